@@ -1,0 +1,359 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself:
+brute force on tiny inputs, closed forms, library routines, invariants the pages
+state, and the cache sizes the pages print.  CPU only."""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import hymba_oracle as O
+from tests import _small
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --- P1: attention equals a brute-force per-query loop (Eq. 1 with scale and mask) ----------
+
+def _attention_loop(q, k, v, s):
+    """Pure-Python scalar loops with math.exp, one query and one key at a time."""
+    L = q.shape[0]
+    H, G, dq, dv = s.n_heads, s.n_kv_heads, s.head_dim_qk, s.head_dim_v
+    out = np.zeros((L, H * dv))
+    for h in range(H):
+        g = h // (H // G)
+        for i in range(L):
+            scores = []
+            for j in range(L):
+                ok = j <= i and (s.is_global or j < s.n_meta or i - j < s.window)
+                if ok:
+                    dot = sum(q[i, h * dq + t] * k[j, g * dq + t] for t in range(dq))
+                    scores.append((j, dot / math.sqrt(dq)))
+            mx = max(sc for _, sc in scores)
+            ws = [(j, math.exp(sc - mx)) for j, sc in scores]
+            tot = sum(w for _, w in ws)
+            for t in range(dv):
+                out[i, h * dv + t] = sum(w * v[j, g * dv + t] for j, w in ws) / tot
+    return out
+
+
+@pytest.mark.parametrize("m,W,glob", [(3, 5, False), (0, 4, False), (2, 100, False), (3, 5, True)])
+def test_p1_attention_bruteforce(m, W, glob):
+    s = _small.spec(m=m, W=W, is_global=glob, H=4, G=2, dq=4, E=16)
+    r = np.random.default_rng(7)
+    L = 13
+    q = r.normal(size=(L, s.n_heads * s.head_dim_qk))
+    k = r.normal(size=(L, s.n_kv_heads * s.head_dim_qk))
+    v = r.normal(size=(L, s.n_kv_heads * s.head_dim_v))
+    np.testing.assert_allclose(O.attention(q, k, v, s), _attention_loop(q, k, v, s),
+                               rtol=0, atol=1e-12)
+
+
+# --- P2: mask special cases -------------------------------------------------------------------
+
+def test_p2_window_covering_sequence_is_global():
+    L = 37
+    for m in (0, 1, 5):
+        for W in (L, L + 1, 1000):
+            np.testing.assert_array_equal(O.mask_matrix(L, m, W, False), O.mask_matrix(L, m, 0, True))
+    s_loc = _small.spec(m=2, W=40)
+    s_glob = _small.spec(m=2, W=1, is_global=True)
+    w = _small.weights(s_loc, seed=3)
+    x = _small.x_tilde(s_loc, 20)
+    np.testing.assert_allclose(O.layer_prefill(x, w, s_loc)["Y"], O.layer_prefill(x, w, s_glob)["Y"],
+                               rtol=0, atol=1e-13)
+
+
+def test_p2_zero_meta_is_plain_sliding_window():
+    L = 29
+    for W in (1, 2, 7, 28, 29):
+        want = np.array([[j <= i and i - j < W for j in range(L)] for i in range(L)])
+        np.testing.assert_array_equal(O.mask_matrix(L, 0, W, False), want)
+
+
+def test_mask_predicate_and_bitmap_match_explicit_loops():
+    for (L, m, W, g) in [(70, 16, 8, False), (33, 0, 1, False), (64, 64, 3, False), (65, 1, 64, False),
+                         (40, 5, 0, True)]:
+        mat = O.mask_matrix(L, m, W, g)
+        for i in range(L):
+            for j in range(L):
+                assert mat[i, j] == O.allowed(i, j, m, W, g)
+        bm = O.mask_bitmap(L, m, W, g)
+        for i in range(L):
+            for j in range(L):
+                assert bool((int(bm[i, j // 32]) >> (j % 32)) & 1) == mat[i, j]
+            # bits past L are zero
+            for j in range(L, bm.shape[1] * 32):
+                assert ((int(bm[i, j // 32]) >> (j % 32)) & 1) == 0
+
+
+# --- P3: beta = 0 isolates one branch (Eq. 3; head-importance analysis of §2.1) ----------------
+
+def test_p3_beta_isolates_branches():
+    s = _small.spec()
+    w = _small.weights(s, seed=5)
+    x = _small.x_tilde(s, 17)
+    base = O.layer_prefill(x, w, s)
+    # beta_ssm = 0: output is W_out(beta_attn * norm(attn) / 2) and does not depend on SSM weights.
+    w_a = dict(w, beta_ssm=np.zeros(s.d_inner))
+    ya = O.layer_prefill(x, w_a, s)["Y"]
+    na = base["o"] / np.sqrt((base["o"] ** 2).mean(1, keepdims=True) + s.eps)
+    np.testing.assert_allclose(ya, (w["beta_attn"] * na / 2) @ w["w_out"].T, atol=1e-12)
+    w_a2 = dict(w_a, conv_w=w["conv_w"] * 3.0, a_log=w["a_log"] * 0.5, w_x=-w["w_x"])
+    np.testing.assert_allclose(O.layer_prefill(x, w_a2, s)["Y"], ya, atol=1e-12)
+    # beta_attn = 0: output does not depend on the Q/K/V rows of W_in.
+    w_s = dict(w, beta_attn=np.zeros(s.d_inner))
+    ys = O.layer_prefill(x, w_s, s)["Y"]
+    nqkv = s.n_heads * s.head_dim_qk + s.n_kv_heads * (s.head_dim_qk + s.head_dim_v)
+    w_in2 = w["w_in"].copy()
+    w_in2[:nqkv] = np.random.default_rng(9).normal(size=(nqkv, s.d_model))
+    np.testing.assert_allclose(O.layer_prefill(x, dict(w_s, w_in=w_in2), s)["Y"], ys, atol=1e-12)
+    ns = base["y_ssm"] / np.sqrt((base["y_ssm"] ** 2).mean(1, keepdims=True) + s.eps)
+    np.testing.assert_allclose(ys, (w["beta_ssm"] * ns / 2) @ w["w_out"].T, atol=1e-12)
+    # Both on: the mean of the two normalised branches (factor 1/2, not a sum).
+    np.testing.assert_allclose(base["Y"], ya + ys, atol=1e-12)
+
+
+# --- P4: constant delta, scalar A, constant B and u -> geometric sum --------------------------
+
+def test_p4_scan_geometric_closed_form():
+    T, E, N = 50, 3, 2
+    dl, a_val, b_val, u_val = 0.3, -1.7, 0.8, 1.3
+    u = np.full((T, E), u_val)
+    delta = np.full((T, E), dl)
+    A = np.full((E, N), a_val)
+    Bm = np.full((T, N), b_val)
+    Cm = np.ones((T, N))
+    y, h = O.selective_scan(u, delta, A, Bm, Cm, np.zeros(E))
+    a = math.exp(dl * a_val)
+    for t in range(T):
+        want = dl * b_val * u_val * (1 - a ** (t + 1)) / (1 - a)
+        np.testing.assert_allclose(y[t], N * want, rtol=1e-13)
+    np.testing.assert_allclose(h, dl * b_val * u_val * (1 - a ** T) / (1 - a), rtol=1e-13)
+
+
+def test_scan_with_zero_A_is_cumulative_sum():
+    r = np.random.default_rng(2)
+    T, E, N = 40, 5, 3
+    u, delta = r.normal(size=(T, E)), r.uniform(0.1, 1, (T, E))
+    Bm, Cm = r.normal(size=(T, N)), r.normal(size=(T, N))
+    y, h = O.selective_scan(u, delta, np.zeros((E, N)), Bm, Cm, np.zeros(E))
+    hs = np.cumsum((delta * u)[:, :, None] * Bm[:, None, :], axis=0)
+    np.testing.assert_allclose(y, np.einsum("ten,tn->te", hs, Cm), rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(h, hs[-1], rtol=1e-12)
+
+
+# --- P5: Eq. 2's materialised operator equals the recurrence ----------------------------------
+
+def test_p5_materialised_eq2_equals_recurrence():
+    r = np.random.default_rng(4)
+    T, E, N = 24, 6, 4
+    u, delta = r.normal(size=(T, E)), r.uniform(0.05, 0.8, (T, E))
+    A = -np.exp(r.uniform(0, math.log(16), (E, N)))
+    Bm, Cm = r.normal(size=(T, N)), r.normal(size=(T, N))
+    Dv = r.normal(size=E)
+    z = r.normal(size=(T, E))
+    y_rec, _ = O.selective_scan(u, delta, A, Bm, Cm, Dv)
+    # alpha^{i,j}[c] = sum_n C_i[n] * prod_{k=j+1..i} exp(A[c,n] delta_k[c]) * B_j[n] * delta_j[c]
+    y_mat = np.zeros((T, E))
+    for i in range(T):
+        for j in range(i + 1):
+            decay = np.exp(A * delta[j + 1:i + 1].sum(axis=0)[:, None])  # empty product -> 1
+            alpha = (Cm[i][None, :] * decay * Bm[j][None, :]).sum(axis=1) * delta[j]
+            y_mat[i] += alpha * u[j]
+        y_mat[i] += Dv * u[i]
+    np.testing.assert_allclose(y_rec, y_mat, rtol=1e-11, atol=1e-12)
+    silu = z / (1 + np.exp(-z))
+    np.testing.assert_allclose(y_rec * silu, y_mat * silu, rtol=1e-11, atol=1e-12)
+
+
+# --- conv: causal depthwise conv equals numpy.convolve; tap order --------------------------------
+
+def test_causal_conv_matches_numpy_convolve():
+    r = np.random.default_rng(6)
+    T, E, K = 19, 4, 4
+    x = r.normal(size=(T, E))
+    w = r.normal(size=(E, K))
+    b = r.normal(size=E)
+    u = O.causal_conv_silu(x, w, b)
+    for c in range(E):
+        pre = np.convolve(x[:, c], w[c, ::-1])[:T] + b[c]
+        np.testing.assert_allclose(u[:, c], pre / (1 + np.exp(-pre)), rtol=1e-13, atol=1e-14)
+    # history rows act as the K-1 inputs before row 0
+    hist = r.normal(size=(K - 1, E))
+    full = O.causal_conv_silu(np.concatenate([hist, x]), w, b)[K - 1:]
+    np.testing.assert_allclose(O.causal_conv_silu(x, w, b, history=hist), full, rtol=1e-13)
+
+
+def test_elementwise_functions_known_values():
+    np.testing.assert_allclose(O.softplus(np.array([0.0, -4.0, 30.0, -50.0])),
+                               [math.log(2.0), math.log1p(math.exp(-4.0)), 30.0 + math.log1p(math.exp(-30.0)),
+                                math.exp(-50.0)], rtol=1e-14)
+    np.testing.assert_allclose(O.silu(np.array([0.0, 1.0, -2.0])),
+                               [0.0, 1 / (1 + math.exp(-1)), -2 / (1 + math.exp(2))], rtol=1e-14)
+
+
+# --- P6: a KV-sharing consumer equals recomputation with the producer's K/V -------------------
+
+def test_p6_kv_shared_consumer_equals_recompute():
+    s = _small.spec(m=2, W=4)
+    wp = _small.weights(s, seed=11)
+    wc = _small.weights(s, seed=12, consumer=True)
+    x = _small.x_tilde(s, 15, seed=3)
+    prod = O.layer_prefill(x, wp, s)
+    cons = O.layer_prefill(x, wc, s, kv_from=prod)
+    # A standalone layer with the consumer's Q/SSM/gate rows and the producer's K/V rows, on the
+    # same input: its own K/V equal the producer's, so it must match the consumer exactly.
+    nq = s.n_heads * s.head_dim_qk
+    nkv = s.n_kv_heads * (s.head_dim_qk + s.head_dim_v)
+    w_in = np.concatenate([wc["w_in"][:nq], wp["w_in"][nq:nq + nkv], wc["w_in"][nq:]], 0)
+    alone = O.layer_prefill(x, dict(wc, w_in=w_in), s)
+    np.testing.assert_allclose(cons["Y"], alone["Y"], atol=1e-13)
+    # With a different consumer input the K/V still come from the producer's input.
+    x2 = _small.x_tilde(s, 15, seed=4)
+    cons2 = O.layer_prefill(x2, wc, s, kv_from=prod)
+    cons3 = O.layer_prefill(x2, wc, s, kv_from=O.layer_prefill(x2, wp, s))
+    assert np.abs(cons2["o"] - cons3["o"]).max() > 1e-3
+
+
+# --- P7: GQA equals MHA with K/V heads repeated per group --------------------------------------
+
+def test_p7_gqa_equals_mha_with_repeated_kv():
+    s = _small.spec(H=4, G=2, dq=4, E=16)
+    w = _small.weights(s, seed=13)
+    x = _small.x_tilde(s, 14)
+    nq = s.n_heads * s.head_dim_qk
+    nk = s.n_kv_heads * s.head_dim_qk
+    nv = s.n_kv_heads * s.head_dim_v
+    Wk = w["w_in"][nq:nq + nk].reshape(s.n_kv_heads, s.head_dim_qk, -1)
+    Wv = w["w_in"][nq + nk:nq + nk + nv].reshape(s.n_kv_heads, s.head_dim_v, -1)
+    rep = s.n_heads // s.n_kv_heads
+    Wk_m = np.repeat(Wk, rep, axis=0).reshape(-1, s.d_model)  # head h <- group h // rep
+    Wv_m = np.repeat(Wv, rep, axis=0).reshape(-1, s.d_model)
+    s_mha = _small.spec(H=4, G=4, dq=4, E=16)
+    w_m = dict(w, w_in=np.concatenate([w["w_in"][:nq], Wk_m, Wv_m, w["w_in"][nq + nk + nv:]], 0))
+    np.testing.assert_allclose(O.layer_prefill(x, w, s)["Y"], O.layer_prefill(x, w_m, s_mha)["Y"],
+                               atol=1e-13)
+
+
+# --- P8: causality, window locality, meta rows ------------------------------------------------
+
+def test_p8_causality_window_and_meta():
+    s = _small.spec(m=3, W=4)
+    w = _small.weights(s, seed=21)
+    L = 18
+    x = _small.x_tilde(s, L)
+    base = O.layer_prefill(x, w, s)
+    t = 9
+    x2 = x.copy()
+    x2[t] += 1.0
+    y2 = O.layer_prefill(x2, w, s)
+    np.testing.assert_array_equal(y2["Y"][:t], base["Y"][:t])
+    assert np.abs(y2["Y"][t:] - base["Y"][t:]).min(axis=1).max() > 0
+    # attention branch alone: a real row only reaches rows [j, j + W - 1]
+    changed = np.abs(y2["o"] - base["o"]).max(axis=1) > 0
+    assert changed.tolist() == [t <= i <= t + s.window - 1 for i in range(L)]
+    # a meta row reaches every later row through attention
+    x3 = x.copy()
+    x3[1] += 1.0
+    ch3 = np.abs(O.layer_prefill(x3, w, s)["o"] - base["o"]).max(axis=1) > 0
+    assert ch3.tolist() == [i >= 1 for i in range(L)]
+    # meta-row outputs do not depend on the real rows
+    x4 = x.copy()
+    x4[s.n_meta:] = _small.x_tilde(s, L - s.n_meta, seed=99)
+    np.testing.assert_array_equal(O.layer_prefill(x4, w, s)["Y"][:s.n_meta], base["Y"][:s.n_meta])
+
+
+# --- P9: prefill(n) then decode == prefill(n + 1) ------------------------------------------------
+
+@pytest.mark.parametrize("glob", [False, True])
+def test_p9_decode_after_prefill(glob):
+    s = _small.spec(m=3, W=4, is_global=glob)
+    wp = _small.weights(s, seed=31)
+    wc = _small.weights(s, seed=32, consumer=True)
+    L = 16
+    x = _small.x_tilde(s, L + 1)
+    cap = L + 1 if glob else None
+    full_p = O.layer_prefill(x, wp, s, capacity=cap)
+    full_c = O.layer_prefill(x, wc, s, kv_from=full_p)
+    pre_p = O.layer_prefill(x[:L], wp, s, capacity=cap)
+    pre_c = O.layer_prefill(x[:L], wc, s, kv_from=pre_p)
+    cache_p = dict(k=pre_p["k_cache"], v=pre_p["v_cache"], ssm=pre_p["h"], conv=pre_p["conv"])
+    y_p, new_p = O.layer_decode(x[L], L, wp, s, cache_p)
+    np.testing.assert_allclose(y_p, full_p["Y"][L], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(new_p["ssm"], full_p["h"], rtol=1e-11, atol=1e-13)
+    np.testing.assert_allclose(new_p["conv"], full_p["conv"], rtol=1e-13, atol=1e-14)
+    cache_c = dict(ssm=pre_c["h"], conv=pre_c["conv"])
+    y_c, _ = O.layer_decode(x[L], L, wc, s, cache_c, kv_cache=new_p)
+    np.testing.assert_allclose(y_c, full_c["Y"][L], rtol=1e-11, atol=1e-12)
+
+
+def test_ring_slots_hold_the_window():
+    """Simulate appending positions one at a time into a ring of W slots after m meta slots;
+    after every append the slots hold exactly the meta rows plus the last W positions."""
+    for m, W in [(0, 1), (3, 4), (5, 7), (128, 1024)]:
+        s = _small.spec(m=m, W=W)
+        store = {}
+        for p in range(m + 3 * W + 5):
+            store[O.kv_slot(p, s)] = p
+            held = sorted(store.values())
+            want = list(range(min(p + 1, m))) + list(range(max(m, p - W + 1), p + 1))
+            assert held == want
+            assert max(store) < m + W
+
+
+# --- P10: the printed cache sizes fix the value head width -------------------------------------
+
+def test_p10_cache_size_reading():
+    g = json.load(open(os.path.join(GOLDEN, "cache_sizes.json")))
+    tokens, b = g["convention"]["tokens"], g["convention"]["bytes_per_value"]
+    ll = g["llama_3_2_3b_public_config"]
+    llama = ll["layers"] * ll["kv_heads"] * ll["head_dim"] * 2 * b * tokens / 1e6
+    assert abs(llama - g["printed"]["llama_3_2_3b_MB"]) / g["printed"]["llama_3_2_3b_MB"] < 0.005
+
+    def hymba(dv):
+        t = g["hymba_1p5b"]
+        full = t["global_layers"] * tokens * t["kv_heads"] * (t["head_dim_qk"] + dv) * b
+        ring = t["swa_kv_producers"] * t["window"] * t["kv_heads"] * (t["head_dim_qk"] + dv) * b
+        ssm = t["layers"] * t["d_inner"] * t["d_state"] * b
+        return (full + ring + ssm) / 1e6
+
+    printed = g["printed"]["hymba_1p5b_MB"]
+    assert abs(hymba(128) - printed) / printed < 0.005
+    assert abs(hymba(64) - printed) / printed > 0.25
+    assert abs(g["printed"]["llama_3_2_3b_MB"] / printed - g["printed"]["ratio_vs_llama"]) < 0.05
+
+
+# --- P11 / P12: softmax rows sum to one; RMS normalisation ------------------------------------
+
+def test_p11_softmax_rows_sum_to_one():
+    s = _small.spec(H=4, G=2, dq=4, E=16)
+    r = np.random.default_rng(8)
+    L = 11
+    q = r.normal(size=(L, s.n_heads * s.head_dim_qk)) * 5
+    k = r.normal(size=(L, s.n_kv_heads * s.head_dim_qk))
+    v = np.ones((L, s.n_kv_heads * s.head_dim_v))
+    np.testing.assert_allclose(O.attention(q, k, v, s), 1.0, atol=1e-14)
+    # a constant added to every score of a row changes nothing: give every key an extra
+    # coordinate equal to 1 and the query a value there
+    s2 = _small.spec(H=4, G=2, dq=5, E=16)
+    v2 = r.normal(size=(L, s.n_kv_heads * s.head_dim_v))
+
+    def widen(a, heads, extra):
+        a = a.reshape(L, heads, 4)
+        return np.concatenate([a, np.broadcast_to(extra, (L, heads, 1))], 2).reshape(L, heads * 5)
+
+    o1 = O.attention(widen(q, 4, 0.0), widen(k, 2, 1.0), v2, s2)
+    o2 = O.attention(widen(q, 4, 3.7), widen(k, 2, 1.0), v2, s2)
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+
+
+def test_p12_rms_normalise():
+    r = np.random.default_rng(1)
+    x = r.normal(size=(7, 300)) * 9.0
+    n = O.rms_normalise(x, 0.0)
+    np.testing.assert_allclose(np.sqrt((n ** 2).mean(1)), 1.0, rtol=1e-14)
+    np.testing.assert_allclose(n * np.sqrt((x ** 2).mean(1, keepdims=True)), x, rtol=1e-14)
