@@ -1,0 +1,503 @@
+#!/usr/bin/env python
+"""Benchmark of the Hymba hybrid-head layer hot path on B200.
+
+One step = the whole hot path over one batch of synthetic input:
+  * prefill of two consecutive sliding-window layers sharing one K/V (layer 2
+    reuses layer 1's K/V), bf16, batch 128, 8192 real tokens + 128 meta tokens,
+    window 1024, 1.5B widths (d_model 1600, 25/5 heads, d_inner 3200, state 16);
+  * one decode step of a 32-layer stack at the same widths, batch 128, 8k
+    context: global attention in layers 0, 15, 31, window 1024 + 128 meta
+    elsewhere, K/V shared by consecutive sliding-window layers, N(0,1) caches.
+`value` is prefill throughput in real tokens per second (B * 8192 tokens through
+both layers per step, whole job over all ranks); decode tokens/s is reported
+beside it.  Inputs are resident in HBM before the timed region; inputs are far
+larger than L2, so no flush is needed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Under torchrun every rank runs its own replica (weak scaling, no collective on
+the data path) and rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+METRIC = "hybrid-layer prefill tok/s @B=128,L=8k bf16 + decode tok/s; % of roofline"
+UNIT = "tok/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks sampled with nvidia-smi during the timed region
+# ---------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except FileNotFoundError:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------------------------
+# our path
+# ---------------------------------------------------------------------------------------------
+class Prefill:
+    """The two KV-sharing prefill layers of the headline workload."""
+
+    def __init__(self, w, dev):
+        import hybrid_attention_ssm_head_b200 as hy
+        import synth
+        self.hy = hy
+        self.w = w
+        d = w.dims
+        B, L, n = w.batch, w.seq_rows, w.n_tokens
+        self.B, self.L, self.n = B, L, n
+        self.wts, self.handles = [], []
+        for layer, consumer in ((0, False), (1, True)):
+            wt = {k: v.contiguous() for k, v in
+                  synth.configs.layer_weights(w, layer, consumer=consumer, device=dev).items()}
+            cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner, d.d_state,
+                                 d.d_conv, d.rank, w.n_meta, w.window, False, "bf16")
+            self.wts.append(wt)
+            self.handles.append(hy.hymba_layer_create(cfg, hy.make_weights(wt)))
+        hy.hymba_kv_share_bind(self.handles[1], self.handles[0])
+        self.x = synth.configs.x_tilde(w, device=dev)
+        self.y1 = torch.empty_like(self.x)
+        self.y2 = torch.empty_like(self.x)
+        self.k = torch.empty(B, L, d.n_kv_heads * d.head_dim_qk, dtype=torch.bfloat16, device=dev)
+        self.v = torch.empty(B, L, d.n_kv_heads * d.head_dim_v, dtype=torch.bfloat16, device=dev)
+        self.kv = hy.hymba_kv_seq(self.k.data_ptr(), self.v.data_ptr(), 0, 0, 0)
+        nb = max(hy.hymba_layer_prefill_workspace(h, B, n) for h in self.handles)
+        self.ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+
+    def run(self, stream, x=None, y=None):
+        hy = self.hy
+        x = self.x if x is None else x
+        y = self.y2 if y is None else y
+        hy.hymba_layer_prefill(self.handles[0], self.B, self.n, x, self.y1, self.kv, None, None,
+                               self.ws, self.ws.numel(), stream)
+        hy.hymba_layer_prefill(self.handles[1], self.B, self.n, self.y1, y, self.kv, None, None,
+                               self.ws, self.ws.numel(), stream)
+
+    def flops(self):
+        """Algorithmic FLOPs of one step (both layers), attention counted on visible pairs only."""
+        d, w = self.w.dims, self.w
+        M = self.B * self.L
+        E, H = d.d_inner, d.n_heads
+        f = 0.0
+        for consumer in (False, True):
+            P = d.in_width(consumer)
+            f += 2.0 * M * P * d.d_model                       # in_proj
+            f += 2.0 * M * d.xproj_width * E                   # x_proj
+            f += 2.0 * M * E * d.rank                          # dt_proj
+            f += 2.0 * M * d.d_model * E                       # out_proj
+            f += self.B * H * 2.0 * (d.head_dim_qk + d.head_dim_v) * visible_pairs(
+                self.L, w.n_meta, w.window, False)             # attention
+        return f
+
+    def in_proj_flops(self):
+        d = self.w.dims
+        M = self.B * self.L
+        return [2.0 * M * d.in_width(False) * d.d_model, 2.0 * M * d.in_width(True) * d.d_model]
+
+
+def visible_pairs(L, m, W, is_global):
+    tot = 0
+    for i in range(L):
+        if is_global:
+            tot += i + 1
+        else:
+            tot += min(i + 1, m) + max(0, i - max(m, i - W + 1) + 1)
+    return tot
+
+
+class Decode:
+    """One decode step of the 32-layer stack (one new token per sequence)."""
+
+    def __init__(self, w, dev):
+        import hybrid_attention_ssm_head_b200 as hy
+        import synth
+        self.hy = hy
+        self.w = w
+        d = w.dims
+        B = w.batch
+        self.B = B
+        self.pos = w.n_meta + w.n_tokens
+        layout = synth.configs.stack_layout(w.n_layers)
+        self.layers = []
+        for l, (is_global, producer) in enumerate(layout):
+            consumer = producer is not None
+            wt = {k: v.contiguous() for k, v in
+                  synth.configs.layer_weights(w, l, consumer=consumer, device=dev).items()}
+            cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner, d.d_state,
+                                 d.d_conv, d.rank, w.n_meta, w.window, is_global, "bf16")
+            h = hy.hymba_layer_create(cfg, hy.make_weights(wt))
+            cap = self.pos + 1 if is_global else w.n_meta + w.window
+            caches = synth.configs.decode_caches(w, l, cap, consumer, device=dev)
+            caches = {k: v.contiguous() for k, v in caches.items()}
+            ent = dict(handle=h, wt=wt, caches=caches, is_global=is_global, producer=producer, cap=cap)
+            ent["ssm"] = hy.hymba_ssm_cache(caches["ssm"].data_ptr(), caches["conv"].data_ptr())
+            if not consumer:
+                ent["kvc"] = hy.hymba_kv_cache(caches["k"].data_ptr(), caches["v"].data_ptr(), B, cap, 0)
+            else:
+                hy.hymba_kv_share_bind(h, self.layers[producer]["handle"])
+            self.layers.append(ent)
+        self.x = synth.configs.decode_tokens(w, device=dev)
+        self.ys = [torch.empty_like(self.x) for _ in range(2)]
+        nb = max(hy.hymba_layer_decode_workspace(e["handle"], B, self.pos) for e in self.layers)
+        self.ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        self.graph = None
+
+    def run(self, stream, x=None, y_out=None):
+        hy = self.hy
+        cur = self.x if x is None else x
+        for l, e in enumerate(self.layers):
+            out = self.ys[l % 2] if (l + 1 < len(self.layers) or y_out is None) else y_out
+            kvc = e["kvc"] if e["producer"] is None else self.layers[e["producer"]]["kvc"]
+            hy.hymba_layer_decode_step(e["handle"], self.B, self.pos, cur, out, kvc, e["ssm"],
+                                       self.ws, self.ws.numel(), stream)
+            cur = out
+        return cur
+
+    def capture(self):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.run(s)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            self.run(torch.cuda.current_stream())
+        self.graph = g
+
+    def hbm_bytes(self):
+        """Minimum HBM traffic of one decode step (bytes)."""
+        d = self.w.dims
+        B = self.B
+        tot = 0
+        for e in self.layers:
+            for k, v in e["wt"].items():
+                tot += v.numel() * v.element_size()
+            tot += 2 * e["caches"]["ssm"].numel() * 4                 # SSM state read + write
+            tot += 2 * e["caches"]["conv"].numel() * 2
+            if e["is_global"]:
+                keys = self.pos + 1
+            else:
+                keys = self.w.n_meta + self.w.window
+            tot += B * d.n_kv_heads * keys * (d.head_dim_qk + d.head_dim_v) * 2  # K/V read
+        return tot
+
+
+def run_ours(args, rank, world, dev):
+    import hybrid_attention_ssm_head_b200 as hy
+    import synth
+    torch.cuda.set_device(dev)
+    w3, w4 = synth.configs.CFG3, synth.configs.CFG4
+    t_setup = time.time()
+    pre = Prefill(w3, dev)
+    dec = Decode(w4, dev)
+    torch.cuda.synchronize()
+    setup_s = time.time() - t_setup
+    stream = torch.cuda.current_stream()
+
+    # warm-up (also first-use costs: function attributes, tensor maps)
+    for _ in range(args.warmup):
+        pre.run(stream)
+        dec.run(stream)
+    hy.hymba_stream_status(stream)
+    dec.capture()
+    dec.graph.replay()
+    hy.hymba_stream_status(stream)
+
+    # timed region: K steps, prefill (eager, per-kernel events on) + decode (graph)
+    peaks, peak_src = load_peaks()
+    sampler = ClockSampler(torch.cuda.current_device())
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    hy.hymba_profile_enable(True)
+    hy.hymba_profile_collect()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * args.steps + 1)]
+    ev[0].record(stream)
+    for s in range(args.steps):
+        pre.run(stream)
+        ev[2 * s + 1].record(stream)
+        dec.graph.replay()
+        ev[2 * s + 2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    prof = hy.hymba_profile_collect()
+    hy.hymba_profile_enable(False)
+    clocks = sampler.stop() if rank == 0 else None
+    hy.hymba_stream_status(stream)
+    pre_ms = sum(ev[2 * s].elapsed_time(ev[2 * s + 1]) for s in range(args.steps))
+    dec_ms = sum(ev[2 * s + 1].elapsed_time(ev[2 * s + 2]) for s in range(args.steps))
+    tot_ms = ev[0].elapsed_time(ev[-1])
+    t = torch.tensor([pre_ms, dec_ms, tot_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    pre_ms, dec_ms, tot_ms = t.tolist()
+
+    # kernel launches of this library in the timed region: prefill launches are counted by the
+    # profiler; the decode graph holds a fixed number per step (counted once below, eagerly)
+    pre_launches = sum(k for _, _, k, _ in prof)
+    hy.hymba_profile_enable(True)
+    hy.hymba_profile_collect()
+    dec.run(stream)
+    dprof = hy.hymba_profile_collect()
+    hy.hymba_profile_enable(False)
+    dec_kernels_per_step = sum(k for _, _, k, _ in dprof)
+
+    tokens = w3.batch * w3.n_tokens
+    value = tokens * args.steps * world / (pre_ms / 1e3)
+    dec_tok_s = w4.batch * args.steps * world / (dec_ms / 1e3)
+
+    # roofline of the dominant kernel: the input projection GEMM (tensor-bound)
+    pmap = {n: (c, ms) for n, c, _, ms in prof}
+    c_in, ms_in = pmap.get("in_proj", (0, 0.0))
+    fl = pre.in_proj_flops()
+    flops_per_launch = sum(fl) / 2.0
+    achieved = (flops_per_launch * c_in) / (ms_in / 1e3) / 1e12 if ms_in > 0 else None
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    roof = {"kernel": "in_proj (gemm_tc_kernel<256,bf16>)", "bound": "tensor",
+            "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": (achieved / peak) if achieved else None, "traffic": None,
+            "peak_source": f"{peak_src} bf16_tflops_sustained"}
+    step_flops = pre.flops()
+    dec_bytes = dec.hbm_bytes()
+
+    # end to end through the C ABI with host buffers: pinned X~ in, Y out, every step
+    e2e = None
+    if not args.no_e2e:
+        xh = torch.empty(pre.x.shape, dtype=pre.x.dtype, pin_memory=True)
+        xh.copy_(pre.x)
+        yh = torch.empty_like(xh, pin_memory=True)
+        xt_h = torch.empty(dec.x.shape, dtype=dec.x.dtype, pin_memory=True)
+        xt_h.copy_(dec.x)
+        yt_h = torch.empty_like(xt_h, pin_memory=True)
+        xd = torch.empty_like(pre.x)
+        xtd = torch.empty_like(dec.x)
+        ytd = torch.empty_like(dec.x)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ed0, ed1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pre_e2e_ms, dec_e2e_ms = 0.0, 0.0
+        steps_e2e = max(1, min(args.steps, 3))
+        for _ in range(steps_e2e):
+            e0.record(stream)
+            xd.copy_(xh, non_blocking=True)
+            pre.run(stream, x=xd)
+            yh.copy_(pre.y2, non_blocking=True)
+            e1.record(stream)
+            ed0.record(stream)
+            xtd.copy_(xt_h, non_blocking=True)
+            dec.run(stream, x=xtd, y_out=ytd)
+            yt_h.copy_(ytd, non_blocking=True)
+            ed1.record(stream)
+            torch.cuda.synchronize()
+            pre_e2e_ms += e0.elapsed_time(e1)
+            dec_e2e_ms += ed0.elapsed_time(ed1)
+        t = torch.tensor([pre_e2e_ms, dec_e2e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        pre_e2e_ms, dec_e2e_ms = t.tolist()
+        e2e = {"value": tokens * steps_e2e * world / (pre_e2e_ms / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": xh.numel() * 2 + xt_h.numel() * 2,
+               "d2h_bytes_per_step": yh.numel() * 2 + yt_h.numel() * 2,
+               "decode_tok_s": w4.batch * steps_e2e * world / (dec_e2e_ms / 1e3)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_sample()
+
+    if rank != 0:
+        return None
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "prefill: 2 KV-sharing SWA layers, B=128, 8192+128 meta rows, W=1024, "
+                               "1.5B widths; decode: 32-layer stack, B=128, 8k context",
+                   "prefill": w3.name, "decode": w4.name, "global_batch": w3.batch * world,
+                   "seq_len": w3.seq_rows, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "prefill_ms_per_step": pre_ms / args.steps,
+        "decode_ms_per_step": dec_ms / args.steps,
+        "decode_tok_s": dec_tok_s,
+        "prefill_tflops": step_flops * args.steps / (pre_ms / 1e3) / 1e12,
+        "prefill_roofline_frac": (step_flops / (peaks.get("bf16_tflops_sustained", 1400) * 1e12))
+                                 / (pre_ms / args.steps / 1e3),
+        "decode_hbm_gbs": dec_bytes * args.steps / (dec_ms / 1e3) / 1e9,
+        "decode_roofline_frac": (dec_bytes / (peaks.get("hbm_gbs", 6650) * 1e9)) / (dec_ms / args.steps / 1e3),
+        "roofline": roof,
+        "steps_profile": {n: {"calls": c, "kernels": k, "ms_per_call": ms / c if c else None}
+                          for n, c, k, ms in prof},
+        "gpu_launches": pre_launches + dec_kernels_per_step * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "setup_s": setup_s,
+    }
+    return out
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands on the host cores, on a bounded sample
+# ---------------------------------------------------------------------------------------------
+CPU_SAMPLE_TOKENS = 2048
+
+
+def cpu_baseline_sample(tokens: int = CPU_SAMPLE_TOKENS):
+    import numpy as np
+    import synth
+    from oracle import hymba_oracle as O
+    w = synth.configs.CFG3
+    d = w.dims
+    spec = O.Spec(d_model=d.d_model, n_heads=d.n_heads, n_kv_heads=d.n_kv_heads,
+                  head_dim_qk=d.head_dim_qk, head_dim_v=d.head_dim_v, d_inner=d.d_inner,
+                  d_state=d.d_state, d_conv=d.d_conv, dt_rank=d.rank, n_meta=w.n_meta,
+                  window=w.window, is_global=False)
+    x = synth.configs.x_tilde(w, batch_index=0)[: w.n_meta + tokens]
+    w0 = {k: v.double().numpy() for k, v in synth.configs.layer_weights(w, 0).items()}
+    w1 = {k: v.double().numpy() for k, v in synth.configs.layer_weights(w, 1, consumer=True).items()}
+    xt = x.double().numpy()
+    t0 = time.perf_counter()
+    r0 = O.layer_prefill(xt, w0, spec)
+    O.layer_prefill(r0["Y"], w1, spec, kv_from=r0)
+    dt = time.perf_counter() - t0
+    cores = torch.get_num_threads()
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max([i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"] or [cores])
+    except Exception:
+        pass
+    return {"value": tokens / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"one sequence (batch row 0) of the prefill workload, first {tokens} real "
+                      f"tokens + {w.n_meta} meta rows, both KV-sharing layers, fp64 numpy",
+            "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    samples = []
+    for _ in range(args.warmup):
+        cpu_baseline_sample(512)
+    for _ in range(args.steps):
+        samples.append(cpu_baseline_sample(512))
+    secs = sum(s["seconds"] for s in samples)
+    value = 512 * args.steps / secs
+    s0 = samples[0]
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": "prefill: 2 KV-sharing SWA layers, B=128, 8192+128 meta rows, "
+                                   "W=1024, 1.5B widths (oracle on a bounded sample per step)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": s0["cores"], "kind": "oracle",
+                             "sample": s0["sample"].replace("2048", "512")},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    out = run_ours(args, rank, world, dev)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,121 @@
+// Fusion of the two branches (Hymba §2.1 Eq. 3): each branch output is
+// RMS-normalised over its d_inner channels, re-scaled per channel by beta and
+// the two are averaged:  f = (beta_1 * o / rms(o) + beta_2 * y / rms(y)) / 2.
+// One CTA per token row; 16-byte vector loads; the second pass re-reads the
+// row from L1/L2, so HBM sees each input once.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace hymba {
+
+template <typename T>
+__device__ __forceinline__ void ld16(const T *p, float (&v)[16 / sizeof(T)]) {
+  uint4 raw = __ldg(reinterpret_cast<const uint4 *>(p));
+  if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __low2float(h[i]);
+      v[2 * i + 1] = __high2float(h[i]);
+    }
+  } else {
+    const float *f = reinterpret_cast<const float *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = f[i];
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) fuse_kernel(FuseArgs a) {
+  constexpr int V = 16 / sizeof(T);
+  __shared__ float red[2][8];
+  const long long row = blockIdx.x;
+  const T *o = reinterpret_cast<const T *>(a.o) + row * a.E;
+  const T *y = reinterpret_cast<const T *>(a.y) + row * a.E;
+  T *f = reinterpret_cast<T *>(a.f) + row * a.E;
+  float so = 0.f, sy = 0.f;
+  for (int c = threadIdx.x * V; c < a.E; c += blockDim.x * V) {
+    float vo[V], vy[V];
+    ld16<T>(o + c, vo);
+    ld16<T>(y + c, vy);
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      so = fmaf(vo[i], vo[i], so);
+      sy = fmaf(vy[i], vy[i], sy);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) {
+    so += __shfl_xor_sync(0xffffffffu, so, off);
+    sy += __shfl_xor_sync(0xffffffffu, sy, off);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    red[0][w] = so;
+    red[1][w] = sy;
+  }
+  __syncthreads();
+  so = 0.f;
+  sy = 0.f;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+    so += red[0][i];
+    sy += red[1][i];
+  }
+  const float ro = 0.5f * rsqrtf(so / a.E + a.eps);
+  const float ry = 0.5f * rsqrtf(sy / a.E + a.eps);
+  for (int c = threadIdx.x * V; c < a.E; c += blockDim.x * V) {
+    float vo[V], vy[V], out[V];
+    ld16<T>(o + c, vo);
+    ld16<T>(y + c, vy);
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+      out[i] = fmaf(a.beta_attn[c + i] * ro, vo[i], a.beta_ssm[c + i] * ry * vy[i]);
+    if constexpr (sizeof(T) == 2) {
+      st_global_v4(f + c, pack_bf16x2(out[0], out[1]), pack_bf16x2(out[2], out[3]),
+                   pack_bf16x2(out[4], out[5]), pack_bf16x2(out[6], out[7]));
+    } else {
+      st_global_v4(f + c, __float_as_uint(out[0]), __float_as_uint(out[1]),
+                   __float_as_uint(out[2]), __float_as_uint(out[3]));
+    }
+  }
+}
+
+hymba_status fuse_branches(const FuseArgs &a, hymba_dtype dt, cudaStream_t s) {
+  if (a.M == 0) return HYMBA_OK;
+  if (dt == HYMBA_BF16)
+    fuse_kernel<__nv_bfloat16><<<a.M, 256, 0, s>>>(a);
+  else
+    fuse_kernel<float><<<a.M, 256, 0, s>>>(a);
+  note_launch(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("fuse launch failed: %s", cudaGetErrorString(e));
+    return HYMBA_ERR_CUDA;
+  }
+  return HYMBA_OK;
+}
+
+template <typename T>
+__global__ void convert_kernel(const float *__restrict__ src, T *__restrict__ dst, long long n) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) dst[i] = Store<T>::from_f(src[i]);
+}
+
+hymba_status convert_f32_to(const float *src, void *dst, long long n, hymba_dtype dt,
+                            cudaStream_t s) {
+  if (n == 0) return HYMBA_OK;
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  if (dt == HYMBA_BF16)
+    convert_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(src, (__nv_bfloat16 *)dst, n);
+  else
+    convert_kernel<float><<<blocks, 256, 0, s>>>(src, (float *)dst, n);
+  note_launch(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("convert launch failed: %s", cudaGetErrorString(e));
+    return HYMBA_ERR_CUDA;
+  }
+  return HYMBA_OK;
+}
+
+}  // namespace hymba

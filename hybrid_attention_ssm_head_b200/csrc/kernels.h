@@ -1,0 +1,154 @@
+// Internal launcher interface between the C ABI host layer and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "hymba.h"
+
+namespace hymba {
+
+// Where a GEMM output column goes.  Column c in [col0, col1) of the product is
+// written to  ptr + row*ld_row + ((c-col0)/inner)*ld_group + (c-col0)%inner
+// (element offsets), as fp32 (f32 = 1) or bf16 (f32 = 0).
+struct EpiSeg {
+  void *ptr;
+  long long ld_row;
+  long long ld_group;
+  int col0, col1;
+  int inner;
+  int f32;
+  int vec_ok;  // 16-byte aligned rows/groups: 8-column vector stores allowed
+};
+
+struct Epilogue {
+  EpiSeg seg[5];
+  int nseg;
+  const float *bias;  // per product column (nullable)
+  int act;            // 0 = identity, 1 = softplus
+  int atomic;         // 1 = fp32 atomicAdd into the destination (split-K)
+};
+
+// out[m, n] = epi( sum_k A[m, k] * B[n, k] )  (A: [M, K], B: [N, K], row-major)
+struct GemmArgs {
+  const void *A;
+  long long lda;
+  const void *B;
+  long long ldb;
+  int M, N, K;
+  int elem;    // 2: bf16 operands; 4: fp32 operands
+  int ksplit;  // >= 1; > 1 requires epi.atomic
+  Epilogue epi;
+};
+
+// Tensor-core path (tcgen05 + TMA).  elem 2 -> kind::f16 (bf16), 4 -> kind::tf32.
+hymba_status gemm_tc(const GemmArgs &g, cudaStream_t s);
+// fp32 CUDA-core path for the fp32 storage configuration.
+hymba_status gemm_simt_f32(const GemmArgs &g, cudaStream_t s);
+
+// ---- SSM branch -----------------------------------------------------------
+struct ConvArgs {
+  const void *x;      // [B, L, E] rows of x_ssm, row stride ld_x elements
+  long long ld_x;
+  void *u;            // [B, L, E] dense
+  const float *w;     // [E, K]
+  const float *bias;  // [E]
+  void *conv_state;   // optional [B, K-1, E]: the last K-1 rows of x
+  int B, L, E, K;
+};
+hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s);
+
+struct ScanArgs {
+  const void *u;       // [B, L, E]
+  const void *delta;   // [B, L, E]
+  const void *z;       // [B, L, E], row stride ld_z
+  long long ld_z;
+  const float *bc;     // [B*L, ld_bc] fp32; B at column bc_col, C at bc_col + N
+  long long ld_bc;
+  int bc_col;
+  const float *a_log;  // [E, N]
+  const float *d_skip; // [E]
+  void *y;             // [B, L, E] gated output
+  float *h_out;        // optional [B, E, N] final state
+  float *h_in;         // optional [B, E, N] initial state (decode), else zero
+  int B, L, E, N;
+  float *chunk_ws;     // workspace for the chunked scan (see scan_workspace_floats)
+};
+size_t scan_workspace_floats(int B, int L, int E, int N, int *chunks_out);
+hymba_status selective_scan(const ScanArgs &a, hymba_dtype dt, cudaStream_t s);
+
+// ---- fused norm / beta / mean -------------------------------------------
+struct FuseArgs {
+  const void *o;       // [M, E]
+  const void *y;       // [M, E]
+  const float *beta_attn, *beta_ssm;
+  void *f;             // [M, E]
+  int M, E;
+  float eps;
+};
+hymba_status fuse_branches(const FuseArgs &a, hymba_dtype dt, cudaStream_t s);
+
+// ---- attention -----------------------------------------------------------
+struct AttnArgs {
+  const void *q;   // [B, L, H*dqk]
+  const void *k;   // [B, L, Hkv*dqk]
+  const void *v;   // [B, L, Hkv*dv]
+  void *o;         // [B, L, H*dv]
+  int B, L, H, Hkv, dqk, dv;
+  int n_meta, window, is_global;
+  float scale;
+};
+hymba_status attention_prefill(const AttnArgs &a, hymba_dtype dt, cudaStream_t s);
+
+struct KvEmitArgs {
+  const void *k_seq, *v_seq;  // [B, L, Hkv*d]
+  void *k_cache, *v_cache;    // [B, Hkv, cap, d]
+  int B, L, Hkv, dqk, dv, cap;
+  int n_meta, window, is_global;
+};
+hymba_status kv_cache_emit(const KvEmitArgs &a, hymba_dtype dt, cudaStream_t s);
+
+struct DecodeAttnArgs {
+  const void *q;             // [B, H*dqk]
+  const void *k_cache, *v_cache;  // [B, Hkv, cap, d]
+  void *o;                   // [B, H*dv]
+  float *partial;            // workspace
+  int B, H, Hkv, dqk, dv, cap;
+  long long pos;
+  int n_meta, window, is_global;
+  float scale;
+};
+size_t decode_attn_workspace_floats(int B, int H, int dv, long long pos, int n_meta, int window,
+                                    int is_global);
+hymba_status attention_decode(const DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s);
+
+struct DecodeConvArgs {
+  const void *x;       // [B, E] x_ssm of the new token, row stride ld_x
+  long long ld_x;
+  void *conv_state;    // [B, K-1, E] in/out
+  void *u;             // [B, E]
+  const float *w, *bias;
+  int B, E, K;
+};
+hymba_status decode_conv(const DecodeConvArgs &a, hymba_dtype dt, cudaStream_t s);
+
+hymba_status mask_bitmap(int L, int n_meta, int window, int is_global, uint32_t *bits,
+                         uint8_t *tile_class, cudaStream_t s);
+
+hymba_status convert_f32_to(const float *src, void *dst, long long n, hymba_dtype dt,
+                            cudaStream_t s);
+
+// Device error word bit for a bounded wait that gave up.
+constexpr unsigned kErrTimeoutHost = 1u;
+// Device error words of every translation unit: read and clear.
+unsigned take_error_gemm();
+unsigned take_error_attn();
+
+// Counts kernel launches of this library (for the optional profiler).
+void note_launch(int n = 1);
+
+// Thread-local reason for the last failure.
+void set_error(const char *fmt, ...);
+
+}  // namespace hymba

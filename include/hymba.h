@@ -1,0 +1,254 @@
+/*
+ * hymba.h — C ABI of the B200 (sm_100a) Hymba hybrid-head layer forward.
+ *
+ * The layer is the fused hybrid-head module of "Hymba: A Hybrid-head
+ * Architecture for Small Language Models" (arXiv 2411.13676), §2.1 Eq. (1)-(3):
+ * one input projection feeds an attention branch (Eq. 1) and a Mamba SSM
+ * branch (Eq. 2) in parallel; each branch is RMS-normalised, re-scaled per
+ * channel by beta, the two are averaged and projected back (Eq. 3).  Meta
+ * tokens are prepended to the input (§2.3 Eq. 4); sliding-window layers use the
+ * "A-shape" mask that always sees the meta tokens, a few layers are global, and
+ * consecutive sliding-window layers share K/V (§2.2; authors' OpenReview reply
+ * "Cache Optimization" / "Meta Tokens").
+ *
+ * Conventions for every entry point:
+ *   - Positions index X~ = [R; X]: rows 0..n_meta-1 are the meta tokens, then the
+ *     real tokens.  A sequence has L = n_meta + n_tokens rows.
+ *   - All tensor pointers are DEVICE pointers owned by the caller, row-major,
+ *     densely packed, with the layouts stated below.  The library never frees,
+ *     copies or retains them beyond the call, except that a layer handle keeps
+ *     the weight pointers given to hymba_layer_create until destroy.
+ *   - Storage dtype HYMBA_BF16: activations, K/V, conv state and the W_in, W_x,
+ *     W_out matrices are bf16 (accumulation in fp32); HYMBA_F32: all fp32.
+ *     Per-channel parameters, W_dt and the SSM state are always fp32.
+ *   - Compute calls are asynchronous on `stream`; they do not allocate, do not
+ *     synchronise and never abort.  Every argument is validated on the host
+ *     before anything is launched; a failed check launches nothing and returns
+ *     an error code (hymba_last_error() gives a one-line reason).  Device-side
+ *     faults and bounded-wait timeouts surface through hymba_stream_status().
+ *   - Device pointers and leading dimensions must be 16-byte aligned (TMA).
+ */
+#ifndef HYMBA_H_
+#define HYMBA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define HYMBA_API __attribute__((visibility("default")))
+#else
+#define HYMBA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *hymba_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  HYMBA_OK = 0,
+  HYMBA_ERR_INVALID_ARG = 1,  /* bad shape, null pointer, misaligned pointer   */
+  HYMBA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement   */
+  HYMBA_ERR_WORKSPACE = 3,    /* workspace smaller than the query returned     */
+  HYMBA_ERR_NOT_BOUND = 4,    /* K/V sharing: consumer/producer mismatch       */
+  HYMBA_ERR_CUDA = 5,         /* a CUDA runtime call failed                    */
+  HYMBA_ERR_TIMEOUT = 6,      /* a device-side bounded wait gave up            */
+  HYMBA_ERR_DEVICE = 7        /* no usable sm_100 device                       */
+} hymba_status;
+
+typedef enum { HYMBA_F32 = 0, HYMBA_BF16 = 1 } hymba_dtype;
+
+/* Layer configuration: shape, attention layout and storage dtype.
+ * Appendix E Table 11 (1.5B): d_model 1600, n_heads 25, n_kv_heads 5 ("query
+ * groups"), d_state 16, window 1024; n_meta 128 (OpenReview reply on meta-token
+ * count).  head_dim_v must equal d_inner / n_heads so the two branches have the
+ * same width in Eq. (3).  dt_rank is the rank of W_delta = W_dt W_x[:dt_rank]
+ * (Mamba's low-rank delta). */
+typedef struct {
+  int d_model;       /* d                                              */
+  int n_heads;       /* H query heads                                  */
+  int n_kv_heads;    /* Hkv; H % Hkv == 0; head h reads kv head h/(H/Hkv) */
+  int head_dim_qk;   /* d_qk (64)                                      */
+  int head_dim_v;    /* d_v = d_inner / n_heads                        */
+  int d_inner;       /* E, SSM channels                                */
+  int d_state;       /* N (16)                                         */
+  int d_conv;        /* K, causal depthwise conv width (4)             */
+  int dt_rank;       /* R                                              */
+  int n_meta;        /* m meta tokens prepended to every sequence      */
+  int window;        /* W: key j visible from query i iff i - j < W or j < m (sliding-window layers) */
+  int is_global;     /* 1: full causal attention (window ignored)      */
+  hymba_dtype dtype;
+  float rms_eps;     /* eps of the per-branch RMS norm                 */
+  float softmax_scale; /* 0 -> 1/sqrt(head_dim_qk) (OpenReview reply Q2) */
+} hymba_layer_config;
+
+/* Weights of one layer (device pointers, kept by the handle, never copied).
+ * P = H*d_qk + Hkv*(d_qk + d_v) + 2E for a layer that owns its K/V, and
+ * P = H*d_qk + 2E for a K/V-sharing consumer (no K/V rows).  Row order of W_in
+ * follows W_in_proj = [W^Q, W^K, W^V, W^SSM, W^G] (§2.1). */
+typedef struct {
+  const void  *w_in;      /* [P, d_model]                 dtype  */
+  const float *conv_w;    /* [d_inner, d_conv]; tap d_conv-1 multiplies the current row */
+  const float *conv_b;    /* [d_inner]                           */
+  const void  *w_x;       /* [dt_rank + 2*d_state, d_inner] dtype; rows: delta_r, B, C */
+  const float *w_dt;      /* [d_inner, dt_rank] fp32 (dt_rank % 4 == 0) */
+  const float *b_dt;      /* [d_inner]                           */
+  const float *a_log;     /* [d_inner, d_state]; A = -exp(a_log) */
+  const float *d_skip;    /* [d_inner] D                          */
+  const float *beta_attn; /* [d_inner] beta_1                     */
+  const float *beta_ssm;  /* [d_inner] beta_2                     */
+  const void  *w_out;     /* [d_model, d_inner]           dtype  */
+} hymba_layer_weights;
+
+typedef struct hymba_layer hymba_layer; /* opaque host handle */
+
+/* Full-length K/V of one prefill: k [batch, L, Hkv*d_qk], v [batch, L, Hkv*d_v]
+ * (token-major, as the input projection produces them).  A layer that owns its
+ * K/V writes them and stamps `owner`, `batch`, `rows`; a consumer bound with
+ * hymba_kv_share_bind reads them in place and checks the stamp. */
+typedef struct {
+  void *k;
+  void *v;
+  int batch;
+  int rows;
+  uint64_t owner;   /* set by the library; 0 = never written */
+} hymba_kv_seq;
+
+/* Decode K/V store of a layer that owns K/V: k [batch, Hkv, capacity, d_qk],
+ * v [batch, Hkv, capacity, d_v].  Slot of position p: p for meta rows
+ * (p < m) and for every row of a global layer; m + (p - m) mod W for real rows
+ * of a sliding-window layer, so capacity >= m + W (window) or >= the largest
+ * position + 1 (global).  `owner` as in hymba_kv_seq. */
+typedef struct {
+  void *k;
+  void *v;
+  int batch;
+  int capacity;
+  uint64_t owner;
+} hymba_kv_cache;
+
+/* Recurrent state of the SSM branch: h [batch, d_inner, d_state] fp32 and the
+ * last d_conv-1 rows of the SSM input x_ssm, conv [batch, d_conv-1, d_inner]
+ * (dtype; oldest row first). */
+typedef struct {
+  float *h;
+  void *conv;
+} hymba_ssm_cache;
+
+/* ---- handles ------------------------------------------------------------ */
+
+/* Validates the configuration, records it and the weight pointers.  No device
+ * work.  Returns INVALID_ARG / UNSUPPORTED with a reason on failure. */
+HYMBA_API hymba_status hymba_layer_create(const hymba_layer_config *cfg, const hymba_layer_weights *w,
+                                hymba_layer **out);
+HYMBA_API void hymba_layer_destroy(hymba_layer *layer);
+/* 1 if this handle reads another layer's K/V. */
+HYMBA_API int hymba_layer_is_consumer(const hymba_layer *layer);
+
+/* Cross-layer K/V sharing (§2.2 "Cross-layer KV sharing"): `consumer` stops
+ * projecting K/V (its W_in must have no K/V rows) and attends over the K/V
+ * written by `producer`.  Host only.  Checks that n_kv_heads, head dims,
+ * n_meta, window and is_global match, that the producer is not itself a
+ * consumer, and that the consumer's W_in width is the consumer width;
+ * returns NOT_BOUND / INVALID_ARG otherwise.  Binding twice rebinds. */
+HYMBA_API hymba_status hymba_kv_share_bind(hymba_layer *consumer, const hymba_layer *producer);
+
+/* ---- prefill ------------------------------------------------------------ */
+
+/* Bytes of device workspace hymba_layer_prefill needs for this batch/length. */
+HYMBA_API hymba_status hymba_layer_prefill_workspace(const hymba_layer *layer, int batch, int n_tokens,
+                                           size_t *bytes);
+
+/* Byte offsets inside the prefill workspace of the intermediates left there by
+ * the last prefill (row-major, M = batch*L rows).  For stage-by-stage checks. */
+typedef struct {
+  size_t q;       /* [M, H*d_qk]          dtype */
+  size_t x_ssm;   /* [M, E]               dtype */
+  size_t z;       /* [M, E]               dtype */
+  size_t u;       /* [M, E] conv+SiLU     dtype */
+  size_t xdbl;    /* [M, R+2N] fp32: delta_r, B, C */
+  size_t delta;   /* [M, E] softplus      dtype */
+  size_t y_ssm;   /* [M, E] gated scan    dtype */
+  size_t o_attn;  /* [M, E] attention     dtype */
+  size_t fused;   /* [M, E] Eq. 3 inside W_out(.)  dtype */
+  size_t total;
+} hymba_prefill_layout;
+HYMBA_API hymba_status hymba_layer_prefill_layout(const hymba_layer *layer, int batch, int n_tokens,
+                                        hymba_prefill_layout *out);
+
+/* One layer over `batch` sequences of L = n_meta + n_tokens rows.
+ *   x   [batch, L, d_model] dtype : X~ (meta rows included; the caller builds
+ *                                   [R; X] for the first layer, later layers
+ *                                   take the previous layer's output as is)
+ *   y   [batch, L, d_model] dtype : Y of Eq. (3) for every row
+ *   kv  full-length K/V: written by a layer that owns K/V (required), read by a
+ *       consumer (must carry its producer's stamp and the same batch/rows)
+ *   kv_cache  optional (NULL): a K/V owner also writes its decode store — the
+ *       meta rows and the rows of the last W positions (all rows if global);
+ *       other slots are left untouched.  Must be NULL for a consumer.
+ *   ssm_cache optional (NULL): final SSM state h_L and the last d_conv-1 x_ssm rows.
+ *   workspace >= hymba_layer_prefill_workspace() bytes, 256-byte aligned. */
+HYMBA_API hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens,
+                                 const void *x, void *y, hymba_kv_seq *kv,
+                                 hymba_kv_cache *kv_cache, hymba_ssm_cache *ssm_cache,
+                                 void *workspace, size_t workspace_bytes, hymba_stream_t stream);
+
+/* ---- decode ------------------------------------------------------------- */
+
+/* Bytes of device workspace hymba_layer_decode_step needs for positions up to max_pos. */
+HYMBA_API hymba_status hymba_layer_decode_workspace(const hymba_layer *layer, int batch, int64_t max_pos,
+                                                    size_t *bytes);
+
+/* One new token per sequence at X~ position `pos` (same for every sequence;
+ * pos >= n_meta).  x_t, y_t [batch, d_model] dtype.
+ *   kv_cache: a K/V owner appends this token's K/V at its slot and attends over
+ *     its own store; a consumer attends over its producer's store (stamp
+ *     checked), which the producer must have updated for this position first.
+ *   ssm_cache: read and updated in place (h and the conv window).
+ * A sliding-window layer attends over positions {0..m-1} and
+ * {max(m, pos-W+1)..pos}; a global layer over 0..pos. */
+HYMBA_API hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
+                                     const void *x_t, void *y_t, hymba_kv_cache *kv_cache,
+                                     hymba_ssm_cache *ssm_cache, void *workspace,
+                                     size_t workspace_bytes, hymba_stream_t stream);
+
+/* ---- status and diagnostics -------------------------------------------- */
+
+/* Synchronises `stream`, then reports a pending CUDA error or a device-side
+ * error word (e.g. a bounded wait that timed out) and clears the word. */
+HYMBA_API hymba_status hymba_stream_status(hymba_stream_t stream);
+/* Reason for the last non-OK status returned on this thread ("" if none). */
+HYMBA_API const char *hymba_last_error(void);
+HYMBA_API const char *hymba_status_string(hymba_status s);
+/* Library version, e.g. "hymba-b200 0.1 sm_100a". */
+HYMBA_API const char *hymba_version(void);
+
+/* The attention mask as the attention kernel evaluates it (same device
+ * predicate), for bit-exact checks.  bits [L, ceil(L/32)] uint32 row-major:
+ * bit j%32 of word j/32 of row i is 1 iff key j is visible from query i.
+ * tile_class (optional) [ceil(L/128), ceil(L/128)] uint8: 0 = skipped (no
+ * visible pair), 1 = fully visible, 2 = partially masked, for 128x128 tiles. */
+HYMBA_API hymba_status hymba_debug_mask_bitmap(int L, int n_meta, int window, int is_global,
+                                     uint32_t *bits, uint8_t *tile_class, hymba_stream_t stream);
+
+/* ---- optional per-kernel timing ---------------------------------------- */
+
+/* When enabled, every kernel launch issued by the compute calls (outside CUDA
+ * graph capture) is bracketed by two CUDA events on its stream; the events come
+ * from a pool created here, so enabling is not a hot call.  Disabled by default. */
+HYMBA_API hymba_status hymba_profile_enable(int on);
+typedef struct {
+  char name[32];     /* pipeline step, e.g. "in_proj", "attention", "scan" */
+  int calls;         /* times the step ran */
+  int kernels;       /* kernels it launched in total */
+  double total_ms;   /* sum of event-measured durations */
+} hymba_profile_entry;
+/* Synchronises the recorded events, accumulates them per step name and clears
+ * the record.  Writes up to `max` entries, *n = number written. */
+HYMBA_API hymba_status hymba_profile_collect(hymba_profile_entry *out, int max, int *n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYMBA_H_ */

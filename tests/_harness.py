@@ -1,0 +1,201 @@
+"""Shared helpers of the GPU parity tests: seeded inputs (synth), the C-ABI
+calls (hybrid_attention_ssm_head_b200), and the fp64 oracle on the same inputs."""
+from __future__ import annotations
+
+import math
+from dataclasses import replace
+
+import numpy as np
+import torch
+
+import hybrid_attention_ssm_head_b200 as hy
+import synth
+from oracle import hymba_oracle as O
+from synth.configs import DEFAULT_STD, Workload
+
+# The workloads' floating-point tolerances: bf16 path |g - o| <= 2e-2 + 2e-2 |o| elementwise;
+# fp32 path 1e-4 relative (elementwise against |o| + the row's rms, and per-row L2).
+BF16_ATOL, BF16_RTOL = 2e-2, 2e-2
+F32_REL = 1e-4
+
+
+def spec_of(w: Workload, is_global: bool | None = None) -> O.Spec:
+    d = w.dims
+    g = (w.window <= 0) if is_global is None else is_global
+    return O.Spec(d_model=d.d_model, n_heads=d.n_heads, n_kv_heads=d.n_kv_heads,
+                  head_dim_qk=d.head_dim_qk, head_dim_v=d.head_dim_v, d_inner=d.d_inner,
+                  d_state=d.d_state, d_conv=d.d_conv, dt_rank=d.rank, n_meta=w.n_meta,
+                  window=max(w.window, 1), is_global=g, eps=1e-6)
+
+
+def to64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def oracle_weights(wt: dict) -> dict:
+    return {k: to64(v) for k, v in wt.items()}
+
+
+class GpuLayer:
+    """One layer: seeded weights on the device and its C-ABI handle."""
+
+    def __init__(self, w: Workload, layer: int, consumer: bool = False, is_global: bool | None = None,
+                 std=DEFAULT_STD, tag: str = "", device="cuda"):
+        self.workload = w
+        self.is_global = (w.window <= 0) if is_global is None else is_global
+        self.consumer = consumer
+        cpu = synth.configs.layer_weights(w, layer, consumer=consumer, std=std, tag=tag)
+        self.cpu = cpu
+        self.dev = {k: v.to(device).contiguous() for k, v in cpu.items()}
+        d = w.dims
+        self.cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner,
+                                  d.d_state, d.d_conv, d.rank, w.n_meta, w.window,
+                                  self.is_global, w.dtype)
+        self.handle = hy.hymba_layer_create(self.cfg, hy.make_weights(self.dev))
+        self.spec = spec_of(w, self.is_global)
+
+    def close(self):
+        if self.handle:
+            hy.hymba_layer_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def torch_dt(w: Workload):
+    return synth.configs.torch_dtype(w.dtype)
+
+
+def alloc_kv_seq(w: Workload, batch: int, L: int, device="cuda"):
+    d = w.dims
+    k = torch.zeros(batch, L, d.n_kv_heads * d.head_dim_qk, dtype=torch_dt(w), device=device)
+    v = torch.zeros(batch, L, d.n_kv_heads * d.head_dim_v, dtype=torch_dt(w), device=device)
+    return k, v, hy.hymba_kv_seq(k.data_ptr(), v.data_ptr(), 0, 0, 0)
+
+
+def alloc_ssm_cache(w: Workload, batch: int, device="cuda"):
+    d = w.dims
+    h = torch.zeros(batch, d.d_inner, d.d_state, dtype=torch.float32, device=device)
+    conv = torch.zeros(batch, d.d_conv - 1, d.d_inner, dtype=torch_dt(w), device=device)
+    return h, conv, hy.hymba_ssm_cache(h.data_ptr(), conv.data_ptr())
+
+
+def alloc_kv_cache(w: Workload, batch: int, capacity: int, device="cuda"):
+    d = w.dims
+    k = torch.zeros(batch, d.n_kv_heads, capacity, d.head_dim_qk, dtype=torch_dt(w), device=device)
+    v = torch.zeros(batch, d.n_kv_heads, capacity, d.head_dim_v, dtype=torch_dt(w), device=device)
+    return k, v, hy.hymba_kv_cache(k.data_ptr(), v.data_ptr(), batch, capacity, 0)
+
+
+def workspace(nbytes: int, device="cuda"):
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def run_prefill(layer: GpuLayer, x: torch.Tensor, kv, kv_cache=None, ssm_cache=None, ws=None):
+    w = layer.workload
+    B, L = x.shape[0], x.shape[1]
+    n = L - w.n_meta
+    y = torch.empty_like(x)
+    need = hy.hymba_layer_prefill_workspace(layer.handle, B, n)
+    if ws is None or ws.numel() < need:
+        ws = workspace(need)
+    hy.hymba_layer_prefill(layer.handle, B, n, x, y, kv, kv_cache, ssm_cache, ws, ws.numel(),
+                           torch.cuda.current_stream())
+    hy.hymba_stream_status(torch.cuda.current_stream())
+    return y, ws
+
+
+def stage(layer: GpuLayer, ws: torch.Tensor, B: int, L: int, name: str) -> torch.Tensor:
+    """A stage's intermediate from the prefill workspace, [B, L, width]."""
+    w = layer.workload
+    lay = hy.hymba_layer_prefill_layout(layer.handle, B, L - w.n_meta)
+    d = w.dims
+    widths = dict(q=d.n_heads * d.head_dim_qk, x_ssm=d.d_inner, z=d.d_inner, u=d.d_inner,
+                  xdbl=d.xproj_width, delta=d.d_inner, y_ssm=d.d_inner, o_attn=d.d_inner,
+                  fused=d.d_inner)
+    dt = torch.float32 if name == "xdbl" else torch_dt(w)
+    es = 4 if dt == torch.float32 else 2
+    off = getattr(lay, name)
+    n = B * L * widths[name]
+    return ws[off:off + n * es].view(dt).view(B, L, widths[name])
+
+
+def close_bf16(g, o, what="", frac_ok=1.0):
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    err = np.abs(g - o)
+    bound = BF16_ATOL + BF16_RTOL * np.abs(o)
+    bad = err > bound
+    if bad.any():
+        idx = np.unravel_index(np.argmax(err - bound), err.shape)
+        raise AssertionError(
+            f"{what}: {bad.sum()} of {bad.size} elements outside 2e-2 + 2e-2|o|; worst at {idx}: "
+            f"gpu {g[idx]:.6g} oracle {o[idx]:.6g}; max |err| {err.max():.3g}")
+
+
+def close_stage(g, o, what=""):
+    """Stage check: the bf16 bound applied to the stage normalised by its rms, so that
+    stages of very different scale (u ~ 1e-2, h ~ 1e-5) are held to the same relative
+    accuracy: |g - o| <= 2e-2 rms(o) + 2e-2 |o|."""
+    o = np.asarray(o, dtype=np.float64)
+    s = float(np.sqrt((o ** 2).mean())) or 1.0
+    close_bf16(np.asarray(g, dtype=np.float64) / s, o / s, what + f" (scaled by rms {s:.3g})")
+
+
+class Checks:
+    """Collects every failed comparison of a test, then fails once with all of them."""
+
+    def __init__(self):
+        self.errors = []
+
+    def __call__(self, fn, *a, **k):
+        try:
+            fn(*a, **k)
+        except AssertionError as e:
+            self.errors.append(str(e).split("\n")[0])
+
+    def done(self):
+        if self.errors:
+            raise AssertionError("\n".join(self.errors))
+
+
+def diag_dump(name: str, arrays: dict):
+    """With HYMBA_DIAG_DIR set, save GPU-side arrays for offline inspection."""
+    import os
+    d = os.environ.get("HYMBA_DIAG_DIR")
+    if not d:
+        return
+    os.makedirs(d, exist_ok=True)
+    np.savez_compressed(os.path.join(d, name + ".npz"),
+                        **{k: np.asarray(v, dtype=np.float32) for k, v in arrays.items()})
+
+
+def close_f32(g, o, what=""):
+    g = np.asarray(g, dtype=np.float64)
+    o = np.asarray(o, dtype=np.float64)
+    g2 = g.reshape(-1, g.shape[-1])
+    o2 = o.reshape(-1, o.shape[-1])
+    rms = np.sqrt((o2 ** 2).mean(axis=1, keepdims=True))
+    err = np.abs(g2 - o2)
+    bound = F32_REL * (np.abs(o2) + rms)
+    assert (err <= bound).all(), f"{what}: elementwise {(err > bound).sum()} bad; max err {err.max():.3g}"
+    rel = np.linalg.norm(g2 - o2, axis=1) / np.maximum(np.linalg.norm(o2, axis=1), 1e-300)
+    assert (rel <= F32_REL).all(), f"{what}: row L2 rel err {rel.max():.3g}"
+
+
+def close(w: Workload, g, o, what=""):
+    if w.dtype == "f32":
+        close_f32(g, o, what)
+    else:
+        close_bf16(g, o, what)
+
+
+def small_workload(name, dtype="bf16", batch=2, n_meta=128, n_tokens=300, window=256, dims=None,
+                   seed=0):
+    from synth.configs import DIMS_1P5B, DIMS_SMALL
+    dims = dims or (DIMS_1P5B if dtype == "bf16" else DIMS_SMALL)
+    return Workload(name, dims, dtype, batch, n_meta, n_tokens, window, seed=seed)

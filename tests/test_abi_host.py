@@ -1,0 +1,168 @@
+"""The C-ABI library: it loads, exports every function include/hymba.h declares,
+and rejects bad arguments on the host before touching a device (CPU only)."""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import hybrid_attention_ssm_head_b200 as hy
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "hymba.h")).read()
+    return sorted(set(re.findall(r"HYMBA_API\s+[\w\s\*]*?\b(hymba_\w+)\s*\(", src)))
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = hy.lib()
+    declared = _declared_functions()
+    assert len(declared) >= 14
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(hy.EXPORTED) == declared
+    assert "sm_100a" in hy.hymba_version()
+
+
+def _cfg(**kw):
+    base = dict(d_model=1600, n_heads=25, n_kv_heads=5, head_dim_qk=64, d_inner=3200, d_state=16,
+                d_conv=4, dt_rank=100, n_meta=128, window=1024, is_global=False, dtype="bf16")
+    base.update(kw)
+    return hy.make_config(**base)
+
+
+def _fake_weights(addr=1 << 40):
+    # aligned, non-null fake device addresses: creation never dereferences them
+    return hy.hymba_layer_weights(*[addr + 4096 * i for i in range(11)])
+
+
+def test_create_validates_configuration():
+    h = hy.hymba_layer_create(_cfg(), _fake_weights())
+    assert h and not hy.hymba_layer_is_consumer(h)
+    hy.hymba_layer_destroy(h)
+    bad = [
+        (dict(n_kv_heads=4), hy.HYMBA_ERR_INVALID_ARG),        # 25 % 4 != 0
+        (dict(d_state=8), hy.HYMBA_ERR_UNSUPPORTED),
+        (dict(dt_rank=101), hy.HYMBA_ERR_UNSUPPORTED),
+        (dict(window=0), hy.HYMBA_ERR_INVALID_ARG),
+        (dict(head_dim_qk=32), hy.HYMBA_ERR_UNSUPPORTED),     # bf16 attention kernel shape
+        (dict(d_conv=5), hy.HYMBA_ERR_UNSUPPORTED),
+    ]
+    for kw, want in bad:
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_create(_cfg(**kw), _fake_weights())
+        assert e.value.status == want, (kw, e.value)
+    cfg = _cfg()
+    cfg.head_dim_v = 64  # branch widths differ: Eq. 3 cannot add them
+    with pytest.raises(hy.HymbaError) as e:
+        hy.hymba_layer_create(cfg, _fake_weights())
+    assert e.value.status == hy.HYMBA_ERR_INVALID_ARG
+    w = _fake_weights()
+    w.w_out = None
+    with pytest.raises(hy.HymbaError):
+        hy.hymba_layer_create(_cfg(), w)
+    w = _fake_weights()
+    w.w_x = (1 << 40) + 8  # misaligned
+    with pytest.raises(hy.HymbaError):
+        hy.hymba_layer_create(_cfg(), w)
+
+
+def test_kv_share_bind_checks_compatibility():
+    p = hy.hymba_layer_create(_cfg(), _fake_weights())
+    c = hy.hymba_layer_create(_cfg(), _fake_weights(1 << 41))
+    other = hy.hymba_layer_create(_cfg(window=512), _fake_weights(1 << 42))
+    glob = hy.hymba_layer_create(_cfg(is_global=True), _fake_weights(1 << 43))
+    try:
+        for prod in (other, glob, c):
+            with pytest.raises(hy.HymbaError) as e:
+                hy.hymba_kv_share_bind(c, prod)
+            assert e.value.status == hy.HYMBA_ERR_NOT_BOUND
+        hy.hymba_kv_share_bind(c, p)
+        assert hy.hymba_layer_is_consumer(c)
+        with pytest.raises(hy.HymbaError) as e:  # a consumer cannot produce
+            hy.hymba_kv_share_bind(other, c)
+        assert e.value.status == hy.HYMBA_ERR_NOT_BOUND
+    finally:
+        for h in (p, c, other, glob):
+            hy.hymba_layer_destroy(h)
+
+
+def test_prefill_rejects_bad_arguments_before_launch():
+    p = hy.hymba_layer_create(_cfg(), _fake_weights())
+    c = hy.hymba_layer_create(_cfg(), _fake_weights(1 << 41))
+    hy.hymba_kv_share_bind(c, p)
+    A = 1 << 44
+    B, n = 2, 300
+    ws = hy.hymba_layer_prefill_workspace(p, B, n)
+    lay = hy.hymba_layer_prefill_layout(p, B, n)
+    assert lay.total == ws and lay.q == 0
+    offs = [lay.q, lay.x_ssm, lay.z, lay.u, lay.xdbl, lay.delta, lay.y_ssm, lay.o_attn, lay.fused]
+    assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
+    M = B * (128 + n)
+    assert lay.x_ssm - lay.q >= M * 1600 * 2 and lay.delta - lay.xdbl >= M * 132 * 4
+    kv = hy.hymba_kv_seq(A, A + (1 << 30), 0, 0, 0)
+    try:
+        # workspace too small
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_prefill(p, B, n, A, A, kv, None, None, A, ws - 256)
+        assert e.value.status == hy.HYMBA_ERR_WORKSPACE
+        # consumer before its producer wrote the K/V
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_prefill(c, B, n, A, A, kv, None, None, A, ws)
+        assert e.value.status == hy.HYMBA_ERR_NOT_BOUND
+        # a stamp from another layer is refused too
+        kv.owner, kv.batch, kv.rows = 987654, B, 128 + n
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_prefill(c, B, n, A, A, kv, None, None, A, ws)
+        assert e.value.status == hy.HYMBA_ERR_NOT_BOUND
+        # misaligned input, null kv, bad batch, small decode store
+        for args in [(p, B, n, A + 2, A, kv, None, None, A, ws),
+                     (p, 0, n, A, A, kv, None, None, A, ws)]:
+            with pytest.raises(hy.HymbaError) as e:
+                hy.hymba_layer_prefill(*args)
+            assert e.value.status == hy.HYMBA_ERR_INVALID_ARG
+        small = hy.hymba_kv_cache(A, A, B, 128 + 1023, 0)
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_prefill(p, B, n, A, A, kv, small, None, A, ws)
+        assert e.value.status == hy.HYMBA_ERR_INVALID_ARG
+    finally:
+        hy.hymba_layer_destroy(p)
+        hy.hymba_layer_destroy(c)
+
+
+def test_decode_rejects_bad_arguments_before_launch():
+    p = hy.hymba_layer_create(_cfg(), _fake_weights())
+    c = hy.hymba_layer_create(_cfg(), _fake_weights(1 << 41))
+    hy.hymba_kv_share_bind(c, p)
+    A = 1 << 44
+    ws = hy.hymba_layer_decode_workspace(p, 4, 2000)
+    kvc = hy.hymba_kv_cache(A, A, 4, 128 + 1024, 0)
+    ssm = hy.hymba_ssm_cache(A, A)
+    try:
+        with pytest.raises(hy.HymbaError) as e:  # meta position
+            hy.hymba_layer_decode_step(p, 4, 5, A, A, kvc, ssm, A, ws)
+        assert e.value.status == hy.HYMBA_ERR_INVALID_ARG
+        with pytest.raises(hy.HymbaError) as e:  # consumer with an unstamped store
+            hy.hymba_layer_decode_step(c, 4, 2000, A, A, kvc, ssm, A, ws)
+        assert e.value.status == hy.HYMBA_ERR_NOT_BOUND
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_decode_step(p, 4, 2000, A, A, kvc, ssm, A, 64)
+        assert e.value.status == hy.HYMBA_ERR_WORKSPACE
+        kvc.capacity = 100
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_decode_step(p, 4, 2000, A, A, kvc, ssm, A, ws)
+        assert e.value.status == hy.HYMBA_ERR_INVALID_ARG
+    finally:
+        hy.hymba_layer_destroy(p)
+        hy.hymba_layer_destroy(c)
+
+
+def test_mask_bitmap_rejects_bad_shape():
+    with pytest.raises(hy.HymbaError):
+        hy.hymba_debug_mask_bitmap(0, 0, 4, False, 1 << 44)
+    with pytest.raises(hy.HymbaError):
+        hy.hymba_debug_mask_bitmap(10, 0, 0, False, 1 << 44)
