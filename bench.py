@@ -402,6 +402,8 @@ def run_ours(args, rank, world, dev):
         "roofline": roof,
         "steps_profile": {n: {"calls": c, "kernels": k, "ms_per_call": ms / c if c else None}
                           for n, c, k, ms in prof},
+        "decode_steps_profile": {n: {"calls": c, "kernels": k, "ms_per_call": ms / c if c else None}
+                                 for n, c, k, ms in dprof},
         "gpu_launches": pre_launches + dec_kernels_per_step * args.steps,
         "clocks": clocks,
         "e2e": e2e,
@@ -470,6 +472,46 @@ def run_reference(args, rank, world):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_case(args, dev):
+    """A smaller workload for profiling: one prefill layer of the given config, or the decode
+    stack alone; prints the per-step profile."""
+    import hybrid_attention_ssm_head_b200 as hy
+    import synth
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    if args.case == "decode":
+        dec = Decode(synth.configs.CFG4, dev)
+        run = lambda: dec.run(stream)  # noqa: E731
+    else:
+        w = {"cfg1": synth.configs.CFG1, "cfg2": synth.configs.CFG2}[args.case]
+        d = w.dims
+        wt = {k: v.contiguous() for k, v in synth.configs.layer_weights(w, 0, device=dev).items()}
+        cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner, d.d_state,
+                             d.d_conv, d.rank, w.n_meta, w.window, w.window <= 0, "bf16")
+        h = hy.hymba_layer_create(cfg, hy.make_weights(wt))
+        B, L = w.batch, w.seq_rows
+        x = synth.configs.x_tilde(w, device=dev)
+        y = torch.empty_like(x)
+        k = torch.empty(B, L, d.n_kv_heads * d.head_dim_qk, dtype=torch.bfloat16, device=dev)
+        v = torch.empty(B, L, d.n_kv_heads * d.head_dim_v, dtype=torch.bfloat16, device=dev)
+        kv = hy.hymba_kv_seq(k.data_ptr(), v.data_ptr(), 0, 0, 0)
+        ws = torch.empty(hy.hymba_layer_prefill_workspace(h, B, w.n_tokens), dtype=torch.uint8, device=dev)
+        run = lambda: hy.hymba_layer_prefill(h, B, w.n_tokens, x, y, kv, None, None, ws,  # noqa: E731
+                                             ws.numel(), stream)
+    for _ in range(args.warmup):
+        run()
+    hy.hymba_stream_status(stream)
+    hy.hymba_profile_enable(True)
+    hy.hymba_profile_collect()
+    for _ in range(args.steps):
+        run()
+    prof = hy.hymba_profile_collect()
+    hy.hymba_profile_enable(False)
+    hy.hymba_stream_status(stream)
+    print(json.dumps({"case": args.case, "steps": args.steps, "profile": {
+        n: {"calls": c, "kernels": kk, "ms_per_call": ms / c} for n, c, kk, ms in prof}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -478,6 +520,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", choices=["headline", "cfg1", "cfg2", "decode"], default="headline",
+                    help="headline: the benchmark; others: a smaller run for profiling")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -492,6 +536,9 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                              device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
+    if args.case != "headline":
+        run_case(args, dev)
+        return
     out = run_ours(args, rank, world, dev)
     if out is not None:
         print(json.dumps(out), flush=True)

@@ -1,8 +1,8 @@
 // Fusion of the two branches (Hymba §2.1 Eq. 3): each branch output is
 // RMS-normalised over its d_inner channels, re-scaled per channel by beta and
 // the two are averaged:  f = (beta_1 * o / rms(o) + beta_2 * y / rms(y)) / 2.
-// One CTA per token row; 16-byte vector loads; the second pass re-reads the
-// row from L1/L2, so HBM sees each input once.
+// One CTA per token row; 16-byte vector loads held in registers across the
+// row reduction, so each input is read once.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -25,8 +25,68 @@ __device__ __forceinline__ void ld16(const T *p, float (&v)[16 / sizeof(T)]) {
   }
 }
 
+// Single read: each of the 128 threads keeps up to NV 16-byte vectors of both
+// branches in registers across the block reduction.
+template <typename T, int NV>
+__global__ void __launch_bounds__(128) fuse_kernel(FuseArgs a) {
+  constexpr int V = 16 / sizeof(T);
+  __shared__ float red[2][4];
+  const long long row = blockIdx.x;
+  const T *o = reinterpret_cast<const T *>(a.o) + row * a.E;
+  const T *y = reinterpret_cast<const T *>(a.y) + row * a.E;
+  T *f = reinterpret_cast<T *>(a.f) + row * a.E;
+  float vo[NV][V], vy[NV][V];
+  float so = 0.f, sy = 0.f;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int c = (threadIdx.x + j * 128) * V;
+    if (c < a.E) {
+      ld16<T>(o + c, vo[j]);
+      ld16<T>(y + c, vy[j]);
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        so = fmaf(vo[j][i], vo[j][i], so);
+        sy = fmaf(vy[j][i], vy[j][i], sy);
+      }
+    }
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) {
+    so += __shfl_xor_sync(0xffffffffu, so, off);
+    sy += __shfl_xor_sync(0xffffffffu, sy, off);
+  }
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    red[0][w] = so;
+    red[1][w] = sy;
+  }
+  __syncthreads();
+  so = red[0][0] + red[0][1] + red[0][2] + red[0][3];
+  sy = red[1][0] + red[1][1] + red[1][2] + red[1][3];
+  const float ro = 0.5f * rsqrtf(so / a.E + a.eps);
+  const float ry = 0.5f * rsqrtf(sy / a.E + a.eps);
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int c = (threadIdx.x + j * 128) * V;
+    if (c < a.E) {
+      float out[V];
+#pragma unroll
+      for (int i = 0; i < V; ++i)
+        out[i] = fmaf(__ldg(a.beta_attn + c + i) * ro, vo[j][i], __ldg(a.beta_ssm + c + i) * ry * vy[j][i]);
+      if constexpr (sizeof(T) == 2) {
+        st_global_v4(f + c, pack_bf16x2(out[0], out[1]), pack_bf16x2(out[2], out[3]),
+                     pack_bf16x2(out[4], out[5]), pack_bf16x2(out[6], out[7]));
+      } else {
+        st_global_v4(f + c, __float_as_uint(out[0]), __float_as_uint(out[1]),
+                     __float_as_uint(out[2]), __float_as_uint(out[3]));
+      }
+    }
+  }
+}
+
+// Rows wider than the register path: two passes, the second from L1/L2.
 template <typename T>
-__global__ void __launch_bounds__(256) fuse_kernel(FuseArgs a) {
+__global__ void __launch_bounds__(256) fuse_wide_kernel(FuseArgs a) {
   constexpr int V = 16 / sizeof(T);
   __shared__ float red[2][8];
   const long long row = blockIdx.x;
@@ -82,10 +142,19 @@ __global__ void __launch_bounds__(256) fuse_kernel(FuseArgs a) {
 
 hymba_status fuse_branches(const FuseArgs &a, hymba_dtype dt, cudaStream_t s) {
   if (a.M == 0) return HYMBA_OK;
-  if (dt == HYMBA_BF16)
-    fuse_kernel<__nv_bfloat16><<<a.M, 256, 0, s>>>(a);
-  else
-    fuse_kernel<float><<<a.M, 256, 0, s>>>(a);
+  const int V = dt == HYMBA_BF16 ? 8 : 4;
+  const bool regs = a.E <= 128 * V * 4;
+  if (dt == HYMBA_BF16) {
+    if (regs)
+      fuse_kernel<__nv_bfloat16, 4><<<a.M, 128, 0, s>>>(a);
+    else
+      fuse_wide_kernel<__nv_bfloat16><<<a.M, 256, 0, s>>>(a);
+  } else {
+    if (regs)
+      fuse_kernel<float, 4><<<a.M, 128, 0, s>>>(a);
+    else
+      fuse_wide_kernel<float><<<a.M, 256, 0, s>>>(a);
+  }
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -8,7 +8,8 @@
 //   warp 1   : TMEM allocator and MMA issuer (one lane): per 128-byte K block,
 //              4 x tcgen05.mma (M=128, N=BN, K=32 bytes) into one of two fp32
 //              accumulators in tensor memory, then tcgen05.commit frees the stage.
-//   warps 2-5: epilogue, one thread per accumulator row: tcgen05.ld, bias /
+//   warps 2-9: epilogue, one thread per accumulator row (two warps per TMEM
+//              lane quarter, alternate 16-column chunks): tcgen05.ld, bias /
 //              softplus, fp32 -> bf16, routed stores (one GEMM writes Q, K, V,
 //              x_ssm and z to their own buffers).  The second accumulator lets
 //              the epilogue of tile i overlap the MMAs of tile i+1.
@@ -34,9 +35,10 @@ __device__ __forceinline__ int find_seg(const Epilogue &e, int n) {
   return s;
 }
 
+// Bias and activation of the fp32 CUDA-core path (full-precision softplus).
 __device__ __forceinline__ float epi_act(const Epilogue &e, int n, float v) {
   if (e.bias) v += __ldg(e.bias + n);
-  if (e.act == 1) v = softplus_f(v);
+  if (e.act == 1) v = softplus_accurate(v);
   return v;
 }
 
@@ -81,6 +83,58 @@ __device__ __forceinline__ void epi_store8(const Epilogue &e, long long m, int n
     if (n + i < N) epi_store_scalar(e, m, n + i, v[i]);
 }
 
+// 16 consecutive product columns n0..n0+15 of row m from raw fp32 accumulator bits.
+// One segment lookup and one bias fetch per chunk on the common path.
+__device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, int n0, int N,
+                                            const uint32_t (&r)[16]) {
+  float v[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  const bool full = n0 + 16 <= N;
+  if (!e.atomic) {
+    if (e.bias) {
+      if (full) {
+        const float4 *bp = reinterpret_cast<const float4 *>(e.bias + n0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 b4 = __ldg(bp + q);
+          v[4 * q] += b4.x;
+          v[4 * q + 1] += b4.y;
+          v[4 * q + 2] += b4.z;
+          v[4 * q + 3] += b4.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          if (n0 + i < N) v[i] += __ldg(e.bias + n0 + i);
+      }
+    }
+    if (e.act == 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = softplus_f(v[i]);
+    }
+  }
+  float a[8], b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    a[i] = v[i];
+    b[i] = v[8 + i];
+  }
+  epi_store8(e, m, n0, N, a);
+  epi_store8(e, m, n0 + 8, N, b);
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05 GEMM
 // ---------------------------------------------------------------------------
@@ -101,7 +155,7 @@ struct TcCfg {
 };
 
 template <int BN, int ELEM>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int M, int N, int K, int ksplit, Epilogue epi) {
   using C = TcCfg<BN, ELEM>;
@@ -130,7 +184,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], 256);
     }
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -233,8 +287,10 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
   } else {
-    // ---------------- epilogue: warps 2..5, one thread per accumulator row ----------------
+    // ---------------- epilogue: warps 2..9, one thread per accumulator row ----------------
+    // Warps w and w+4 share a TMEM lane quarter and take alternate 16-column chunks.
     const int quarter = warp & 3;  // TMEM lanes this warp may access
+    const int half = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -249,38 +305,13 @@ __global__ void __launch_bounds__(192, 1)
       const long long m = (long long)mt * C::BM + row;
       const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        if (c + 32 <= BN) {
-          tmem_ld32(t_row + c, r);
-        } else {
-          // BN % 32 == 16: last 16 columns (the remaining registers are unused)
-          asm volatile(
-              "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-              "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-              : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
-                "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-              : "r"(t_row + c)
-              : "memory");
-        }
+      for (int c = half * 16; c < BN; c += 32) {
+        const int n0 = nt * BN + c;
+        if (n0 >= N) break;  // uniform across the warp
+        uint32_t r[16];
+        tmem_ld16(t_row + c, r);
         tmem_wait_ld();
-        if (m < M) {
-          const int ncols = min(32, BN - c);
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            if (h * 8 >= ncols) break;
-            const int n = nt * BN + c + h * 8;
-            float v[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const int nn = min(n + i, N - 1);
-              const float raw = __uint_as_float(r[h * 8 + i]);
-              v[i] = epi.atomic ? raw : epi_act(epi, nn, raw);
-            }
-            epi_store8(epi, m, n, N, v);
-          }
-        }
+        if (m < M) epi_store16(epi, m, n0, N, r);
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -334,7 +365,7 @@ static hymba_status launch_tc(const GemmArgs &g, cudaStream_t s) {
   if (!make_tmap(&tb, g.B, dt, 2, db, sb, bb)) return HYMBA_ERR_CUDA;
   const long long tiles = (long long)((g.M + 127) / 128) * ((g.N + BN - 1) / BN) * g.ksplit;
   const int grid = (int)std::min<long long>(tiles, num_sms());
-  gemm_tc_kernel<BN, ELEM><<<grid, 192, C::SMEM, s>>>(ta, tb, g.M, g.N, g.K, g.ksplit, g.epi);
+  gemm_tc_kernel<BN, ELEM><<<grid, 320, C::SMEM, s>>>(ta, tb, g.M, g.N, g.K, g.ksplit, g.epi);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -67,11 +67,15 @@ __device__ __forceinline__ void store_vec(T *p, const float (&v)[Vec16<T>::N]) {
   *reinterpret_cast<uint4 *>(p) = raw;
 }
 
-constexpr int kConvTB = 16;
+constexpr int kConvTB = 8;
 
+// One thread: VEC channels x kConvTB rows.  The kConvTB + 3 input rows it needs are
+// loaded up front (16-byte vectors, coalesced across the warp) so that all loads
+// are in flight together.
 template <typename T>
-__global__ void conv_silu_kernel(ConvArgs a) {
+__global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
   constexpr int V = Vec16<T>::N;
+  constexpr int NR = kConvTB + 3;
   const int nvec = a.E / V;
   const int tblocks = (a.L + kConvTB - 1) / kConvTB;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -82,6 +86,19 @@ __global__ void conv_silu_kernel(ConvArgs a) {
   const int b = int(rest / tblocks);
   const int c0 = cv * V;
   const int K = a.K;
+  const T *x = reinterpret_cast<const T *>(a.x);
+  T *u = reinterpret_cast<T *>(a.u);
+  const int t0 = tb * kConvTB;
+  // raw[r] = x[t0 - 3 + r] (zero outside the sequence)
+  uint4 raw[NR];
+#pragma unroll
+  for (int r = 0; r < NR; ++r) {
+    const int t = t0 - 3 + r;
+    if (t >= 0 && t < a.L)
+      raw[r] = __ldg(reinterpret_cast<const uint4 *>(x + ((long long)b * a.L + t) * a.ld_x + c0));
+    else
+      raw[r] = make_uint4(0, 0, 0, 0);
+  }
   float w[4][V], bias[V];
 #pragma unroll
   for (int i = 0; i < V; ++i) {
@@ -89,47 +106,38 @@ __global__ void conv_silu_kernel(ConvArgs a) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) w[k][i] = k < K ? a.w[(c0 + i) * K + k] : 0.f;
   }
-  const T *x = reinterpret_cast<const T *>(a.x);
-  T *u = reinterpret_cast<T *>(a.u);
-  const int t0 = tb * kConvTB, t1 = min(a.L, t0 + kConvTB);
-  // hist[2] = x[t-1], hist[1] = x[t-2], hist[0] = x[t-3] (zero before the sequence)
-  float hist[3][V];
+  auto val = [&](int r, int i) -> float {
+    if constexpr (sizeof(T) == 2) {
+      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw[r]);
+      return (i & 1) ? __high2float(h[i >> 1]) : __low2float(h[i >> 1]);
+    } else {
+      return reinterpret_cast<const float *>(&raw[r])[i];
+    }
+  };
 #pragma unroll
-  for (int d = 1; d <= 3; ++d) {
-    const int t = t0 - d;
-    if (t >= 0)
-      load_vec<T>(x + ((long long)b * a.L + t) * a.ld_x + c0, hist[3 - d]);
-    else
-#pragma unroll
-      for (int i = 0; i < V; ++i) hist[3 - d][i] = 0.f;
-  }
-  for (int t = t0; t < t1; ++t) {
-    float cur[V], o[V];
-    load_vec<T>(x + ((long long)b * a.L + t) * a.ld_x + c0, cur);
+  for (int tt = 0; tt < kConvTB; ++tt) {
+    const int t = t0 + tt;
+    if (t >= a.L) break;
+    float o[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) {
-      // tap k multiplies x[t - (K-1) + k]
-      float acc = bias[i] + w[K - 1][i] * cur[i];
-      if (K >= 2) acc = fmaf(w[K - 2][i], hist[2][i], acc);
-      if (K >= 3) acc = fmaf(w[K - 3][i], hist[1][i], acc);
-      if (K >= 4) acc = fmaf(w[K - 4][i], hist[0][i], acc);
+      // tap k multiplies x[t - (K-1) + k] = raw[tt + 3 - (K-1) + k]
+      float acc = bias[i];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        if (k < K) acc = fmaf(w[k][i], val(tt + 4 - K + k, i), acc);
       o[i] = silu_f(acc);
     }
     store_vec<T>(u + ((long long)b * a.L + t) * a.E + c0, o);
-#pragma unroll
-    for (int i = 0; i < V; ++i) {
-      hist[0][i] = hist[1][i];
-      hist[1][i] = hist[2][i];
-      hist[2][i] = cur[i];
-    }
   }
-  if (a.conv_state && t1 == a.L) {
-    // the last K-1 rows of x, oldest first (hist holds rows L-3, L-2, L-1)
+  if (a.conv_state && t0 + kConvTB >= a.L) {
+    // the last K-1 rows of x, oldest first: x[L-K+1 .. L-1] = raw[L-K+1 - t0 + 3 ..]
     T *cs = reinterpret_cast<T *>(a.conv_state);
     for (int r = 0; r < K - 1; ++r) {
+      const int rr = a.L - (K - 1) + r - t0 + 3;
       float v[V];
 #pragma unroll
-      for (int i = 0; i < V; ++i) v[i] = hist[3 - (K - 1) + r][i];
+      for (int i = 0; i < V; ++i) v[i] = (rr >= 0 && rr < NR) ? val(rr, i) : 0.f;
       store_vec<T>(cs + ((long long)b * (K - 1) + r) * a.E + c0, v);
     }
   }

@@ -32,21 +32,21 @@ def _check_prefill(w, lay, x, y, ws, k, v, h=None, conv=None, rows=(0,), stages=
         if stages:
             for name, key in STAGES:
                 got[key] = H.to64(H.stage(lay, ws, B, L, name)[b])
-                chk(H.close_stage, got[key], ref[key], f"{name}[b={b}]")
+                chk(H.close_stage_dist, got[key], ref[key], f"{name}[b={b}]")
             xd = H.to64(H.stage(lay, ws, B, L, "xdbl")[b])
             R = lay.spec.dt_rank
             got["B"], got["C"] = xd[:, R:R + 16], xd[:, R + 16:]
-            chk(H.close_stage, got["B"], ref["B"], "B")
-            chk(H.close_stage, got["C"], ref["C"], "C")
+            chk(H.close_stage_dist, got["B"], ref["B"], "B")
+            chk(H.close_stage_dist, got["C"], ref["C"], "C")
             if kv_from is None:
-                chk(H.close_stage, H.to64(k[b]), ref["k"], "k")
-                chk(H.close_stage, H.to64(v[b]), ref["v"], "v")
+                chk(H.close_stage_dist, H.to64(k[b]), ref["k"], "k")
+                chk(H.close_stage_dist, H.to64(v[b]), ref["v"], "v")
         got["Y"] = H.to64(y[b])
         chk(H.close_bf16, got["Y"], ref["Y"], f"Y[b={b}]")
         if h is not None:
             got["h"], got["conv"] = H.to64(h[b]), H.to64(conv[b])
-            chk(H.close_stage, got["h"], ref["h"], "h_final")
-            chk(H.close_stage, got["conv"], ref["conv"], "conv_state")
+            chk(H.close_stage_dist, got["h"], ref["h"], "h_final")
+            chk(H.close_stage_dist, got["conv"], ref["conv"], "conv_state")
         if diag and chk.errors:
             H.diag_dump(f"{diag}_b{b}", got)
         chk.done()
@@ -85,23 +85,28 @@ def test_bf16_scan_stress_parity():
 
 
 def test_bf16_kv_shared_pair():
+    """Layer 2 attends over layer 1's K/V and projects none of its own.  Strict parity with
+    an independent seeded input for each layer; the chained case (layer 2 fed layer 1's
+    bf16 output) against the two-layer bound."""
     w = H.small_workload("t_bf16_pair_b2_n300", window=256)
     prod = H.GpuLayer(w, 0)
     cons = H.GpuLayer(w, 1, consumer=True)
     hy.hymba_kv_share_bind(cons.handle, prod.handle)
     B, L = w.batch, w.seq_rows
     x = synth.configs.x_tilde(w).cuda()
+    x2 = synth.gen.normal_tensor((B, L, w.dims.d_model), 0, "t_bf16_pair/x2", device="cuda").to(torch.bfloat16)
     k, v, kv = H.alloc_kv_seq(w, B, L)
     y1, ws = H.run_prefill(prod, x, kv)
-    y2, ws = H.run_prefill(cons, y1, kv, ws=ws)
+    y2, ws = H.run_prefill(cons, x2, kv, ws=ws)
+    y2c, ws = H.run_prefill(cons, y1, kv, ws=ws)
     for b in range(B):
         ref1 = O.layer_prefill(H.to64(x[b]), H.oracle_weights(prod.cpu), prod.spec)
         H.close_bf16(H.to64(y1[b]), ref1["Y"], "producer Y")
-        # the consumer's input is the producer's output: the oracle uses its own
-        ref2 = O.layer_prefill(ref1["Y"], H.oracle_weights(cons.cpu), cons.spec, kv_from=ref1)
-        if os.environ.get("HYMBA_DIAG_DIR"):
-            H.diag_dump(f"pair_b{b}", dict(y1=H.to64(y1[b]), y2=H.to64(y2[b])))
+        ref2 = O.layer_prefill(H.to64(x2[b]), H.oracle_weights(cons.cpu), cons.spec, kv_from=ref1)
         H.close_bf16(H.to64(y2[b]), ref2["Y"], "consumer Y")
+        # chained: the oracle chains its own fp64 output
+        ref2c = O.layer_prefill(ref1["Y"], H.oracle_weights(cons.cpu), cons.spec, kv_from=ref1)
+        H.close_chain2(H.to64(y2c[b]), ref2c["Y"], "chained consumer Y")
     # the consumer refuses a K/V store its producer did not stamp
     kv2 = hy.hymba_kv_seq(kv.k, kv.v, B, L, 12345)
     with pytest.raises(hy.HymbaError):
@@ -127,15 +132,19 @@ def test_bf16_decode_after_prefill(kind):
         cons = H.GpuLayer(w, 1, consumer=True)
         hy.hymba_kv_share_bind(cons.handle, prod.handle)
         h2, conv2, ssm2 = H.alloc_ssm_cache(w, B)
-        y2, ws = H.run_prefill(cons, y, kv, None, ssm2, ws=ws)
+        xs2 = synth.gen.normal_tensor((B, L, w.dims.d_model), 0, "t_bf16_dec/x2",
+                                      device="cuda").to(torch.bfloat16)
+        y2, ws = H.run_prefill(cons, xs2, kv, None, ssm2, ws=ws)
     dws = H.workspace(hy.hymba_layer_decode_workspace(prod.handle, B, L))
     yt = torch.empty_like(x_new)
     hy.hymba_layer_decode_step(prod.handle, B, L, x_new, yt, kvc, ssm, dws, dws.numel(),
                                torch.cuda.current_stream())
     hy.hymba_stream_status(torch.cuda.current_stream())
     if kind == "consumer":
+        x_new2 = synth.gen.normal_tensor((B, w.dims.d_model), 0, "t_bf16_dec/xnew2",
+                                         device="cuda").to(torch.bfloat16)
         yt2 = torch.empty_like(x_new)
-        hy.hymba_layer_decode_step(cons.handle, B, L, yt, yt2, kvc, ssm2, dws, dws.numel(),
+        hy.hymba_layer_decode_step(cons.handle, B, L, x_new2, yt2, kvc, ssm2, dws, dws.numel(),
                                    torch.cuda.current_stream())
         hy.hymba_stream_status(torch.cuda.current_stream())
     for b in range(B):
@@ -143,15 +152,15 @@ def test_bf16_decode_after_prefill(kind):
         cache = dict(k=refp["k_cache"], v=refp["v_cache"], ssm=refp["h"], conv=refp["conv"])
         yo, newc = O.layer_decode(H.to64(x_new[b]), L, H.oracle_weights(prod.cpu), prod.spec, cache)
         H.close_bf16(H.to64(yt[b]), yo, f"decode y[b={b}]")
-        H.close_stage(H.to64(h[b]), newc["ssm"], "decode h")
-        H.close_stage(H.to64(conv[b]), newc["conv"], "decode conv")
+        H.close_stage_dist(H.to64(h[b]), newc["ssm"], "decode h")
+        H.close_stage_dist(H.to64(conv[b]), newc["conv"], "decode conv")
         # the appended K/V row sits at its slot
         sl = O.kv_slot(L, prod.spec)
         H.close_bf16(H.to64(kc[b][:, sl]), newc["k"][:, sl], "appended k")
         H.close_bf16(H.to64(vc[b][:, sl]), newc["v"][:, sl], "appended v")
         if kind == "consumer":
-            refc = O.layer_prefill(refp["Y"], H.oracle_weights(cons.cpu), cons.spec, kv_from=refp)
-            yc, _ = O.layer_decode(yo, L, H.oracle_weights(cons.cpu), cons.spec,
+            refc = O.layer_prefill(H.to64(xs2[b]), H.oracle_weights(cons.cpu), cons.spec, kv_from=refp)
+            yc, _ = O.layer_decode(H.to64(x_new2[b]), L, H.oracle_weights(cons.cpu), cons.spec,
                                    dict(ssm=refc["h"], conv=refc["conv"]), kv_cache=newc)
             H.close_bf16(H.to64(yt2[b]), yc, f"consumer decode y[b={b}]")
     prod.close()
