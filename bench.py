@@ -479,11 +479,19 @@ def run_case(args, dev):
     import synth
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    if args.case == "decode":
-        dec = Decode(synth.configs.CFG4, dev)
+    if args.case in ("decode", "decode-b32"):
+        from dataclasses import replace as _replace
+        w4 = synth.configs.CFG4 if args.case == "decode" else \
+            _replace(synth.configs.CFG4, name="decode_b32", batch=32)
+        dec = Decode(w4, dev)
         run = lambda: dec.run(stream)  # noqa: E731
     else:
-        w = {"cfg1": synth.configs.CFG1, "cfg2": synth.configs.CFG2}[args.case]
+        from dataclasses import replace as _replace
+        w = {"cfg1": synth.configs.CFG1, "cfg2": synth.configs.CFG2,
+             # prefill layer at the headline widths, batch 32, 1024 tokens: every kernel in the
+             # single-pass configuration of the headline run, with a few GB on the device
+             "b32": _replace(synth.configs.CFG3, name="b32_n1024", batch=32, n_tokens=1024,
+                             n_layers=1, kv_shared_pair=False)}[args.case]
         d = w.dims
         wt = {k: v.contiguous() for k, v in synth.configs.layer_weights(w, 0, device=dev).items()}
         cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner, d.d_state,
@@ -520,7 +528,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", choices=["headline", "cfg1", "cfg2", "decode"], default="headline",
+    ap.add_argument("--case", choices=["headline", "cfg1", "cfg2", "b32", "decode", "decode-b32"], default="headline",
                     help="headline: the benchmark; others: a smaller run for profiling")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -9,7 +9,7 @@
 //   warp 1     : TMEM allocation and MMA issue.  Per key tile and query tile:
 //                S = Q K^T (tcgen05, M=128, N=128, K=64) and O += P V
 //                (M=128, N=128, K=128; V read MN-major from its natural layout).
-//   warps 2-5, 6-9 : one softmax warpgroup per query tile, one thread per row:
+//   warps 4-7, 8-11 : one softmax warpgroup per query tile, one thread per row:
 //                row max over S (tcgen05.ld), lazy rescaling of O in TMEM only
 //                when the max grows by more than 2^8, exp2, P (bf16) written to
 //                shared memory in the 128-byte swizzled K-major layout.
@@ -51,9 +51,13 @@ constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
 constexpr int OFF_V = OFF_K + 2 * K_BYTES;
 constexpr int OFF_P = OFF_V + 2 * V_BYTES;
 constexpr int OFF_BAR = OFF_P + NQ * P_BYTES;
-constexpr int NBAR = 1 + 2 + 2 + 2 + 2 + NQ * 3 + 1;
+constexpr int NBAR = 1 + 2 + 2 + 2 + 2 + NQ * 4 + 1;
 constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
-constexpr int THREADS = 64 + NQ * 128;
+constexpr int THREADS = 128 + NQ * 128;  // warpgroup 0: TMA + MMA; one softmax warpgroup per query tile
+// Register split (setmaxnreg): launch 168 per thread = 64,512; warpgroup 0 drops to 56,
+// the softmax warpgroups rise to 224: 128 * 56 + 256 * 224 = 64,512.
+constexpr int REG_CTRL = 56;
+constexpr int REG_SOFTMAX = 224;
 constexpr uint32_t IDESC_S = make_idesc(128, 1, 0, 0);
 constexpr uint32_t IDESC_PV = make_idesc(128, 1, 0, 1);
 }  // namespace fa
@@ -63,8 +67,69 @@ __device__ __forceinline__ int fa_tile_class(int qtile, int kt, int L, int n_met
                                              int is_global) {
   return seq_tile_class(qtile, kt, L, n_meta, window, is_global);
 }
-__device__ __forceinline__ bool fa_streamed(int qa, int kt, int L, int m, int w, int g) {
-  return fa_tile_class(qa, kt, L, m, w, g) != 0 || fa_tile_class(qa + 1, kt, L, m, w, g) != 0;
+// Key tiles streamed for the query-tile pair (qa, qa+1): every tile holding a pair
+// visible from some row of the pair.  The keys visible from rows [i0, i1] are
+// [0, min(m, i1+1)) and [i0 - W + 1, i1] (all of [0, i1] for a global layer), so
+// the tiles are [0, a_end) followed by [lo, hi].  Same sequence in every role.
+struct FaTiles {
+  int a_end, lo, hi;
+  __device__ __forceinline__ int first() const { return a_end > 0 ? 0 : lo; }
+  __device__ __forceinline__ int next(int kt) const { return kt + 1 < a_end ? kt + 1 : max(kt + 1, lo); }
+};
+__device__ __forceinline__ FaTiles fa_tiles(int qa, int L, int n_meta, int window, int is_global) {
+  FaTiles t;
+  const long long i0 = (long long)qa * fa::QT;
+  const long long i1 = min((long long)(qa + 2) * fa::QT, (long long)L) - 1;
+  t.hi = (int)(i1 / fa::KT);
+  if (is_global) {
+    t.a_end = 0;
+    t.lo = 0;
+    return t;
+  }
+  const long long me = min((long long)n_meta, i1 + 1);
+  t.a_end = (int)((me + fa::KT - 1) / fa::KT);
+  t.lo = (int)(max(0LL, i0 - window + 1) / fa::KT);
+  if (t.lo < t.a_end) t.lo = t.a_end;
+  return t;
+}
+
+template <int N>
+__device__ __forceinline__ void mask_cols(uint32_t (&v)[N], int col0, int hi1, int lo2, int hi2) {
+#pragma unroll
+  for (int e = 0; e < N; ++e) {
+    const int cc = col0 + e;
+    const bool keep = (cc < hi1) | ((cc >= lo2) & (cc < hi2));
+    if (!keep) v[e] = __float_as_uint(-INFINITY);
+  }
+}
+__device__ __forceinline__ float max32(const uint32_t (&v)[32]) {
+  float m[8];
+#pragma unroll
+  for (int t = 0; t < 8; ++t) m[t] = __uint_as_float(v[t]);
+#pragma unroll
+  for (int e = 8; e < 32; ++e) m[e & 7] = fmaxf(m[e & 7], __uint_as_float(v[e]));
+  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+}
+// P for keys c*32 .. c*32+31 of row r: exp2, bf16, swizzled K-major store; returns the sum.
+__device__ __forceinline__ float p_chunk(const uint32_t (&v)[32], int c, int r, uint32_t p_base,
+                                         float scale_log2, float nm) {
+  uint32_t pk[16];
+  float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int e = 0; e < 32; e += 2) {
+    const float p0 = ex2(fmaf(__uint_as_float(v[e]), scale_log2, nm));
+    const float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale_log2, nm));
+    ls[(e >> 1) & 3] += p0 + p1;
+    pk[e >> 1] = pack_bf16x2(p0, p1);
+  }
+  const uint32_t atom = p_base + (c >> 1) * (fa::P_BYTES / 2) + r * 128;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const int chunk = (c & 1) * 4 + t;
+    st_shared_v4(atom + ((chunk ^ (r & 7)) << 4), pk[4 * t], pk[4 * t + 1], pk[4 * t + 2],
+                 pk[4 * t + 3]);
+  }
+  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
 }
 
 __global__ void __launch_bounds__(fa::THREADS, 1)
@@ -83,6 +148,7 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
   uint64_t *p_full = bars + 9 + NQ;       // [NQ]
   uint64_t *o_done = bars + 9 + 2 * NQ;   // [NQ]
   uint64_t *drain = bars + 9 + 3 * NQ;
+  uint64_t *s_free = bars + 10 + 3 * NQ;  // [NQ]: S of the tile is in registers
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBAR);
 
   const int warp = warp_id(), lane = lane_id();
@@ -94,7 +160,6 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
   const int b = rest / npairs;
   const int g = h / (H / Hkv);
   const int qa = 2 * pair;
-  const int kt_last = min(qa + 1, (L - 1) / KT);
 
   if (warp == 0 && lane == 0) {
     mbar_init(q_full, 1);
@@ -109,6 +174,7 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
       mbar_init(&s_full[q], 1);
       mbar_init(&p_full[q], 4);
       mbar_init(&o_done[q], 1);
+      mbar_init(&s_free[q], 4);
     }
     fence_barrier_init();
     tma_prefetch_desc(&tmQ);
@@ -125,41 +191,43 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S of tile q at 256q, O of tile q at 256q + 128.
 
-  // Number of streamed key tiles (same count in every role).
-  int nstream = 0;
-  for (int kt = 0; kt <= kt_last; ++kt)
-    if (fa_streamed(qa, kt, L, n_meta, window, is_global)) ++nstream;
 
-  if (warp == 0) {
+  // Streamed key tiles (same sequence in every role).
+  const FaTiles tiles = fa_tiles(qa, L, n_meta, window, is_global);
+  int nstream = 0;
+  for (int kt = tiles.first(); kt <= tiles.hi; kt = tiles.next(kt)) ++nstream;
+
+  if (warp < 4) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_CTRL));
+   if (warp == 0) {
     if (lane == 0) {
       bool ok = true;
-      uint32_t k_issued[2] = {0, 0}, v_issued[2] = {0, 0};
+      uint32_t k_issued0 = 0, k_issued1 = 0, v_issued0 = 0, v_issued1 = 0;
       mbar_arrive_expect_tx(q_full, NQ * Q_BYTES);
       for (int q = 0; q < NQ; ++q)
         tma_load_3d(smem + OFF_Q + q * Q_BYTES, &tmQ, q_full, h * 64, (qa + q) * QT, b);
       int j = 0;
-      for (int kt = 0; kt <= kt_last && ok; ++kt) {
-        if (!fa_streamed(qa, kt, L, n_meta, window, is_global)) continue;
+      for (int kt = tiles.first(); kt <= tiles.hi && ok; kt = tiles.next(kt)) {
         const int st = j & 1;
         const uint32_t ph = (uint32_t(j) >> 1) & 1u;
         if (!mbar_wait(&k_empty[st], ph ^ 1u, &g_err_attn)) { ok = false; break; }
         mbar_arrive_expect_tx(&k_full[st], K_BYTES);
         tma_load_3d(smem + OFF_K + st * K_BYTES, &tmK, &k_full[st], g * 64, kt * KT, b);
-        ++k_issued[st];
+        if (st) ++k_issued1; else ++k_issued0;
         if (!mbar_wait(&v_empty[st], ph ^ 1u, &g_err_attn)) { ok = false; break; }
         mbar_arrive_expect_tx(&v_full[st], V_BYTES);
         uint8_t *vdst = smem + OFF_V + st * V_BYTES;
         tma_load_3d(vdst, &tmV, &v_full[st], g * 128, kt * KT, b);
         tma_load_3d(vdst + V_BYTES / 2, &tmV, &v_full[st], g * 128 + 64, kt * KT, b);
-        ++v_issued[st];
+        if (st) ++v_issued1; else ++v_issued0;
         ++j;
       }
       if (!ok) {
-        mbar_wait(q_full, 0, &g_err_attn);
-        for (int s = 0; s < 2; ++s) {
-          if (k_issued[s]) mbar_wait(&k_full[s], (k_issued[s] - 1) & 1u, &g_err_attn);
-          if (v_issued[s]) mbar_wait(&v_full[s], (v_issued[s] - 1) & 1u, &g_err_attn);
-        }
+        mbar_wait_drain(q_full, 0, &g_err_attn);
+        if (k_issued0) mbar_wait_drain(&k_full[0], (k_issued0 - 1) & 1u, &g_err_attn);
+        if (k_issued1) mbar_wait_drain(&k_full[1], (k_issued1 - 1) & 1u, &g_err_attn);
+        if (v_issued0) mbar_wait_drain(&v_full[0], (v_issued0 - 1) & 1u, &g_err_attn);
+        if (v_issued1) mbar_wait_drain(&v_full[1], (v_issued1 - 1) & 1u, &g_err_attn);
       }
     }
   } else if (warp == 1) {
@@ -193,34 +261,44 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         for (int q = 0; q < NQ; ++q) issue_S(q, 0);
         mma_commit(&k_empty[0]);
       }
+      // Per key tile j: S(j+1) of both query tiles as soon as their softmax holds S(j)
+      // in registers, then PV(j) as soon as P(j) is in shared memory.  S(j+1) thus
+      // overlaps the exponentials of tile j.
       for (int j = 0; j < nstream && ok; ++j) {
         const int st = j & 1;
         const uint32_t ph = (uint32_t(j) >> 1) & 1u;
-        for (int q = 0; q < NQ && ok; ++q) {
-          if (!mbar_wait(&p_full[q], uint32_t(j) & 1u, &g_err_attn)) { ok = false; break; }
-          if (q == 0 && !mbar_wait(&v_full[st], ph, &g_err_attn)) { ok = false; break; }
-          tc_fence_after();
-          issue_PV(q, st, j > 0);
-          if (q == NQ - 1) mma_commit(&v_empty[st]);
-          if (j + 1 < nstream) {
-            const int st1 = (j + 1) & 1;
-            const uint32_t ph1 = (uint32_t(j + 1) >> 1) & 1u;
-            if (q == 0 && !mbar_wait(&k_full[st1], ph1, &g_err_attn)) { ok = false; break; }
+        if (j + 1 < nstream) {
+          const int st1 = (j + 1) & 1;
+          const uint32_t ph1 = (uint32_t(j + 1) >> 1) & 1u;
+          if (!mbar_wait(&k_full[st1], ph1, &g_err_attn)) { ok = false; break; }
+          for (int q = 0; q < NQ && ok; ++q) {
+            if (!mbar_wait(&s_free[q], uint32_t(j) & 1u, &g_err_attn)) { ok = false; break; }
             tc_fence_after();
             issue_S(q, st1);
-            if (q == NQ - 1) mma_commit(&k_empty[st1]);
           }
+          if (!ok) break;
+          mma_commit(&k_empty[st1]);
         }
+        if (!mbar_wait(&v_full[st], ph, &g_err_attn)) { ok = false; break; }
+        for (int q = 0; q < NQ && ok; ++q) {
+          if (!mbar_wait(&p_full[q], uint32_t(j) & 1u, &g_err_attn)) { ok = false; break; }
+          tc_fence_after();
+          issue_PV(q, st, j > 0);
+        }
+        if (!ok) break;
+        mma_commit(&v_empty[st]);
       }
       if (!ok) {
         // Drain issued MMAs before tensor memory is released.
         mma_commit(drain);
-        mbar_wait(drain, 0, &g_err_attn);
+        mbar_wait_drain(drain, 0, &g_err_attn);
       }
     }
+   }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_SOFTMAX));
     // ---------------- softmax warpgroups ----------------
-    const int q = (warp - 2) >> 2;        // query tile of this warpgroup
+    const int q = (warp - 4) >> 2;        // query tile of this warpgroup
     const int quarter = warp & 3;         // TMEM lane quarter
     const int r = quarter * 32 + lane;    // row within the tile
     const long long i = (long long)(qa + q) * QT + r;  // query position
@@ -229,32 +307,41 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
     const uint32_t tO = tS + 128;
     const uint32_t p_base = smem_u32(smem + OFF_P + q * P_BYTES);
     const int qtile = qa + q;
+    // Visible keys of row i: [0, meta_end) and [win_lo, i] (positions).
+    const long long meta_end = is_global ? 0 : min((long long)n_meta, i + 1);
+    const long long win_lo = is_global ? 0 : max((long long)n_meta, i - window + 1);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     int j = 0;
-    for (int kt = 0; kt <= kt_last && ok; ++kt) {
-      if (!fa_streamed(qa, kt, L, n_meta, window, is_global)) continue;
-      const int cls = fa_tile_class(qtile, kt, L, n_meta, window, is_global);
-      const long long key0 = (long long)kt * KT;
+    for (int kt = tiles.first(); kt <= tiles.hi && ok; kt = tiles.next(kt)) {
+      const int cls = fa_tile_class(qtile, kt, L, n_meta, window, is_global);  // uniform
       if (!mbar_wait(&s_full[q], uint32_t(j) & 1u, &g_err_attn)) { ok = false; break; }
       tc_fence_after();
-      // pass 1: row maximum of the scaled, masked scores
-      float mx = -INFINITY;
-      if (cls != 0) {
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tS + c * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            float x = __uint_as_float(v[e]) * scale_log2;
-            if (cls == 2 && !mask_allowed(i, key0 + c * 32 + e, n_meta, window, is_global))
-              x = -INFINITY;
-            mx = fmaxf(mx, x);
-          }
-        }
+      // the whole S row in registers: four loads, one wait
+      uint32_t s0[32], s1[32], s2[32], s3[32];
+      tmem_ld32(tS, s0);
+      tmem_ld32(tS + 32, s1);
+      tmem_ld32(tS + 64, s2);
+      tmem_ld32(tS + 96, s3);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[q]);  // the MMA warp may overwrite S now
+      if (cls != 1) {
+        // partial tile: keep the column ranges [0, hi1) and [lo2, hi2); skipped tile: none
+        const long long key0 = (long long)kt * KT;
+        int hi1 = (int)max(0LL, min(128LL, meta_end - key0));
+        int lo2 = (int)max(0LL, min(128LL, win_lo - key0));
+        int hi2 = (int)max(0LL, min(128LL, i + 1 - key0));
+        if (cls == 0) hi1 = hi2 = 0;
+        mask_cols(s0, 0, hi1, lo2, hi2);
+        mask_cols(s1, 32, hi1, lo2, hi2);
+        mask_cols(s2, 64, hi1, lo2, hi2);
+        mask_cols(s3, 96, hi1, lo2, hi2);
       }
+      // row max (scale > 0, so the max commutes with the scaling)
+      float mx = fmaxf(fmaxf(max32(s0), max32(s1)), fmaxf(max32(s2), max32(s3)));
+      mx *= scale_log2;
       // lazy rescale decision
       float alpha = 1.f;
       bool resc = false;
@@ -282,42 +369,10 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
           tmem_wait_st();
         }
       }
-      // pass 2: P = exp2(x - m), bf16, into the swizzled K-major tile
-      const float mref = (m_run == -INFINITY) ? 0.f : m_run;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        if (cls != 0) {
-          tmem_ld32(tS + c * 32, v);
-          tmem_wait_ld();
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p0 = 0.f, p1 = 0.f;
-          if (cls != 0) {
-            float x0 = __uint_as_float(v[e]) * scale_log2;
-            float x1 = __uint_as_float(v[e + 1]) * scale_log2;
-            if (cls == 2) {
-              if (!mask_allowed(i, key0 + c * 32 + e, n_meta, window, is_global)) x0 = -INFINITY;
-              if (!mask_allowed(i, key0 + c * 32 + e + 1, n_meta, window, is_global)) x1 = -INFINITY;
-            }
-            p0 = ex2(x0 - mref);
-            p1 = ex2(x1 - mref);
-          }
-          __nv_bfloat162 pb = __floats2bfloat162_rn(p0, p1);
-          l_run += __low2float(pb) + __high2float(pb);
-          pk[e >> 1] = *reinterpret_cast<uint32_t *>(&pb);
-        }
-        // keys c*32 .. c*32+31 -> atom c/2, 16-byte chunks (c%2)*4 .. +3
-        const uint32_t atom = p_base + (c >> 1) * (P_BYTES / 2) + r * 128;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int chunk = (c & 1) * 4 + t;
-          st_shared_v4(atom + ((chunk ^ (r & 7)) << 4), pk[4 * t], pk[4 * t + 1], pk[4 * t + 2],
-                       pk[4 * t + 3]);
-        }
-      }
+      // P = exp2(s * scale - m) -> bf16 into the swizzled K-major tile; fp32 row sum
+      const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+      l_run += (p_chunk(s0, 0, r, p_base, scale_log2, nm) + p_chunk(s1, 1, r, p_base, scale_log2, nm)) +
+               (p_chunk(s2, 2, r, p_base, scale_log2, nm) + p_chunk(s3, 3, r, p_base, scale_log2, nm));
       fence_proxy_async();
       tc_fence_before();
       __syncwarp();
@@ -476,44 +531,71 @@ hymba_status attention_prefill(const AttnArgs &a, hymba_dtype dt, cudaStream_t s
 
 // ---------------------------------------------------------------------------
 // Decode attention: one query per sequence over the layer's K/V store.
-// Split over key chunks (partial softmax per chunk), then a combine kernel.
-// The query heads of one kv group share every K/V read.
+// A CTA takes 64 consecutive slots of one (sequence, kv head) and all the query
+// heads of that group, so every K/V byte is read once: the slots' K and V rows are
+// contiguous and arrive in shared memory by two bulk copies.  Softmax does not depend
+// on key order, so the slots are streamed in memory order: a sliding-window
+// store's slots are exactly the visible positions once the context fills the
+// window; before that, slot validity masks the unwritten ones.  Partial
+// (max, sum, unnormalised output) per chunk, merged by a combine kernel.
 // ---------------------------------------------------------------------------
-constexpr int DEC_CHUNK = 256;
+constexpr int DEC_CHUNK = 64;
 constexpr int DEC_MAXREP = 8;
 
-__host__ __device__ __forceinline__ long long dec_visible(long long pos, int n_meta, int window,
-                                                          int is_global, long long *win0) {
-  // visible positions: [0, meta_end) and [win0, pos]
-  if (is_global) {
-    *win0 = 0;
-    return pos + 1;
-  }
-  const long long meta_end = n_meta < pos + 1 ? n_meta : pos + 1;
-  long long w0 = pos - window + 1;
-  if (w0 < meta_end) w0 = meta_end;
-  *win0 = w0;
-  return meta_end + (pos - w0 + 1);
-}
-__host__ __device__ __forceinline__ long long dec_position(long long vi, int n_meta,
-                                                           long long pos, long long win0,
-                                                           int is_global) {
-  if (is_global) return vi;
-  const long long meta_end = n_meta < pos + 1 ? n_meta : pos + 1;
-  return vi < meta_end ? vi : win0 + (vi - meta_end);
-}
 __host__ __device__ __forceinline__ long long kv_slot_of(long long p, int n_meta, int window,
                                                          int is_global) {
   if (is_global || p < n_meta) return p;
   return n_meta + (p - n_meta) % window;
 }
+// Slots a query at `pos` may read: every position of a global store, the meta
+// rows and the ring of a sliding-window store.
+__host__ __device__ __forceinline__ long long dec_slots(long long pos, int n_meta, int window,
+                                                       int is_global) {
+  return is_global ? pos + 1 : (long long)n_meta + window;
+}
+// Whether slot s holds a position visible from `pos`.
+__device__ __forceinline__ bool dec_slot_valid(long long s, long long pos, int n_meta, int window,
+                                               int is_global) {
+  if (is_global) return s <= pos;
+  if (s < n_meta) return s <= pos;
+  // the most recent position p <= pos stored in ring slot s
+  long long back = (pos - s) % window;
+  if (back < 0) back += window;
+  return pos - back >= n_meta;
+}
 
 size_t decode_attn_workspace_floats(int B, int H, int dv, long long pos, int n_meta, int window,
                                     int is_global) {
-  long long w0;
-  const long long nvis = dec_visible(pos, n_meta, window, is_global, &w0);
-  const long long nsplit = (nvis + DEC_CHUNK - 1) / DEC_CHUNK;
+  const long long nslots = dec_slots(pos, n_meta, window, is_global);
+  const long long nsplit = (nslots + DEC_CHUNK - 1) / DEC_CHUNK;
   return (size_t)B * H * nsplit * (dv + 2);
+}
+
+template <typename T>
+__device__ __forceinline__ void ld_row16(const T *p, float (&v)[16 / sizeof(T)]) {
+  uint4 raw = __ldg(reinterpret_cast<const uint4 *>(p));
+  if constexpr (sizeof(T) == 2) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __low2float(h[i]);
+      v[2 * i + 1] = __high2float(h[i]);
+    }
+  } else {
+    const float *f = reinterpret_cast<const float *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = f[i];
+  }
+}
+
+// Bulk copy global -> shared (contiguous, 16-byte aligned, size % 16 == 0), completion
+// counted on an mbarrier.  Plain (no multicast) form.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
 template <typename T>
@@ -522,89 +604,164 @@ __global__ void __launch_bounds__(128)
                                const T *__restrict__ vc, float *__restrict__ part, int H, int Hkv,
                                int dqk, int dv, int cap, long long pos, int n_meta, int window,
                                int is_global, float scale_log2, int nsplit) {
+  constexpr int V = 16 / sizeof(T);
+  extern __shared__ __align__(128) uint8_t dsm[];
+  T *sk = reinterpret_cast<T *>(dsm);                               // [DEC_CHUNK][dqk]
+  T *sv = reinterpret_cast<T *>(dsm + DEC_CHUNK * dqk * sizeof(T));  // [DEC_CHUNK][dv]
   __shared__ float qs[DEC_MAXREP][128];
   __shared__ float sc[DEC_MAXREP][DEC_CHUNK];
   __shared__ float red[DEC_MAXREP][4];
-  __shared__ float mxs[DEC_MAXREP], sums[DEC_MAXREP];
+  __shared__ float stat[DEC_MAXREP][2];
+  __shared__ float opart[DEC_MAXREP][128];
+  __shared__ uint64_t bar;
   const int split = blockIdx.y;
   const int bg = blockIdx.x;
   const int b = bg / Hkv, g = bg % Hkv;
   const int rep = H / Hkv;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const long long s0 = (long long)split * DEC_CHUNK;
+  const long long nslots = dec_slots(pos, n_meta, window, is_global);
+  const int ns = (int)min((long long)DEC_CHUNK, nslots - s0);
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (tid == 0) {
+    const uint32_t kb = (uint32_t)(ns * dqk * sizeof(T)), vb = (uint32_t)(ns * dv * sizeof(T));
+    mbar_arrive_expect_tx(&bar, kb + vb);
+    bulk_load(sk, kc + (((long long)b * Hkv + g) * cap + s0) * dqk, kb, &bar);
+    bulk_load(sv, vc + (((long long)b * Hkv + g) * cap + s0) * dv, vb, &bar);
+  }
   for (int idx = tid; idx < rep * dqk; idx += 128) {
     const int r = idx / dqk, d = idx % dqk;
     qs[r][d] = Store<T>::to_f(q[(long long)b * H * dqk + (g * rep + r) * dqk + d]) * scale_log2;
   }
   __syncthreads();
-  long long w0;
-  const long long nvis = dec_visible(pos, n_meta, window, is_global, &w0);
-  const long long v0 = (long long)split * DEC_CHUNK;
-  const int nk = (int)min((long long)DEC_CHUNK, nvis - v0);
-  const T *kbase = kc + ((long long)b * Hkv + g) * cap * dqk;
-  const T *vbase = vc + ((long long)b * Hkv + g) * cap * dv;
-  for (int t = tid; t < DEC_CHUNK; t += 128) {
-    if (t < nk) {
-      const long long p = dec_position(v0 + t, n_meta, pos, w0, is_global);
-      const T *kr = kbase + kv_slot_of(p, n_meta, window, is_global) * dqk;
-      float acc[DEC_MAXREP];
+  bool ok = mbar_wait(&bar, 0, &g_err_attn);
+  if (!ok && tid == 0) mbar_wait_drain(&bar, 0, &g_err_attn);  // no copy outlives the CTA
+  __syncthreads();
+  // scores: two threads per key, each half of the head dim (16-byte pieces read in a
+  // rotated order, conflict-free), combined by a shuffle
+  {
+    const int key = tid >> 1, part_ = tid & 1;
+    const bool valid = ok && key < ns && dec_slot_valid(s0 + key, pos, n_meta, window, is_global);
+    float acc[DEC_MAXREP];
 #pragma unroll
-      for (int r = 0; r < DEC_MAXREP; ++r) acc[r] = 0.f;
-      for (int d = 0; d < dqk; ++d) {
-        const float kv = Store<T>::to_f(kr[d]);
+    for (int r = 0; r < DEC_MAXREP; ++r) acc[r] = 0.f;
+    if (valid) {
+      const int npc = dqk / V / 2;  // pieces in this thread's half
+      const T *kr = sk + key * dqk + part_ * (dqk / 2);
+      for (int pc0 = 0; pc0 < npc; ++pc0) {
+        const int pc = (pc0 + key) % npc;
+        const uint4 raw = *reinterpret_cast<const uint4 *>(kr + pc * V);
+        float kv[V];
+        if constexpr (sizeof(T) == 2) {
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-        for (int r = 0; r < DEC_MAXREP; ++r)
-          if (r < rep) acc[r] = fmaf(qs[r][d], kv, acc[r]);
+          for (int i = 0; i < 4; ++i) {
+            kv[2 * i] = bf16_lo(w[i]);
+            kv[2 * i + 1] = bf16_hi(w[i]);
+          }
+        } else {
+          const float *f = reinterpret_cast<const float *>(&raw);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) kv[i] = f[i];
+        }
+        const int d0 = part_ * (dqk / 2) + pc * V;
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+#pragma unroll
+          for (int r = 0; r < DEC_MAXREP; ++r)
+            if (r < rep) acc[r] = fmaf(qs[r][d0 + i], kv[i], acc[r]);
       }
-      for (int r = 0; r < rep; ++r) sc[r][t] = acc[r];
-    } else {
-      for (int r = 0; r < rep; ++r) sc[r][t] = -INFINITY;
+    }
+#pragma unroll
+    for (int r = 0; r < DEC_MAXREP; ++r) acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 1);
+    if (part_ == 0) {
+#pragma unroll
+      for (int r = 0; r < DEC_MAXREP; ++r)
+        if (r < rep) sc[r][key] = valid ? acc[r] : -INFINITY;
     }
   }
   __syncthreads();
   // per-head max and sum over the chunk
   for (int r = 0; r < rep; ++r) {
-    float m = fmaxf(sc[r][tid], sc[r][tid + 128]);
+    float m = tid < DEC_CHUNK ? sc[r][tid] : -INFINITY;
 #pragma unroll
     for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
     if (lane == 0) red[r][wid] = m;
   }
   __syncthreads();
-  if (tid < rep) mxs[tid] = fmaxf(fmaxf(red[tid][0], red[tid][1]), fmaxf(red[tid][2], red[tid][3]));
+  if (tid < rep) stat[tid][0] = fmaxf(fmaxf(red[tid][0], red[tid][1]), fmaxf(red[tid][2], red[tid][3]));
   __syncthreads();
   for (int r = 0; r < rep; ++r) {
-    const float p0 = ex2(sc[r][tid] - mxs[r]);
-    const float p1 = ex2(sc[r][tid + 128] - mxs[r]);
-    sc[r][tid] = p0;
-    sc[r][tid + 128] = p1;
-    float s = p0 + p1;
+    const float mr = stat[r][0];
+    float p = 0.f;
+    if (tid < DEC_CHUNK) {
+      p = mr == -INFINITY ? 0.f : ex2(sc[r][tid] - mr);
+      sc[r][tid] = p;
+    }
+    float sum = p;
 #pragma unroll
-    for (int off = 16; off; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) red[r][wid] = s;
+    for (int off = 16; off; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane == 0) red[r][wid] = sum;
   }
   __syncthreads();
-  if (tid < rep) sums[tid] = red[tid][0] + red[tid][1] + red[tid][2] + red[tid][3];
-  __syncthreads();
-  // o[r][d] = sum_t p[r][t] V[t][d]
-  for (int d = tid; d < dv; d += 128) {
-    float acc[DEC_MAXREP];
+  if (tid < rep) stat[tid][1] = (red[tid][0] + red[tid][1]) + (red[tid][2] + red[tid][3]);
+  // o[r][d] = sum_t p[r][t] V[t][d]: thread = (column pair, half of the keys)
+  const int npair = dv / 2;
+  const int half = tid / 64, cp = tid % 64;
+  for (int c0 = 0; c0 < npair; c0 += 64) {  // uniform trip count: barriers inside
+    const int c = c0 + cp;
+    const bool active = ok && c < npair;
+    float acc0[DEC_MAXREP], acc1[DEC_MAXREP];
 #pragma unroll
-    for (int r = 0; r < DEC_MAXREP; ++r) acc[r] = 0.f;
-    for (int t = 0; t < nk; ++t) {
-      const long long p = dec_position(v0 + t, n_meta, pos, w0, is_global);
-      const float vv = Store<T>::to_f(vbase[kv_slot_of(p, n_meta, window, is_global) * dv + d]);
+    for (int r = 0; r < DEC_MAXREP; ++r) acc0[r] = acc1[r] = 0.f;
+    const int t0 = half * (DEC_CHUNK / 2), t1 = active ? min(ns, t0 + DEC_CHUNK / 2) : t0;
+    for (int t = t0; t < t1; ++t) {
+      float v0, v1;
+      if constexpr (sizeof(T) == 2) {
+        const __nv_bfloat162 v2 = *reinterpret_cast<const __nv_bfloat162 *>(sv + t * dv + 2 * c);
+        v0 = __low2float(v2);
+        v1 = __high2float(v2);
+      } else {
+        const float2 v2 = *reinterpret_cast<const float2 *>(sv + t * dv + 2 * c);
+        v0 = v2.x;
+        v1 = v2.y;
+      }
 #pragma unroll
       for (int r = 0; r < DEC_MAXREP; ++r)
-        if (r < rep) acc[r] = fmaf(sc[r][t], vv, acc[r]);
+        if (r < rep) {
+          const float p = sc[r][t];
+          acc0[r] = fmaf(p, v0, acc0[r]);
+          acc1[r] = fmaf(p, v1, acc1[r]);
+        }
     }
-    for (int r = 0; r < rep; ++r) {
-      float *dst = part + (((long long)b * H + g * rep + r) * nsplit + split) * (dv + 2);
-      dst[2 + d] = acc[r];
+    if (half == 1) {
+#pragma unroll
+      for (int r = 0; r < DEC_MAXREP; ++r)
+        if (r < rep) {
+          opart[r][2 * cp] = acc0[r];
+          opart[r][2 * cp + 1] = acc1[r];
+        }
     }
+    __syncthreads();
+    if (half == 0 && active) {
+#pragma unroll
+      for (int r = 0; r < DEC_MAXREP; ++r)
+        if (r < rep) {
+          float *dst = part + (((long long)b * H + g * rep + r) * nsplit + split) * (dv + 2);
+          dst[2 + 2 * c] = acc0[r] + opart[r][2 * cp];
+          dst[2 + 2 * c + 1] = acc1[r] + opart[r][2 * cp + 1];
+        }
+    }
+    __syncthreads();
   }
   if (tid < rep) {
     float *dst = part + (((long long)b * H + g * rep + tid) * nsplit + split) * (dv + 2);
-    dst[0] = mxs[tid];
-    dst[1] = sums[tid];
+    dst[0] = stat[tid][0];
+    dst[1] = stat[tid][1];
   }
 }
 
@@ -616,34 +773,54 @@ __global__ void attn_decode_combine_kernel(const float *__restrict__ part, T *__
   float M = -INFINITY;
   for (int s = 0; s < nsplit; ++s) M = fmaxf(M, base[s * (dv + 2)]);
   float Lsum = 0.f;
-  for (int s = 0; s < nsplit; ++s) Lsum += base[s * (dv + 2) + 1] * ex2(base[s * (dv + 2)] - M);
+  for (int s = 0; s < nsplit; ++s) {
+    const float ms = base[s * (dv + 2)];
+    if (ms != -INFINITY) Lsum += base[s * (dv + 2) + 1] * ex2(ms - M);
+  }
   for (int d = threadIdx.x; d < dv; d += blockDim.x) {
     float acc = 0.f;
-    for (int s = 0; s < nsplit; ++s)
-      acc += base[s * (dv + 2) + 2 + d] * ex2(base[s * (dv + 2)] - M);
+    for (int s = 0; s < nsplit; ++s) {
+      const float ms = base[s * (dv + 2)];
+      if (ms != -INFINITY) acc += base[s * (dv + 2) + 2 + d] * ex2(ms - M);
+    }
     o[(long long)bh * dv + d] = Store<T>::from_f(acc / Lsum);
   }
 }
 
 hymba_status attention_decode(const DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s) {
   const int rep = a.H / a.Hkv;
-  if (rep > DEC_MAXREP || a.dqk > 128) {
-    set_error("decode attention supports H/Hkv <= 8 and head_dim_qk <= 128");
+  const int V = dt == HYMBA_BF16 ? 8 : 4;
+  if (rep > DEC_MAXREP || a.dqk > 128 || a.dqk % V || a.dv > 256 || a.dv % 2) {
+    set_error("decode attention supports H/Hkv <= 8, head_dim_qk <= 128 (multiple of 16 bytes), "
+              "even head_dim_v <= 256");
     return HYMBA_ERR_UNSUPPORTED;
   }
-  long long w0;
-  const long long nvis = dec_visible(a.pos, a.n_meta, a.window, a.is_global, &w0);
-  const int nsplit = (int)((nvis + DEC_CHUNK - 1) / DEC_CHUNK);
+  const long long nslots = dec_slots(a.pos, a.n_meta, a.window, a.is_global);
+  const int nsplit = (int)((nslots + DEC_CHUNK - 1) / DEC_CHUNK);
   dim3 grid(a.B * a.Hkv, nsplit);
   const float sl2 = a.scale * 1.4426950408889634f;
+  const int esz = dt == HYMBA_BF16 ? 2 : 4;
+  const int dsmem = DEC_CHUNK * (a.dqk + a.dv) * esz;
+  {
+    static unsigned attr_set = 0;  // one bit per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!(attr_set & (1u << (dev & 31)))) {
+      const int most = DEC_CHUNK * (128 + 256) * 4;
+      cudaFuncSetAttribute(attn_decode_partial_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      cudaFuncSetAttribute(attn_decode_partial_kernel<__nv_bfloat16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      attr_set |= 1u << (dev & 31);
+    }
+  }
   if (dt == HYMBA_BF16) {
-    attn_decode_partial_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(
+    attn_decode_partial_kernel<__nv_bfloat16><<<grid, 128, dsmem, s>>>(
         (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k_cache, (const __nv_bfloat16 *)a.v_cache,
         a.partial, a.H, a.Hkv, a.dqk, a.dv, a.cap, a.pos, a.n_meta, a.window, a.is_global, sl2, nsplit);
     attn_decode_combine_kernel<__nv_bfloat16><<<a.B * a.H, 128, 0, s>>>(
         a.partial, (__nv_bfloat16 *)a.o, a.H, a.dv, nsplit);
   } else {
-    attn_decode_partial_kernel<float><<<grid, 128, 0, s>>>(
+    attn_decode_partial_kernel<float><<<grid, 128, dsmem, s>>>(
         (const float *)a.q, (const float *)a.k_cache, (const float *)a.v_cache, a.partial, a.H,
         a.Hkv, a.dqk, a.dv, a.cap, a.pos, a.n_meta, a.window, a.is_global, sl2, nsplit);
     attn_decode_combine_kernel<float><<<a.B * a.H, 128, 0, s>>>(a.partial, (float *)a.o, a.H,

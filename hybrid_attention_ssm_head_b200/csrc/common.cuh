@@ -32,11 +32,33 @@ template <> struct Store<float> {
   static __device__ __forceinline__ float from_f(float v) { return v; }
 };
 template <> struct Store<__nv_bfloat16> {
-  static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+  static __device__ __forceinline__ float to_f(__nv_bfloat16 v) {
+    return __uint_as_float(uint32_t(*reinterpret_cast<const unsigned short *>(&v)) << 16);
+  }
   static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
 };
 
-__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + __expf(-x)); }
+// x * sigmoid(x) with the fast exp and division (about 2 ulp; 0 for x -> -inf).
+__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+// bf16 -> fp32 is a 16-bit shift of the bits (exact): an integer-pipe operation.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+// Two fp32 fused multiply-adds in one instruction (d = a * b + c, elementwise).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)),
+        "l"(*reinterpret_cast<uint64_t *>(&c)));
+  return *reinterpret_cast<float2 *>(&d);
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&d);
+}
 // log(1 + e^x) with the fast exp/log: x above 20 returns x; below -8 returns e^x
 // (relative error e^x / 2 < 2e-4); in between log(1 + e^x) with 1 + e^x >= 1 + 3e-4,
 // so the fp32 rounding of the sum costs at most ~2e-4 relative.
@@ -140,6 +162,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
       return false;
     }
   }
+}
+
+// Drain wait for the abort path: waits (bounded) for copies or MMAs already
+// issued by this CTA, even when another CTA has recorded an error.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, unsigned int *err) {
+  long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) {
+      atomicOr(err, kErrTimeout);
+      return false;
+    }
+  }
+  return true;
 }
 
 // ---------------------------------------------------------------------------

@@ -8,8 +8,8 @@
 //   warp 1   : TMEM allocator and MMA issuer (one lane): per 128-byte K block,
 //              4 x tcgen05.mma (M=128, N=BN, K=32 bytes) into one of two fp32
 //              accumulators in tensor memory, then tcgen05.commit frees the stage.
-//   warps 2-9: epilogue, one thread per accumulator row (two warps per TMEM
-//              lane quarter, alternate 16-column chunks): tcgen05.ld, bias /
+//   warps 2-17: epilogue, one thread per accumulator row (four warps per TMEM
+//              lane quarter, every fourth 16-column chunk): tcgen05.ld, bias /
 //              softplus, fp32 -> bf16, routed stores (one GEMM writes Q, K, V,
 //              x_ssm and z to their own buffers).  The second accumulator lets
 //              the epilogue of tile i overlap the MMAs of tile i+1.
@@ -149,13 +149,13 @@ struct TcCfg {
   static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
   static constexpr uint32_t IDESC = make_idesc(BN, ELEM == 2 ? 1 : 2, 0, 0);
-  static constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 16;
+  static constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 16;  // + static smem: Epilogue
   static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0, N <= 256");
 };
 
 template <int BN, int ELEM>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(576, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int M, int N, int K, int ksplit, Epilogue epi) {
   using C = TcCfg<BN, ELEM>;
@@ -168,6 +168,10 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t *tfull = empty + C::STAGES;
   uint64_t *tempty = tfull + 2;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  // Segment table in shared memory: per-column routing then indexes smem, not
+  // kernel parameters.
+  __shared__ Epilogue s_epi;
+  if (threadIdx.x == 0) s_epi = epi;
 
   const int warp = warp_id();
   const int lane = lane_id();
@@ -184,7 +188,7 @@ __global__ void __launch_bounds__(320, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 256);
+      mbar_init(&tempty[a], 512);
     }
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
@@ -229,7 +233,7 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok) {
         // Leave no copy in flight into shared memory that is about to be released.
         for (int s = 0; s < C::STAGES; ++s)
-          if (issued[s]) mbar_wait(&full[s], (issued[s] - 1) & 1u, &g_err_gemm);
+          if (issued[s]) mbar_wait_drain(&full[s], (issued[s] - 1) & 1u, &g_err_gemm);
       }
     }
   } else if (warp == 1) {
@@ -283,14 +287,15 @@ __global__ void __launch_bounds__(320, 1)
       if (!ok) {
         // Drain issued MMAs before tensor memory is released.
         mma_commit(&tfull[acc]);
-        mbar_wait(&tfull[acc], acc_phase, &g_err_gemm);
+        mbar_wait_drain(&tfull[acc], acc_phase, &g_err_gemm);
       }
     }
   } else {
     // ---------------- epilogue: warps 2..9, one thread per accumulator row ----------------
-    // Warps w and w+4 share a TMEM lane quarter and take alternate 16-column chunks.
+    // Warps w, w+4, w+8, w+12 share a TMEM lane quarter and take every fourth
+    // 16-column chunk.
     const int quarter = warp & 3;  // TMEM lanes this warp may access
-    const int half = (warp - 2) >> 2;
+    const int sub = (warp - 2) >> 2;
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
@@ -305,13 +310,13 @@ __global__ void __launch_bounds__(320, 1)
       const long long m = (long long)mt * C::BM + row;
       const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
 #pragma unroll 1
-      for (int c = half * 16; c < BN; c += 32) {
+      for (int c = sub * 16; c < BN; c += 64) {
         const int n0 = nt * BN + c;
         if (n0 >= N) break;  // uniform across the warp
         uint32_t r[16];
         tmem_ld16(t_row + c, r);
         tmem_wait_ld();
-        if (m < M) epi_store16(epi, m, n0, N, r);
+        if (m < M) epi_store16(s_epi, m, n0, N, r);
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -365,7 +370,7 @@ static hymba_status launch_tc(const GemmArgs &g, cudaStream_t s) {
   if (!make_tmap(&tb, g.B, dt, 2, db, sb, bb)) return HYMBA_ERR_CUDA;
   const long long tiles = (long long)((g.M + 127) / 128) * ((g.N + BN - 1) / BN) * g.ksplit;
   const int grid = (int)std::min<long long>(tiles, num_sms());
-  gemm_tc_kernel<BN, ELEM><<<grid, 320, C::SMEM, s>>>(ta, tb, g.M, g.N, g.K, g.ksplit, g.epi);
+  gemm_tc_kernel<BN, ELEM><<<grid, 576, C::SMEM, s>>>(ta, tb, g.M, g.N, g.K, g.ksplit, g.epi);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

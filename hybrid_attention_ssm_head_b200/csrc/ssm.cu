@@ -5,8 +5,8 @@
 // [delta, B, C] come from the projection GEMMs; A = -exp(A_log).
 //
 // Scan layout: one thread per (sequence, channel) carrying the d_state = 16
-// states in registers; B_t and C_t (shared by all channels of a sequence) are
-// staged through shared memory 32 steps at a time.  When there are too few
+// states in registers; u, delta, z and B_t, C_t (shared by all channels of a
+// sequence) are staged through shared memory 16 steps at a time by cp.async.  When there are too few
 // (sequence, channel) pairs to fill the GPU, time is split into chunks:
 // pass 1 scans each chunk from zero and records its end state and sum of
 // delta (the chunk's decay is exp(A * sum delta)); pass 2 chains the chunk
@@ -20,7 +20,7 @@
 namespace hymba {
 
 constexpr int kStates = 16;
-constexpr int kScanTB = 32;
+constexpr int kScanTB = 16;
 
 __device__ __forceinline__ float ex2f_(float x) {
   float y;
@@ -67,13 +67,29 @@ __device__ __forceinline__ void store_vec(T *p, const float (&v)[Vec16<T>::N]) {
   *reinterpret_cast<uint4 *>(p) = raw;
 }
 
-constexpr int kConvTB = 8;
+constexpr int kConvTB = 4;
 
-// One thread: VEC channels x kConvTB rows.  The kConvTB + 3 input rows it needs are
-// loaded up front (16-byte vectors, coalesced across the warp) so that all loads
-// are in flight together.
 template <typename T>
-__global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
+__device__ __forceinline__ void unpack16(const uint4 &raw, float (&v)[16 / sizeof(T)]) {
+  if constexpr (sizeof(T) == 2) {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = bf16_lo(w[i]);
+      v[2 * i + 1] = bf16_hi(w[i]);
+    }
+  } else {
+    const float *f = reinterpret_cast<const float *>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = f[i];
+  }
+}
+
+// One thread: VEC channels x kConvTB rows.  Its kConvTB + 3 input rows are loaded
+// up front as 16-byte vectors (coalesced across the warp); the overlap with the
+// neighbouring row blocks is served by L2.
+template <typename T>
+__global__ void __launch_bounds__(256) conv_silu_kernel(ConvArgs a) {
   constexpr int V = Vec16<T>::N;
   constexpr int NR = kConvTB + 3;
   const int nvec = a.E / V;
@@ -89,56 +105,59 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
   const T *x = reinterpret_cast<const T *>(a.x);
   T *u = reinterpret_cast<T *>(a.u);
   const int t0 = tb * kConvTB;
-  // raw[r] = x[t0 - 3 + r] (zero outside the sequence)
-  uint4 raw[NR];
+  uint4 raw[NR];  // raw[r] = x[t0 - 3 + r], zero outside the sequence
 #pragma unroll
   for (int r = 0; r < NR; ++r) {
     const int t = t0 - 3 + r;
-    if (t >= 0 && t < a.L)
-      raw[r] = __ldg(reinterpret_cast<const uint4 *>(x + ((long long)b * a.L + t) * a.ld_x + c0));
-    else
-      raw[r] = make_uint4(0, 0, 0, 0);
+    raw[r] = (t >= 0 && t < a.L)
+                 ? __ldg(reinterpret_cast<const uint4 *>(x + ((long long)b * a.L + t) * a.ld_x + c0))
+                 : make_uint4(0, 0, 0, 0);
   }
-  float w[4][V], bias[V];
+  float acc[kConvTB][V];
 #pragma unroll
   for (int i = 0; i < V; ++i) {
-    bias[i] = a.bias[c0 + i];
+    const float bi = __ldg(a.bias + c0 + i);
 #pragma unroll
-    for (int k = 0; k < 4; ++k) w[k][i] = k < K ? a.w[(c0 + i) * K + k] : 0.f;
+    for (int tt = 0; tt < kConvTB; ++tt) acc[tt][i] = bi;
   }
-  auto val = [&](int r, int i) -> float {
-    if constexpr (sizeof(T) == 2) {
-      const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw[r]);
-      return (i & 1) ? __high2float(h[i >> 1]) : __low2float(h[i >> 1]);
-    } else {
-      return reinterpret_cast<const float *>(&raw[r])[i];
+  // wj multiplies x[t - 3 + j] (taps right-aligned so every index is static)
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int k = j - (4 - K);
+    if (k < 0) continue;
+    float wj[V];
+#pragma unroll
+    for (int i = 0; i < V; ++i) wj[i] = __ldg(a.w + (c0 + i) * K + k);
+#pragma unroll
+    for (int tt = 0; tt < kConvTB; ++tt) {
+      float xv[V];
+      unpack16<T>(raw[tt + j], xv);
+#pragma unroll
+      for (int i = 0; i < V; ++i) acc[tt][i] = fmaf(wj[i], xv[i], acc[tt][i]);
     }
-  };
+  }
 #pragma unroll
   for (int tt = 0; tt < kConvTB; ++tt) {
     const int t = t0 + tt;
-    if (t >= a.L) break;
-    float o[V];
+    if (t < a.L) {
+      float o[V];
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-      // tap k multiplies x[t - (K-1) + k] = raw[tt + 3 - (K-1) + k]
-      float acc = bias[i];
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        if (k < K) acc = fmaf(w[k][i], val(tt + 4 - K + k, i), acc);
-      o[i] = silu_f(acc);
+      for (int i = 0; i < V; ++i) o[i] = silu_f(acc[tt][i]);
+      store_vec<T>(u + ((long long)b * a.L + t) * a.E + c0, o);
     }
-    store_vec<T>(u + ((long long)b * a.L + t) * a.E + c0, o);
   }
   if (a.conv_state && t0 + kConvTB >= a.L) {
-    // the last K-1 rows of x, oldest first: x[L-K+1 .. L-1] = raw[L-K+1 - t0 + 3 ..]
+    // the last K-1 rows of x, oldest first: x[L-K+1+r] = raw[L-K+4+r-t0]
     T *cs = reinterpret_cast<T *>(a.conv_state);
-    for (int r = 0; r < K - 1; ++r) {
-      const int rr = a.L - (K - 1) + r - t0 + 3;
-      float v[V];
+    const int base = a.L - K + 4 - t0;
 #pragma unroll
-      for (int i = 0; i < V; ++i) v[i] = (rr >= 0 && rr < NR) ? val(rr, i) : 0.f;
-      store_vec<T>(cs + ((long long)b * (K - 1) + r) * a.E + c0, v);
+    for (int rr = 0; rr < NR; ++rr) {
+      const int r = rr - base;
+      if (r >= 0 && r < K - 1) {
+        float v[V];
+        unpack16<T>(raw[rr], v);
+        store_vec<T>(cs + ((long long)b * (K - 1) + r) * a.E + c0, v);
+      }
     }
   }
 }
@@ -147,11 +166,11 @@ hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s) {
   const int V = dt == HYMBA_BF16 ? 8 : 4;
   const long long n = (long long)a.B * ((a.L + kConvTB - 1) / kConvTB) * (a.E / V);
   if (n == 0) return HYMBA_OK;
-  const unsigned blocks = (unsigned)((n + 127) / 128);
+  const unsigned blocks = (unsigned)((n + 255) / 256);
   if (dt == HYMBA_BF16)
-    conv_silu_kernel<__nv_bfloat16><<<blocks, 128, 0, s>>>(a);
+    conv_silu_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(a);
   else
-    conv_silu_kernel<float><<<blocks, 128, 0, s>>>(a);
+    conv_silu_kernel<float><<<blocks, 256, 0, s>>>(a);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -202,14 +221,33 @@ hymba_status decode_conv(const DecodeConvArgs &a, hymba_dtype dt, cudaStream_t s
 // ---------------------------------------------------------------------------
 // mode 0: scan from the chunk's start state and write y (and the final state);
 // mode 1: scan from zero, record the chunk's end state and sum of delta.
+// u, delta, z and [B, C] of kScanTB steps are staged in shared memory with
+// cp.async (double-buffered) while the previous steps are being scanned.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
 template <typename T>
 __global__ void __launch_bounds__(128)
     scan_kernel(ScanArgs a, int chunks, int Tc, int mode, const float *__restrict__ hstart,
                 float *__restrict__ hend, float *__restrict__ dsum_out) {
-  __shared__ float sbc[kScanTB][2 * kStates];
+  extern __shared__ __align__(16) uint8_t scan_smem[];
+  const int bs = blockDim.x;
+  // layout per buffer: u [TB][bs], delta [TB][bs], z [TB][bs] (T), bc [TB][2N] (fp32)
+  const int arr_bytes = kScanTB * bs * (int)sizeof(T);
+  const int buf_bytes = 3 * arr_bytes + kScanTB * 2 * kStates * 4;
   const int E = a.E;
-  const int cblocks = E / blockDim.x;
-  const int c = (blockIdx.x % cblocks) * blockDim.x + threadIdx.x;
+  const int cblocks = E / bs;
+  const int cbase = (blockIdx.x % cblocks) * bs;
+  const int c = cbase + threadIdx.x;
   const int rest = blockIdx.x / cblocks;
   const int k = rest % chunks;
   const int b = rest / chunks;
@@ -219,6 +257,28 @@ __global__ void __launch_bounds__(128)
   const T *z = reinterpret_cast<const T *>(a.z);
   T *y = reinterpret_cast<T *>(a.y);
 
+  // issue the copies of steps [tb, tb + nt) into buffer `buf`
+  auto stage = [&](int tb, int nt, int buf) {
+    uint8_t *base = scan_smem + buf * buf_bytes;
+    const int row_chunks = bs * (int)sizeof(T) / 16;  // 16-byte pieces of one row of bs channels
+    const int n_act = nt * row_chunks;
+    for (int e = threadIdx.x; e < 3 * n_act; e += bs) {
+      const int arr = e / n_act, w = e % n_act;
+      const int tt = w / row_chunks, piece = w % row_chunks;
+      const long long row = (long long)b * a.L + tb + tt;
+      const T *src = arr == 0 ? u + row * E : arr == 1 ? dl + row * E : z + row * a.ld_z;
+      cp_async16(base + arr * arr_bytes + (tt * bs) * (int)sizeof(T) + piece * 16,
+                 src + cbase + piece * (16 / (int)sizeof(T)));
+    }
+    float *sbc = reinterpret_cast<float *>(base + 3 * arr_bytes);
+    for (int e = threadIdx.x; e < nt * 8; e += bs) {  // 2N floats = 8 pieces per step
+      const int tt = e / 8, piece = e % 8;
+      cp_async16(sbc + tt * 2 * kStates + piece * 4,
+                 a.bc + ((long long)b * a.L + tb + tt) * a.ld_bc + a.bc_col + piece * 4);
+    }
+    cp_async_commit();
+  };
+
   float A2[kStates], h[kStates];
 #pragma unroll
   for (int n = 0; n < kStates; ++n) A2[n] = -__expf(a.a_log[c * kStates + n]) * 1.4426950408889634f;
@@ -227,51 +287,75 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int n = 0; n < kStates; ++n) h[n] = hstart[sidx + n];
   } else if (mode == 0 && a.h_in) {
+    const float4 *hp = reinterpret_cast<const float4 *>(a.h_in + ((long long)b * E + c) * kStates);
 #pragma unroll
-    for (int n = 0; n < kStates; ++n) h[n] = a.h_in[((long long)b * E + c) * kStates + n];
+    for (int n = 0; n < kStates; n += 4) {
+      const float4 v4 = hp[n >> 2];
+      h[n] = v4.x;
+      h[n + 1] = v4.y;
+      h[n + 2] = v4.z;
+      h[n + 3] = v4.w;
+    }
   } else {
 #pragma unroll
     for (int n = 0; n < kStates; ++n) h[n] = 0.f;
   }
   const float Dc = a.d_skip[c];
   float dsum = 0.f;
-  for (int tb = t0; tb < t1; tb += kScanTB) {
+  const int nblk = (t1 - t0 + kScanTB - 1) / kScanTB;
+  if (nblk > 0) stage(t0, min(kScanTB, t1 - t0), 0);
+  for (int kb = 0; kb < nblk; ++kb) {
+    const int tb = t0 + kb * kScanTB;
     const int nt = min(kScanTB, t1 - tb);
-    __syncthreads();
-    for (int e = threadIdx.x; e < nt * 2 * kStates; e += blockDim.x) {
-      const int tt = e / (2 * kStates), j = e % (2 * kStates);
-      sbc[tt][j] = a.bc[((long long)b * a.L + tb + tt) * a.ld_bc + a.bc_col + j];
+    if (kb + 1 < nblk) {
+      stage(tb + kScanTB, min(kScanTB, t1 - tb - kScanTB), (kb + 1) & 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
+    const uint8_t *base = scan_smem + (kb & 1) * buf_bytes;
+    const T *su = reinterpret_cast<const T *>(base);
+    const T *sd = reinterpret_cast<const T *>(base + arr_bytes);
+    const T *sz = reinterpret_cast<const T *>(base + 2 * arr_bytes);
+    const float *sbc = reinterpret_cast<const float *>(base + 3 * arr_bytes);
 #pragma unroll 2
     for (int tt = 0; tt < nt; ++tt) {
-      const long long row = (long long)b * a.L + tb + tt;
-      const float d = Store<T>::to_f(dl[row * E + c]);
-      const float uu = Store<T>::to_f(u[row * E + c]);
+      const float d = Store<T>::to_f(sd[tt * bs + threadIdx.x]);
+      const float uu = Store<T>::to_f(su[tt * bs + threadIdx.x]);
       const float du = d * uu;
-      float acc = 0.f;
+      const float2 *bc2 = reinterpret_cast<const float2 *>(sbc + tt * 2 * kStates);
+      const float2 d2 = make_float2(d, d), du2 = make_float2(du, du);
+      float2 acc2 = make_float2(0.f, 0.f);
 #pragma unroll
-      for (int n = 0; n < kStates; ++n) {
-        const float dA = ex2f_(d * A2[n]);
-        h[n] = fmaf(dA, h[n], du * sbc[tt][n]);
-        acc = fmaf(sbc[tt][kStates + n], h[n], acc);
+      for (int n = 0; n < kStates; n += 2) {
+        const float2 x2 = fmul2(d2, make_float2(A2[n], A2[n + 1]));
+        const float2 dA2 = make_float2(ex2f_(x2.x), ex2f_(x2.y));
+        const float2 hb = fmul2(du2, bc2[n >> 1]);
+        float2 hv = ffma2(dA2, make_float2(h[n], h[n + 1]), hb);
+        h[n] = hv.x;
+        h[n + 1] = hv.y;
+        acc2 = ffma2(bc2[(kStates + n) >> 1], hv, acc2);
       }
+      float acc = acc2.x + acc2.y;
       if (mode == 0) {
         acc = fmaf(Dc, uu, acc);
-        const float zz = Store<T>::to_f(z[row * a.ld_z + c]);
-        y[row * E + c] = Store<T>::from_f(acc * silu_f(zz));
+        const float zz = Store<T>::to_f(sz[tt * bs + threadIdx.x]);
+        y[((long long)b * a.L + tb + tt) * E + c] = Store<T>::from_f(acc * silu_f(zz));
       } else {
         dsum += d;
       }
     }
+    __syncthreads();  // the buffer is refilled two blocks later
   }
   if (mode == 1) {
 #pragma unroll
     for (int n = 0; n < kStates; ++n) hend[sidx + n] = h[n];
     dsum_out[((long long)b * chunks + k) * E + c] = dsum;
   } else if (k == chunks - 1 && a.h_out) {
+    float4 *hp = reinterpret_cast<float4 *>(a.h_out + ((long long)b * E + c) * kStates);
 #pragma unroll
-    for (int n = 0; n < kStates; ++n) a.h_out[((long long)b * E + c) * kStates + n] = h[n];
+    for (int n = 0; n < kStates; n += 4) hp[n >> 2] = make_float4(h[n], h[n + 1], h[n + 2], h[n + 3]);
   }
 }
 
@@ -336,11 +420,24 @@ hymba_status selective_scan(const ScanArgs &a, hymba_dtype dt, cudaStream_t s) {
     hstart = hend + st;
     dsum = hstart + st;
   }
+  const int esz = dt == HYMBA_BF16 ? 2 : 4;
+  const int smem = 2 * (3 * kScanTB * bs * esz + kScanTB * 2 * kStates * 4);
+  {
+    static unsigned attr_set = 0;  // one bit per device
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!(attr_set & (1u << (dev & 31)))) {
+      const int most = 2 * (3 * kScanTB * 128 * 4 + kScanTB * 2 * kStates * 4);
+      cudaFuncSetAttribute(scan_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      cudaFuncSetAttribute(scan_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      attr_set |= 1u << (dev & 31);
+    }
+  }
   auto launch = [&](int mode) {
     if (dt == HYMBA_BF16)
-      scan_kernel<__nv_bfloat16><<<blocks, bs, 0, s>>>(a, chunks, Tc, mode, hstart, hend, dsum);
+      scan_kernel<__nv_bfloat16><<<blocks, bs, smem, s>>>(a, chunks, Tc, mode, hstart, hend, dsum);
     else
-      scan_kernel<float><<<blocks, bs, 0, s>>>(a, chunks, Tc, mode, hstart, hend, dsum);
+      scan_kernel<float><<<blocks, bs, smem, s>>>(a, chunks, Tc, mode, hstart, hend, dsum);
   };
   if (chunks > 1) {
     launch(1);
