@@ -91,6 +91,9 @@ _SIGS = {
     "hymba_version": (C.c_char_p, []),
     "hymba_debug_mask_bitmap": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_void_p,
                                           C.c_void_p, C.c_void_p]),
+    "hymba_layer_decode_step_static": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_void_p, C.c_void_p,
+                                                 C.POINTER(hymba_kv_cache), C.POINTER(hymba_ssm_cache),
+                                                 C.c_void_p]),
     "hymba_profile_enable": (C.c_int, [C.c_int]),
     "hymba_profile_collect": (C.c_int, [C.POINTER(hymba_profile_entry), C.c_int, C.POINTER(C.c_int)]),
 }
@@ -193,6 +196,18 @@ def hymba_layer_decode_step(layer: int, batch: int, pos: int, x_t, y_t, kv_cache
     check(lib().hymba_layer_decode_step(layer, batch, pos, _ptr(x_t), _ptr(y_t), C.byref(kv_cache),
                                         C.byref(ssm_cache), _ptr(workspace), workspace_bytes,
                                         _stream(stream)), "hymba_layer_decode_step")
+
+
+HYMBA_DECODE_STATIC_SCRATCH_BYTES = 40 << 20
+
+
+def hymba_layer_decode_step_static(layer: int, batch: int, pos: int, x_t, y_t,
+                                   kv_cache: hymba_kv_cache, ssm_cache: hymba_ssm_cache,
+                                   stream=None) -> None:
+    """hymba_layer_decode_step with the library's static scratch instead of a workspace."""
+    check(lib().hymba_layer_decode_step_static(layer, batch, pos, _ptr(x_t), _ptr(y_t),
+                                               C.byref(kv_cache), C.byref(ssm_cache),
+                                               _stream(stream)), "hymba_layer_decode_step_static")
 
 
 def hymba_stream_status(stream=None) -> None:

@@ -213,6 +213,32 @@ HYMBA_API hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, in
                                      hymba_ssm_cache *ssm_cache, void *workspace,
                                      size_t workspace_bytes, hymba_stream_t stream);
 
+/* Decode step that allocates nothing and takes no workspace argument.
+ *
+ * For callers that cannot call cudaMalloc: code whose device memory is all
+ * carved up in advance by another owner (an inference server's memory pool,
+ * an engine's arena) and that has no way to ask it for a workspace, or a
+ * latency-critical loop that must not pay for cudaMalloc's implicit device
+ * synchronisation.  This entry point has no counterpart on the paper's pages.
+ *
+ * It runs exactly hymba_layer_decode_step (same arguments, same results) with
+ * its scratch in a buffer of HYMBA_DECODE_STATIC_SCRATCH_BYTES that the
+ * library holds in device memory of every GPU that loads it, until exit.
+ * A request needing more scratch than that (hymba_layer_decode_workspace) is
+ * rejected with HYMBA_ERR_WORKSPACE before anything is launched; 40 MiB covers
+ * a batch of 128 on a sliding-window layer of the 1.5B shape (m + W = 1152).
+ * The first call on a device looks up the buffer's device address (with that
+ * device current); make that first call before any stream capture.  All calls
+ * share the one buffer, which keeps the last call's contents (the step zeroes
+ * what it accumulates into): calls that may overlap on the GPU race, so issue
+ * them in order on one stream. */
+#define HYMBA_DECODE_STATIC_SCRATCH_BYTES (40u << 20)
+HYMBA_API hymba_status hymba_layer_decode_step_static(hymba_layer *layer, int batch, int64_t pos,
+                                                      const void *x_t, void *y_t,
+                                                      hymba_kv_cache *kv_cache,
+                                                      hymba_ssm_cache *ssm_cache,
+                                                      hymba_stream_t stream);
+
 /* ---- status and diagnostics -------------------------------------------- */
 
 /* Synchronises `stream`, then reports a pending CUDA error or a device-side
