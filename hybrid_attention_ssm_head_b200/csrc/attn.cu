@@ -765,6 +765,185 @@ __global__ void __launch_bounds__(128)
   }
 }
 
+// ---- bf16 decode attention on the tensor cores (mma.sync m16n8k16) ---------------
+// CTA = 128 slots of one (sequence, kv head); the K and V chunks arrive by 3-D TMA
+// (128-byte swizzle, rows past the store's capacity read as zero); warp w takes keys
+// 32w..32w+31: S = Q K^T with the query heads of the group in rows 0..rep-1 of a
+// 16-row tile, softmax in registers, O += P V with V fragments from ldmatrix.trans.
+// The four warps' partial results are merged in shared memory.
+namespace dtc {
+constexpr int SLOTS = 128;
+constexpr int K_BYTES = SLOTS * 128;        // 64 bf16 per slot
+constexpr int V_BYTES = SLOTS * 256;        // two 64-column boxes
+constexpr int SMEM = K_BYTES + V_BYTES + 4 * 8 * 130 * 4 + 64 + 1024;
+}  // namespace dtc
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                          uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// byte offset of 16-byte chunk `ch` (0..7) of row `row` in a 128-byte-swizzled tile
+__device__ __forceinline__ uint32_t sw128(int row, int ch) {
+  return uint32_t(row * 128 + ((ch ^ (row & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(128)
+    attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                          const __nv_bfloat16 *__restrict__ q, float *__restrict__ part, int H,
+                          int Hkv, long long pos, int n_meta, int window, int is_global,
+                          float scale_log2, int nsplit) {
+  using namespace dtc;
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t *sm = dsm_raw + ((1024 - (smem_u32(dsm_raw) & 1023)) & 1023);
+  float *om = reinterpret_cast<float *>(sm + K_BYTES + V_BYTES);  // [4 warps][8 rows][130]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(om + 4 * 8 * 130);
+  const int split = blockIdx.y, bg = blockIdx.x;
+  const int b = bg / Hkv, g = bg % Hkv;
+  const int rep = H / Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gr = lane >> 2, gc = lane & 3;  // mma group row / column pair
+  const long long s0 = (long long)split * SLOTS;
+  const long long nslots = dec_slots(pos, n_meta, window, is_global);
+  const int ns = (int)min((long long)SLOTS, nslots - s0);
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar, K_BYTES + V_BYTES);
+    tma_load_3d(sm, &tmK, bar, 0, (int)s0, bg);
+    tma_load_3d(sm + K_BYTES, &tmV, bar, 0, (int)s0, bg);
+    tma_load_3d(sm + K_BYTES + V_BYTES / 2, &tmV, bar, 64, (int)s0, bg);
+  }
+  // Q fragments (row = query head of the group, zero beyond rep), from global memory
+  uint32_t qa[4][2];  // [k-step][a0a1 / a4a5]; rows 8..15 are zero
+  {
+    const bool live = gr < rep;
+    const uint32_t *qr = reinterpret_cast<const uint32_t *>(q + ((long long)b * H + g * rep + (live ? gr : 0)) * 64);
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      qa[ks][0] = live ? __ldg(qr + ks * 8 + gc) : 0u;
+      qa[ks][1] = live ? __ldg(qr + ks * 8 + 4 + gc) : 0u;
+    }
+  }
+  bool ok = mbar_wait(bar, 0, &g_err_attn);
+  if (!ok && tid == 0) mbar_wait_drain(bar, 0, &g_err_attn);
+  const uint32_t kb = smem_u32(sm), vb = smem_u32(sm + K_BYTES);
+  // ---- S = Q K^T for this warp's 32 keys (4 n-tiles of 8 keys) ----
+  float sacc[4][4];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+    const int key = warp * 32 + nt * 8 + (lane & 7);
+#pragma unroll
+    for (int kp = 0; kp < 2; ++kp) {  // two k-steps per ldmatrix.x4
+      const int ch = kp * 4 + (lane >> 3);  // 16-byte chunk of the key row (8 dims)
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(kb + sw128(key, ch), b0, b1, b2, b3);
+      mma16816(sacc[nt], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b0, b1);
+      mma16816(sacc[nt], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b2, b3);
+    }
+  }
+  // ---- softmax over the warp's keys, row gr (values sacc[nt][0..1], keys 8nt + 2gc + {0,1}) ----
+  float mx = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int key = warp * 32 + nt * 8 + 2 * gc + e;
+      const bool valid = ok && key < ns && dec_slot_valid(s0 + key, pos, n_meta, window, is_global);
+      const float x = valid ? sacc[nt][e] * scale_log2 : -INFINITY;
+      sacc[nt][e] = x;
+      mx = fmaxf(mx, x);
+    }
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+  const float mref = mx == -INFINITY ? 0.f : mx;
+  float lsum = 0.f;
+  uint32_t pa[4];  // P as A fragments: [k-step kk][a0a1 (n-tile 2kk) / a4a5 (n-tile 2kk+1)]
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+    const float p0 = ex2(sacc[nt][0] - mref), p1 = ex2(sacc[nt][1] - mref);
+    lsum += p0 + p1;
+    pa[nt] = pack_bf16x2(p0, p1);
+  }
+  lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+  lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+  // ---- O = P V (16 n-tiles of 8 value columns, 2 k-steps of 16 keys) ----
+  float oacc[16][4];
+#pragma unroll
+  for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) oacc[nt][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < 2; ++kk) {
+    const int key = warp * 32 + kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int np = 0; np < 8; ++np) {  // pairs of n-tiles per ldmatrix.x4.trans
+      const int chg = np * 2 + (lane >> 4);  // 16-byte chunk of value columns (0..15)
+      const uint32_t addr = vb + (chg >> 3) * (V_BYTES / 2) + sw128(key, chg & 7);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4_t(addr, b0, b1, b2, b3);
+      mma16816(oacc[2 * np], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b0, b1);
+      mma16816(oacc[2 * np + 1], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b2, b3);
+    }
+  }
+  // ---- merge the four warps: rows 0..rep-1 ----
+  float *mw = om;  // per warp: [8 rows][130] = m, l, o[128]
+  if (gr < 8) {
+    float *row = mw + (warp * 8 + gr) * 130;
+    if (gc == 0) {
+      row[0] = mx;
+      row[1] = lsum;
+    }
+#pragma unroll
+    for (int nt = 0; nt < 16; ++nt) {
+      row[2 + nt * 8 + 2 * gc] = oacc[nt][0];
+      row[2 + nt * 8 + 2 * gc + 1] = oacc[nt][1];
+    }
+  }
+  __syncthreads();
+  for (int idx = tid; idx < rep * 130; idx += 128) {
+    const int r = idx / 130, col = idx % 130;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, mw[(w * 8 + r) * 130]);
+    float acc = 0.f;
+    if (col == 0) {
+      acc = M;
+    } else {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float mw_ = mw[(w * 8 + r) * 130];
+        if (mw_ != -INFINITY) acc += mw[(w * 8 + r) * 130 + col] * ex2(mw_ - M);
+      }
+    }
+    part[(((long long)b * H + g * rep + r) * nsplit + split) * 130 + col] = acc;
+  }
+}
+
 template <typename T>
 __global__ void attn_decode_combine_kernel(const float *__restrict__ part, T *__restrict__ o, int H,
                                            int dv, int nsplit) {
@@ -813,7 +992,30 @@ hymba_status attention_decode(const DecodeAttnArgs &a, hymba_dtype dt, cudaStrea
       attr_set |= 1u << (dev & 31);
     }
   }
-  if (dt == HYMBA_BF16) {
+  if (dt == HYMBA_BF16 && a.dqk == 64 && a.dv == 128) {
+    static unsigned attr_tc = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!(attr_tc & (1u << (dev & 31)))) {
+      cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dtc::SMEM);
+      attr_tc |= 1u << (dev & 31);
+    }
+    CUtensorMap tk, tv;
+    const uint64_t dk[3] = {64, (uint64_t)a.cap, (uint64_t)a.B * a.Hkv};
+    const uint64_t sk[2] = {64 * 2, (uint64_t)a.cap * 64 * 2};
+    const uint64_t dvv[3] = {128, (uint64_t)a.cap, (uint64_t)a.B * a.Hkv};
+    const uint64_t svv[2] = {128 * 2, (uint64_t)a.cap * 128 * 2};
+    const uint32_t box[3] = {64, (uint32_t)dtc::SLOTS, 1};
+    if (!make_tmap(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dk, sk, box)) return HYMBA_ERR_CUDA;
+    if (!make_tmap(&tv, a.v_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dvv, svv, box)) return HYMBA_ERR_CUDA;
+    const int ns_tc = (int)((nslots + dtc::SLOTS - 1) / dtc::SLOTS);
+    dim3 grid_tc(a.B * a.Hkv, ns_tc);
+    attn_decode_tc_kernel<<<grid_tc, 128, dtc::SMEM, s>>>(tk, tv, (const __nv_bfloat16 *)a.q, a.partial,
+                                                         a.H, a.Hkv, a.pos, a.n_meta, a.window,
+                                                         a.is_global, sl2, ns_tc);
+    attn_decode_combine_kernel<__nv_bfloat16><<<a.B * a.H, 128, 0, s>>>(
+        a.partial, (__nv_bfloat16 *)a.o, a.H, a.dv, ns_tc);
+  } else if (dt == HYMBA_BF16) {
     attn_decode_partial_kernel<__nv_bfloat16><<<grid, 128, dsmem, s>>>(
         (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k_cache, (const __nv_bfloat16 *)a.v_cache,
         a.partial, a.H, a.Hkv, a.dqk, a.dv, a.cap, a.pos, a.n_meta, a.window, a.is_global, sl2, nsplit);

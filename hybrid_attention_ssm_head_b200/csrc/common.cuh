@@ -63,9 +63,9 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
 // (relative error e^x / 2 < 2e-4); in between log(1 + e^x) with 1 + e^x >= 1 + 3e-4,
 // so the fp32 rounding of the sum costs at most ~2e-4 relative.
 __device__ __forceinline__ float softplus_f(float x) {
-  if (x > 20.0f) return x;
-  const float e = __expf(x);
-  return x < -8.0f ? e : __logf(1.0f + e);
+  const float e = __expf(fminf(x, 20.0f));
+  const float l = __logf(1.0f + e);
+  return x > 20.0f ? x : (x < -8.0f ? e : l);  // selects, no divergence
 }
 // Full-precision variant for the fp32 storage path.
 __device__ __forceinline__ float softplus_accurate(float x) {

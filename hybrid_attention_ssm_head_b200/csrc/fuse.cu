@@ -12,11 +12,11 @@ template <typename T>
 __device__ __forceinline__ void ld16(const T *p, float (&v)[16 / sizeof(T)]) {
   uint4 raw = __ldg(reinterpret_cast<const uint4 *>(p));
   if constexpr (sizeof(T) == 2) {
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __low2float(h[i]);
-      v[2 * i + 1] = __high2float(h[i]);
+      v[2 * i] = bf16_lo(w[i]);
+      v[2 * i + 1] = bf16_hi(w[i]);
     }
   } else {
     const float *f = reinterpret_cast<const float *>(&raw);
@@ -69,10 +69,16 @@ __global__ void __launch_bounds__(128) fuse_kernel(FuseArgs a) {
   for (int j = 0; j < NV; ++j) {
     const int c = (threadIdx.x + j * 128) * V;
     if (c < a.E) {
-      float out[V];
+      float ba[V], bs[V], out[V];
 #pragma unroll
-      for (int i = 0; i < V; ++i)
-        out[i] = fmaf(__ldg(a.beta_attn + c + i) * ro, vo[j][i], __ldg(a.beta_ssm + c + i) * ry * vy[j][i]);
+      for (int i = 0; i < V; i += 4) {  // per-channel beta as 16-byte loads
+        const float4 a4 = __ldg(reinterpret_cast<const float4 *>(a.beta_attn + c + i));
+        const float4 s4 = __ldg(reinterpret_cast<const float4 *>(a.beta_ssm + c + i));
+        ba[i] = a4.x; ba[i + 1] = a4.y; ba[i + 2] = a4.z; ba[i + 3] = a4.w;
+        bs[i] = s4.x; bs[i + 1] = s4.y; bs[i + 2] = s4.z; bs[i + 3] = s4.w;
+      }
+#pragma unroll
+      for (int i = 0; i < V; ++i) out[i] = fmaf(ba[i] * ro, vo[j][i], bs[i] * ry * vy[j][i]);
       if constexpr (sizeof(T) == 2) {
         st_global_v4(f + c, pack_bf16x2(out[0], out[1]), pack_bf16x2(out[2], out[3]),
                      pack_bf16x2(out[4], out[5]), pack_bf16x2(out[6], out[7]));

@@ -114,6 +114,27 @@ __device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, int 
       for (int i = 0; i < 16; ++i) v[i] = softplus_f(v[i]);
     }
   }
+  // common case: the 16 columns lie in one segment and one group, 16-byte aligned rows
+  const int sidx = find_seg(e, n0);
+  const EpiSeg &g = e.seg[sidx];
+  const int local = n0 - g.col0;
+  if (full && !e.atomic && g.vec_ok && n0 + 16 <= g.col1 && (local % g.inner) + 16 <= g.inner) {
+    const long long off = m * g.ld_row + (long long)(local / g.inner) * g.ld_group + (local % g.inner);
+    if (g.f32) {
+      float *p = reinterpret_cast<float *>(g.ptr) + off;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        st_global_v4(p + 4 * q, __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                     __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+    } else {
+      __nv_bfloat16 *p = reinterpret_cast<__nv_bfloat16 *>(g.ptr) + off;
+      st_global_v4(p, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                   pack_bf16x2(v[6], v[7]));
+      st_global_v4(p + 8, pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                   pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+    }
+    return;
+  }
   float a[8], b[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {

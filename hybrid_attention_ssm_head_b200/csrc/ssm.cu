@@ -28,6 +28,14 @@ __device__ __forceinline__ float ex2f_(float x) {
   return y;
 }
 
+// Decay factors exp2(x) of two states, fp32 MUFU.  (A packed f16 exp2 halves the
+// MUFU work but resolves factors near 1 only to ~5e-4 absolute, which moves slowly
+// decaying states by 1-2%: not used.)
+template <typename T>
+__device__ __forceinline__ float2 decay2(float2 x) {
+  return make_float2(ex2f_(x.x), ex2f_(x.y));
+}
+
 // ---------------------------------------------------------------------------
 // causal conv + SiLU (prefill)
 // ---------------------------------------------------------------------------
@@ -67,7 +75,7 @@ __device__ __forceinline__ void store_vec(T *p, const float (&v)[Vec16<T>::N]) {
   *reinterpret_cast<uint4 *>(p) = raw;
 }
 
-constexpr int kConvTB = 4;
+constexpr int kConvTB = 16;
 
 template <typename T>
 __device__ __forceinline__ void unpack16(const uint4 &raw, float (&v)[16 / sizeof(T)]) {
@@ -86,10 +94,10 @@ __device__ __forceinline__ void unpack16(const uint4 &raw, float (&v)[16 / sizeo
 }
 
 // One thread: VEC channels x kConvTB rows.  Its kConvTB + 3 input rows are loaded
-// up front as 16-byte vectors (coalesced across the warp); the overlap with the
-// neighbouring row blocks is served by L2.
+// up front as 16-byte vectors (coalesced across the warp); the taps (one 16-byte
+// vector per channel) and the bias are fetched once for all kConvTB rows.
 template <typename T>
-__global__ void __launch_bounds__(256) conv_silu_kernel(ConvArgs a) {
+__global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
   constexpr int V = Vec16<T>::N;
   constexpr int NR = kConvTB + 3;
   const int nvec = a.E / V;
@@ -113,36 +121,54 @@ __global__ void __launch_bounds__(256) conv_silu_kernel(ConvArgs a) {
                  ? __ldg(reinterpret_cast<const uint4 *>(x + ((long long)b * a.L + t) * a.ld_x + c0))
                  : make_uint4(0, 0, 0, 0);
   }
-  float acc[kConvTB][V];
+  // wj[j][i] multiplies x[t - 3 + j] for channel c0 + i (taps right-aligned)
+  float wj[4][V], bias[V];
+  if (K == 4) {
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const float bi = __ldg(a.bias + c0 + i);
-#pragma unroll
-    for (int tt = 0; tt < kConvTB; ++tt) acc[tt][i] = bi;
-  }
-  // wj multiplies x[t - 3 + j] (taps right-aligned so every index is static)
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int k = j - (4 - K);
-    if (k < 0) continue;
-    float wj[V];
-#pragma unroll
-    for (int i = 0; i < V; ++i) wj[i] = __ldg(a.w + (c0 + i) * K + k);
-#pragma unroll
-    for (int tt = 0; tt < kConvTB; ++tt) {
-      float xv[V];
-      unpack16<T>(raw[tt + j], xv);
-#pragma unroll
-      for (int i = 0; i < V; ++i) acc[tt][i] = fmaf(wj[i], xv[i], acc[tt][i]);
+    for (int i = 0; i < V; ++i) {
+      const float4 w4 = __ldg(reinterpret_cast<const float4 *>(a.w + (c0 + i) * 4));
+      wj[0][i] = w4.x;
+      wj[1][i] = w4.y;
+      wj[2][i] = w4.z;
+      wj[3][i] = w4.w;
     }
+  } else {
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int k = j - (4 - K);
+        wj[j][i] = k >= 0 ? __ldg(a.w + (c0 + i) * K + k) : 0.f;
+      }
   }
+#pragma unroll
+  for (int i = 0; i < V; i += 4) {
+    const float4 b4 = __ldg(reinterpret_cast<const float4 *>(a.bias + c0 + i));
+    bias[i] = b4.x;
+    bias[i + 1] = b4.y;
+    bias[i + 2] = b4.z;
+    bias[i + 3] = b4.w;
+  }
+  float xv[4][V];  // rolling window of converted rows t-3 .. t
+#pragma unroll
+  for (int j = 0; j < 3; ++j) unpack16<T>(raw[j], xv[j + 1]);
 #pragma unroll
   for (int tt = 0; tt < kConvTB; ++tt) {
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+#pragma unroll
+      for (int i = 0; i < V; ++i) xv[j][i] = xv[j + 1][i];
+    unpack16<T>(raw[tt + 3], xv[3]);
     const int t = t0 + tt;
     if (t < a.L) {
       float o[V];
 #pragma unroll
-      for (int i = 0; i < V; ++i) o[i] = silu_f(acc[tt][i]);
+      for (int i = 0; i < V; ++i) {
+        float acc = bias[i];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc = fmaf(wj[j][i], xv[j][i], acc);
+        o[i] = silu_f(acc);
+      }
       store_vec<T>(u + ((long long)b * a.L + t) * a.E + c0, o);
     }
   }
@@ -166,11 +192,11 @@ hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s) {
   const int V = dt == HYMBA_BF16 ? 8 : 4;
   const long long n = (long long)a.B * ((a.L + kConvTB - 1) / kConvTB) * (a.E / V);
   if (n == 0) return HYMBA_OK;
-  const unsigned blocks = (unsigned)((n + 255) / 256);
+  const unsigned blocks = (unsigned)((n + 127) / 128);
   if (dt == HYMBA_BF16)
-    conv_silu_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(a);
+    conv_silu_kernel<__nv_bfloat16><<<blocks, 128, 0, s>>>(a);
   else
-    conv_silu_kernel<float><<<blocks, 256, 0, s>>>(a);
+    conv_silu_kernel<float><<<blocks, 128, 0, s>>>(a);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -279,26 +305,27 @@ __global__ void __launch_bounds__(128)
     cp_async_commit();
   };
 
-  float A2[kStates], h[kStates];
+  // state and A (pre-scaled by log2 e) as register pairs for the packed fp32x2 ops
+  float2 A2[kStates / 2], h[kStates / 2];
 #pragma unroll
-  for (int n = 0; n < kStates; ++n) A2[n] = -__expf(a.a_log[c * kStates + n]) * 1.4426950408889634f;
+  for (int n = 0; n < kStates; n += 2)
+    A2[n / 2] = make_float2(-__expf(a.a_log[c * kStates + n]) * 1.4426950408889634f,
+                            -__expf(a.a_log[c * kStates + n + 1]) * 1.4426950408889634f);
   const long long sidx = (((long long)b * chunks + k) * E + c) * kStates;
-  if (mode == 0 && chunks > 1) {
-#pragma unroll
-    for (int n = 0; n < kStates; ++n) h[n] = hstart[sidx + n];
-  } else if (mode == 0 && a.h_in) {
-    const float4 *hp = reinterpret_cast<const float4 *>(a.h_in + ((long long)b * E + c) * kStates);
+  const float *h0 = nullptr;
+  if (mode == 0 && chunks > 1) h0 = hstart + sidx;
+  else if (mode == 0 && a.h_in) h0 = a.h_in + ((long long)b * E + c) * kStates;
+  if (h0) {
+    const float4 *hp = reinterpret_cast<const float4 *>(h0);
 #pragma unroll
     for (int n = 0; n < kStates; n += 4) {
       const float4 v4 = hp[n >> 2];
-      h[n] = v4.x;
-      h[n + 1] = v4.y;
-      h[n + 2] = v4.z;
-      h[n + 3] = v4.w;
+      h[n / 2] = make_float2(v4.x, v4.y);
+      h[n / 2 + 1] = make_float2(v4.z, v4.w);
     }
   } else {
 #pragma unroll
-    for (int n = 0; n < kStates; ++n) h[n] = 0.f;
+    for (int n = 0; n < kStates / 2; ++n) h[n] = make_float2(0.f, 0.f);
   }
   const float Dc = a.d_skip[c];
   float dsum = 0.f;
@@ -324,20 +351,23 @@ __global__ void __launch_bounds__(128)
       const float d = Store<T>::to_f(sd[tt * bs + threadIdx.x]);
       const float uu = Store<T>::to_f(su[tt * bs + threadIdx.x]);
       const float du = d * uu;
-      const float2 *bc2 = reinterpret_cast<const float2 *>(sbc + tt * 2 * kStates);
+      const float4 *bc4 = reinterpret_cast<const float4 *>(sbc + tt * 2 * kStates);
       const float2 d2 = make_float2(d, d), du2 = make_float2(du, du);
-      float2 acc2 = make_float2(0.f, 0.f);
+      float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};  // two chains
 #pragma unroll
-      for (int n = 0; n < kStates; n += 2) {
-        const float2 x2 = fmul2(d2, make_float2(A2[n], A2[n + 1]));
-        const float2 dA2 = make_float2(ex2f_(x2.x), ex2f_(x2.y));
-        const float2 hb = fmul2(du2, bc2[n >> 1]);
-        float2 hv = ffma2(dA2, make_float2(h[n], h[n + 1]), hb);
-        h[n] = hv.x;
-        h[n + 1] = hv.y;
-        acc2 = ffma2(bc2[(kStates + n) >> 1], hv, acc2);
+      for (int qd = 0; qd < kStates / 4; ++qd) {
+        const float4 B4 = bc4[qd], C4 = bc4[kStates / 4 + qd];
+        const float2 Bp[2] = {make_float2(B4.x, B4.y), make_float2(B4.z, B4.w)};
+        const float2 Cp[2] = {make_float2(C4.x, C4.y), make_float2(C4.z, C4.w)};
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int n2 = 2 * qd + e;
+          const float2 dA = decay2<T>(fmul2(d2, A2[n2]));
+          h[n2] = ffma2(dA, h[n2], fmul2(du2, Bp[e]));
+          acc2[e] = ffma2(Cp[e], h[n2], acc2[e]);
+        }
       }
-      float acc = acc2.x + acc2.y;
+      float acc = (acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y);
       if (mode == 0) {
         acc = fmaf(Dc, uu, acc);
         const float zz = Store<T>::to_f(sz[tt * bs + threadIdx.x]);
@@ -350,13 +380,51 @@ __global__ void __launch_bounds__(128)
   }
   if (mode == 1) {
 #pragma unroll
-    for (int n = 0; n < kStates; ++n) hend[sidx + n] = h[n];
+    for (int n = 0; n < kStates; n += 2) {
+      hend[sidx + n] = h[n / 2].x;
+      hend[sidx + n + 1] = h[n / 2].y;
+    }
     dsum_out[((long long)b * chunks + k) * E + c] = dsum;
   } else if (k == chunks - 1 && a.h_out) {
     float4 *hp = reinterpret_cast<float4 *>(a.h_out + ((long long)b * E + c) * kStates);
 #pragma unroll
-    for (int n = 0; n < kStates; n += 4) hp[n >> 2] = make_float4(h[n], h[n + 1], h[n + 2], h[n + 3]);
+    for (int n = 0; n < kStates; n += 4)
+      hp[n >> 2] = make_float4(h[n / 2].x, h[n / 2].y, h[n / 2 + 1].x, h[n / 2 + 1].y);
   }
+}
+
+// One decode step (L = 1) from the stored state: thread per (sequence, channel),
+// the 16 states as four 16-byte loads and stores.
+template <typename T>
+__global__ void __launch_bounds__(256) scan_step_kernel(ScanArgs a) {
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)a.B * a.E) return;
+  const int c = int(idx % a.E), b = int(idx / a.E);
+  const T *u = reinterpret_cast<const T *>(a.u);
+  const T *dl = reinterpret_cast<const T *>(a.delta);
+  const T *z = reinterpret_cast<const T *>(a.z);
+  const float d = Store<T>::to_f(dl[(long long)b * a.E + c]);
+  const float uu = Store<T>::to_f(u[(long long)b * a.E + c]);
+  const float zz = Store<T>::to_f(z[(long long)b * a.ld_z + c]);
+  const float4 *bc4 = reinterpret_cast<const float4 *>(a.bc + (long long)b * a.ld_bc + a.bc_col);
+  const float4 *al4 = reinterpret_cast<const float4 *>(a.a_log + (long long)c * kStates);
+  const float4 *hi4 = reinterpret_cast<const float4 *>(a.h_in + ((long long)b * a.E + c) * kStates);
+  float4 *ho4 = reinterpret_cast<float4 *>(a.h_out + ((long long)b * a.E + c) * kStates);
+  const float du = d * uu;
+  float acc = 0.f;
+#pragma unroll
+  for (int q4 = 0; q4 < kStates / 4; ++q4) {
+    const float4 hv = hi4[q4], al = __ldg(al4 + q4), Bv = __ldg(bc4 + q4), Cv = __ldg(bc4 + kStates / 4 + q4);
+    float4 hn;
+    hn.x = fmaf(ex2f_(-__expf(al.x) * 1.4426950408889634f * d), hv.x, du * Bv.x);
+    hn.y = fmaf(ex2f_(-__expf(al.y) * 1.4426950408889634f * d), hv.y, du * Bv.y);
+    hn.z = fmaf(ex2f_(-__expf(al.z) * 1.4426950408889634f * d), hv.z, du * Bv.z);
+    hn.w = fmaf(ex2f_(-__expf(al.w) * 1.4426950408889634f * d), hv.w, du * Bv.w);
+    acc = fmaf(Cv.x, hn.x, fmaf(Cv.y, hn.y, fmaf(Cv.z, hn.z, fmaf(Cv.w, hn.w, acc))));
+    ho4[q4] = hn;
+  }
+  acc = fmaf(a.d_skip[c], uu, acc);
+  reinterpret_cast<T *>(a.y)[(long long)b * a.E + c] = Store<T>::from_f(acc * silu_f(zz));
 }
 
 // Chains chunk start states: H_0 = h_in (or 0); H_{k+1} = exp(A * dsum_k) H_k + hend_k.
@@ -408,6 +476,21 @@ static int scan_block(int E) {
 }
 
 hymba_status selective_scan(const ScanArgs &a, hymba_dtype dt, cudaStream_t s) {
+  if (a.L == 1 && a.h_in && a.h_out) {
+    const long long n = (long long)a.B * a.E;
+    const unsigned blocks = (unsigned)((n + 255) / 256);
+    if (dt == HYMBA_BF16)
+      scan_step_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(a);
+    else
+      scan_step_kernel<float><<<blocks, 256, 0, s>>>(a);
+    note_launch(1);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      set_error("scan step launch failed: %s", cudaGetErrorString(e));
+      return HYMBA_ERR_CUDA;
+    }
+    return HYMBA_OK;
+  }
   int chunks = 1;
   scan_workspace_floats(a.B, a.L, a.E, a.N, &chunks);
   const int Tc = (a.L + chunks - 1) / chunks;
