@@ -36,6 +36,13 @@ import torch  # noqa: E402
 METRIC = "hybrid-layer prefill tok/s @B=128,L=8k bf16 + decode tok/s; % of roofline"
 UNIT = "tok/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one in_proj launch: ncu dram__bytes_{read,write}.sum of the
+# in_proj launch of `bench.py --case b32` (36,864 rows: 156.06 MB + 616.80 MB, see
+# profiles/gemm_b32.md), scaled by rows to one producer launch of the headline prefill
+# (1,064,960 rows).  The algorithmic minimum is 22.5 GB (read X~ and W_in, write the
+# 8960 output columns), so the kernel re-reads nothing.
+IN_PROJ_TRAFFIC = (156.06e6 + 616.80e6) * 1064960 / 36864
+IN_PROJ_TRAFFIC_BASIS = "ncu b32 in_proj capture scaled by rows to one producer launch"
 
 
 def load_peaks():
@@ -331,7 +338,8 @@ def run_ours(args, rank, world, dev):
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     roof = {"kernel": "in_proj (gemm_tc_kernel<256,bf16>)", "bound": "tensor",
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": (achieved / peak) if achieved else None, "traffic": None,
+            "frac": (achieved / peak) if achieved else None, "traffic": IN_PROJ_TRAFFIC,
+            "traffic_basis": IN_PROJ_TRAFFIC_BASIS,
             "peak_source": f"{peak_src} bf16_tflops_sustained"}
     step_flops = pre.flops()
     dec_bytes = dec.hbm_bytes()

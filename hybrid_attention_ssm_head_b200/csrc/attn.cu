@@ -110,10 +110,9 @@ __device__ __forceinline__ float max32(const uint32_t (&v)[32]) {
   for (int e = 8; e < 32; ++e) m[e & 7] = fmaxf(m[e & 7], __uint_as_float(v[e]));
   return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
 }
-// P for keys c*32 .. c*32+31 of row r: exp2, bf16, swizzled K-major store; returns the sum.
-__device__ __forceinline__ float p_chunk(const uint32_t (&v)[32], int c, int r, uint32_t p_base,
-                                         float scale_log2, float nm) {
-  uint32_t pk[16];
+// P for 32 keys of a row: exp2(s * scale - m) packed to bf16 pairs; returns the fp32 sum.
+__device__ __forceinline__ float p_pack(const uint32_t (&v)[32], uint32_t (&pk)[16], float scale_log2,
+                                        float nm) {
   float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
@@ -122,6 +121,11 @@ __device__ __forceinline__ float p_chunk(const uint32_t (&v)[32], int c, int r, 
     ls[(e >> 1) & 3] += p0 + p1;
     pk[e >> 1] = pack_bf16x2(p0, p1);
   }
+  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
+}
+// Keys c*32 .. c*32+31 of row r into the 128-byte swizzled K-major P tile
+// (atom c/2, 16-byte chunks (c%2)*4 .. +3).
+__device__ __forceinline__ void p_store(const uint32_t (&pk)[16], int c, int r, uint32_t p_base) {
   const uint32_t atom = p_base + (c >> 1) * (fa::P_BYTES / 2) + r * 128;
 #pragma unroll
   for (int t = 0; t < 4; ++t) {
@@ -129,7 +133,6 @@ __device__ __forceinline__ float p_chunk(const uint32_t (&v)[32], int c, int r, 
     st_shared_v4(atom + ((chunk ^ (r & 7)) << 4), pk[4 * t], pk[4 * t + 1], pk[4 * t + 2],
                  pk[4 * t + 3]);
   }
-  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
 }
 
 __global__ void __launch_bounds__(fa::THREADS, 1)
@@ -353,6 +356,12 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         resc = true;
       }
       l_run *= alpha;
+      // P = exp2(s * scale - m) into packed bf16 registers first, so that the wait for
+      // the previous tile's P V (which still reads the P buffer) overlaps the exps
+      const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+      uint32_t pk0[16], pk1[16], pk2[16], pk3[16];
+      l_run += (p_pack(s0, pk0, scale_log2, nm) + p_pack(s1, pk1, scale_log2, nm)) +
+               (p_pack(s2, pk2, scale_log2, nm) + p_pack(s3, pk3, scale_log2, nm));
       if (j > 0) {
         if (!mbar_wait(&o_done[q], uint32_t(j - 1) & 1u, &g_err_attn)) { ok = false; break; }
         tc_fence_after();
@@ -369,10 +378,10 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
           tmem_wait_st();
         }
       }
-      // P = exp2(s * scale - m) -> bf16 into the swizzled K-major tile; fp32 row sum
-      const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-      l_run += (p_chunk(s0, 0, r, p_base, scale_log2, nm) + p_chunk(s1, 1, r, p_base, scale_log2, nm)) +
-               (p_chunk(s2, 2, r, p_base, scale_log2, nm) + p_chunk(s3, 3, r, p_base, scale_log2, nm));
+      p_store(pk0, 0, r, p_base);
+      p_store(pk1, 1, r, p_base);
+      p_store(pk2, 2, r, p_base);
+      p_store(pk3, 3, r, p_base);
       fence_proxy_async();
       tc_fence_before();
       __syncwarp();
