@@ -527,7 +527,7 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
 // decode
 // ---------------------------------------------------------------------------
 struct DecodeLayout {
-  size_t q, x_ssm, z, u, xdbl, delta, y_ssm, o, f, y32, part, total;
+  size_t q, x_ssm, z, u, xdbl, y_ssm, o, f, y32, part, total;
 };
 
 static DecodeLayout decode_layout(const hymba_layer_config &c, int batch, long long pos) {
@@ -544,7 +544,6 @@ static DecodeLayout decode_layout(const hymba_layer_config &c, int batch, long l
   d.z = take(B * E * es);
   d.u = take(B * E * es);
   d.xdbl = take(B * xdbl_width(c) * 4);
-  d.delta = take(B * E * es);
   d.y_ssm = take(B * E * es);
   d.o = take(B * E * es);
   d.f = take(B * E * es);
@@ -604,7 +603,7 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
   char *ws = reinterpret_cast<char *>(workspace);
   void *q = ws + d.q, *xs = ws + d.x_ssm, *z = ws + d.z, *u = ws + d.u;
   float *xdbl = reinterpret_cast<float *>(ws + d.xdbl);
-  void *delta = ws + d.delta, *yssm = ws + d.y_ssm, *o = ws + d.o, *f = ws + d.f;
+  void *yssm = ws + d.y_ssm, *o = ws + d.o, *f = ws + d.f;
   float *y32 = reinterpret_cast<float *>(ws + d.y32);
   float *part = reinterpret_cast<float *>(ws + d.part);
   hymba_status st;
@@ -632,84 +631,32 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
                              cap * c.head_dim_qk, cap * c.head_dim_v, xs, z, E);
     if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
   }
-  // 2. conv over the stored window + SiLU
+  // 2-5. SSM branch: conv + x_proj, then dt_proj + softplus + one scan step + gate
   {
-    ProfScope prof_scope(stream, "dec_conv");
-    DecodeConvArgs a{};
+    ProfScope prof_scope(stream, "dec_ssm");
+    DecodeSsmArgs a{};
     a.x = xs;
     a.ld_x = E;
+    a.z = z;
+    a.ld_z = E;
     a.conv_state = ssm_cache->conv;
+    a.conv_w = layer->w.conv_w;
+    a.conv_b = layer->w.conv_b;
+    a.w_x = layer->w.w_x;
+    a.xdbl = xdbl;
     a.u = u;
-    a.w = layer->w.conv_w;
-    a.bias = layer->w.conv_b;
+    a.w_dt = layer->w.w_dt;
+    a.b_dt = layer->w.b_dt;
+    a.a_log = layer->w.a_log;
+    a.d_skip = layer->w.d_skip;
+    a.h = ssm_cache->h;
+    a.y = yssm;
     a.B = batch;
     a.E = E;
     a.K = c.d_conv;
-    if ((st = decode_conv(a, c.dtype, stream)) != HYMBA_OK) return st;
-  }
-  // 3. x_proj, split over K into a zeroed fp32 buffer
-  {
-    ProfScope prof_scope(stream, "dec_x_proj");
-    const int ksplit = c.dtype == HYMBA_BF16 ? std::max(1, std::min(32, E / 128)) : 4;
-    if (cudaMemsetAsync(xdbl, 0, (size_t)batch * xdbl_width(c) * 4, stream) != cudaSuccess)
-      FAIL(HYMBA_ERR_CUDA, "memset failed");
-    GemmArgs g{};
-    g.A = u;
-    g.lda = E;
-    g.B = layer->w.w_x;
-    g.ldb = E;
-    g.M = batch;
-    g.N = xdbl_width(c);
-    g.K = E;
-    g.elem = (int)es;
-    g.ksplit = ksplit;
-    g.epi.seg[0] = seg(xdbl, xdbl_width(c), 0, xdbl_width(c), 1, es);
-    g.epi.nseg = 1;
-    g.epi.atomic = 1;
-    if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
-  }
-  // 4. dt_proj + softplus
-  {
-    ProfScope prof_scope(stream, "dec_dt_proj");
-    GemmArgs g{};
-    g.A = xdbl;
-    g.lda = xdbl_width(c);
-    g.B = layer->w.w_dt;
-    g.ldb = c.dt_rank;
-    g.M = batch;
-    g.N = E;
-    g.K = c.dt_rank;
-    g.elem = 4;
-    g.ksplit = 1;
-    g.epi.seg[0] = seg(delta, E, 0, E, c.dtype == HYMBA_F32, es);
-    g.epi.nseg = 1;
-    g.epi.bias = layer->w.b_dt;
-    g.epi.act = 1;
-    st = c.dtype == HYMBA_BF16 ? gemm_tc(g, stream) : gemm_simt_f32(g, stream);
-    if (st != HYMBA_OK) return st;
-  }
-  // 5. one scan step from the stored state (updated in place)
-  {
-    ProfScope prof_scope(stream, "dec_scan");
-    ScanArgs a{};
-    a.u = u;
-    a.delta = delta;
-    a.z = z;
-    a.ld_z = E;
-    a.bc = xdbl;
-    a.ld_bc = xdbl_width(c);
-    a.bc_col = c.dt_rank;
-    a.a_log = layer->w.a_log;
-    a.d_skip = layer->w.d_skip;
-    a.y = yssm;
-    a.h_in = ssm_cache->h;
-    a.h_out = ssm_cache->h;
-    a.B = batch;
-    a.L = 1;
-    a.E = E;
+    a.R = c.dt_rank;
     a.N = c.d_state;
-    a.chunk_ws = nullptr;
-    if ((st = selective_scan(a, c.dtype, stream)) != HYMBA_OK) return st;
+    if ((st = decode_ssm(a, c.dtype, stream)) != HYMBA_OK) return st;
   }
   // 6. single-query attention over the store
   {

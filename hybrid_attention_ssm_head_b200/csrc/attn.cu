@@ -102,26 +102,40 @@ __device__ __forceinline__ void mask_cols(uint32_t (&v)[N], int col0, int hi1, i
     if (!keep) v[e] = __float_as_uint(-INFINITY);
   }
 }
-__device__ __forceinline__ float max32(const uint32_t (&v)[32]) {
+// Row max over the 128 scores of one row: eight chains of three-input maxima.
+__device__ __forceinline__ float row_max128(const uint32_t (&s0)[32], const uint32_t (&s1)[32],
+                                            const uint32_t (&s2)[32], const uint32_t (&s3)[32]) {
   float m[8];
 #pragma unroll
-  for (int t = 0; t < 8; ++t) m[t] = __uint_as_float(v[t]);
+  for (int t = 0; t < 8; ++t) m[t] = fmaxf(__uint_as_float(s0[t]), __uint_as_float(s0[t + 8]));
 #pragma unroll
-  for (int e = 8; e < 32; ++e) m[e & 7] = fmaxf(m[e & 7], __uint_as_float(v[e]));
-  return fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])), fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+  for (int t = 0; t < 8; ++t) m[t] = fmax3(m[t], __uint_as_float(s0[t + 16]), __uint_as_float(s0[t + 24]));
+#pragma unroll
+  for (int e = 0; e < 32; e += 16)
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      m[t] = fmax3(m[t], __uint_as_float(s1[e + t]), __uint_as_float(s1[e + t + 8]));
+      m[t] = fmax3(m[t], __uint_as_float(s2[e + t]), __uint_as_float(s2[e + t + 8]));
+      m[t] = fmax3(m[t], __uint_as_float(s3[e + t]), __uint_as_float(s3[e + t + 8]));
+    }
+  return fmaxf(fmax3(m[0], m[1], m[2]), fmax3(fmax3(m[3], m[4], m[5]), m[6], m[7]));
 }
-// P for 32 keys of a row: exp2(s * scale - m) packed to bf16 pairs; returns the fp32 sum.
-__device__ __forceinline__ float p_pack(const uint32_t (&v)[32], uint32_t (&pk)[16], float scale_log2,
-                                        float nm) {
-  float ls[4] = {0.f, 0.f, 0.f, 0.f};
+// P for 32 keys of a row: exp2(s * scale - m) packed to bf16 pairs; returns the fp32
+// sum as a pair of partial sums.  Scale and shift run as packed fp32x2 FMAs; one key
+// pair in four takes its exponentials from the degree-3 polynomial on the FMA pipe
+// (relative error 7.5e-5, well inside the bf16 rounding of P) and the others from
+// the MUFU, so that the two pipes share the exponentials.
+__device__ __forceinline__ float2 p_pack(const uint32_t (&v)[32], uint32_t (&pk)[16], float2 scale2,
+                                         float2 nm2) {
+  float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
-    const float p0 = ex2(fmaf(__uint_as_float(v[e]), scale_log2, nm));
-    const float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale_log2, nm));
-    ls[(e >> 1) & 3] += p0 + p1;
-    pk[e >> 1] = pack_bf16x2(p0, p1);
+    const float2 x = ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scale2, nm2);
+    const float2 p = ((e >> 1) & 3) == 0 ? exp2_poly2<3>(x) : make_float2(ex2(x.x), ex2(x.y));
+    ls[(e >> 1) & 1] = fadd2(ls[(e >> 1) & 1], p);
+    pk[e >> 1] = pack_bf16x2(p.x, p.y);
   }
-  return (ls[0] + ls[1]) + (ls[2] + ls[3]);
+  return fadd2(ls[0], ls[1]);
 }
 // Keys c*32 .. c*32+31 of row r into the 128-byte swizzled K-major P tile
 // (atom c/2, 16-byte chunks (c%2)*4 .. +3).
@@ -343,8 +357,7 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         mask_cols(s3, 96, hi1, lo2, hi2);
       }
       // row max (scale > 0, so the max commutes with the scaling)
-      float mx = fmaxf(fmaxf(max32(s0), max32(s1)), fmaxf(max32(s2), max32(s3)));
-      mx *= scale_log2;
+      const float mx = row_max128(s0, s1, s2, s3) * scale_log2;
       // lazy rescale decision
       float alpha = 1.f;
       bool resc = false;
@@ -359,9 +372,11 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
       // P = exp2(s * scale - m) into packed bf16 registers first, so that the wait for
       // the previous tile's P V (which still reads the P buffer) overlaps the exps
       const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+      const float2 nm2 = make_float2(nm, nm), scale2 = make_float2(scale_log2, scale_log2);
       uint32_t pk0[16], pk1[16], pk2[16], pk3[16];
-      l_run += (p_pack(s0, pk0, scale_log2, nm) + p_pack(s1, pk1, scale_log2, nm)) +
-               (p_pack(s2, pk2, scale_log2, nm) + p_pack(s3, pk3, scale_log2, nm));
+      const float2 ps = fadd2(fadd2(p_pack(s0, pk0, scale2, nm2), p_pack(s1, pk1, scale2, nm2)),
+                              fadd2(p_pack(s2, pk2, scale2, nm2), p_pack(s3, pk3, scale2, nm2)));
+      l_run += ps.x + ps.y;
       if (j > 0) {
         if (!mbar_wait(&o_done[q], uint32_t(j - 1) & 1u, &g_err_attn)) { ok = false; break; }
         tc_fence_after();
@@ -775,16 +790,21 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---- bf16 decode attention on the tensor cores (mma.sync m16n8k16) ---------------
-// CTA = 128 slots of one (sequence, kv head); the K and V chunks arrive by 3-D TMA
-// (128-byte swizzle, rows past the store's capacity read as zero); warp w takes keys
-// 32w..32w+31: S = Q K^T with the query heads of the group in rows 0..rep-1 of a
-// 16-row tile, softmax in registers, O += P V with V fragments from ldmatrix.trans.
-// The four warps' partial results are merged in shared memory.
+// CTA = a run of CPC consecutive 128-slot chunks of one (sequence, kv head).  The
+// chunks stream through two shared-memory stages by 3-D TMA (128-byte swizzle, rows
+// past the store's capacity read as zero), the next chunk's copy in flight while the
+// current one is computed.  Warp w takes keys 32w..32w+31 of every chunk: S = Q K^T
+// with the query heads of the group in rows 0..rep-1 of a 16-row tile, an online
+// softmax in registers (running max and sum per row, O rescaled when the max grows),
+// O += P V with V fragments from ldmatrix.trans.  At the end the four warps' states are
+// merged in shared memory into one partial (max, sum, O) per query head and run.
 namespace dtc {
 constexpr int SLOTS = 128;
 constexpr int K_BYTES = SLOTS * 128;        // 64 bf16 per slot
 constexpr int V_BYTES = SLOTS * 256;        // two 64-column boxes
-constexpr int SMEM = K_BYTES + V_BYTES + 4 * 8 * 130 * 4 + 64 + 1024;
+constexpr int STAGE = K_BYTES + V_BYTES;
+constexpr int SMEM = 2 * STAGE + 64 + 1024;  // the final merge reuses stage 0: two CTAs per SM
+constexpr int MAX_CPC = 4;                   // chunks per CTA
 }  // namespace dtc
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
@@ -816,32 +836,40 @@ __global__ void __launch_bounds__(128)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                           const __nv_bfloat16 *__restrict__ q, float *__restrict__ part, int H,
                           int Hkv, long long pos, int n_meta, int window, int is_global,
-                          float scale_log2, int nsplit) {
+                          float scale_log2, int nsplit, int cpc) {
   using namespace dtc;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t *sm = dsm_raw + ((1024 - (smem_u32(dsm_raw) & 1023)) & 1023);
-  float *om = reinterpret_cast<float *>(sm + K_BYTES + V_BYTES);  // [4 warps][8 rows][130]
-  uint64_t *bar = reinterpret_cast<uint64_t *>(om + 4 * 8 * 130);
+  float *om = reinterpret_cast<float *>(sm);  // [4 warps][8 rows][130], after the last chunk
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + 2 * STAGE);  // [2]
   const int split = blockIdx.y, bg = blockIdx.x;
   const int b = bg / Hkv, g = bg % Hkv;
   const int rep = H / Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = lane >> 2, gc = lane & 3;  // mma group row / column pair
-  const long long s0 = (long long)split * SLOTS;
   const long long nslots = dec_slots(pos, n_meta, window, is_global);
-  const int ns = (int)min((long long)SLOTS, nslots - s0);
+  const long long nchunks = (nslots + SLOTS - 1) / SLOTS;
+  const int c0 = split * cpc;
+  const int nch = (int)max(0LL, min((long long)cpc, nchunks - c0));
+  auto issue = [&](int i) {  // chunk c0 + i into stage i & 1
+    uint8_t *dst = sm + (i & 1) * STAGE;
+    const int s0 = (c0 + i) * SLOTS;
+    mbar_arrive_expect_tx(&full[i & 1], STAGE);
+    tma_load_3d(dst, &tmK, &full[i & 1], 0, s0, bg);
+    tma_load_3d(dst + K_BYTES, &tmV, &full[i & 1], 0, s0, bg);
+    tma_load_3d(dst + K_BYTES + V_BYTES / 2, &tmV, &full[i & 1], 64, s0, bg);
+  };
   if (tid == 0) {
-    mbar_init(bar, 1);
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
   }
   __syncthreads();
+  int issued = 0;
   if (tid == 0) {
-    mbar_arrive_expect_tx(bar, K_BYTES + V_BYTES);
-    tma_load_3d(sm, &tmK, bar, 0, (int)s0, bg);
-    tma_load_3d(sm + K_BYTES, &tmV, bar, 0, (int)s0, bg);
-    tma_load_3d(sm + K_BYTES + V_BYTES / 2, &tmV, bar, 64, (int)s0, bg);
+    for (; issued < min(2, nch); ++issued) issue(issued);
   }
   // Q fragments (row = query head of the group, zero beyond rep), from global memory
   uint32_t qa[4][2];  // [k-step][a0a1 / a4a5]; rows 8..15 are zero
@@ -854,78 +882,107 @@ __global__ void __launch_bounds__(128)
       qa[ks][1] = live ? __ldg(qr + ks * 8 + 4 + gc) : 0u;
     }
   }
-  bool ok = mbar_wait(bar, 0, &g_err_attn);
-  if (!ok && tid == 0) mbar_wait_drain(bar, 0, &g_err_attn);
-  const uint32_t kb = smem_u32(sm), vb = smem_u32(sm + K_BYTES);
-  // ---- S = Q K^T for this warp's 32 keys (4 n-tiles of 8 keys) ----
-  float sacc[4][4];
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
-    const int key = warp * 32 + nt * 8 + (lane & 7);
-#pragma unroll
-    for (int kp = 0; kp < 2; ++kp) {  // two k-steps per ldmatrix.x4
-      const int ch = kp * 4 + (lane >> 3);  // 16-byte chunk of the key row (8 dims)
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(kb + sw128(key, ch), b0, b1, b2, b3);
-      mma16816(sacc[nt], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b0, b1);
-      mma16816(sacc[nt], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b2, b3);
-    }
-  }
-  // ---- softmax over the warp's keys, row gr (values sacc[nt][0..1], keys 8nt + 2gc + {0,1}) ----
-  float mx = -INFINITY;
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int key = warp * 32 + nt * 8 + 2 * gc + e;
-      const bool valid = ok && key < ns && dec_slot_valid(s0 + key, pos, n_meta, window, is_global);
-      const float x = valid ? sacc[nt][e] * scale_log2 : -INFINITY;
-      sacc[nt][e] = x;
-      mx = fmaxf(mx, x);
-    }
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-  mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-  const float mref = mx == -INFINITY ? 0.f : mx;
-  float lsum = 0.f;
-  uint32_t pa[4];  // P as A fragments: [k-step kk][a0a1 (n-tile 2kk) / a4a5 (n-tile 2kk+1)]
-#pragma unroll
-  for (int nt = 0; nt < 4; ++nt) {
-    const float p0 = ex2(sacc[nt][0] - mref), p1 = ex2(sacc[nt][1] - mref);
-    lsum += p0 + p1;
-    pa[nt] = pack_bf16x2(p0, p1);
-  }
-  lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
-  lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
-  // ---- O = P V (16 n-tiles of 8 value columns, 2 k-steps of 16 keys) ----
+  float m_run = -INFINITY, l_run = 0.f;  // row gr of this warp
   float oacc[16][4];
 #pragma unroll
   for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
     for (int e = 0; e < 4; ++e) oacc[nt][e] = 0.f;
+  bool ok = true;
+  int i = 0;
+  for (; i < nch; ++i) {
+    const int st = i & 1;
+    ok = mbar_wait(&full[st], uint32_t(i >> 1) & 1u, &g_err_attn);
+    if (__syncthreads_or(!ok)) { ok = false; break; }
+    const uint32_t kb = smem_u32(sm + st * STAGE), vb = kb + K_BYTES;
+    const long long s0 = (long long)(c0 + i) * SLOTS;
+    const int ns = (int)min((long long)SLOTS, nslots - s0);
+    // ---- S = Q K^T for this warp's 32 keys (4 n-tiles of 8 keys) ----
+    float sacc[4][4];
 #pragma unroll
-  for (int kk = 0; kk < 2; ++kk) {
-    const int key = warp * 32 + kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-    for (int np = 0; np < 8; ++np) {  // pairs of n-tiles per ldmatrix.x4.trans
-      const int chg = np * 2 + (lane >> 4);  // 16-byte chunk of value columns (0..15)
-      const uint32_t addr = vb + (chg >> 3) * (V_BYTES / 2) + sw128(key, chg & 7);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4_t(addr, b0, b1, b2, b3);
-      mma16816(oacc[2 * np], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b0, b1);
-      mma16816(oacc[2 * np + 1], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b2, b3);
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int key = warp * 32 + nt * 8 + (lane & 7);
+#pragma unroll
+      for (int kp = 0; kp < 2; ++kp) {  // two k-steps per ldmatrix.x4
+        const int ch = kp * 4 + (lane >> 3);  // 16-byte chunk of the key row (8 dims)
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + sw128(key, ch), b0, b1, b2, b3);
+        mma16816(sacc[nt], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b0, b1);
+        mma16816(sacc[nt], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b2, b3);
+      }
     }
+    // ---- online softmax, row gr (values sacc[nt][0..1], keys 8nt + 2gc + {0,1}) ----
+    float mx = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int key = warp * 32 + nt * 8 + 2 * gc + e;
+        const bool valid = key < ns && dec_slot_valid(s0 + key, pos, n_meta, window, is_global);
+        const float x = valid ? sacc[nt][e] * scale_log2 : -INFINITY;
+        sacc[nt][e] = x;
+        mx = fmaxf(mx, x);
+      }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    const float mref = m_new == -INFINITY ? 0.f : m_new;
+    const float alpha = m_run == -INFINITY ? 0.f : ex2(m_run - mref);
+    m_run = m_new;
+    float lsum = 0.f;
+    uint32_t pa[4];  // P as A fragments: [k-step kk][a0a1 (n-tile 2kk) / a4a5 (n-tile 2kk+1)]
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const float p0 = ex2(sacc[nt][0] - mref), p1 = ex2(sacc[nt][1] - mref);
+      lsum += p0 + p1;
+      pa[nt] = pack_bf16x2(p0, p1);
+    }
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+    lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+    l_run = fmaf(l_run, alpha, lsum);
+    if (i > 0) {
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt) {
+        oacc[nt][0] *= alpha;
+        oacc[nt][1] *= alpha;
+      }
+    }
+    // ---- O += P V (16 n-tiles of 8 value columns, 2 k-steps of 16 keys) ----
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      const int key = warp * 32 + kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int np = 0; np < 8; ++np) {  // pairs of n-tiles per ldmatrix.x4.trans
+        const int chg = np * 2 + (lane >> 4);  // 16-byte chunk of value columns (0..15)
+        const uint32_t addr = vb + (chg >> 3) * (V_BYTES / 2) + sw128(key, chg & 7);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(addr, b0, b1, b2, b3);
+        mma16816(oacc[2 * np], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b0, b1);
+        mma16816(oacc[2 * np + 1], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b2, b3);
+      }
+    }
+    __syncthreads();  // every warp is done with stage st
+    if (tid == 0 && issued < nch) issue(issued++);
   }
-  // ---- merge the four warps: rows 0..rep-1 ----
+  if (!ok) {
+    // copies issued past the failed wait must land before the CTA leaves
+    if (tid == 0)
+      for (int k = i; k < issued; ++k) mbar_wait_drain(&full[k & 1], uint32_t(k >> 1) & 1u, &g_err_attn);
+    m_run = -INFINITY;
+    l_run = 0.f;
+  }
+  // ---- merge the four warps: rows 0..rep-1 (stage 0 is free: every copy has landed) ----
+  __syncthreads();
   float *mw = om;  // per warp: [8 rows][130] = m, l, o[128]
   if (gr < 8) {
     float *row = mw + (warp * 8 + gr) * 130;
     if (gc == 0) {
-      row[0] = mx;
-      row[1] = lsum;
+      row[0] = m_run;
+      row[1] = l_run;
     }
 #pragma unroll
     for (int nt = 0; nt < 16; ++nt) {
@@ -1017,11 +1074,15 @@ hymba_status attention_decode(const DecodeAttnArgs &a, hymba_dtype dt, cudaStrea
     const uint32_t box[3] = {64, (uint32_t)dtc::SLOTS, 1};
     if (!make_tmap(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dk, sk, box)) return HYMBA_ERR_CUDA;
     if (!make_tmap(&tv, a.v_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dvv, svv, box)) return HYMBA_ERR_CUDA;
-    const int ns_tc = (int)((nslots + dtc::SLOTS - 1) / dtc::SLOTS);
+    // runs of up to MAX_CPC chunks, as even as the chunk count allows
+    const int nchunks = (int)((nslots + dtc::SLOTS - 1) / dtc::SLOTS);
+    const int runs = (nchunks + dtc::MAX_CPC - 1) / dtc::MAX_CPC;
+    const int cpc = (nchunks + runs - 1) / runs;
+    const int ns_tc = (nchunks + cpc - 1) / cpc;
     dim3 grid_tc(a.B * a.Hkv, ns_tc);
     attn_decode_tc_kernel<<<grid_tc, 128, dtc::SMEM, s>>>(tk, tv, (const __nv_bfloat16 *)a.q, a.partial,
                                                          a.H, a.Hkv, a.pos, a.n_meta, a.window,
-                                                         a.is_global, sl2, ns_tc);
+                                                         a.is_global, sl2, ns_tc, cpc);
     attn_decode_combine_kernel<__nv_bfloat16><<<a.B * a.H, 128, 0, s>>>(
         a.partial, (__nv_bfloat16 *)a.o, a.H, a.dv, ns_tc);
   } else if (dt == HYMBA_BF16) {

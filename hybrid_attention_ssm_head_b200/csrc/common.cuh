@@ -38,8 +38,27 @@ template <> struct Store<__nv_bfloat16> {
   static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
 };
 
-// x * sigmoid(x) with the fast exp and division (about 2 ulp; 0 for x -> -inf).
-__device__ __forceinline__ float silu_f(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
+// The MUFU approximations with subnormal inputs and results flushed to zero: one
+// instruction each (the non-flushing forms add range fix-ups around the MUFU).
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float lg2_ftz(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp_ftz(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+// x * sigmoid(x) = x / (1 + 2^(-x log2 e)); 0 for x -> -inf (the reciprocal of +inf).
+__device__ __forceinline__ float silu_f(float x) { return x * rcp_ftz(1.0f + ex2_ftz(-kLog2e * x)); }
 // bf16 -> fp32 is a 16-bit shift of the bits (exact): an integer-pipe operation.
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -59,12 +78,63 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
       : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
   return *reinterpret_cast<float2 *>(&d);
 }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&d);
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t *>(&a)), "l"(*reinterpret_cast<uint64_t *>(&b)));
+  return *reinterpret_cast<float2 *>(&d);
+}
+// max of three in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// 2^x on the FMA pipe, two lanes per instruction (Cody-Waite style reduction):
+// j = rint(x) through the 1.5 * 2^23 rounding constant, f = x - j in [-1/2, 1/2],
+// 2^f by a polynomial of degree DEG, j added into the exponent field.  The
+// coefficients are relative-error minimax fits of 2^f on [-1/2, 1/2] made for this
+// library (fp32 Horner evaluation: max relative error 7.5e-5 at degree 3, 2.4e-7 at
+// degree 5, the size of the MUFU's own error).  x is clamped below at -125 so the
+// exponent stays in range (the result is then 2^-125 instead of smaller); no upper
+// clamp, valid for x < 128.
+template <int DEG>
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  static_assert(DEG == 3 || DEG == 5, "fitted degrees");
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 rnd = make_float2(12582912.f, 12582912.f);
+  const float2 t = fadd2(x, rnd);
+  const float2 f = fsub2(x, fsub2(t, rnd));
+  float2 p;
+  if constexpr (DEG == 5) {
+    p = ffma2(make_float2(1.3276470e-3f, 1.3276470e-3f), f, make_float2(9.6755419e-3f, 9.6755419e-3f));
+    p = ffma2(p, f, make_float2(5.5507135e-2f, 5.5507135e-2f));
+    p = ffma2(p, f, make_float2(2.4022120e-1f, 2.4022120e-1f));
+    p = ffma2(p, f, make_float2(6.9314694e-1f, 6.9314694e-1f));
+    p = ffma2(p, f, make_float2(1.0000001f, 1.0000001f));
+  } else {
+    p = ffma2(make_float2(5.5171657e-2f, 5.5171657e-2f), f, make_float2(2.4261114e-1f, 2.4261114e-1f));
+    p = ffma2(p, f, make_float2(6.9326097e-1f, 6.9326097e-1f));
+    p = ffma2(p, f, make_float2(9.9992806e-1f, 9.9992806e-1f));
+  }
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
 // log(1 + e^x) with the fast exp/log: x above 20 returns x; below -8 returns e^x
 // (relative error e^x / 2 < 2e-4); in between log(1 + e^x) with 1 + e^x >= 1 + 3e-4,
 // so the fp32 rounding of the sum costs at most ~2e-4 relative.
 __device__ __forceinline__ float softplus_f(float x) {
-  const float e = __expf(fminf(x, 20.0f));
-  const float l = __logf(1.0f + e);
+  const float e = ex2_ftz(kLog2e * fminf(x, 20.0f));
+  const float l = kLn2 * lg2_ftz(1.0f + e);
   return x > 20.0f ? x : (x < -8.0f ? e : l);  // selects, no divergence
 }
 // Full-precision variant for the fp32 storage path.

@@ -123,15 +123,25 @@ size_t decode_attn_workspace_floats(int B, int H, int dv, long long pos, int n_m
                                     int is_global);
 hymba_status attention_decode(const DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s);
 
-struct DecodeConvArgs {
+
+// ---- decode SSM branch: conv + x_proj, then dt_proj + softplus + scan step + gate ----
+struct DecodeSsmArgs {
   const void *x;       // [B, E] x_ssm of the new token, row stride ld_x
   long long ld_x;
+  const void *z;       // [B, E] gate input, row stride ld_z
+  long long ld_z;
   void *conv_state;    // [B, K-1, E] in/out
-  void *u;             // [B, E]
-  const float *w, *bias;
-  int B, E, K;
+  const float *conv_w, *conv_b;  // [E, K], [E]
+  const void *w_x;     // [R + 2N, E]
+  float *xdbl;         // [B, R + 2N] fp32, zeroed before the first kernel
+  void *u;             // [B, E] conv + SiLU output
+  const float *w_dt, *b_dt;      // [E, R], [E]
+  const float *a_log, *d_skip;   // [E, N], [E]
+  float *h;            // [B, E, N] fp32 state, updated in place
+  void *y;             // [B, E] gated output
+  int B, E, K, R, N;
 };
-hymba_status decode_conv(const DecodeConvArgs &a, hymba_dtype dt, cudaStream_t s);
+hymba_status decode_ssm(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s);
 
 hymba_status mask_bitmap(int L, int n_meta, int window, int is_global, uint32_t *bits,
                          uint8_t *tile_class, cudaStream_t s);
