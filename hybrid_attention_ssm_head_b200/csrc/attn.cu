@@ -41,23 +41,24 @@ __device__ __forceinline__ float ex2(float x) {
 namespace fa {
 constexpr int QT = 128;          // query rows per tile
 constexpr int KT = 128;          // keys per tile
-constexpr int NQ = 2;            // query tiles per CTA
+constexpr int NQ = 2;            // query tiles per work item
 constexpr int Q_BYTES = QT * 128;        // 64 bf16 per row
 constexpr int K_BYTES = KT * 128;
 constexpr int V_BYTES = KT * 256;        // two 64-column boxes
 constexpr int P_BYTES = QT * 256;        // two 64-key swizzle atoms
-constexpr int OFF_Q = 0;
-constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
+constexpr int OFF_Q = 0;                 // two buffers (this item's and the next one's)
+constexpr int OFF_K = OFF_Q + 2 * NQ * Q_BYTES;
 constexpr int OFF_V = OFF_K + 2 * K_BYTES;
 constexpr int OFF_P = OFF_V + 2 * V_BYTES;
 constexpr int OFF_BAR = OFF_P + NQ * P_BYTES;
-constexpr int NBAR = 1 + 2 + 2 + 2 + 2 + NQ * 4 + 1;
+constexpr int NBAR = 2 * 10 + 1 + 2 * NQ;
 constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
+static_assert(SMEM <= 232448, "attention shared memory");
 constexpr int THREADS = 128 + NQ * 128;  // warpgroup 0: TMA + MMA; one softmax warpgroup per query tile
-// Register split (setmaxnreg): launch 168 per thread = 64,512; warpgroup 0 drops to 56,
-// the softmax warpgroups rise to 224: 128 * 56 + 256 * 224 = 64,512.
-constexpr int REG_CTRL = 56;
-constexpr int REG_SOFTMAX = 224;
+// Register split (setmaxnreg): launch 168 per thread = 64,512; warpgroup 0 drops to 72,
+// the softmax warpgroups rise to 216: 128 * 72 + 256 * 216 = 64,512.
+constexpr int REG_CTRL = 72;
+constexpr int REG_SOFTMAX = 216;
 constexpr uint32_t IDESC_S = make_idesc(128, 1, 0, 0);
 constexpr uint32_t IDESC_PV = make_idesc(128, 1, 0, 1);
 }  // namespace fa
@@ -93,14 +94,32 @@ __device__ __forceinline__ FaTiles fa_tiles(int qa, int L, int n_meta, int windo
   return t;
 }
 
-template <int N>
-__device__ __forceinline__ void mask_cols(uint32_t (&v)[N], int col0, int hi1, int lo2, int hi2) {
+// Work item of the persistent kernel: (sequence, head, query-tile pair).  Pairs run
+// from the last (the most key tiles in a causal layer) to the first, heads fastest so
+// that the heads of one kv group run side by side and share K/V tiles through L2.
+struct FaItem {
+  int b, h, qa;  // qa: first query tile of the pair
+};
+__device__ __forceinline__ FaItem fa_item(long long it, int H, int BH, int npairs) {
+  const int pair = npairs - 1 - (int)(it / BH);
+  const int rest = (int)(it % BH);
+  return {rest / H, rest % H, 2 * pair};
+}
+__device__ __forceinline__ int fa_count(const FaTiles &t) {
+  int n = 0;
+  for (int kt = t.first(); kt <= t.hi; kt = t.next(kt)) ++n;
+  return n;
+}
+
+// Keep-mask of the 32 columns col0..col0+31 for the column ranges [0, hi1) and [lo2, hi2).
+__device__ __forceinline__ uint32_t low_bits(int n) {
+  return n <= 0 ? 0u : (n >= 32 ? 0xffffffffu : (1u << n) - 1u);
+}
+__device__ __forceinline__ void mask_cols(uint32_t (&v)[32], int col0, int hi1, int lo2, int hi2) {
+  const uint32_t keep = low_bits(hi1 - col0) | (low_bits(hi2 - col0) & ~low_bits(lo2 - col0));
 #pragma unroll
-  for (int e = 0; e < N; ++e) {
-    const int cc = col0 + e;
-    const bool keep = (cc < hi1) | ((cc >= lo2) & (cc < hi2));
-    if (!keep) v[e] = __float_as_uint(-INFINITY);
-  }
+  for (int e = 0; e < 32; ++e)
+    if (!(keep & (1u << e))) v[e] = __float_as_uint(-INFINITY);
 }
 // Row max over the 128 scores of one row: eight chains of three-input maxima.
 __device__ __forceinline__ float row_max128(const uint32_t (&s0)[32], const uint32_t (&s1)[32],
@@ -149,43 +168,41 @@ __device__ __forceinline__ void p_store(const uint32_t (&pk)[16], int c, int r, 
   }
 }
 
+// Persistent: one CTA per SM walks the work items blockIdx.x, + gridDim.x, ...; the
+// K/V ring and every per-tile barrier count tiles across item boundaries, so the next
+// item's Q and first K/V tiles stream in, and its first S = Q K^T is issued, while the
+// current item's last tile is still in the softmax; the softmax warpgroups write the
+// finished item's O between its last tile and the next item's first.
 __global__ void __launch_bounds__(fa::THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                       const __grid_constant__ CUtensorMap tmV, __nv_bfloat16 *__restrict__ out,
-                       int L, int H, int Hkv, int n_meta, int window, int is_global, float scale_log2,
-                       int npairs) {
+                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                       int L, int B, int H, int Hkv, int n_meta, int window, int is_global,
+                       float scale_log2, int npairs) {
   using namespace fa;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
-  uint64_t *q_full = bars + 0;
-  uint64_t *k_full = bars + 1, *k_empty = bars + 3;
-  uint64_t *v_full = bars + 5, *v_empty = bars + 7;
-  uint64_t *s_full = bars + 9;            // [NQ]
-  uint64_t *p_full = bars + 9 + NQ;       // [NQ]
-  uint64_t *o_done = bars + 9 + 2 * NQ;   // [NQ]
-  uint64_t *drain = bars + 9 + 3 * NQ;
-  uint64_t *s_free = bars + 10 + 3 * NQ;  // [NQ]: S of the tile is in registers
+  uint64_t *q_full = bars + 0, *q_empty = bars + 2;    // [2]: Q buffers
+  uint64_t *k_full = bars + 4, *k_empty = bars + 6;    // [2]: K stages
+  uint64_t *v_full = bars + 8, *v_empty = bars + 10;   // [2]: V stages
+  uint64_t *s_full = bars + 12, *p_full = bars + 14;   // [NQ]
+  uint64_t *o_done = bars + 16, *s_free = bars + 18;   // [NQ]: PV retired / S in registers
+  uint64_t *drain = bars + 20;
+  uint64_t *o_staged = bars + 21, *o_stored = bars + 23;  // [NQ]: O rows in the P buffer / stored
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBAR);
 
   const int warp = warp_id(), lane = lane_id();
-  // block -> (head fastest, then query-tile pair, then batch): the heads of one
-  // kv group run together and share K/V tiles through L2.
-  const int h = blockIdx.x % H;
-  const int rest = blockIdx.x / H;
-  const int pair = rest % npairs;
-  const int b = rest / npairs;
-  const int g = h / (H / Hkv);
-  const int qa = 2 * pair;
+  const int BH = B * H;
+  const long long n_items = (long long)BH * npairs;
 
   if (warp == 0 && lane == 0) {
-    mbar_init(q_full, 1);
-    mbar_init(drain, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&q_full[x], 1);
+      mbar_init(&q_empty[x], 1);
+      mbar_init(&k_full[x], 1);
+      mbar_init(&k_empty[x], 1);
+      mbar_init(&v_full[x], 1);
+      mbar_init(&v_empty[x], 1);
     }
     for (int q = 0; q < NQ; ++q) {
       mbar_init(&s_full[q], 1);
@@ -193,10 +210,16 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
       mbar_init(&o_done[q], 1);
       mbar_init(&s_free[q], 4);
     }
+    mbar_init(drain, 1);
+    for (int q = 0; q < NQ; ++q) {
+      mbar_init(&o_staged[q], 128);
+      mbar_init(&o_stored[q], 1);
+    }
     fence_barrier_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -208,52 +231,54 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S of tile q at 256q, O of tile q at 256q + 128.
 
-
-  // Streamed key tiles (same sequence in every role).
-  const FaTiles tiles = fa_tiles(qa, L, n_meta, window, is_global);
-  int nstream = 0;
-  for (int kt = tiles.first(); kt <= tiles.hi; kt = tiles.next(kt)) ++nstream;
-
   if (warp < 4) {
    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_CTRL));
    if (warp == 0) {
     if (lane == 0) {
+      // ---------------- TMA producer ----------------
       bool ok = true;
-      uint32_t k_issued0 = 0, k_issued1 = 0, v_issued0 = 0, v_issued1 = 0;
-      mbar_arrive_expect_tx(q_full, NQ * Q_BYTES);
-      for (int q = 0; q < NQ; ++q)
-        tma_load_3d(smem + OFF_Q + q * Q_BYTES, &tmQ, q_full, h * 64, (qa + q) * QT, b);
-      int j = 0;
-      for (int kt = tiles.first(); kt <= tiles.hi && ok; kt = tiles.next(kt)) {
-        const int st = j & 1;
-        const uint32_t ph = (uint32_t(j) >> 1) & 1u;
-        if (!mbar_wait(&k_empty[st], ph ^ 1u, &g_err_attn)) { ok = false; break; }
-        mbar_arrive_expect_tx(&k_full[st], K_BYTES);
-        tma_load_3d(smem + OFF_K + st * K_BYTES, &tmK, &k_full[st], g * 64, kt * KT, b);
-        if (st) ++k_issued1; else ++k_issued0;
-        if (!mbar_wait(&v_empty[st], ph ^ 1u, &g_err_attn)) { ok = false; break; }
-        mbar_arrive_expect_tx(&v_full[st], V_BYTES);
-        uint8_t *vdst = smem + OFF_V + st * V_BYTES;
-        tma_load_3d(vdst, &tmV, &v_full[st], g * 128, kt * KT, b);
-        tma_load_3d(vdst + V_BYTES / 2, &tmV, &v_full[st], g * 128 + 64, kt * KT, b);
-        if (st) ++v_issued1; else ++v_issued0;
-        ++j;
+      long long g = 0;  // tiles issued so far (all items)
+      uint32_t nq[2] = {0, 0}, nk[2] = {0, 0}, nv[2] = {0, 0};
+      int itk = 0;
+      for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++itk) {
+        const FaItem w = fa_item(it, H, BH, npairs);
+        const int gkv = w.h / (H / Hkv);
+        const int qb = itk & 1;
+        if (!mbar_wait(&q_empty[qb], ((uint32_t(itk) >> 1) & 1u) ^ 1u, &g_err_attn)) { ok = false; break; }
+        mbar_arrive_expect_tx(&q_full[qb], NQ * Q_BYTES);
+        for (int q = 0; q < NQ; ++q)
+          tma_load_3d(smem + OFF_Q + (qb * NQ + q) * Q_BYTES, &tmQ, &q_full[qb], w.h * 64, (w.qa + q) * QT, w.b);
+        ++nq[qb];
+        const FaTiles t = fa_tiles(w.qa, L, n_meta, window, is_global);
+        for (int kt = t.first(); kt <= t.hi; kt = t.next(kt), ++g) {
+          const int st = int(g & 1);
+          const uint32_t ph = uint32_t(g >> 1) & 1u;
+          if (!mbar_wait(&k_empty[st], ph ^ 1u, &g_err_attn)) { ok = false; break; }
+          mbar_arrive_expect_tx(&k_full[st], K_BYTES);
+          tma_load_3d(smem + OFF_K + st * K_BYTES, &tmK, &k_full[st], gkv * 64, kt * KT, w.b);
+          ++nk[st];
+          if (!mbar_wait(&v_empty[st], ph ^ 1u, &g_err_attn)) { ok = false; break; }
+          mbar_arrive_expect_tx(&v_full[st], V_BYTES);
+          uint8_t *vdst = smem + OFF_V + st * V_BYTES;
+          tma_load_3d(vdst, &tmV, &v_full[st], gkv * 128, kt * KT, w.b);
+          tma_load_3d(vdst + V_BYTES / 2, &tmV, &v_full[st], gkv * 128 + 64, kt * KT, w.b);
+          ++nv[st];
+        }
       }
       if (!ok) {
-        mbar_wait_drain(q_full, 0, &g_err_attn);
-        if (k_issued0) mbar_wait_drain(&k_full[0], (k_issued0 - 1) & 1u, &g_err_attn);
-        if (k_issued1) mbar_wait_drain(&k_full[1], (k_issued1 - 1) & 1u, &g_err_attn);
-        if (v_issued0) mbar_wait_drain(&v_full[0], (v_issued0 - 1) & 1u, &g_err_attn);
-        if (v_issued1) mbar_wait_drain(&v_full[1], (v_issued1 - 1) & 1u, &g_err_attn);
+        for (int x = 0; x < 2; ++x) {
+          if (nq[x]) mbar_wait_drain(&q_full[x], (nq[x] - 1) & 1u, &g_err_attn);
+          if (nk[x]) mbar_wait_drain(&k_full[x], (nk[x] - 1) & 1u, &g_err_attn);
+          if (nv[x]) mbar_wait_drain(&v_full[x], (nv[x] - 1) & 1u, &g_err_attn);
+        }
       }
     }
-  } else if (warp == 1) {
-    if (lane == 0 && nstream > 0) {
-      bool ok = mbar_wait(q_full, 0, &g_err_attn);
-      const uint32_t q_addr0 = smem_u32(smem + OFF_Q);
+   } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer: one flat walk over the tiles of all items ----------------
       const uint32_t p_addr0 = smem_u32(smem + OFF_P);
-      auto issue_S = [&](int q, int st) {
-        const uint32_t qa_ = q_addr0 + q * Q_BYTES;
+      auto issue_S = [&](int q, int st, int qb) {
+        const uint32_t qa_ = smem_u32(smem + OFF_Q) + (qb * NQ + q) * Q_BYTES;
         const uint32_t ka = smem_u32(smem + OFF_K + st * K_BYTES);
 #pragma unroll
         for (int k = 0; k < 4; ++k)
@@ -272,38 +297,69 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         }
         mma_commit(&o_done[q]);
       };
-      if (ok) ok = mbar_wait(&k_full[0], 0, &g_err_attn);
-      if (ok) {
-        tc_fence_after();
-        for (int q = 0; q < NQ; ++q) issue_S(q, 0);
-        mma_commit(&k_empty[0]);
-      }
-      // Per key tile j: S(j+1) of both query tiles as soon as their softmax holds S(j)
-      // in registers, then PV(j) as soon as P(j) is in shared memory.  S(j+1) thus
-      // overlaps the exponentials of tile j.
-      for (int j = 0; j < nstream && ok; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (uint32_t(j) >> 1) & 1u;
-        if (j + 1 < nstream) {
-          const int st1 = (j + 1) & 1;
-          const uint32_t ph1 = (uint32_t(j + 1) >> 1) & 1u;
-          if (!mbar_wait(&k_full[st1], ph1, &g_err_attn)) { ok = false; break; }
+      bool ok = true;
+      long long it = blockIdx.x;
+      int itk = 0;
+      if (it < n_items) {
+        FaItem w = fa_item(it, H, BH, npairs);
+        int n = fa_count(fa_tiles(w.qa, L, n_meta, window, is_global));
+        // S of the first tile
+        ok = mbar_wait(&q_full[0], 0, &g_err_attn) && mbar_wait(&k_full[0], 0, &g_err_attn);
+        if (ok) {
+          tc_fence_after();
+          for (int q = 0; q < NQ; ++q) issue_S(q, 0, 0);
+          mma_commit(&k_empty[0]);
+          if (n == 1) mma_commit(&q_empty[0]);
+        }
+        long long g = 0;  // current tile (all items)
+        int j = 0;        // its index within the item
+        while (ok) {
+          // the next tile: the same item's, or the first of the next item
+          const bool same = j + 1 < n;
+          const long long it_next = same ? it : it + gridDim.x;
+          const bool has_next = it_next < n_items;
+          int n_next = n;
+          if (has_next) {
+            const int qb_next = same ? (itk & 1) : ((itk + 1) & 1);
+            if (!same) {
+              const FaItem wn = fa_item(it_next, H, BH, npairs);
+              n_next = fa_count(fa_tiles(wn.qa, L, n_meta, window, is_global));
+              if (!mbar_wait(&q_full[qb_next], (uint32_t(itk + 1) >> 1) & 1u, &g_err_attn)) { ok = false; break; }
+            }
+            const long long g1 = g + 1;
+            const int st1 = int(g1 & 1);
+            if (!mbar_wait(&k_full[st1], uint32_t(g1 >> 1) & 1u, &g_err_attn)) { ok = false; break; }
+            for (int q = 0; q < NQ && ok; ++q) {
+              if (!mbar_wait(&s_free[q], uint32_t(g) & 1u, &g_err_attn)) { ok = false; break; }
+              tc_fence_after();
+              issue_S(q, st1, qb_next);
+            }
+            if (!ok) break;
+            mma_commit(&k_empty[st1]);
+            // the last S of an item releases its Q buffer once it has run
+            if ((same ? j + 1 : 0) == (same ? n : n_next) - 1) mma_commit(&q_empty[qb_next]);
+          }
+          // P V of the current tile
+          const int st = int(g & 1);
+          if (!mbar_wait(&v_full[st], uint32_t(g >> 1) & 1u, &g_err_attn)) { ok = false; break; }
           for (int q = 0; q < NQ && ok; ++q) {
-            if (!mbar_wait(&s_free[q], uint32_t(j) & 1u, &g_err_attn)) { ok = false; break; }
+            if (!mbar_wait(&p_full[q], uint32_t(g) & 1u, &g_err_attn)) { ok = false; break; }
             tc_fence_after();
-            issue_S(q, st1);
+            issue_PV(q, st, j > 0);
           }
           if (!ok) break;
-          mma_commit(&k_empty[st1]);
+          mma_commit(&v_empty[st]);
+          if (!has_next) break;
+          ++g;
+          if (same) {
+            ++j;
+          } else {
+            it = it_next;
+            ++itk;
+            n = n_next;
+            j = 0;
+          }
         }
-        if (!mbar_wait(&v_full[st], ph, &g_err_attn)) { ok = false; break; }
-        for (int q = 0; q < NQ && ok; ++q) {
-          if (!mbar_wait(&p_full[q], uint32_t(j) & 1u, &g_err_attn)) { ok = false; break; }
-          tc_fence_after();
-          issue_PV(q, st, j > 0);
-        }
-        if (!ok) break;
-        mma_commit(&v_empty[st]);
       }
       if (!ok) {
         // Drain issued MMAs before tensor memory is released.
@@ -318,114 +374,156 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
     const int q = (warp - 4) >> 2;        // query tile of this warpgroup
     const int quarter = warp & 3;         // TMEM lane quarter
     const int r = quarter * 32 + lane;    // row within the tile
-    const long long i = (long long)(qa + q) * QT + r;  // query position
     const uint32_t lane_off = uint32_t(quarter * 32) << 16;
     const uint32_t tS = tmem + 256 * q + lane_off;
     const uint32_t tO = tS + 128;
     const uint32_t p_base = smem_u32(smem + OFF_P + q * P_BYTES);
-    const int qtile = qa + q;
-    // Visible keys of row i: [0, meta_end) and [win_lo, i] (positions).
-    const long long meta_end = is_global ? 0 : min((long long)n_meta, i + 1);
-    const long long win_lo = is_global ? 0 : max((long long)n_meta, i - window + 1);
-    float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    int j = 0;
-    for (int kt = tiles.first(); kt <= tiles.hi && ok; kt = tiles.next(kt)) {
-      const int cls = fa_tile_class(qtile, kt, L, n_meta, window, is_global);  // uniform
-      if (!mbar_wait(&s_full[q], uint32_t(j) & 1u, &g_err_attn)) { ok = false; break; }
-      tc_fence_after();
-      // the whole S row in registers: four loads, one wait
-      uint32_t s0[32], s1[32], s2[32], s3[32];
-      tmem_ld32(tS, s0);
-      tmem_ld32(tS + 32, s1);
-      tmem_ld32(tS + 64, s2);
-      tmem_ld32(tS + 96, s3);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[q]);  // the MMA warp may overwrite S now
-      if (cls != 1) {
-        // partial tile: keep the column ranges [0, hi1) and [lo2, hi2); skipped tile: none
-        const long long key0 = (long long)kt * KT;
-        int hi1 = (int)max(0LL, min(128LL, meta_end - key0));
-        int lo2 = (int)max(0LL, min(128LL, win_lo - key0));
-        int hi2 = (int)max(0LL, min(128LL, i + 1 - key0));
-        if (cls == 0) hi1 = hi2 = 0;
-        mask_cols(s0, 0, hi1, lo2, hi2);
-        mask_cols(s1, 32, hi1, lo2, hi2);
-        mask_cols(s2, 64, hi1, lo2, hi2);
-        mask_cols(s3, 96, hi1, lo2, hi2);
-      }
-      // row max (scale > 0, so the max commutes with the scaling)
-      const float mx = row_max128(s0, s1, s2, s3) * scale_log2;
-      // lazy rescale decision
-      float alpha = 1.f;
-      bool resc = false;
-      if (m_run == -INFINITY) {
-        m_run = mx;
-      } else if (mx > m_run + 8.f) {
-        alpha = ex2(m_run - mx);
-        m_run = mx;
-        resc = true;
-      }
-      l_run *= alpha;
-      // P = exp2(s * scale - m) into packed bf16 registers first, so that the wait for
-      // the previous tile's P V (which still reads the P buffer) overlaps the exps
-      const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-      const float2 nm2 = make_float2(nm, nm), scale2 = make_float2(scale_log2, scale_log2);
-      uint32_t pk0[16], pk1[16], pk2[16], pk3[16];
-      const float2 ps = fadd2(fadd2(p_pack(s0, pk0, scale2, nm2), p_pack(s1, pk1, scale2, nm2)),
-                              fadd2(p_pack(s2, pk2, scale2, nm2), p_pack(s3, pk3, scale2, nm2)));
-      l_run += ps.x + ps.y;
-      if (j > 0) {
-        if (!mbar_wait(&o_done[q], uint32_t(j - 1) & 1u, &g_err_attn)) { ok = false; break; }
+    long long g = 0;  // tiles done (all items)
+    int itk = 0;      // items done
+    for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++itk) {
+      const FaItem w = fa_item(it, H, BH, npairs);
+      const int qtile = w.qa + q;
+      const long long i = (long long)qtile * QT + r;  // query position
+      // Visible keys of row i: [0, meta_end) and [win_lo, i] (positions).
+      const long long meta_end = is_global ? 0 : min((long long)n_meta, i + 1);
+      const long long win_lo = is_global ? 0 : max((long long)n_meta, i - window + 1);
+      const FaTiles tiles = fa_tiles(w.qa, L, n_meta, window, is_global);
+      float m_run = -INFINITY, l_run = 0.f;
+      int j = 0;
+      for (int kt = tiles.first(); kt <= tiles.hi; kt = tiles.next(kt), ++g, ++j) {
+        const int cls = fa_tile_class(qtile, kt, L, n_meta, window, is_global);  // uniform
+        if (!mbar_wait(&s_full[q], uint32_t(g) & 1u, &g_err_attn)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
-#pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tO + c * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-            tmem_st32(tO + c * 32, v);
+        if (cls == 0) {
+          // no visible pair in this tile (or the query tile lies past the sequence):
+          // S is released unread and P is zero; the running max and sum are unchanged
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&s_free[q]);
+          if (g > 0) {
+            if (!mbar_wait(&o_done[q], uint32_t(g - 1) & 1u, &g_err_attn)) { ok = false; break; }
+            tc_fence_after();
           }
-          tmem_wait_st();
+          uint32_t zero[16];
+#pragma unroll
+          for (int t = 0; t < 16; ++t) zero[t] = 0u;
+          p_store(zero, 0, r, p_base);
+          p_store(zero, 1, r, p_base);
+          p_store(zero, 2, r, p_base);
+          p_store(zero, 3, r, p_base);
+          fence_proxy_async();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&p_full[q]);
+          continue;
         }
+        // the whole S row in registers: four loads, one wait
+        uint32_t s0[32], s1[32], s2[32], s3[32];
+        tmem_ld32(tS, s0);
+        tmem_ld32(tS + 32, s1);
+        tmem_ld32(tS + 64, s2);
+        tmem_ld32(tS + 96, s3);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_free[q]);  // the MMA warp may overwrite S now
+        if (cls != 1) {
+          // partial tile: keep the column ranges [0, hi1) and [lo2, hi2)
+          const long long key0 = (long long)kt * KT;
+          const int hi1 = (int)max(0LL, min(128LL, meta_end - key0));
+          const int lo2 = (int)max(0LL, min(128LL, win_lo - key0));
+          const int hi2 = (int)max(0LL, min(128LL, i + 1 - key0));
+          mask_cols(s0, 0, hi1, lo2, hi2);
+          mask_cols(s1, 32, hi1, lo2, hi2);
+          mask_cols(s2, 64, hi1, lo2, hi2);
+          mask_cols(s3, 96, hi1, lo2, hi2);
+        }
+        // row max (scale > 0, so the max commutes with the scaling)
+        const float mx = row_max128(s0, s1, s2, s3) * scale_log2;
+        // lazy rescale decision
+        float alpha = 1.f;
+        bool resc = false;
+        if (m_run == -INFINITY) {
+          m_run = mx;
+        } else if (mx > m_run + 8.f) {
+          alpha = ex2(m_run - mx);
+          m_run = mx;
+          resc = true;
+        }
+        l_run *= alpha;
+        // P = exp2(s * scale - m) into packed bf16 registers first, so that the wait for
+        // the previous tile's P V (which still reads the P buffer) overlaps the exps
+        const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+        const float2 nm2 = make_float2(nm, nm), scale2 = make_float2(scale_log2, scale_log2);
+        uint32_t pk0[16], pk1[16], pk2[16], pk3[16];
+        const float2 ps = fadd2(fadd2(p_pack(s0, pk0, scale2, nm2), p_pack(s1, pk1, scale2, nm2)),
+                                fadd2(p_pack(s2, pk2, scale2, nm2), p_pack(s3, pk3, scale2, nm2)));
+        l_run += ps.x + ps.y;
+        if (g > 0) {
+          if (!mbar_wait(&o_done[q], uint32_t(g - 1) & 1u, &g_err_attn)) { ok = false; break; }
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t v[32];
+              tmem_ld32(tO + c * 32, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+              tmem_st32(tO + c * 32, v);
+            }
+            tmem_wait_st();
+          }
+        }
+        p_store(pk0, 0, r, p_base);
+        p_store(pk1, 1, r, p_base);
+        p_store(pk2, 2, r, p_base);
+        p_store(pk3, 3, r, p_base);
+        fence_proxy_async();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[q]);
       }
-      p_store(pk0, 0, r, p_base);
-      p_store(pk1, 1, r, p_base);
-      p_store(pk2, 2, r, p_base);
-      p_store(pk3, 3, r, p_base);
-      fence_proxy_async();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[q]);
-      ++j;
-    }
-    // epilogue: O / l -> bf16 rows of the output
-    if (ok && nstream > 0 && mbar_wait(&o_done[q], uint32_t(nstream - 1) & 1u, &g_err_attn)) {
+      if (!ok) break;
+      // the item's output once its last P V has retired: O / l -> bf16 rows written into
+      // this tile's P buffer (idle until the next item's first P) as two 128-byte-swizzled
+      // 64-column boxes, then two TMA tile stores (rows past the sequence are not written)
+      if (!mbar_wait(&o_done[q], uint32_t(g - 1) & 1u, &g_err_attn)) { ok = false; break; }
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      const int E = H * 128;
-      __nv_bfloat16 *dst = out + ((long long)b * L + i) * E + h * 128;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tO + c * 32, v);
-        tmem_wait_ld();
-        if (i < L) {
+      {
+        uint32_t v[4][32];
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            st_global_v4(dst + c * 32 + t * 8,
-                         pack_bf16x2(__uint_as_float(v[8 * t]) * inv, __uint_as_float(v[8 * t + 1]) * inv),
-                         pack_bf16x2(__uint_as_float(v[8 * t + 2]) * inv, __uint_as_float(v[8 * t + 3]) * inv),
-                         pack_bf16x2(__uint_as_float(v[8 * t + 4]) * inv, __uint_as_float(v[8 * t + 5]) * inv),
-                         pack_bf16x2(__uint_as_float(v[8 * t + 6]) * inv, __uint_as_float(v[8 * t + 7]) * inv));
-          }
+        for (int c = 0; c < 4; ++c) tmem_ld32(tO + c * 32, v[c]);
+        tmem_wait_ld();
+        tc_fence_before();  // O is in registers: the next item's first P V may overwrite it
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(v[c][2 * e]) * inv, __uint_as_float(v[c][2 * e + 1]) * inv);
+          p_store(pk, c, r, p_base);
         }
       }
+      fence_proxy_async();
+      mbar_arrive(&o_staged[q]);
+      if (quarter == 0 && lane == 0) {
+        // every row of the tile staged -> two stores; the buffer is released once they
+        // have read it (released on a failed wait too, so that no thread waits forever)
+        if (mbar_wait(&o_staged[q], uint32_t(itk) & 1u, &g_err_attn)) {
+          const uint8_t *stage = smem + OFF_P + q * P_BYTES;
+          tma_store_3d(&tmO, stage, w.h * 128, qtile * QT, w.b);
+          tma_store_3d(&tmO, stage + P_BYTES / 2, w.h * 128 + 64, qtile * QT, w.b);
+          bulk_commit();
+          bulk_wait_read();
+        }
+        mbar_arrive(&o_stored[q]);
+      }
+      if (!mbar_wait(&o_stored[q], uint32_t(itk) & 1u, &g_err_attn)) { ok = false; break; }
     }
+    if (quarter == 0 && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -449,7 +547,12 @@ static hymba_status attention_prefill_tc(const AttnArgs &a, cudaStream_t s) {
     }
     attr_set |= 1u << (dev & 31);
   }
-  CUtensorMap tq, tk, tv;
+  static int sms = 0;
+  if (sms == 0) {
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  CUtensorMap tq, tk, tv, to;
   const uint64_t dq[3] = {(uint64_t)a.H * 64, (uint64_t)a.L, (uint64_t)a.B};
   const uint64_t sq[2] = {(uint64_t)a.H * 64 * 2, (uint64_t)a.L * a.H * 64 * 2};
   const uint64_t dk[3] = {(uint64_t)a.Hkv * 64, (uint64_t)a.L, (uint64_t)a.B};
@@ -460,15 +563,16 @@ static hymba_status attention_prefill_tc(const AttnArgs &a, cudaStream_t s) {
   if (!make_tmap(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dq, sq, box)) return HYMBA_ERR_CUDA;
   if (!make_tmap(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dk, sk, box)) return HYMBA_ERR_CUDA;
   if (!make_tmap(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dv, sv, box)) return HYMBA_ERR_CUDA;
+  const uint64_t dout[3] = {(uint64_t)a.H * 128, (uint64_t)a.L, (uint64_t)a.B};
+  const uint64_t sout[2] = {(uint64_t)a.H * 128 * 2, (uint64_t)a.L * a.H * 128 * 2};
+  if (!make_tmap(&to, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dout, sout, box)) return HYMBA_ERR_CUDA;
   const int nqt = (a.L + QT - 1) / QT;
   const int npairs = (nqt + 1) / 2;
-  const long long blocks = (long long)npairs * a.H * a.B;
-  if (blocks > 0x7fffffffLL) {
-    set_error("attention grid too large");
-    return HYMBA_ERR_UNSUPPORTED;
-  }
-  attn_fwd_tc_kernel<<<(unsigned)blocks, THREADS, SMEM, s>>>(
-      tq, tk, tv, reinterpret_cast<__nv_bfloat16 *>(a.o), a.L, a.H, a.Hkv, a.n_meta, a.window,
+  const long long items = (long long)npairs * a.H * a.B;
+  if (items == 0) return HYMBA_OK;
+  const unsigned grid = (unsigned)std::min<long long>(items, sms);
+  attn_fwd_tc_kernel<<<grid, THREADS, SMEM, s>>>(
+      tq, tk, tv, to, a.L, a.B, a.H, a.Hkv, a.n_meta, a.window,
       a.is_global, a.scale * 1.4426950408889634f, npairs);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
@@ -790,22 +894,34 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---- bf16 decode attention on the tensor cores (mma.sync m16n8k16) ---------------
-// CTA = a run of CPC consecutive 128-slot chunks of one (sequence, kv head).  The
-// chunks stream through two shared-memory stages by 3-D TMA (128-byte swizzle, rows
-// past the store's capacity read as zero), the next chunk's copy in flight while the
-// current one is computed.  Warp w takes keys 32w..32w+31 of every chunk: S = Q K^T
-// with the query heads of the group in rows 0..rep-1 of a 16-row tile, an online
-// softmax in registers (running max and sum per row, O rescaled when the max grows),
-// O += P V with V fragments from ldmatrix.trans.  At the end the four warps' states are
-// merged in shared memory into one partial (max, sum, O) per query head and run.
+// Persistent: the work is the list of 128-slot chunks of every (sequence, kv head),
+// item i = (b * Hkv + g) * nchunks + chunk, cut into equal contiguous ranges, one per
+// CTA (two CTAs per SM).  A CTA streams its chunks through two shared-memory stages by
+// 3-D TMA (128-byte swizzle, rows past the store's capacity read as zero), the copy of
+// the next chunk in flight while the current one is computed, across (sequence, kv
+// head) boundaries too.  Warp w takes keys 32w..32w+31 of every chunk: S = Q K^T with
+// the query heads of the group in rows 0..rep-1 of a 16-row tile, an online softmax in
+// registers, O += P V with V fragments from ldmatrix.trans.  Where a run of chunks of
+// one (sequence, kv head) ends inside the CTA's range, the four warps' states are
+// merged in shared memory into one partial (max, sum, O) per query head, stored at the
+// slot of the run's first chunk; the combine kernel reads the run-start slots.
 namespace dtc {
 constexpr int SLOTS = 128;
 constexpr int K_BYTES = SLOTS * 128;        // 64 bf16 per slot
 constexpr int V_BYTES = SLOTS * 256;        // two 64-column boxes
 constexpr int STAGE = K_BYTES + V_BYTES;
-constexpr int SMEM = 2 * STAGE + 64 + 1024;  // the final merge reuses stage 0: two CTAs per SM
-constexpr int MAX_CPC = 4;                   // chunks per CTA
+constexpr int MAXREP = 8;
+// merge buffer [4 warps][rep][130] floats after the stages: two CTAs per SM for rep <= 5
+__host__ __device__ constexpr int merge_bytes(int rep) { return 4 * rep * 130 * 4; }
+__host__ __device__ constexpr int smem_bytes(int rep) { return 2 * STAGE + merge_bytes(rep) + 64 + 1024; }
+constexpr int CTAS_PER_SM = 2;
 }  // namespace dtc
+
+// First chunk of every run: a run starts at chunk 0 of a (sequence, kv head) or at the
+// first item of a CTA's range.
+__host__ __device__ __forceinline__ bool dec_run_start(long long item, int chunk, long long per) {
+  return chunk == 0 || item % per == 0;
+}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
                                         uint32_t &r3) {
@@ -836,28 +952,29 @@ __global__ void __launch_bounds__(128)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                           const __nv_bfloat16 *__restrict__ q, float *__restrict__ part, int H,
                           int Hkv, long long pos, int n_meta, int window, int is_global,
-                          float scale_log2, int nsplit, int cpc) {
+                          float scale_log2, long long n_items, long long per) {
   using namespace dtc;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t *sm = dsm_raw + ((1024 - (smem_u32(dsm_raw) & 1023)) & 1023);
-  float *om = reinterpret_cast<float *>(sm);  // [4 warps][8 rows][130], after the last chunk
-  uint64_t *full = reinterpret_cast<uint64_t *>(sm + 2 * STAGE);  // [2]
-  const int split = blockIdx.y, bg = blockIdx.x;
-  const int b = bg / Hkv, g = bg % Hkv;
   const int rep = H / Hkv;
+  float *mw = reinterpret_cast<float *>(sm + 2 * STAGE);                         // [4 warps][rep][130]
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + 2 * STAGE + merge_bytes(rep));  // [2]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = lane >> 2, gc = lane & 3;  // mma group row / column pair
   const long long nslots = dec_slots(pos, n_meta, window, is_global);
-  const long long nchunks = (nslots + SLOTS - 1) / SLOTS;
-  const int c0 = split * cpc;
-  const int nch = (int)max(0LL, min((long long)cpc, nchunks - c0));
-  auto issue = [&](int i) {  // chunk c0 + i into stage i & 1
-    uint8_t *dst = sm + (i & 1) * STAGE;
-    const int s0 = (c0 + i) * SLOTS;
-    mbar_arrive_expect_tx(&full[i & 1], STAGE);
-    tma_load_3d(dst, &tmK, &full[i & 1], 0, s0, bg);
-    tma_load_3d(dst + K_BYTES, &tmV, &full[i & 1], 0, s0, bg);
-    tma_load_3d(dst + K_BYTES + V_BYTES / 2, &tmV, &full[i & 1], 64, s0, bg);
+  const int nchunks = (int)((nslots + SLOTS - 1) / SLOTS);
+  const long long i0 = (long long)blockIdx.x * per;
+  const long long i1 = min(n_items, i0 + per);
+  if (i0 >= i1) return;
+  const int nloc = (int)(i1 - i0);
+  auto issue = [&](int k) {  // item i0 + k into stage k & 1
+    const long long it = i0 + k;
+    const int bg = (int)(it / nchunks), s0 = (int)(it % nchunks) * SLOTS;
+    uint8_t *dst = sm + (k & 1) * STAGE;
+    mbar_arrive_expect_tx(&full[k & 1], STAGE);
+    tma_load_3d(dst, &tmK, &full[k & 1], 0, s0, bg);
+    tma_load_3d(dst + K_BYTES, &tmV, &full[k & 1], 0, s0, bg);
+    tma_load_3d(dst + K_BYTES + V_BYTES / 2, &tmV, &full[k & 1], 64, s0, bg);
   };
   if (tid == 0) {
     mbar_init(&full[0], 1);
@@ -868,34 +985,38 @@ __global__ void __launch_bounds__(128)
   }
   __syncthreads();
   int issued = 0;
-  if (tid == 0) {
-    for (; issued < min(2, nch); ++issued) issue(issued);
-  }
-  // Q fragments (row = query head of the group, zero beyond rep), from global memory
-  uint32_t qa[4][2];  // [k-step][a0a1 / a4a5]; rows 8..15 are zero
-  {
-    const bool live = gr < rep;
-    const uint32_t *qr = reinterpret_cast<const uint32_t *>(q + ((long long)b * H + g * rep + (live ? gr : 0)) * 64);
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      qa[ks][0] = live ? __ldg(qr + ks * 8 + gc) : 0u;
-      qa[ks][1] = live ? __ldg(qr + ks * 8 + 4 + gc) : 0u;
-    }
-  }
+  if (tid == 0)
+    for (; issued < min(2, nloc); ++issued) issue(issued);
   float m_run = -INFINITY, l_run = 0.f;  // row gr of this warp
   float oacc[16][4];
-#pragma unroll
-  for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) oacc[nt][e] = 0.f;
+  uint32_t qa[4][2];  // Q fragments [k-step][a0a1 / a4a5]; rows 8..15 are zero
   bool ok = true;
-  int i = 0;
-  for (; i < nch; ++i) {
-    const int st = i & 1;
-    ok = mbar_wait(&full[st], uint32_t(i >> 1) & 1u, &g_err_attn);
+  int k = 0;
+  for (; k < nloc; ++k) {
+    const long long it = i0 + k;
+    const int bg = (int)(it / nchunks), chunk = (int)(it % nchunks);
+    const int b = bg / Hkv, g = bg % Hkv;
+    if (k == 0 || chunk == 0) {  // a run starts: fresh state, the group's queries
+      m_run = -INFINITY;
+      l_run = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < 16; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) oacc[nt][e] = 0.f;
+      const bool live = gr < rep;
+      const uint32_t *qr =
+          reinterpret_cast<const uint32_t *>(q + ((long long)b * H + g * rep + (live ? gr : 0)) * 64);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks) {
+        qa[ks][0] = live ? __ldg(qr + ks * 8 + gc) : 0u;
+        qa[ks][1] = live ? __ldg(qr + ks * 8 + 4 + gc) : 0u;
+      }
+    }
+    const int st = k & 1;
+    ok = mbar_wait(&full[st], uint32_t(k >> 1) & 1u, &g_err_attn);
     if (__syncthreads_or(!ok)) { ok = false; break; }
     const uint32_t kb = smem_u32(sm + st * STAGE), vb = kb + K_BYTES;
-    const long long s0 = (long long)(c0 + i) * SLOTS;
+    const long long s0 = (long long)chunk * SLOTS;
     const int ns = (int)min((long long)SLOTS, nslots - s0);
     // ---- S = Q K^T for this warp's 32 keys (4 n-tiles of 8 keys) ----
     float sacc[4][4];
@@ -944,12 +1065,10 @@ __global__ void __launch_bounds__(128)
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
     l_run = fmaf(l_run, alpha, lsum);
-    if (i > 0) {
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt) {
-        oacc[nt][0] *= alpha;
-        oacc[nt][1] *= alpha;
-      }
+    for (int nt = 0; nt < 16; ++nt) {
+      oacc[nt][0] *= alpha;
+      oacc[nt][1] *= alpha;
     }
     // ---- O += P V (16 n-tiles of 8 value columns, 2 k-steps of 16 keys) ----
 #pragma unroll
@@ -966,47 +1085,46 @@ __global__ void __launch_bounds__(128)
       }
     }
     __syncthreads();  // every warp is done with stage st
-    if (tid == 0 && issued < nch) issue(issued++);
-  }
-  if (!ok) {
-    // copies issued past the failed wait must land before the CTA leaves
-    if (tid == 0)
-      for (int k = i; k < issued; ++k) mbar_wait_drain(&full[k & 1], uint32_t(k >> 1) & 1u, &g_err_attn);
-    m_run = -INFINITY;
-    l_run = 0.f;
-  }
-  // ---- merge the four warps: rows 0..rep-1 (stage 0 is free: every copy has landed) ----
-  __syncthreads();
-  float *mw = om;  // per warp: [8 rows][130] = m, l, o[128]
-  if (gr < 8) {
-    float *row = mw + (warp * 8 + gr) * 130;
-    if (gc == 0) {
-      row[0] = m_run;
-      row[1] = l_run;
-    }
+    if (tid == 0 && issued < nloc) issue(issued++);
+    if (chunk == nchunks - 1 || k == nloc - 1) {
+      // the run ends: merge the four warps, rows 0..rep-1, into the run-start slot
+      if (gr < rep) {
+        float *row = mw + (warp * rep + gr) * 130;
+        if (gc == 0) {
+          row[0] = m_run;
+          row[1] = l_run;
+        }
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      row[2 + nt * 8 + 2 * gc] = oacc[nt][0];
-      row[2 + nt * 8 + 2 * gc + 1] = oacc[nt][1];
-    }
-  }
-  __syncthreads();
-  for (int idx = tid; idx < rep * 130; idx += 128) {
-    const int r = idx / 130, col = idx % 130;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, mw[(w * 8 + r) * 130]);
-    float acc = 0.f;
-    if (col == 0) {
-      acc = M;
-    } else {
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float mw_ = mw[(w * 8 + r) * 130];
-        if (mw_ != -INFINITY) acc += mw[(w * 8 + r) * 130 + col] * ex2(mw_ - M);
+        for (int nt = 0; nt < 16; ++nt) {
+          row[2 + nt * 8 + 2 * gc] = oacc[nt][0];
+          row[2 + nt * 8 + 2 * gc + 1] = oacc[nt][1];
+        }
       }
+      __syncthreads();
+      const int run_chunk = (int)(max(i0, it - chunk) - (it - chunk));  // the run began at item max(i0, it - chunk)
+      for (int idx = tid; idx < rep * 130; idx += 128) {
+        const int r = idx / 130, col = idx % 130;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, mw[(w * rep + r) * 130]);
+        float acc = 0.f;
+        if (col == 0) {
+          acc = M;
+        } else {
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const float mw_ = mw[(w * rep + r) * 130];
+            if (mw_ != -INFINITY) acc += mw[(w * rep + r) * 130 + col] * ex2(mw_ - M);
+          }
+        }
+        part[(((long long)b * H + g * rep + r) * nchunks + run_chunk) * 130 + col] = acc;
+      }
+      __syncthreads();  // the merge buffer is reused by the next run
     }
-    part[(((long long)b * H + g * rep + r) * nsplit + split) * 130 + col] = acc;
+  }
+  if (!ok && tid == 0) {
+    // copies issued past the failed wait must land before the CTA leaves
+    for (int kk = k; kk < issued; ++kk) mbar_wait_drain(&full[kk & 1], uint32_t(kk >> 1) & 1u, &g_err_attn);
   }
 }
 
@@ -1027,6 +1145,38 @@ __global__ void attn_decode_combine_kernel(const float *__restrict__ part, T *__
     for (int s = 0; s < nsplit; ++s) {
       const float ms = base[s * (dv + 2)];
       if (ms != -INFINITY) acc += base[s * (dv + 2) + 2 + d] * ex2(ms - M);
+    }
+    o[(long long)bh * dv + d] = Store<T>::from_f(acc / Lsum);
+  }
+}
+
+// Merges the run partials of one (sequence, query head): the slots of the chunks that
+// start a run of the persistent tensor-core kernel, i.e. chunk 0 and every chunk whose
+// item index is a multiple of `per` (the first at per - item0 % per, then every per).
+template <typename T>
+__global__ void attn_decode_combine_runs_kernel(const float *__restrict__ part, T *__restrict__ o, int H,
+                                                int Hkv, int dv, int nchunks, long long per) {
+  const int bh = blockIdx.x;
+  const int b = bh / H, h = bh % H, g = h / (H / Hkv);
+  const long long item0 = ((long long)b * Hkv + g) * nchunks;
+  const long long r0 = item0 % per;
+  const long long cfirst = r0 == 0 ? per : per - r0;  // first run start after chunk 0
+  const float *base = part + (long long)bh * nchunks * (dv + 2);
+  auto slot = [&](long long k) { return k == 0 ? 0LL : cfirst + (k - 1) * per; };
+  long long nruns = 1;
+  if (cfirst < nchunks) nruns += 1 + (nchunks - 1 - cfirst) / per;
+  float M = -INFINITY;
+  for (long long k = 0; k < nruns; ++k) M = fmaxf(M, base[slot(k) * (dv + 2)]);
+  float Lsum = 0.f;
+  for (long long k = 0; k < nruns; ++k) {
+    const float ms = base[slot(k) * (dv + 2)];
+    if (ms != -INFINITY) Lsum += base[slot(k) * (dv + 2) + 1] * ex2(ms - M);
+  }
+  for (int d = threadIdx.x; d < dv; d += blockDim.x) {
+    float acc = 0.f;
+    for (long long k = 0; k < nruns; ++k) {
+      const float ms = base[slot(k) * (dv + 2)];
+      if (ms != -INFINITY) acc += base[slot(k) * (dv + 2) + 2 + d] * ex2(ms - M);
     }
     o[(long long)bh * dv + d] = Store<T>::from_f(acc / Lsum);
   }
@@ -1063,7 +1213,8 @@ hymba_status attention_decode(const DecodeAttnArgs &a, hymba_dtype dt, cudaStrea
     int dev = 0;
     cudaGetDevice(&dev);
     if (!(attr_tc & (1u << (dev & 31)))) {
-      cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, dtc::SMEM);
+      cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           dtc::smem_bytes(dtc::MAXREP));
       attr_tc |= 1u << (dev & 31);
     }
     CUtensorMap tk, tv;
@@ -1074,17 +1225,21 @@ hymba_status attention_decode(const DecodeAttnArgs &a, hymba_dtype dt, cudaStrea
     const uint32_t box[3] = {64, (uint32_t)dtc::SLOTS, 1};
     if (!make_tmap(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dk, sk, box)) return HYMBA_ERR_CUDA;
     if (!make_tmap(&tv, a.v_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dvv, svv, box)) return HYMBA_ERR_CUDA;
-    // runs of up to MAX_CPC chunks, as even as the chunk count allows
+    // equal contiguous ranges of the (sequence, kv head, chunk) items, two CTAs per SM
+    static int sms = 0;
+    if (sms == 0) {
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (sms <= 0) sms = 148;
+    }
     const int nchunks = (int)((nslots + dtc::SLOTS - 1) / dtc::SLOTS);
-    const int runs = (nchunks + dtc::MAX_CPC - 1) / dtc::MAX_CPC;
-    const int cpc = (nchunks + runs - 1) / runs;
-    const int ns_tc = (nchunks + cpc - 1) / cpc;
-    dim3 grid_tc(a.B * a.Hkv, ns_tc);
-    attn_decode_tc_kernel<<<grid_tc, 128, dtc::SMEM, s>>>(tk, tv, (const __nv_bfloat16 *)a.q, a.partial,
-                                                         a.H, a.Hkv, a.pos, a.n_meta, a.window,
-                                                         a.is_global, sl2, ns_tc, cpc);
-    attn_decode_combine_kernel<__nv_bfloat16><<<a.B * a.H, 128, 0, s>>>(
-        a.partial, (__nv_bfloat16 *)a.o, a.H, a.dv, ns_tc);
+    const long long n_items = (long long)a.B * a.Hkv * nchunks;
+    const long long grid_tc = std::min<long long>(n_items, (long long)dtc::CTAS_PER_SM * sms);
+    const long long per = (n_items + grid_tc - 1) / grid_tc;
+    attn_decode_tc_kernel<<<(unsigned)((n_items + per - 1) / per), 128, dtc::smem_bytes(rep), s>>>(
+        tk, tv, (const __nv_bfloat16 *)a.q, a.partial, a.H, a.Hkv, a.pos, a.n_meta, a.window,
+        a.is_global, sl2, n_items, per);
+    attn_decode_combine_runs_kernel<__nv_bfloat16><<<a.B * a.H, 128, 0, s>>>(
+        a.partial, (__nv_bfloat16 *)a.o, a.H, a.Hkv, a.dv, nchunks, per);
   } else if (dt == HYMBA_BF16) {
     attn_decode_partial_kernel<__nv_bfloat16><<<grid, 128, dsmem, s>>>(
         (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k_cache, (const __nv_bfloat16 *)a.v_cache,

@@ -35,6 +35,24 @@ __device__ __forceinline__ int find_seg(const Epilogue &e, int n) {
   return s;
 }
 
+// Column `local` of a segment -> (group, offset in group) without a division on the
+// common layouts: one group, or a power-of-two group width.
+__device__ __forceinline__ long long seg_offset(const EpiSeg &g, long long m, int local) {
+  int grp, lin;
+  if (g.inner >= g.col1 - g.col0) {
+    grp = 0;
+    lin = local;
+  } else if ((g.inner & (g.inner - 1)) == 0) {
+    const int sh = __ffs(g.inner) - 1;
+    grp = local >> sh;
+    lin = local & (g.inner - 1);
+  } else {
+    grp = local / g.inner;
+    lin = local - grp * g.inner;
+  }
+  return m * g.ld_row + (long long)grp * g.ld_group + lin;
+}
+
 // Bias and activation of the fp32 CUDA-core path (full-precision softplus).
 __device__ __forceinline__ float epi_act(const Epilogue &e, int n, float v) {
   if (e.bias) v += __ldg(e.bias + n);
@@ -44,8 +62,7 @@ __device__ __forceinline__ float epi_act(const Epilogue &e, int n, float v) {
 
 __device__ __forceinline__ void epi_store_scalar(const Epilogue &e, long long m, int n, float v) {
   const EpiSeg &g = e.seg[find_seg(e, n)];
-  int local = n - g.col0;
-  long long off = m * g.ld_row + (long long)(local / g.inner) * g.ld_group + (local % g.inner);
+  const long long off = seg_offset(g, m, n - g.col0);
   if (e.atomic) {
     atomicAdd(reinterpret_cast<float *>(g.ptr) + off, v);
   } else if (g.f32) {
@@ -64,7 +81,7 @@ __device__ __forceinline__ void epi_store8(const Epilogue &e, long long m, int n
   bool vec = !e.atomic && g.vec_ok && (n + 8 <= N) && (n + 8 <= g.col1) && (local % 8 == 0) &&
              ((local % g.inner) + 8 <= g.inner);
   if (vec) {
-    long long off = m * g.ld_row + (long long)(local / g.inner) * g.ld_group + (local % g.inner);
+    const long long off = seg_offset(g, m, local);
     if (g.f32) {
       float *p = reinterpret_cast<float *>(g.ptr) + off;
       st_global_v4(p, __float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
@@ -83,31 +100,37 @@ __device__ __forceinline__ void epi_store8(const Epilogue &e, long long m, int n
     if (n + i < N) epi_store_scalar(e, m, n + i, v[i]);
 }
 
-// 16 consecutive product columns n0..n0+15 of row m from raw fp32 accumulator bits.
-// One segment lookup and one bias fetch per chunk on the common path.
+// Bias of columns n0..n0+15 (zero past N).
+__device__ __forceinline__ void epi_bias16(const Epilogue &e, int n0, int N, float (&b)[16]) {
+  if (n0 + 16 <= N) {
+    const float4 *bp = reinterpret_cast<const float4 *>(e.bias + n0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 b4 = __ldg(bp + q);
+      b[4 * q] = b4.x;
+      b[4 * q + 1] = b4.y;
+      b[4 * q + 2] = b4.z;
+      b[4 * q + 3] = b4.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) b[i] = n0 + i < N ? __ldg(e.bias + n0 + i) : 0.f;
+  }
+}
+
+// 16 consecutive product columns n0..n0+15 of row m from raw fp32 accumulator bits,
+// plus the bias (when the epilogue has one).  One segment lookup per chunk on the
+// common path.
 __device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, int n0, int N,
-                                            const uint32_t (&r)[16]) {
+                                            const uint32_t (&r)[16], const float (&bias)[16]) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
   const bool full = n0 + 16 <= N;
   if (!e.atomic) {
     if (e.bias) {
-      if (full) {
-        const float4 *bp = reinterpret_cast<const float4 *>(e.bias + n0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 b4 = __ldg(bp + q);
-          v[4 * q] += b4.x;
-          v[4 * q + 1] += b4.y;
-          v[4 * q + 2] += b4.z;
-          v[4 * q + 3] += b4.w;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          if (n0 + i < N) v[i] += __ldg(e.bias + n0 + i);
-      }
+      for (int i = 0; i < 16; ++i) v[i] += bias[i];
     }
     if (e.act == 1) {
 #pragma unroll
@@ -118,8 +141,9 @@ __device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, int 
   const int sidx = find_seg(e, n0);
   const EpiSeg &g = e.seg[sidx];
   const int local = n0 - g.col0;
-  if (full && !e.atomic && g.vec_ok && n0 + 16 <= g.col1 && (local % g.inner) + 16 <= g.inner) {
-    const long long off = m * g.ld_row + (long long)(local / g.inner) * g.ld_group + (local % g.inner);
+  if (full && !e.atomic && g.vec_ok && n0 + 16 <= g.col1 &&
+      (g.inner >= g.col1 - g.col0 || ((g.inner & 15) == 0 && (local & 15) == 0))) {
+    const long long off = seg_offset(g, m, local);
     if (g.f32) {
       float *p = reinterpret_cast<float *>(g.ptr) + off;
 #pragma unroll
@@ -326,21 +350,30 @@ __global__ void __launch_bounds__(576, 1)
       const int kb0 = ks * kb_per, kb1 = min(kblocks, kb0 + kb_per);
       if (kb0 >= kb1) continue;
       const int mt = int(tile / n_tiles), nt = int(tile % n_tiles);
+      constexpr int NCH = (BN + 63) / 64;
       if (!mbar_wait(&tfull[acc], acc_phase, &g_err_gemm)) break;
       tc_fence_after();
       const long long m = (long long)mt * C::BM + row;
       const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
-#pragma unroll 1
-      for (int c = sub * 16; c < BN; c += 64) {
-        const int n0 = nt * BN + c;
-        if (n0 >= N) break;  // uniform across the warp
-        uint32_t r[16];
-        tmem_ld16(t_row + c, r);
-        tmem_wait_ld();
-        if (m < M) epi_store16(s_epi, m, n0, N, r);
-      }
+      // all of this warp's chunks in one round of loads, then the accumulator is handed
+      // back to the MMA warp before the activation math and the stores
+      uint32_t r[NCH][16];
+#pragma unroll
+      for (int k = 0; k < NCH; ++k)
+        if (sub * 16 + 64 * k < BN) tmem_ld16(t_row + sub * 16 + 64 * k, r[k]);  // uniform per warp
+      tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
+#pragma unroll
+      for (int k = 0; k < NCH; ++k) {
+        const int c = sub * 16 + 64 * k;
+        const int n0 = nt * BN + c;
+        if (c < BN && n0 < N && m < M) {
+          float bias[16];
+          if (s_epi.bias) epi_bias16(s_epi, n0, N, bias);
+          epi_store16(s_epi, m, n0, N, r[k], bias);
+        }
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1u;

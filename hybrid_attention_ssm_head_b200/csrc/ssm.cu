@@ -218,63 +218,103 @@ hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s) {
 // (1) CTA = 16 sequences x CH channels: u = SiLU(conv(window, x) + b) for its
 //     channels (window advanced in conv_state, u stored), then its share of
 //     x_proj, xdbl[b, j] += sum over its channels of u[b, c] W_x[j, c], added
-//     atomically (E / CH partial sums per output).
+//     atomically (E / CH partial sums per output).  The W_x slice arrives by cp.async
+//     while the convolution runs; every global load of the convolution is issued
+//     before the first store.
 constexpr int kDecRows = 16;
 template <typename T, int CH>
 __global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
-  extern __shared__ __align__(16) float dsmem[];
-  float *us = dsmem;                   // [CH][kDecRows] u, channel-major (broadcast reads)
-  float *wt = dsmem + CH * kDecRows;   // [CH][NJP] W_x slice, transposed (odd stride)
-  const int NJ = a.R + 2 * a.N, NJP = NJ | 1;
+  constexpr int ROWB = CH * (int)sizeof(T) + 16;  // padded row of the W_x slice (conflict-free 16-byte reads)
+  constexpr int PIECES = CH * (int)sizeof(T) / 16;
+  constexpr int RPT = kDecRows * CH / 256;         // conv rows per thread
+  extern __shared__ __align__(16) uint8_t dsm_x[];
+  float *us = reinterpret_cast<float *>(dsm_x);    // [CH][kDecRows] u, channel-major (broadcast reads)
+  uint8_t *wxs = dsm_x + CH * kDecRows * 4;        // [NJ][ROWB] W_x slice
+  const int NJ = a.R + 2 * a.N;
   const int cbase = blockIdx.x * CH;
   const int b0 = blockIdx.y * kDecRows;
   const int tid = threadIdx.x;
   const T *wx = reinterpret_cast<const T *>(a.w_x);
-  for (int idx = tid; idx < NJ * CH; idx += 256) {
-    const int j = idx / CH, ch = idx % CH;  // coalesced along the channels of row j
-    wt[ch * NJP + j] = Store<T>::to_f(wx[(long long)j * a.E + cbase + ch]);
+  for (int idx = tid; idx < NJ * PIECES; idx += 256) {
+    const int j = idx / PIECES, pc = idx % PIECES;
+    cp_async16(wxs + j * ROWB + pc * 16, wx + (long long)j * a.E + cbase + pc * (16 / (int)sizeof(T)));
   }
-  // conv + SiLU: thread -> (channel, rows ch/CH-strided)
+  cp_async_commit();
+  // conv + SiLU: thread -> channel tid % CH, rows tid / CH + k * (256 / CH)
   {
     const int K = a.K;
     T *cs = reinterpret_cast<T *>(a.conv_state);
     const T *x = reinterpret_cast<const T *>(a.x);
     T *u = reinterpret_cast<T *>(a.u);
-    for (int idx = tid; idx < kDecRows * CH; idx += 256) {
-      const int ch = idx % CH, r = idx / CH;
-      const int b = b0 + r;
+    const int ch = tid % CH, c = cbase + ch;
+    float w[4], win[RPT][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[k] = k < K ? a.conv_w[c * K + k] : 0.f;
+    const float bias = a.conv_b[c];
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int b = b0 + tid / CH + k * (256 / CH);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        float v = 0.f;
+        if (b < a.B && t < K - 1) v = Store<T>::to_f(cs[((long long)b * (K - 1) + t) * a.E + c]);
+        else if (b < a.B && t == K - 1) v = Store<T>::to_f(x[(long long)b * a.ld_x + c]);
+        win[k][t] = v;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int r = tid / CH + k * (256 / CH), b = b0 + r;
       float uv = 0.f;
       if (b < a.B) {
-        const int c = cbase + ch;
-        float win[4];
-        for (int k = 0; k < K - 1; ++k) win[k] = Store<T>::to_f(cs[((long long)b * (K - 1) + k) * a.E + c]);
-        win[K - 1] = Store<T>::to_f(x[(long long)b * a.ld_x + c]);
-        float acc = a.conv_b[c];
-        for (int k = 0; k < K; ++k) acc = fmaf(a.conv_w[c * K + k], win[k], acc);
+        float acc = bias;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) acc = fmaf(w[t], win[k][t], acc);
         uv = silu_f(acc);
         u[(long long)b * a.E + c] = Store<T>::from_f(uv);
-        for (int k = 0; k < K - 1; ++k) cs[((long long)b * (K - 1) + k) * a.E + c] = Store<T>::from_f(win[k + 1]);
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+          if (t < K - 1) cs[((long long)b * (K - 1) + t) * a.E + c] = Store<T>::from_f(win[k][t + 1]);
       }
       us[ch * kDecRows + r] = uv;
     }
   }
+  cp_async_wait<0>();
   __syncthreads();
-  // x_proj share: thread -> output column j, all 16 rows
+  // x_proj share: thread -> output column j, all 16 rows, 16-byte reads of the W_x row
   for (int j = tid; j < NJ; j += 256) {
     float acc[kDecRows];
 #pragma unroll
     for (int r = 0; r < kDecRows; ++r) acc[r] = 0.f;
-#pragma unroll 4
-    for (int ch = 0; ch < CH; ++ch) {
-      const float w = wt[ch * NJP + j];
-      const float4 *u4 = reinterpret_cast<const float4 *>(us + ch * kDecRows);
+    const uint8_t *wrow = wxs + j * ROWB;
+#pragma unroll 2
+    for (int pc = 0; pc < PIECES; ++pc) {
+      const uint4 raw = *reinterpret_cast<const uint4 *>(wrow + pc * 16);
+      float wv[16 / sizeof(T)];
+      if constexpr (sizeof(T) == 2) {
+        const uint32_t q[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-      for (int q = 0; q < kDecRows / 4; ++q) {
-        const float4 v = u4[q];
-        acc[4 * q] = fmaf(v.x, w, acc[4 * q]);
-        acc[4 * q + 1] = fmaf(v.y, w, acc[4 * q + 1]);
-        acc[4 * q + 2] = fmaf(v.z, w, acc[4 * q + 2]);
-        acc[4 * q + 3] = fmaf(v.w, w, acc[4 * q + 3]);
+        for (int i = 0; i < 4; ++i) {
+          wv[2 * i] = bf16_lo(q[i]);
+          wv[2 * i + 1] = bf16_hi(q[i]);
+        }
+      } else {
+        wv[0] = __uint_as_float(raw.x);
+        wv[1] = __uint_as_float(raw.y);
+        wv[2] = __uint_as_float(raw.z);
+        wv[3] = __uint_as_float(raw.w);
+      }
+#pragma unroll
+      for (int i = 0; i < (int)(16 / sizeof(T)); ++i) {
+        const float4 *u4 = reinterpret_cast<const float4 *>(us + (pc * (16 / (int)sizeof(T)) + i) * kDecRows);
+#pragma unroll
+        for (int q = 0; q < kDecRows / 4; ++q) {
+          const float4 v = u4[q];
+          acc[4 * q] = fmaf(v.x, wv[i], acc[4 * q]);
+          acc[4 * q + 1] = fmaf(v.y, wv[i], acc[4 * q + 1]);
+          acc[4 * q + 2] = fmaf(v.z, wv[i], acc[4 * q + 2]);
+          acc[4 * q + 3] = fmaf(v.w, wv[i], acc[4 * q + 3]);
+        }
       }
     }
 #pragma unroll
@@ -284,9 +324,10 @@ __global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
 }
 
 // (2) CTA = 8 sequences x 128 channels, thread per channel: delta = softplus(b_dt +
-//     W_dt[c] . dt_low[b]) in fp32 (W_dt transposed in shared memory), then one step
-//     of the recurrence from the stored state (h_t = exp(delta A) h + delta B u,
-//     y = C . h + D u, gated by SiLU(z)), state written back in place.
+//     W_dt[c] . dt_low[b]) in fp32, then one step of the recurrence from the stored
+//     state (h_t = exp(delta A) h + delta B u, y = C . h + D u, gated by SiLU(z)), state
+//     written back in place.  The W_dt slice (contiguous rows) and the xdbl rows arrive
+//     by cp.async; W_dt rows are read 16 bytes at a time (conflict-free for R % 4 == 0).
 constexpr int kDecScanRows = 8;
 template <typename T>
 __device__ __forceinline__ float softplus_dec(float x) {
@@ -294,44 +335,28 @@ __device__ __forceinline__ float softplus_dec(float x) {
   else return softplus_accurate(x);
 }
 template <typename T>
-__global__ void __launch_bounds__(128) dec_dt_scan_kernel(DecodeSsmArgs a) {
+__global__ void __launch_bounds__(128, 4) dec_dt_scan_kernel(DecodeSsmArgs a) {
   extern __shared__ __align__(16) float dsmem[];
   const int R = a.R, NJ = a.R + 2 * kStates;
-  float *wdt = dsmem;                       // [R][129] transposed W_dt slice
-  float *xs = dsmem + R * 129;              // [NJ][kDecScanRows] xdbl rows, row-fastest
+  float *wdt = dsmem;               // [128][R] W_dt slice
+  float *xs = dsmem + 128 * R;      // [kDecScanRows][NJ] xdbl rows
   const int cbase = blockIdx.x * 128;
   const int b0 = blockIdx.y * kDecScanRows;
   const int tid = threadIdx.x;
-  for (int idx = tid; idx < 128 * R; idx += 128) {
-    const int ch = idx / R, r = idx % R;  // coalesced along r of channel ch
-    wdt[r * 129 + ch] = a.w_dt[(long long)(cbase + ch) * R + r];
-  }
-  for (int idx = tid; idx < kDecScanRows * NJ; idx += 128) {
-    const int rr = idx / NJ, j = idx % NJ;
-    xs[j * kDecScanRows + rr] = b0 + rr < a.B ? a.xdbl[(long long)(b0 + rr) * NJ + j] : 0.f;
-  }
-  __syncthreads();
-  const int c = cbase + tid;
-  if (c >= a.E) return;
-  float dtv[kDecScanRows];
-#pragma unroll
-  for (int rr = 0; rr < kDecScanRows; ++rr) dtv[rr] = 0.f;
-#pragma unroll 4
-  for (int r = 0; r < R; ++r) {
-    const float w = wdt[r * 129 + tid];
-    const float4 x0 = *reinterpret_cast<const float4 *>(xs + r * kDecScanRows);
-    const float4 x1 = *reinterpret_cast<const float4 *>(xs + r * kDecScanRows + 4);
-    dtv[0] = fmaf(x0.x, w, dtv[0]);
-    dtv[1] = fmaf(x0.y, w, dtv[1]);
-    dtv[2] = fmaf(x0.z, w, dtv[2]);
-    dtv[3] = fmaf(x0.w, w, dtv[3]);
-    dtv[4] = fmaf(x1.x, w, dtv[4]);
-    dtv[5] = fmaf(x1.y, w, dtv[5]);
-    dtv[6] = fmaf(x1.z, w, dtv[6]);
-    dtv[7] = fmaf(x1.w, w, dtv[7]);
-  }
-  float A2[kStates];
+  const int nrows = min(kDecScanRows, a.B - b0);
   {
+    const float *src = a.w_dt + (long long)cbase * R;
+    const int nw = min(128, a.E - cbase) * R / 4;
+    for (int idx = tid; idx < nw; idx += 128) cp_async16(wdt + idx * 4, src + idx * 4);
+    const float *xsrc = a.xdbl + (long long)b0 * NJ;
+    for (int idx = tid; idx < nrows * NJ / 4; idx += 128) cp_async16(xs + idx * 4, xsrc + idx * 4);
+    cp_async_commit();
+  }
+  const int c = cbase + tid;
+  const bool live = c < a.E;
+  float A2[kStates];
+  float bdt = 0.f, Dc = 0.f;
+  if (live) {
     const float4 *al4 = reinterpret_cast<const float4 *>(a.a_log + (long long)c * kStates);
 #pragma unroll
     for (int q = 0; q < kStates / 4; ++q) {
@@ -341,33 +366,65 @@ __global__ void __launch_bounds__(128) dec_dt_scan_kernel(DecodeSsmArgs a) {
       A2[4 * q + 2] = -kLog2e * ex2_ftz(kLog2e * v.z);
       A2[4 * q + 3] = -kLog2e * ex2_ftz(kLog2e * v.w);
     }
+    bdt = a.b_dt[c];
+    Dc = a.d_skip[c];
   }
-  const float bdt = a.b_dt[c], Dc = a.d_skip[c];
+  cp_async_wait<0>();
+  __syncthreads();
+  if (!live) return;
+  float dtv[kDecScanRows];
+#pragma unroll
+  for (int rr = 0; rr < kDecScanRows; ++rr) dtv[rr] = bdt;
+  const float4 *w4 = reinterpret_cast<const float4 *>(wdt + tid * R);
+#pragma unroll 2
+  for (int r4 = 0; r4 < R / 4; ++r4) {
+    const float4 w = w4[r4];
+#pragma unroll
+    for (int rr = 0; rr < kDecScanRows; ++rr) {
+      const float4 x = *reinterpret_cast<const float4 *>(xs + rr * NJ + 4 * r4);
+      dtv[rr] = fmaf(x.x, w.x, fmaf(x.y, w.y, fmaf(x.z, w.z, fmaf(x.w, w.w, dtv[rr]))));
+    }
+  }
   const T *u = reinterpret_cast<const T *>(a.u);
   const T *z = reinterpret_cast<const T *>(a.z);
   T *y = reinterpret_cast<T *>(a.y);
+  // the state, u and z of row rr + 1 are loaded before row rr's state is stored (the
+  // compiler cannot move loads above stores through the same pointer type itself)
+  float4 hn[kStates / 4];
+  float un = 0.f, zn = 0.f;
+  auto load_row = [&](int rr) {
+    const int b = b0 + rr;
+    const float4 *hp = reinterpret_cast<const float4 *>(a.h + ((long long)b * a.E + c) * kStates);
+#pragma unroll
+    for (int q = 0; q < kStates / 4; ++q) hn[q] = hp[q];
+    un = Store<T>::to_f(u[(long long)b * a.E + c]);
+    zn = Store<T>::to_f(z[(long long)b * a.ld_z + c]);
+  };
+  if (nrows > 0) load_row(0);
 #pragma unroll
   for (int rr = 0; rr < kDecScanRows; ++rr) {
     const int b = b0 + rr;
-    if (b >= a.B) continue;
-    const float d = softplus_dec<T>(dtv[rr] + bdt);
-    const float uu = Store<T>::to_f(u[(long long)b * a.E + c]);
-    const float zz = Store<T>::to_f(z[(long long)b * a.ld_z + c]);
+    if (rr >= nrows) continue;
+    float4 hv[kStates / 4];
+#pragma unroll
+    for (int q = 0; q < kStates / 4; ++q) hv[q] = hn[q];
+    const float uu = un, zz = zn;
+    if (rr + 1 < nrows) load_row(rr + 1);
+    const float d = softplus_dec<T>(dtv[rr]);
     const float du = d * uu;
     float4 *hp = reinterpret_cast<float4 *>(a.h + ((long long)b * a.E + c) * kStates);
+    const float *Bv = xs + rr * NJ + R, *Cv = Bv + kStates;
     float acc = 0.f;
 #pragma unroll
     for (int q = 0; q < kStates / 4; ++q) {
-      float4 hv = hp[q];
-      const float *Bq = xs + (R + 4 * q) * kDecScanRows + rr;
-      const float *Cq = xs + (R + kStates + 4 * q) * kDecScanRows + rr;
-      hv.x = fmaf(ex2_ftz(A2[4 * q] * d), hv.x, du * Bq[0]);
-      hv.y = fmaf(ex2_ftz(A2[4 * q + 1] * d), hv.y, du * Bq[kDecScanRows]);
-      hv.z = fmaf(ex2_ftz(A2[4 * q + 2] * d), hv.z, du * Bq[2 * kDecScanRows]);
-      hv.w = fmaf(ex2_ftz(A2[4 * q + 3] * d), hv.w, du * Bq[3 * kDecScanRows]);
-      acc = fmaf(Cq[0], hv.x, fmaf(Cq[kDecScanRows], hv.y,
-                 fmaf(Cq[2 * kDecScanRows], hv.z, fmaf(Cq[3 * kDecScanRows], hv.w, acc))));
-      hp[q] = hv;
+      const float4 B4 = *reinterpret_cast<const float4 *>(Bv + 4 * q);
+      const float4 C4 = *reinterpret_cast<const float4 *>(Cv + 4 * q);
+      hv[q].x = fmaf(ex2_ftz(A2[4 * q] * d), hv[q].x, du * B4.x);
+      hv[q].y = fmaf(ex2_ftz(A2[4 * q + 1] * d), hv[q].y, du * B4.y);
+      hv[q].z = fmaf(ex2_ftz(A2[4 * q + 2] * d), hv[q].z, du * B4.z);
+      hv[q].w = fmaf(ex2_ftz(A2[4 * q + 3] * d), hv[q].w, du * B4.w);
+      acc = fmaf(C4.x, hv[q].x, fmaf(C4.y, hv[q].y, fmaf(C4.z, hv[q].z, fmaf(C4.w, hv[q].w, acc))));
+      hp[q] = hv[q];
     }
     y[(long long)b * a.E + c] = Store<T>::from_f(fmaf(Dc, uu, acc) * silu_f(zz));
   }
@@ -376,8 +433,8 @@ __global__ void __launch_bounds__(128) dec_dt_scan_kernel(DecodeSsmArgs a) {
 template <typename T, int CH>
 static hymba_status decode_ssm_t(const DecodeSsmArgs &a, cudaStream_t s) {
   const int NJ = a.R + 2 * a.N;
-  const int smem1 = (CH * kDecRows + CH * (NJ | 1)) * 4;
-  const int smem2 = (a.R * 129 + kDecScanRows * NJ) * 4;
+  const int smem1 = CH * kDecRows * 4 + NJ * (CH * (int)sizeof(T) + 16);
+  const int smem2 = (128 * a.R + kDecScanRows * NJ) * 4;
   if (smem1 > 200 * 1024 || smem2 > 200 * 1024) {
     set_error("decode SSM: dt_rank %d too large for the fused decode kernels", a.R);
     return HYMBA_ERR_UNSUPPORTED;
@@ -428,17 +485,6 @@ hymba_status decode_ssm(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s) 
 // mode 1: scan from zero, record the chunk's end state and sum of delta.
 // u, delta, z and [B, C] of kScanTB steps are staged in shared memory with
 // cp.async (double-buffered) while the previous steps are being scanned.
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 // Two adjacent channels of one staged row.
 template <typename T>
