@@ -269,6 +269,8 @@ static EpiSeg seg(void *ptr, long long ld_row, int col0, int col1, int f32, size
   const size_t b = f32 ? 4 : es;
   s.vec_ok = aligned16(ptr) && ((ld_row * b) % 16 == 0) && ((ld_group * b) % 16 == 0) &&
              (s.inner % 8 == 0);
+  s.vec32 = s.vec_ok && (reinterpret_cast<uintptr_t>(ptr) % 32 == 0) && ((ld_row * b) % 32 == 0) &&
+            ((ld_group * b) % 32 == 0) && (s.inner % 16 == 0) && (col0 % 16 == 0);
   return s;
 }
 

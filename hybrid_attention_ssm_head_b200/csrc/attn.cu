@@ -11,10 +11,12 @@
 //                (M=128, N=128, K=128; V read MN-major from its natural layout).
 //   warps 4-7, 8-11 : one softmax warpgroup per query tile, one thread per row:
 //                row max over S (tcgen05.ld), lazy rescaling of O in TMEM only
-//                when the max grows by more than 2^8, exp2, P (bf16) written to
-//                shared memory in the 128-byte swizzled K-major layout.
-// The two query tiles ping-pong: while one warpgroup computes softmax the
-// tensor core runs the other tile's MMAs.  Key tiles with no visible pair are
+//                when the max grows by more than 2^8, exp2, P (bf16) written back
+//                into the first 64 columns of its own S (tcgen05.st), from where
+//                the P V MMA reads it as its A operand.
+// The two query tiles ping-pong: the MMA order per key tile is P V then the next
+// S for one query tile, then the same for the other, so while one warpgroup
+// computes its softmax the tensor core runs the other tile's MMAs.  Key tiles with no visible pair are
 // never loaded; fully visible tiles skip the per-element mask.
 //
 // fp32 path and decode: CUDA-core kernels (small or bandwidth-bound work).
@@ -45,13 +47,13 @@ constexpr int NQ = 2;            // query tiles per work item
 constexpr int Q_BYTES = QT * 128;        // 64 bf16 per row
 constexpr int K_BYTES = KT * 128;
 constexpr int V_BYTES = KT * 256;        // two 64-column boxes
-constexpr int P_BYTES = QT * 256;        // two 64-key swizzle atoms
+constexpr int P_BYTES = QT * 256;        // O staging of one query tile: two 64-column swizzle atoms
 constexpr int OFF_Q = 0;                 // two buffers (this item's and the next one's)
 constexpr int OFF_K = OFF_Q + 2 * NQ * Q_BYTES;
 constexpr int OFF_V = OFF_K + 2 * K_BYTES;
-constexpr int OFF_P = OFF_V + 2 * V_BYTES;
+constexpr int OFF_P = OFF_V + 2 * V_BYTES;  // O staging for the TMA stores
 constexpr int OFF_BAR = OFF_P + NQ * P_BYTES;
-constexpr int NBAR = 2 * 10 + 1 + 2 * NQ;
+constexpr int NBAR = 2 * 6 + 3 * NQ + 1 + 2 * NQ;
 constexpr int SMEM = OFF_BAR + NBAR * 8 + 16 + 1024;
 static_assert(SMEM <= 232448, "attention shared memory");
 constexpr int THREADS = 128 + NQ * 128;  // warpgroup 0: TMA + MMA; one softmax warpgroup per query tile
@@ -94,16 +96,20 @@ __device__ __forceinline__ FaTiles fa_tiles(int qa, int L, int n_meta, int windo
   return t;
 }
 
-// Work item of the persistent kernel: (sequence, head, query-tile pair).  Pairs run
-// from the last (the most key tiles in a causal layer) to the first, heads fastest so
-// that the heads of one kv group run side by side and share K/V tiles through L2.
+// Work item of the persistent kernel: (sequence, head, query-tile pair), heads fastest,
+// then pairs from the last (the most key tiles in a causal layer) to the first, then
+// sequences: the items running at one time are neighbouring pairs of one sequence with
+// all their heads, so a K/V tile is read from DRAM once and then shared through L2 by
+// the query heads of its group and by the overlapping windows of neighbouring pairs.
 struct FaItem {
   int b, h, qa;  // qa: first query tile of the pair
 };
 __device__ __forceinline__ FaItem fa_item(long long it, int H, int BH, int npairs) {
-  const int pair = npairs - 1 - (int)(it / BH);
-  const int rest = (int)(it % BH);
-  return {rest / H, rest % H, 2 * pair};
+  (void)BH;
+  const int h = (int)(it % H);
+  const long long rest = it / H;
+  const int pair = npairs - 1 - (int)(rest % npairs);
+  return {(int)(rest / npairs), h, 2 * pair};
 }
 __device__ __forceinline__ int fa_count(const FaTiles &t) {
   int n = 0;
@@ -185,10 +191,10 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
   uint64_t *q_full = bars + 0, *q_empty = bars + 2;    // [2]: Q buffers
   uint64_t *k_full = bars + 4, *k_empty = bars + 6;    // [2]: K stages
   uint64_t *v_full = bars + 8, *v_empty = bars + 10;   // [2]: V stages
-  uint64_t *s_full = bars + 12, *p_full = bars + 14;   // [NQ]
-  uint64_t *o_done = bars + 16, *s_free = bars + 18;   // [NQ]: PV retired / S in registers
-  uint64_t *drain = bars + 20;
-  uint64_t *o_staged = bars + 21, *o_stored = bars + 23;  // [NQ]: O rows in the P buffer / stored
+  uint64_t *s_full = bars + 12, *p_full = bars + 14;   // [NQ]: S ready / P written over it
+  uint64_t *o_done = bars + 16;                        // [NQ]: P V retired
+  uint64_t *drain = bars + 18;
+  uint64_t *o_staged = bars + 19, *o_stored = bars + 21;  // [NQ]: O rows staged / stored
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NBAR);
 
   const int warp = warp_id(), lane = lane_id();
@@ -208,7 +214,6 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
       mbar_init(&s_full[q], 1);
       mbar_init(&p_full[q], 4);
       mbar_init(&o_done[q], 1);
-      mbar_init(&s_free[q], 4);
     }
     mbar_init(drain, 1);
     for (int q = 0; q < NQ; ++q) {
@@ -276,7 +281,6 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
    } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer: one flat walk over the tiles of all items ----------------
-      const uint32_t p_addr0 = smem_u32(smem + OFF_P);
       auto issue_S = [&](int q, int st, int qb) {
         const uint32_t qa_ = smem_u32(smem + OFF_Q) + (qb * NQ + q) * Q_BYTES;
         const uint32_t ka = smem_u32(smem + OFF_K + st * K_BYTES);
@@ -286,14 +290,14 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
                       make_sdesc(ka + 32 * k, 16, 1024), IDESC_S, k > 0 ? 1u : 0u);
         mma_commit(&s_full[q]);
       };
+      // O += P V with P (bf16 pairs) in the first 64 columns of the tile's S
       auto issue_PV = [&](int q, int st, bool acc_prev) {
-        const uint32_t pa = p_addr0 + q * P_BYTES;
         const uint32_t va = smem_u32(smem + OFF_V + st * V_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t ad = make_sdesc(pa + (kk >> 2) * (P_BYTES / 2) + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = make_sdesc(va + kk * 2048, V_BYTES / 2, 1024);
-          mma_bf16_ss(tmem + 256 * q + 128, ad, bd, IDESC_PV, (acc_prev || kk > 0) ? 1u : 0u);
+          mma_bf16_ts(tmem + 256 * q + 128, tmem + 256 * q + 8 * kk, bd, IDESC_PV,
+                      (acc_prev || kk > 0) ? 1u : 0u);
         }
         mma_commit(&o_done[q]);
       };
@@ -318,39 +322,34 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
           const bool same = j + 1 < n;
           const long long it_next = same ? it : it + gridDim.x;
           const bool has_next = it_next < n_items;
+          const int qb_next = same ? (itk & 1) : ((itk + 1) & 1);
           int n_next = n;
+          const long long g1 = g + 1;
+          const int st = int(g & 1), st1 = int(g1 & 1);
           if (has_next) {
-            const int qb_next = same ? (itk & 1) : ((itk + 1) & 1);
             if (!same) {
               const FaItem wn = fa_item(it_next, H, BH, npairs);
               n_next = fa_count(fa_tiles(wn.qa, L, n_meta, window, is_global));
               if (!mbar_wait(&q_full[qb_next], (uint32_t(itk + 1) >> 1) & 1u, &g_err_attn)) { ok = false; break; }
             }
-            const long long g1 = g + 1;
-            const int st1 = int(g1 & 1);
             if (!mbar_wait(&k_full[st1], uint32_t(g1 >> 1) & 1u, &g_err_attn)) { ok = false; break; }
-            for (int q = 0; q < NQ && ok; ++q) {
-              if (!mbar_wait(&s_free[q], uint32_t(g) & 1u, &g_err_attn)) { ok = false; break; }
-              tc_fence_after();
-              issue_S(q, st1, qb_next);
-            }
-            if (!ok) break;
-            mma_commit(&k_empty[st1]);
-            // the last S of an item releases its Q buffer once it has run
-            if ((same ? j + 1 : 0) == (same ? n : n_next) - 1) mma_commit(&q_empty[qb_next]);
           }
-          // P V of the current tile
-          const int st = int(g & 1);
           if (!mbar_wait(&v_full[st], uint32_t(g >> 1) & 1u, &g_err_attn)) { ok = false; break; }
+          // per query tile: P V of this tile, then S of the next one into the same columns
+          // (the tensor core runs them in order, so P is read before S overwrites it)
           for (int q = 0; q < NQ && ok; ++q) {
             if (!mbar_wait(&p_full[q], uint32_t(g) & 1u, &g_err_attn)) { ok = false; break; }
             tc_fence_after();
             issue_PV(q, st, j > 0);
+            if (has_next) issue_S(q, st1, qb_next);
           }
           if (!ok) break;
           mma_commit(&v_empty[st]);
           if (!has_next) break;
-          ++g;
+          mma_commit(&k_empty[st1]);
+          // the last S of an item releases its Q buffer once it has run
+          if ((same ? j + 1 : 0) == (same ? n : n_next) - 1) mma_commit(&q_empty[qb_next]);
+          g = g1;
           if (same) {
             ++j;
           } else {
@@ -397,22 +396,13 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         tc_fence_after();
         if (cls == 0) {
           // no visible pair in this tile (or the query tile lies past the sequence):
-          // S is released unread and P is zero; the running max and sum are unchanged
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&s_free[q]);
-          if (g > 0) {
-            if (!mbar_wait(&o_done[q], uint32_t(g - 1) & 1u, &g_err_attn)) { ok = false; break; }
-            tc_fence_after();
-          }
+          // S is not read and P is zero; the running max and sum are unchanged
           uint32_t zero[16];
 #pragma unroll
           for (int t = 0; t < 16; ++t) zero[t] = 0u;
-          p_store(zero, 0, r, p_base);
-          p_store(zero, 1, r, p_base);
-          p_store(zero, 2, r, p_base);
-          p_store(zero, 3, r, p_base);
-          fence_proxy_async();
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_st16(tS + 16 * c, zero);
+          tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&p_full[q]);
@@ -425,9 +415,6 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         tmem_ld32(tS + 64, s2);
         tmem_ld32(tS + 96, s3);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_free[q]);  // the MMA warp may overwrite S now
         if (cls != 1) {
           // partial tile: keep the column ranges [0, hi1) and [lo2, hi2)
           const long long key0 = (long long)kt * KT;
@@ -452,35 +439,34 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
           resc = true;
         }
         l_run *= alpha;
-        // P = exp2(s * scale - m) into packed bf16 registers first, so that the wait for
-        // the previous tile's P V (which still reads the P buffer) overlaps the exps
+        // P = exp2(s * scale - m) as packed bf16 pairs
         const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
         const float2 nm2 = make_float2(nm, nm), scale2 = make_float2(scale_log2, scale_log2);
         uint32_t pk0[16], pk1[16], pk2[16], pk3[16];
         const float2 ps = fadd2(fadd2(p_pack(s0, pk0, scale2, nm2), p_pack(s1, pk1, scale2, nm2)),
                                 fadd2(p_pack(s2, pk2, scale2, nm2), p_pack(s3, pk3, scale2, nm2)));
         l_run += ps.x + ps.y;
-        if (g > 0) {
+        if (__any_sync(0xffffffffu, resc)) {
+          // O grows by the new max: rescale it once the previous tile's P V has retired
           if (!mbar_wait(&o_done[q], uint32_t(g - 1) & 1u, &g_err_attn)) { ok = false; break; }
           tc_fence_after();
-          if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-              uint32_t v[32];
-              tmem_ld32(tO + c * 32, v);
-              tmem_wait_ld();
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tO + c * 32, v);
+            tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-              tmem_st32(tO + c * 32, v);
-            }
-            tmem_wait_st();
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+            tmem_st32(tO + c * 32, v);
           }
         }
-        p_store(pk0, 0, r, p_base);
-        p_store(pk1, 1, r, p_base);
-        p_store(pk2, 2, r, p_base);
-        p_store(pk3, 3, r, p_base);
-        fence_proxy_async();
+        // P over the first 64 columns of S (already in registers; the previous tile's
+        // P V read its P before this tile's S was written)
+        tmem_st16(tS, pk0);
+        tmem_st16(tS + 16, pk1);
+        tmem_st16(tS + 32, pk2);
+        tmem_st16(tS + 48, pk3);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&p_full[q]);

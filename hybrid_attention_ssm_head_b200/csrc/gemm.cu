@@ -146,16 +146,31 @@ __device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, int 
     const long long off = seg_offset(g, m, local);
     if (g.f32) {
       float *p = reinterpret_cast<float *>(g.ptr) + off;
+      if (g.vec32) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-        st_global_v4(p + 4 * q, __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                     __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+        for (int q = 0; q < 2; ++q)
+          st_global_v8(p + 8 * q, __float_as_uint(v[8 * q]), __float_as_uint(v[8 * q + 1]),
+                       __float_as_uint(v[8 * q + 2]), __float_as_uint(v[8 * q + 3]),
+                       __float_as_uint(v[8 * q + 4]), __float_as_uint(v[8 * q + 5]),
+                       __float_as_uint(v[8 * q + 6]), __float_as_uint(v[8 * q + 7]));
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          st_global_v4(p + 4 * q, __float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                       __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3]));
+      }
     } else {
       __nv_bfloat16 *p = reinterpret_cast<__nv_bfloat16 *>(g.ptr) + off;
-      st_global_v4(p, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                   pack_bf16x2(v[6], v[7]));
-      st_global_v4(p + 8, pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
-                   pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+      if (g.vec32) {
+        st_global_v8(p, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                     pack_bf16x2(v[6], v[7]), pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                     pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+      } else {
+        st_global_v4(p, pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                     pack_bf16x2(v[6], v[7]));
+        st_global_v4(p + 8, pack_bf16x2(v[8], v[9]), pack_bf16x2(v[10], v[11]),
+                     pack_bf16x2(v[12], v[13]), pack_bf16x2(v[14], v[15]));
+      }
     }
     return;
   }
@@ -355,23 +370,31 @@ __global__ void __launch_bounds__(576, 1)
       tc_fence_after();
       const long long m = (long long)mt * C::BM + row;
       const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
-      // all of this warp's chunks in one round of loads, then the accumulator is handed
-      // back to the MMA warp before the activation math and the stores
-      uint32_t r[NCH][16];
+      // this warp's chunks in rounds of at most two loads; the accumulator is handed back
+      // to the MMA warp after the last round's loads, before its activation math and stores
+      constexpr int BATCH = NCH > 2 ? 2 : NCH;
 #pragma unroll
-      for (int k = 0; k < NCH; ++k)
-        if (sub * 16 + 64 * k < BN) tmem_ld16(t_row + sub * 16 + 64 * k, r[k]);  // uniform per warp
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      for (int k0 = 0; k0 < NCH; k0 += BATCH) {
+        uint32_t r[BATCH][16];
 #pragma unroll
-      for (int k = 0; k < NCH; ++k) {
-        const int c = sub * 16 + 64 * k;
-        const int n0 = nt * BN + c;
-        if (c < BN && n0 < N && m < M) {
-          float bias[16];
-          if (s_epi.bias) epi_bias16(s_epi, n0, N, bias);
-          epi_store16(s_epi, m, n0, N, r[k], bias);
+        for (int k = 0; k < BATCH; ++k) {
+          const int c = sub * 16 + 64 * (k0 + k);
+          if (k0 + k < NCH && c < BN) tmem_ld16(t_row + c, r[k]);  // uniform per warp
+        }
+        tmem_wait_ld();
+        if (k0 + BATCH >= NCH) {
+          tc_fence_before();
+          mbar_arrive(&tempty[acc]);
+        }
+#pragma unroll
+        for (int k = 0; k < BATCH; ++k) {
+          const int c = sub * 16 + 64 * (k0 + k);
+          const int n0 = nt * BN + c;
+          if (k0 + k < NCH && c < BN && n0 < N && m < M) {
+            float bias[16];
+            if (s_epi.bias) epi_bias16(s_epi, n0, N, bias);
+            epi_store16(s_epi, m, n0, N, r[k], bias);
+          }
         }
       }
       if (++acc == 2) {

@@ -20,6 +20,7 @@ struct EpiSeg {
   int inner;
   int f32;
   int vec_ok;  // 16-byte aligned rows/groups: 8-column vector stores allowed
+  int vec32;   // 32-byte aligned rows/groups: whole-sector (256-bit) stores allowed
 };
 
 struct Epilogue {
