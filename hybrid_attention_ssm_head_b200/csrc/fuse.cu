@@ -1,8 +1,8 @@
 // Fusion of the two branches (Hymba §2.1 Eq. 3): each branch output is
 // RMS-normalised over its d_inner channels, re-scaled per channel by beta and
 // the two are averaged:  f = (beta_1 * o / rms(o) + beta_2 * y / rms(y)) / 2.
-// One CTA per token row; 16-byte vector loads held in registers across the
-// row reduction, so each input is read once.
+// One CTA per token row; 16-byte vector loads held (packed) in registers across
+// the row reduction, so each input is read once.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -25,8 +25,26 @@ __device__ __forceinline__ void ld16(const T *p, float (&v)[16 / sizeof(T)]) {
   }
 }
 
+template <typename T>
+__device__ __forceinline__ void unpack16(const uint4 &raw, float (&v)[16 / sizeof(T)]) {
+  if constexpr (sizeof(T) == 2) {
+    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = bf16_lo(w[i]);
+      v[2 * i + 1] = bf16_hi(w[i]);
+    }
+  } else {
+    v[0] = __uint_as_float(raw.x);
+    v[1] = __uint_as_float(raw.y);
+    v[2] = __uint_as_float(raw.z);
+    v[3] = __uint_as_float(raw.w);
+  }
+}
+
 // Single read: each of the 128 threads keeps up to NV 16-byte vectors of both
-// branches in registers across the block reduction.
+// branches in registers across the block reduction, as raw (packed) words, so that
+// more rows fit on an SM; they are unpacked again for the output pass.
 template <typename T, int NV>
 __global__ void __launch_bounds__(128) fuse_kernel(FuseArgs a) {
   constexpr int V = 16 / sizeof(T);
@@ -35,18 +53,27 @@ __global__ void __launch_bounds__(128) fuse_kernel(FuseArgs a) {
   const T *o = reinterpret_cast<const T *>(a.o) + row * a.E;
   const T *y = reinterpret_cast<const T *>(a.y) + row * a.E;
   T *f = reinterpret_cast<T *>(a.f) + row * a.E;
-  float vo[NV][V], vy[NV][V];
+  uint4 ro_[NV], ry_[NV];
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int c = (threadIdx.x + j * 128) * V;
+    if (c < a.E) {
+      ro_[j] = __ldg(reinterpret_cast<const uint4 *>(o + c));
+      ry_[j] = __ldg(reinterpret_cast<const uint4 *>(y + c));
+    }
+  }
   float so = 0.f, sy = 0.f;
 #pragma unroll
   for (int j = 0; j < NV; ++j) {
     const int c = (threadIdx.x + j * 128) * V;
     if (c < a.E) {
-      ld16<T>(o + c, vo[j]);
-      ld16<T>(y + c, vy[j]);
+      float vo[V], vy[V];
+      unpack16<T>(ro_[j], vo);
+      unpack16<T>(ry_[j], vy);
 #pragma unroll
       for (int i = 0; i < V; ++i) {
-        so = fmaf(vo[j][i], vo[j][i], so);
-        sy = fmaf(vy[j][i], vy[j][i], sy);
+        so = fmaf(vo[i], vo[i], so);
+        sy = fmaf(vy[i], vy[i], sy);
       }
     }
   }
@@ -69,7 +96,9 @@ __global__ void __launch_bounds__(128) fuse_kernel(FuseArgs a) {
   for (int j = 0; j < NV; ++j) {
     const int c = (threadIdx.x + j * 128) * V;
     if (c < a.E) {
-      float ba[V], bs[V], out[V];
+      float vo[V], vy[V], ba[V], bs[V], out[V];
+      unpack16<T>(ro_[j], vo);
+      unpack16<T>(ry_[j], vy);
 #pragma unroll
       for (int i = 0; i < V; i += 4) {  // per-channel beta as 16-byte loads
         const float4 a4 = __ldg(reinterpret_cast<const float4 *>(a.beta_attn + c + i));
@@ -78,7 +107,7 @@ __global__ void __launch_bounds__(128) fuse_kernel(FuseArgs a) {
         bs[i] = s4.x; bs[i + 1] = s4.y; bs[i + 2] = s4.z; bs[i + 3] = s4.w;
       }
 #pragma unroll
-      for (int i = 0; i < V; ++i) out[i] = fmaf(ba[i] * ro, vo[j][i], bs[i] * ry * vy[j][i]);
+      for (int i = 0; i < V; ++i) out[i] = fmaf(ba[i] * ro, vo[i], bs[i] * ry * vy[i]);
       if constexpr (sizeof(T) == 2) {
         st_global_v4(f + c, pack_bf16x2(out[0], out[1]), pack_bf16x2(out[2], out[3]),
                      pack_bf16x2(out[4], out[5]), pack_bf16x2(out[6], out[7]));
