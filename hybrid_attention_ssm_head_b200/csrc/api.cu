@@ -545,11 +545,11 @@ static DecodeLayout decode_layout(const hymba_layer_config &c, int batch, long l
   d.x_ssm = take(B * E * es);
   d.z = take(B * E * es);
   d.u = take(B * E * es);
-  d.xdbl = take(B * xdbl_width(c) * 4);
+  d.xdbl = take(B * xdbl_width(c) * 4);  // xdbl and y32 adjacent: zeroed in one range
+  d.y32 = take(B * c.d_model * 4);
   d.y_ssm = take(B * E * es);
   d.o = take(B * E * es);
   d.f = take(B * E * es);
-  d.y32 = take(B * c.d_model * 4);
   d.part = take(decode_attn_workspace_floats(batch, c.n_heads, c.head_dim_v, pos, c.n_meta,
                                              c.window, c.is_global) * 4);
   d.total = off;
@@ -631,6 +631,9 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
                              (long long)c.n_kv_heads * cap * c.head_dim_qk,
                              (long long)c.n_kv_heads * cap * c.head_dim_v,
                              cap * c.head_dim_qk, cap * c.head_dim_v, xs, z, E);
+    // the split-K accumulators of x_proj and out_proj (adjacent) start at zero
+    g.epi.zero = xdbl;
+    g.epi.zero_n = (long long)((d.y32 - d.xdbl) / 4) + (long long)batch * c.d_model;
     if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
   }
   // 2-5. SSM branch: conv + x_proj, then dt_proj + softplus + one scan step + gate
@@ -700,8 +703,6 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
   {
     ProfScope prof_scope(stream, "dec_out_proj");
     const int ksplit = 4;
-    if (cudaMemsetAsync(y32, 0, (size_t)batch * c.d_model * 4, stream) != cudaSuccess)
-      FAIL(HYMBA_ERR_CUDA, "memset failed");
     GemmArgs g{};
     g.A = f;
     g.lda = E;

@@ -262,6 +262,11 @@ __global__ void __launch_bounds__(576, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  if (epi.zero && warp >= 2) {
+    for (long long i = (long long)blockIdx.x * 512 + (threadIdx.x - 64); i < epi.zero_n;
+         i += (long long)gridDim.x * 512)
+      epi.zero[i] = 0.f;
+  }
 
   if (warp == 0) {
     if (lane == 0) {
@@ -486,6 +491,11 @@ __global__ void __launch_bounds__(256)
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
   const int tid = threadIdx.x;
+  if (epi.zero) {
+    const long long nb = (long long)gridDim.x * gridDim.y * gridDim.z;
+    const long long bid = blockIdx.x + (long long)gridDim.x * (blockIdx.y + (long long)gridDim.y * blockIdx.z);
+    for (long long i = bid * 256 + tid; i < epi.zero_n; i += nb * 256) epi.zero[i] = 0.f;
+  }
   const int tx = tid & 15, ty = tid >> 4;
   const long long m0 = (long long)blockIdx.y * 64;
   const int n0 = blockIdx.x * 64;

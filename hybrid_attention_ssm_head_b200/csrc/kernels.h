@@ -9,6 +9,7 @@
 
 namespace hymba {
 
+
 // Where a GEMM output column goes.  Column c in [col0, col1) of the product is
 // written to  ptr + row*ld_row + ((c-col0)/inner)*ld_group + (c-col0)%inner
 // (element offsets), as fp32 (f32 = 1) or bf16 (f32 = 0).
@@ -29,6 +30,8 @@ struct Epilogue {
   const float *bias;  // per product column (nullable)
   int act;            // 0 = identity, 1 = softplus
   int atomic;         // 1 = fp32 atomicAdd into the destination (split-K)
+  float *zero;        // optional: zeroed by the GEMM (after the previous kernels), for
+  long long zero_n;   // split-K destinations of later kernels of the same step
 };
 
 // out[m, n] = epi( sum_k A[m, k] * B[n, k] )  (A: [M, K], B: [N, K], row-major)
@@ -134,7 +137,7 @@ struct DecodeSsmArgs {
   void *conv_state;    // [B, K-1, E] in/out
   const float *conv_w, *conv_b;  // [E, K], [E]
   const void *w_x;     // [R + 2N, E]
-  float *xdbl;         // [B, R + 2N] fp32, zeroed before the first kernel
+  float *xdbl;         // [B, R + 2N] fp32, zero on entry (the caller zeroes it)
   void *u;             // [B, E] conv + SiLU output
   const float *w_dt, *b_dt;      // [E, R], [E]
   const float *a_log, *d_skip;   // [E, N], [E]

@@ -121,12 +121,13 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
   const int t0 = tb * kConvTB;
   uint4 raw[NR];  // raw[r] = x[t0 - 3 + r], zero outside the sequence
 #pragma unroll
-  for (int r = 0; r < NR; ++r) {
-    const int t = t0 - 3 + r;
-    raw[r] = (t >= 0 && t < a.L)
-                 ? __ldg(reinterpret_cast<const uint4 *>(x + ((long long)b * a.L + t) * a.ld_x + c0))
-                 : make_uint4(0, 0, 0, 0);
+  for (int r = 0; r < NR; ++r) {  // unconditional loads (clamped row), zeroed afterwards
+    const int t = min(max(t0 - 3 + r, 0), a.L - 1);
+    raw[r] = __ldg(reinterpret_cast<const uint4 *>(x + ((long long)b * a.L + t) * a.ld_x + c0));
   }
+#pragma unroll
+  for (int r = 0; r < NR; ++r)
+    if (t0 - 3 + r < 0 || t0 - 3 + r >= a.L) raw[r] = make_uint4(0, 0, 0, 0);
   // wj[j][i] multiplies x[t - 3 + j] for channel c0 + i (taps right-aligned)
   float wj[4][V], bias[V];
   if (K == 4) {
@@ -240,41 +241,52 @@ __global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
     cp_async16(wxs + j * ROWB + pc * 16, wx + (long long)j * a.E + cbase + pc * (16 / (int)sizeof(T)));
   }
   cp_async_commit();
-  // conv + SiLU: thread -> channel tid % CH, rows tid / CH + k * (256 / CH)
+  // conv + SiLU: thread -> channel tid % CH, rows tid / CH + k * (256 / CH).  Every load
+  // is issued unconditionally (rows past the batch read a valid row and are discarded)
+  // and kept raw until all of them are in flight, so their latencies overlap.
   {
     const int K = a.K;
     T *cs = reinterpret_cast<T *>(a.conv_state);
     const T *x = reinterpret_cast<const T *>(a.x);
     T *u = reinterpret_cast<T *>(a.u);
     const int ch = tid % CH, c = cbase + ch;
-    float w[4], win[RPT][4];
+    float w[3];  // taps of the window rows (oldest first); wlast multiplies the new row
 #pragma unroll
-    for (int k = 0; k < 4; ++k) w[k] = k < K ? a.conv_w[c * K + k] : 0.f;
+    for (int k = 0; k < 3; ++k) w[k] = k < K - 1 ? a.conv_w[c * K + k] : 0.f;
+    const float wlast = a.conv_w[c * K + K - 1];
     const float bias = a.conv_b[c];
+    T raw[RPT][4];  // window rows oldest first; the new row x last
 #pragma unroll
     for (int k = 0; k < RPT; ++k) {
-      const int b = b0 + tid / CH + k * (256 / CH);
+      const int bb = min(b0 + tid / CH + k * (256 / CH), a.B - 1);
+      if (K > 1) {  // uniform: no window rows at all for a one-tap convolution
 #pragma unroll
-      for (int t = 0; t < 4; ++t) {
-        float v = 0.f;
-        if (b < a.B && t < K - 1) v = Store<T>::to_f(cs[((long long)b * (K - 1) + t) * a.E + c]);
-        else if (b < a.B && t == K - 1) v = Store<T>::to_f(x[(long long)b * a.ld_x + c]);
-        win[k][t] = v;
+        for (int t = 0; t < 3; ++t) raw[k][t] = cs[((long long)bb * (K - 1) + min(t, K - 2)) * a.E + c];
       }
+      raw[k][3] = x[(long long)bb * a.ld_x + c];
     }
 #pragma unroll
     for (int k = 0; k < RPT; ++k) {
       const int r = tid / CH + k * (256 / CH), b = b0 + r;
+      float win[3];
+#pragma unroll
+      for (int t = 0; t < 3; ++t) win[t] = 0.f;
+#pragma unroll
+      for (int t = 0; t < 3; ++t)
+        if (t < K - 1) win[t] = Store<T>::to_f(raw[k][t]);
+      float acc = bias;
+#pragma unroll
+      for (int t = 0; t < 3; ++t) acc = fmaf(w[t], win[t], acc);
+      acc = fmaf(wlast, Store<T>::to_f(raw[k][3]), acc);
       float uv = 0.f;
       if (b < a.B) {
-        float acc = bias;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) acc = fmaf(w[t], win[k][t], acc);
         uv = silu_f(acc);
         u[(long long)b * a.E + c] = Store<T>::from_f(uv);
+        // the window advances by one row: rows 1..K-2 move down, x becomes the newest
 #pragma unroll
         for (int t = 0; t < 3; ++t)
-          if (t < K - 1) cs[((long long)b * (K - 1) + t) * a.E + c] = Store<T>::from_f(win[k][t + 1]);
+          if (t < K - 1)
+            cs[((long long)b * (K - 1) + t) * a.E + c] = t + 1 < K - 1 ? raw[k][t + 1] : raw[k][3];
       }
       us[ch * kDecRows + r] = uv;
     }
@@ -323,37 +335,83 @@ __global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
   }
 }
 
-// (2) CTA = 8 sequences x 128 channels, thread per channel: delta = softplus(b_dt +
-//     W_dt[c] . dt_low[b]) in fp32, then one step of the recurrence from the stored
-//     state (h_t = exp(delta A) h + delta B u, y = C . h + D u, gated by SiLU(z)), state
-//     written back in place.  The W_dt slice (contiguous rows) and the xdbl rows arrive
-//     by cp.async; W_dt rows are read 16 bytes at a time (conflict-free for R % 4 == 0).
+// (2) CTA = 8 sequences x 128 channels.  dt_low (rank R) times the W_dt slice on the
+//     tensor cores (mma.sync m16n8k8, tf32 in, fp32 accumulate; rows 8..15 of the
+//     16-row tile are zero), then thread per channel: delta = softplus(. + b_dt), one
+//     step of the recurrence from the stored state (h_t = exp(delta A) h + delta B u,
+//     y = C . h + D u, gated by SiLU(z)), state written back in place.  W_dt (contiguous
+//     rows) and the xdbl rows arrive by cp.async; shared row strides are 4 mod 8 floats,
+//     so the tf32 fragment loads are free of bank conflicts.
 constexpr int kDecScanRows = 8;
 template <typename T>
 __device__ __forceinline__ float softplus_dec(float x) {
   if constexpr (sizeof(T) == 2) return softplus_f(x);
   else return softplus_accurate(x);
 }
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32_16808(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// shared layout of the dt_proj stage, in floats
+struct DecDtLayout {
+  int RP, WS, XS, NJ;  // rank padded to 8, W_dt row stride, xdbl row stride, xdbl width
+  __host__ __device__ DecDtLayout(int R, int N) {
+    RP = (R + 7) / 8 * 8;
+    WS = RP + 4;
+    NJ = R + 2 * N;
+    XS = (NJ + 7) / 8 * 8 + 4;
+  }
+  __host__ __device__ int wdt() const { return 0; }
+  __host__ __device__ int xs() const { return 128 * WS; }
+  __host__ __device__ int dts() const { return 128 * WS + 16 * XS; }
+  __host__ __device__ int floats() const { return 128 * WS + 16 * XS + kDecScanRows * 132; }
+};
 template <typename T>
-__global__ void __launch_bounds__(128, 4) dec_dt_scan_kernel(DecodeSsmArgs a) {
+__global__ void __launch_bounds__(128, 3) dec_dt_scan_kernel(DecodeSsmArgs a) {
   extern __shared__ __align__(16) float dsmem[];
-  const int R = a.R, NJ = a.R + 2 * kStates;
-  float *wdt = dsmem;               // [128][R] W_dt slice
-  float *xs = dsmem + 128 * R;      // [kDecScanRows][NJ] xdbl rows
+  const int R = a.R;
+  const DecDtLayout lay(R, kStates);
+  const int NJ = lay.NJ;
+  float *wdt = dsmem + lay.wdt();  // [128][WS] W_dt slice, columns R..RP-1 zero
+  float *xs = dsmem + lay.xs();    // [16][XS] xdbl rows (rows past the batch zero)
+  float *dts = dsmem + lay.dts();  // [kDecScanRows][132] dt_proj result
   const int cbase = blockIdx.x * 128;
   const int b0 = blockIdx.y * kDecScanRows;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nrows = min(kDecScanRows, a.B - b0);
+  const int nch = min(128, a.E - cbase);
   {
     const float *src = a.w_dt + (long long)cbase * R;
-    const int nw = min(128, a.E - cbase) * R / 4;
-    for (int idx = tid; idx < nw; idx += 128) cp_async16(wdt + idx * 4, src + idx * 4);
+    const int per_row = R / 4;
+    for (int idx = tid; idx < nch * per_row; idx += 128) {
+      const int ch = idx / per_row, pc = idx % per_row;
+      cp_async16(wdt + ch * lay.WS + pc * 4, src + (long long)ch * R + pc * 4);
+    }
+    for (int idx = tid; idx < 128 * (lay.RP - R); idx += 128) {
+      const int ch = idx / (lay.RP - R), k = R + idx % (lay.RP - R);
+      wdt[ch * lay.WS + k] = 0.f;
+    }
+    for (int idx = tid; idx < (128 - nch) * R; idx += 128) wdt[(nch + idx / R) * lay.WS + idx % R] = 0.f;
     const float *xsrc = a.xdbl + (long long)b0 * NJ;
-    for (int idx = tid; idx < nrows * NJ / 4; idx += 128) cp_async16(xs + idx * 4, xsrc + idx * 4);
+    for (int idx = tid; idx < nrows * (NJ / 4); idx += 128) {
+      const int r = idx / (NJ / 4), pc = idx % (NJ / 4);
+      cp_async16(xs + r * lay.XS + pc * 4, xsrc + (long long)r * NJ + pc * 4);
+    }
+    for (int idx = tid; idx < (16 - nrows) * lay.RP; idx += 128)
+      xs[(nrows + idx / lay.RP) * lay.XS + idx % lay.RP] = 0.f;
     cp_async_commit();
   }
   const int c = cbase + tid;
-  const bool live = c < a.E;
+  const bool live = tid < nch;
   float A2[kStates];
   float bdt = 0.f, Dc = 0.f;
   if (live) {
@@ -371,58 +429,70 @@ __global__ void __launch_bounds__(128, 4) dec_dt_scan_kernel(DecodeSsmArgs a) {
   }
   cp_async_wait<0>();
   __syncthreads();
-  if (!live) return;
-  float dtv[kDecScanRows];
+  // dt_proj on the tensor cores: warp w -> channels 32w..32w+31 (four 8-column tiles)
+  {
+    const int g = lane >> 2, t = lane & 3;
+    float d[4][4];
 #pragma unroll
-  for (int rr = 0; rr < kDecScanRows; ++rr) dtv[rr] = bdt;
-  const float4 *w4 = reinterpret_cast<const float4 *>(wdt + tid * R);
-#pragma unroll 2
-  for (int r4 = 0; r4 < R / 4; ++r4) {
-    const float4 w = w4[r4];
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-    for (int rr = 0; rr < kDecScanRows; ++rr) {
-      const float4 x = *reinterpret_cast<const float4 *>(xs + rr * NJ + 4 * r4);
-      dtv[rr] = fmaf(x.x, w.x, fmaf(x.y, w.y, fmaf(x.z, w.z, fmaf(x.w, w.w, dtv[rr]))));
+      for (int e = 0; e < 4; ++e) d[nt][e] = 0.f;
+    for (int k0 = 0; k0 < lay.RP; k0 += 8) {
+      const uint32_t a0 = to_tf32(xs[g * lay.XS + k0 + t]), a1 = to_tf32(xs[(g + 8) * lay.XS + k0 + t]);
+      const uint32_t a2 = to_tf32(xs[g * lay.XS + k0 + t + 4]), a3 = to_tf32(xs[(g + 8) * lay.XS + k0 + t + 4]);
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const float *wr = wdt + (warp * 32 + nt * 8 + g) * lay.WS + k0;
+        mma_tf32_16808(d[nt], a0, a1, a2, a3, to_tf32(wr[t]), to_tf32(wr[t + 4]));
+      }
+    }
+    if (g < kDecScanRows) {
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+        *reinterpret_cast<float2 *>(dts + g * 132 + warp * 32 + nt * 8 + 2 * t) = make_float2(d[nt][0], d[nt][1]);
     }
   }
+  __syncthreads();
+  if (!live) return;
   const T *u = reinterpret_cast<const T *>(a.u);
   const T *z = reinterpret_cast<const T *>(a.z);
   T *y = reinterpret_cast<T *>(a.y);
-  // the state, u and z of row rr + 1 are loaded before row rr's state is stored (the
-  // compiler cannot move loads above stores through the same pointer type itself)
+  // raw loads, converted at their use, so that the loads of row rr + 1 stay in flight
+  // while row rr is computed (rows past the batch read the last row and are discarded)
   float4 hn[kStates / 4];
-  float un = 0.f, zn = 0.f;
+  T un, zn;
   auto load_row = [&](int rr) {
-    const int b = b0 + rr;
+    const int b = min(b0 + rr, a.B - 1);
     const float4 *hp = reinterpret_cast<const float4 *>(a.h + ((long long)b * a.E + c) * kStates);
 #pragma unroll
     for (int q = 0; q < kStates / 4; ++q) hn[q] = hp[q];
-    un = Store<T>::to_f(u[(long long)b * a.E + c]);
-    zn = Store<T>::to_f(z[(long long)b * a.ld_z + c]);
+    un = u[(long long)b * a.E + c];
+    zn = z[(long long)b * a.ld_z + c];
   };
-  if (nrows > 0) load_row(0);
+  load_row(0);
 #pragma unroll
   for (int rr = 0; rr < kDecScanRows; ++rr) {
     const int b = b0 + rr;
-    if (rr >= nrows) continue;
     float4 hv[kStates / 4];
 #pragma unroll
     for (int q = 0; q < kStates / 4; ++q) hv[q] = hn[q];
-    const float uu = un, zz = zn;
-    if (rr + 1 < nrows) load_row(rr + 1);
-    const float d = softplus_dec<T>(dtv[rr]);
-    const float du = d * uu;
+    const T ur = un, zr = zn;
+    if (rr + 1 < kDecScanRows) load_row(rr + 1);
+    if (rr >= nrows) continue;
+    const float uu = Store<T>::to_f(ur), zz = Store<T>::to_f(zr);
+    const float dl = softplus_dec<T>(dts[rr * 132 + tid] + bdt);
+    const float du = dl * uu;
     float4 *hp = reinterpret_cast<float4 *>(a.h + ((long long)b * a.E + c) * kStates);
-    const float *Bv = xs + rr * NJ + R, *Cv = Bv + kStates;
+    const float *Bv = xs + rr * lay.XS + R, *Cv = Bv + kStates;
     float acc = 0.f;
 #pragma unroll
     for (int q = 0; q < kStates / 4; ++q) {
       const float4 B4 = *reinterpret_cast<const float4 *>(Bv + 4 * q);
       const float4 C4 = *reinterpret_cast<const float4 *>(Cv + 4 * q);
-      hv[q].x = fmaf(ex2_ftz(A2[4 * q] * d), hv[q].x, du * B4.x);
-      hv[q].y = fmaf(ex2_ftz(A2[4 * q + 1] * d), hv[q].y, du * B4.y);
-      hv[q].z = fmaf(ex2_ftz(A2[4 * q + 2] * d), hv[q].z, du * B4.z);
-      hv[q].w = fmaf(ex2_ftz(A2[4 * q + 3] * d), hv[q].w, du * B4.w);
+      hv[q].x = fmaf(ex2_ftz(A2[4 * q] * dl), hv[q].x, du * B4.x);
+      hv[q].y = fmaf(ex2_ftz(A2[4 * q + 1] * dl), hv[q].y, du * B4.y);
+      hv[q].z = fmaf(ex2_ftz(A2[4 * q + 2] * dl), hv[q].z, du * B4.z);
+      hv[q].w = fmaf(ex2_ftz(A2[4 * q + 3] * dl), hv[q].w, du * B4.w);
       acc = fmaf(C4.x, hv[q].x, fmaf(C4.y, hv[q].y, fmaf(C4.z, hv[q].z, fmaf(C4.w, hv[q].w, acc))));
       hp[q] = hv[q];
     }
@@ -434,7 +504,7 @@ template <typename T, int CH>
 static hymba_status decode_ssm_t(const DecodeSsmArgs &a, cudaStream_t s) {
   const int NJ = a.R + 2 * a.N;
   const int smem1 = CH * kDecRows * 4 + NJ * (CH * (int)sizeof(T) + 16);
-  const int smem2 = (128 * a.R + kDecScanRows * NJ) * 4;
+  const int smem2 = DecDtLayout(a.R, a.N).floats() * 4;
   if (smem1 > 200 * 1024 || smem2 > 200 * 1024) {
     set_error("decode SSM: dt_rank %d too large for the fused decode kernels", a.R);
     return HYMBA_ERR_UNSUPPORTED;
@@ -458,10 +528,6 @@ hymba_status decode_ssm(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s) 
   if (a.N != kStates || a.K > 4 || a.E % 32) {
     set_error("decode SSM needs d_state 16, d_conv <= 4, d_inner %% 32 == 0");
     return HYMBA_ERR_UNSUPPORTED;
-  }
-  if (cudaMemsetAsync(a.xdbl, 0, (size_t)a.B * (a.R + 2 * a.N) * 4, s) != cudaSuccess) {
-    set_error("decode SSM: memset failed");
-    return HYMBA_ERR_CUDA;
   }
   hymba_status st;
   if (dt == HYMBA_BF16)
