@@ -664,6 +664,8 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
     if ((st = decode_ssm(a, c.dtype, stream)) != HYMBA_OK) return st;
   }
   // 6. single-query attention over the store
+  int fuse_nchunks = 0;
+  long long fuse_per = 1;
   {
     ProfScope prof_scope(stream, "dec_attention");
     DecodeAttnArgs a{};
@@ -683,10 +685,31 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
     a.window = c.window;
     a.is_global = c.is_global;
     a.scale = score_scale(c);
+    // bf16: the fuse below merges the attention's run partials itself
+    a.fuse_later = c.dtype == HYMBA_BF16 && c.n_heads <= 32 && c.head_dim_v == 128 &&
+                   (long long)c.n_heads * c.head_dim_v == E;
     if ((st = attention_decode(a, c.dtype, stream)) != HYMBA_OK) return st;
+    fuse_nchunks = a.nchunks_out;
+    fuse_per = a.per_out;
   }
   // 7. norm, beta, mean
-  {
+  if (fuse_nchunks > 0) {
+    ProfScope prof_scope(stream, "dec_fuse");
+    FuseDecodeArgs a{};
+    a.part = part;
+    a.H = c.n_heads;
+    a.Hkv = c.n_kv_heads;
+    a.dv = c.head_dim_v;
+    a.nchunks = fuse_nchunks;
+    a.per = fuse_per;
+    a.y = yssm;
+    a.beta_attn = layer->w.beta_attn;
+    a.beta_ssm = layer->w.beta_ssm;
+    a.f = f;
+    a.B = batch;
+    a.eps = c.rms_eps;
+    if ((st = fuse_decode(a, stream)) != HYMBA_OK) return st;
+  } else {
     ProfScope prof_scope(stream, "dec_fuse");
     FuseArgs a{};
     a.o = o;

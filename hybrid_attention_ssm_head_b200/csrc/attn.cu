@@ -1168,7 +1168,8 @@ __global__ void attn_decode_combine_runs_kernel(const float *__restrict__ part, 
   }
 }
 
-hymba_status attention_decode(const DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s) {
+hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s) {
+  a.nchunks_out = 0;
   const int rep = a.H / a.Hkv;
   const int V = dt == HYMBA_BF16 ? 8 : 4;
   if (rep > DEC_MAXREP || a.dqk > 128 || a.dqk % V || a.dv > 256 || a.dv % 2) {
@@ -1224,8 +1225,21 @@ hymba_status attention_decode(const DecodeAttnArgs &a, hymba_dtype dt, cudaStrea
     attn_decode_tc_kernel<<<(unsigned)((n_items + per - 1) / per), 128, dtc::smem_bytes(rep), s>>>(
         tk, tv, (const __nv_bfloat16 *)a.q, a.partial, a.H, a.Hkv, a.pos, a.n_meta, a.window,
         a.is_global, sl2, n_items, per);
-    attn_decode_combine_runs_kernel<__nv_bfloat16><<<a.B * a.H, 128, 0, s>>>(
-        a.partial, (__nv_bfloat16 *)a.o, a.H, a.Hkv, a.dv, nchunks, per);
+    if (a.fuse_later) {
+      a.nchunks_out = nchunks;
+      a.per_out = per;
+      note_launch(1);
+    } else {
+      attn_decode_combine_runs_kernel<__nv_bfloat16><<<a.B * a.H, 128, 0, s>>>(
+          a.partial, (__nv_bfloat16 *)a.o, a.H, a.Hkv, a.dv, nchunks, per);
+      note_launch(2);
+    }
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+      set_error("decode attention launch failed: %s", cudaGetErrorString(e));
+      return HYMBA_ERR_CUDA;
+    }
+    return HYMBA_OK;
   } else if (dt == HYMBA_BF16) {
     attn_decode_partial_kernel<__nv_bfloat16><<<grid, 128, dsmem, s>>>(
         (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k_cache, (const __nv_bfloat16 *)a.v_cache,

@@ -222,4 +222,85 @@ hymba_status convert_f32_to(const float *src, void *dst, long long n, hymba_dtyp
   return HYMBA_OK;
 }
 
+// Decode fuse straight from the attention's run partials: CTA = one sequence, thread =
+// one value column d of every head.  Per head the runs' (max, sum) pairs give the merge
+// weights 2^(m_r - M) / L; the merged O stays in registers (fp32) for the two RMS norms
+// (the SSM row is read twice, the second time from cache).
+template <int MAXH>
+__global__ void __launch_bounds__(128) fuse_decode_kernel(FuseDecodeArgs a) {
+  __shared__ float red[2][4];
+  const int b = blockIdx.x, d = threadIdx.x;  // blockDim == dv == 128
+  const int rep = a.H / a.Hkv, E = a.H * a.dv;
+  float o[MAXH];
+  float so = 0.f;
+#pragma unroll
+  for (int h = 0; h < MAXH; ++h) {
+    o[h] = 0.f;
+    if (h >= a.H) continue;
+    const int g = h / rep;
+    const long long item0 = ((long long)b * a.Hkv + g) * a.nchunks;
+    const long long r0 = item0 % a.per;
+    const long long cfirst = r0 == 0 ? a.per : a.per - r0;
+    long long nruns = 1;
+    if (cfirst < a.nchunks) nruns += 1 + (a.nchunks - 1 - cfirst) / a.per;
+    const float *base = a.part + ((long long)b * a.H + h) * a.nchunks * (a.dv + 2);
+    float M = -INFINITY;
+    for (long long k = 0; k < nruns; ++k) M = fmaxf(M, base[(k == 0 ? 0 : cfirst + (k - 1) * a.per) * (a.dv + 2)]);
+    float Ls = 0.f, acc = 0.f;
+    for (long long k = 0; k < nruns; ++k) {
+      const float *r = base + (k == 0 ? 0 : cfirst + (k - 1) * a.per) * (a.dv + 2);
+      if (r[0] != -INFINITY) {
+        const float wgt = ex2_ftz(r[0] - M);
+        Ls = fmaf(r[1], wgt, Ls);
+        acc = fmaf(r[2 + d], wgt, acc);
+      }
+    }
+    o[h] = acc / Ls;
+    so = fmaf(o[h], o[h], so);
+  }
+  const __nv_bfloat16 *y = reinterpret_cast<const __nv_bfloat16 *>(a.y) + (long long)b * E;
+  float sy = 0.f;
+#pragma unroll
+  for (int h = 0; h < MAXH; ++h) {
+    const float yv = h < a.H ? __bfloat162float(y[h * a.dv + d]) : 0.f;
+    sy = fmaf(yv, yv, sy);
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) {
+    so += __shfl_xor_sync(0xffffffffu, so, off);
+    sy += __shfl_xor_sync(0xffffffffu, sy, off);
+  }
+  if ((d & 31) == 0) {
+    red[0][d >> 5] = so;
+    red[1][d >> 5] = sy;
+  }
+  __syncthreads();
+  so = red[0][0] + red[0][1] + red[0][2] + red[0][3];
+  sy = red[1][0] + red[1][1] + red[1][2] + red[1][3];
+  const float ro = 0.5f * rsqrtf(so / E + a.eps);
+  const float ry = 0.5f * rsqrtf(sy / E + a.eps);
+  __nv_bfloat16 *f = reinterpret_cast<__nv_bfloat16 *>(a.f) + (long long)b * E;
+#pragma unroll
+  for (int h = 0; h < MAXH; ++h) {
+    if (h >= a.H) continue;
+    const int c = h * a.dv + d;
+    f[c] = __float2bfloat16_rn(fmaf(a.beta_attn[c] * ro, o[h], a.beta_ssm[c] * ry * __bfloat162float(y[c])));
+  }
+}
+
+hymba_status fuse_decode(const FuseDecodeArgs &a, cudaStream_t s) {
+  if (a.dv != 128 || a.H > 32) {
+    set_error("fuse_decode needs d_v 128 and at most 32 heads");
+    return HYMBA_ERR_UNSUPPORTED;
+  }
+  fuse_decode_kernel<32><<<a.B, 128, 0, s>>>(a);
+  note_launch(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("decode fuse launch failed: %s", cudaGetErrorString(e));
+    return HYMBA_ERR_CUDA;
+  }
+  return HYMBA_OK;
+}
+
 }  // namespace hymba

@@ -92,6 +92,21 @@ struct FuseArgs {
   float eps;
 };
 hymba_status fuse_branches(const FuseArgs &a, hymba_dtype dt, cudaStream_t s);
+// Decode: the attention output is merged from the run partials of the tensor-core
+// decode attention (per (sequence, head): nchunks slots of (max, sum, O[dv]), the run
+// starts at chunk 0 and at every chunk whose item index is a multiple of per), then
+// fused with the SSM branch as fuse_branches does.
+struct FuseDecodeArgs {
+  const float *part;
+  int H, Hkv, dv, nchunks;
+  long long per;
+  const void *y;       // [B, H*dv]
+  const float *beta_attn, *beta_ssm;
+  void *f;             // [B, H*dv]
+  int B;
+  float eps;
+};
+hymba_status fuse_decode(const FuseDecodeArgs &a, cudaStream_t s);
 
 // ---- attention -----------------------------------------------------------
 struct AttnArgs {
@@ -122,10 +137,15 @@ struct DecodeAttnArgs {
   long long pos;
   int n_meta, window, is_global;
   float scale;
+  int fuse_later;            // bf16 tensor-core path: leave the run partials for fuse_decode
+  // out (fuse_later): where the run partials of (sequence, head) start, see fuse_decode
+  int nchunks_out;
+  long long per_out;
 };
 size_t decode_attn_workspace_floats(int B, int H, int dv, long long pos, int n_meta, int window,
                                     int is_global);
-hymba_status attention_decode(const DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s);
+// a.nchunks_out > 0 on return: the partials were left for fuse_decode (no output written)
+hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s);
 
 
 // ---- decode SSM branch: conv + x_proj, then dt_proj + softplus + scan step + gate ----
