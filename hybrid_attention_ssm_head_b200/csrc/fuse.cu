@@ -222,70 +222,95 @@ hymba_status convert_f32_to(const float *src, void *dst, long long n, hymba_dtyp
   return HYMBA_OK;
 }
 
-// Decode fuse straight from the attention's run partials: CTA = one sequence, thread =
-// one value column d of every head.  Per head the runs' (max, sum) pairs give the merge
-// weights 2^(m_r - M) / L; the merged O stays in registers (fp32) for the two RMS norms
-// (the SSM row is read twice, the second time from cache).
-template <int MAXH>
-__global__ void __launch_bounds__(128) fuse_decode_kernel(FuseDecodeArgs a) {
-  __shared__ float red[2][4];
-  const int b = blockIdx.x, d = threadIdx.x;  // blockDim == dv == 128
+// Decode fuse straight from the attention's run partials: CTA = one sequence, warp h =
+// head h, lane = four value columns.  Per head the runs' (max, sum) pairs give the merge
+// weights 2^(m_r - M) / L; the merged O (fp32, four values per lane) stays in registers
+// for the two RMS norms.
+__global__ void __launch_bounds__(1024) fuse_decode_kernel(FuseDecodeArgs a) {
+  __shared__ float red[2][32];
+  const int b = blockIdx.x, h = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rep = a.H / a.Hkv, E = a.H * a.dv;
-  float o[MAXH];
-  float so = 0.f;
-#pragma unroll
-  for (int h = 0; h < MAXH; ++h) {
-    o[h] = 0.f;
-    if (h >= a.H) continue;
+  const bool live = h < a.H;
+  float4 ov = make_float4(0.f, 0.f, 0.f, 0.f), yv = ov;
+  float so = 0.f, sy = 0.f;
+  if (live) {
     const int g = h / rep;
     const long long item0 = ((long long)b * a.Hkv + g) * a.nchunks;
     const long long r0 = item0 % a.per;
     const long long cfirst = r0 == 0 ? a.per : a.per - r0;
-    long long nruns = 1;
-    if (cfirst < a.nchunks) nruns += 1 + (a.nchunks - 1 - cfirst) / a.per;
+    int nruns = 1;
+    if (cfirst < a.nchunks) nruns += 1 + (int)((a.nchunks - 1 - cfirst) / a.per);
     const float *base = a.part + ((long long)b * a.H + h) * a.nchunks * (a.dv + 2);
+    auto run = [&](long long k) { return base + (k == 0 ? 0 : cfirst + (k - 1) * a.per) * (a.dv + 2); };
+    // the runs' (max, sum) pairs, 32 runs per round across the lanes
     float M = -INFINITY;
-    for (long long k = 0; k < nruns; ++k) M = fmaxf(M, base[(k == 0 ? 0 : cfirst + (k - 1) * a.per) * (a.dv + 2)]);
-    float Ls = 0.f, acc = 0.f;
-    for (long long k = 0; k < nruns; ++k) {
-      const float *r = base + (k == 0 ? 0 : cfirst + (k - 1) * a.per) * (a.dv + 2);
-      if (r[0] != -INFINITY) {
-        const float wgt = ex2_ftz(r[0] - M);
-        Ls = fmaf(r[1], wgt, Ls);
-        acc = fmaf(r[2 + d], wgt, acc);
+    for (int k0 = 0; k0 < nruns; k0 += 32)
+      if (k0 + lane < nruns) M = fmaxf(M, run(k0 + lane)[0]);
+#pragma unroll
+    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float L = 0.f;
+    for (int k0 = 0; k0 < nruns; k0 += 32) {
+      if (k0 + lane < nruns) {
+        const float *r = run(k0 + lane);
+        if (r[0] != -INFINITY) L = fmaf(r[1], ex2_ftz(r[0] - M), L);
       }
     }
-    o[h] = acc / Ls;
-    so = fmaf(o[h], o[h], so);
-  }
-  const __nv_bfloat16 *y = reinterpret_cast<const __nv_bfloat16 *>(a.y) + (long long)b * E;
-  float sy = 0.f;
 #pragma unroll
-  for (int h = 0; h < MAXH; ++h) {
-    const float yv = h < a.H ? __bfloat162float(y[h * a.dv + d]) : 0.f;
-    sy = fmaf(yv, yv, sy);
+    for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    for (int k = 0; k < nruns; ++k) {
+      const float *r = run(k);
+      const float mk = r[0];
+      if (mk == -INFINITY) continue;
+      const float w = ex2_ftz(mk - M) * inv;
+      // O starts at offset 2 (8-byte aligned): two float2 loads per lane
+      const float2 p0 = *reinterpret_cast<const float2 *>(r + 2 + 4 * lane);
+      const float2 p1 = *reinterpret_cast<const float2 *>(r + 2 + 4 * lane + 2);
+      ov.x = fmaf(p0.x, w, ov.x);
+      ov.y = fmaf(p0.y, w, ov.y);
+      ov.z = fmaf(p1.x, w, ov.z);
+      ov.w = fmaf(p1.y, w, ov.w);
+    }
+    so = ov.x * ov.x + ov.y * ov.y + ov.z * ov.z + ov.w * ov.w;
+    const uint2 raw = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(a.y) +
+                                                       (long long)b * E + h * a.dv + 4 * lane);
+    yv = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
+    sy = yv.x * yv.x + yv.y * yv.y + yv.z * yv.z + yv.w * yv.w;
   }
 #pragma unroll
   for (int off = 16; off; off >>= 1) {
     so += __shfl_xor_sync(0xffffffffu, so, off);
     sy += __shfl_xor_sync(0xffffffffu, sy, off);
   }
-  if ((d & 31) == 0) {
-    red[0][d >> 5] = so;
-    red[1][d >> 5] = sy;
+  if (lane == 0) {
+    red[0][h] = so;
+    red[1][h] = sy;
   }
   __syncthreads();
-  so = red[0][0] + red[0][1] + red[0][2] + red[0][3];
-  sy = red[1][0] + red[1][1] + red[1][2] + red[1][3];
-  const float ro = 0.5f * rsqrtf(so / E + a.eps);
-  const float ry = 0.5f * rsqrtf(sy / E + a.eps);
-  __nv_bfloat16 *f = reinterpret_cast<__nv_bfloat16 *>(a.f) + (long long)b * E;
+  if (h == 0) {
+    float a0 = lane < (int)(blockDim.x >> 5) ? red[0][lane] : 0.f;
+    float a1 = lane < (int)(blockDim.x >> 5) ? red[1][lane] : 0.f;
 #pragma unroll
-  for (int h = 0; h < MAXH; ++h) {
-    if (h >= a.H) continue;
-    const int c = h * a.dv + d;
-    f[c] = __float2bfloat16_rn(fmaf(a.beta_attn[c] * ro, o[h], a.beta_ssm[c] * ry * __bfloat162float(y[c])));
+    for (int off = 16; off; off >>= 1) {
+      a0 += __shfl_xor_sync(0xffffffffu, a0, off);
+      a1 += __shfl_xor_sync(0xffffffffu, a1, off);
+    }
+    if (lane == 0) {
+      red[0][0] = a0;
+      red[1][0] = a1;
+    }
   }
+  __syncthreads();
+  if (!live) return;
+  const float ro = 0.5f * rsqrtf(red[0][0] / E + a.eps);
+  const float ry = 0.5f * rsqrtf(red[1][0] / E + a.eps);
+  const int c = h * a.dv + 4 * lane;
+  const float4 ba = *reinterpret_cast<const float4 *>(a.beta_attn + c);
+  const float4 bs = *reinterpret_cast<const float4 *>(a.beta_ssm + c);
+  uint2 outw;
+  outw.x = pack_bf16x2(fmaf(ba.x * ro, ov.x, bs.x * ry * yv.x), fmaf(ba.y * ro, ov.y, bs.y * ry * yv.y));
+  outw.y = pack_bf16x2(fmaf(ba.z * ro, ov.z, bs.z * ry * yv.z), fmaf(ba.w * ro, ov.w, bs.w * ry * yv.w));
+  *reinterpret_cast<uint2 *>(reinterpret_cast<__nv_bfloat16 *>(a.f) + (long long)b * E + c) = outw;
 }
 
 hymba_status fuse_decode(const FuseDecodeArgs &a, cudaStream_t s) {
@@ -293,7 +318,7 @@ hymba_status fuse_decode(const FuseDecodeArgs &a, cudaStream_t s) {
     set_error("fuse_decode needs d_v 128 and at most 32 heads");
     return HYMBA_ERR_UNSUPPORTED;
   }
-  fuse_decode_kernel<32><<<a.B, 128, 0, s>>>(a);
+  fuse_decode_kernel<<<a.B, 32 * a.H, 0, s>>>(a);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

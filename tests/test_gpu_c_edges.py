@@ -99,3 +99,26 @@ def test_nan_inputs_propagate_without_fault():
     ref = O.layer_prefill(H.to64(x[1]), H.oracle_weights(lay.cpu), lay.spec)
     H.close_bf16(H.to64(y[1]), ref["Y"], "clean sequence")
     lay.close()
+
+
+def test_decode_global_more_runs_than_a_warp():
+    """Batch 1 on a long global layer: few (sequence, kv head, chunk) items, so every chunk
+    of the store becomes its own run of the persistent decode attention (35 runs per head),
+    more than one warp merges in one round."""
+    w = synth.configs.Workload("edge_dec_runs", DIMS_BF16_SMALL, "bf16", 1, 128, 4300, 0)
+    lay = H.GpuLayer(w, 0, is_global=True)
+    pos = w.n_meta + w.n_tokens
+    cap = pos + 1
+    c = {k: t.contiguous() for k, t in synth.configs.decode_caches(w, 0, cap, False, device="cuda").items()}
+    kvc = hy.hymba_kv_cache(c["k"].data_ptr(), c["v"].data_ptr(), 1, cap, 0)
+    ssm = hy.hymba_ssm_cache(c["ssm"].data_ptr(), c["conv"].data_ptr())
+    dws = H.workspace(hy.hymba_layer_decode_workspace(lay.handle, 1, pos))
+    xt = synth.gen.normal_tensor((1, w.dims.d_model), 0, "edge_dec_runs/x", device="cuda").to(torch.bfloat16)
+    yt = torch.empty_like(xt)
+    hy.hymba_layer_decode_step(lay.handle, 1, pos, xt, yt, kvc, ssm, dws, dws.numel(),
+                               torch.cuda.current_stream())
+    hy.hymba_stream_status(torch.cuda.current_stream())
+    cache = {k: H.to64(t) for k, t in synth.configs.decode_caches(w, 0, cap, False, batch_index=0).items()}
+    yo, _ = O.layer_decode(H.to64(xt[0]), pos, H.oracle_weights(lay.cpu), lay.spec, cache)
+    H.close_bf16(H.to64(yt[0]), yo, "decode y, 35 runs")
+    lay.close()
