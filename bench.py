@@ -41,7 +41,7 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # profiles/gemm_b32.md), scaled by rows to one producer launch of the headline prefill
 # (1,064,960 rows).  The algorithmic minimum is 22.5 GB (read X~ and W_in, write the
 # 8960 output columns), so the kernel re-reads nothing.
-IN_PROJ_TRAFFIC = (156.06e6 + 616.80e6) * 1064960 / 36864
+IN_PROJ_TRAFFIC = (152.7e6 + 627.8e6) * 1064960 / 36864
 IN_PROJ_TRAFFIC_BASIS = "ncu b32 in_proj capture scaled by rows to one producer launch"
 
 
