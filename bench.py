@@ -37,7 +37,7 @@ METRIC = "hybrid-layer prefill tok/s @B=128,L=8k bf16 + decode tok/s; % of roofl
 UNIT = "tok/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one in_proj launch: ncu dram__bytes_{read,write}.sum of the
-# in_proj launch of `bench.py --case b32` (36,864 rows: 156.06 MB + 616.80 MB, see
+# in_proj launch of `bench.py --case b32` (36,864 rows: 152.7 MB + 627.8 MB, see
 # profiles/gemm_b32.md), scaled by rows to one producer launch of the headline prefill
 # (1,064,960 rows).  The algorithmic minimum is 22.5 GB (read X~ and W_in, write the
 # 8960 output columns), so the kernel re-reads nothing.
