@@ -45,6 +45,19 @@ IN_PROJ_TRAFFIC = (152.7e6 + 627.8e6) * 1064960 / 36864
 IN_PROJ_TRAFFIC_BASIS = "ncu b32 in_proj capture scaled by rows to one producer launch"
 
 
+def max_over_ranks(vals, device, world: int):
+    """This rank's device times -> the slowest rank's, elementwise (one MAX all-reduce)."""
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_rate(units_per_rank_step: float, steps: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the units every replica processed over the slowest rank's time."""
+    return units_per_rank_step * steps * world / (ms / 1e3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -310,10 +323,7 @@ def run_ours(args, rank, world, dev):
     pre_ms = sum(ev[2 * s].elapsed_time(ev[2 * s + 1]) for s in range(args.steps))
     dec_ms = sum(ev[2 * s + 1].elapsed_time(ev[2 * s + 2]) for s in range(args.steps))
     tot_ms = ev[0].elapsed_time(ev[-1])
-    t = torch.tensor([pre_ms, dec_ms, tot_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    pre_ms, dec_ms, tot_ms = t.tolist()
+    pre_ms, dec_ms, tot_ms = max_over_ranks([pre_ms, dec_ms, tot_ms], dev, world)
 
     # kernel launches of this library in the timed region: prefill launches are counted by the
     # profiler; the decode graph holds a fixed number per step (counted once below, eagerly)
@@ -326,8 +336,8 @@ def run_ours(args, rank, world, dev):
     dec_kernels_per_step = sum(k for _, _, k, _ in dprof)
 
     tokens = w3.batch * w3.n_tokens
-    value = tokens * args.steps * world / (pre_ms / 1e3)
-    dec_tok_s = w4.batch * args.steps * world / (dec_ms / 1e3)
+    value = job_rate(tokens, args.steps, world, pre_ms)
+    dec_tok_s = job_rate(w4.batch, args.steps, world, dec_ms)
 
     # roofline of the dominant kernel: the input projection GEMM (tensor-bound)
     pmap = {n: (c, ms) for n, c, _, ms in prof}
@@ -399,14 +409,11 @@ def run_ours(args, rank, world, dev):
             ed1.record(stream)
             torch.cuda.synchronize()
             dec_e2e_ms += ed0.elapsed_time(ed1)
-        t = torch.tensor([pre_e2e_ms, dec_e2e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        pre_e2e_ms, dec_e2e_ms = t.tolist()
-        e2e = {"value": tokens * steps_e2e * world / (pre_e2e_ms / 1e3), "unit": UNIT,
+        pre_e2e_ms, dec_e2e_ms = max_over_ranks([pre_e2e_ms, dec_e2e_ms], dev, world)
+        e2e = {"value": job_rate(tokens, steps_e2e, world, pre_e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": xh.numel() * 2 + xt_h.numel() * 2,
                "d2h_bytes_per_step": yh.numel() * 2 + yt_h.numel() * 2,
-               "decode_tok_s": w4.batch * steps_e2e * world / (dec_e2e_ms / 1e3),
+               "decode_tok_s": job_rate(w4.batch, steps_e2e, world, dec_e2e_ms),
                "copies": "overlapped with compute on two copy streams, device buffers double-buffered"}
 
     cpu = None
