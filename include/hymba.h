@@ -49,7 +49,7 @@ typedef struct CUstream_st *hymba_stream_t; /* a cudaStream_t; NULL = legacy def
 typedef enum {
   HYMBA_OK = 0,
   HYMBA_ERR_INVALID_ARG = 1,  /* bad shape, null pointer, misaligned pointer   */
-  HYMBA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement   */
+  HYMBA_ERR_UNSUPPORTED = 2,  /* valid request the library does not implement */
   HYMBA_ERR_WORKSPACE = 3,    /* workspace smaller than the query returned     */
   HYMBA_ERR_NOT_BOUND = 4,    /* K/V sharing: consumer/producer mismatch       */
   HYMBA_ERR_CUDA = 5,         /* a CUDA runtime call failed                    */
