@@ -28,8 +28,11 @@ the design notes of this repository):
   * norm = RMS over all d_inner channels with no weight, eps as configured;
   * Eq. (3)'s two branches are averaged (divided by 2) as the text says;
   * no biases in the in/x/out projections; no RoPE.
-Parity unpinned (fixed only by these readings, not by the pages): the conv,
-the low-rank delta, the SiLU gate, the RMS form of "norm" and D.
+The pages print no value that checks the readings of the conv, the low-rank
+delta, the SiLU gate, the RMS form of "norm" and D; the functions themselves are
+pinned by the tests through special cases with closed forms or library routines
+(the conv against numpy.convolve; D and the gate with the C rows at zero; delta
+with W_dt = 0 and with a full-rank identity; the norm against its closed form).
 """
 from __future__ import annotations
 

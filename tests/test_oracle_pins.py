@@ -196,6 +196,68 @@ def test_elementwise_functions_known_values():
                                [0.0, 1 / (1 + math.exp(-1)), -2 / (1 + math.exp(2))], rtol=1e-14)
 
 
+# --- the SSM readings (Mamba-1 form) reduced to closed forms by special weights --------------
+
+def _silu_scalar(x):
+    return x / (1.0 + math.exp(-x))
+
+
+def _softplus_scalar(x):
+    return math.log1p(math.exp(x)) if x < 30 else x + math.log1p(math.exp(-x))
+
+
+def test_ssm_with_C_zero_is_the_D_skip_times_the_gate():
+    """With the C rows of W_x at zero the recurrence term of y vanishes: y = D * u (D acts on
+    the conv output, not on x_ssm) and y_ssm = D * u * SiLU(z), whatever A, delta and B are."""
+    s = _small.spec()
+    w = _small.weights(s, seed=11)
+    R, N = s.dt_rank, s.d_state
+    w_x = w["w_x"].copy()
+    w_x[R + N:R + 2 * N] = 0.0
+    w0 = dict(w, w_x=w_x)
+    x = _small.x_tilde(s, 14, seed=3)
+    r0 = O.layer_prefill(x, w0, s)
+    T, E = r0["u"].shape
+    for t in range(T):
+        for c in range(E):
+            want_y = w["d_skip"][c] * r0["u"][t, c]
+            assert abs(r0["y"][t, c] - want_y) <= 1e-13 * (1 + abs(want_y))
+            want = want_y * _silu_scalar(r0["z"][t, c])
+            assert abs(r0["y_ssm"][t, c] - want) <= 1e-13 * (1 + abs(want))
+    # the recurrence inputs no longer matter
+    w_x2 = w_x.copy()
+    w_x2[:R + N] *= -2.5
+    w1 = dict(w0, w_x=w_x2, a_log=w["a_log"][::-1].copy(), b_dt=w["b_dt"] + 1.0, w_dt=-w["w_dt"])
+    np.testing.assert_allclose(O.layer_prefill(x, w1, s)["y_ssm"], r0["y_ssm"], rtol=1e-13, atol=1e-14)
+
+
+def test_delta_with_zero_W_dt_is_softplus_of_the_bias():
+    """delta = softplus(delta_r W_dt^T + b_dt): with W_dt = 0 every row is softplus(b_dt)."""
+    s = _small.spec()
+    w = dict(_small.weights(s, seed=12), w_dt=np.zeros((s.d_inner, s.dt_rank)))
+    r = O.layer_prefill(_small.x_tilde(s, 9), w, s)
+    for c in range(s.d_inner):
+        want = _softplus_scalar(w["b_dt"][c])
+        assert np.all(np.abs(r["delta"][:, c] - want) <= 1e-14 * want)
+
+
+def test_full_rank_delta_of_the_conv_output():
+    """R = E with W_x[:R] = I and W_dt = I: delta = softplus(u + b_dt) elementwise, so delta is
+    driven by the conv + SiLU output u (not by x_ssm), through W_x first and W_dt second."""
+    E = 16
+    s = _small.spec(E=E, R=E)
+    w = _small.weights(s, seed=13)
+    w_x = w["w_x"].copy()
+    w_x[:E] = np.eye(E)
+    w = dict(w, w_x=w_x, w_dt=np.eye(E))
+    r = O.layer_prefill(_small.x_tilde(s, 11), w, s)
+    T = r["u"].shape[0]
+    for t in range(T):
+        for c in range(E):
+            want = _softplus_scalar(r["u"][t, c] + w["b_dt"][c])
+            assert abs(r["delta"][t, c] - want) <= 1e-14 * (1 + want)
+
+
 # --- P6: a KV-sharing consumer equals recomputation with the producer's K/V -------------------
 
 def test_p6_kv_shared_consumer_equals_recompute():
