@@ -166,3 +166,46 @@ def test_mask_bitmap_rejects_bad_shape():
         hy.hymba_debug_mask_bitmap(0, 0, 4, False, 1 << 44)
     with pytest.raises(hy.HymbaError):
         hy.hymba_debug_mask_bitmap(10, 0, 0, False, 1 << 44)
+
+
+def _c_kind(decl: str) -> str:
+    decl = decl.strip()
+    if "*" in decl or decl.startswith("hymba_stream_t"):
+        return "ptr"
+    if decl.startswith("int64_t"):
+        return "i64"
+    if decl.startswith("size_t"):
+        return "size"
+    if decl.startswith("int") or decl.startswith("hymba_status"):
+        return "int"
+    raise AssertionError(f"unclassified parameter {decl!r}")
+
+
+def _ctypes_kind(t) -> str:
+    import ctypes as C
+    if t in (C.c_void_p, C.c_char_p) or (isinstance(t, type) and issubclass(t, C._Pointer)):
+        return "ptr"
+    if t is C.c_int64:
+        return "i64"
+    if t is C.c_size_t:
+        return "size"
+    if t is C.c_int:
+        return "int"
+    raise AssertionError(f"unclassified ctypes type {t!r}")
+
+
+def test_binding_signatures_match_the_header():
+    """Every declaration's parameter list (count and kind: pointer, int, int64, size_t) and
+    return kind agree with the argument types the binding gives ctypes."""
+    import ctypes as C
+    from hybrid_attention_ssm_head_b200 import _abi
+    src = open(os.path.join(ROOT, "include", "hymba.h")).read()
+    decls = re.findall(r"HYMBA_API\s+([\w\s\*]+?)\b(hymba_\w+)\s*\(([^)]*)\)\s*;", src)
+    assert len(decls) == len(_abi._SIGS)
+    for ret, name, params in decls:
+        res, args = _abi._SIGS[name]
+        plist = [p for p in params.split(",") if p.strip() and p.strip() != "void"]
+        assert [_c_kind(p) for p in plist] == [_ctypes_kind(a) for a in args], name
+        ret = ret.strip()
+        want = {"hymba_status": C.c_int, "int": C.c_int, "void": None, "const char *": C.c_char_p}[ret]
+        assert res is want, name
