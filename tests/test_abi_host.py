@@ -209,3 +209,43 @@ def test_binding_signatures_match_the_header():
         ret = ret.strip()
         want = {"hymba_status": C.c_int, "int": C.c_int, "void": None, "const char *": C.c_char_p}[ret]
         assert res is want, name
+
+
+@pytest.mark.parametrize("kw", [
+    dict(),
+    dict(dtype="f32"),
+    dict(is_global=True),
+    dict(d_model=256, n_heads=4, n_kv_heads=2, d_inner=512, dt_rank=16, n_meta=16, window=64),
+    dict(d_model=256, n_heads=4, n_kv_heads=2, d_inner=512, dt_rank=16, n_meta=0, window=64, dtype="f32"),
+])
+def test_prefill_workspace_holds_every_documented_intermediate(kw):
+    """The workspace layout gives each intermediate the [M, width] extent the header documents,
+    256-byte aligned and in order without overlap, for producers and consumers of either dtype;
+    an empty sequence is refused."""
+    cfg = _cfg(**kw)
+    es = 4 if kw.get("dtype") == "f32" else 2
+    E, N, R = cfg.d_inner, cfg.d_state, cfg.dt_rank
+    for consumer in (False, True):
+        h = hy.hymba_layer_create(cfg, _fake_weights())
+        prod = hy.hymba_layer_create(cfg, _fake_weights(1 << 41)) if consumer else None
+        if consumer:
+            hy.hymba_kv_share_bind(h, prod)
+        for B, n in [(1, 1), (3, 127), (2, 300), (128, 8192)]:
+            if cfg.n_meta + n < 1:
+                continue
+            M = B * (cfg.n_meta + n)
+            lay = hy.hymba_layer_prefill_layout(h, B, n)
+            assert lay.total == hy.hymba_layer_prefill_workspace(h, B, n)
+            regions = [(lay.q, M * cfg.n_heads * cfg.head_dim_qk * es), (lay.x_ssm, M * E * es),
+                       (lay.z, M * E * es), (lay.u, M * E * es), (lay.xdbl, M * (R + 2 * N) * 4),
+                       (lay.delta, M * E * es), (lay.y_ssm, M * E * es), (lay.o_attn, M * E * es),
+                       (lay.fused, M * E * es)]
+            for (o, size), (o_next, _) in zip(regions, regions[1:] + [(lay.total, 0)]):
+                assert o % 256 == 0 and o + size <= o_next, (kw, consumer, B, n)
+        if cfg.n_meta == 0:
+            with pytest.raises(hy.HymbaError) as e:
+                hy.hymba_layer_prefill_layout(h, 1, 0)
+            assert e.value.status == hy.HYMBA_ERR_INVALID_ARG
+        hy.hymba_layer_destroy(h)
+        if prod:
+            hy.hymba_layer_destroy(prod)
