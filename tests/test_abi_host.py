@@ -249,3 +249,21 @@ def test_prefill_workspace_holds_every_documented_intermediate(kw):
         hy.hymba_layer_destroy(h)
         if prod:
             hy.hymba_layer_destroy(prod)
+
+
+@pytest.mark.parametrize("glob", [False, True])
+def test_decode_workspace_never_shrinks_as_the_position_grows(glob):
+    """A workspace sized for max_pos serves every earlier step: the size is non-decreasing in
+    the position, and constant for a sliding-window layer once the window is full."""
+    h = hy.hymba_layer_create(_cfg(is_global=glob), _fake_weights())
+    sizes = [hy.hymba_layer_decode_workspace(h, 128, p) for p in range(128, 128 + 20000, 97)]
+    assert all(a <= b for a, b in zip(sizes, sizes[1:]))
+    if glob:
+        assert sizes[-1] > sizes[0]
+    else:
+        tail = [hy.hymba_layer_decode_workspace(h, 128, p) for p in range(128 + 1024, 128 + 9000, 331)]
+        assert len(set(tail)) == 1
+    with pytest.raises(hy.HymbaError) as e:
+        hy.hymba_layer_decode_workspace(h, 128, 127)   # a meta position
+    assert e.value.status == hy.HYMBA_ERR_INVALID_ARG
+    hy.hymba_layer_destroy(h)
