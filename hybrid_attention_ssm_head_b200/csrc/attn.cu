@@ -522,22 +522,20 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
 
 static hymba_status attention_prefill_tc(const AttnArgs &a, cudaStream_t s) {
   using namespace fa;
-  static unsigned attr_set = 0;
+  static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(attr_set & (1u << (dev & 31)))) {
+  if (!attr_set.done(dev)) {
     if (cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
         cudaSuccess) {
       set_error("cudaFuncSetAttribute(attention smem) failed");
       return HYMBA_ERR_CUDA;
     }
-    attr_set |= 1u << (dev & 31);
+    attr_set.mark(dev);
   }
-  static int sms = 0;
-  if (sms == 0) {
-    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (sms <= 0) sms = 148;
-  }
+  int sms = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
   CUtensorMap tq, tk, tv, to;
   const uint64_t dq[3] = {(uint64_t)a.H * 64, (uint64_t)a.L, (uint64_t)a.B};
   const uint64_t sq[2] = {(uint64_t)a.H * 64 * 2, (uint64_t)a.L * a.H * 64 * 2};
@@ -1184,25 +1182,25 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
   const int esz = dt == HYMBA_BF16 ? 2 : 4;
   const int dsmem = DEC_CHUNK * (a.dqk + a.dv) * esz;
   {
-    static unsigned attr_set = 0;  // one bit per device
+    static DeviceOnce attr_set;
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!(attr_set & (1u << (dev & 31)))) {
+    if (!attr_set.done(dev)) {
       const int most = DEC_CHUNK * (128 + 256) * 4;
       cudaFuncSetAttribute(attn_decode_partial_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
       cudaFuncSetAttribute(attn_decode_partial_kernel<__nv_bfloat16>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, most);
-      attr_set |= 1u << (dev & 31);
+      attr_set.mark(dev);
     }
   }
   if (dt == HYMBA_BF16 && a.dqk == 64 && a.dv == 128) {
-    static unsigned attr_tc = 0;
+    static DeviceOnce attr_tc;
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!(attr_tc & (1u << (dev & 31)))) {
+    if (!attr_tc.done(dev)) {
       cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            dtc::smem_bytes(dtc::MAXREP));
-      attr_tc |= 1u << (dev & 31);
+      attr_tc.mark(dev);
     }
     CUtensorMap tk, tv;
     const uint64_t dk[3] = {64, (uint64_t)a.cap, (uint64_t)a.B * a.Hkv};
@@ -1213,11 +1211,9 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
     if (!make_tmap(&tk, a.k_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dk, sk, box)) return HYMBA_ERR_CUDA;
     if (!make_tmap(&tv, a.v_cache, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dvv, svv, box)) return HYMBA_ERR_CUDA;
     // equal contiguous ranges of the (sequence, kv head, chunk) items, two CTAs per SM
-    static int sms = 0;
-    if (sms == 0) {
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-      if (sms <= 0) sms = 148;
-    }
+    int sms = 0;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
     const int nchunks = (int)((nslots + dtc::SLOTS - 1) / dtc::SLOTS);
     const long long n_items = (long long)a.B * a.Hkv * nchunks;
     const long long grid_tc = std::min<long long>(n_items, (long long)dtc::CTAS_PER_SM * sms);

@@ -417,30 +417,27 @@ __global__ void __launch_bounds__(576, 1)
   }
 }
 
+// SM count of the current device (queried per launch: devices may differ between calls)
 static int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
 }
 
 template <int BN, int ELEM>
 static hymba_status launch_tc(const GemmArgs &g, cudaStream_t s) {
   using C = TcCfg<BN, ELEM>;
-  static unsigned attr_set = 0;  // one bit per device
+  static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(attr_set & (1u << (dev & 31)))) {
+  if (!attr_set.done(dev)) {
     if (cudaFuncSetAttribute(gemm_tc_kernel<BN, ELEM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM) != cudaSuccess) {
       set_error("cudaFuncSetAttribute(gemm smem %d) failed", C::SMEM);
       return HYMBA_ERR_CUDA;
     }
-    attr_set |= 1u << (dev & 31);
+    attr_set.mark(dev);
   }
   CUtensorMapDataType dt = ELEM == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   CUtensorMap ta, tb;

@@ -5,9 +5,20 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "hymba.h"
 
 namespace hymba {
+
+// One bit per device (ordinal mod 32), set once a kernel's launch attributes have been
+// configured on that device.  Atomic, so that first launches from several host threads at
+// once are well defined: each may then set the (idempotent) attribute.
+struct DeviceOnce {
+  std::atomic<unsigned> bits{0};
+  bool done(int dev) const { return bits.load(std::memory_order_acquire) & (1u << (dev & 31)); }
+  void mark(int dev) { bits.fetch_or(1u << (dev & 31), std::memory_order_acq_rel); }
+};
 
 
 // Where a GEMM output column goes.  Column c in [col0, col1) of the product is

@@ -509,13 +509,13 @@ static hymba_status decode_ssm_t(const DecodeSsmArgs &a, cudaStream_t s) {
     set_error("decode SSM: dt_rank %d too large for the fused decode kernels", a.R);
     return HYMBA_ERR_UNSUPPORTED;
   }
-  static unsigned attr_set = 0;  // one bit per device
+  static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (!(attr_set & (1u << (dev & 31)))) {
+  if (!attr_set.done(dev)) {
     cudaFuncSetAttribute(dec_conv_xproj_kernel<T, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     cudaFuncSetAttribute(dec_dt_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    attr_set |= 1u << (dev & 31);
+    attr_set.mark(dev);
   }
   dim3 g1(a.E / CH, (a.B + kDecRows - 1) / kDecRows);
   dec_conv_xproj_kernel<T, CH><<<g1, 256, smem1, s>>>(a);
@@ -826,10 +826,10 @@ hymba_status selective_scan(const ScanArgs &a, hymba_dtype dt, cudaStream_t s) {
     dsum = hstart + st;
   }
   {
-    static unsigned attr_set = 0;  // one bit per device
+    static DeviceOnce attr_set;
     int dev = 0;
     cudaGetDevice(&dev);
-    if (!(attr_set & (1u << (dev & 31)))) {
+    if (!attr_set.done(dev)) {
       const int most = 2 * (3 * kScanTB * 128 * 4 + kScanTB * 2 * kStates * 4);
       scan_set_smem<float, 128, 0>(most);
       scan_set_smem<float, 64, 0>(most);
@@ -837,7 +837,7 @@ hymba_status selective_scan(const ScanArgs &a, hymba_dtype dt, cudaStream_t s) {
       scan_set_smem<__nv_bfloat16, 128, kScanPolyStates>(most);
       scan_set_smem<__nv_bfloat16, 64, kScanPolyStates>(most);
       scan_set_smem<__nv_bfloat16, 32, kScanPolyStates>(most);
-      attr_set |= 1u << (dev & 31);
+      attr_set.mark(dev);
     }
   }
   auto launch = [&](int mode) {
