@@ -4,7 +4,10 @@
 One step = the whole hot path over one batch of synthetic input:
   * prefill of two consecutive sliding-window layers sharing one K/V (layer 2
     reuses layer 1's K/V), bf16, batch 128, 8192 real tokens + 128 meta tokens,
-    window 1024, 1.5B widths (d_model 1600, 25/5 heads, d_inner 3200, state 16);
+    window 1024, 1.5B widths (d_model 1600, 25/5 heads, d_inner 3200, state 16):
+    the two layers' meta-token caches are computed (batch 1, the meta rows being the
+    same in every sequence), then the real rows of both layers are prefilled from them;
+    the same prefill without the meta cache is timed beside it for comparison;
   * one decode step of a 32-layer stack at the same widths, batch 128, 8k
     context: global attention in layers 0, 15, 31, window 1024 + 128 meta
     elsewhere, K/V shared by consecutive sliding-window layers, N(0,1) caches.
@@ -36,13 +39,12 @@ import torch  # noqa: E402
 METRIC = "hybrid-layer prefill tok/s @B=128,L=8k bf16 + decode tok/s; % of roofline"
 UNIT = "tok/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one in_proj launch: ncu dram__bytes_{read,write}.sum of the
-# in_proj launch of `bench.py --case b32` (36,864 rows: 152.7 MB + 627.8 MB, see
-# profiles/gemm_b32.md), scaled by rows to one producer launch of the headline prefill
-# (1,064,960 rows).  The algorithmic minimum is 22.5 GB (read X~ and W_in, write the
-# 8960 output columns), so the kernel re-reads nothing.
-IN_PROJ_TRAFFIC = (152.7e6 + 627.8e6) * 1064960 / 36864
-IN_PROJ_TRAFFIC_BASIS = "ncu b32 in_proj capture scaled by rows to one producer launch"
+# DRAM bytes (read + write) of one in_proj launch from an ncu capture of the current kernel
+# (dram__bytes_{read,write}.sum of the in_proj launch of `bench.py --case b32`), scaled by
+# rows to one producer launch of the headline prefill (B x n = 1,048,576 real rows); None
+# while the kernel has changed since the last capture.
+IN_PROJ_TRAFFIC = None
+IN_PROJ_TRAFFIC_BASIS = "no capture of the current kernel yet"
 
 
 def max_over_ranks(vals, device, world: int):
@@ -127,7 +129,9 @@ class ClockSampler:
 # our path
 # ---------------------------------------------------------------------------------------------
 class Prefill:
-    """The two KV-sharing prefill layers of the headline workload."""
+    """The two KV-sharing prefill layers of the headline workload.  A step computes the
+    two layers' meta-token caches (batch 1: the m meta rows are the same in every sequence,
+    Hymba §2.3) and then prefills the B x n real rows of both layers from them."""
 
     def __init__(self, w, dev):
         import hybrid_attention_ssm_head_b200 as hy
@@ -146,29 +150,73 @@ class Prefill:
             self.wts.append(wt)
             self.handles.append(hy.hymba_layer_create(cfg, hy.make_weights(wt)))
         hy.hymba_kv_share_bind(self.handles[1], self.handles[0])
-        self.x = synth.configs.x_tilde(w, device=dev)
+        m = w.n_meta
+        self.m = m
+        self.meta_x = synth.configs.meta_tokens(w, device=dev)          # R [m, d]
+        self.x = synth.configs.real_rows(w, device=dev).contiguous()     # X [B, n, d]
         self.y1 = torch.empty_like(self.x)
         self.y2 = torch.empty_like(self.x)
         self.k = torch.empty(B, L, d.n_kv_heads * d.head_dim_qk, dtype=torch.bfloat16, device=dev)
         self.v = torch.empty(B, L, d.n_kv_heads * d.head_dim_v, dtype=torch.bfloat16, device=dev)
         self.kv = hy.hymba_kv_seq(self.k.data_ptr(), self.v.data_ptr(), 0, 0, 0)
-        nb = max(hy.hymba_layer_prefill_workspace(h, B, n) for h in self.handles)
+        # meta caches of the two layers (the consumer's K/V are its producer's)
+        self.meta_bufs, self.metas = [], []
+        for layer in range(2):
+            bufs = dict(h=torch.empty(d.d_inner, d.d_state, dtype=torch.float32, device=dev),
+                        conv=torch.empty(d.d_conv - 1, d.d_inner, dtype=torch.bfloat16, device=dev),
+                        y=torch.empty(m, d.d_model, dtype=torch.bfloat16, device=dev))
+            if layer == 0:
+                bufs["k"] = torch.empty(m, d.n_kv_heads * d.head_dim_qk, dtype=torch.bfloat16, device=dev)
+                bufs["v"] = torch.empty(m, d.n_kv_heads * d.head_dim_v, dtype=torch.bfloat16, device=dev)
+            self.meta_bufs.append(bufs)
+            self.metas.append(hy.hymba_meta_cache(
+                bufs["k"].data_ptr() if layer == 0 else None, bufs["v"].data_ptr() if layer == 0 else None,
+                bufs["h"].data_ptr(), bufs["conv"].data_ptr(), bufs["y"].data_ptr(), 0))
+        nb = max(max(hy.hymba_layer_prefill_cached_workspace(h, B, n), hy.hymba_layer_meta_workspace(h))
+                 for h in self.handles)
         self.ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        self._full = None
 
     def run(self, stream, x=None, y=None):
+        """One step: both layers' meta caches, then both layers over the real rows."""
         hy = self.hy
         x = self.x if x is None else x
         y = self.y2 if y is None else y
-        hy.hymba_layer_prefill(self.handles[0], self.B, self.n, x, self.y1, self.kv, None, None,
-                               self.ws, self.ws.numel(), stream)
-        hy.hymba_layer_prefill(self.handles[1], self.B, self.n, self.y1, y, self.kv, None, None,
-                               self.ws, self.ws.numel(), stream)
+        hy.hymba_layer_meta_precompute(self.handles[0], self.meta_x, self.metas[0], None, self.ws,
+                                       self.ws.numel(), stream)
+        hy.hymba_layer_meta_precompute(self.handles[1], self.meta_bufs[0]["y"], self.metas[1], self.metas[0],
+                                       self.ws, self.ws.numel(), stream)
+        hy.hymba_layer_prefill_cached(self.handles[0], self.B, self.n, x, self.y1, self.metas[0], self.kv, None,
+                                      None, self.ws, self.ws.numel(), stream)
+        hy.hymba_layer_prefill_cached(self.handles[1], self.B, self.n, self.y1, y, self.metas[1], self.kv, None,
+                                      None, self.ws, self.ws.numel(), stream)
+
+    def run_full(self, stream):
+        """The same two layers without the meta cache: every sequence's L = m + n rows."""
+        hy = self.hy
+        if self._full is None:
+            import synth
+            xf = synth.configs.x_tilde(self.w, device=self.x.device)
+            nb = max(hy.hymba_layer_prefill_workspace(h, self.B, self.n) for h in self.handles)
+            self._full = dict(x=xf, y1=torch.empty_like(xf), y2=torch.empty_like(xf),
+                              ws=torch.empty(nb, dtype=torch.uint8, device=self.x.device))
+        f = self._full
+        hy.hymba_layer_prefill(self.handles[0], self.B, self.n, f["x"], f["y1"], self.kv, None, None,
+                               f["ws"], f["ws"].numel(), stream)
+        hy.hymba_layer_prefill(self.handles[1], self.B, self.n, f["y1"], f["y2"], self.kv, None, None,
+                               f["ws"], f["ws"].numel(), stream)
+
+    def release_full(self):
+        self._full = None
 
     def flops(self):
-        """Algorithmic FLOPs of one step (both layers), attention counted on visible pairs only."""
+        """Algorithmic FLOPs of one step (both layers): the meta rows once and the real rows of
+        every sequence; attention counted on visible pairs only."""
         d, w = self.w.dims, self.w
-        M = self.B * self.L
+        M = self.B * self.n + self.m
         E, H = d.d_inner, d.n_heads
+        meta_pairs = visible_pairs(self.m, w.n_meta, w.window, False)
+        real_pairs = visible_pairs(self.L, w.n_meta, w.window, False) - meta_pairs
         f = 0.0
         for consumer in (False, True):
             P = d.in_width(consumer)
@@ -176,13 +224,13 @@ class Prefill:
             f += 2.0 * M * d.xproj_width * E                   # x_proj
             f += 2.0 * M * E * d.rank                          # dt_proj
             f += 2.0 * M * d.d_model * E                       # out_proj
-            f += self.B * H * 2.0 * (d.head_dim_qk + d.head_dim_v) * visible_pairs(
-                self.L, w.n_meta, w.window, False)             # attention
+            f += H * 2.0 * (d.head_dim_qk + d.head_dim_v) * (self.B * real_pairs + meta_pairs)  # attention
         return f
 
     def in_proj_flops(self):
+        """Per launch over the real rows: [producer, consumer]."""
         d = self.w.dims
-        M = self.B * self.L
+        M = self.B * self.n
         return [2.0 * M * d.in_width(False) * d.d_model, 2.0 * M * d.in_width(True) * d.d_model]
 
 
@@ -274,6 +322,68 @@ class Decode:
         return tot
 
 
+MUFU_OPS_PER_CLK_SM = 16  # MUFU (ex2/rcp/lg2) results per clock per SM on sm_100
+SCAN_MUFU_PER_CHANNEL_STEP = 16  # the 16 decays exp2(delta A) (the gate SiLU(z) comes precomputed)
+
+
+def kernel_fractions(pre, dec, prof, dprof, peaks, sm_mhz, sms):
+    """Each hot kernel's achieved rate against its bound: algorithmic FLOPs (tensor-bound
+    kernels) or bytes (memory-bound kernels) over the CUDA-event time the library's
+    profiler measured for it inside the timed region.  The scan is also reported against
+    its MUFU floor (its 16 MUFU operations per channel-step at the sampled SM clock)."""
+    d, w = pre.w.dims, pre.w
+    B, L = pre.B, pre.L
+    M = B * pre.n  # the prefill's main launches run over the real rows (the meta rows are cached)
+    E, H, R, N = d.d_inner, d.n_heads, d.rank, d.d_state
+    hbm = peaks.get("hbm_gbs", 6650.0)
+    tens = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1400.0))
+    pm = {n: ms / c for n, c, _, ms in prof if c}
+    out = {}
+
+    def tensor(name, flops):
+        if name in pm:
+            a = flops / (pm[name] / 1e3) / 1e12
+            out[name] = {"bound": "tensor", "achieved": a, "peak": tens, "unit": "TFLOP/s", "frac": a / tens,
+                         "ms": pm[name]}
+
+    def mem(name, nbytes, table=None, extra=None):
+        t = (table or pm)
+        if name in t:
+            a = nbytes / (t[name] / 1e3) / 1e9
+            out[name] = {"bound": "hbm", "achieved": a, "peak": hbm, "unit": "GB/s", "frac": a / hbm,
+                         "ms": t[name]}
+            if extra:
+                out[name].update(extra)
+
+    fl_in = sum(pre.in_proj_flops()) / 2.0
+    tensor("in_proj", fl_in)
+    tensor("out_proj", 2.0 * M * d.d_model * E)
+    tensor("attention", B * H * 2.0 * (d.head_dim_qk + d.head_dim_v) *
+           (visible_pairs(L, w.n_meta, w.window, False) - visible_pairs(w.n_meta, w.n_meta, w.window, False)))
+    mem("conv", 2.0 * M * E * 2)
+    mem("x_proj", M * E * 2 + M * (R + 2 * N) * 4)
+    mem("dt_proj", M * (R + 2 * N) * 4 + M * E * 2)
+    mem("fuse", 3.0 * M * E * 2)
+    if "scan" in pm and sm_mhz:
+        floor_ms = M * E * SCAN_MUFU_PER_CHANNEL_STEP / (MUFU_OPS_PER_CLK_SM * sms * sm_mhz * 1e6) * 1e3
+        mem("scan", 4.0 * M * E * 2 + M * 2 * N * 4,
+            extra={"mufu_floor_ms": floor_ms, "mufu_frac": floor_ms / pm["scan"]})
+    # decode, per layer (the stack's 32 layers averaged)
+    dm = {n: ms / c for n, c, _, ms in dprof if c}
+    nl = len(dec.layers)
+    wbytes = lambda key: sum(e["wt"][key].numel() * e["wt"][key].element_size() for e in dec.layers) / nl  # noqa: E731
+    kv_bytes = 0
+    for e in dec.layers:
+        keys = dec.pos + 1 if e["is_global"] else dec.w.n_meta + dec.w.window
+        kv_bytes += dec.B * d.n_kv_heads * keys * (d.head_dim_qk + d.head_dim_v) * 2
+    mem("dec_in_proj", wbytes("w_in"), dm)
+    mem("dec_out_proj", wbytes("w_out"), dm)
+    mem("dec_attention", kv_bytes / nl, dm)
+    mem("dec_ssm", 2.0 * dec.B * E * N * 4 + wbytes("w_x") + wbytes("w_dt") + 2.0 * dec.B * (d.d_conv - 1) * E * 2,
+        dm)
+    return out
+
+
 def run_ours(args, rank, world, dev):
     import hybrid_attention_ssm_head_b200 as hy
     import synth
@@ -319,6 +429,18 @@ def run_ours(args, rank, world, dev):
     prof = hy.hymba_profile_collect()
     hy.hymba_profile_enable(False)
     clocks = sampler.stop() if rank == 0 else None
+    # for comparison: the same two layers without the meta cache (every sequence's m + n rows)
+    steps_full = max(1, min(args.steps, 3))
+    pre.run_full(stream)
+    torch.cuda.synchronize()
+    ef0, ef1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ef0.record(stream)
+    for _ in range(steps_full):
+        pre.run_full(stream)
+    ef1.record(stream)
+    torch.cuda.synchronize()
+    full_ms = max_over_ranks([ef0.elapsed_time(ef1) / steps_full], dev, world)[0]
+    pre.release_full()
     hy.hymba_stream_status(stream)
     pre_ms = sum(ev[2 * s].elapsed_time(ev[2 * s + 1]) for s in range(args.steps))
     dec_ms = sum(ev[2 * s + 1].elapsed_time(ev[2 * s + 2]) for s in range(args.steps))
@@ -373,7 +495,7 @@ def run_ours(args, rank, world, dev):
         ytd = torch.empty_like(dec.x)
         s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
         torch.cuda.synchronize()
-        steps_e2e = max(1, min(args.steps, 3))
+        steps_e2e = args.steps
         ev = lambda: torch.cuda.Event(enable_timing=False)  # noqa: E731
         in_ready = [ev(), ev()]
         done = [ev(), ev()]
@@ -420,6 +542,10 @@ def run_ours(args, rank, world, dev):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_sample()
 
+    sm_mhz = clocks.get("sm_mhz") if clocks else None
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    kernels = kernel_fractions(pre, dec, prof, dprof, peaks, sm_mhz, sms)
+
     if rank != 0:
         return None
     out = {
@@ -427,11 +553,13 @@ def run_ours(args, rank, world, dev):
         "warmup": args.warmup, "ms_per_step": tot_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "prefill: 2 KV-sharing SWA layers, B=128, 8192+128 meta rows, W=1024, "
-                               "1.5B widths; decode: 32-layer stack, B=128, 8k context",
+                               "1.5B widths, meta rows computed once per step (batch 1) and the "
+                               "real rows prefilled from them; decode: 32-layer stack, B=128, 8k context",
                    "prefill": w3.name, "decode": w4.name, "global_batch": w3.batch * world,
                    "seq_len": w3.seq_rows, "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (no flush)"},
         "prefill_ms_per_step": pre_ms / args.steps,
+        "prefill_without_meta_cache_ms_per_step": full_ms,
         "decode_ms_per_step": dec_ms / args.steps,
         "decode_tok_s": dec_tok_s,
         "prefill_tflops": step_flops * args.steps / (pre_ms / 1e3) / 1e12,
@@ -444,6 +572,7 @@ def run_ours(args, rank, world, dev):
                           for n, c, k, ms in prof},
         "decode_steps_profile": {n: {"calls": c, "kernels": k, "ms_per_call": ms / c if c else None}
                                  for n, c, k, ms in dprof},
+        "kernels": kernels,
         "gpu_launches": pre_launches + dec_kernels_per_step * args.steps,
         "clocks": clocks,
         "e2e": e2e,

@@ -28,7 +28,8 @@ class hymba_layer_config(C.Structure):
                 ("head_dim_qk", C.c_int), ("head_dim_v", C.c_int), ("d_inner", C.c_int),
                 ("d_state", C.c_int), ("d_conv", C.c_int), ("dt_rank", C.c_int),
                 ("n_meta", C.c_int), ("window", C.c_int), ("is_global", C.c_int),
-                ("dtype", C.c_int), ("rms_eps", C.c_float), ("softmax_scale", C.c_float)]
+                ("dtype", C.c_int), ("rms_eps", C.c_float), ("softmax_scale", C.c_float),
+                ("rope_base", C.c_float)]
 
 
 class hymba_layer_weights(C.Structure):
@@ -50,9 +51,14 @@ class hymba_ssm_cache(C.Structure):
     _fields_ = [("h", C.c_void_p), ("conv", C.c_void_p)]
 
 
+class hymba_meta_cache(C.Structure):
+    _fields_ = [("k", C.c_void_p), ("v", C.c_void_p), ("h", C.c_void_p), ("conv", C.c_void_p),
+                ("y", C.c_void_p), ("owner", C.c_uint64)]
+
+
 class hymba_prefill_layout(C.Structure):
-    _fields_ = [(n, C.c_size_t) for n in ("q", "x_ssm", "z", "u", "xdbl", "delta", "y_ssm",
-                                          "o_attn", "fused", "total")]
+    _fields_ = [(n, C.c_size_t) for n in ("q", "x_ssm", "gate", "u", "xdbl", "delta", "y_ssm",
+                                          "o_attn", "fused", "rope", "total")]
 
 
 class hymba_profile_entry(C.Structure):
@@ -81,6 +87,16 @@ _SIGS = {
     "hymba_layer_prefill": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p,
                                       C.POINTER(hymba_kv_seq), C.POINTER(hymba_kv_cache),
                                       C.POINTER(hymba_ssm_cache), C.c_void_p, C.c_size_t, C.c_void_p]),
+    "hymba_layer_meta_workspace": (C.c_int, [C.c_void_p, C.POINTER(C.c_size_t)]),
+    "hymba_layer_meta_precompute": (C.c_int, [C.c_void_p, C.c_void_p, C.POINTER(hymba_meta_cache),
+                                              C.POINTER(hymba_meta_cache), C.c_void_p, C.c_size_t,
+                                              C.c_void_p]),
+    "hymba_layer_prefill_cached_workspace": (C.c_int, [C.c_void_p, C.c_int, C.c_int,
+                                                       C.POINTER(C.c_size_t)]),
+    "hymba_layer_prefill_cached": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_void_p, C.c_void_p,
+                                             C.POINTER(hymba_meta_cache), C.POINTER(hymba_kv_seq),
+                                             C.POINTER(hymba_kv_cache), C.POINTER(hymba_ssm_cache),
+                                             C.c_void_p, C.c_size_t, C.c_void_p]),
     "hymba_layer_decode_workspace": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.POINTER(C.c_size_t)]),
     "hymba_layer_decode_step": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_void_p, C.c_void_p,
                                           C.POINTER(hymba_kv_cache), C.POINTER(hymba_ssm_cache),
@@ -89,11 +105,16 @@ _SIGS = {
     "hymba_last_error": (C.c_char_p, []),
     "hymba_status_string": (C.c_char_p, [C.c_int]),
     "hymba_version": (C.c_char_p, []),
-    "hymba_debug_mask_bitmap": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_void_p,
+    "hymba_debug_mask_bitmap": (C.c_int, [C.c_int, C.c_int, C.c_int, C.c_int, C.c_int, C.c_void_p,
                                           C.c_void_p, C.c_void_p]),
+    "hymba_debug_decode_mask": (C.c_int, [C.c_int64, C.c_int, C.c_int, C.c_int, C.c_int, C.c_void_p,
+                                          C.c_void_p]),
+    "hymba_debug_exp2_poly": (C.c_int, [C.c_int, C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p]),
     "hymba_layer_decode_step_static": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_void_p, C.c_void_p,
                                                  C.POINTER(hymba_kv_cache), C.POINTER(hymba_ssm_cache),
                                                  C.c_void_p]),
+    "hymba_set_wait_limit": (C.c_int, [C.c_int64, C.POINTER(C.c_int64)]),
+    "hymba_debug_stall_next_prefill": (C.c_int, [C.c_int]),
     "hymba_profile_enable": (C.c_int, [C.c_int]),
     "hymba_profile_collect": (C.c_int, [C.POINTER(hymba_profile_entry), C.c_int, C.POINTER(C.c_int)]),
 }
@@ -183,6 +204,38 @@ def hymba_layer_prefill(layer: int, batch: int, n_tokens: int, x, y, kv: hymba_k
         _ptr(workspace), workspace_bytes, _stream(stream)), "hymba_layer_prefill")
 
 
+def hymba_layer_meta_workspace(layer: int) -> int:
+    out = C.c_size_t()
+    check(lib().hymba_layer_meta_workspace(layer, C.byref(out)), "hymba_layer_meta_workspace")
+    return out.value
+
+
+def hymba_layer_meta_precompute(layer: int, x_meta, meta: hymba_meta_cache,
+                                producer_meta: hymba_meta_cache | None, workspace, workspace_bytes: int,
+                                stream=None) -> None:
+    check(lib().hymba_layer_meta_precompute(
+        layer, _ptr(x_meta), C.byref(meta), C.byref(producer_meta) if producer_meta is not None else None,
+        _ptr(workspace), workspace_bytes, _stream(stream)), "hymba_layer_meta_precompute")
+
+
+def hymba_layer_prefill_cached_workspace(layer: int, batch: int, n_tokens: int) -> int:
+    out = C.c_size_t()
+    check(lib().hymba_layer_prefill_cached_workspace(layer, batch, n_tokens, C.byref(out)),
+          "hymba_layer_prefill_cached_workspace")
+    return out.value
+
+
+def hymba_layer_prefill_cached(layer: int, batch: int, n_tokens: int, x, y, meta: hymba_meta_cache,
+                               kv: hymba_kv_seq, kv_cache: hymba_kv_cache | None,
+                               ssm_cache: hymba_ssm_cache | None, workspace, workspace_bytes: int,
+                               stream=None) -> None:
+    check(lib().hymba_layer_prefill_cached(
+        layer, batch, n_tokens, _ptr(x), _ptr(y), C.byref(meta), C.byref(kv),
+        C.byref(kv_cache) if kv_cache is not None else None,
+        C.byref(ssm_cache) if ssm_cache is not None else None,
+        _ptr(workspace), workspace_bytes, _stream(stream)), "hymba_layer_prefill_cached")
+
+
 def hymba_layer_decode_workspace(layer: int, batch: int, max_pos: int) -> int:
     out = C.c_size_t()
     check(lib().hymba_layer_decode_workspace(layer, batch, max_pos, C.byref(out)),
@@ -227,9 +280,31 @@ def hymba_version() -> str:
 
 
 def hymba_debug_mask_bitmap(L: int, n_meta: int, window: int, is_global: bool, bits,
-                            tile_class=None, stream=None) -> None:
-    check(lib().hymba_debug_mask_bitmap(L, n_meta, window, int(is_global), _ptr(bits),
+                            tile_class=None, stream=None, path: int = 0) -> None:
+    check(lib().hymba_debug_mask_bitmap(L, n_meta, window, int(is_global), path, _ptr(bits),
                                         _ptr(tile_class), _stream(stream)), "hymba_debug_mask_bitmap")
+
+
+def hymba_debug_decode_mask(pos: int, n_meta: int, window: int, is_global: bool, capacity: int, bits,
+                            stream=None) -> None:
+    check(lib().hymba_debug_decode_mask(pos, n_meta, window, int(is_global), capacity, _ptr(bits),
+                                        _stream(stream)), "hymba_debug_decode_mask")
+
+
+def hymba_debug_exp2_poly(degree: int, x, y, n: int, stream=None) -> None:
+    check(lib().hymba_debug_exp2_poly(degree, _ptr(x), _ptr(y), n, _stream(stream)),
+          "hymba_debug_exp2_poly")
+
+
+def hymba_set_wait_limit(cycles: int) -> int:
+    """Sets the bounded-wait limit (0: default); returns the limit now in force."""
+    out = C.c_int64()
+    check(lib().hymba_set_wait_limit(cycles, C.byref(out)), "hymba_set_wait_limit")
+    return out.value
+
+
+def hymba_debug_stall_next_prefill(count: int) -> None:
+    check(lib().hymba_debug_stall_next_prefill(count), "hymba_debug_stall_next_prefill")
 
 
 def hymba_profile_enable(on: bool) -> None:
@@ -248,11 +323,11 @@ def hymba_profile_collect(max_entries: int = 64) -> list[tuple[str, int, int, fl
 # ---- marshalling helpers ---------------------------------------------------------------
 
 def make_config(d_model, n_heads, n_kv_heads, head_dim_qk, d_inner, d_state, d_conv, dt_rank,
-                n_meta, window, is_global, dtype: str, rms_eps=1e-6, softmax_scale=0.0):
+                n_meta, window, is_global, dtype: str, rms_eps=1e-6, softmax_scale=0.0, rope_base=0.0):
     return hymba_layer_config(d_model, n_heads, n_kv_heads, head_dim_qk, d_inner // n_heads, d_inner,
                               d_state, d_conv, dt_rank, n_meta, window if not is_global else 0,
                               int(bool(is_global)), HYMBA_BF16 if dtype == "bf16" else HYMBA_F32,
-                              rms_eps, softmax_scale)
+                              rms_eps, softmax_scale, rope_base)
 
 
 def make_weights(w: dict) -> hymba_layer_weights:

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -21,6 +22,30 @@ static thread_local char g_msg[512] = "";
 
 static std::atomic<unsigned long long> g_launches{0};
 void note_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
+
+constexpr long long kDefaultWaitLimit = 1000000000LL;  // ~0.5 s at 2 GHz
+constexpr long long kMinWaitLimit = 100000LL;
+static std::atomic<long long> g_wait_limit{0};  // 0: not set through the ABI
+static long long env_wait_limit() {
+  static const long long v = [] {
+    const char *e = getenv("HYMBA_WAIT_LIMIT");
+    return e ? atoll(e) : 0LL;
+  }();
+  return v;
+}
+long long wait_limit_cycles() {
+  long long v = g_wait_limit.load(std::memory_order_relaxed);
+  if (v <= 0) v = env_wait_limit();
+  if (v <= 0) v = kDefaultWaitLimit;
+  return std::max(v, kMinWaitLimit);
+}
+static std::atomic<int> g_stall{0};
+int take_debug_stall() {
+  int v = g_stall.load();
+  while (v > 0 && !g_stall.compare_exchange_weak(v, v - 1)) {
+  }
+  return v > 0 ? 1 : 0;
+}
 
 void set_error(const char *fmt, ...) {
   va_list ap;
@@ -152,6 +177,9 @@ hymba_status hymba_layer_create(const hymba_layer_config *cfg, const hymba_layer
   if (c.n_meta < 0) FAIL(HYMBA_ERR_INVALID_ARG, "n_meta < 0");
   if (!c.is_global && c.window < 1) FAIL(HYMBA_ERR_INVALID_ARG, "window < 1 on a sliding-window layer");
   if (!(c.rms_eps >= 0.f) || !(c.softmax_scale >= 0.f)) FAIL(HYMBA_ERR_INVALID_ARG, "eps/scale < 0");
+  if (!(c.rope_base >= 0.f) || !std::isfinite(c.rope_base)) FAIL(HYMBA_ERR_INVALID_ARG, "rope_base < 0");
+  if (c.rope_base > 0.f && (c.rope_base <= 1.f || (c.head_dim_qk & (c.head_dim_qk - 1)) || c.head_dim_qk < 2))
+    FAIL(HYMBA_ERR_UNSUPPORTED, "rotary embedding needs a base > 1 and a power-of-two head_dim_qk");
   if (c.d_state != 16) FAIL(HYMBA_ERR_UNSUPPORTED, "d_state must be 16");
   if (c.d_conv > 4) FAIL(HYMBA_ERR_UNSUPPORTED, "d_conv must be <= 4");
   if (c.dt_rank % 4) FAIL(HYMBA_ERR_UNSUPPORTED, "dt_rank must be a multiple of 4 (16-byte rows of W_dt)");
@@ -196,9 +224,10 @@ hymba_status hymba_kv_share_bind(hymba_layer *consumer, const hymba_layer *produ
   const hymba_layer_config &c = consumer->cfg, &p = producer->cfg;
   if (c.n_kv_heads != p.n_kv_heads || c.head_dim_qk != p.head_dim_qk ||
       c.head_dim_v != p.head_dim_v || c.n_meta != p.n_meta || c.is_global != p.is_global ||
-      (!c.is_global && c.window != p.window) || c.dtype != p.dtype || c.n_heads != p.n_heads)
+      (!c.is_global && c.window != p.window) || c.dtype != p.dtype || c.n_heads != p.n_heads ||
+      c.rope_base != p.rope_base)
     FAIL(HYMBA_ERR_NOT_BOUND, "producer and consumer differ in heads, head dims, n_meta, window, "
-                              "global flag or dtype");
+                              "global flag, dtype or rotary base");
   consumer->producer = producer;
   consumer->producer_id = producer->id;
   return HYMBA_OK;
@@ -207,15 +236,16 @@ hymba_status hymba_kv_share_bind(hymba_layer *consumer, const hymba_layer *produ
 // ---------------------------------------------------------------------------
 // prefill
 // ---------------------------------------------------------------------------
-static hymba_status prefill_layout(const hymba_layer *layer, int batch, int n_tokens,
-                                   hymba_prefill_layout *o, size_t *scan_floats) {
+// Workspace of a prefill whose intermediates have `rows` rows per sequence: all L = m + n
+// rows, or the n real rows when the meta rows come from a precomputed meta cache.
+static hymba_status prefill_layout_rows(const hymba_layer *layer, int batch, long long rows,
+                                        hymba_prefill_layout *o, size_t *scan_floats) {
   if (!layer) FAIL(HYMBA_ERR_INVALID_ARG, "null layer");
-  if (batch < 1 || n_tokens < 0) FAIL(HYMBA_ERR_INVALID_ARG, "batch < 1 or n_tokens < 0");
+  if (batch < 1) FAIL(HYMBA_ERR_INVALID_ARG, "batch < 1");
   const hymba_layer_config &c = layer->cfg;
-  const long long L = (long long)c.n_meta + n_tokens;
-  if (L < 1) FAIL(HYMBA_ERR_INVALID_ARG, "a sequence needs at least one row");
-  if (L > (1LL << 30)) FAIL(HYMBA_ERR_UNSUPPORTED, "sequence too long");
-  const size_t M = (size_t)batch * L, es = esize(c.dtype), E = c.d_inner;
+  if (rows < 1) FAIL(HYMBA_ERR_INVALID_ARG, "a sequence needs at least one row");
+  if (rows + c.n_meta > (1LL << 30)) FAIL(HYMBA_ERR_UNSUPPORTED, "sequence too long");
+  const size_t M = (size_t)batch * rows, es = esize(c.dtype), E = c.d_inner;
   size_t off = 0;
   auto take = [&](size_t bytes) {
     size_t at = off;
@@ -224,18 +254,27 @@ static hymba_status prefill_layout(const hymba_layer *layer, int batch, int n_to
   };
   o->q = take(M * qk_width(c) * es);
   o->x_ssm = take(M * E * es);
-  o->z = take(M * E * es);
+  o->gate = take(M * E * es);
   o->u = take(M * E * es);
   o->xdbl = take(M * xdbl_width(c) * 4);
   o->delta = take(M * E * es);
   o->y_ssm = take(M * E * es);
   o->o_attn = take(M * E * es);
   o->fused = take(M * E * es);
-  size_t sf = scan_workspace_floats(batch, (int)L, c.d_inner, c.d_state, nullptr);
+  size_t sf = scan_workspace_floats(batch, (int)rows, c.d_inner, c.d_state, nullptr);
   if (scan_floats) *scan_floats = sf;
   take(sf * 4);  // scan chunk states, after `fused`
+  // rotary table of the positions 0..L-1 (none without a rotary embedding)
+  o->rope = take(c.rope_base > 0.f ? (size_t)(rows + c.n_meta) * (c.head_dim_qk / 2) * 8 : 0);
   o->total = off;
   return HYMBA_OK;
+}
+
+static hymba_status prefill_layout(const hymba_layer *layer, int batch, int n_tokens,
+                                   hymba_prefill_layout *o, size_t *scan_floats) {
+  if (!layer) FAIL(HYMBA_ERR_INVALID_ARG, "null layer");
+  if (n_tokens < 0) FAIL(HYMBA_ERR_INVALID_ARG, "n_tokens < 0");
+  return prefill_layout_rows(layer, batch, (long long)layer->cfg.n_meta + n_tokens, o, scan_floats);
 }
 
 hymba_status hymba_layer_prefill_layout(const hymba_layer *layer, int batch, int n_tokens,
@@ -258,7 +297,7 @@ hymba_status hymba_layer_prefill_workspace(const hymba_layer *layer, int batch, 
 
 static EpiSeg seg(void *ptr, long long ld_row, int col0, int col1, int f32, size_t es,
                   long long ld_group = 0, int inner = 0) {
-  EpiSeg s;
+  EpiSeg s{};
   s.ptr = ptr;
   s.ld_row = ld_row;
   s.col0 = col0;
@@ -278,8 +317,13 @@ static hymba_status gemm(const GemmArgs &g, hymba_dtype dt, cudaStream_t s) {
   if (dt == HYMBA_BF16) return gemm_tc(g, s);
   return gemm_simt_f32(g, s);
 }
+// The decode step's projections: a few activation rows against a whole weight matrix.
+static hymba_status gemm_decode(const GemmArgs &g, hymba_dtype dt, cudaStream_t s) {
+  if (dt == HYMBA_BF16 && g.M <= 256) return gemm_ws(g, s);
+  return gemm(g, dt, s);
+}
 
-// in_proj: one GEMM, columns routed to Q, (K, V), x_ssm, z.
+// in_proj: one GEMM, columns routed to Q, (K, V), x_ssm and the gate SiLU(z).
 static Epilogue in_proj_epilogue(const hymba_layer_config &c, bool consumer, void *q, long long ldq,
                                  void *k, void *v, long long ld_k_row, long long ld_v_row,
                                  long long k_group, long long v_group, void *xs, void *z,
@@ -298,65 +342,58 @@ static Epilogue in_proj_epilogue(const hymba_layer_config &c, bool consumer, voi
   }
   e.seg[n++] = seg(xs, ld_e, col, col + c.d_inner, f32, es);
   col += c.d_inner;
-  e.seg[n++] = seg(z, ld_e, col, col + c.d_inner, f32, es);
+  // the gate's SiLU is applied here, so the scan multiplies by a stored SiLU(z)
+  e.seg[n] = seg(z, ld_e, col, col + c.d_inner, f32, es);
+  e.seg[n++].act = 2;
   e.nseg = n;
   return e;
 }
 
-hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, const void *x, void *y,
-                                 hymba_kv_seq *kv, hymba_kv_cache *kv_cache,
-                                 hymba_ssm_cache *ssm_cache, void *workspace, size_t workspace_bytes,
-                                 hymba_stream_t stream_) {
-  g_msg[0] = 0;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
-  hymba_prefill_layout lay;
-  size_t scan_floats = 0;
-  hymba_status st = prefill_layout(layer, batch, n_tokens, &lay, &scan_floats);
-  if (st != HYMBA_OK) return st;
+// The launch sequence of one prefill over `rows` rows per sequence whose first row is X~
+// position q_off: the whole sequence (q_off = 0, rows = L), or its real rows after a
+// precomputed meta cache (q_off = m, rows = n; the meta rows' K/V are then in kv already,
+// and their SSM state and conv history come from `meta`).  Arguments validated.
+struct PrefillRun {
+  const void *x;  // [B, rows, d]
+  void *y;        // [B, rows, d]
+  int rows, q_off;
+  const float *h0;    // broadcast initial SSM state [E, N] or null
+  const void *conv0;  // broadcast conv history [K-1, E] or null
+  bool meta;          // the meta-cache precompute: its steps are profiled under "meta_*" names
+};
+// Profiler step name of a prefill step (the meta-cache precompute has its own names).
+static const char *step_name(const PrefillRun &r, int step) {
+  static const char *const names[2][9] = {
+      {"in_proj", "conv", "x_proj", "dt_proj", "scan", "attention", "fuse", "out_proj", "kv_emit"},
+      {"meta_in_proj", "meta_conv", "meta_x_proj", "meta_dt_proj", "meta_scan", "meta_attention",
+       "meta_fuse", "meta_out_proj", "meta_kv_emit"}};
+  return names[r.meta ? 1 : 0][step];
+}
+
+static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun &r, hymba_kv_seq *kv,
+                                hymba_kv_cache *kv_cache, hymba_ssm_cache *ssm_cache, void *workspace,
+                                const hymba_prefill_layout &lay, cudaStream_t stream) {
   const hymba_layer_config &c = layer->cfg;
   const bool consumer = layer->producer != nullptr;
-  const int L = c.n_meta + n_tokens;
-  const long long M = (long long)batch * L;
+  const int L = r.q_off + r.rows;
+  const long long M = (long long)batch * r.rows;
   const size_t es = esize(c.dtype);
   const int E = c.d_inner;
-  if (!x || !y || !aligned16(x) || !aligned16(y)) FAIL(HYMBA_ERR_INVALID_ARG, "x/y null or misaligned");
-  if (!kv || !kv->k || !kv->v || !aligned16(kv->k) || !aligned16(kv->v))
-    FAIL(HYMBA_ERR_INVALID_ARG, "kv buffers null or misaligned");
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
-    FAIL(HYMBA_ERR_INVALID_ARG, "workspace null or not 256-byte aligned");
-  if (workspace_bytes < lay.total)
-    FAIL(HYMBA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, lay.total);
-  if (consumer) {
-    if (kv->owner != layer->producer_id || layer->producer->id != layer->producer_id)
-      FAIL(HYMBA_ERR_NOT_BOUND, "kv was not written by this consumer's producer");
-    if (kv->batch != batch || kv->rows != L)
-      FAIL(HYMBA_ERR_NOT_BOUND, "producer K/V has batch %d rows %d, consumer needs %d x %d",
-           kv->batch, kv->rows, batch, L);
-    if (kv_cache) FAIL(HYMBA_ERR_INVALID_ARG, "a consumer does not write a decode K/V store");
-  }
-  if (kv_cache) {
-    const long long need = c.is_global ? L : (long long)c.n_meta + c.window;
-    if (!kv_cache->k || !kv_cache->v || !aligned16(kv_cache->k) || !aligned16(kv_cache->v))
-      FAIL(HYMBA_ERR_INVALID_ARG, "kv_cache buffers null or misaligned");
-    if (kv_cache->batch != batch || kv_cache->capacity < need)
-      FAIL(HYMBA_ERR_INVALID_ARG, "kv_cache batch %d capacity %d; need batch %d capacity >= %lld",
-           kv_cache->batch, kv_cache->capacity, batch, need);
-  }
-  if (ssm_cache && (!ssm_cache->h || !ssm_cache->conv || !aligned16(ssm_cache->h) ||
-                    !aligned16(ssm_cache->conv)))
-    FAIL(HYMBA_ERR_INVALID_ARG, "ssm_cache buffers null or misaligned");
+  hymba_status st;
+  if (M > 0x7fffffffLL) FAIL(HYMBA_ERR_UNSUPPORTED, "too many rows");
 
   char *ws = reinterpret_cast<char *>(workspace);
-  void *q = ws + lay.q, *xs = ws + lay.x_ssm, *z = ws + lay.z, *u = ws + lay.u;
+  void *q = ws + lay.q, *xs = ws + lay.x_ssm, *z = ws + lay.gate, *u = ws + lay.u;
   float *xdbl = reinterpret_cast<float *>(ws + lay.xdbl);
   void *delta = ws + lay.delta, *yssm = ws + lay.y_ssm, *o = ws + lay.o_attn, *f = ws + lay.fused;
   float *scan_ws = reinterpret_cast<float *>(ws + lay.fused + up256((size_t)M * E * es));
 
-  // 1. input projection (§2.1 W_in_proj) -> Q, K, V, x_ssm, z
+  // 1. input projection (§2.1 W_in_proj) -> Q, K, V, x_ssm, SiLU(z); K and V go to their
+  //    rows q_off.. of each sequence of the full-length K/V
   {
-    ProfScope prof_scope(stream, "in_proj");
+    ProfScope prof_scope(stream, step_name(r, 0));
     GemmArgs g{};
-    g.A = x;
+    g.A = r.x;
     g.lda = c.d_model;
     g.B = layer->w.w_in;
     g.ldb = c.d_model;
@@ -367,12 +404,28 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
     g.ksplit = 1;
     g.epi = in_proj_epilogue(c, consumer, q, qk_width(c), kv->k, kv->v, k_width(c), v_width(c), 0, 0,
                              xs, z, E);
-    if (M > 0x7fffffffLL) FAIL(HYMBA_ERR_UNSUPPORTED, "too many rows");
+    if (!consumer && r.q_off > 0) {
+      g.epi.seg[1].rmap = g.epi.seg[2].rmap = 1;
+      g.epi.rmap_rows = r.rows;
+      g.epi.rmap_stride = L;
+      g.epi.rmap_off = r.q_off;
+    }
+    if (c.rope_base > 0.f) {
+      // Q and K rotated in the epilogue (§2.5 RoPE), positions q_off.. of each sequence
+      float2 *tab = reinterpret_cast<float2 *>(ws + lay.rope);
+      if ((st = rope_table(tab, L, 0, c.head_dim_qk, c.rope_base, stream)) != HYMBA_OK) return st;
+      g.epi.rope_tab = tab;
+      g.epi.rope_rows = r.rows;
+      g.epi.rope_off = r.q_off;
+      g.epi.rope_hd = c.head_dim_qk;
+      g.epi.seg[0].rope = 1;
+      if (!consumer) g.epi.seg[1].rope = 1;
+    }
     if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
   }
   // 2. causal conv + SiLU -> u (and the conv state)
   {
-    ProfScope prof_scope(stream, "conv");
+    ProfScope prof_scope(stream, step_name(r, 1));
     ConvArgs a{};
     a.x = xs;
     a.ld_x = E;
@@ -380,15 +433,16 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
     a.w = layer->w.conv_w;
     a.bias = layer->w.conv_b;
     a.conv_state = ssm_cache ? ssm_cache->conv : nullptr;
+    a.hist = r.conv0;
     a.B = batch;
-    a.L = L;
+    a.L = r.rows;
     a.E = E;
     a.K = c.d_conv;
     if ((st = conv_silu(a, c.dtype, stream)) != HYMBA_OK) return st;
   }
   // 3. x_proj -> [delta_r, B, C] (fp32)
   {
-    ProfScope prof_scope(stream, "x_proj");
+    ProfScope prof_scope(stream, step_name(r, 2));
     GemmArgs g{};
     g.A = u;
     g.lda = E;
@@ -405,7 +459,7 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
   }
   // 4. dt_proj + bias + softplus -> delta (tf32 on the tensor cores for the bf16 path)
   {
-    ProfScope prof_scope(stream, "dt_proj");
+    ProfScope prof_scope(stream, step_name(r, 3));
     GemmArgs g{};
     g.A = xdbl;
     g.lda = xdbl_width(c);
@@ -423,9 +477,9 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
     st = c.dtype == HYMBA_BF16 ? gemm_tc(g, stream) : gemm_simt_f32(g, stream);
     if (st != HYMBA_OK) return st;
   }
-  // 5. selective scan + D skip + SiLU(z) gate -> y_ssm (and the final state)
+  // 5. selective scan + D skip, times the gate SiLU(z) -> y_ssm (and the final state)
   {
-    ProfScope prof_scope(stream, "scan");
+    ProfScope prof_scope(stream, step_name(r, 4));
     ScanArgs a{};
     a.u = u;
     a.delta = delta;
@@ -438,9 +492,10 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
     a.d_skip = layer->w.d_skip;
     a.y = yssm;
     a.h_out = ssm_cache ? ssm_cache->h : nullptr;
-    a.h_in = nullptr;
+    a.h_in = r.h0;
+    a.h_in_bstride = 0;
     a.B = batch;
-    a.L = L;
+    a.L = r.rows;
     a.E = E;
     a.N = c.d_state;
     a.chunk_ws = scan_ws;
@@ -448,7 +503,7 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
   }
   // 6. attention heads over the own or the producer's K/V
   {
-    ProfScope prof_scope(stream, "attention");
+    ProfScope prof_scope(stream, step_name(r, 5));
     AttnArgs a{};
     a.q = q;
     a.k = kv->k;
@@ -456,6 +511,8 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
     a.o = o;
     a.B = batch;
     a.L = L;
+    a.q_off = r.q_off;
+    a.Lq = r.rows;
     a.H = c.n_heads;
     a.Hkv = c.n_kv_heads;
     a.dqk = c.head_dim_qk;
@@ -468,7 +525,7 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
   }
   // 7. norm, beta, mean (Eq. 3)
   {
-    ProfScope prof_scope(stream, "fuse");
+    ProfScope prof_scope(stream, step_name(r, 6));
     FuseArgs a{};
     a.o = o;
     a.y = yssm;
@@ -482,7 +539,7 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
   }
   // 8. output projection
   {
-    ProfScope prof_scope(stream, "out_proj");
+    ProfScope prof_scope(stream, step_name(r, 7));
     GemmArgs g{};
     g.A = f;
     g.lda = E;
@@ -493,13 +550,14 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
     g.K = E;
     g.elem = (int)es;
     g.ksplit = 1;
-    g.epi.seg[0] = seg(y, c.d_model, 0, c.d_model, c.dtype == HYMBA_F32, es);
+    g.epi.seg[0] = seg(r.y, c.d_model, 0, c.d_model, c.dtype == HYMBA_F32, es);
     g.epi.nseg = 1;
+    g.stall = take_debug_stall();
     if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
   }
   // 9. decode K/V store
   if (kv_cache) {
-    ProfScope prof_scope(stream, "kv_emit");
+    ProfScope prof_scope(stream, step_name(r, 8));
     KvEmitArgs a{};
     a.k_seq = kv->k;
     a.v_seq = kv->v;
@@ -525,11 +583,187 @@ hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, co
   return HYMBA_OK;
 }
 
+// Checks shared by both prefill entry points: K/V of L rows per sequence (written by an
+// owner, stamped by the producer for a consumer), the optional decode stores.
+static hymba_status check_prefill_kv(const hymba_layer *layer, int batch, int L, const hymba_kv_seq *kv,
+                                     const hymba_kv_cache *kv_cache, const hymba_ssm_cache *ssm_cache) {
+  const hymba_layer_config &c = layer->cfg;
+  const bool consumer = layer->producer != nullptr;
+  if (!kv || !kv->k || !kv->v || !aligned16(kv->k) || !aligned16(kv->v))
+    FAIL(HYMBA_ERR_INVALID_ARG, "kv buffers null or misaligned");
+  if (consumer) {
+    if (kv->owner != layer->producer_id || layer->producer->id != layer->producer_id)
+      FAIL(HYMBA_ERR_NOT_BOUND, "kv was not written by this consumer's producer");
+    if (kv->batch != batch || kv->rows != L)
+      FAIL(HYMBA_ERR_NOT_BOUND, "producer K/V has batch %d rows %d, consumer needs %d x %d",
+           kv->batch, kv->rows, batch, L);
+    if (kv_cache) FAIL(HYMBA_ERR_INVALID_ARG, "a consumer does not write a decode K/V store");
+  }
+  if (kv_cache) {
+    const long long need = c.is_global ? L : (long long)c.n_meta + c.window;
+    if (!kv_cache->k || !kv_cache->v || !aligned16(kv_cache->k) || !aligned16(kv_cache->v))
+      FAIL(HYMBA_ERR_INVALID_ARG, "kv_cache buffers null or misaligned");
+    if (kv_cache->batch != batch || kv_cache->capacity < need)
+      FAIL(HYMBA_ERR_INVALID_ARG, "kv_cache batch %d capacity %d; need batch %d capacity >= %lld",
+           kv_cache->batch, kv_cache->capacity, batch, need);
+  }
+  if (ssm_cache && (!ssm_cache->h || !ssm_cache->conv || !aligned16(ssm_cache->h) ||
+                    !aligned16(ssm_cache->conv)))
+    FAIL(HYMBA_ERR_INVALID_ARG, "ssm_cache buffers null or misaligned");
+  return HYMBA_OK;
+}
+
+hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_tokens, const void *x, void *y,
+                                 hymba_kv_seq *kv, hymba_kv_cache *kv_cache,
+                                 hymba_ssm_cache *ssm_cache, void *workspace, size_t workspace_bytes,
+                                 hymba_stream_t stream_) {
+  g_msg[0] = 0;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  hymba_prefill_layout lay;
+  hymba_status st = prefill_layout(layer, batch, n_tokens, &lay, nullptr);
+  if (st != HYMBA_OK) return st;
+  const int L = layer->cfg.n_meta + n_tokens;
+  if (!x || !y || !aligned16(x) || !aligned16(y)) FAIL(HYMBA_ERR_INVALID_ARG, "x/y null or misaligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    FAIL(HYMBA_ERR_INVALID_ARG, "workspace null or not 256-byte aligned");
+  if (workspace_bytes < lay.total)
+    FAIL(HYMBA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, lay.total);
+  if ((st = check_prefill_kv(layer, batch, L, kv, kv_cache, ssm_cache)) != HYMBA_OK) return st;
+  PrefillRun r{};
+  r.x = x;
+  r.y = y;
+  r.rows = L;
+  r.q_off = 0;
+  return prefill_run(layer, batch, r, kv, kv_cache, ssm_cache, workspace, lay, stream);
+}
+
+// ---------------------------------------------------------------------------
+// meta-token cache (§2.3: the meta rows do not depend on the input, so their K/V, SSM
+// state and conv history are computed once and every prefill starts from them)
+// ---------------------------------------------------------------------------
+hymba_status hymba_layer_meta_workspace(const hymba_layer *layer, size_t *bytes) {
+  g_msg[0] = 0;
+  if (!layer || !bytes) FAIL(HYMBA_ERR_INVALID_ARG, "null argument");
+  if (layer->cfg.n_meta < 1) FAIL(HYMBA_ERR_INVALID_ARG, "the layer has no meta tokens");
+  return hymba_layer_prefill_workspace(layer, 1, 0, bytes);
+}
+
+hymba_status hymba_layer_meta_precompute(hymba_layer *layer, const void *x_meta, hymba_meta_cache *meta,
+                                         const hymba_meta_cache *producer_meta, void *workspace,
+                                         size_t workspace_bytes, hymba_stream_t stream) {
+  g_msg[0] = 0;
+  if (!layer || !meta) FAIL(HYMBA_ERR_INVALID_ARG, "null argument");
+  const hymba_layer_config &c = layer->cfg;
+  const bool consumer = layer->producer != nullptr;
+  if (c.n_meta < 1) FAIL(HYMBA_ERR_INVALID_ARG, "the layer has no meta tokens");
+  if (!meta->y || !meta->h || !meta->conv || !aligned16(meta->y) || !aligned16(meta->h) ||
+      !aligned16(meta->conv))
+    FAIL(HYMBA_ERR_INVALID_ARG, "meta cache y/h/conv null or misaligned");
+  hymba_kv_seq kv{};
+  if (consumer) {
+    if (!producer_meta || producer_meta->owner != layer->producer_id)
+      FAIL(HYMBA_ERR_NOT_BOUND, "a consumer needs its producer's meta cache");
+    kv.k = producer_meta->k;
+    kv.v = producer_meta->v;
+    kv.batch = 1;
+    kv.rows = c.n_meta;
+    kv.owner = producer_meta->owner;
+  } else {
+    if (producer_meta) FAIL(HYMBA_ERR_INVALID_ARG, "a layer that owns its K/V takes no producer cache");
+    kv.k = meta->k;
+    kv.v = meta->v;
+  }
+  hymba_ssm_cache ssm{meta->h, meta->conv};
+  meta->owner = 0;
+  hymba_prefill_layout lay;
+  hymba_status st = prefill_layout(layer, 1, 0, &lay, nullptr);
+  if (st != HYMBA_OK) return st;
+  if (!x_meta || !aligned16(x_meta)) FAIL(HYMBA_ERR_INVALID_ARG, "x_meta null or misaligned");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    FAIL(HYMBA_ERR_INVALID_ARG, "workspace null or not 256-byte aligned");
+  if (workspace_bytes < lay.total)
+    FAIL(HYMBA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, lay.total);
+  if ((st = check_prefill_kv(layer, 1, c.n_meta, &kv, nullptr, &ssm)) != HYMBA_OK) return st;
+  PrefillRun r{};
+  r.x = x_meta;
+  r.y = meta->y;
+  r.rows = c.n_meta;
+  r.q_off = 0;
+  r.meta = true;
+  st = prefill_run(layer, 1, r, &kv, nullptr, &ssm, workspace, lay, reinterpret_cast<cudaStream_t>(stream));
+  if (st != HYMBA_OK) return st;
+  meta->owner = layer->id;
+  return HYMBA_OK;
+}
+
+hymba_status hymba_layer_prefill_cached_workspace(const hymba_layer *layer, int batch, int n_tokens,
+                                                  size_t *bytes) {
+  g_msg[0] = 0;
+  if (!bytes) FAIL(HYMBA_ERR_INVALID_ARG, "null output");
+  if (n_tokens < 1) FAIL(HYMBA_ERR_INVALID_ARG, "n_tokens < 1");
+  hymba_prefill_layout lay;
+  hymba_status st = prefill_layout_rows(layer, batch, n_tokens, &lay, nullptr);
+  if (st != HYMBA_OK) return st;
+  *bytes = lay.total;
+  return HYMBA_OK;
+}
+
+hymba_status hymba_layer_prefill_cached(hymba_layer *layer, int batch, int n_tokens, const void *x,
+                                        void *y, const hymba_meta_cache *meta, hymba_kv_seq *kv,
+                                        hymba_kv_cache *kv_cache, hymba_ssm_cache *ssm_cache,
+                                        void *workspace, size_t workspace_bytes, hymba_stream_t stream_) {
+  g_msg[0] = 0;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (!layer) FAIL(HYMBA_ERR_INVALID_ARG, "null layer");
+  const hymba_layer_config &c = layer->cfg;
+  const bool consumer = layer->producer != nullptr;
+  if (n_tokens < 1) FAIL(HYMBA_ERR_INVALID_ARG, "n_tokens < 1");
+  if (c.n_meta < 1) FAIL(HYMBA_ERR_INVALID_ARG, "the layer has no meta tokens");
+  hymba_prefill_layout lay;
+  hymba_status st = prefill_layout_rows(layer, batch, n_tokens, &lay, nullptr);
+  if (st != HYMBA_OK) return st;
+  const int L = c.n_meta + n_tokens;
+  if (!x || !y || !aligned16(x) || !aligned16(y)) FAIL(HYMBA_ERR_INVALID_ARG, "x/y null or misaligned");
+  if (!meta || meta->owner != layer->id) FAIL(HYMBA_ERR_NOT_BOUND, "meta cache not computed by this layer");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    FAIL(HYMBA_ERR_INVALID_ARG, "workspace null or not 256-byte aligned");
+  if (workspace_bytes < lay.total)
+    FAIL(HYMBA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, lay.total);
+  if ((st = check_prefill_kv(layer, batch, L, kv, kv_cache, ssm_cache)) != HYMBA_OK) return st;
+  if (!consumer) {
+    // the meta rows' K/V into rows 0..m-1 of every sequence
+    if (!meta->k || !meta->v || !aligned16(meta->k) || !aligned16(meta->v))
+      FAIL(HYMBA_ERR_INVALID_ARG, "meta cache K/V null or misaligned");
+    if ((k_width(c) * esize(c.dtype)) % 16 || (v_width(c) * esize(c.dtype)) % 16)
+      FAIL(HYMBA_ERR_UNSUPPORTED, "K/V rows must be multiples of 16 bytes");
+    ProfScope prof_scope(stream, "kv_meta");
+    KvBroadcastArgs a{};
+    a.k_meta = meta->k;
+    a.v_meta = meta->v;
+    a.k_seq = kv->k;
+    a.v_seq = kv->v;
+    a.B = batch;
+    a.L = L;
+    a.m = c.n_meta;
+    a.kw = k_width(c);
+    a.vw = v_width(c);
+    if ((st = kv_broadcast_meta(a, c.dtype, stream)) != HYMBA_OK) return st;
+  }
+  PrefillRun r{};
+  r.x = x;
+  r.y = y;
+  r.rows = n_tokens;
+  r.q_off = c.n_meta;
+  r.h0 = meta->h;
+  r.conv0 = meta->conv;
+  return prefill_run(layer, batch, r, kv, kv_cache, ssm_cache, workspace, lay, stream);
+}
+
 // ---------------------------------------------------------------------------
 // decode
 // ---------------------------------------------------------------------------
 struct DecodeLayout {
-  size_t q, x_ssm, z, u, xdbl, y_ssm, o, f, y32, part, total;
+  size_t q, x_ssm, z, u, xdbl, y_ssm, o, f, part, rope, total;
 };
 
 static DecodeLayout decode_layout(const hymba_layer_config &c, int batch, long long pos) {
@@ -545,13 +779,13 @@ static DecodeLayout decode_layout(const hymba_layer_config &c, int batch, long l
   d.x_ssm = take(B * E * es);
   d.z = take(B * E * es);
   d.u = take(B * E * es);
-  d.xdbl = take(B * xdbl_width(c) * 4);  // xdbl and y32 adjacent: zeroed in one range
-  d.y32 = take(B * c.d_model * 4);
+  d.xdbl = take(B * xdbl_width(c) * 4);
   d.y_ssm = take(B * E * es);
   d.o = take(B * E * es);
   d.f = take(B * E * es);
   d.part = take(decode_attn_workspace_floats(batch, c.n_heads, c.head_dim_v, pos, c.n_meta,
                                              c.window, c.is_global) * 4);
+  d.rope = take(c.rope_base > 0.f ? (size_t)(c.head_dim_qk / 2) * 8 : 0);
   d.total = off;
   return d;
 }
@@ -606,7 +840,6 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
   void *q = ws + d.q, *xs = ws + d.x_ssm, *z = ws + d.z, *u = ws + d.u;
   float *xdbl = reinterpret_cast<float *>(ws + d.xdbl);
   void *yssm = ws + d.y_ssm, *o = ws + d.o, *f = ws + d.f;
-  float *y32 = reinterpret_cast<float *>(ws + d.y32);
   float *part = reinterpret_cast<float *>(ws + d.part);
   hymba_status st;
   const long long slot = (c.is_global || pos < c.n_meta) ? pos : c.n_meta + (pos - c.n_meta) % c.window;
@@ -631,10 +864,21 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
                              (long long)c.n_kv_heads * cap * c.head_dim_qk,
                              (long long)c.n_kv_heads * cap * c.head_dim_v,
                              cap * c.head_dim_qk, cap * c.head_dim_v, xs, z, E);
-    // the split-K accumulators of x_proj and out_proj (adjacent) start at zero
+    if (c.rope_base > 0.f) {
+      // the new token's Q and K rotated by the angles of its position
+      float2 *tab = reinterpret_cast<float2 *>(ws + d.rope);
+      if ((st = rope_table(tab, 1, pos, c.head_dim_qk, c.rope_base, stream)) != HYMBA_OK) return st;
+      g.epi.rope_tab = tab;
+      g.epi.rope_rows = 1;
+      g.epi.rope_off = 0;
+      g.epi.rope_hd = c.head_dim_qk;
+      g.epi.seg[0].rope = 1;
+      if (!consumer) g.epi.seg[1].rope = 1;
+    }
+    // x_proj's accumulators (summed by the SSM kernel's channel blocks) start at zero
     g.epi.zero = xdbl;
-    g.epi.zero_n = (long long)((d.y32 - d.xdbl) / 4) + (long long)batch * c.d_model;
-    if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
+    g.epi.zero_n = (long long)batch * xdbl_width(c);
+    if ((st = gemm_decode(g, c.dtype, stream)) != HYMBA_OK) return st;
   }
   // 2-5. SSM branch: conv + x_proj, then dt_proj + softplus + one scan step + gate
   {
@@ -722,10 +966,9 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
     a.eps = c.rms_eps;
     if ((st = fuse_branches(a, c.dtype, stream)) != HYMBA_OK) return st;
   }
-  // 8. output projection, split over K into fp32, then to the storage dtype
+  // 8. output projection, straight into y_t
   {
     ProfScope prof_scope(stream, "dec_out_proj");
-    const int ksplit = 4;
     GemmArgs g{};
     g.A = f;
     g.lda = E;
@@ -735,13 +978,10 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
     g.N = c.d_model;
     g.K = E;
     g.elem = (int)es;
-    g.ksplit = ksplit;
-    g.epi.seg[0] = seg(y32, c.d_model, 0, c.d_model, 1, es);
+    g.ksplit = 1;
+    g.epi.seg[0] = seg(y_t, c.d_model, 0, c.d_model, c.dtype == HYMBA_F32, es);
     g.epi.nseg = 1;
-    g.epi.atomic = 1;
-    if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
-    if ((st = convert_f32_to(y32, y_t, (long long)batch * c.d_model, c.dtype, stream)) != HYMBA_OK)
-      return st;
+    if ((st = gemm_decode(g, c.dtype, stream)) != HYMBA_OK) return st;
   }
   if (!consumer) kv_cache->owner = layer->id;
   return HYMBA_OK;
@@ -758,6 +998,21 @@ hymba_status hymba_stream_status(hymba_stream_t stream) {
   if (e != cudaSuccess) FAIL(HYMBA_ERR_CUDA, "%s", cudaGetErrorString(e));
   const unsigned err = take_error_gemm() | take_error_attn();
   if (err & kErrTimeoutHost) FAIL(HYMBA_ERR_TIMEOUT, "a device-side wait timed out");
+  return HYMBA_OK;
+}
+
+hymba_status hymba_set_wait_limit(int64_t cycles, int64_t *applied) {
+  g_msg[0] = 0;
+  if (cycles < 0) FAIL(HYMBA_ERR_INVALID_ARG, "negative wait limit");
+  g_wait_limit.store(cycles);
+  if (applied) *applied = wait_limit_cycles();
+  return HYMBA_OK;
+}
+
+hymba_status hymba_debug_stall_next_prefill(int count) {
+  g_msg[0] = 0;
+  if (count < 0) FAIL(HYMBA_ERR_INVALID_ARG, "negative count");
+  g_stall.store(count);
   return HYMBA_OK;
 }
 
@@ -814,13 +1069,34 @@ hymba_status hymba_profile_collect(hymba_profile_entry *out, int max, int *n) {
   return HYMBA_OK;
 }
 
-hymba_status hymba_debug_mask_bitmap(int L, int n_meta, int window, int is_global, uint32_t *bits,
-                                     uint8_t *tile_class, hymba_stream_t stream) {
+hymba_status hymba_debug_mask_bitmap(int L, int n_meta, int window, int is_global, int path,
+                                     uint32_t *bits, uint8_t *tile_class, hymba_stream_t stream) {
   g_msg[0] = 0;
   if (L < 1 || n_meta < 0 || (!is_global && window < 1)) FAIL(HYMBA_ERR_INVALID_ARG, "bad mask shape");
+  if (path != 0 && path != 1) FAIL(HYMBA_ERR_INVALID_ARG, "path must be 0 (tensor-core) or 1 (fp32)");
   if (!bits) FAIL(HYMBA_ERR_INVALID_ARG, "null bits");
-  return mask_bitmap(L, n_meta, window, is_global, bits, tile_class,
+  return mask_bitmap(L, n_meta, window, is_global, path, bits, tile_class,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+hymba_status hymba_debug_decode_mask(int64_t pos, int n_meta, int window, int is_global,
+                                     int capacity, uint32_t *bits, hymba_stream_t stream) {
+  g_msg[0] = 0;
+  if (n_meta < 0 || pos < n_meta || (!is_global && window < 1) || capacity < 1)
+    FAIL(HYMBA_ERR_INVALID_ARG, "bad decode mask shape");
+  const long long need = is_global ? pos + 1 : (long long)n_meta + window;
+  if (capacity < need) FAIL(HYMBA_ERR_INVALID_ARG, "capacity %d < %lld slots read", capacity, need);
+  if (!bits) FAIL(HYMBA_ERR_INVALID_ARG, "null bits");
+  return decode_mask(pos, n_meta, window, is_global, capacity, bits,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+hymba_status hymba_debug_exp2_poly(int degree, const float *x, float *y, int64_t n,
+                                   hymba_stream_t stream) {
+  g_msg[0] = 0;
+  if (degree != 3 && degree != 5) FAIL(HYMBA_ERR_INVALID_ARG, "degree must be 3 or 5");
+  if (n < 0 || (n > 0 && (!x || !y))) FAIL(HYMBA_ERR_INVALID_ARG, "null buffer or n < 0");
+  return exp2_poly_eval(degree, x, y, n, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -66,12 +66,12 @@ constexpr uint32_t IDESC_PV = make_idesc(128, 1, 0, 1);
 }  // namespace fa
 
 // Class of the (query tile, key tile) pair as the prefill kernel sees it.
-__device__ __forceinline__ int fa_tile_class(int qtile, int kt, int L, int n_meta, int window,
+__device__ __forceinline__ int fa_tile_class(int qtile, int kt, int L, int q_off, int n_meta, int window,
                                              int is_global) {
-  return seq_tile_class(qtile, kt, L, n_meta, window, is_global);
+  return seq_tile_class(qtile, kt, L, q_off, n_meta, window, is_global);
 }
-// Key tiles streamed for the query-tile pair (qa, qa+1): every tile holding a pair
-// visible from some row of the pair.  The keys visible from rows [i0, i1] are
+// Key tiles streamed for the query-tile pair (qa, qa+1) (query positions from
+// q_off + 128 qa): every tile holding a pair visible from some row of the pair.  The keys visible from rows [i0, i1] are
 // [0, min(m, i1+1)) and [i0 - W + 1, i1] (all of [0, i1] for a global layer), so
 // the tiles are [0, a_end) followed by [lo, hi].  Same sequence in every role.
 struct FaTiles {
@@ -79,10 +79,10 @@ struct FaTiles {
   __device__ __forceinline__ int first() const { return a_end > 0 ? 0 : lo; }
   __device__ __forceinline__ int next(int kt) const { return kt + 1 < a_end ? kt + 1 : max(kt + 1, lo); }
 };
-__device__ __forceinline__ FaTiles fa_tiles(int qa, int L, int n_meta, int window, int is_global) {
+__device__ __forceinline__ FaTiles fa_tiles(int qa, int L, int q_off, int n_meta, int window, int is_global) {
   FaTiles t;
-  const long long i0 = (long long)qa * fa::QT;
-  const long long i1 = min((long long)(qa + 2) * fa::QT, (long long)L) - 1;
+  const long long i0 = (long long)q_off + (long long)qa * fa::QT;
+  const long long i1 = min((long long)q_off + (long long)(qa + 2) * fa::QT, (long long)L) - 1;
   t.hi = (int)(i1 / fa::KT);
   if (is_global) {
     t.a_end = 0;
@@ -117,12 +117,30 @@ __device__ __forceinline__ int fa_count(const FaTiles &t) {
   return n;
 }
 
-// Keep-mask of the 32 columns col0..col0+31 for the column ranges [0, hi1) and [lo2, hi2).
+// Visible keys of query position i inside the 128-key tile that starts at key0, as column
+// ranges of the tile: [0, hi1) (meta keys) and [lo2, hi2) (the window, up to the query
+// itself).  A global layer has hi1 = lo2 = 0.
+struct FaCols {
+  int hi1, lo2, hi2;
+};
+__device__ __forceinline__ FaCols fa_cols(long long i, long long key0, int n_meta, int window,
+                                          int is_global) {
+  const long long meta_end = is_global ? 0 : min((long long)n_meta, i + 1);
+  const long long win_lo = is_global ? 0 : max((long long)n_meta, i - window + 1);
+  FaCols c;
+  c.hi1 = (int)max(0LL, min(128LL, meta_end - key0));
+  c.lo2 = (int)max(0LL, min(128LL, win_lo - key0));
+  c.hi2 = (int)max(0LL, min(128LL, i + 1 - key0));
+  return c;
+}
 __device__ __forceinline__ uint32_t low_bits(int n) {
   return n <= 0 ? 0u : (n >= 32 ? 0xffffffffu : (1u << n) - 1u);
 }
-__device__ __forceinline__ void mask_cols(uint32_t (&v)[32], int col0, int hi1, int lo2, int hi2) {
-  const uint32_t keep = low_bits(hi1 - col0) | (low_bits(hi2 - col0) & ~low_bits(lo2 - col0));
+// Keep-mask of the 32 columns col0..col0+31 of a partially visible tile.
+__device__ __forceinline__ uint32_t fa_keep32(const FaCols &c, int col0) {
+  return low_bits(c.hi1 - col0) | (low_bits(c.hi2 - col0) & ~low_bits(c.lo2 - col0));
+}
+__device__ __forceinline__ void mask_cols(uint32_t (&v)[32], uint32_t keep) {
 #pragma unroll
   for (int e = 0; e < 32; ++e)
     if (!(keep & (1u << e))) v[e] = __float_as_uint(-INFINITY);
@@ -182,8 +200,8 @@ __device__ __forceinline__ void p_store(const uint32_t (&pk)[16], int c, int r, 
 __global__ void __launch_bounds__(fa::THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                       int L, int B, int H, int Hkv, int n_meta, int window, int is_global,
-                       float scale_log2, int npairs) {
+                       int L, int q_off, int B, int H, int Hkv, int n_meta, int window, int is_global,
+                       float scale_log2, int npairs, long long wlim) {
   using namespace fa;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -249,20 +267,20 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         const FaItem w = fa_item(it, H, BH, npairs);
         const int gkv = w.h / (H / Hkv);
         const int qb = itk & 1;
-        if (!mbar_wait(&q_empty[qb], ((uint32_t(itk) >> 1) & 1u) ^ 1u, &g_err_attn)) { ok = false; break; }
+        if (!mbar_wait(&q_empty[qb], ((uint32_t(itk) >> 1) & 1u) ^ 1u, &g_err_attn, wlim)) { ok = false; break; }
         mbar_arrive_expect_tx(&q_full[qb], NQ * Q_BYTES);
         for (int q = 0; q < NQ; ++q)
           tma_load_3d(smem + OFF_Q + (qb * NQ + q) * Q_BYTES, &tmQ, &q_full[qb], w.h * 64, (w.qa + q) * QT, w.b);
         ++nq[qb];
-        const FaTiles t = fa_tiles(w.qa, L, n_meta, window, is_global);
+        const FaTiles t = fa_tiles(w.qa, L, q_off, n_meta, window, is_global);
         for (int kt = t.first(); kt <= t.hi; kt = t.next(kt), ++g) {
           const int st = int(g & 1);
           const uint32_t ph = uint32_t(g >> 1) & 1u;
-          if (!mbar_wait(&k_empty[st], ph ^ 1u, &g_err_attn)) { ok = false; break; }
+          if (!mbar_wait(&k_empty[st], ph ^ 1u, &g_err_attn, wlim)) { ok = false; break; }
           mbar_arrive_expect_tx(&k_full[st], K_BYTES);
           tma_load_3d(smem + OFF_K + st * K_BYTES, &tmK, &k_full[st], gkv * 64, kt * KT, w.b);
           ++nk[st];
-          if (!mbar_wait(&v_empty[st], ph ^ 1u, &g_err_attn)) { ok = false; break; }
+          if (!mbar_wait(&v_empty[st], ph ^ 1u, &g_err_attn, wlim)) { ok = false; break; }
           mbar_arrive_expect_tx(&v_full[st], V_BYTES);
           uint8_t *vdst = smem + OFF_V + st * V_BYTES;
           tma_load_3d(vdst, &tmV, &v_full[st], gkv * 128, kt * KT, w.b);
@@ -272,9 +290,9 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
       }
       if (!ok) {
         for (int x = 0; x < 2; ++x) {
-          if (nq[x]) mbar_wait_drain(&q_full[x], (nq[x] - 1) & 1u, &g_err_attn);
-          if (nk[x]) mbar_wait_drain(&k_full[x], (nk[x] - 1) & 1u, &g_err_attn);
-          if (nv[x]) mbar_wait_drain(&v_full[x], (nv[x] - 1) & 1u, &g_err_attn);
+          if (nq[x]) mbar_wait_drain(&q_full[x], (nq[x] - 1) & 1u, &g_err_attn, wlim);
+          if (nk[x]) mbar_wait_drain(&k_full[x], (nk[x] - 1) & 1u, &g_err_attn, wlim);
+          if (nv[x]) mbar_wait_drain(&v_full[x], (nv[x] - 1) & 1u, &g_err_attn, wlim);
         }
       }
     }
@@ -306,9 +324,9 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
       int itk = 0;
       if (it < n_items) {
         FaItem w = fa_item(it, H, BH, npairs);
-        int n = fa_count(fa_tiles(w.qa, L, n_meta, window, is_global));
+        int n = fa_count(fa_tiles(w.qa, L, q_off, n_meta, window, is_global));
         // S of the first tile
-        ok = mbar_wait(&q_full[0], 0, &g_err_attn) && mbar_wait(&k_full[0], 0, &g_err_attn);
+        ok = mbar_wait(&q_full[0], 0, &g_err_attn, wlim) && mbar_wait(&k_full[0], 0, &g_err_attn, wlim);
         if (ok) {
           tc_fence_after();
           for (int q = 0; q < NQ; ++q) issue_S(q, 0, 0);
@@ -329,16 +347,16 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
           if (has_next) {
             if (!same) {
               const FaItem wn = fa_item(it_next, H, BH, npairs);
-              n_next = fa_count(fa_tiles(wn.qa, L, n_meta, window, is_global));
-              if (!mbar_wait(&q_full[qb_next], (uint32_t(itk + 1) >> 1) & 1u, &g_err_attn)) { ok = false; break; }
+              n_next = fa_count(fa_tiles(wn.qa, L, q_off, n_meta, window, is_global));
+              if (!mbar_wait(&q_full[qb_next], (uint32_t(itk + 1) >> 1) & 1u, &g_err_attn, wlim)) { ok = false; break; }
             }
-            if (!mbar_wait(&k_full[st1], uint32_t(g1 >> 1) & 1u, &g_err_attn)) { ok = false; break; }
+            if (!mbar_wait(&k_full[st1], uint32_t(g1 >> 1) & 1u, &g_err_attn, wlim)) { ok = false; break; }
           }
-          if (!mbar_wait(&v_full[st], uint32_t(g >> 1) & 1u, &g_err_attn)) { ok = false; break; }
+          if (!mbar_wait(&v_full[st], uint32_t(g >> 1) & 1u, &g_err_attn, wlim)) { ok = false; break; }
           // per query tile: P V of this tile, then S of the next one into the same columns
           // (the tensor core runs them in order, so P is read before S overwrites it)
           for (int q = 0; q < NQ && ok; ++q) {
-            if (!mbar_wait(&p_full[q], uint32_t(g) & 1u, &g_err_attn)) { ok = false; break; }
+            if (!mbar_wait(&p_full[q], uint32_t(g) & 1u, &g_err_attn, wlim)) { ok = false; break; }
             tc_fence_after();
             issue_PV(q, st, j > 0);
             if (has_next) issue_S(q, st1, qb_next);
@@ -363,7 +381,7 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
       if (!ok) {
         // Drain issued MMAs before tensor memory is released.
         mma_commit(drain);
-        mbar_wait_drain(drain, 0, &g_err_attn);
+        mbar_wait_drain(drain, 0, &g_err_attn, wlim);
       }
     }
    }
@@ -383,16 +401,13 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
     for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++itk) {
       const FaItem w = fa_item(it, H, BH, npairs);
       const int qtile = w.qa + q;
-      const long long i = (long long)qtile * QT + r;  // query position
-      // Visible keys of row i: [0, meta_end) and [win_lo, i] (positions).
-      const long long meta_end = is_global ? 0 : min((long long)n_meta, i + 1);
-      const long long win_lo = is_global ? 0 : max((long long)n_meta, i - window + 1);
-      const FaTiles tiles = fa_tiles(w.qa, L, n_meta, window, is_global);
+      const long long i = (long long)q_off + (long long)qtile * QT + r;  // query position
+      const FaTiles tiles = fa_tiles(w.qa, L, q_off, n_meta, window, is_global);
       float m_run = -INFINITY, l_run = 0.f;
       int j = 0;
       for (int kt = tiles.first(); kt <= tiles.hi; kt = tiles.next(kt), ++g, ++j) {
-        const int cls = fa_tile_class(qtile, kt, L, n_meta, window, is_global);  // uniform
-        if (!mbar_wait(&s_full[q], uint32_t(g) & 1u, &g_err_attn)) { ok = false; break; }
+        const int cls = fa_tile_class(qtile, kt, L, q_off, n_meta, window, is_global);  // uniform
+        if (!mbar_wait(&s_full[q], uint32_t(g) & 1u, &g_err_attn, wlim)) { ok = false; break; }
         tc_fence_after();
         if (cls == 0) {
           // no visible pair in this tile (or the query tile lies past the sequence):
@@ -416,15 +431,12 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         tmem_ld32(tS + 96, s3);
         tmem_wait_ld();
         if (cls != 1) {
-          // partial tile: keep the column ranges [0, hi1) and [lo2, hi2)
-          const long long key0 = (long long)kt * KT;
-          const int hi1 = (int)max(0LL, min(128LL, meta_end - key0));
-          const int lo2 = (int)max(0LL, min(128LL, win_lo - key0));
-          const int hi2 = (int)max(0LL, min(128LL, i + 1 - key0));
-          mask_cols(s0, 0, hi1, lo2, hi2);
-          mask_cols(s1, 32, hi1, lo2, hi2);
-          mask_cols(s2, 64, hi1, lo2, hi2);
-          mask_cols(s3, 96, hi1, lo2, hi2);
+          // partial tile: keep the column ranges of this row
+          const FaCols fc = fa_cols(i, (long long)kt * KT, n_meta, window, is_global);
+          mask_cols(s0, fa_keep32(fc, 0));
+          mask_cols(s1, fa_keep32(fc, 32));
+          mask_cols(s2, fa_keep32(fc, 64));
+          mask_cols(s3, fa_keep32(fc, 96));
         }
         // row max (scale > 0, so the max commutes with the scaling)
         const float mx = row_max128(s0, s1, s2, s3) * scale_log2;
@@ -448,7 +460,7 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         l_run += ps.x + ps.y;
         if (__any_sync(0xffffffffu, resc)) {
           // O grows by the new max: rescale it once the previous tile's P V has retired
-          if (!mbar_wait(&o_done[q], uint32_t(g - 1) & 1u, &g_err_attn)) { ok = false; break; }
+          if (!mbar_wait(&o_done[q], uint32_t(g - 1) & 1u, &g_err_attn, wlim)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
@@ -475,7 +487,7 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
       // the item's output once its last P V has retired: O / l -> bf16 rows written into
       // this tile's P buffer (idle until the next item's first P) as two 128-byte-swizzled
       // 64-column boxes, then two TMA tile stores (rows past the sequence are not written)
-      if (!mbar_wait(&o_done[q], uint32_t(g - 1) & 1u, &g_err_attn)) { ok = false; break; }
+      if (!mbar_wait(&o_done[q], uint32_t(g - 1) & 1u, &g_err_attn, wlim)) { ok = false; break; }
       tc_fence_after();
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
       {
@@ -498,7 +510,7 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
       if (quarter == 0 && lane == 0) {
         // every row of the tile staged -> two stores; the buffer is released once they
         // have read it (released on a failed wait too, so that no thread waits forever)
-        if (mbar_wait(&o_staged[q], uint32_t(itk) & 1u, &g_err_attn)) {
+        if (mbar_wait(&o_staged[q], uint32_t(itk) & 1u, &g_err_attn, wlim)) {
           const uint8_t *stage = smem + OFF_P + q * P_BYTES;
           tma_store_3d(&tmO, stage, w.h * 128, qtile * QT, w.b);
           tma_store_3d(&tmO, stage + P_BYTES / 2, w.h * 128 + 64, qtile * QT, w.b);
@@ -507,7 +519,7 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         }
         mbar_arrive(&o_stored[q]);
       }
-      if (!mbar_wait(&o_stored[q], uint32_t(itk) & 1u, &g_err_attn)) { ok = false; break; }
+      if (!mbar_wait(&o_stored[q], uint32_t(itk) & 1u, &g_err_attn, wlim)) { ok = false; break; }
     }
     if (quarter == 0 && lane == 0) bulk_wait_all();
   }
@@ -537,8 +549,8 @@ static hymba_status attention_prefill_tc(const AttnArgs &a, cudaStream_t s) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (sms <= 0) sms = 148;
   CUtensorMap tq, tk, tv, to;
-  const uint64_t dq[3] = {(uint64_t)a.H * 64, (uint64_t)a.L, (uint64_t)a.B};
-  const uint64_t sq[2] = {(uint64_t)a.H * 64 * 2, (uint64_t)a.L * a.H * 64 * 2};
+  const uint64_t dq[3] = {(uint64_t)a.H * 64, (uint64_t)a.Lq, (uint64_t)a.B};
+  const uint64_t sq[2] = {(uint64_t)a.H * 64 * 2, (uint64_t)a.Lq * a.H * 64 * 2};
   const uint64_t dk[3] = {(uint64_t)a.Hkv * 64, (uint64_t)a.L, (uint64_t)a.B};
   const uint64_t sk[2] = {(uint64_t)a.Hkv * 64 * 2, (uint64_t)a.L * a.Hkv * 64 * 2};
   const uint64_t dv[3] = {(uint64_t)a.Hkv * 128, (uint64_t)a.L, (uint64_t)a.B};
@@ -547,17 +559,17 @@ static hymba_status attention_prefill_tc(const AttnArgs &a, cudaStream_t s) {
   if (!make_tmap(&tq, a.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dq, sq, box)) return HYMBA_ERR_CUDA;
   if (!make_tmap(&tk, a.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dk, sk, box)) return HYMBA_ERR_CUDA;
   if (!make_tmap(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dv, sv, box)) return HYMBA_ERR_CUDA;
-  const uint64_t dout[3] = {(uint64_t)a.H * 128, (uint64_t)a.L, (uint64_t)a.B};
-  const uint64_t sout[2] = {(uint64_t)a.H * 128 * 2, (uint64_t)a.L * a.H * 128 * 2};
+  const uint64_t dout[3] = {(uint64_t)a.H * 128, (uint64_t)a.Lq, (uint64_t)a.B};
+  const uint64_t sout[2] = {(uint64_t)a.H * 128 * 2, (uint64_t)a.Lq * a.H * 128 * 2};
   if (!make_tmap(&to, a.o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, dout, sout, box)) return HYMBA_ERR_CUDA;
-  const int nqt = (a.L + QT - 1) / QT;
+  const int nqt = (a.Lq + QT - 1) / QT;
   const int npairs = (nqt + 1) / 2;
   const long long items = (long long)npairs * a.H * a.B;
   if (items == 0) return HYMBA_OK;
   const unsigned grid = (unsigned)std::min<long long>(items, sms);
   attn_fwd_tc_kernel<<<grid, THREADS, SMEM, s>>>(
-      tq, tk, tv, to, a.L, a.B, a.H, a.Hkv, a.n_meta, a.window,
-      a.is_global, a.scale * 1.4426950408889634f, npairs);
+      tq, tk, tv, to, a.L, a.q_off, a.B, a.H, a.Hkv, a.n_meta, a.window,
+      a.is_global, a.scale * 1.4426950408889634f, npairs, wait_limit_cycles());
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -572,18 +584,19 @@ static hymba_status attention_prefill_tc(const AttnArgs &a, cudaStream_t s) {
 // ---------------------------------------------------------------------------
 template <typename T>
 __global__ void attn_fwd_simt_kernel(const T *__restrict__ q, const T *__restrict__ k,
-                                     const T *__restrict__ v, T *__restrict__ o, int B, int L, int H,
-                                     int Hkv, int dqk, int dv, int n_meta, int window, int is_global,
-                                     float scale) {
+                                     const T *__restrict__ v, T *__restrict__ o, int B, int L, int q_off,
+                                     int Lq, int H, int Hkv, int dqk, int dv, int n_meta, int window,
+                                     int is_global, float scale) {
   const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (wid >= (long long)B * L * H) return;
+  if (wid >= (long long)B * Lq * H) return;
   const int h = int(wid % H);
   const long long bi = wid / H;
-  const int i = int(bi % L);
-  const int b = int(bi / L);
+  const int row = int(bi % Lq);
+  const int i = q_off + row;  // query position
+  const int b = int(bi / Lq);
   const int g = h / (H / Hkv);
-  const T *qr = q + ((long long)b * L + i) * H * dqk + h * dqk;
+  const T *qr = q + ((long long)b * Lq + row) * H * dqk + h * dqk;
   float mx = -INFINITY, l = 0.f;
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};  // dv <= 256: lane owns columns lane + 32*t
   for (int j = 0; j <= i; ++j) {
@@ -606,7 +619,7 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ q, const T *__restric
     }
     mx = mn;
   }
-  T *orow = o + ((long long)b * L + i) * H * dv + h * dv;
+  T *orow = o + ((long long)b * Lq + row) * H * dv + h * dv;
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
     const int d = lane + 32 * t;
@@ -626,12 +639,12 @@ hymba_status attention_prefill(const AttnArgs &a, hymba_dtype dt, cudaStream_t s
     set_error("fp32 attention supports head_dim_v <= 256");
     return HYMBA_ERR_UNSUPPORTED;
   }
-  const long long warps = (long long)a.B * a.L * a.H;
+  const long long warps = (long long)a.B * a.Lq * a.H;
   const int tpb = 256;
   const long long blocks = (warps * 32 + tpb - 1) / tpb;
   attn_fwd_simt_kernel<float><<<(unsigned)blocks, tpb, 0, s>>>(
-      (const float *)a.q, (const float *)a.k, (const float *)a.v, (float *)a.o, a.B, a.L, a.H,
-      a.Hkv, a.dqk, a.dv, a.n_meta, a.window, a.is_global, a.scale);
+      (const float *)a.q, (const float *)a.k, (const float *)a.v, (float *)a.o, a.B, a.L, a.q_off, a.Lq,
+      a.H, a.Hkv, a.dqk, a.dv, a.n_meta, a.window, a.is_global, a.scale);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -676,6 +689,14 @@ __device__ __forceinline__ bool dec_slot_valid(long long s, long long pos, int n
   return pos - back >= n_meta;
 }
 
+// Whether key slot s takes part in the decode attention of the query at `pos`: inside the
+// slots the query may read and holding a visible position.  Both decode kernels mask with
+// this predicate.
+__device__ __forceinline__ bool dec_key_valid(long long s, long long nslots, long long pos, int n_meta,
+                                              int window, int is_global) {
+  return s < nslots && dec_slot_valid(s, pos, n_meta, window, is_global);
+}
+
 size_t decode_attn_workspace_floats(int B, int H, int dv, long long pos, int n_meta, int window,
                                     int is_global) {
   const long long nslots = dec_slots(pos, n_meta, window, is_global);
@@ -715,7 +736,7 @@ __global__ void __launch_bounds__(128)
     attn_decode_partial_kernel(const T *__restrict__ q, const T *__restrict__ kc,
                                const T *__restrict__ vc, float *__restrict__ part, int H, int Hkv,
                                int dqk, int dv, int cap, long long pos, int n_meta, int window,
-                               int is_global, float scale_log2, int nsplit) {
+                               int is_global, float scale_log2, int nsplit, long long wlim) {
   constexpr int V = 16 / sizeof(T);
   extern __shared__ __align__(128) uint8_t dsm[];
   T *sk = reinterpret_cast<T *>(dsm);                               // [DEC_CHUNK][dqk]
@@ -750,14 +771,14 @@ __global__ void __launch_bounds__(128)
     qs[r][d] = Store<T>::to_f(q[(long long)b * H * dqk + (g * rep + r) * dqk + d]) * scale_log2;
   }
   __syncthreads();
-  bool ok = mbar_wait(&bar, 0, &g_err_attn);
-  if (!ok && tid == 0) mbar_wait_drain(&bar, 0, &g_err_attn);  // no copy outlives the CTA
+  bool ok = mbar_wait(&bar, 0, &g_err_attn, wlim);
+  if (!ok && tid == 0) mbar_wait_drain(&bar, 0, &g_err_attn, wlim);  // no copy outlives the CTA
   __syncthreads();
   // scores: two threads per key, each half of the head dim (16-byte pieces read in a
   // rotated order, conflict-free), combined by a shuffle
   {
     const int key = tid >> 1, part_ = tid & 1;
-    const bool valid = ok && key < ns && dec_slot_valid(s0 + key, pos, n_meta, window, is_global);
+    const bool valid = ok && dec_key_valid(s0 + key, nslots, pos, n_meta, window, is_global);
     float acc[DEC_MAXREP];
 #pragma unroll
     for (int r = 0; r < DEC_MAXREP; ++r) acc[r] = 0.f;
@@ -936,7 +957,7 @@ __global__ void __launch_bounds__(128)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                           const __nv_bfloat16 *__restrict__ q, float *__restrict__ part, int H,
                           int Hkv, long long pos, int n_meta, int window, int is_global,
-                          float scale_log2, long long n_items, long long per) {
+                          float scale_log2, long long n_items, long long per, long long wlim) {
   using namespace dtc;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t *sm = dsm_raw + ((1024 - (smem_u32(dsm_raw) & 1023)) & 1023);
@@ -997,11 +1018,10 @@ __global__ void __launch_bounds__(128)
       }
     }
     const int st = k & 1;
-    ok = mbar_wait(&full[st], uint32_t(k >> 1) & 1u, &g_err_attn);
+    ok = mbar_wait(&full[st], uint32_t(k >> 1) & 1u, &g_err_attn, wlim);
     if (__syncthreads_or(!ok)) { ok = false; break; }
     const uint32_t kb = smem_u32(sm + st * STAGE), vb = kb + K_BYTES;
     const long long s0 = (long long)chunk * SLOTS;
-    const int ns = (int)min((long long)SLOTS, nslots - s0);
     // ---- S = Q K^T for this warp's 32 keys (4 n-tiles of 8 keys) ----
     float sacc[4][4];
 #pragma unroll
@@ -1027,7 +1047,7 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int key = warp * 32 + nt * 8 + 2 * gc + e;
-        const bool valid = key < ns && dec_slot_valid(s0 + key, pos, n_meta, window, is_global);
+        const bool valid = dec_key_valid(s0 + key, nslots, pos, n_meta, window, is_global);
         const float x = valid ? sacc[nt][e] * scale_log2 : -INFINITY;
         sacc[nt][e] = x;
         mx = fmaxf(mx, x);
@@ -1108,7 +1128,7 @@ __global__ void __launch_bounds__(128)
   }
   if (!ok && tid == 0) {
     // copies issued past the failed wait must land before the CTA leaves
-    for (int kk = k; kk < issued; ++kk) mbar_wait_drain(&full[kk & 1], uint32_t(kk >> 1) & 1u, &g_err_attn);
+    for (int kk = k; kk < issued; ++kk) mbar_wait_drain(&full[kk & 1], uint32_t(kk >> 1) & 1u, &g_err_attn, wlim);
   }
 }
 
@@ -1187,9 +1207,13 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
     cudaGetDevice(&dev);
     if (!attr_set.done(dev)) {
       const int most = DEC_CHUNK * (128 + 256) * 4;
-      cudaFuncSetAttribute(attn_decode_partial_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, most);
-      cudaFuncSetAttribute(attn_decode_partial_kernel<__nv_bfloat16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, most);
+      if (cudaFuncSetAttribute(attn_decode_partial_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               most) != cudaSuccess ||
+          cudaFuncSetAttribute(attn_decode_partial_kernel<__nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, most) != cudaSuccess) {
+        set_error("cudaFuncSetAttribute(decode attention smem) failed");
+        return HYMBA_ERR_CUDA;
+      }
       attr_set.mark(dev);
     }
   }
@@ -1198,8 +1222,11 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
     int dev = 0;
     cudaGetDevice(&dev);
     if (!attr_tc.done(dev)) {
-      cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           dtc::smem_bytes(dtc::MAXREP));
+      if (cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               dtc::smem_bytes(dtc::MAXREP)) != cudaSuccess) {
+        set_error("cudaFuncSetAttribute(decode attention smem) failed");
+        return HYMBA_ERR_CUDA;
+      }
       attr_tc.mark(dev);
     }
     CUtensorMap tk, tv;
@@ -1220,7 +1247,7 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
     const long long per = (n_items + grid_tc - 1) / grid_tc;
     attn_decode_tc_kernel<<<(unsigned)((n_items + per - 1) / per), 128, dtc::smem_bytes(rep), s>>>(
         tk, tv, (const __nv_bfloat16 *)a.q, a.partial, a.H, a.Hkv, a.pos, a.n_meta, a.window,
-        a.is_global, sl2, n_items, per);
+        a.is_global, sl2, n_items, per, wait_limit_cycles());
     if (a.fuse_later) {
       a.nchunks_out = nchunks;
       a.per_out = per;
@@ -1239,13 +1266,14 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
   } else if (dt == HYMBA_BF16) {
     attn_decode_partial_kernel<__nv_bfloat16><<<grid, 128, dsmem, s>>>(
         (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k_cache, (const __nv_bfloat16 *)a.v_cache,
-        a.partial, a.H, a.Hkv, a.dqk, a.dv, a.cap, a.pos, a.n_meta, a.window, a.is_global, sl2, nsplit);
+        a.partial, a.H, a.Hkv, a.dqk, a.dv, a.cap, a.pos, a.n_meta, a.window, a.is_global, sl2, nsplit,
+        wait_limit_cycles());
     attn_decode_combine_kernel<__nv_bfloat16><<<a.B * a.H, 128, 0, s>>>(
         a.partial, (__nv_bfloat16 *)a.o, a.H, a.dv, nsplit);
   } else {
     attn_decode_partial_kernel<float><<<grid, 128, dsmem, s>>>(
         (const float *)a.q, (const float *)a.k_cache, (const float *)a.v_cache, a.partial, a.H,
-        a.Hkv, a.dqk, a.dv, a.cap, a.pos, a.n_meta, a.window, a.is_global, sl2, nsplit);
+        a.Hkv, a.dqk, a.dv, a.cap, a.pos, a.n_meta, a.window, a.is_global, sl2, nsplit, wait_limit_cycles());
     attn_decode_combine_kernel<float><<<a.B * a.H, 128, 0, s>>>(a.partial, (float *)a.o, a.H,
                                                                  a.dv, nsplit);
   }
@@ -1253,6 +1281,39 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error("decode attention launch failed: %s", cudaGetErrorString(e));
+    return HYMBA_ERR_CUDA;
+  }
+  return HYMBA_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Meta rows of K/V into every sequence (prefill from a precomputed meta cache)
+// ---------------------------------------------------------------------------
+__global__ void kv_broadcast_kernel(const uint4 *__restrict__ src, uint4 *__restrict__ dst, int B,
+                                    long long seq_vecs, long long meta_vecs) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (long long)B * meta_vecs) return;
+  const long long b = i / meta_vecs, r = i - b * meta_vecs;
+  dst[b * seq_vecs + r] = __ldg(src + r);
+}
+
+hymba_status kv_broadcast_meta(const KvBroadcastArgs &a, hymba_dtype dt, cudaStream_t s) {
+  const int es = dt == HYMBA_BF16 ? 2 : 4;
+  const void *src[2] = {a.k_meta, a.v_meta};
+  void *dst[2] = {a.k_seq, a.v_seq};
+  const int width[2] = {a.kw, a.vw};
+  for (int t = 0; t < 2; ++t) {
+    const long long row_bytes = (long long)width[t] * es;  // a multiple of 16 (validated by the caller)
+    const long long meta_vecs = (long long)a.m * row_bytes / 16, seq_vecs = (long long)a.L * row_bytes / 16;
+    const long long n = (long long)a.B * meta_vecs;
+    if (n == 0) continue;
+    kv_broadcast_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const uint4 *>(src[t]), reinterpret_cast<uint4 *>(dst[t]), a.B, seq_vecs, meta_vecs);
+    note_launch(1);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("meta K/V broadcast launch failed: %s", cudaGetErrorString(e));
     return HYMBA_ERR_CUDA;
   }
   return HYMBA_OK;
@@ -1318,9 +1379,32 @@ hymba_status kv_cache_emit(const KvEmitArgs &a, hymba_dtype dt, cudaStream_t s) 
 }
 
 // ---------------------------------------------------------------------------
-// Mask bitmap dump (same predicate and tile classification as the kernels).
+// Mask dumps for bit-exact checks, produced by the kernels' own masking code.
 // ---------------------------------------------------------------------------
-__global__ void mask_bits_kernel(int L, int n_meta, int window, int is_global, uint32_t *bits) {
+// Tensor-core prefill kernel: a key of row i is visible iff its 128-key tile is among the
+// tiles fa_tiles() streams for the row's query-tile pair, the tile is not skipped by its
+// class, and, in a partially visible tile, its column is in the keep-mask the softmax
+// applies.  One thread per (row, 32-key word).
+__global__ void mask_bits_tc_kernel(int L, int n_meta, int window, int is_global, uint32_t *bits) {
+  const int words = (L + 31) / 32;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)L * words) return;
+  const int i = int(idx / words), w = int(idx % words);
+  const int qtile = i / fa::QT, kt = (w * 32) / fa::KT;
+  const FaTiles t = fa_tiles(qtile & ~1, L, 0, n_meta, window, is_global);
+  bool streamed = false;
+  for (int k = t.first(); k <= t.hi; k = t.next(k)) streamed |= (k == kt);
+  uint32_t v = 0;
+  if (streamed) {
+    const int cls = fa_tile_class(qtile, kt, L, 0, n_meta, window, is_global);
+    if (cls == 1) v = 0xffffffffu;
+    else if (cls == 2) v = fa_keep32(fa_cols(i, (long long)kt * fa::KT, n_meta, window, is_global),
+                                     (w * 32) % fa::KT);
+  }
+  bits[idx] = v;
+}
+// CUDA-core (fp32) prefill kernel: the per-pair predicate it evaluates.
+__global__ void mask_bits_simt_kernel(int L, int n_meta, int window, int is_global, uint32_t *bits) {
   const int words = (L + 31) / 32;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)L * words) return;
@@ -1328,7 +1412,7 @@ __global__ void mask_bits_kernel(int L, int n_meta, int window, int is_global, u
   uint32_t v = 0;
   for (int t = 0; t < 32; ++t) {
     const int j = w * 32 + t;
-    if (j < L && mask_allowed(i, j, n_meta, window, is_global)) v |= 1u << t;
+    if (j < L && j <= i && mask_allowed(i, j, n_meta, window, is_global)) v |= 1u << t;
   }
   bits[idx] = v;
 }
@@ -1337,13 +1421,32 @@ __global__ void mask_tiles_kernel(int L, int n_meta, int window, int is_global, 
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= nt * nt) return;
   const int qt = idx / nt, kt = idx % nt;
-  cls[idx] = (uint8_t)seq_tile_class(qt, kt, L, n_meta, window, is_global);
+  cls[idx] = (uint8_t)fa_tile_class(qt, kt, L, 0, n_meta, window, is_global);
+}
+// Decode kernels: bit s of the dump is set iff slot s takes part (dec_key_valid).
+__global__ void decode_mask_kernel(long long pos, int n_meta, int window, int is_global, int capacity,
+                                   uint32_t *bits) {
+  const int words = (capacity + 31) / 32;
+  const int w = blockIdx.x * blockDim.x + threadIdx.x;
+  if (w >= words) return;
+  const long long nslots = dec_slots(pos, n_meta, window, is_global);
+  uint32_t v = 0;
+  for (int e = 0; e < 32; ++e) {
+    const long long s = (long long)w * 32 + e;
+    if (s < capacity && dec_key_valid(s, nslots, pos, n_meta, window, is_global)) v |= 1u << e;
+  }
+  bits[w] = v;
 }
 
-hymba_status mask_bitmap(int L, int n_meta, int window, int is_global, uint32_t *bits,
+hymba_status mask_bitmap(int L, int n_meta, int window, int is_global, int path, uint32_t *bits,
                          uint8_t *tile_class, cudaStream_t s) {
   const long long n = (long long)L * ((L + 31) / 32);
-  if (n > 0) mask_bits_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(L, n_meta, window, is_global, bits);
+  if (n > 0) {
+    if (path == 0)
+      mask_bits_tc_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(L, n_meta, window, is_global, bits);
+    else
+      mask_bits_simt_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(L, n_meta, window, is_global, bits);
+  }
   if (tile_class) {
     const int nt = (L + 127) / 128;
     if (nt > 0)
@@ -1353,6 +1456,19 @@ hymba_status mask_bitmap(int L, int n_meta, int window, int is_global, uint32_t 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error("mask bitmap launch failed: %s", cudaGetErrorString(e));
+    return HYMBA_ERR_CUDA;
+  }
+  return HYMBA_OK;
+}
+
+hymba_status decode_mask(long long pos, int n_meta, int window, int is_global, int capacity,
+                         uint32_t *bits, cudaStream_t s) {
+  const int words = (capacity + 31) / 32;
+  decode_mask_kernel<<<(words + 127) / 128, 128, 0, s>>>(pos, n_meta, window, is_global, capacity, bits);
+  note_launch(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("decode mask launch failed: %s", cudaGetErrorString(e));
     return HYMBA_ERR_CUDA;
   }
   return HYMBA_OK;

@@ -19,9 +19,9 @@ namespace hymba {
 #define HYMBA_DEVICE_ERROR_WORD(name) static __device__ unsigned int name = 0u
 
 constexpr unsigned kErrTimeout = 1u;
-// Spin limit of every mbarrier wait, in SM clock cycles (about 0.5 s at 2 GHz).
-// Legitimate waits in these kernels last microseconds.
-constexpr long long kWaitLimitCycles = 1000000000LL;
+// Every mbarrier wait gives up after a limit in SM clock cycles that the launching host
+// code passes to the kernel (wait_limit_cycles(): 1e9 cycles, about 0.5 s at 2 GHz, unless
+// set otherwise).  Legitimate waits in these kernels last microseconds.
 
 // ---------------------------------------------------------------------------
 // Small math helpers
@@ -168,12 +168,13 @@ __host__ __device__ __forceinline__ int mask_tile_class(long long i0, long long 
   return (causal_full && win_full) ? 1 : 2;
 }
 
-// Class of 128-row query tile qt against 128-key tile kt of a sequence of L rows:
-// rows past the sequence are ignored (their outputs are never stored); keys past
-// it are not (they are zero-filled by TMA and must stay masked).
-__host__ __device__ __forceinline__ int seq_tile_class(int qt, int kt, int L, int n_meta,
+// Class of 128-row query tile qt (query positions q_off + 128 qt ...) against 128-key
+// tile kt of a sequence of L positions: rows past the sequence are ignored (their
+// outputs are never stored); keys past it are not (they are zero-filled by TMA and must
+// stay masked).
+__host__ __device__ __forceinline__ int seq_tile_class(int qt, int kt, int L, int q_off, int n_meta,
                                                        int window, int is_global) {
-  const long long i0 = (long long)qt * 128;
+  const long long i0 = (long long)q_off + (long long)qt * 128;
   if (i0 >= L) return 0;
   const long long i1 = (i0 + 127 < L - 1) ? i0 + 127 : L - 1;
   const long long j0 = (long long)kt * 128, j1 = j0 + 127;
@@ -233,18 +234,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitCycles, records kErrTimeout in *err and returns false.
+// Waits for the phase with the given parity to complete.  Gives up after `limit`
+// cycles, records kErrTimeout in *err and returns false.
 // Also gives up at once when another CTA has already recorded a timeout, so a
 // broken pipeline ends after one limit instead of one limit per wave of CTAs.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsigned int *err,
+                                          long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   unsigned spins = 0;
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((++spins & 3u) == 0 && *reinterpret_cast<volatile unsigned *>(err) != 0u) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(err, kErrTimeout);
       return false;
     }
@@ -253,10 +255,11 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, unsign
 
 // Drain wait for the abort path: waits (bounded) for copies or MMAs already
 // issued by this CTA, even when another CTA has recorded an error.
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, unsigned int *err) {
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t *bar, uint32_t parity, unsigned int *err,
+                                                long long limit) {
   long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       atomicOr(err, kErrTimeout);
       return false;
     }
@@ -432,6 +435,30 @@ __device__ __forceinline__ void tmem_wait_ld() {
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Thread-block clusters: rank, cluster-wide barrier, distributed shared memory
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Every thread of every CTA of the cluster arrives (release) and waits (acquire).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// The shared::cluster address of this CTA's shared-memory address saddr in CTA `rank`.
+__device__ __forceinline__ uint32_t map_shared_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ int warp_id() { return threadIdx.x >> 5; }

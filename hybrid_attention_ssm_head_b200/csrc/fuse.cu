@@ -199,29 +199,6 @@ hymba_status fuse_branches(const FuseArgs &a, hymba_dtype dt, cudaStream_t s) {
   return HYMBA_OK;
 }
 
-template <typename T>
-__global__ void convert_kernel(const float *__restrict__ src, T *__restrict__ dst, long long n) {
-  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i < n) dst[i] = Store<T>::from_f(src[i]);
-}
-
-hymba_status convert_f32_to(const float *src, void *dst, long long n, hymba_dtype dt,
-                            cudaStream_t s) {
-  if (n == 0) return HYMBA_OK;
-  const unsigned blocks = (unsigned)((n + 255) / 256);
-  if (dt == HYMBA_BF16)
-    convert_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>(src, (__nv_bfloat16 *)dst, n);
-  else
-    convert_kernel<float><<<blocks, 256, 0, s>>>(src, (float *)dst, n);
-  note_launch(1);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) {
-    set_error("convert launch failed: %s", cudaGetErrorString(e));
-    return HYMBA_ERR_CUDA;
-  }
-  return HYMBA_OK;
-}
-
 // Decode fuse straight from the attention's run partials: CTA = one sequence, warp h =
 // head h, lane = four value columns.  Per head the runs' (max, sum) pairs give the merge
 // weights 2^(m_r - M) / L; the merged O (fp32, four values per lane) stays in registers

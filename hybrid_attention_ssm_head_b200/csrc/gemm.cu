@@ -37,6 +37,13 @@ __device__ __forceinline__ int find_seg(const Epilogue &e, int n) {
 
 // Column `local` of a segment -> (group, offset in group) without a division on the
 // common layouts: one group, or a power-of-two group width.
+// Destination row of product row m for the segments with a row remap.
+__device__ __forceinline__ long long remap_row(const Epilogue &e, long long m) {
+  if (e.rmap_rows <= 0) return m;
+  const unsigned q = (unsigned)m / (unsigned)e.rmap_rows, r = (unsigned)m - q * (unsigned)e.rmap_rows;
+  return (long long)q * e.rmap_stride + r + e.rmap_off;
+}
+
 __device__ __forceinline__ long long seg_offset(const EpiSeg &g, long long m, int local) {
   int grp, lin;
   if (g.inner >= g.col1 - g.col0) {
@@ -60,9 +67,36 @@ __device__ __forceinline__ float epi_act(const Epilogue &e, int n, float v) {
   return v;
 }
 
-__device__ __forceinline__ void epi_store_scalar(const Epilogue &e, long long m, int n, float v) {
+// Position of product row m for the rotary embedding.
+__device__ __forceinline__ int rope_pos(const Epilogue &e, long long m) {
+  if (!e.rope_tab) return 0;
+  return (int)((unsigned)m % (unsigned)e.rope_rows) + e.rope_off;
+}
+// Rotates the column pairs of v[0..2*NP) (columns n, n+1, ... of segment g, n even) by the
+// rotary angles of position pos.
+template <int NP>
+__device__ __forceinline__ void rope_rotate(const Epilogue &e, const EpiSeg &g, int n, int pos, float *v) {
+  const int hp = e.rope_hd >> 1;
+  const int pair0 = ((n - g.col0) & (e.rope_hd - 1)) >> 1;
+  const float2 *cs = e.rope_tab + (long long)pos * hp + pair0;
+#pragma unroll
+  for (int i = 0; i < NP; ++i) {
+    const float2 c = __ldg(cs + i);
+    const float a = v[2 * i], b = v[2 * i + 1];
+    v[2 * i] = a * c.x - b * c.y;
+    v[2 * i + 1] = fmaf(a, c.y, b * c.x);
+  }
+}
+
+// The segment's own activation (not on split-K partial sums).
+__device__ __forceinline__ float seg_act(const EpiSeg &g, float v) { return g.act == 2 ? silu_f(v) : v; }
+
+// m: the product row; mk: its remapped row (used by segments with rmap).
+__device__ __forceinline__ void epi_store_scalar(const Epilogue &e, long long m, long long mk, int n,
+                                                 float v) {
   const EpiSeg &g = e.seg[find_seg(e, n)];
-  const long long off = seg_offset(g, m, n - g.col0);
+  const long long off = seg_offset(g, g.rmap ? mk : m, n - g.col0);
+  if (!e.atomic) v = seg_act(g, v);
   if (e.atomic) {
     atomicAdd(reinterpret_cast<float *>(g.ptr) + off, v);
   } else if (g.f32) {
@@ -73,15 +107,22 @@ __device__ __forceinline__ void epi_store_scalar(const Epilogue &e, long long m,
 }
 
 // Stores 8 consecutive columns n..n+7 of row m (values already activated).
-__device__ __forceinline__ void epi_store8(const Epilogue &e, long long m, int n, int N,
-                                           const float (&v)[8]) {
+__device__ __forceinline__ void epi_store8(const Epilogue &e, long long m, long long mk, int rp, int n,
+                                           int N, const float (&v_raw)[8]) {
   if (n >= N) return;
   const EpiSeg &g = e.seg[find_seg(e, n)];
+  float v_in[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v_in[i] = v_raw[i];
+  if (g.rope && !e.atomic && n + 8 <= g.col1) rope_rotate<4>(e, g, n, rp, v_in);
   int local = n - g.col0;
   bool vec = !e.atomic && g.vec_ok && (n + 8 <= N) && (n + 8 <= g.col1) && (local % 8 == 0) &&
              ((local % g.inner) + 8 <= g.inner);
   if (vec) {
-    const long long off = seg_offset(g, m, local);
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = seg_act(g, v_in[i]);
+    const long long off = seg_offset(g, g.rmap ? mk : m, local);
     if (g.f32) {
       float *p = reinterpret_cast<float *>(g.ptr) + off;
       st_global_v4(p, __float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]),
@@ -97,7 +138,7 @@ __device__ __forceinline__ void epi_store8(const Epilogue &e, long long m, int n
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    if (n + i < N) epi_store_scalar(e, m, n + i, v[i]);
+    if (n + i < N) epi_store_scalar(e, m, mk, n + i, v_in[i]);
 }
 
 // Bias of columns n0..n0+15 (zero past N).
@@ -121,8 +162,8 @@ __device__ __forceinline__ void epi_bias16(const Epilogue &e, int n0, int N, flo
 // 16 consecutive product columns n0..n0+15 of row m from raw fp32 accumulator bits,
 // plus the bias (when the epilogue has one).  One segment lookup per chunk on the
 // common path.
-__device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, int n0, int N,
-                                            const uint32_t (&r)[16], const float (&bias)[16]) {
+__device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, long long mk, int rp, int n0,
+                                            int N, const uint32_t (&r)[16], const float (&bias)[16]) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
@@ -143,7 +184,12 @@ __device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, int 
   const int local = n0 - g.col0;
   if (full && !e.atomic && g.vec_ok && n0 + 16 <= g.col1 &&
       (g.inner >= g.col1 - g.col0 || ((g.inner & 15) == 0 && (local & 15) == 0))) {
-    const long long off = seg_offset(g, m, local);
+    if (g.act) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] = seg_act(g, v[i]);
+    }
+    if (g.rope) rope_rotate<8>(e, g, n0, rp, v);
+    const long long off = seg_offset(g, g.rmap ? mk : m, local);
     if (g.f32) {
       float *p = reinterpret_cast<float *>(g.ptr) + off;
       if (g.vec32) {
@@ -180,8 +226,8 @@ __device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, int 
     a[i] = v[i];
     b[i] = v[8 + i];
   }
-  epi_store8(e, m, n0, N, a);
-  epi_store8(e, m, n0 + 8, N, b);
+  epi_store8(e, m, mk, rp, n0, N, a);
+  epi_store8(e, m, mk, rp, n0 + 8, N, b);
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -209,7 +255,7 @@ struct TcCfg {
   static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
   static constexpr uint32_t IDESC = make_idesc(BN, ELEM == 2 ? 1 : 2, 0, 0);
-  static constexpr int BAR_BYTES = (2 * STAGES + 4) * 8 + 16;  // + static smem: Epilogue
+  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8 + 16;  // + static smem: Epilogue
   static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0, N <= 256");
 };
@@ -217,7 +263,7 @@ struct TcCfg {
 template <int BN, int ELEM>
 __global__ void __launch_bounds__(576, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   int M, int N, int K, int ksplit, Epilogue epi) {
+                   int M, int N, int K, int ksplit, Epilogue epi, long long wlim, int stall) {
   using C = TcCfg<BN, ELEM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -227,7 +273,8 @@ __global__ void __launch_bounds__(576, 1)
   uint64_t *empty = full + C::STAGES;
   uint64_t *tfull = empty + C::STAGES;
   uint64_t *tempty = tfull + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(tempty + 2);
+  uint64_t *never = tempty + 2;  // nothing arrives on it: the wait of a stalled MMA warp
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(never + 1);
   // Segment table in shared memory: per-column routing then indexes smem, not
   // kernel parameters.
   __shared__ Epilogue s_epi;
@@ -250,6 +297,7 @@ __global__ void __launch_bounds__(576, 1)
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 512);
     }
+    mbar_init(never, 1);
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
@@ -281,7 +329,7 @@ __global__ void __launch_bounds__(576, 1)
         const int mt = int(tile / n_tiles), nt = int(tile % n_tiles);
         const int kb0 = ks * kb_per, kb1 = min(kblocks, kb0 + kb_per);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, &g_err_gemm)) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, &g_err_gemm, wlim)) {
             ok = false;
             break;
           }
@@ -298,7 +346,7 @@ __global__ void __launch_bounds__(576, 1)
       if (!ok) {
         // Leave no copy in flight into shared memory that is about to be released.
         for (int s = 0; s < C::STAGES; ++s)
-          if (issued[s]) mbar_wait_drain(&full[s], (issued[s] - 1) & 1u, &g_err_gemm);
+          if (issued[s]) mbar_wait_drain(&full[s], (issued[s] - 1) & 1u, &g_err_gemm, wlim);
       }
     }
   } else if (warp == 1) {
@@ -308,19 +356,21 @@ __global__ void __launch_bounds__(576, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
-      bool ok = true;
+      // A stalled launch (the bounded-wait test) waits for an arrival that never comes
+      // instead of issuing its first MMA; it then takes the abort path below.
+      bool ok = !stall || mbar_wait(never, 0, &g_err_gemm, wlim);
       for (long long u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const int ks = int(u % ksplit);
         const int kb0 = ks * kb_per, kb1 = min(kblocks, kb0 + kb_per);
         if (kb0 >= kb1) continue;
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, &g_err_gemm)) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, &g_err_gemm, wlim)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&full[stage], phase, &g_err_gemm)) {
+          if (!mbar_wait(&full[stage], phase, &g_err_gemm, wlim)) {
             ok = false;
             break;
           }
@@ -352,7 +402,7 @@ __global__ void __launch_bounds__(576, 1)
       if (!ok) {
         // Drain issued MMAs before tensor memory is released.
         mma_commit(&tfull[acc]);
-        mbar_wait_drain(&tfull[acc], acc_phase, &g_err_gemm);
+        mbar_wait_drain(&tfull[acc], acc_phase, &g_err_gemm, wlim);
       }
     }
   } else {
@@ -371,9 +421,11 @@ __global__ void __launch_bounds__(576, 1)
       if (kb0 >= kb1) continue;
       const int mt = int(tile / n_tiles), nt = int(tile % n_tiles);
       constexpr int NCH = (BN + 63) / 64;
-      if (!mbar_wait(&tfull[acc], acc_phase, &g_err_gemm)) break;
+      if (!mbar_wait(&tfull[acc], acc_phase, &g_err_gemm, wlim)) break;
       tc_fence_after();
       const long long m = (long long)mt * C::BM + row;
+      const long long mk = remap_row(s_epi, m);
+      const int rp = rope_pos(s_epi, m);
       const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
       // this warp's chunks in rounds of at most two loads; the accumulator is handed back
       // to the MMA warp after the last round's loads, before its activation math and stores
@@ -398,7 +450,7 @@ __global__ void __launch_bounds__(576, 1)
           if (k0 + k < NCH && c < BN && n0 < N && m < M) {
             float bias[16];
             if (s_epi.bias) epi_bias16(s_epi, n0, N, bias);
-            epi_store16(s_epi, m, n0, N, r[k], bias);
+            epi_store16(s_epi, m, mk, rp, n0, N, r[k], bias);
           }
         }
       }
@@ -425,6 +477,255 @@ static int num_sms() {
   return n > 0 ? n : 148;
 }
 
+// ---------------------------------------------------------------------------
+// Weight-streaming GEMM for a few activation rows (the decode step):
+//   out[b, n] = epi( sum_k X[b, k] W[n, k] ),   b < B <= 256 (one tile of rows)
+// computed transposed on the tensor cores, D[n, b] = W[n, :] . X[b, :], with the weights
+// as the M = 128 operand: a cluster of CL CTAs shares one 128-row weight tile, each CTA
+// streaming a disjoint 1/CL of K, so every weight byte is read from HBM once by one SM
+// while the few activation rows come from L2.  The CL partial accumulators are reduced
+// through distributed shared memory: every CTA puts its partial tile in its own shared
+// memory, then CTA r sums the CL partials of weight rows [r*128/CL, (r+1)*128/CL) for all
+// activation rows and stores them through the routed epilogue (one thread per activation
+// row, 16 output columns per store).  No atomics, no second pass.
+//   warp 0, one lane : TMA producer (weight tile and activation rows, 4-stage ring)
+//   warp 1, one lane : tcgen05.mma (M = 128, N = BN) into tensor memory
+//   all four warps   : tensor memory -> shared partial tile; the cluster reduction
+// ---------------------------------------------------------------------------
+namespace wsg {
+constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int W_BYTES = BM * 128;
+template <int BN>
+struct Cfg {
+  static constexpr int X_BYTES = BN * 128;
+  static constexpr int STAGE = W_BYTES + X_BYTES;
+  static constexpr int PSTRIDE = BN + 1;  // floats per partial row: conflict-free both ways
+  static constexpr int P_BYTES = BM * PSTRIDE * 4;
+  static constexpr int BODY = STAGE * STAGES > P_BYTES ? STAGE * STAGES : P_BYTES;
+  static constexpr int SMEM = BODY + (2 * STAGES + 1) * 8 + 16 + 1024;
+  static constexpr uint32_t IDESC = make_idesc(BN, 1, 0, 0);
+};
+}  // namespace wsg
+
+template <int BN, int CL>
+__global__ void __launch_bounds__(128, 1)
+    gemm_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int Nout,
+                   int B, int K, Epilogue epi, long long wlim) {
+  using C = wsg::Cfg<BN>;
+  using namespace wsg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BODY);
+  uint64_t *empty = full + STAGES;
+  uint64_t *done = empty + STAGES;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(done + 1);
+  float *part = reinterpret_cast<float *>(smem);  // [BM][PSTRIDE], over the stages once the MMAs are done
+  __shared__ Epilogue s_epi;
+  const int warp = warp_id(), lane = lane_id(), tid = threadIdx.x;
+  const uint32_t rank = cluster_ctarank();
+  const int mt = blockIdx.y;
+  const int kblocks = (K + BK - 1) / BK;
+  const int kb_per = (kblocks + CL - 1) / CL;
+  const int kb0 = min(kblocks, (int)rank * kb_per), kb1 = min(kblocks, kb0 + kb_per);
+  if (tid == 0) {
+    s_epi = epi;
+    for (int st = 0; st < STAGES; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
+    }
+    mbar_init(done, 1);
+    fence_barrier_init();
+    tma_prefetch_desc(&tmW);
+    tma_prefetch_desc(&tmX);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tmem_relinquish();
+  }
+  if (epi.zero) {  // accumulators of a later kernel of the same step start at zero
+    const long long nct = (long long)gridDim.x * gridDim.y, bid = (long long)blockIdx.y * gridDim.x + blockIdx.x;
+    for (long long i = bid * 128 + tid; i < epi.zero_n; i += nct * 128) epi.zero[i] = 0.f;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer ----------------
+    int st = 0;
+    uint32_t ph = 0, issued[STAGES] = {0, 0, 0, 0};
+    bool ok = true;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&empty[st], ph ^ 1u, &g_err_gemm, wlim)) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx(&full[st], C::STAGE);
+      tma_load_2d(smem + st * C::STAGE, &tmW, &full[st], kb * BK, mt * BM);
+      tma_load_2d(smem + st * C::STAGE + W_BYTES, &tmX, &full[st], kb * BK, 0);
+      ++issued[st];
+      if (++st == STAGES) {
+        st = 0;
+        ph ^= 1u;
+      }
+    }
+    if (!ok)  // no copy may still be landing in the stages that the partial tile reuses
+      for (int x = 0; x < STAGES; ++x)
+        if (issued[x]) mbar_wait_drain(&full[x], (issued[x] - 1) & 1u, &g_err_gemm, wlim);
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    int st = 0;
+    uint32_t ph = 0;
+    for (int kb = kb0; kb < kb1; ++kb) {
+      if (!mbar_wait(&full[st], ph, &g_err_gemm, wlim)) break;
+      tc_fence_after();
+      const uint32_t a = smem_u32(smem + st * C::STAGE), b = a + W_BYTES;
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        mma_bf16_ss(tmem, make_sdesc(a + 32 * k, 16, 1024), make_sdesc(b + 32 * k, 16, 1024), C::IDESC,
+                    (kb > kb0 || k > 0) ? 1u : 0u);
+      mma_commit(&empty[st]);
+      if (++st == STAGES) {
+        st = 0;
+        ph ^= 1u;
+      }
+    }
+    mma_commit(done);  // arrives once every MMA issued above has finished (at once if none)
+  }
+  __syncwarp();
+  const bool acc_ok = mbar_wait(done, 0, &g_err_gemm, wlim) && kb1 > kb0;
+  __syncthreads();  // the producer has drained: the stages are free for the partial tile
+  tc_fence_after();
+  {
+    // tensor memory -> this CTA's partial tile, part[row of W][activation row]
+    const int f = warp * 32 + lane;
+    const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16);
+#pragma unroll 1
+    for (int c = 0; c < BN; c += 32) {
+      uint32_t r[32];
+      tmem_ld32(t_row + c, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 32; ++j) part[f * C::PSTRIDE + c + j] = acc_ok ? __uint_as_float(r[j]) : 0.f;
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // every partial tile of the cluster is written
+  {
+    constexpr int F = BM / CL;  // weight rows this CTA reduces and stores
+    const uint32_t pbase = smem_u32(part);
+#pragma unroll 1
+    for (int b = tid; b < B && b < BN; b += 128) {
+      const long long m = b;
+      const long long mk = remap_row(s_epi, m);
+      const int rp = rope_pos(s_epi, m);
+#pragma unroll 1
+      for (int j = 0; j < F; j += 16) {
+        const int f0 = (int)rank * F + j;
+        const int n0 = mt * BM + f0;
+        if (n0 >= Nout) break;
+        float acc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int c = 0; c < CL; ++c) {
+          const uint32_t remote = map_shared_rank(pbase, (uint32_t)c);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            acc[i] += ld_shared_cluster_f32(remote + (uint32_t)(((f0 + i) * C::PSTRIDE + b) * 4));
+        }
+        uint32_t bits[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) bits[i] = __float_as_uint(acc[i]);
+        float bias[16];
+        if (s_epi.bias) epi_bias16(s_epi, n0, Nout, bias);
+        epi_store16(s_epi, m, mk, rp, n0, Nout, bits, bias);
+      }
+    }
+  }
+  cluster_sync();  // no CTA leaves while the others still read its partial tile
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
+template <int BN, int CL>
+static hymba_status launch_ws(const GemmArgs &g, cudaStream_t s) {
+  using C = wsg::Cfg<BN>;
+  static DeviceOnce attr_set;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set.done(dev)) {
+    if (cudaFuncSetAttribute(gemm_ws_kernel<BN, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess) {
+      set_error("cudaFuncSetAttribute(weight-streaming gemm smem %d) failed", C::SMEM);
+      return HYMBA_ERR_CUDA;
+    }
+    attr_set.mark(dev);
+  }
+  CUtensorMap tw, tx;
+  // W = the product's B operand [N, K]; X = its A operand [M, K] (the activation rows)
+  const uint64_t dw[2] = {(uint64_t)g.K, (uint64_t)g.N}, sw[1] = {(uint64_t)g.ldb * 2};
+  const uint32_t bw[2] = {(uint32_t)wsg::BK, (uint32_t)wsg::BM};
+  const uint64_t dx[2] = {(uint64_t)g.K, (uint64_t)g.M}, sx[1] = {(uint64_t)g.lda * 2};
+  const uint32_t bx[2] = {(uint32_t)wsg::BK, (uint32_t)BN};
+  if (!make_tmap(&tw, g.B, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dw, sw, bw)) return HYMBA_ERR_CUDA;
+  if (!make_tmap(&tx, g.A, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dx, sx, bx)) return HYMBA_ERR_CUDA;
+  const int m_tiles = (g.N + wsg::BM - 1) / wsg::BM;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL, m_tiles, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_ws_kernel<BN, CL>, tw, tx, g.N, g.M, g.K, g.epi,
+                                     wait_limit_cycles());
+  note_launch(1);
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("weight-streaming gemm launch failed: %s", cudaGetErrorString(e));
+    return HYMBA_ERR_CUDA;
+  }
+  return HYMBA_OK;
+}
+
+template <int BN>
+static hymba_status launch_ws_cl(const GemmArgs &g, int cl, cudaStream_t s) {
+  switch (cl) {
+    case 8: return launch_ws<BN, 8>(g, s);
+    case 4: return launch_ws<BN, 4>(g, s);
+    case 2: return launch_ws<BN, 2>(g, s);
+    default: return launch_ws<BN, 1>(g, s);
+  }
+}
+
+// Decode-sized products (at most 256 activation rows, bf16, no split-K or atomic epilogue).
+hymba_status gemm_ws(const GemmArgs &g, cudaStream_t s) {
+  if (g.elem != 2 || g.M < 1 || g.M > 256 || g.ksplit != 1 || g.epi.atomic || g.stall) {
+    set_error("gemm_ws: unsupported product (bf16, <= 256 rows, no split-K)");
+    return HYMBA_ERR_UNSUPPORTED;
+  }
+  // cluster size: enough CTAs to put most SMs on the weight stream, at most one K block each
+  const int m_tiles = (g.N + wsg::BM - 1) / wsg::BM;
+  const int kblocks = (g.K + wsg::BK - 1) / wsg::BK;
+  int cl = 1;
+  while (cl < 8 && m_tiles * cl * 2 <= num_sms() + num_sms() / 8 && kblocks >= cl * 2) cl *= 2;
+  if (g.M <= 32) return launch_ws_cl<32>(g, cl, s);
+  if (g.M <= 64) return launch_ws_cl<64>(g, cl, s);
+  if (g.M <= 128) return launch_ws_cl<128>(g, cl, s);
+  return launch_ws_cl<256>(g, cl, s);
+}
+
 template <int BN, int ELEM>
 static hymba_status launch_tc(const GemmArgs &g, cudaStream_t s) {
   using C = TcCfg<BN, ELEM>;
@@ -449,7 +750,8 @@ static hymba_status launch_tc(const GemmArgs &g, cudaStream_t s) {
   if (!make_tmap(&tb, g.B, dt, 2, db, sb, bb)) return HYMBA_ERR_CUDA;
   const long long tiles = (long long)((g.M + 127) / 128) * ((g.N + BN - 1) / BN) * g.ksplit;
   const int grid = (int)std::min<long long>(tiles, num_sms());
-  gemm_tc_kernel<BN, ELEM><<<grid, 576, C::SMEM, s>>>(ta, tb, g.M, g.N, g.K, g.ksplit, g.epi);
+  gemm_tc_kernel<BN, ELEM><<<grid, 576, C::SMEM, s>>>(ta, tb, g.M, g.N, g.K, g.ksplit, g.epi,
+                                                     wait_limit_cycles(), g.stall);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -529,14 +831,25 @@ __global__ void __launch_bounds__(256)
   for (int i = 0; i < 4; ++i) {
     const long long m = m0 + ty * 4 + i;
     if (m >= M) continue;
+    float v[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx * 4 + j;
-      if (n < N) {
-        float v = acc[i][j];
-        if (!epi.atomic) v = epi_act(epi, n, v);
-        epi_store_scalar(epi, m, n, v);
+      v[j] = (n < N && !epi.atomic) ? epi_act(epi, n, acc[i][j]) : acc[i][j];
+    }
+    // rotary pairs (2i, 2i+1) are both in this thread's four columns
+#pragma unroll
+    for (int j = 0; j < 4; j += 2) {
+      const int n = n0 + tx * 4 + j;
+      if (n + 1 < N && !epi.atomic) {
+        const EpiSeg &g = epi.seg[find_seg(epi, n)];
+        if (g.rope && n + 1 < g.col1) rope_rotate<1>(epi, g, n, rope_pos(epi, m), v + j);
       }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = n0 + tx * 4 + j;
+      if (n < N) epi_store_scalar(epi, m, remap_row(epi, m), n, v[j]);
     }
   }
 }

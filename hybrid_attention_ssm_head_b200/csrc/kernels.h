@@ -11,13 +11,19 @@
 
 namespace hymba {
 
-// One bit per device (ordinal mod 32), set once a kernel's launch attributes have been
-// configured on that device.  Atomic, so that first launches from several host threads at
-// once are well defined: each may then set the (idempotent) attribute.
+// One flag per device ordinal, set once a kernel's launch attributes have been configured
+// on that device.  Atomic, so that first launches from several host threads at once are
+// well defined: each may then set the (idempotent) attribute.  Ordinals past the table
+// are never marked, so their attributes are set on every launch.
 struct DeviceOnce {
-  std::atomic<unsigned> bits{0};
-  bool done(int dev) const { return bits.load(std::memory_order_acquire) & (1u << (dev & 31)); }
-  void mark(int dev) { bits.fetch_or(1u << (dev & 31), std::memory_order_acq_rel); }
+  static constexpr int kMaxDevices = 256;
+  std::atomic<bool> flag[kMaxDevices] = {};
+  bool done(int dev) const {
+    return dev >= 0 && dev < kMaxDevices && flag[dev].load(std::memory_order_acquire);
+  }
+  void mark(int dev) {
+    if (dev >= 0 && dev < kMaxDevices) flag[dev].store(true, std::memory_order_release);
+  }
 };
 
 
@@ -33,11 +39,25 @@ struct EpiSeg {
   int f32;
   int vec_ok;  // 16-byte aligned rows/groups: 8-column vector stores allowed
   int vec32;   // 32-byte aligned rows/groups: whole-sector (256-bit) stores allowed
+  int act;     // activation of this segment's columns: 0 none, 2 SiLU (after the GEMM's own)
+  int rmap;    // 1: rows go through the epilogue's row remap
+  int rope;    // 1: rotary position embedding of this segment's heads (pairs of columns)
 };
 
 struct Epilogue {
   EpiSeg seg[5];
   int nseg;
+  // Row remap of the segments with rmap set: product row r is stored at row
+  // (r / rmap_rows) * rmap_stride + r % rmap_rows + rmap_off of that segment (rows of
+  // sequences that sit after a prefix of rmap_off rows in a longer destination).
+  int rmap_rows;
+  long long rmap_stride;
+  int rmap_off;
+  // Rotary position embedding of the segments with rope set: product row r is at position
+  // r % rope_rows + rope_off; column pair i of a head (head width rope_hd, a power of two)
+  // is rotated by rope_tab[pos * rope_hd / 2 + i] = (cos, sin).
+  const float2 *rope_tab;
+  int rope_rows, rope_off, rope_hd;
   const float *bias;  // per product column (nullable)
   int act;            // 0 = identity, 1 = softplus
   int atomic;         // 1 = fp32 atomicAdd into the destination (split-K)
@@ -55,10 +75,14 @@ struct GemmArgs {
   int elem;    // 2: bf16 operands; 4: fp32 operands
   int ksplit;  // >= 1; > 1 requires epi.atomic
   Epilogue epi;
+  int stall;   // tensor-core path: the MMA warp waits for an arrival that never comes
 };
 
 // Tensor-core path (tcgen05 + TMA).  elem 2 -> kind::f16 (bf16), 4 -> kind::tf32.
 hymba_status gemm_tc(const GemmArgs &g, cudaStream_t s);
+// Weight-streaming tensor-core path for at most 256 activation rows (decode): clusters of
+// CTAs split K, partials reduced through distributed shared memory.  bf16 only.
+hymba_status gemm_ws(const GemmArgs &g, cudaStream_t s);
 // fp32 CUDA-core path for the fp32 storage configuration.
 hymba_status gemm_simt_f32(const GemmArgs &g, cudaStream_t s);
 
@@ -70,6 +94,8 @@ struct ConvArgs {
   const float *w;     // [E, K]
   const float *bias;  // [E]
   void *conv_state;   // optional [B, K-1, E]: the last K-1 rows of x
+  const void *hist;   // optional [K-1, E]: the rows before row 0 (the same for every
+                      // sequence; zero rows when null)
   int B, L, E, K;
 };
 hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s);
@@ -77,7 +103,7 @@ hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s);
 struct ScanArgs {
   const void *u;       // [B, L, E]
   const void *delta;   // [B, L, E]
-  const void *z;       // [B, L, E], row stride ld_z
+  const void *z;       // [B, L, E] the gate SiLU(z), row stride ld_z
   long long ld_z;
   const float *bc;     // [B*L, ld_bc] fp32; B at column bc_col, C at bc_col + N
   long long ld_bc;
@@ -86,7 +112,8 @@ struct ScanArgs {
   const float *d_skip; // [E]
   void *y;             // [B, L, E] gated output
   float *h_out;        // optional [B, E, N] final state
-  float *h_in;         // optional [B, E, N] initial state (decode), else zero
+  const float *h_in;   // optional initial state: [E, N] per sequence, h_in_bstride floats
+  long long h_in_bstride;  // apart (0: one state for every sequence); zero when null
   int B, L, E, N;
   float *chunk_ws;     // workspace for the chunked scan (see scan_workspace_floats)
 };
@@ -120,16 +147,27 @@ struct FuseDecodeArgs {
 hymba_status fuse_decode(const FuseDecodeArgs &a, cudaStream_t s);
 
 // ---- attention -----------------------------------------------------------
+// Queries are the positions q_off .. q_off + Lq - 1 of sequences of L = q_off + Lq rows,
+// stored from row 0 of q and o; keys are all L positions.
 struct AttnArgs {
-  const void *q;   // [B, L, H*dqk]
+  const void *q;   // [B, Lq, H*dqk]
   const void *k;   // [B, L, Hkv*dqk]
   const void *v;   // [B, L, Hkv*dv]
-  void *o;         // [B, L, H*dv]
+  void *o;         // [B, Lq, H*dv]
   int B, L, H, Hkv, dqk, dv;
+  int q_off, Lq;
   int n_meta, window, is_global;
   float scale;
 };
 hymba_status attention_prefill(const AttnArgs &a, hymba_dtype dt, cudaStream_t s);
+
+// Copies one sequence's first m rows of K and V (the meta rows) into every sequence.
+struct KvBroadcastArgs {
+  const void *k_meta, *v_meta;  // [m, Hkv*dqk], [m, Hkv*dv]
+  void *k_seq, *v_seq;          // [B, L, Hkv*dqk], [B, L, Hkv*dv]
+  int B, L, m, kw, vw;          // kw, vw: row widths in elements
+};
+hymba_status kv_broadcast_meta(const KvBroadcastArgs &a, hymba_dtype dt, cudaStream_t s);
 
 struct KvEmitArgs {
   const void *k_seq, *v_seq;  // [B, L, Hkv*d]
@@ -163,7 +201,7 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
 struct DecodeSsmArgs {
   const void *x;       // [B, E] x_ssm of the new token, row stride ld_x
   long long ld_x;
-  const void *z;       // [B, E] gate input, row stride ld_z
+  const void *z;       // [B, E] the gate SiLU(z), row stride ld_z
   long long ld_z;
   void *conv_state;    // [B, K-1, E] in/out
   const float *conv_w, *conv_b;  // [E, K], [E]
@@ -178,11 +216,24 @@ struct DecodeSsmArgs {
 };
 hymba_status decode_ssm(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s);
 
-hymba_status mask_bitmap(int L, int n_meta, int window, int is_global, uint32_t *bits,
+// path 0: the tensor-core (bf16) prefill kernel's tile enumeration, tile classes and
+// column keep-masks; path 1: the CUDA-core (fp32) kernel's per-pair predicate.
+hymba_status mask_bitmap(int L, int n_meta, int window, int is_global, int path, uint32_t *bits,
                          uint8_t *tile_class, cudaStream_t s);
+// The decode kernels' slot predicate for the query at `pos`, one bit per slot.
+hymba_status decode_mask(long long pos, int n_meta, int window, int is_global, int capacity,
+                         uint32_t *bits, cudaStream_t s);
+// Rotary table: tab[p * hd/2 + i] = (cos, sin)((pos0 + p) * base^(-2i/hd)), p < npos.
+hymba_status rope_table(float2 *tab, int npos, long long pos0, int hd, float base, cudaStream_t s);
+// exp2 of n floats by the polynomial the attention softmax uses (degree 3 or 5).
+hymba_status exp2_poly_eval(int degree, const float *x, float *y, long long n, cudaStream_t s);
 
-hymba_status convert_f32_to(const float *src, void *dst, long long n, hymba_dtype dt,
-                            cudaStream_t s);
+
+// Cycle limit the kernels' bounded waits are launched with: HYMBA_WAIT_LIMIT from the
+// environment, else hymba_set_wait_limit()'s value, else 1e9; never below 1e5.
+long long wait_limit_cycles();
+// One-shot diagnostic: 1 if the next prefill's output projection is to stall (consumed).
+int take_debug_stall();
 
 // Device error word bit for a bounded wait that gave up.
 constexpr unsigned kErrTimeoutHost = 1u;

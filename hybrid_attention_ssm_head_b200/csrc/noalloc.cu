@@ -1,5 +1,7 @@
 // Decode step without a caller-provided workspace: its scratch lives in a
 // file-scope device buffer, so the call allocates nothing.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "kernels.h"
@@ -12,7 +14,27 @@ static __device__ __align__(256) unsigned char g_decode_scratch[HYMBA_DECODE_STA
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
+// The address is looked up once per device and CUDA context: a context torn down and
+// created again (cudaDeviceReset) maps the module afresh, so the cached address is
+// re-derived whenever the current context is not the one it was taken in.
 void *g_scratch_addr[kMaxDevices] = {};
+void *g_scratch_ctx[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+void *current_context() {
+  static std::once_flag once;
+  static CtxGetCurrentFn fn = nullptr;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
 
 }  // namespace
 
@@ -38,7 +60,9 @@ extern "C" HYMBA_API hymba_status hymba_layer_decode_step_static(hymba_layer *la
   void *scratch = nullptr;
   {
     std::lock_guard<std::mutex> g(g_mu);
-    if (!g_scratch_addr[dev]) {
+    // the runtime makes the device's primary context current on its first call above
+    void *ctx = current_context();
+    if (!g_scratch_addr[dev] || ctx != g_scratch_ctx[dev]) {
       void *p = nullptr;
       const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
       if (e != cudaSuccess || !p) {
@@ -46,6 +70,7 @@ extern "C" HYMBA_API hymba_status hymba_layer_decode_step_static(hymba_layer *la
         return HYMBA_ERR_CUDA;
       }
       g_scratch_addr[dev] = p;
+      g_scratch_ctx[dev] = ctx;
     }
     scratch = g_scratch_addr[dev];
   }

@@ -2,7 +2,8 @@
 //   u = SiLU(causal depthwise conv_K(x_ssm) + b)
 //   h_t = exp(delta_t A) * h_{t-1} + delta_t B_t u_t,   y_t = C_t . h_t + D u_t
 //   y_ssm = y * SiLU(z)
-// [delta, B, C] come from the projection GEMMs; A = -exp(A_log).
+// [delta, B, C] come from the projection GEMMs; A = -exp(A_log).  The gate SiLU(z) is
+// applied by the input projection's epilogue, so the scans read it ready-made.
 //
 // Prefill scan layout: a thread carries two adjacent channels of one sequence with
 // their d_state = 16 states in registers as fp32 pairs (packed fp32x2 FMAs); u,
@@ -119,15 +120,27 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
   const T *x = reinterpret_cast<const T *>(a.x);
   T *u = reinterpret_cast<T *>(a.u);
   const int t0 = tb * kConvTB;
-  uint4 raw[NR];  // raw[r] = x[t0 - 3 + r], zero outside the sequence
+  static_assert(kConvTB >= 3, "the history rows must fall in the first block");
+  uint4 raw[NR];  // raw[r] = x[t0 - 3 + r]: the history rows before row 0, zero past the end
 #pragma unroll
-  for (int r = 0; r < NR; ++r) {  // unconditional loads (clamped row), zeroed afterwards
+  for (int r = 0; r < NR; ++r) {  // unconditional loads (clamped row), replaced afterwards
     const int t = min(max(t0 - 3 + r, 0), a.L - 1);
     raw[r] = __ldg(reinterpret_cast<const uint4 *>(x + ((long long)b * a.L + t) * a.ld_x + c0));
   }
 #pragma unroll
-  for (int r = 0; r < NR; ++r)
-    if (t0 - 3 + r < 0 || t0 - 3 + r >= a.L) raw[r] = make_uint4(0, 0, 0, 0);
+  for (int r = 0; r < 3; ++r) {  // rows before 0 exist only in the first block
+    const int t = t0 - 3 + r;
+    if (t < 0) {
+      const int hr = K - 1 + t;  // history row (oldest first); taps past K are zero
+      raw[r] = (a.hist && hr >= 0)
+                   ? __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const T *>(a.hist) +
+                                                           (long long)hr * a.E + c0))
+                   : make_uint4(0, 0, 0, 0);
+    }
+  }
+#pragma unroll
+  for (int r = 3; r < NR; ++r)
+    if (t0 - 3 + r >= a.L) raw[r] = make_uint4(0, 0, 0, 0);
   // wj[j][i] multiplies x[t - 3 + j] for channel c0 + i (taps right-aligned)
   float wj[4][V], bias[V];
   if (K == 4) {
@@ -339,7 +352,7 @@ __global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
 //     tensor cores (mma.sync m16n8k8, tf32 in, fp32 accumulate; rows 8..15 of the
 //     16-row tile are zero), then thread per channel: delta = softplus(. + b_dt), one
 //     step of the recurrence from the stored state (h_t = exp(delta A) h + delta B u,
-//     y = C . h + D u, gated by SiLU(z)), state written back in place.  W_dt (contiguous
+//     y = C . h + D u, times the gate SiLU(z)), state written back in place.  W_dt (contiguous
 //     rows) and the xdbl rows arrive by cp.async; shared row strides are 4 mod 8 floats,
 //     so the tf32 fragment loads are free of bank conflicts.
 constexpr int kDecScanRows = 8;
@@ -496,7 +509,7 @@ __global__ void __launch_bounds__(128, 3) dec_dt_scan_kernel(DecodeSsmArgs a) {
       acc = fmaf(C4.x, hv[q].x, fmaf(C4.y, hv[q].y, fmaf(C4.z, hv[q].z, fmaf(C4.w, hv[q].w, acc))));
       hp[q] = hv[q];
     }
-    y[(long long)b * a.E + c] = Store<T>::from_f(fmaf(Dc, uu, acc) * silu_f(zz));
+    y[(long long)b * a.E + c] = Store<T>::from_f(fmaf(Dc, uu, acc) * zz);
   }
 }
 
@@ -513,8 +526,13 @@ static hymba_status decode_ssm_t(const DecodeSsmArgs &a, cudaStream_t s) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set.done(dev)) {
-    cudaFuncSetAttribute(dec_conv_xproj_kernel<T, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    cudaFuncSetAttribute(dec_dt_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    if (cudaFuncSetAttribute(dec_conv_xproj_kernel<T, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             200 * 1024) != cudaSuccess ||
+        cudaFuncSetAttribute(dec_dt_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             200 * 1024) != cudaSuccess) {
+      set_error("cudaFuncSetAttribute(decode SSM smem) failed");
+      return HYMBA_ERR_CUDA;
+    }
     attr_set.mark(dev);
   }
   dim3 g1(a.E / CH, (a.B + kDecRows - 1) / kDecRows);
@@ -572,10 +590,11 @@ __device__ __forceinline__ void st_pair(T *p, float a, float b) {
 
 // CB channels per block, two per thread.  MODE 0: scan from the chunk's start
 // state and write y (and the final state); MODE 1: scan from zero, record the
-// chunk's end state and sum of delta.  The first NPOLY states of each channel take
-// their decay from the degree-5 exp2_poly2 (FMA pipe), the others from the MUFU: the two pipes
-// then share the exponentials, which bound this kernel.
-template <typename T, int CB, int MODE, int NPOLY>
+// chunk's end state and sum of delta.  Every decay is one MUFU exp2: a polynomial
+// share on the FMA pipe was measured slower (0, 2, 4 states: 4.71, 4.98, 5.45 ms on a
+// batch-32 layer), since at ~80 instructions per channel-step each polynomial pair's ten
+// extra instructions cost more issue slots than the MUFU time they free.
+template <typename T, int CB, int MODE>
 __global__ void __launch_bounds__(CB / 2)
     scan_kernel(ScanArgs a, int chunks, int Tc, const float *__restrict__ hstart,
                 float *__restrict__ hend, float *__restrict__ dsum_out) {
@@ -584,7 +603,6 @@ __global__ void __launch_bounds__(CB / 2)
   constexpr int ROW_PIECES = CB * (int)sizeof(T) / 16;  // 16-byte pieces per staged row
   constexpr int ARR_BYTES = TB * CB * (int)sizeof(T);
   constexpr int BUF_BYTES = 3 * ARR_BYTES + TB * 2 * kStates * 4;
-  static_assert(NPOLY % 2 == 0 && NPOLY <= kStates, "polynomial states come in pairs");
   extern __shared__ __align__(16) uint8_t scan_smem[];
   const int E = a.E;
   const int cblocks = E / CB;
@@ -637,7 +655,7 @@ __global__ void __launch_bounds__(CB / 2)
   const long long sidx = (((long long)b * chunks + k) * E + c) * kStates;  // channel c; c + 1 follows
   const float *h0 = nullptr;
   if (MODE == 0 && chunks > 1) h0 = hstart + sidx;
-  else if (MODE == 0 && a.h_in) h0 = a.h_in + ((long long)b * E + c) * kStates;
+  else if (MODE == 0 && a.h_in) h0 = a.h_in + (long long)b * a.h_in_bstride + (long long)c * kStates;
 #pragma unroll
   for (int ch = 0; ch < 2; ++ch) {
 #pragma unroll
@@ -690,7 +708,7 @@ __global__ void __launch_bounds__(CB / 2)
 #pragma unroll
         for (int n2 = 0; n2 < kStates / 2; ++n2) {
           const float2 x = fmul2(d2, A2[ch][n2]);
-          const float2 dA = 2 * n2 < NPOLY ? exp2_poly2<5>(x) : make_float2(ex2_ftz(x.x), ex2_ftz(x.y));
+          const float2 dA = make_float2(ex2_ftz(x.x), ex2_ftz(x.y));
           h[ch][n2] = ffma2(dA, h[ch][n2], fmul2(du2, Bp[n2]));
           acc[n2 & 1] = ffma2(Cp[n2], h[ch][n2], acc[n2 & 1]);
         }
@@ -698,8 +716,7 @@ __global__ void __launch_bounds__(CB / 2)
       }
       if (MODE == 0) {
         const float2 zz = ld_pair(sz + tt * CB);
-        st_pair(yp + (long long)tt * E, fmaf(Dc.x, uu.x, yv[0]) * silu_f(zz.x),
-                fmaf(Dc.y, uu.y, yv[1]) * silu_f(zz.y));
+        st_pair(yp + (long long)tt * E, fmaf(Dc.x, uu.x, yv[0]) * zz.x, fmaf(Dc.y, uu.y, yv[1]) * zz.y);
       } else {
         dsum.x += dd.x;
         dsum.y += dd.y;
@@ -737,8 +754,9 @@ __global__ void __launch_bounds__(CB / 2)
 
 // Chains chunk start states: H_0 = h_in (or 0); H_{k+1} = exp(A * dsum_k) H_k + hend_k.
 __global__ void scan_combine_kernel(const float *__restrict__ a_log, const float *__restrict__ h_in,
-                                    const float *__restrict__ hend, const float *__restrict__ dsum,
-                                    float *__restrict__ hstart, int B, int E, int chunks) {
+                                    long long h_in_bstride, const float *__restrict__ hend,
+                                    const float *__restrict__ dsum, float *__restrict__ hstart, int B,
+                                    int E, int chunks) {
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)B * E) return;
   const int c = int(idx % E), b = int(idx / E);
@@ -746,7 +764,7 @@ __global__ void scan_combine_kernel(const float *__restrict__ a_log, const float
 #pragma unroll
   for (int n = 0; n < kStates; ++n) {
     A2[n] = -__expf(a_log[c * kStates + n]) * 1.4426950408889634f;
-    H[n] = h_in ? h_in[((long long)b * E + c) * kStates + n] : 0.f;
+    H[n] = h_in ? h_in[(long long)b * h_in_bstride + (long long)c * kStates + n] : 0.f;
   }
   for (int k = 0; k < chunks; ++k) {
     const long long sidx = (((long long)b * chunks + k) * E + c) * kStates;
@@ -777,37 +795,30 @@ size_t scan_workspace_floats(int B, int L, int E, int N, int *chunks_out) {
   return (size_t)B * ch * E * (2 * N + 1);
 }
 
-// Polynomial-exp2 states per channel in the bf16 scan (the fp32 path keeps the MUFU for all).
-// Measured on B200 at batch 32, 8320 rows, d_inner 3200: 0 states 4.71 ms, 2 states
-// 4.98 ms, 4 states 5.45 ms.  With 80 instructions per channel-step the scan is bound
-// by issue and latency rather than by the MUFU, and each polynomial pair costs ten more
-// instructions, so all decays stay on the MUFU.
-constexpr int kScanPolyStates = 0;
-
-template <typename T, int CB, int NPOLY>
+template <typename T, int CB>
 static void scan_set_smem(int bytes) {
-  cudaFuncSetAttribute(scan_kernel<T, CB, 0, NPOLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  cudaFuncSetAttribute(scan_kernel<T, CB, 1, NPOLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  cudaFuncSetAttribute(scan_kernel<T, CB, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  cudaFuncSetAttribute(scan_kernel<T, CB, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
-template <typename T, int CB, int NPOLY>
+template <typename T, int CB>
 static void scan_launch(const ScanArgs &a, int mode, int chunks, int Tc, const float *hstart,
                         float *hend, float *dsum, cudaStream_t s) {
   const unsigned blocks = (unsigned)((long long)a.B * chunks * (a.E / CB));
   const int smem = 2 * (3 * kScanTB * CB * (int)sizeof(T) + kScanTB * 2 * kStates * 4);
   if (mode == 0)
-    scan_kernel<T, CB, 0, NPOLY><<<blocks, CB / 2, smem, s>>>(a, chunks, Tc, hstart, hend, dsum);
+    scan_kernel<T, CB, 0><<<blocks, CB / 2, smem, s>>>(a, chunks, Tc, hstart, hend, dsum);
   else
-    scan_kernel<T, CB, 1, NPOLY><<<blocks, CB / 2, smem, s>>>(a, chunks, Tc, hstart, hend, dsum);
+    scan_kernel<T, CB, 1><<<blocks, CB / 2, smem, s>>>(a, chunks, Tc, hstart, hend, dsum);
 }
-template <typename T, int NPOLY>
+template <typename T>
 static void scan_launch_cb(const ScanArgs &a, int mode, int chunks, int Tc, const float *hstart,
                            float *hend, float *dsum, cudaStream_t s) {
   if (a.E % 128 == 0)
-    scan_launch<T, 128, NPOLY>(a, mode, chunks, Tc, hstart, hend, dsum, s);
+    scan_launch<T, 128>(a, mode, chunks, Tc, hstart, hend, dsum, s);
   else if (a.E % 64 == 0)
-    scan_launch<T, 64, NPOLY>(a, mode, chunks, Tc, hstart, hend, dsum, s);
+    scan_launch<T, 64>(a, mode, chunks, Tc, hstart, hend, dsum, s);
   else
-    scan_launch<T, 32, NPOLY>(a, mode, chunks, Tc, hstart, hend, dsum, s);
+    scan_launch<T, 32>(a, mode, chunks, Tc, hstart, hend, dsum, s);
 }
 
 hymba_status selective_scan(const ScanArgs &a, hymba_dtype dt, cudaStream_t s) {
@@ -831,26 +842,26 @@ hymba_status selective_scan(const ScanArgs &a, hymba_dtype dt, cudaStream_t s) {
     cudaGetDevice(&dev);
     if (!attr_set.done(dev)) {
       const int most = 2 * (3 * kScanTB * 128 * 4 + kScanTB * 2 * kStates * 4);
-      scan_set_smem<float, 128, 0>(most);
-      scan_set_smem<float, 64, 0>(most);
-      scan_set_smem<float, 32, 0>(most);
-      scan_set_smem<__nv_bfloat16, 128, kScanPolyStates>(most);
-      scan_set_smem<__nv_bfloat16, 64, kScanPolyStates>(most);
-      scan_set_smem<__nv_bfloat16, 32, kScanPolyStates>(most);
+      scan_set_smem<float, 128>(most);
+      scan_set_smem<float, 64>(most);
+      scan_set_smem<float, 32>(most);
+      scan_set_smem<__nv_bfloat16, 128>(most);
+      scan_set_smem<__nv_bfloat16, 64>(most);
+      scan_set_smem<__nv_bfloat16, 32>(most);
       attr_set.mark(dev);
     }
   }
   auto launch = [&](int mode) {
     if (dt == HYMBA_BF16)
-      scan_launch_cb<__nv_bfloat16, kScanPolyStates>(a, mode, chunks, Tc, hstart, hend, dsum, s);
+      scan_launch_cb<__nv_bfloat16>(a, mode, chunks, Tc, hstart, hend, dsum, s);
     else
-      scan_launch_cb<float, 0>(a, mode, chunks, Tc, hstart, hend, dsum, s);
+      scan_launch_cb<float>(a, mode, chunks, Tc, hstart, hend, dsum, s);
   };
   if (chunks > 1) {
     launch(1);
     const long long n = (long long)a.B * a.E;
-    scan_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.a_log, a.h_in, hend, dsum,
-                                                                    hstart, a.B, a.E, chunks);
+    scan_combine_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a.a_log, a.h_in, a.h_in_bstride, hend,
+                                                                    dsum, hstart, a.B, a.E, chunks);
   }
   launch(0);
   note_launch(chunks > 1 ? 3 : 1);

@@ -81,6 +81,11 @@ typedef struct {
   hymba_dtype dtype;
   float rms_eps;     /* eps of the per-branch RMS norm                 */
   float softmax_scale; /* 0 -> 1/sqrt(head_dim_qk) (OpenReview reply Q2) */
+  float rope_base;   /* rotary position embedding of Q and K (§2.5 changes "the RoPE base";
+                        no value is given): 0 = none; > 1: pair (2i, 2i+1) of every head
+                        turned by p * rope_base^(-2i/head_dim_qk) at X~ position p, applied
+                        by the input projection (head_dim_qk a power of two).  Layers that
+                        share K/V must use the same base. */
 } hymba_layer_config;
 
 /* Weights of one layer (device pointers, kept by the handle, never copied).
@@ -165,19 +170,23 @@ HYMBA_API hymba_status hymba_layer_prefill_workspace(const hymba_layer *layer, i
 typedef struct {
   size_t q;       /* [M, H*d_qk]          dtype */
   size_t x_ssm;   /* [M, E]               dtype */
-  size_t z;       /* [M, E]               dtype */
+  size_t gate;    /* [M, E] SiLU(z)       dtype */
   size_t u;       /* [M, E] conv+SiLU     dtype */
   size_t xdbl;    /* [M, R+2N] fp32: delta_r, B, C */
   size_t delta;   /* [M, E] softplus      dtype */
   size_t y_ssm;   /* [M, E] gated scan    dtype */
   size_t o_attn;  /* [M, E] attention     dtype */
   size_t fused;   /* [M, E] Eq. 3 inside W_out(.)  dtype */
+  size_t rope;    /* [L, d_qk/2] (cos, sin) fp32 pairs of the rotary embedding (if any) */
   size_t total;
 } hymba_prefill_layout;
 HYMBA_API hymba_status hymba_layer_prefill_layout(const hymba_layer *layer, int batch, int n_tokens,
                                         hymba_prefill_layout *out);
 
-/* One layer over `batch` sequences of L = n_meta + n_tokens rows.
+/* One layer over `batch` sequences of L = n_meta + n_tokens rows: the hybrid-head
+ * module of §2.1 (Eq. 3 over the attention heads of Eq. 1 and the SSM heads of Eq. 2)
+ * on X~ = [R; X] (§2.3 Eq. 4), with the A-shape or global mask of §2.2 and, for a
+ * bound consumer, the producer's K/V ("Cross-layer KV sharing", §2.2).
  *   x   [batch, L, d_model] dtype : X~ (meta rows included; the caller builds
  *                                   [R; X] for the first layer, later layers
  *                                   take the previous layer's output as is)
@@ -194,6 +203,65 @@ HYMBA_API hymba_status hymba_layer_prefill(hymba_layer *layer, int batch, int n_
                                  hymba_kv_cache *kv_cache, hymba_ssm_cache *ssm_cache,
                                  void *workspace, size_t workspace_bytes, hymba_stream_t stream);
 
+/* ---- meta-token cache --------------------------------------------------- */
+
+/* The meta tokens are the same rows at the head of every sequence (§2.3 Eq. 4), so
+ * their part of a layer's work does not depend on the input: the paper notes that it can
+ * be done offline, the meta tokens acting as a learned initialisation of the K/V cache
+ * and the SSM state (§2.3, "Initialization for KV cache and SSM state").  A meta cache
+ * holds that part for one layer, computed once (batch 1):
+ *   k, v  [n_meta, Hkv*d_qk] / [n_meta, Hkv*d_v] dtype: the meta rows' K/V (a layer that
+ *         owns its K/V; unused for a consumer, which reads its producer's)
+ *   h     [d_inner, d_state] fp32: the SSM state after the meta rows
+ *   conv  [d_conv-1, d_inner] dtype: the last d_conv-1 x_ssm rows of the meta rows
+ *   y     [n_meta, d_model] dtype: the layer's output for the meta rows, which is the
+ *         next layer's meta input
+ *   owner set by hymba_layer_meta_precompute (0 = not computed).
+ * Device buffers owned by the caller, 16-byte aligned. */
+typedef struct {
+  void *k;
+  void *v;
+  float *h;
+  void *conv;
+  void *y;
+  uint64_t owner;
+} hymba_meta_cache;
+
+/* Workspace bytes of hymba_layer_meta_precompute (a batch-1 prefill of the meta rows). */
+HYMBA_API hymba_status hymba_layer_meta_workspace(const hymba_layer *layer, size_t *bytes);
+
+/* Fills `meta` for this layer from x_meta [n_meta, d_model] dtype: the meta tokens R
+ * for the first layer, the previous layer's meta->y for later ones.  A consumer passes
+ * its producer's meta cache (stamp checked, NOT_BOUND otherwise); a K/V owner passes
+ * NULL.  Asynchronous on `stream`; INVALID_ARG if the layer has no meta tokens. */
+HYMBA_API hymba_status hymba_layer_meta_precompute(hymba_layer *layer, const void *x_meta,
+                                                   hymba_meta_cache *meta,
+                                                   const hymba_meta_cache *producer_meta,
+                                                   void *workspace, size_t workspace_bytes,
+                                                   hymba_stream_t stream);
+
+/* Workspace bytes of hymba_layer_prefill_cached (intermediates of the real rows only). */
+HYMBA_API hymba_status hymba_layer_prefill_cached_workspace(const hymba_layer *layer, int batch,
+                                                            int n_tokens, size_t *bytes);
+
+/* hymba_layer_prefill for the real rows only, starting from this layer's meta cache:
+ *   x, y  [batch, n_tokens, d_model] dtype: the real rows of X~ (positions n_meta..L-1)
+ *         and their outputs (the meta rows' outputs are meta->y, the same for every
+ *         sequence)
+ *   meta  computed by hymba_layer_meta_precompute for this layer (NOT_BOUND otherwise)
+ *   kv    full-length K/V as for hymba_layer_prefill (L = n_meta + n_tokens rows per
+ *         sequence): a K/V owner copies its meta rows' K/V into rows 0..n_meta-1 of each
+ *         sequence and writes rows n_meta..L-1; a consumer reads its producer's.
+ *   kv_cache, ssm_cache, workspace as for hymba_layer_prefill (ssm_cache receives the
+ *         state after the whole sequence).
+ * Same results as hymba_layer_prefill on X~ = [R; X] for rows n_meta..L-1, with the
+ * meta rows' work done once instead of once per sequence.  n_tokens >= 1. */
+HYMBA_API hymba_status hymba_layer_prefill_cached(hymba_layer *layer, int batch, int n_tokens,
+                                                  const void *x, void *y, const hymba_meta_cache *meta,
+                                                  hymba_kv_seq *kv, hymba_kv_cache *kv_cache,
+                                                  hymba_ssm_cache *ssm_cache, void *workspace,
+                                                  size_t workspace_bytes, hymba_stream_t stream);
+
 /* ---- decode ------------------------------------------------------------- */
 
 /* Bytes of device workspace hymba_layer_decode_step needs for positions up to max_pos. */
@@ -201,7 +269,10 @@ HYMBA_API hymba_status hymba_layer_decode_workspace(const hymba_layer *layer, in
                                                     size_t *bytes);
 
 /* One new token per sequence at X~ position `pos` (same for every sequence;
- * pos >= n_meta).  x_t, y_t [batch, d_model] dtype.
+ * pos >= n_meta): the same module for a single row, reading the layer's caches — the
+ * meta rows plus the sliding window of K/V, or every row for a global layer (§2.2, §2.3
+ * "learned cache initialization"), and the constant-size SSM state of Eq. 2's
+ * recurrence (§2.1).  x_t, y_t [batch, d_model] dtype.
  *   kv_cache: a K/V owner appends this token's K/V at its slot and attends over
  *     its own store; a consumer attends over its producer's store (stamp
  *     checked), which the producer must have updated for this position first.
@@ -228,7 +299,8 @@ HYMBA_API hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, in
  * rejected with HYMBA_ERR_WORKSPACE before anything is launched; 40 MiB covers
  * a batch of 128 on a sliding-window layer of the 1.5B shape (m + W = 1152).
  * The first call on a device looks up the buffer's device address (with that
- * device current); make that first call before any stream capture.  All calls
+ * device current), and so does the first call after that device's context has been
+ * torn down and created again; make such a first call before any stream capture.  All calls
  * share the one buffer, which keeps the last call's contents (the step zeroes
  * what it accumulates into): calls that may overlap on the GPU race, so issue
  * them in order on one stream. */
@@ -244,19 +316,60 @@ HYMBA_API hymba_status hymba_layer_decode_step_static(hymba_layer *layer, int ba
 /* Synchronises `stream`, then reports a pending CUDA error or a device-side
  * error word (e.g. a bounded wait that timed out) and clears the word. */
 HYMBA_API hymba_status hymba_stream_status(hymba_stream_t stream);
+/* Bounded device waits.  Every wait of the tensor-core kernels on an mbarrier (a TMA
+ * copy, an MMA, a pipeline stage) gives up after a limit in SM clock cycles, records a
+ * timeout in the library's device error word, drains what its CTA has in flight, releases
+ * its tensor memory and returns; hymba_stream_status() then reports HYMBA_ERR_TIMEOUT.
+ * This sets the limit for launches issued from now on: `cycles` >= 1e5 (smaller values
+ * are raised to 1e5); 0 restores the default, which is the HYMBA_WAIT_LIMIT environment
+ * variable when set, else 1e9 cycles (about half a second).  *applied (optional) receives
+ * the limit now in force.  Host only; not a hot call. */
+HYMBA_API hymba_status hymba_set_wait_limit(int64_t cycles, int64_t *applied);
+
+/* Diagnostic of the bounded-wait path: in the next `count` calls of hymba_layer_prefill
+ * (bf16 path), the output projection's MMA warp waits for an arrival that never comes
+ * instead of issuing its first MMA, so that kernel's waits run out: it records a timeout,
+ * drains and returns (its output rows are then undefined), and hymba_stream_status()
+ * reports HYMBA_ERR_TIMEOUT.  No fault and no unbounded wait is involved.  0 cancels. */
+HYMBA_API hymba_status hymba_debug_stall_next_prefill(int count);
+
 /* Reason for the last non-OK status returned on this thread ("" if none). */
 HYMBA_API const char *hymba_last_error(void);
 HYMBA_API const char *hymba_status_string(hymba_status s);
 /* Library version, e.g. "hymba-b200 0.1 sm_100a". */
 HYMBA_API const char *hymba_version(void);
 
-/* The attention mask as the attention kernel evaluates it (same device
- * predicate), for bit-exact checks.  bits [L, ceil(L/32)] uint32 row-major:
- * bit j%32 of word j/32 of row i is 1 iff key j is visible from query i.
- * tile_class (optional) [ceil(L/128), ceil(L/128)] uint8: 0 = skipped (no
- * visible pair), 1 = fully visible, 2 = partially masked, for 128x128 tiles. */
-HYMBA_API hymba_status hymba_debug_mask_bitmap(int L, int n_meta, int window, int is_global,
-                                     uint32_t *bits, uint8_t *tile_class, hymba_stream_t stream);
+/* The prefill attention mask exactly as an attention kernel applies it, for bit-exact
+ * checks against the definition (Hymba §2.1 Eq. 1 under the A-shape mask of the authors'
+ * OpenReview reply, or causal for a global layer, §2.2).
+ *   path 0: the bf16 tensor-core kernel: a key is visible iff its 128-key tile is among
+ *           the tiles the kernel streams for the query's pair of 128-row tiles, the
+ *           tile's class is not "skipped", and (partially visible tile) its column is
+ *           in the keep-mask the softmax applies.  The dump calls the kernel's own
+ *           device functions for each of these decisions.
+ *   path 1: the fp32 CUDA-core kernel: its per-pair predicate.
+ * bits [L, ceil(L/32)] uint32 (device) row-major: bit j%32 of word j/32 of row i is 1 iff
+ * key j is visible from query i.  tile_class (optional, device) [ceil(L/128)]^2 uint8:
+ * 0 = skipped (no visible pair), 1 = fully visible, 2 = partially masked, as the tensor-
+ * core kernel classifies 128x128 tiles.  INVALID_ARG for a bad shape or path. */
+HYMBA_API hymba_status hymba_debug_mask_bitmap(int L, int n_meta, int window, int is_global, int path,
+                                               uint32_t *bits, uint8_t *tile_class,
+                                               hymba_stream_t stream);
+
+/* The decode attention's key-slot mask for the query at X~ position `pos` (the predicate
+ * both decode kernels apply to every slot of the K/V store; slot rule as for
+ * hymba_kv_cache).  bits [ceil(capacity/32)] uint32 (device): bit s%32 of word s/32 is 1
+ * iff slot s holds a position visible from pos.  capacity must cover the slots the query
+ * reads (m + W, or pos + 1 for a global layer), else INVALID_ARG. */
+HYMBA_API hymba_status hymba_debug_decode_mask(int64_t pos, int n_meta, int window, int is_global,
+                                               int capacity, uint32_t *bits, hymba_stream_t stream);
+
+/* 2^x of n floats (device buffers) by the FMA-pipe polynomial (degree 3 or 5) that the
+ * prefill attention softmax uses for a share of its exponentials.  For checking the
+ * stated bound: relative error <= 7.5e-5 (degree 3) or 2.4e-7 (degree 5) for
+ * -125 <= x < 128 beyond fp32 rounding; x < -125 returns 2^-125. */
+HYMBA_API hymba_status hymba_debug_exp2_poly(int degree, const float *x, float *y, int64_t n,
+                                             hymba_stream_t stream);
 
 /* ---- optional per-kernel timing ---------------------------------------- */
 

@@ -27,7 +27,11 @@ the design notes of this repository):
     A = -exp(A_log), y = C.h + D u, gated by SiLU(z);
   * norm = RMS over all d_inner channels with no weight, eps as configured;
   * Eq. (3)'s two branches are averaged (divided by 2) as the text says;
-  * no biases in the in/x/out projections; no RoPE.
+  * no biases in the in/x/out projections;
+  * rotary position embedding of Q and K (§2.5 changes "the ROPE base" for the 8k
+    extension; base not given): off unless a base is configured; when on, the rotation
+    of the original rotary-embedding definition, each consecutive pair (2i, 2i+1) of a
+    head turned by the angle p * base^(-2i/d_qk) at X~ position p (meta rows included).
 The pages print no value that checks the readings of the conv, the low-rank
 delta, the SiLU gate, the RMS form of "norm" and D; the functions themselves are
 pinned by the tests through special cases with closed forms or library routines
@@ -58,6 +62,7 @@ class Spec:
     is_global: bool
     eps: float = 1e-6
     scale: float = 0.0   # 0 -> 1/sqrt(head_dim_qk)
+    rope_base: float = 0.0  # 0 -> no rotary position embedding
 
     @property
     def score_scale(self) -> float:
@@ -138,6 +143,25 @@ def in_proj(xt: np.ndarray, w_in: np.ndarray, s: Spec, consumer: bool):
     z = p[:, c + E:c + 2 * E]
     assert p.shape[1] == c + 2 * E
     return q, k, v, xs, z
+
+
+# ---------------------------------------------------------------------------
+# Rotary position embedding of Q and K (Hymba §2.5 / §3: a RoPE base changed for the
+# 8k-context extension)
+# ---------------------------------------------------------------------------
+
+def rope(x: np.ndarray, positions: np.ndarray, head_dim: int, base: float) -> np.ndarray:
+    """x [rows, n_heads*head_dim] at X~ positions [rows]: in every head, pair (2i, 2i+1)
+    rotated by the angle pos * base^(-2i/head_dim)."""
+    rows = x.shape[0]
+    xh = x.reshape(rows, -1, head_dim // 2, 2)
+    i = np.arange(head_dim // 2)
+    ang = np.asarray(positions, dtype=np.float64)[:, None] * base ** (-2.0 * i / head_dim)[None, :]
+    c, s = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    out = np.empty_like(xh)
+    out[..., 0] = xh[..., 0] * c - xh[..., 1] * s
+    out[..., 1] = xh[..., 0] * s + xh[..., 1] * c
+    return out.reshape(rows, -1)
 
 
 # ---------------------------------------------------------------------------
@@ -237,6 +261,18 @@ def kv_capacity(s: Spec, max_rows: int) -> int:
     return max_rows if s.is_global else s.n_meta + s.window
 
 
+def decode_slot_bitmap(pos: int, s: Spec, capacity: int) -> np.ndarray:
+    """Slots of the decode K/V store that a query at position pos attends to: the slot of
+    every position visible from pos.  [ceil(capacity/32)] uint32; bit (k % 32) of word
+    k // 32 is slot k."""
+    words = np.zeros((capacity + 31) // 32, dtype=np.uint32)
+    for j in range(pos + 1):
+        if allowed(pos, j, s.n_meta, s.window, s.is_global):
+            k = kv_slot(j, s)
+            words[k // 32] |= np.uint32(1 << (k % 32))
+    return words
+
+
 # ---------------------------------------------------------------------------
 # Whole layer
 # ---------------------------------------------------------------------------
@@ -256,6 +292,10 @@ def layer_prefill(xt, w: dict, s: Spec, kv_from: dict | None = None, capacity: i
     L = xt.shape[0]
     consumer = kv_from is not None
     q, k, v, xs, z = in_proj(xt, _f64(w["w_in"]), s, consumer)
+    if s.rope_base > 0:
+        q = rope(q, np.arange(L), s.head_dim_qk, s.rope_base)
+        if not consumer:
+            k = rope(k, np.arange(L), s.head_dim_qk, s.rope_base)
     if consumer:
         k, v = kv_from["k"], kv_from["v"]
     o = attention(q, k, v, s)
@@ -297,6 +337,10 @@ def layer_decode(x_t, pos: int, w: dict, s: Spec, cache: dict, kv_cache: dict | 
     x_t = _f64(x_t)[None, :]
     consumer = kv_cache is not None
     q, k, v, xs, z = in_proj(x_t, _f64(w["w_in"]), s, consumer)
+    if s.rope_base > 0:
+        q = rope(q, np.array([pos]), s.head_dim_qk, s.rope_base)
+        if not consumer:
+            k = rope(k, np.array([pos]), s.head_dim_qk, s.rope_base)
     new = {key: _f64(val).copy() for key, val in cache.items()}
     if consumer:
         kc, vc = _f64(kv_cache["k"]), _f64(kv_cache["v"])

@@ -63,6 +63,7 @@ class Workload:
     kv_shared_pair: bool = False
     decode: bool = False
     seed: int = 0
+    rope_base: float = 0.0  # rotary position embedding of Q and K: 0 = none
 
     @property
     def seq_rows(self) -> int:
@@ -130,6 +131,10 @@ DEFAULT_STD = WeightStd()
 # "Scan-stress" set: u, B and C of order one and D = 0, so that the recurrence
 # term dominates the SSM output instead of the D*u skip.
 STRESS_STD = replace(DEFAULT_STD, conv_w=0.5, conv_b=0.5, w_x_bc_unit_gain=True, d_skip=0.0)
+# The same with a dt projection of std 0.2, so that delta varies by a factor of several
+# along the sequence (with the default weights it is nearly constant: softplus(b_dt) plus
+# a ~5e-3 input term), which makes the decay's use of delta visible.
+STRESS_DELTA_STD = replace(STRESS_STD, w_dt=0.2)
 
 
 def layer_weights(w: Workload, layer: int, consumer: bool = False, device="cpu",

@@ -25,7 +25,7 @@ def spec_of(w: Workload, is_global: bool | None = None) -> O.Spec:
     return O.Spec(d_model=d.d_model, n_heads=d.n_heads, n_kv_heads=d.n_kv_heads,
                   head_dim_qk=d.head_dim_qk, head_dim_v=d.head_dim_v, d_inner=d.d_inner,
                   d_state=d.d_state, d_conv=d.d_conv, dt_rank=d.rank, n_meta=w.n_meta,
-                  window=max(w.window, 1), is_global=g, eps=1e-6)
+                  window=max(w.window, 1), is_global=g, eps=1e-6, rope_base=w.rope_base)
 
 
 def to64(t: torch.Tensor) -> np.ndarray:
@@ -50,7 +50,7 @@ class GpuLayer:
         d = w.dims
         self.cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner,
                                   d.d_state, d.d_conv, d.rank, w.n_meta, w.window,
-                                  self.is_global, w.dtype)
+                                  self.is_global, w.dtype, rope_base=w.rope_base)
         self.handle = hy.hymba_layer_create(self.cfg, hy.make_weights(self.dev))
         self.spec = spec_of(w, self.is_global)
 
@@ -114,7 +114,7 @@ def stage(layer: GpuLayer, ws: torch.Tensor, B: int, L: int, name: str) -> torch
     w = layer.workload
     lay = hy.hymba_layer_prefill_layout(layer.handle, B, L - w.n_meta)
     d = w.dims
-    widths = dict(q=d.n_heads * d.head_dim_qk, x_ssm=d.d_inner, z=d.d_inner, u=d.d_inner,
+    widths = dict(q=d.n_heads * d.head_dim_qk, x_ssm=d.d_inner, gate=d.d_inner, u=d.d_inner,
                   xdbl=d.xproj_width, delta=d.d_inner, y_ssm=d.d_inner, o_attn=d.d_inner,
                   fused=d.d_inner)
     dt = torch.float32 if name == "xdbl" else torch_dt(w)
@@ -146,31 +146,39 @@ def close_stage(g, o, what=""):
     close_bf16(np.asarray(g, dtype=np.float64) / s, o / s, what + f" (scaled by rms {s:.3g})")
 
 
-def close_stage_dist(g, o, what="", max_frac=2e-4, max_ratio=5.0, max_rel_l2=1e-2):
-    """Intermediate-stage check.  Intermediates are conditioning-limited: y_ssm = C.h sums
-    16 products that can cancel, so bf16 rounding of u or x_ssm upstream can move a near-zero
-    element by several per cent of the stage's rms.  A wrong index, sign or term moves most
-    elements; so: at most max_frac of the elements may exceed the scaled bf16 bound, none by
-    more than max_ratio times, and the relative L2 error stays below max_rel_l2."""
+def close_rel_l2(g, o, tol=1e-2, what=""):
+    """Relative L2 distance of the whole array: catches a mistake spread thinly over many
+    elements of a stage whose elementwise bound is set by cancellation."""
     g = np.asarray(g, dtype=np.float64)
     o = np.asarray(o, dtype=np.float64)
-    s = float(np.sqrt((o ** 2).mean())) or 1.0
-    err = np.abs(g - o) / s
-    bound = BF16_ATOL + BF16_RTOL * np.abs(o) / s
-    ratio = err / bound
-    frac = float((ratio > 1).mean())
     rel = float(np.linalg.norm(g - o) / max(np.linalg.norm(o), 1e-300))
-    if frac > max_frac or ratio.max() > max_ratio or rel > max_rel_l2:
-        idx = np.unravel_index(np.argmax(ratio), ratio.shape)
-        raise AssertionError(f"{what}: {frac:.2e} of elements outside the scaled bound, worst "
-                             f"{ratio.max():.2f}x at {idx} (gpu {g[idx]:.5g}, oracle {o[idx]:.5g}); "
-                             f"rel L2 {rel:.2e}")
+    assert rel <= tol, f"{what}: relative L2 error {rel:.3g} > {tol:g}"
 
 
-# Two chained layers: the consumer receives the producer's bf16 output, whose rounding
-# (error std ~0.4% of rms(Y)) adds in quadrature to the layer's own (~0.4%): the chain's
-# error std is ~sqrt(2) larger, so its elementwise bound is taken 1.5x the single-layer one
-# (about 7 standard deviations at Y = 0).
+def conv_state_from_stage(x_ssm_stage: torch.Tensor, K: int) -> torch.Tensor:
+    """The conv state a prefill must return, taken from the x_ssm rows the same call
+    produced: its last K-1 rows (zero rows in front when the sequence is shorter)."""
+    L, E = x_ssm_stage.shape
+    out = torch.zeros((K - 1, E), dtype=x_ssm_stage.dtype, device=x_ssm_stage.device)
+    take = min(K - 1, L)
+    if take:
+        out[K - 1 - take:] = x_ssm_stage[L - take:]
+    return out
+
+
+def assert_bits_equal(a: torch.Tensor, b: torch.Tensor, what=""):
+    """Bit-for-bit equality of two tensors of the same dtype (any dtype, bf16 included)."""
+    assert a.dtype == b.dtype and a.shape == b.shape, (what, a.dtype, b.dtype, a.shape, b.shape)
+    ia = a.contiguous().view(torch.int16 if a.element_size() == 2 else torch.int32)
+    ib = b.contiguous().view(torch.int16 if b.element_size() == 2 else torch.int32)
+    n = int((ia != ib).sum())
+    assert n == 0, f"{what}: {n} of {a.numel()} elements differ in their bits"
+
+
+# Two chained layers (the consumer fed the producer's bf16 output): the chain's error is
+# larger than one layer's by the ratio of the error spreads, which the bf16 rounding model
+# (tests/_bf16_emulation.py, checked in tests/test_rounding_model.py) puts at 1.47 on the
+# pair workload; the chained bound is the single-layer bound times 1.5.
 CHAIN2_ATOL, CHAIN2_RTOL = 3e-2, 3e-2
 
 

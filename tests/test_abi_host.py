@@ -100,7 +100,7 @@ def test_prefill_rejects_bad_arguments_before_launch():
     ws = hy.hymba_layer_prefill_workspace(p, B, n)
     lay = hy.hymba_layer_prefill_layout(p, B, n)
     assert lay.total == ws and lay.q == 0
-    offs = [lay.q, lay.x_ssm, lay.z, lay.u, lay.xdbl, lay.delta, lay.y_ssm, lay.o_attn, lay.fused]
+    offs = [lay.q, lay.x_ssm, lay.gate, lay.u, lay.xdbl, lay.delta, lay.y_ssm, lay.o_attn, lay.fused]
     assert offs == sorted(offs) and all(o % 256 == 0 for o in offs)
     M = B * (128 + n)
     assert lay.x_ssm - lay.q >= M * 1600 * 2 and lay.delta - lay.xdbl >= M * 132 * 4
@@ -237,7 +237,7 @@ def test_prefill_workspace_holds_every_documented_intermediate(kw):
             lay = hy.hymba_layer_prefill_layout(h, B, n)
             assert lay.total == hy.hymba_layer_prefill_workspace(h, B, n)
             regions = [(lay.q, M * cfg.n_heads * cfg.head_dim_qk * es), (lay.x_ssm, M * E * es),
-                       (lay.z, M * E * es), (lay.u, M * E * es), (lay.xdbl, M * (R + 2 * N) * 4),
+                       (lay.gate, M * E * es), (lay.u, M * E * es), (lay.xdbl, M * (R + 2 * N) * 4),
                        (lay.delta, M * E * es), (lay.y_ssm, M * E * es), (lay.o_attn, M * E * es),
                        (lay.fused, M * E * es)]
             for (o, size), (o_next, _) in zip(regions, regions[1:] + [(lay.total, 0)]):
@@ -267,3 +267,68 @@ def test_decode_workspace_never_shrinks_as_the_position_grows(glob):
         hy.hymba_layer_decode_workspace(h, 128, 127)   # a meta position
     assert e.value.status == hy.HYMBA_ERR_INVALID_ARG
     hy.hymba_layer_destroy(h)
+
+
+def test_wait_limit_is_clamped_and_restorable():
+    assert hy.hymba_set_wait_limit(10) == 100000
+    assert hy.hymba_set_wait_limit(5_000_000) == 5_000_000
+    default = hy.hymba_set_wait_limit(0)
+    assert default >= 100000
+    with pytest.raises(hy.HymbaError):
+        hy.hymba_set_wait_limit(-1)
+    hy.hymba_debug_stall_next_prefill(0)
+    with pytest.raises(hy.HymbaError):
+        hy.hymba_debug_stall_next_prefill(-1)
+
+
+def test_meta_cache_calls_check_their_stamps_before_launch():
+    p = hy.hymba_layer_create(_cfg(), _fake_weights())
+    c = hy.hymba_layer_create(_cfg(), _fake_weights(1 << 41))
+    hy.hymba_kv_share_bind(c, p)
+    A = 1 << 44
+    try:
+        assert hy.hymba_layer_meta_workspace(p) == hy.hymba_layer_prefill_workspace(p, 1, 0)
+        assert hy.hymba_layer_prefill_cached_workspace(p, 4, 300) < hy.hymba_layer_prefill_workspace(p, 4, 300)
+        meta = hy.hymba_meta_cache(A, A, A, A, A, 0)
+        # a consumer needs its producer's meta cache, stamped by the producer
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_meta_precompute(c, A, meta, None, A, 1 << 30)
+        assert e.value.status == hy.HYMBA_ERR_NOT_BOUND
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_meta_precompute(c, A, meta, hy.hymba_meta_cache(A, A, A, A, A, 42), A, 1 << 30)
+        assert e.value.status == hy.HYMBA_ERR_NOT_BOUND
+        # a prefill from a meta cache this layer did not compute
+        kv = hy.hymba_kv_seq(A, A, 0, 0, 0)
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_prefill_cached(p, 2, 100, A, A, meta, kv, None, None, A, 1 << 34)
+        assert e.value.status == hy.HYMBA_ERR_NOT_BOUND
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_layer_prefill_cached(p, 2, 0, A, A, meta, kv, None, None, A, 1 << 34)
+        assert e.value.status == hy.HYMBA_ERR_INVALID_ARG
+        # no meta tokens, no meta cache
+        nom = hy.hymba_layer_create(_cfg(n_meta=0), _fake_weights(1 << 42))
+        with pytest.raises(hy.HymbaError):
+            hy.hymba_layer_meta_workspace(nom)
+        hy.hymba_layer_destroy(nom)
+    finally:
+        hy.hymba_layer_destroy(p)
+        hy.hymba_layer_destroy(c)
+
+
+def test_rope_configuration_is_validated():
+    h = hy.hymba_layer_create(_cfg(rope_base=10000.0), _fake_weights())
+    plain = hy.hymba_layer_create(_cfg(), _fake_weights(1 << 41))
+    try:
+        for bad, want in ((-1.0, hy.HYMBA_ERR_INVALID_ARG), (0.5, hy.HYMBA_ERR_UNSUPPORTED)):
+            with pytest.raises(hy.HymbaError) as e:
+                hy.hymba_layer_create(_cfg(rope_base=bad), _fake_weights(1 << 42))
+            assert e.value.status == want
+        # K/V sharing needs the same rotation on both sides
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_kv_share_bind(plain, h)
+        assert e.value.status == hy.HYMBA_ERR_NOT_BOUND
+        # the rotary table lives in the workspace
+        assert hy.hymba_layer_prefill_workspace(h, 2, 100) > hy.hymba_layer_prefill_workspace(plain, 2, 100)
+    finally:
+        hy.hymba_layer_destroy(h)
+        hy.hymba_layer_destroy(plain)

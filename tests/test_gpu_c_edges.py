@@ -10,6 +10,7 @@ import hybrid_attention_ssm_head_b200 as hy
 import synth
 from oracle import hymba_oracle as O
 from synth.configs import LayerDims
+from tests import _bounds as BD
 from tests import _harness as H
 
 pytestmark = pytest.mark.gpu
@@ -50,7 +51,10 @@ def test_edge_prefill(dtype, B, m, n, W):
         if dtype == "f32":
             H.close_f32(H.to64(h[b]), ref["h"], "h_final")
         else:
-            H.close_stage_dist(H.to64(h[b]), ref["h"], "h_final")
+            mag = BD.ssm_magnitudes(H.oracle_weights(lay.cpu), lay.spec, ref)
+            BD.close_mag(H.to64(h[b]), ref["h"], mag["h"], "h_final")
+            H.close_rel_l2(H.to64(h[b]), ref["h"], 1e-2, "h_final")
+            H.close_bf16(H.to64(conv[b]), ref["conv"], "conv_state")
     lay.close()
 
 
@@ -121,4 +125,27 @@ def test_decode_global_more_runs_than_a_warp():
     cache = {k: H.to64(t) for k, t in synth.configs.decode_caches(w, 0, cap, False, batch_index=0).items()}
     yo, _ = O.layer_decode(H.to64(xt[0]), pos, H.oracle_weights(lay.cpu), lay.spec, cache)
     H.close_bf16(H.to64(yt[0]), yo, "decode y, 35 runs")
+    lay.close()
+
+
+@pytest.mark.parametrize("batch", [129, 200])
+def test_decode_batch_over_128_rows(batch):
+    """More than 128 sequences: the decode projections take 256-row activation tiles."""
+    w = synth.configs.Workload(f"edge_dec_b{batch}", DIMS_BF16_SMALL, "bf16", batch, 16, 40, 32)
+    lay = H.GpuLayer(w, 0)
+    pos = w.n_meta + w.n_tokens
+    cap = w.n_meta + w.window
+    c = {k: t.contiguous() for k, t in synth.configs.decode_caches(w, 0, cap, False, device="cuda").items()}
+    kvc = hy.hymba_kv_cache(c["k"].data_ptr(), c["v"].data_ptr(), batch, cap, 0)
+    ssm = hy.hymba_ssm_cache(c["ssm"].data_ptr(), c["conv"].data_ptr())
+    dws = H.workspace(hy.hymba_layer_decode_workspace(lay.handle, batch, pos))
+    xt = synth.gen.normal_tensor((batch, w.dims.d_model), 0, f"edge_dec_b{batch}/x", device="cuda").to(torch.bfloat16)
+    yt = torch.empty_like(xt)
+    hy.hymba_layer_decode_step(lay.handle, batch, pos, xt, yt, kvc, ssm, dws, dws.numel(),
+                               torch.cuda.current_stream())
+    hy.hymba_stream_status(torch.cuda.current_stream())
+    for b in (0, 127, 128, batch - 1):
+        cache = {k: H.to64(t) for k, t in synth.configs.decode_caches(w, 0, cap, False, batch_index=b).items()}
+        yo, _ = O.layer_decode(H.to64(xt[b]), pos, H.oracle_weights(lay.cpu), lay.spec, cache)
+        H.close_bf16(H.to64(yt[b]), yo, f"decode y b={b}")
     lay.close()

@@ -13,6 +13,7 @@ import hybrid_attention_ssm_head_b200 as hy
 import synth
 from oracle import hymba_oracle as O
 from synth.configs import CFG0, CFG1, CFG2, CFG3, CFG4
+from tests import _bounds as BD
 from tests import _harness as H
 
 pytestmark = pytest.mark.gpu
@@ -29,7 +30,13 @@ def _prefill_workload(w, rows):
         xb = synth.configs.x_tilde(w, batch_index=b)  # regenerated on the CPU, same values
         ref = O.layer_prefill(H.to64(xb), H.oracle_weights(lay.cpu), lay.spec)
         H.close(w, H.to64(y[b]), ref["Y"], f"{w.name} Y[b={b}]")
-        H.close_stage_dist(H.to64(h[b]), ref["h"], f"{w.name} h_final[b={b}]")
+        if w.dtype == "f32":
+            H.close_f32(H.to64(h[b]), ref["h"], f"{w.name} h_final[b={b}]")
+        else:
+            mag = BD.ssm_magnitudes(H.oracle_weights(lay.cpu), lay.spec, ref)
+            BD.close_mag(H.to64(h[b]), ref["h"], mag["h"], f"{w.name} h_final[b={b}]")
+            H.close_rel_l2(H.to64(h[b]), ref["h"], 1e-2, f"{w.name} h_final[b={b}]")
+            H.close_bf16(H.to64(conv[b]), ref["conv"], f"{w.name} conv_state[b={b}]")
     lay.close()
 
 
@@ -126,10 +133,15 @@ def test_cfg4_decode_stack_full_sampled():
             if not consumer:
                 new_store[l] = newc
             H.close_bf16(H.to64(outs[l][b]), yo, f"layer {l} y_t[b={b}]")
-            H.close_stage_dist(H.to64(caches[l]["ssm"][b]), newc["ssm"], f"layer {l} h[b={b}]")
+            hm = BD.decode_state_magnitude(H.to64(xs[l][b]), pos, H.oracle_weights(lay.cpu), lay.spec, cache,
+                                           consumer)
+            BD.close_mag(H.to64(caches[l]["ssm"][b]), newc["ssm"], hm, f"layer {l} h[b={b}]")
+            H.close_rel_l2(H.to64(caches[l]["ssm"][b]), newc["ssm"], 1e-2, f"layer {l} h[b={b}]")
             np.testing.assert_array_equal(H.to64(caches[l]["conv"][b][:-1]), cache["conv"][1:])
+            H.close_bf16(H.to64(caches[l]["conv"][b][-1]), newc["conv"][-1], f"layer {l} conv new row")
             if not consumer:
                 sl = O.kv_slot(pos, lay.spec)
-                H.close_stage_dist(H.to64(caches[l]["k"][b][:, sl]), newc["k"][:, sl], f"layer {l} k slot")
+                H.close_bf16(H.to64(caches[l]["k"][b][:, sl]), newc["k"][:, sl], f"layer {l} k slot")
+                H.close_bf16(H.to64(caches[l]["v"][b][:, sl]), newc["v"][:, sl], f"layer {l} v slot")
     for lay in layers:
         lay.close()

@@ -7,6 +7,8 @@ import json
 import math
 import os
 
+from dataclasses import replace
+
 import numpy as np
 import pytest
 
@@ -331,9 +333,11 @@ def test_p8_causality_window_and_meta():
 
 # --- P9: prefill(n) then decode == prefill(n + 1) ------------------------------------------------
 
-@pytest.mark.parametrize("glob", [False, True])
-def test_p9_decode_after_prefill(glob):
+@pytest.mark.parametrize("glob,rope_base", [(False, 0.0), (True, 0.0), (False, 100.0), (True, 10000.0)])
+def test_p9_decode_after_prefill(glob, rope_base):
     s = _small.spec(m=3, W=4, is_global=glob)
+    if rope_base:
+        s = replace(s, rope_base=rope_base)
     wp = _small.weights(s, seed=31)
     wc = _small.weights(s, seed=32, consumer=True)
     L = 16
@@ -353,6 +357,43 @@ def test_p9_decode_after_prefill(glob):
     np.testing.assert_allclose(y_c, full_c["Y"][L], rtol=1e-11, atol=1e-12)
 
 
+# --- rotary position embedding (Hymba §2.5: a RoPE base; off in the five workloads) -------------
+
+def test_rope_closed_forms():
+    """Position 0 is the identity; every head keeps its norm; pair i at position p is the
+    complex product (x_2i + j x_2i+1) exp(j p base^(-2i/d)), computed here with Python's
+    complex numbers."""
+    rng = np.random.default_rng(7)
+    d, heads, base = 8, 3, 500.0
+    x = rng.normal(size=(5, heads * d))
+    pos = np.array([0, 1, 7, 1000, 8319])
+    r = O.rope(x, pos, d, base)
+    np.testing.assert_array_equal(r[0], x[0])
+    np.testing.assert_allclose(np.linalg.norm(r.reshape(5, heads, d), axis=2),
+                               np.linalg.norm(x.reshape(5, heads, d), axis=2), rtol=1e-13)
+    import cmath
+    for row, p in enumerate(pos):
+        for h in range(heads):
+            for i in range(d // 2):
+                z = complex(x[row, h * d + 2 * i], x[row, h * d + 2 * i + 1]) * cmath.exp(
+                    1j * p * base ** (-2.0 * i / d))
+                assert abs(complex(r[row, h * d + 2 * i], r[row, h * d + 2 * i + 1]) - z) <= 1e-9 * (1 + abs(z))
+
+
+def test_rope_scores_depend_only_on_the_relative_position():
+    rng = np.random.default_rng(8)
+    d, base = 16, 10000.0
+    q, k = rng.normal(size=(1, d)), rng.normal(size=(1, d))
+    for i, j, shift in [(5, 2, 100), (300, 0, 7), (8000, 7990, 123)]:
+        a = (O.rope(q, [i], d, base) @ O.rope(k, [j], d, base).T).item()
+        b = (O.rope(q, [i + shift], d, base) @ O.rope(k, [j + shift], d, base).T).item()
+        assert abs(a - b) <= 1e-9 * (1 + abs(a))
+    # and they do depend on it
+    a = (O.rope(q, [10], d, base) @ O.rope(k, [3], d, base).T).item()
+    b = (O.rope(q, [10], d, base) @ O.rope(k, [4], d, base).T).item()
+    assert abs(a - b) > 1e-3
+
+
 def test_ring_slots_hold_the_window():
     """Simulate appending positions one at a time into a ring of W slots after m meta slots;
     after every append the slots hold exactly the meta rows plus the last W positions."""
@@ -365,6 +406,25 @@ def test_ring_slots_hold_the_window():
             want = list(range(min(p + 1, m))) + list(range(max(m, p - W + 1), p + 1))
             assert held == want
             assert max(store) < m + W
+
+
+def test_decode_slot_bitmap_by_ring_simulation():
+    """The decode slot mask against a simulated store: append positions 0..pos one at a
+    time (each overwrites its slot), then mark the slots whose held position is visible
+    from pos under the mask predicate; before and after the ring wraps, and global."""
+    for m, W, glob in [(0, 1, False), (3, 4, False), (5, 7, False), (16, 64, False), (4, 1, True),
+                       (7, 0, True)]:
+        s = _small.spec(m=m, W=max(W, 1), is_global=glob)
+        for pos in range(m, m + 3 * max(W, 1) + 9):
+            cap = pos + 1 if glob else m + W
+            store = {}
+            for p in range(pos + 1):
+                store[p if glob or p < m else m + (p - m) % W] = p
+            want = np.zeros((cap + 31) // 32, dtype=np.uint32)
+            for slot, p in store.items():
+                if O.allowed(pos, p, m, max(W, 1), glob):
+                    want[slot // 32] |= np.uint32(1 << (slot % 32))
+            np.testing.assert_array_equal(O.decode_slot_bitmap(pos, s, cap), want)
 
 
 # --- P10: the printed cache sizes fix the value head width -------------------------------------
