@@ -56,6 +56,11 @@ class hymba_meta_cache(C.Structure):
                 ("y", C.c_void_p), ("owner", C.c_uint64)]
 
 
+class hymba_block_weights(C.Structure):
+    _fields_ = [("norm1", C.c_void_p), ("norm2", C.c_void_p), ("w_gate_up", C.c_void_p),
+                ("w_down", C.c_void_p), ("mlp_hidden", C.c_int)]
+
+
 class hymba_prefill_layout(C.Structure):
     _fields_ = [(n, C.c_size_t) for n in ("q", "x_ssm", "gate", "u", "xdbl", "delta", "y_ssm",
                                           "o_attn", "fused", "rope", "total")]
@@ -97,6 +102,15 @@ _SIGS = {
                                              C.POINTER(hymba_meta_cache), C.POINTER(hymba_kv_seq),
                                              C.POINTER(hymba_kv_cache), C.POINTER(hymba_ssm_cache),
                                              C.c_void_p, C.c_size_t, C.c_void_p]),
+    "hymba_block_prefill_workspace": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_int, C.POINTER(C.c_size_t)]),
+    "hymba_block_prefill": (C.c_int, [C.c_void_p, C.POINTER(hymba_block_weights), C.c_int, C.c_int,
+                                      C.c_void_p, C.c_void_p, C.POINTER(hymba_kv_seq),
+                                      C.POINTER(hymba_kv_cache), C.POINTER(hymba_ssm_cache), C.c_void_p,
+                                      C.c_size_t, C.c_void_p]),
+    "hymba_block_decode_workspace": (C.c_int, [C.c_void_p, C.c_int, C.c_int, C.c_int64, C.POINTER(C.c_size_t)]),
+    "hymba_block_decode_step": (C.c_int, [C.c_void_p, C.POINTER(hymba_block_weights), C.c_int, C.c_int64,
+                                          C.c_void_p, C.c_void_p, C.POINTER(hymba_kv_cache),
+                                          C.POINTER(hymba_ssm_cache), C.c_void_p, C.c_size_t, C.c_void_p]),
     "hymba_layer_decode_workspace": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.POINTER(C.c_size_t)]),
     "hymba_layer_decode_step": (C.c_int, [C.c_void_p, C.c_int, C.c_int64, C.c_void_p, C.c_void_p,
                                           C.POINTER(hymba_kv_cache), C.POINTER(hymba_ssm_cache),
@@ -234,6 +248,44 @@ def hymba_layer_prefill_cached(layer: int, batch: int, n_tokens: int, x, y, meta
         C.byref(kv_cache) if kv_cache is not None else None,
         C.byref(ssm_cache) if ssm_cache is not None else None,
         _ptr(workspace), workspace_bytes, _stream(stream)), "hymba_layer_prefill_cached")
+
+
+def make_block_weights(w: dict) -> hymba_block_weights:
+    """From device tensors norm1, norm2 [d] fp32, w_gate_up [2F, d] (rows interleaved), w_down [d, F]."""
+    return hymba_block_weights(_ptr(w["norm1"]), _ptr(w["norm2"]), _ptr(w["w_gate_up"]), _ptr(w["w_down"]),
+                               int(w["w_down"].shape[1]))
+
+
+def hymba_block_prefill_workspace(layer: int, mlp_hidden: int, batch: int, n_tokens: int) -> int:
+    out = C.c_size_t()
+    check(lib().hymba_block_prefill_workspace(layer, mlp_hidden, batch, n_tokens, C.byref(out)),
+          "hymba_block_prefill_workspace")
+    return out.value
+
+
+def hymba_block_prefill(layer: int, bw: hymba_block_weights, batch: int, n_tokens: int, x, y, kv: hymba_kv_seq,
+                        kv_cache: hymba_kv_cache | None, ssm_cache: hymba_ssm_cache | None, workspace,
+                        workspace_bytes: int, stream=None) -> None:
+    check(lib().hymba_block_prefill(
+        layer, C.byref(bw), batch, n_tokens, _ptr(x), _ptr(y), C.byref(kv),
+        C.byref(kv_cache) if kv_cache is not None else None,
+        C.byref(ssm_cache) if ssm_cache is not None else None,
+        _ptr(workspace), workspace_bytes, _stream(stream)), "hymba_block_prefill")
+
+
+def hymba_block_decode_workspace(layer: int, mlp_hidden: int, batch: int, max_pos: int) -> int:
+    out = C.c_size_t()
+    check(lib().hymba_block_decode_workspace(layer, mlp_hidden, batch, max_pos, C.byref(out)),
+          "hymba_block_decode_workspace")
+    return out.value
+
+
+def hymba_block_decode_step(layer: int, bw: hymba_block_weights, batch: int, pos: int, x_t, y_t,
+                            kv_cache: hymba_kv_cache, ssm_cache: hymba_ssm_cache, workspace, workspace_bytes: int,
+                            stream=None) -> None:
+    check(lib().hymba_block_decode_step(layer, C.byref(bw), batch, pos, _ptr(x_t), _ptr(y_t), C.byref(kv_cache),
+                                        C.byref(ssm_cache), _ptr(workspace), workspace_bytes, _stream(stream)),
+          "hymba_block_decode_step")
 
 
 def hymba_layer_decode_workspace(layer: int, batch: int, max_pos: int) -> int:

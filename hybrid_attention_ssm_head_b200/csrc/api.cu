@@ -360,6 +360,7 @@ struct PrefillRun {
   const float *h0;    // broadcast initial SSM state [E, N] or null
   const void *conv0;  // broadcast conv history [K-1, E] or null
   bool meta;          // the meta-cache precompute: its steps are profiled under "meta_*" names
+  const void *resid;  // [B, rows, d] added to the output by the output projection (block) or null
 };
 // Profiler step name of a prefill step (the meta-cache precompute has its own names).
 static const char *step_name(const PrefillRun &r, int step) {
@@ -401,7 +402,6 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
     g.N = qk_width(c) + (consumer ? 0 : k_width(c) + v_width(c)) + 2 * E;
     g.K = c.d_model;
     g.elem = (int)es;
-    g.ksplit = 1;
     g.epi = in_proj_epilogue(c, consumer, q, qk_width(c), kv->k, kv->v, k_width(c), v_width(c), 0, 0,
                              xs, z, E);
     if (!consumer && r.q_off > 0) {
@@ -452,7 +452,6 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
     g.N = xdbl_width(c);
     g.K = E;
     g.elem = (int)es;
-    g.ksplit = 1;
     g.epi.seg[0] = seg(xdbl, xdbl_width(c), 0, xdbl_width(c), 1, es);
     g.epi.nseg = 1;
     if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
@@ -469,7 +468,6 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
     g.N = E;
     g.K = c.dt_rank;
     g.elem = 4;
-    g.ksplit = 1;
     g.epi.seg[0] = seg(delta, E, 0, E, c.dtype == HYMBA_F32, es);
     g.epi.nseg = 1;
     g.epi.bias = layer->w.b_dt;
@@ -549,8 +547,9 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
     g.N = c.d_model;
     g.K = E;
     g.elem = (int)es;
-    g.ksplit = 1;
     g.epi.seg[0] = seg(r.y, c.d_model, 0, c.d_model, c.dtype == HYMBA_F32, es);
+    g.epi.seg[0].resid = r.resid;
+    g.epi.seg[0].ld_resid = c.d_model;
     g.epi.nseg = 1;
     g.stall = take_debug_stall();
     if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
@@ -802,12 +801,11 @@ hymba_status hymba_layer_decode_workspace(const hymba_layer *layer, int batch, i
   return HYMBA_OK;
 }
 
-hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos, const void *x_t,
-                                     void *y_t, hymba_kv_cache *kv_cache, hymba_ssm_cache *ssm_cache,
-                                     void *workspace, size_t workspace_bytes,
-                                     hymba_stream_t stream_) {
-  g_msg[0] = 0;
-  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+// The decode step of the mixer; `resid` (optional, [batch, d_model]) is added to its output
+// by the output projection (the block's residual).
+static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const void *x_t, void *y_t,
+                               const void *resid, hymba_kv_cache *kv_cache, hymba_ssm_cache *ssm_cache,
+                               void *workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!layer) FAIL(HYMBA_ERR_INVALID_ARG, "null layer");
   const hymba_layer_config &c = layer->cfg;
   const bool consumer = layer->producer != nullptr;
@@ -857,7 +855,6 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
     g.N = qk_width(c) + (consumer ? 0 : k_width(c) + v_width(c)) + 2 * E;
     g.K = c.d_model;
     g.elem = (int)es;
-    g.ksplit = 1;
     char *kbase = reinterpret_cast<char *>(kv_cache->k) + (size_t)slot * c.head_dim_qk * es;
     char *vbase = reinterpret_cast<char *>(kv_cache->v) + (size_t)slot * c.head_dim_v * es;
     g.epi = in_proj_epilogue(c, consumer, q, qk_width(c), kbase, vbase,
@@ -875,12 +872,9 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
       g.epi.seg[0].rope = 1;
       if (!consumer) g.epi.seg[1].rope = 1;
     }
-    // x_proj's accumulators (summed by the SSM kernel's channel blocks) start at zero
-    g.epi.zero = xdbl;
-    g.epi.zero_n = (long long)batch * xdbl_width(c);
     if ((st = gemm_decode(g, c.dtype, stream)) != HYMBA_OK) return st;
   }
-  // 2-5. SSM branch: conv + x_proj, then dt_proj + softplus + one scan step + gate
+  // 2-5. SSM branch: conv + SiLU, x_proj, then dt_proj + softplus + one scan step + gate
   {
     ProfScope prof_scope(stream, "dec_ssm");
     DecodeSsmArgs a{};
@@ -891,7 +885,6 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
     a.conv_state = ssm_cache->conv;
     a.conv_w = layer->w.conv_w;
     a.conv_b = layer->w.conv_b;
-    a.w_x = layer->w.w_x;
     a.xdbl = xdbl;
     a.u = u;
     a.w_dt = layer->w.w_dt;
@@ -905,7 +898,20 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
     a.K = c.d_conv;
     a.R = c.dt_rank;
     a.N = c.d_state;
-    if ((st = decode_ssm(a, c.dtype, stream)) != HYMBA_OK) return st;
+    if ((st = decode_conv(a, c.dtype, stream)) != HYMBA_OK) return st;
+    GemmArgs g{};
+    g.A = u;
+    g.lda = E;
+    g.B = layer->w.w_x;
+    g.ldb = E;
+    g.M = batch;
+    g.N = xdbl_width(c);
+    g.K = E;
+    g.elem = (int)es;
+    g.epi.seg[0] = seg(xdbl, xdbl_width(c), 0, xdbl_width(c), 1, es);
+    g.epi.nseg = 1;
+    if ((st = gemm_decode(g, c.dtype, stream)) != HYMBA_OK) return st;
+    if ((st = decode_scan(a, c.dtype, stream)) != HYMBA_OK) return st;
   }
   // 6. single-query attention over the store
   int fuse_nchunks = 0;
@@ -978,13 +984,193 @@ hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos,
     g.N = c.d_model;
     g.K = E;
     g.elem = (int)es;
-    g.ksplit = 1;
     g.epi.seg[0] = seg(y_t, c.d_model, 0, c.d_model, c.dtype == HYMBA_F32, es);
+    g.epi.seg[0].resid = resid;
+    g.epi.seg[0].ld_resid = c.d_model;
     g.epi.nseg = 1;
     if ((st = gemm_decode(g, c.dtype, stream)) != HYMBA_OK) return st;
   }
   if (!consumer) kv_cache->owner = layer->id;
   return HYMBA_OK;
+}
+
+hymba_status hymba_layer_decode_step(hymba_layer *layer, int batch, int64_t pos, const void *x_t,
+                                     void *y_t, hymba_kv_cache *kv_cache, hymba_ssm_cache *ssm_cache,
+                                     void *workspace, size_t workspace_bytes,
+                                     hymba_stream_t stream) {
+  g_msg[0] = 0;
+  return decode_run(layer, batch, pos, x_t, y_t, nullptr, kv_cache, ssm_cache, workspace, workspace_bytes,
+                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------------------------
+// the Hymba block: x + mixer(norm1(x)), then + MLP(norm2(.)) (Fig. 4 (b); Table 11)
+// ---------------------------------------------------------------------------
+static hymba_status check_block(const hymba_layer *layer, const hymba_block_weights *bw) {
+  if (!layer || !bw) FAIL(HYMBA_ERR_INVALID_ARG, "null layer or block weights");
+  const hymba_layer_config &c = layer->cfg;
+  if (!bw->norm1 || !bw->norm2 || !bw->w_gate_up || !bw->w_down || !aligned16(bw->norm1) ||
+      !aligned16(bw->norm2) || !aligned16(bw->w_gate_up) || !aligned16(bw->w_down))
+    FAIL(HYMBA_ERR_INVALID_ARG, "block weights null or misaligned");
+  if (bw->mlp_hidden < 8 || bw->mlp_hidden % 8) FAIL(HYMBA_ERR_UNSUPPORTED, "mlp_hidden must be a multiple of 8");
+  const int V = c.dtype == HYMBA_BF16 ? 8 : 4;
+  if (c.d_model % V || c.d_model / V > 256) FAIL(HYMBA_ERR_UNSUPPORTED, "d_model too wide for the block's norm");
+  return HYMBA_OK;
+}
+
+// Block workspace: the mixer's own, then the normed rows [M, d] and the MLP's hidden rows [M, F].
+struct BlockLayout {
+  size_t mixer, xn, hid, total;
+};
+static BlockLayout block_layout(size_t mixer_bytes, const hymba_layer_config &c, long long M, int F) {
+  BlockLayout b{};
+  b.mixer = 0;
+  b.xn = up256(mixer_bytes);
+  b.hid = b.xn + up256((size_t)M * c.d_model * esize(c.dtype));
+  b.total = b.hid + up256((size_t)M * F * esize(c.dtype));
+  return b;
+}
+
+hymba_status hymba_block_prefill_workspace(const hymba_layer *layer, int mlp_hidden, int batch, int n_tokens,
+                                           size_t *bytes) {
+  g_msg[0] = 0;
+  if (!bytes || mlp_hidden < 1) FAIL(HYMBA_ERR_INVALID_ARG, "null output or mlp_hidden < 1");
+  hymba_prefill_layout lay;
+  hymba_status st = prefill_layout(layer, batch, n_tokens, &lay, nullptr);
+  if (st != HYMBA_OK) return st;
+  const long long M = (long long)batch * (layer->cfg.n_meta + n_tokens);
+  *bytes = block_layout(lay.total, layer->cfg, M, mlp_hidden).total;
+  return HYMBA_OK;
+}
+
+// MLP of M rows: hid = SiLU(hn W_gate^T) * (hn W_up^T); y += hid W_down^T (y holds h).
+static hymba_status block_mlp(const hymba_layer *layer, const hymba_block_weights *bw, long long M, const void *hn,
+                              void *hid, void *y, bool decode, cudaStream_t stream) {
+  const hymba_layer_config &c = layer->cfg;
+  const size_t es = esize(c.dtype);
+  const int F = bw->mlp_hidden;
+  hymba_status st;
+  {
+    ProfScope prof_scope(stream, decode ? "dec_mlp_up" : "mlp_up");
+    GemmArgs g{};
+    g.A = hn;
+    g.lda = c.d_model;
+    g.B = bw->w_gate_up;
+    g.ldb = c.d_model;
+    g.M = (int)M;
+    g.N = 2 * F;
+    g.K = c.d_model;
+    g.elem = (int)es;
+    g.epi.seg[0] = seg(hid, F, 0, 2 * F, c.dtype == HYMBA_F32, es);
+    g.epi.seg[0].act = 3;
+    g.epi.nseg = 1;
+    if ((st = decode ? gemm_decode(g, c.dtype, stream) : gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
+  }
+  {
+    ProfScope prof_scope(stream, decode ? "dec_mlp_down" : "mlp_down");
+    GemmArgs g{};
+    g.A = hid;
+    g.lda = F;
+    g.B = bw->w_down;
+    g.ldb = F;
+    g.M = (int)M;
+    g.N = c.d_model;
+    g.K = F;
+    g.elem = (int)es;
+    g.epi.seg[0] = seg(y, c.d_model, 0, c.d_model, c.dtype == HYMBA_F32, es);
+    g.epi.seg[0].resid = y;  // in place: each element is read, then written, by one thread
+    g.epi.seg[0].ld_resid = c.d_model;
+    g.epi.nseg = 1;
+    if ((st = decode ? gemm_decode(g, c.dtype, stream) : gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
+  }
+  return HYMBA_OK;
+}
+
+hymba_status hymba_block_prefill(hymba_layer *layer, const hymba_block_weights *bw, int batch, int n_tokens,
+                                 const void *x, void *y, hymba_kv_seq *kv, hymba_kv_cache *kv_cache,
+                                 hymba_ssm_cache *ssm_cache, void *workspace, size_t workspace_bytes,
+                                 hymba_stream_t stream_) {
+  g_msg[0] = 0;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  hymba_status st = check_block(layer, bw);
+  if (st != HYMBA_OK) return st;
+  hymba_prefill_layout lay;
+  if ((st = prefill_layout(layer, batch, n_tokens, &lay, nullptr)) != HYMBA_OK) return st;
+  const hymba_layer_config &c = layer->cfg;
+  const int L = c.n_meta + n_tokens;
+  const long long M = (long long)batch * L;
+  const BlockLayout bl = block_layout(lay.total, c, M, bw->mlp_hidden);
+  if (!x || !y || !aligned16(x) || !aligned16(y) || x == y) FAIL(HYMBA_ERR_INVALID_ARG, "x/y null, misaligned or the same");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    FAIL(HYMBA_ERR_INVALID_ARG, "workspace null or not 256-byte aligned");
+  if (workspace_bytes < bl.total)
+    FAIL(HYMBA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, bl.total);
+  if ((st = check_prefill_kv(layer, batch, L, kv, kv_cache, ssm_cache)) != HYMBA_OK) return st;
+  char *ws = reinterpret_cast<char *>(workspace);
+  void *xn = ws + bl.xn, *hid = ws + bl.hid;
+  {
+    ProfScope prof_scope(stream, "norm1");
+    if ((st = rms_norm_rows(x, bw->norm1, xn, M, c.d_model, c.rms_eps, c.dtype, stream)) != HYMBA_OK) return st;
+  }
+  PrefillRun r{};
+  r.x = xn;
+  r.y = y;
+  r.rows = L;
+  r.q_off = 0;
+  r.resid = x;  // y = x + mixer(norm1(x))
+  if ((st = prefill_run(layer, batch, r, kv, kv_cache, ssm_cache, workspace, lay, stream)) != HYMBA_OK) return st;
+  {
+    ProfScope prof_scope(stream, "norm2");
+    if ((st = rms_norm_rows(y, bw->norm2, xn, M, c.d_model, c.rms_eps, c.dtype, stream)) != HYMBA_OK) return st;
+  }
+  return block_mlp(layer, bw, M, xn, hid, y, false, stream);
+}
+
+hymba_status hymba_block_decode_workspace(const hymba_layer *layer, int mlp_hidden, int batch, int64_t max_pos,
+                                          size_t *bytes) {
+  g_msg[0] = 0;
+  size_t mixer = 0;
+  hymba_status st = hymba_layer_decode_workspace(layer, batch, max_pos, &mixer);
+  if (st != HYMBA_OK) return st;
+  if (mlp_hidden < 1) FAIL(HYMBA_ERR_INVALID_ARG, "mlp_hidden < 1");
+  *bytes = block_layout(mixer, layer->cfg, batch, mlp_hidden).total;
+  return HYMBA_OK;
+}
+
+hymba_status hymba_block_decode_step(hymba_layer *layer, const hymba_block_weights *bw, int batch, int64_t pos,
+                                     const void *x_t, void *y_t, hymba_kv_cache *kv_cache,
+                                     hymba_ssm_cache *ssm_cache, void *workspace, size_t workspace_bytes,
+                                     hymba_stream_t stream_) {
+  g_msg[0] = 0;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  hymba_status st = check_block(layer, bw);
+  if (st != HYMBA_OK) return st;
+  const hymba_layer_config &c = layer->cfg;
+  if (batch < 1 || pos < c.n_meta) FAIL(HYMBA_ERR_INVALID_ARG, "batch < 1 or pos is a meta position");
+  const size_t mixer = decode_layout(c, batch, pos).total;
+  const BlockLayout bl = block_layout(mixer, c, batch, bw->mlp_hidden);
+  if (!x_t || !y_t || !aligned16(x_t) || !aligned16(y_t) || x_t == y_t)
+    FAIL(HYMBA_ERR_INVALID_ARG, "x_t/y_t null, misaligned or the same");
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    FAIL(HYMBA_ERR_INVALID_ARG, "workspace null or not 256-byte aligned");
+  if (workspace_bytes < bl.total)
+    FAIL(HYMBA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, bl.total);
+  char *ws = reinterpret_cast<char *>(workspace);
+  void *xn = ws + bl.xn, *hid = ws + bl.hid;
+  {
+    ProfScope prof_scope(stream, "dec_norm1");
+    if ((st = rms_norm_rows(x_t, bw->norm1, xn, batch, c.d_model, c.rms_eps, c.dtype, stream)) != HYMBA_OK)
+      return st;
+  }
+  if ((st = decode_run(layer, batch, pos, xn, y_t, x_t, kv_cache, ssm_cache, workspace, mixer, stream)) !=
+      HYMBA_OK)
+    return st;
+  {
+    ProfScope prof_scope(stream, "dec_norm2");
+    if ((st = rms_norm_rows(y_t, bw->norm2, xn, batch, c.d_model, c.rms_eps, c.dtype, stream)) != HYMBA_OK)
+      return st;
+  }
+  return block_mlp(layer, bw, batch, xn, hid, y_t, true, stream);
 }
 
 // ---------------------------------------------------------------------------

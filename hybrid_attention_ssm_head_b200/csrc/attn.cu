@@ -21,6 +21,7 @@
 //
 // fp32 path and decode: CUDA-core kernels (small or bandwidth-bound work).
 #include <algorithm>
+#include <cstdlib>
 #include <math.h>
 
 #include "common.cuh"
@@ -168,13 +169,14 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s0)[32], const uint
 // pair in four takes its exponentials from the degree-3 polynomial on the FMA pipe
 // (relative error 7.5e-5, well inside the bf16 rounding of P) and the others from
 // the MUFU, so that the two pipes share the exponentials.
+template <int POLY8>
 __device__ __forceinline__ float2 p_pack(const uint32_t (&v)[32], uint32_t (&pk)[16], float2 scale2,
                                          float2 nm2) {
   float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     const float2 x = ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scale2, nm2);
-    const float2 p = ((e >> 1) & 3) == 0 ? exp2_poly2<3>(x) : make_float2(ex2(x.x), ex2(x.y));
+    const float2 p = ((e >> 1) & 7) < POLY8 ? exp2_poly2<3>(x) : make_float2(ex2(x.x), ex2(x.y));
     ls[(e >> 1) & 1] = fadd2(ls[(e >> 1) & 1], p);
     pk[e >> 1] = pack_bf16x2(p.x, p.y);
   }
@@ -197,6 +199,7 @@ __device__ __forceinline__ void p_store(const uint32_t (&pk)[16], int c, int r, 
 // item's Q and first K/V tiles stream in, and its first S = Q K^T is issued, while the
 // current item's last tile is still in the softmax; the softmax warpgroups write the
 // finished item's O between its last tile and the next item's first.
+template <int POLY8>
 __global__ void __launch_bounds__(fa::THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -455,8 +458,8 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
         const float2 nm2 = make_float2(nm, nm), scale2 = make_float2(scale_log2, scale_log2);
         uint32_t pk0[16], pk1[16], pk2[16], pk3[16];
-        const float2 ps = fadd2(fadd2(p_pack(s0, pk0, scale2, nm2), p_pack(s1, pk1, scale2, nm2)),
-                                fadd2(p_pack(s2, pk2, scale2, nm2), p_pack(s3, pk3, scale2, nm2)));
+        const float2 ps = fadd2(fadd2(p_pack<POLY8>(s0, pk0, scale2, nm2), p_pack<POLY8>(s1, pk1, scale2, nm2)),
+                                fadd2(p_pack<POLY8>(s2, pk2, scale2, nm2), p_pack<POLY8>(s3, pk3, scale2, nm2)));
         l_run += ps.x + ps.y;
         if (__any_sync(0xffffffffu, resc)) {
           // O grows by the new max: rescale it once the previous tile's P V has retired
@@ -532,13 +535,14 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
   }
 }
 
+template <int POLY8>
 static hymba_status attention_prefill_tc(const AttnArgs &a, cudaStream_t s) {
   using namespace fa;
   static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set.done(dev)) {
-    if (cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
+    if (cudaFuncSetAttribute(attn_fwd_tc_kernel<POLY8>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
         cudaSuccess) {
       set_error("cudaFuncSetAttribute(attention smem) failed");
       return HYMBA_ERR_CUDA;
@@ -567,7 +571,7 @@ static hymba_status attention_prefill_tc(const AttnArgs &a, cudaStream_t s) {
   const long long items = (long long)npairs * a.H * a.B;
   if (items == 0) return HYMBA_OK;
   const unsigned grid = (unsigned)std::min<long long>(items, sms);
-  attn_fwd_tc_kernel<<<grid, THREADS, SMEM, s>>>(
+  attn_fwd_tc_kernel<POLY8><<<grid, THREADS, SMEM, s>>>(
       tq, tk, tv, to, a.L, a.q_off, a.B, a.H, a.Hkv, a.n_meta, a.window,
       a.is_global, a.scale * 1.4426950408889634f, npairs, wait_limit_cycles());
   note_launch(1);
@@ -633,7 +637,14 @@ hymba_status attention_prefill(const AttnArgs &a, hymba_dtype dt, cudaStream_t s
       set_error("bf16 attention kernel supports head_dim_qk 64 and head_dim_v 128 only");
       return HYMBA_ERR_UNSUPPORTED;
     }
-    return attention_prefill_tc(a, s);
+    static const int poly8 = [] { const char *e = getenv("HYMBA_EXP_POLY8"); return e ? atoi(e) : 2; }();
+    switch (poly8) {
+      case 3: return attention_prefill_tc<3>(a, s);
+      case 4: return attention_prefill_tc<4>(a, s);
+      case 5: return attention_prefill_tc<5>(a, s);
+      case 6: return attention_prefill_tc<6>(a, s);
+      default: return attention_prefill_tc<2>(a, s);
+    }
   }
   if (a.dv > 256) {
     set_error("fp32 attention supports head_dim_v <= 256");
@@ -899,27 +910,29 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---- bf16 decode attention on the tensor cores (mma.sync m16n8k16) ---------------
-// Persistent: the work is the list of 128-slot chunks of every (sequence, kv head),
+// Persistent: the work is the list of 64-slot chunks of every (sequence, kv head),
 // item i = (b * Hkv + g) * nchunks + chunk, cut into equal contiguous ranges, one per
-// CTA (two CTAs per SM).  A CTA streams its chunks through two shared-memory stages by
-// 3-D TMA (128-byte swizzle, rows past the store's capacity read as zero), the copy of
-// the next chunk in flight while the current one is computed, across (sequence, kv
-// head) boundaries too.  Warp w takes keys 32w..32w+31 of every chunk: S = Q K^T with
+// CTA (two CTAs per SM).  A CTA streams its chunks through four shared-memory stages by
+// 3-D TMA (128-byte swizzle, rows past the store's capacity read as zero), the copies of
+// the next three chunks in flight while the current one is computed, across (sequence, kv
+// head) boundaries too.  Warp w takes keys 16w..16w+15 of every chunk: S = Q K^T with
 // the query heads of the group in rows 0..rep-1 of a 16-row tile, an online softmax in
 // registers, O += P V with V fragments from ldmatrix.trans.  Where a run of chunks of
 // one (sequence, kv head) ends inside the CTA's range, the four warps' states are
 // merged in shared memory into one partial (max, sum, O) per query head, stored at the
 // slot of the run's first chunk; the combine kernel reads the run-start slots.
 namespace dtc {
-constexpr int SLOTS = 128;
+constexpr int SLOTS = 64;                   // slots per chunk: 16 per warp
+constexpr int STAGES = 4;                   // chunks in flight per CTA: three ahead of the one computed
 constexpr int K_BYTES = SLOTS * 128;        // 64 bf16 per slot
 constexpr int V_BYTES = SLOTS * 256;        // two 64-column boxes
 constexpr int STAGE = K_BYTES + V_BYTES;
 constexpr int MAXREP = 8;
 // merge buffer [4 warps][rep][130] floats after the stages: two CTAs per SM for rep <= 5
 __host__ __device__ constexpr int merge_bytes(int rep) { return 4 * rep * 130 * 4; }
-__host__ __device__ constexpr int smem_bytes(int rep) { return 2 * STAGE + merge_bytes(rep) + 64 + 1024; }
+__host__ __device__ constexpr int smem_bytes(int rep) { return STAGES * STAGE + merge_bytes(rep) + 8 * STAGES + 1024; }
 constexpr int CTAS_PER_SM = 2;
+static_assert(SLOTS == 64, "the warps' key mapping takes 16 slots each");
 }  // namespace dtc
 
 // First chunk of every run: a run starts at chunk 0 of a (sequence, kv head) or at the
@@ -962,8 +975,8 @@ __global__ void __launch_bounds__(128)
   extern __shared__ uint8_t dsm_raw[];
   uint8_t *sm = dsm_raw + ((1024 - (smem_u32(dsm_raw) & 1023)) & 1023);
   const int rep = H / Hkv;
-  float *mw = reinterpret_cast<float *>(sm + 2 * STAGE);                         // [4 warps][rep][130]
-  uint64_t *full = reinterpret_cast<uint64_t *>(sm + 2 * STAGE + merge_bytes(rep));  // [2]
+  float *mw = reinterpret_cast<float *>(sm + STAGES * STAGE);                         // [4 warps][rep][130]
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + STAGES * STAGE + merge_bytes(rep));  // [STAGES]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = lane >> 2, gc = lane & 3;  // mma group row / column pair
   const long long nslots = dec_slots(pos, n_meta, window, is_global);
@@ -972,18 +985,18 @@ __global__ void __launch_bounds__(128)
   const long long i1 = min(n_items, i0 + per);
   if (i0 >= i1) return;
   const int nloc = (int)(i1 - i0);
-  auto issue = [&](int k) {  // item i0 + k into stage k & 1
+  auto issue = [&](int k) {  // item i0 + k into stage k % STAGES
     const long long it = i0 + k;
     const int bg = (int)(it / nchunks), s0 = (int)(it % nchunks) * SLOTS;
-    uint8_t *dst = sm + (k & 1) * STAGE;
-    mbar_arrive_expect_tx(&full[k & 1], STAGE);
-    tma_load_3d(dst, &tmK, &full[k & 1], 0, s0, bg);
-    tma_load_3d(dst + K_BYTES, &tmV, &full[k & 1], 0, s0, bg);
-    tma_load_3d(dst + K_BYTES + V_BYTES / 2, &tmV, &full[k & 1], 64, s0, bg);
+    const int st = k % STAGES;
+    uint8_t *dst = sm + st * STAGE;
+    mbar_arrive_expect_tx(&full[st], STAGE);
+    tma_load_3d(dst, &tmK, &full[st], 0, s0, bg);
+    tma_load_3d(dst + K_BYTES, &tmV, &full[st], 0, s0, bg);
+    tma_load_3d(dst + K_BYTES + V_BYTES / 2, &tmV, &full[st], 64, s0, bg);
   };
   if (tid == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
+    for (int st = 0; st < STAGES; ++st) mbar_init(&full[st], 1);
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -991,7 +1004,7 @@ __global__ void __launch_bounds__(128)
   __syncthreads();
   int issued = 0;
   if (tid == 0)
-    for (; issued < min(2, nloc); ++issued) issue(issued);
+    for (; issued < min(STAGES, nloc); ++issued) issue(issued);
   float m_run = -INFINITY, l_run = 0.f;  // row gr of this warp
   float oacc[16][4];
   uint32_t qa[4][2];  // Q fragments [k-step][a0a1 / a4a5]; rows 8..15 are zero
@@ -1017,20 +1030,20 @@ __global__ void __launch_bounds__(128)
         qa[ks][1] = live ? __ldg(qr + ks * 8 + 4 + gc) : 0u;
       }
     }
-    const int st = k & 1;
-    ok = mbar_wait(&full[st], uint32_t(k >> 1) & 1u, &g_err_attn, wlim);
+    const int st = k % STAGES;
+    ok = mbar_wait(&full[st], uint32_t(k / STAGES) & 1u, &g_err_attn, wlim);
     if (__syncthreads_or(!ok)) { ok = false; break; }
     const uint32_t kb = smem_u32(sm + st * STAGE), vb = kb + K_BYTES;
     const long long s0 = (long long)chunk * SLOTS;
-    // ---- S = Q K^T for this warp's 32 keys (4 n-tiles of 8 keys) ----
-    float sacc[4][4];
+    // ---- S = Q K^T for this warp's 16 keys (2 n-tiles of 8 keys) ----
+    float sacc[2][4];
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const int key = warp * 32 + nt * 8 + (lane & 7);
+    for (int nt = 0; nt < 2; ++nt) {
+      const int key = warp * 16 + nt * 8 + (lane & 7);
 #pragma unroll
       for (int kp = 0; kp < 2; ++kp) {  // two k-steps per ldmatrix.x4
         const int ch = kp * 4 + (lane >> 3);  // 16-byte chunk of the key row (8 dims)
@@ -1043,10 +1056,10 @@ __global__ void __launch_bounds__(128)
     // ---- online softmax, row gr (values sacc[nt][0..1], keys 8nt + 2gc + {0,1}) ----
     float mx = -INFINITY;
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int key = warp * 32 + nt * 8 + 2 * gc + e;
+        const int key = warp * 16 + nt * 8 + 2 * gc + e;
         const bool valid = dec_key_valid(s0 + key, nslots, pos, n_meta, window, is_global);
         const float x = valid ? sacc[nt][e] * scale_log2 : -INFINITY;
         sacc[nt][e] = x;
@@ -1059,9 +1072,9 @@ __global__ void __launch_bounds__(128)
     const float alpha = m_run == -INFINITY ? 0.f : ex2(m_run - mref);
     m_run = m_new;
     float lsum = 0.f;
-    uint32_t pa[4];  // P as A fragments: [k-step kk][a0a1 (n-tile 2kk) / a4a5 (n-tile 2kk+1)]
+    uint32_t pa[2];  // P as the A fragment of one 16-key step: a0a1 (n-tile 0) / a4a5 (n-tile 1)
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
+    for (int nt = 0; nt < 2; ++nt) {
       const float p0 = ex2(sacc[nt][0] - mref), p1 = ex2(sacc[nt][1] - mref);
       lsum += p0 + p1;
       pa[nt] = pack_bf16x2(p0, p1);
@@ -1074,10 +1087,10 @@ __global__ void __launch_bounds__(128)
       oacc[nt][0] *= alpha;
       oacc[nt][1] *= alpha;
     }
-    // ---- O += P V (16 n-tiles of 8 value columns, 2 k-steps of 16 keys) ----
-#pragma unroll
-    for (int kk = 0; kk < 2; ++kk) {
-      const int key = warp * 32 + kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    // ---- O += P V (16 n-tiles of 8 value columns, one k-step of 16 keys) ----
+    {
+      const int kk = 0;
+      const int key = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int np = 0; np < 8; ++np) {  // pairs of n-tiles per ldmatrix.x4.trans
         const int chg = np * 2 + (lane >> 4);  // 16-byte chunk of value columns (0..15)
@@ -1086,6 +1099,7 @@ __global__ void __launch_bounds__(128)
         ldsm_x4_t(addr, b0, b1, b2, b3);
         mma16816(oacc[2 * np], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b0, b1);
         mma16816(oacc[2 * np + 1], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b2, b3);
+        (void)kk;
       }
     }
     __syncthreads();  // every warp is done with stage st
@@ -1128,7 +1142,8 @@ __global__ void __launch_bounds__(128)
   }
   if (!ok && tid == 0) {
     // copies issued past the failed wait must land before the CTA leaves
-    for (int kk = k; kk < issued; ++kk) mbar_wait_drain(&full[kk & 1], uint32_t(kk >> 1) & 1u, &g_err_attn, wlim);
+    for (int kk = k; kk < issued; ++kk)
+      mbar_wait_drain(&full[kk % STAGES], uint32_t(kk / STAGES) & 1u, &g_err_attn, wlim);
   }
 }
 

@@ -305,4 +305,85 @@ hymba_status fuse_decode(const FuseDecodeArgs &a, cudaStream_t s) {
   return HYMBA_OK;
 }
 
+
+// ---------------------------------------------------------------------------
+// RMS norm with a learnable weight (the Hymba block's pre-norms):
+//   y[r, :] = x[r, :] / sqrt(mean(x[r, :]^2) + eps) * w
+// One warp per row; the row stays in registers as packed 16-byte vectors between the
+// reduction and the scaling, so it is read once.
+// ---------------------------------------------------------------------------
+template <typename T, int NV>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const T *__restrict__ x, const float *__restrict__ w,
+                                                      T *__restrict__ y, long long M, int d, float eps) {
+  constexpr int V = 16 / sizeof(T);
+  const long long row = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  const int nvec = d / V;
+  const T *xr = x + row * d;
+  uint4 raw[NV];
+  float ss = 0.f;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int v = lane + 32 * j;
+    if (v < nvec) {
+      raw[j] = __ldg(reinterpret_cast<const uint4 *>(xr + v * V));
+      float f[V];
+      unpack16<T>(raw[j], f);
+#pragma unroll
+      for (int i = 0; i < V; ++i) ss = fmaf(f[i], f[i], ss);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+  const float inv = rsqrtf(ss / d + eps);
+  T *yr = y + row * d;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int v = lane + 32 * j;
+    if (v < nvec) {
+      float f[V];
+      unpack16<T>(raw[j], f);
+#pragma unroll
+      for (int i = 0; i < V; i += 4) {
+        const float4 w4 = __ldg(reinterpret_cast<const float4 *>(w + v * V + i));
+        f[i] *= inv * w4.x;
+        f[i + 1] *= inv * w4.y;
+        f[i + 2] *= inv * w4.z;
+        f[i + 3] *= inv * w4.w;
+      }
+      if constexpr (sizeof(T) == 2) {
+        st_global_v4(yr + v * V, pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                     pack_bf16x2(f[6], f[7]));
+      } else {
+        st_global_v4(yr + v * V, __float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                     __float_as_uint(f[3]));
+      }
+    }
+  }
+}
+
+hymba_status rms_norm_rows(const void *x, const float *w, void *y, long long M, int d, float eps, hymba_dtype dt,
+                           cudaStream_t s) {
+  const int V = dt == HYMBA_BF16 ? 8 : 4;
+  if (d % V || d / V > 32 * 8) {
+    set_error("rms norm rows of %d elements: need a multiple of %d, at most %d", d, V, 32 * 8 * V);
+    return HYMBA_ERR_UNSUPPORTED;
+  }
+  if (M == 0) return HYMBA_OK;
+  const unsigned blocks = (unsigned)((M * 32 + 255) / 256);
+  if (dt == HYMBA_BF16)
+    rmsnorm_kernel<__nv_bfloat16, 8><<<blocks, 256, 0, s>>>((const __nv_bfloat16 *)x, w, (__nv_bfloat16 *)y, M,
+                                                              d, eps);
+  else
+    rmsnorm_kernel<float, 8><<<blocks, 256, 0, s>>>((const float *)x, w, (float *)y, M, d, eps);
+  note_launch(1);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error("rms norm launch failed: %s", cudaGetErrorString(e));
+    return HYMBA_ERR_CUDA;
+  }
+  return HYMBA_OK;
+}
+
 }  // namespace hymba

@@ -10,10 +10,12 @@
 //              accumulators in tensor memory, then tcgen05.commit frees the stage.
 //   warps 2-17: epilogue, one thread per accumulator row (four warps per TMEM
 //              lane quarter, every fourth 16-column chunk): tcgen05.ld, bias /
-//              softplus, fp32 -> bf16, routed stores (one GEMM writes Q, K, V,
-//              x_ssm and z to their own buffers).  The second accumulator lets
-//              the epilogue of tile i overlap the MMAs of tile i+1.
+//              softplus, per-segment SiLU and rotary embedding, fp32 -> bf16, routed
+//              stores (one GEMM writes Q, K, V, x_ssm and the gate SiLU(z) to their own
+//              buffers).  The second accumulator lets the epilogue of tile i overlap
+//              the MMAs of tile i+1.
 // Tiles are visited N-fastest so the CTAs in flight share A rows in L2.
+// Decode-sized products (<= 256 rows) use the weight-streaming kernel further down.
 // fp32 path: a plain CUDA-core tiled kernel with the same epilogue.
 #include <algorithm>
 
@@ -88,18 +90,44 @@ __device__ __forceinline__ void rope_rotate(const Epilogue &e, const EpiSeg &g, 
   }
 }
 
-// The segment's own activation (not on split-K partial sums).
+// The segment's own activation.
 __device__ __forceinline__ float seg_act(const EpiSeg &g, float v) { return g.act == 2 ? silu_f(v) : v; }
 
+// Residual of column `local` of segment g at product row m.
+__device__ __forceinline__ float resid_at(const EpiSeg &g, long long m, int local) {
+  const long long o = m * g.ld_resid + local;
+  if (g.f32) return __ldg(reinterpret_cast<const float *>(g.resid) + o);
+  return bf16_lo((uint32_t)__ldg(reinterpret_cast<const unsigned short *>(g.resid) + o));
+}
+// Residual of 8 consecutive columns (16-byte aligned, bf16 or fp32).
+__device__ __forceinline__ void resid8(const EpiSeg &g, long long m, int local, float (&r)[8]) {
+  const long long o = m * g.ld_resid + local;
+  if (g.f32) {
+    const float4 *p = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(g.resid) + o);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    r[0] = a.x; r[1] = a.y; r[2] = a.z; r[3] = a.w; r[4] = b.x; r[5] = b.y; r[6] = b.z; r[7] = b.w;
+  } else {
+    const uint4 w = __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const __nv_bfloat16 *>(g.resid) + o));
+    const uint32_t q[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      r[2 * i] = bf16_lo(q[i]);
+      r[2 * i + 1] = bf16_hi(q[i]);
+    }
+  }
+}
+
 // m: the product row; mk: its remapped row (used by segments with rmap).
+template <int EPI>
 __device__ __forceinline__ void epi_store_scalar(const Epilogue &e, long long m, long long mk, int n,
                                                  float v) {
   const EpiSeg &g = e.seg[find_seg(e, n)];
   const long long off = seg_offset(g, g.rmap ? mk : m, n - g.col0);
-  if (!e.atomic) v = seg_act(g, v);
-  if (e.atomic) {
-    atomicAdd(reinterpret_cast<float *>(g.ptr) + off, v);
-  } else if (g.f32) {
+  v = seg_act(g, v);
+  if constexpr ((EPI & kEpiResid) != 0) {
+    if (g.resid) v += resid_at(g, m, n - g.col0);
+  }
+  if (g.f32) {
     reinterpret_cast<float *>(g.ptr)[off] = v;
   } else {
     reinterpret_cast<__nv_bfloat16 *>(g.ptr)[off] = __float2bfloat16_rn(v);
@@ -107,6 +135,11 @@ __device__ __forceinline__ void epi_store_scalar(const Epilogue &e, long long m,
 }
 
 // Stores 8 consecutive columns n..n+7 of row m (values already activated).
+// EPI (kEpi* flags): the features this instantiation carries; the plain one (one segment,
+// no routing) keeps fewer registers live.  The 8-column path takes what the 16-column
+// fast path cannot (segment edges, unaligned destinations); it does no gated SiLU (the
+// host keeps such segments on whole 16-column chunks).
+template <int EPI>
 __device__ __forceinline__ void epi_store8(const Epilogue &e, long long m, long long mk, int rp, int n,
                                            int N, const float (&v_raw)[8]) {
   if (n >= N) return;
@@ -114,14 +147,24 @@ __device__ __forceinline__ void epi_store8(const Epilogue &e, long long m, long 
   float v_in[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) v_in[i] = v_raw[i];
-  if (g.rope && !e.atomic && n + 8 <= g.col1) rope_rotate<4>(e, g, n, rp, v_in);
+  if constexpr ((EPI & kEpiRoute) != 0) {
+    if (g.rope && n + 8 <= g.col1) rope_rotate<4>(e, g, n, rp, v_in);
+  }
   int local = n - g.col0;
-  bool vec = !e.atomic && g.vec_ok && (n + 8 <= N) && (n + 8 <= g.col1) && (local % 8 == 0) &&
+  bool vec = g.vec_ok && (n + 8 <= N) && (n + 8 <= g.col1) && (local % 8 == 0) &&
              ((local % g.inner) + 8 <= g.inner);
   if (vec) {
     float v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = seg_act(g, v_in[i]);
+    if constexpr ((EPI & kEpiResid) != 0) {
+      if (g.resid) {
+        float rr[8];
+        resid8(g, m, local, rr);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] += rr[i];
+      }
+    }
     const long long off = seg_offset(g, g.rmap ? mk : m, local);
     if (g.f32) {
       float *p = reinterpret_cast<float *>(g.ptr) + off;
@@ -138,7 +181,7 @@ __device__ __forceinline__ void epi_store8(const Epilogue &e, long long m, long 
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i)
-    if (n + i < N) epi_store_scalar(e, m, mk, n + i, v_in[i]);
+    if (n + i < N) epi_store_scalar<EPI>(e, m, mk, n + i, v_in[i]);
 }
 
 // Bias of columns n0..n0+15 (zero past N).
@@ -162,34 +205,65 @@ __device__ __forceinline__ void epi_bias16(const Epilogue &e, int n0, int N, flo
 // 16 consecutive product columns n0..n0+15 of row m from raw fp32 accumulator bits,
 // plus the bias (when the epilogue has one).  One segment lookup per chunk on the
 // common path.
+template <int EPI>
 __device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, long long mk, int rp, int n0,
                                             int N, const uint32_t (&r)[16], const float (&bias)[16]) {
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
   const bool full = n0 + 16 <= N;
-  if (!e.atomic) {
-    if (e.bias) {
+  if (e.bias) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] += bias[i];
-    }
-    if (e.act == 1) {
+    for (int i = 0; i < 16; ++i) v[i] += bias[i];
+  }
+  if (e.act == 1) {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) v[i] = softplus_f(v[i]);
-    }
+    for (int i = 0; i < 16; ++i) v[i] = softplus_f(v[i]);
   }
   // common case: the 16 columns lie in one segment and one group, 16-byte aligned rows
   const int sidx = find_seg(e, n0);
   const EpiSeg &g = e.seg[sidx];
   const int local = n0 - g.col0;
-  if (full && !e.atomic && g.vec_ok && n0 + 16 <= g.col1 &&
+  if (full && g.vec_ok && n0 + 16 <= g.col1 &&
       (g.inner >= g.col1 - g.col0 || ((g.inner & 15) == 0 && (local & 15) == 0))) {
+    if constexpr ((EPI & kEpiGlu) != 0) {
+      if (g.act == 3) {
+        // gated SiLU: product columns (2i, 2i+1) -> output column local/2 + i
+        float o[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = silu_f(v[2 * i]) * v[2 * i + 1];
+        const long long off = m * g.ld_row + (local >> 1);
+        if (g.f32) {
+          float *p = reinterpret_cast<float *>(g.ptr) + off;
+          st_global_v4(p, __float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]), __float_as_uint(o[3]));
+          st_global_v4(p + 4, __float_as_uint(o[4]), __float_as_uint(o[5]), __float_as_uint(o[6]),
+                       __float_as_uint(o[7]));
+        } else {
+          st_global_v4(reinterpret_cast<__nv_bfloat16 *>(g.ptr) + off, pack_bf16x2(o[0], o[1]),
+                       pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]), pack_bf16x2(o[6], o[7]));
+        }
+        return;
+      }
+    }
     if (g.act) {
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] = seg_act(g, v[i]);
     }
-    if (g.rope) rope_rotate<8>(e, g, n0, rp, v);
-    const long long off = seg_offset(g, g.rmap ? mk : m, local);
+    if constexpr ((EPI & kEpiRoute) != 0) {
+      if (g.rope) rope_rotate<8>(e, g, n0, rp, v);
+    }
+    if constexpr ((EPI & kEpiResid) != 0) {
+      if (g.resid) {
+        float rr[8];
+        resid8(g, m, local, rr);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] += rr[i];
+        resid8(g, m, local + 8, rr);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[8 + i] += rr[i];
+      }
+    }
+    const long long off = seg_offset(g, ((EPI & kEpiRoute) && g.rmap) ? mk : m, local);
     if (g.f32) {
       float *p = reinterpret_cast<float *>(g.ptr) + off;
       if (g.vec32) {
@@ -226,8 +300,8 @@ __device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, long
     a[i] = v[i];
     b[i] = v[8 + i];
   }
-  epi_store8(e, m, mk, rp, n0, N, a);
-  epi_store8(e, m, mk, rp, n0 + 8, N, b);
+  epi_store8<EPI>(e, m, mk, rp, n0, N, a);
+  epi_store8<EPI>(e, m, mk, rp, n0 + 8, N, b);
 }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -260,10 +334,10 @@ struct TcCfg {
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0, N <= 256");
 };
 
-template <int BN, int ELEM>
+template <int BN, int ELEM, int EPI>
 __global__ void __launch_bounds__(576, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   int M, int N, int K, int ksplit, Epilogue epi, long long wlim, int stall) {
+                   int M, int N, int K, Epilogue epi, long long wlim, int stall) {
   using C = TcCfg<BN, ELEM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -285,8 +359,7 @@ __global__ void __launch_bounds__(576, 1)
   const int m_tiles = (M + C::BM - 1) / C::BM;
   const int n_tiles = (N + BN - 1) / BN;
   const int kblocks = (K + C::BK - 1) / C::BK;
-  const int kb_per = (kblocks + ksplit - 1) / ksplit;
-  const long long units = (long long)m_tiles * n_tiles * ksplit;
+  const long long units = (long long)m_tiles * n_tiles;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -310,11 +383,6 @@ __global__ void __launch_bounds__(576, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  if (epi.zero && warp >= 2) {
-    for (long long i = (long long)blockIdx.x * 512 + (threadIdx.x - 64); i < epi.zero_n;
-         i += (long long)gridDim.x * 512)
-      epi.zero[i] = 0.f;
-  }
 
   if (warp == 0) {
     if (lane == 0) {
@@ -324,11 +392,8 @@ __global__ void __launch_bounds__(576, 1)
       uint32_t issued[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       bool ok = true;
       for (long long u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const int ks = int(u % ksplit);
-        const long long tile = u / ksplit;
-        const int mt = int(tile / n_tiles), nt = int(tile % n_tiles);
-        const int kb0 = ks * kb_per, kb1 = min(kblocks, kb0 + kb_per);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        const int mt = int(u / n_tiles), nt = int(u % n_tiles);
+        for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, &g_err_gemm, wlim)) {
             ok = false;
             break;
@@ -360,16 +425,13 @@ __global__ void __launch_bounds__(576, 1)
       // instead of issuing its first MMA; it then takes the abort path below.
       bool ok = !stall || mbar_wait(never, 0, &g_err_gemm, wlim);
       for (long long u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const int ks = int(u % ksplit);
-        const int kb0 = ks * kb_per, kb1 = min(kblocks, kb0 + kb_per);
-        if (kb0 >= kb1) continue;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, &g_err_gemm, wlim)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + uint32_t(acc * BN);
-        for (int kb = kb0; kb < kb1; ++kb) {
+        for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&full[stage], phase, &g_err_gemm, wlim)) {
             ok = false;
             break;
@@ -382,9 +444,9 @@ __global__ void __launch_bounds__(576, 1)
             const uint64_t ad = make_sdesc(a_addr + k * 32, 16, 1024);
             const uint64_t bd = make_sdesc(b_addr + k * 32, 16, 1024);
             if (ELEM == 2)
-              mma_bf16_ss(d_tmem, ad, bd, C::IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+              mma_bf16_ss(d_tmem, ad, bd, C::IDESC, (kb > 0 || k > 0) ? 1u : 0u);
             else
-              mma_tf32_ss(d_tmem, ad, bd, C::IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+              mma_tf32_ss(d_tmem, ad, bd, C::IDESC, (kb > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit(&empty[stage]);
           if (++stage == C::STAGES) {
@@ -415,17 +477,13 @@ __global__ void __launch_bounds__(576, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (long long u = blockIdx.x; u < units; u += gridDim.x) {
-      const int ks = int(u % ksplit);
-      const long long tile = u / ksplit;
-      const int kb0 = ks * kb_per, kb1 = min(kblocks, kb0 + kb_per);
-      if (kb0 >= kb1) continue;
-      const int mt = int(tile / n_tiles), nt = int(tile % n_tiles);
+      const int mt = int(u / n_tiles), nt = int(u % n_tiles);
       constexpr int NCH = (BN + 63) / 64;
       if (!mbar_wait(&tfull[acc], acc_phase, &g_err_gemm, wlim)) break;
       tc_fence_after();
       const long long m = (long long)mt * C::BM + row;
-      const long long mk = remap_row(s_epi, m);
-      const int rp = rope_pos(s_epi, m);
+      const long long mk = (EPI & kEpiRoute) ? remap_row(s_epi, m) : m;
+      const int rp = (EPI & kEpiRoute) ? rope_pos(s_epi, m) : 0;
       const uint32_t t_row = tmem_base + (uint32_t(quarter * 32) << 16) + uint32_t(acc * BN);
       // this warp's chunks in rounds of at most two loads; the accumulator is handed back
       // to the MMA warp after the last round's loads, before its activation math and stores
@@ -450,7 +508,7 @@ __global__ void __launch_bounds__(576, 1)
           if (k0 + k < NCH && c < BN && n0 < N && m < M) {
             float bias[16];
             if (s_epi.bias) epi_bias16(s_epi, n0, N, bias);
-            epi_store16(s_epi, m, mk, rp, n0, N, r[k], bias);
+            epi_store16<EPI>(s_epi, m, mk, rp, n0, N, r[k], bias);
           }
         }
       }
@@ -541,10 +599,6 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 1) {
     tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
-  }
-  if (epi.zero) {  // accumulators of a later kernel of the same step start at zero
-    const long long nct = (long long)gridDim.x * gridDim.y, bid = (long long)blockIdx.y * gridDim.x + blockIdx.x;
-    for (long long i = bid * 128 + tid; i < epi.zero_n; i += nct * 128) epi.zero[i] = 0.f;
   }
   tc_fence_before();
   __syncthreads();
@@ -640,7 +694,7 @@ __global__ void __launch_bounds__(128, 1)
         for (int i = 0; i < 16; ++i) bits[i] = __float_as_uint(acc[i]);
         float bias[16];
         if (s_epi.bias) epi_bias16(s_epi, n0, Nout, bias);
-        epi_store16(s_epi, m, mk, rp, n0, Nout, bits, bias);
+        epi_store16<kEpiRoute | kEpiResid | kEpiGlu>(s_epi, m, mk, rp, n0, Nout, bits, bias);
       }
     }
   }
@@ -711,8 +765,8 @@ static hymba_status launch_ws_cl(const GemmArgs &g, int cl, cudaStream_t s) {
 
 // Decode-sized products (at most 256 activation rows, bf16, no split-K or atomic epilogue).
 hymba_status gemm_ws(const GemmArgs &g, cudaStream_t s) {
-  if (g.elem != 2 || g.M < 1 || g.M > 256 || g.ksplit != 1 || g.epi.atomic || g.stall) {
-    set_error("gemm_ws: unsupported product (bf16, <= 256 rows, no split-K)");
+  if (g.elem != 2 || g.M < 1 || g.M > 256 || g.stall) {
+    set_error("gemm_ws: unsupported product (bf16, at most 256 rows)");
     return HYMBA_ERR_UNSUPPORTED;
   }
   // cluster size: enough CTAs to put most SMs on the weight stream, at most one K block each
@@ -726,14 +780,26 @@ hymba_status gemm_ws(const GemmArgs &g, cudaStream_t s) {
   return launch_ws_cl<256>(g, cl, s);
 }
 
-template <int BN, int ELEM>
+// The epilogue features a product needs (kEpi* flags).
+static int epi_flags(const Epilogue &e) {
+  int f = 0;
+  if (e.nseg > 1 || e.rmap_rows > 0 || e.rope_tab) f |= kEpiRoute;
+  for (int i = 0; i < e.nseg; ++i) {
+    if (e.seg[i].rmap || e.seg[i].rope) f |= kEpiRoute;
+    if (e.seg[i].resid) f |= kEpiResid;
+    if (e.seg[i].act == 3) f |= kEpiGlu;
+  }
+  return f;
+}
+
+template <int BN, int ELEM, int EPI>
 static hymba_status launch_tc(const GemmArgs &g, cudaStream_t s) {
   using C = TcCfg<BN, ELEM>;
   static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set.done(dev)) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<BN, ELEM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(gemm_tc_kernel<BN, ELEM, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              C::SMEM) != cudaSuccess) {
       set_error("cudaFuncSetAttribute(gemm smem %d) failed", C::SMEM);
       return HYMBA_ERR_CUDA;
@@ -748,9 +814,9 @@ static hymba_status launch_tc(const GemmArgs &g, cudaStream_t s) {
   uint32_t bb[2] = {(uint32_t)C::BK, (uint32_t)BN};
   if (!make_tmap(&ta, g.A, dt, 2, da, sa, ba)) return HYMBA_ERR_CUDA;
   if (!make_tmap(&tb, g.B, dt, 2, db, sb, bb)) return HYMBA_ERR_CUDA;
-  const long long tiles = (long long)((g.M + 127) / 128) * ((g.N + BN - 1) / BN) * g.ksplit;
+  const long long tiles = (long long)((g.M + 127) / 128) * ((g.N + BN - 1) / BN);
   const int grid = (int)std::min<long long>(tiles, num_sms());
-  gemm_tc_kernel<BN, ELEM><<<grid, 576, C::SMEM, s>>>(ta, tb, g.M, g.N, g.K, g.ksplit, g.epi,
+  gemm_tc_kernel<BN, ELEM, EPI><<<grid, 576, C::SMEM, s>>>(ta, tb, g.M, g.N, g.K, g.epi,
                                                      wait_limit_cycles(), g.stall);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
@@ -766,16 +832,33 @@ hymba_status gemm_tc(const GemmArgs &g, cudaStream_t s) {
   // (decode) so that more CTAs stream the weights.
   const bool small_m = g.M <= 128;
   if (g.elem == 2) {
-    if (g.N <= 144) return launch_tc<144, 2>(g, s);
-    if (small_m) return launch_tc<64, 2>(g, s);
-    if (g.N % 256 == 0 || g.N > 4096) return launch_tc<256, 2>(g, s);
-    if (g.N % 160 == 0) return launch_tc<160, 2>(g, s);
-    return launch_tc<128, 2>(g, s);
+    const int f = epi_flags(g.epi);
+    if (f == kEpiRoute) {  // the input projection
+      if (small_m) return launch_tc<64, 2, kEpiRoute>(g, s);
+      return launch_tc<256, 2, kEpiRoute>(g, s);
+    }
+    if (f == kEpiResid) {  // a projection back into the residual stream (the 160-wide tile spills)
+      if (small_m) return launch_tc<64, 2, kEpiResid>(g, s);
+      return launch_tc<128, 2, kEpiResid>(g, s);
+    }
+    if (f == kEpiGlu) {  // the MLP's gated up projection
+      if (small_m) return launch_tc<64, 2, kEpiGlu>(g, s);
+      return launch_tc<256, 2, kEpiGlu>(g, s);
+    }
+    if (f != 0) {
+      set_error("gemm_tc: unsupported combination of epilogue features %d", f);
+      return HYMBA_ERR_UNSUPPORTED;
+    }
+    if (g.N <= 144) return launch_tc<144, 2, 0>(g, s);
+    if (small_m) return launch_tc<64, 2, 0>(g, s);
+    if (g.N % 256 == 0 || g.N > 4096) return launch_tc<256, 2, 0>(g, s);
+    if (g.N % 160 == 0) return launch_tc<160, 2, 0>(g, s);
+    return launch_tc<128, 2, 0>(g, s);
   }
   if (g.elem == 4) {
-    if (small_m) return launch_tc<64, 4>(g, s);
-    if (g.N % 160 == 0) return launch_tc<160, 4>(g, s);
-    return launch_tc<128, 4>(g, s);
+    if (small_m) return launch_tc<64, 4, 0>(g, s);
+    if (g.N % 160 == 0) return launch_tc<160, 4, 0>(g, s);
+    return launch_tc<128, 4, 0>(g, s);
   }
   set_error("gemm_tc: unsupported element size %d", g.elem);
   return HYMBA_ERR_UNSUPPORTED;
@@ -786,22 +869,16 @@ hymba_status gemm_tc(const GemmArgs &g, cudaStream_t s) {
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256)
     gemm_simt_f32_kernel(const float *__restrict__ A, long long lda, const float *__restrict__ B,
-                         long long ldb, int M, int N, int K, int kb_per, Epilogue epi) {
+                         long long ldb, int M, int N, int K, Epilogue epi) {
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
   const int tid = threadIdx.x;
-  if (epi.zero) {
-    const long long nb = (long long)gridDim.x * gridDim.y * gridDim.z;
-    const long long bid = blockIdx.x + (long long)gridDim.x * (blockIdx.y + (long long)gridDim.y * blockIdx.z);
-    for (long long i = bid * 256 + tid; i < epi.zero_n; i += nb * 256) epi.zero[i] = 0.f;
-  }
   const int tx = tid & 15, ty = tid >> 4;
   const long long m0 = (long long)blockIdx.y * 64;
   const int n0 = blockIdx.x * 64;
-  const int kbeg = blockIdx.z * kb_per * 16;
-  const int kend = min(K, kbeg + kb_per * 16);
+  const int kend = K;
   float acc[4][4] = {};
-  for (int k0 = kbeg; k0 < kend; k0 += 16) {
+  for (int k0 = 0; k0 < kend; k0 += 16) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int idx = tid + i * 256;
@@ -835,32 +912,43 @@ __global__ void __launch_bounds__(256)
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx * 4 + j;
-      v[j] = (n < N && !epi.atomic) ? epi_act(epi, n, acc[i][j]) : acc[i][j];
+      v[j] = n < N ? epi_act(epi, n, acc[i][j]) : acc[i][j];
     }
     // rotary pairs (2i, 2i+1) are both in this thread's four columns
 #pragma unroll
     for (int j = 0; j < 4; j += 2) {
       const int n = n0 + tx * 4 + j;
-      if (n + 1 < N && !epi.atomic) {
+      if (n + 1 < N) {
         const EpiSeg &g = epi.seg[find_seg(epi, n)];
         if (g.rope && n + 1 < g.col1) rope_rotate<1>(epi, g, n, rope_pos(epi, m), v + j);
+      }
+    }
+    // gated SiLU pairs (both columns in this thread) write one output column each
+    bool done_pair[2] = {false, false};
+#pragma unroll
+    for (int j = 0; j < 4; j += 2) {
+      const int n = n0 + tx * 4 + j;
+      if (n + 1 < N) {
+        const EpiSeg &g = epi.seg[find_seg(epi, n)];
+        if (g.act == 3 && n + 1 < g.col1) {
+          reinterpret_cast<float *>(g.ptr)[m * g.ld_row + ((n - g.col0) >> 1)] = silu_f(v[j]) * v[j + 1];
+          done_pair[j >> 1] = true;
+        }
       }
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = n0 + tx * 4 + j;
-      if (n < N) epi_store_scalar(epi, m, remap_row(epi, m), n, v[j]);
+      if (n < N && !done_pair[j >> 1]) epi_store_scalar<kEpiRoute | kEpiResid>(epi, m, remap_row(epi, m), n, v[j]);
     }
   }
 }
 
 hymba_status gemm_simt_f32(const GemmArgs &g, cudaStream_t s) {
-  const int kblocks = (g.K + 15) / 16;
-  const int kb_per = (kblocks + g.ksplit - 1) / g.ksplit;
-  dim3 grid((g.N + 63) / 64, (g.M + 63) / 64, g.ksplit);
+  dim3 grid((g.N + 63) / 64, (g.M + 63) / 64);
   gemm_simt_f32_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float *>(g.A), g.lda,
                                             reinterpret_cast<const float *>(g.B), g.ldb, g.M, g.N,
-                                            g.K, kb_per, g.epi);
+                                            g.K, g.epi);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

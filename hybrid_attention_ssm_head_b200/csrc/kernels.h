@@ -39,10 +39,18 @@ struct EpiSeg {
   int f32;
   int vec_ok;  // 16-byte aligned rows/groups: 8-column vector stores allowed
   int vec32;   // 32-byte aligned rows/groups: whole-sector (256-bit) stores allowed
-  int act;     // activation of this segment's columns: 0 none, 2 SiLU (after the GEMM's own)
+  int act;     // activation of this segment's columns (after the GEMM's own): 0 none, 2 SiLU,
+               // 3 gated SiLU: product columns (2i, 2i+1) = (gate_i, up_i) give output column
+               // i = SiLU(gate_i) * up_i (the segment's destination has half its columns)
   int rmap;    // 1: rows go through the epilogue's row remap
   int rope;    // 1: rotary position embedding of this segment's heads (pairs of columns)
+  const void *resid;  // optional residual added to the result: same dtype as the destination,
+  long long ld_resid; // [rows, col1 - col0] with row stride ld_resid (one group only)
 };
+// Epilogue features a GEMM instantiation carries (bit flags).
+constexpr int kEpiRoute = 1;  // several segments, row remap, rotary embedding
+constexpr int kEpiResid = 2;  // residual add
+constexpr int kEpiGlu = 4;    // gated SiLU of column pairs
 
 struct Epilogue {
   EpiSeg seg[5];
@@ -60,9 +68,6 @@ struct Epilogue {
   int rope_rows, rope_off, rope_hd;
   const float *bias;  // per product column (nullable)
   int act;            // 0 = identity, 1 = softplus
-  int atomic;         // 1 = fp32 atomicAdd into the destination (split-K)
-  float *zero;        // optional: zeroed by the GEMM (after the previous kernels), for
-  long long zero_n;   // split-K destinations of later kernels of the same step
 };
 
 // out[m, n] = epi( sum_k A[m, k] * B[n, k] )  (A: [M, K], B: [N, K], row-major)
@@ -73,7 +78,6 @@ struct GemmArgs {
   long long ldb;
   int M, N, K;
   int elem;    // 2: bf16 operands; 4: fp32 operands
-  int ksplit;  // >= 1; > 1 requires epi.atomic
   Epilogue epi;
   int stall;   // tensor-core path: the MMA warp waits for an arrival that never comes
 };
@@ -146,6 +150,10 @@ struct FuseDecodeArgs {
 };
 hymba_status fuse_decode(const FuseDecodeArgs &a, cudaStream_t s);
 
+// y = x / rms(x) * w per row of d elements (the block's pre-norms).
+hymba_status rms_norm_rows(const void *x, const float *w, void *y, long long M, int d, float eps, hymba_dtype dt,
+                           cudaStream_t s);
+
 // ---- attention -----------------------------------------------------------
 // Queries are the positions q_off .. q_off + Lq - 1 of sequences of L = q_off + Lq rows,
 // stored from row 0 of q and o; keys are all L positions.
@@ -197,7 +205,7 @@ size_t decode_attn_workspace_floats(int B, int H, int dv, long long pos, int n_m
 hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s);
 
 
-// ---- decode SSM branch: conv + x_proj, then dt_proj + softplus + scan step + gate ----
+// ---- decode SSM branch: conv + SiLU; x_proj (a GEMM); dt_proj + softplus + scan step + gate ----
 struct DecodeSsmArgs {
   const void *x;       // [B, E] x_ssm of the new token, row stride ld_x
   long long ld_x;
@@ -205,8 +213,7 @@ struct DecodeSsmArgs {
   long long ld_z;
   void *conv_state;    // [B, K-1, E] in/out
   const float *conv_w, *conv_b;  // [E, K], [E]
-  const void *w_x;     // [R + 2N, E]
-  float *xdbl;         // [B, R + 2N] fp32, zero on entry (the caller zeroes it)
+  const float *xdbl;   // [B, R + 2N] fp32: delta_r, B, C of the new token
   void *u;             // [B, E] conv + SiLU output
   const float *w_dt, *b_dt;      // [E, R], [E]
   const float *a_log, *d_skip;   // [E, N], [E]
@@ -214,10 +221,11 @@ struct DecodeSsmArgs {
   void *y;             // [B, E] gated output
   int B, E, K, R, N;
 };
-hymba_status decode_ssm(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s);
+// u = SiLU(conv(window, x) + b); the conv window advanced in place.
+hymba_status decode_conv(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s);
+// delta = softplus(delta_r W_dt^T + b_dt), one recurrence step, y = (C.h + D u) * gate.
+hymba_status decode_scan(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s);
 
-// path 0: the tensor-core (bf16) prefill kernel's tile enumeration, tile classes and
-// column keep-masks; path 1: the CUDA-core (fp32) kernel's per-pair predicate.
 hymba_status mask_bitmap(int L, int n_meta, int window, int is_global, int path, uint32_t *bits,
                          uint8_t *tile_class, cudaStream_t s);
 // The decode kernels' slot predicate for the query at `pos`, one bit per slot.

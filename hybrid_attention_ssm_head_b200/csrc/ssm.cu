@@ -16,9 +16,8 @@
 // (the chunk's decay is exp(A * sum delta)); pass 2 chains the chunk start states;
 // pass 3 rescans each chunk from its true start and writes y.
 //
-// Decode: two kernels for the whole branch of one new token: conv + SiLU + a share
-// of x_proj (atomic partial sums), then dt_proj + softplus + one recurrence step +
-// gate from the stored state.
+// Decode: conv + SiLU (one kernel), x_proj (the decode GEMM), then dt_proj + softplus +
+// one recurrence step + gate from the stored state (one kernel).
 #include <algorithm>
 
 #include "common.cuh"
@@ -227,135 +226,55 @@ hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
-// decode SSM branch in two kernels
+// decode SSM branch: conv + SiLU, then (after the x_proj GEMM) dt_proj + softplus +
+// one recurrence step + gate
 // ---------------------------------------------------------------------------
-// (1) CTA = 16 sequences x CH channels: u = SiLU(conv(window, x) + b) for its
-//     channels (window advanced in conv_state, u stored), then its share of
-//     x_proj, xdbl[b, j] += sum over its channels of u[b, c] W_x[j, c], added
-//     atomically (E / CH partial sums per output).  The W_x slice arrives by cp.async
-//     while the convolution runs; every global load of the convolution is issued
-//     before the first store.
-constexpr int kDecRows = 16;
-template <typename T, int CH>
-__global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
-  constexpr int ROWB = CH * (int)sizeof(T) + 16;  // padded row of the W_x slice (conflict-free 16-byte reads)
-  constexpr int PIECES = CH * (int)sizeof(T) / 16;
-  constexpr int RPT = kDecRows * CH / 256;         // conv rows per thread
-  extern __shared__ __align__(16) uint8_t dsm_x[];
-  float *us = reinterpret_cast<float *>(dsm_x);    // [CH][kDecRows] u, channel-major (broadcast reads)
-  uint8_t *wxs = dsm_x + CH * kDecRows * 4;        // [NJ][ROWB] W_x slice
-  const int NJ = a.R + 2 * a.N;
-  const int cbase = blockIdx.x * CH;
-  const int b0 = blockIdx.y * kDecRows;
-  const int tid = threadIdx.x;
-  const T *wx = reinterpret_cast<const T *>(a.w_x);
-  for (int idx = tid; idx < NJ * PIECES; idx += 256) {
-    const int j = idx / PIECES, pc = idx % PIECES;
-    cp_async16(wxs + j * ROWB + pc * 16, wx + (long long)j * a.E + cbase + pc * (16 / (int)sizeof(T)));
+// (1) One thread per (sequence, 8 channels): u = SiLU(conv(window, x) + b), the window
+//     advanced by one row in conv_state.  16-byte loads and stores.
+template <typename T>
+__global__ void __launch_bounds__(256) dec_conv_kernel(DecodeSsmArgs a) {
+  constexpr int V = 16 / sizeof(T);
+  const int nv = a.E / V;
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)a.B * nv) return;
+  const int b = (int)(idx / nv), c0 = (int)(idx % nv) * V;
+  const int K = a.K;
+  T *cs = reinterpret_cast<T *>(a.conv_state) + (long long)b * (K - 1) * a.E + c0;
+  uint4 raw[4];  // window rows (oldest first), then the new row x
+#pragma unroll
+  for (int t = 0; t < 3; ++t)
+    raw[t] = t < K - 1 ? *reinterpret_cast<const uint4 *>(cs + (long long)t * a.E) : make_uint4(0, 0, 0, 0);
+  raw[3] = __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const T *>(a.x) + (long long)b * a.ld_x + c0));
+  float xv[4][V];
+#pragma unroll
+  for (int t = 0; t < 4; ++t) unpack16<T>(raw[t], xv[t]);
+  float o[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const float *w = a.conv_w + (long long)(c0 + i) * K;
+    float acc = __ldg(a.conv_b + c0 + i);
+#pragma unroll
+    for (int t = 0; t < 3; ++t)
+      if (t < K - 1) acc = fmaf(__ldg(w + t), xv[t][i], acc);
+    acc = fmaf(__ldg(w + K - 1), xv[3][i], acc);
+    o[i] = silu_f(acc);
   }
-  cp_async_commit();
-  // conv + SiLU: thread -> channel tid % CH, rows tid / CH + k * (256 / CH).  Every load
-  // is issued unconditionally (rows past the batch read a valid row and are discarded)
-  // and kept raw until all of them are in flight, so their latencies overlap.
-  {
-    const int K = a.K;
-    T *cs = reinterpret_cast<T *>(a.conv_state);
-    const T *x = reinterpret_cast<const T *>(a.x);
-    T *u = reinterpret_cast<T *>(a.u);
-    const int ch = tid % CH, c = cbase + ch;
-    float w[3];  // taps of the window rows (oldest first); wlast multiplies the new row
+  store_vec<T>(reinterpret_cast<T *>(a.u) + (long long)b * a.E + c0, o);
+  // the window advances by one row: rows 1..K-2 move down, x becomes the newest
 #pragma unroll
-    for (int k = 0; k < 3; ++k) w[k] = k < K - 1 ? a.conv_w[c * K + k] : 0.f;
-    const float wlast = a.conv_w[c * K + K - 1];
-    const float bias = a.conv_b[c];
-    T raw[RPT][4];  // window rows oldest first; the new row x last
-#pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-      const int bb = min(b0 + tid / CH + k * (256 / CH), a.B - 1);
-      if (K > 1) {  // uniform: no window rows at all for a one-tap convolution
-#pragma unroll
-        for (int t = 0; t < 3; ++t) raw[k][t] = cs[((long long)bb * (K - 1) + min(t, K - 2)) * a.E + c];
-      }
-      raw[k][3] = x[(long long)bb * a.ld_x + c];
-    }
-#pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-      const int r = tid / CH + k * (256 / CH), b = b0 + r;
-      float win[3];
-#pragma unroll
-      for (int t = 0; t < 3; ++t) win[t] = 0.f;
-#pragma unroll
-      for (int t = 0; t < 3; ++t)
-        if (t < K - 1) win[t] = Store<T>::to_f(raw[k][t]);
-      float acc = bias;
-#pragma unroll
-      for (int t = 0; t < 3; ++t) acc = fmaf(w[t], win[t], acc);
-      acc = fmaf(wlast, Store<T>::to_f(raw[k][3]), acc);
-      float uv = 0.f;
-      if (b < a.B) {
-        uv = silu_f(acc);
-        u[(long long)b * a.E + c] = Store<T>::from_f(uv);
-        // the window advances by one row: rows 1..K-2 move down, x becomes the newest
-#pragma unroll
-        for (int t = 0; t < 3; ++t)
-          if (t < K - 1)
-            cs[((long long)b * (K - 1) + t) * a.E + c] = t + 1 < K - 1 ? raw[k][t + 1] : raw[k][3];
-      }
-      us[ch * kDecRows + r] = uv;
-    }
-  }
-  cp_async_wait<0>();
-  __syncthreads();
-  // x_proj share: thread -> output column j, all 16 rows, 16-byte reads of the W_x row
-  for (int j = tid; j < NJ; j += 256) {
-    float acc[kDecRows];
-#pragma unroll
-    for (int r = 0; r < kDecRows; ++r) acc[r] = 0.f;
-    const uint8_t *wrow = wxs + j * ROWB;
-#pragma unroll 2
-    for (int pc = 0; pc < PIECES; ++pc) {
-      const uint4 raw = *reinterpret_cast<const uint4 *>(wrow + pc * 16);
-      float wv[16 / sizeof(T)];
-      if constexpr (sizeof(T) == 2) {
-        const uint32_t q[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          wv[2 * i] = bf16_lo(q[i]);
-          wv[2 * i + 1] = bf16_hi(q[i]);
-        }
-      } else {
-        wv[0] = __uint_as_float(raw.x);
-        wv[1] = __uint_as_float(raw.y);
-        wv[2] = __uint_as_float(raw.z);
-        wv[3] = __uint_as_float(raw.w);
-      }
-#pragma unroll
-      for (int i = 0; i < (int)(16 / sizeof(T)); ++i) {
-        const float4 *u4 = reinterpret_cast<const float4 *>(us + (pc * (16 / (int)sizeof(T)) + i) * kDecRows);
-#pragma unroll
-        for (int q = 0; q < kDecRows / 4; ++q) {
-          const float4 v = u4[q];
-          acc[4 * q] = fmaf(v.x, wv[i], acc[4 * q]);
-          acc[4 * q + 1] = fmaf(v.y, wv[i], acc[4 * q + 1]);
-          acc[4 * q + 2] = fmaf(v.z, wv[i], acc[4 * q + 2]);
-          acc[4 * q + 3] = fmaf(v.w, wv[i], acc[4 * q + 3]);
-        }
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < kDecRows; ++r)
-      if (b0 + r < a.B) atomicAdd(&a.xdbl[(long long)(b0 + r) * NJ + j], acc[r]);
-  }
+  for (int t = 0; t < 3; ++t)
+    if (t < K - 1) *reinterpret_cast<uint4 *>(cs + (long long)t * a.E) = t + 1 < K - 1 ? raw[t + 1] : raw[3];
 }
 
-// (2) CTA = 8 sequences x 128 channels.  dt_low (rank R) times the W_dt slice on the
-//     tensor cores (mma.sync m16n8k8, tf32 in, fp32 accumulate; rows 8..15 of the
-//     16-row tile are zero), then thread per channel: delta = softplus(. + b_dt), one
-//     step of the recurrence from the stored state (h_t = exp(delta A) h + delta B u,
-//     y = C . h + D u, times the gate SiLU(z)), state written back in place.  W_dt (contiguous
-//     rows) and the xdbl rows arrive by cp.async; shared row strides are 4 mod 8 floats,
-//     so the tf32 fragment loads are free of bank conflicts.
-constexpr int kDecScanRows = 8;
+// (2) CTA = 16 sequences x 32 channels, 128 threads; thread (channel c, rows 4g..4g+3).
+//     The four rows' states are loaded first (all in flight while the rest runs).  Then
+//     dt_low [16 rows, R] times the W_dt slice on the tensor cores (mma.sync m16n8k8, tf32,
+//     fp32 accumulate; one 8-channel tile per warp), softplus, one step of the recurrence
+//     from the stored state (h_t = exp(delta A) h + delta B u, y = C . h + D u, times the
+//     gate SiLU(z)), and the state written back in place.  W_dt rows and the xdbl rows
+//     arrive by cp.async; shared row strides are 12 mod 32 floats, so the tf32 fragment
+//     loads are free of bank conflicts.
+constexpr int kScanRows = 16, kScanCh = 32;
 template <typename T>
 __device__ __forceinline__ float softplus_dec(float x) {
   if constexpr (sizeof(T) == 2) return softplus_f(x);
@@ -374,60 +293,65 @@ __device__ __forceinline__ void mma_tf32_16808(float (&d)[4], uint32_t a0, uint3
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
-// shared layout of the dt_proj stage, in floats
-struct DecDtLayout {
+// shared layout of the scan-step kernel, in floats
+struct DecScanLayout {
   int RP, WS, XS, NJ;  // rank padded to 8, W_dt row stride, xdbl row stride, xdbl width
-  __host__ __device__ DecDtLayout(int R, int N) {
+  __host__ __device__ DecScanLayout(int R, int N) {
     RP = (R + 7) / 8 * 8;
-    WS = RP + 4;
+    WS = RP + ((12 - RP % 32) % 32 + 32) % 32;
     NJ = R + 2 * N;
-    XS = (NJ + 7) / 8 * 8 + 4;
+    const int xp = (NJ + 7) / 8 * 8;
+    XS = xp + ((12 - xp % 32) % 32 + 32) % 32;
   }
   __host__ __device__ int wdt() const { return 0; }
-  __host__ __device__ int xs() const { return 128 * WS; }
-  __host__ __device__ int dts() const { return 128 * WS + 16 * XS; }
-  __host__ __device__ int floats() const { return 128 * WS + 16 * XS + kDecScanRows * 132; }
+  __host__ __device__ int xs() const { return kScanCh * WS; }
+  __host__ __device__ int dts() const { return kScanCh * WS + kScanRows * XS; }
+  __host__ __device__ int floats() const { return kScanCh * WS + kScanRows * XS + kScanRows * (kScanCh + 4); }
 };
 template <typename T>
-__global__ void __launch_bounds__(128, 3) dec_dt_scan_kernel(DecodeSsmArgs a) {
+__global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
   extern __shared__ __align__(16) float dsmem[];
   const int R = a.R;
-  const DecDtLayout lay(R, kStates);
+  const DecScanLayout lay(R, kStates);
   const int NJ = lay.NJ;
-  float *wdt = dsmem + lay.wdt();  // [128][WS] W_dt slice, columns R..RP-1 zero
+  float *wdt = dsmem + lay.wdt();  // [32][WS] W_dt slice, columns R..RP-1 zero
   float *xs = dsmem + lay.xs();    // [16][XS] xdbl rows (rows past the batch zero)
-  float *dts = dsmem + lay.dts();  // [kDecScanRows][132] dt_proj result
-  const int cbase = blockIdx.x * 128;
-  const int b0 = blockIdx.y * kDecScanRows;
+  float *dts = dsmem + lay.dts();  // [16][36] dt_proj result
+  const int cbase = blockIdx.x * kScanCh;
+  const int b0 = blockIdx.y * kScanRows;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nrows = min(kDecScanRows, a.B - b0);
-  const int nch = min(128, a.E - cbase);
+  const int nrows = min(kScanRows, a.B - b0);
+  const int ch = tid % kScanCh, rg = tid / kScanCh;  // channel, group of four rows
+  const int c = cbase + ch;
+  // the states of this thread's four rows: issued first, consumed last
+  float4 hv[4][kStates / 4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int b = min(b0 + rg * 4 + k, a.B - 1);  // rows past the batch re-read the last row
+    const float4 *hp = reinterpret_cast<const float4 *>(a.h + ((long long)b * a.E + c) * kStates);
+#pragma unroll
+    for (int q = 0; q < kStates / 4; ++q) hv[k][q] = hp[q];
+  }
   {
     const float *src = a.w_dt + (long long)cbase * R;
     const int per_row = R / 4;
-    for (int idx = tid; idx < nch * per_row; idx += 128) {
-      const int ch = idx / per_row, pc = idx % per_row;
-      cp_async16(wdt + ch * lay.WS + pc * 4, src + (long long)ch * R + pc * 4);
+    for (int idx = tid; idx < kScanCh * per_row; idx += 128) {
+      const int r = idx / per_row, pc = idx % per_row;
+      cp_async16(wdt + r * lay.WS + pc * 4, src + (long long)r * R + pc * 4);
     }
-    for (int idx = tid; idx < 128 * (lay.RP - R); idx += 128) {
-      const int ch = idx / (lay.RP - R), k = R + idx % (lay.RP - R);
-      wdt[ch * lay.WS + k] = 0.f;
-    }
-    for (int idx = tid; idx < (128 - nch) * R; idx += 128) wdt[(nch + idx / R) * lay.WS + idx % R] = 0.f;
+    for (int idx = tid; idx < kScanCh * (lay.RP - R); idx += 128)
+      wdt[(idx / (lay.RP - R)) * lay.WS + R + idx % (lay.RP - R)] = 0.f;
     const float *xsrc = a.xdbl + (long long)b0 * NJ;
     for (int idx = tid; idx < nrows * (NJ / 4); idx += 128) {
       const int r = idx / (NJ / 4), pc = idx % (NJ / 4);
       cp_async16(xs + r * lay.XS + pc * 4, xsrc + (long long)r * NJ + pc * 4);
     }
-    for (int idx = tid; idx < (16 - nrows) * lay.RP; idx += 128)
+    for (int idx = tid; idx < (kScanRows - nrows) * lay.RP; idx += 128)
       xs[(nrows + idx / lay.RP) * lay.XS + idx % lay.RP] = 0.f;
     cp_async_commit();
   }
-  const int c = cbase + tid;
-  const bool live = tid < nch;
   float A2[kStates];
-  float bdt = 0.f, Dc = 0.f;
-  if (live) {
+  {
     const float4 *al4 = reinterpret_cast<const float4 *>(a.a_log + (long long)c * kStates);
 #pragma unroll
     for (int q = 0; q < kStates / 4; ++q) {
@@ -437,129 +361,124 @@ __global__ void __launch_bounds__(128, 3) dec_dt_scan_kernel(DecodeSsmArgs a) {
       A2[4 * q + 2] = -kLog2e * ex2_ftz(kLog2e * v.z);
       A2[4 * q + 3] = -kLog2e * ex2_ftz(kLog2e * v.w);
     }
-    bdt = a.b_dt[c];
-    Dc = a.d_skip[c];
+  }
+  const float bdt = __ldg(a.b_dt + c), Dc = __ldg(a.d_skip + c);
+  const T *u = reinterpret_cast<const T *>(a.u);
+  const T *z = reinterpret_cast<const T *>(a.z);
+  T ur[4], zr[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int b = min(b0 + rg * 4 + k, a.B - 1);
+    ur[k] = u[(long long)b * a.E + c];
+    zr[k] = z[(long long)b * a.ld_z + c];
   }
   cp_async_wait<0>();
   __syncthreads();
-  // dt_proj on the tensor cores: warp w -> channels 32w..32w+31 (four 8-column tiles)
+  // dt_proj: warp w -> channels 8w..8w+7 of the slice, all 16 rows
   {
     const int g = lane >> 2, t = lane & 3;
-    float d[4][4];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) d[nt][e] = 0.f;
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    const float *wr = wdt + (warp * 8 + g) * lay.WS;
     for (int k0 = 0; k0 < lay.RP; k0 += 8) {
       const uint32_t a0 = to_tf32(xs[g * lay.XS + k0 + t]), a1 = to_tf32(xs[(g + 8) * lay.XS + k0 + t]);
       const uint32_t a2 = to_tf32(xs[g * lay.XS + k0 + t + 4]), a3 = to_tf32(xs[(g + 8) * lay.XS + k0 + t + 4]);
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt) {
-        const float *wr = wdt + (warp * 32 + nt * 8 + g) * lay.WS + k0;
-        mma_tf32_16808(d[nt], a0, a1, a2, a3, to_tf32(wr[t]), to_tf32(wr[t + 4]));
-      }
+      mma_tf32_16808(d, a0, a1, a2, a3, to_tf32(wr[k0 + t]), to_tf32(wr[k0 + t + 4]));
     }
-    if (g < kDecScanRows) {
-#pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-        *reinterpret_cast<float2 *>(dts + g * 132 + warp * 32 + nt * 8 + 2 * t) = make_float2(d[nt][0], d[nt][1]);
-    }
+    *reinterpret_cast<float2 *>(dts + g * (kScanCh + 4) + warp * 8 + 2 * t) = make_float2(d[0], d[1]);
+    *reinterpret_cast<float2 *>(dts + (g + 8) * (kScanCh + 4) + warp * 8 + 2 * t) = make_float2(d[2], d[3]);
   }
   __syncthreads();
-  if (!live) return;
-  const T *u = reinterpret_cast<const T *>(a.u);
-  const T *z = reinterpret_cast<const T *>(a.z);
   T *y = reinterpret_cast<T *>(a.y);
-  // raw loads, converted at their use, so that the loads of row rr + 1 stay in flight
-  // while row rr is computed (rows past the batch read the last row and are discarded)
-  float4 hn[kStates / 4];
-  T un, zn;
-  auto load_row = [&](int rr) {
-    const int b = min(b0 + rr, a.B - 1);
-    const float4 *hp = reinterpret_cast<const float4 *>(a.h + ((long long)b * a.E + c) * kStates);
 #pragma unroll
-    for (int q = 0; q < kStates / 4; ++q) hn[q] = hp[q];
-    un = u[(long long)b * a.E + c];
-    zn = z[(long long)b * a.ld_z + c];
-  };
-  load_row(0);
-#pragma unroll
-  for (int rr = 0; rr < kDecScanRows; ++rr) {
-    const int b = b0 + rr;
-    float4 hv[kStates / 4];
-#pragma unroll
-    for (int q = 0; q < kStates / 4; ++q) hv[q] = hn[q];
-    const T ur = un, zr = zn;
-    if (rr + 1 < kDecScanRows) load_row(rr + 1);
-    if (rr >= nrows) continue;
-    const float uu = Store<T>::to_f(ur), zz = Store<T>::to_f(zr);
-    const float dl = softplus_dec<T>(dts[rr * 132 + tid] + bdt);
+  for (int k = 0; k < 4; ++k) {
+    const int r = rg * 4 + k, b = b0 + r;
+    if (r >= nrows) break;
+    const float uu = Store<T>::to_f(ur[k]), gate = Store<T>::to_f(zr[k]);
+    const float dl = softplus_dec<T>(dts[r * (kScanCh + 4) + ch] + bdt);
     const float du = dl * uu;
+    const float *Bv = xs + r * lay.XS + R, *Cv = Bv + kStates;
     float4 *hp = reinterpret_cast<float4 *>(a.h + ((long long)b * a.E + c) * kStates);
-    const float *Bv = xs + rr * lay.XS + R, *Cv = Bv + kStates;
     float acc = 0.f;
 #pragma unroll
     for (int q = 0; q < kStates / 4; ++q) {
       const float4 B4 = *reinterpret_cast<const float4 *>(Bv + 4 * q);
       const float4 C4 = *reinterpret_cast<const float4 *>(Cv + 4 * q);
-      hv[q].x = fmaf(ex2_ftz(A2[4 * q] * dl), hv[q].x, du * B4.x);
-      hv[q].y = fmaf(ex2_ftz(A2[4 * q + 1] * dl), hv[q].y, du * B4.y);
-      hv[q].z = fmaf(ex2_ftz(A2[4 * q + 2] * dl), hv[q].z, du * B4.z);
-      hv[q].w = fmaf(ex2_ftz(A2[4 * q + 3] * dl), hv[q].w, du * B4.w);
-      acc = fmaf(C4.x, hv[q].x, fmaf(C4.y, hv[q].y, fmaf(C4.z, hv[q].z, fmaf(C4.w, hv[q].w, acc))));
-      hp[q] = hv[q];
+      float4 h = hv[k][q];
+      h.x = fmaf(ex2_ftz(A2[4 * q] * dl), h.x, du * B4.x);
+      h.y = fmaf(ex2_ftz(A2[4 * q + 1] * dl), h.y, du * B4.y);
+      h.z = fmaf(ex2_ftz(A2[4 * q + 2] * dl), h.z, du * B4.z);
+      h.w = fmaf(ex2_ftz(A2[4 * q + 3] * dl), h.w, du * B4.w);
+      acc = fmaf(C4.x, h.x, fmaf(C4.y, h.y, fmaf(C4.z, h.z, fmaf(C4.w, h.w, acc))));
+      hp[q] = h;
     }
-    y[(long long)b * a.E + c] = Store<T>::from_f(fmaf(Dc, uu, acc) * zz);
+    y[(long long)b * a.E + c] = Store<T>::from_f(fmaf(Dc, uu, acc) * gate);
   }
 }
 
-template <typename T, int CH>
-static hymba_status decode_ssm_t(const DecodeSsmArgs &a, cudaStream_t s) {
-  const int NJ = a.R + 2 * a.N;
-  const int smem1 = CH * kDecRows * 4 + NJ * (CH * (int)sizeof(T) + 16);
-  const int smem2 = DecDtLayout(a.R, a.N).floats() * 4;
-  if (smem1 > 200 * 1024 || smem2 > 200 * 1024) {
-    set_error("decode SSM: dt_rank %d too large for the fused decode kernels", a.R);
+template <typename T>
+static hymba_status decode_conv_t(const DecodeSsmArgs &a, cudaStream_t s) {
+  constexpr int V = 16 / sizeof(T);
+  const long long n = (long long)a.B * (a.E / V);
+  dec_conv_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a);
+  return HYMBA_OK;
+}
+
+template <typename T>
+static hymba_status decode_scan_t(const DecodeSsmArgs &a, cudaStream_t s) {
+  const int smem = DecScanLayout(a.R, a.N).floats() * 4;
+  if (smem > 200 * 1024) {
+    set_error("decode SSM: dt_rank %d too large for the scan-step kernel", a.R);
     return HYMBA_ERR_UNSUPPORTED;
   }
   static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set.done(dev)) {
-    if (cudaFuncSetAttribute(dec_conv_xproj_kernel<T, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             200 * 1024) != cudaSuccess ||
-        cudaFuncSetAttribute(dec_dt_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             200 * 1024) != cudaSuccess) {
-      set_error("cudaFuncSetAttribute(decode SSM smem) failed");
+    if (cudaFuncSetAttribute(dec_scan_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024) !=
+        cudaSuccess) {
+      set_error("cudaFuncSetAttribute(decode scan smem) failed");
       return HYMBA_ERR_CUDA;
     }
     attr_set.mark(dev);
   }
-  dim3 g1(a.E / CH, (a.B + kDecRows - 1) / kDecRows);
-  dec_conv_xproj_kernel<T, CH><<<g1, 256, smem1, s>>>(a);
-  dim3 g2((a.E + 127) / 128, (a.B + kDecScanRows - 1) / kDecScanRows);
-  dec_dt_scan_kernel<T><<<g2, 128, smem2, s>>>(a);
+  dim3 grid(a.E / kScanCh, (a.B + kScanRows - 1) / kScanRows);
+  dec_scan_kernel<T><<<grid, 128, smem, s>>>(a);
   return HYMBA_OK;
 }
 
-hymba_status decode_ssm(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s) {
-  if (a.N != kStates || a.K > 4 || a.E % 32) {
-    set_error("decode SSM needs d_state 16, d_conv <= 4, d_inner %% 32 == 0");
+static hymba_status decode_check(const DecodeSsmArgs &a, hymba_dtype dt) {
+  const int V = dt == HYMBA_BF16 ? 8 : 4;
+  if (a.N != kStates || a.K > 4 || a.K < 1 || a.E % kScanCh || a.E % V || a.R % 4) {
+    set_error("decode SSM needs d_state 16, 1 <= d_conv <= 4, d_inner %% 32 == 0, dt_rank %% 4 == 0");
     return HYMBA_ERR_UNSUPPORTED;
   }
-  hymba_status st;
-  if (dt == HYMBA_BF16)
-    st = a.E % 128 == 0 ? decode_ssm_t<__nv_bfloat16, 128>(a, s) : decode_ssm_t<__nv_bfloat16, 32>(a, s);
-  else
-    st = a.E % 128 == 0 ? decode_ssm_t<float, 128>(a, s) : decode_ssm_t<float, 32>(a, s);
-  if (st != HYMBA_OK) return st;
-  note_launch(2);
+  return HYMBA_OK;
+}
+
+static hymba_status launched(const char *what) {
+  note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
-    set_error("decode SSM launch failed: %s", cudaGetErrorString(e));
+    set_error("decode %s launch failed: %s", what, cudaGetErrorString(e));
     return HYMBA_ERR_CUDA;
   }
   return HYMBA_OK;
+}
+
+hymba_status decode_conv(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s) {
+  hymba_status st = decode_check(a, dt);
+  if (st != HYMBA_OK) return st;
+  st = dt == HYMBA_BF16 ? decode_conv_t<__nv_bfloat16>(a, s) : decode_conv_t<float>(a, s);
+  if (st != HYMBA_OK) return st;
+  return launched("conv");
+}
+
+hymba_status decode_scan(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s) {
+  hymba_status st = decode_check(a, dt);
+  if (st != HYMBA_OK) return st;
+  st = dt == HYMBA_BF16 ? decode_scan_t<__nv_bfloat16>(a, s) : decode_scan_t<float>(a, s);
+  if (st != HYMBA_OK) return st;
+  return launched("scan step");
 }
 
 // ---------------------------------------------------------------------------

@@ -311,6 +311,45 @@ HYMBA_API hymba_status hymba_layer_decode_step_static(hymba_layer *layer, int ba
                                                       hymba_ssm_cache *ssm_cache,
                                                       hymba_stream_t stream);
 
+/* ---- the Hymba block ------------------------------------------------------ */
+
+/* A block of the model (Fig. 4 (b); Appendix E Table 11: MLP hidden 5504 at 1.5B): the
+ * hybrid-head module and an MLP, each behind an RMS norm with a learnable weight and
+ * inside a residual:
+ *     h = x + M(norm1(x)),   out = h + W_down (SiLU(W_gate n) * (W_up n)),  n = norm2(h)
+ * (the pages give the caption and the MLP width only; this gated form is the one whose
+ * parameter count gives the printed 1.52B).  The mixer M is the layer of `layer` (its
+ * weights, K/V sharing, caches and RoPE as for hymba_layer_prefill / _decode_step).
+ *   norm1, norm2  [d_model] fp32
+ *   w_gate_up     [2 * mlp_hidden, d_model] dtype: row 2i is W_gate's row i, row 2i+1 W_up's
+ *   w_down        [d_model, mlp_hidden] dtype
+ * mlp_hidden a multiple of 8.  Device pointers, 16-byte aligned, owned by the caller. */
+typedef struct {
+  const float *norm1;
+  const float *norm2;
+  const void *w_gate_up;
+  const void *w_down;
+  int mlp_hidden;
+} hymba_block_weights;
+
+HYMBA_API hymba_status hymba_block_prefill_workspace(const hymba_layer *layer, int mlp_hidden, int batch,
+                                                     int n_tokens, size_t *bytes);
+/* The block over `batch` sequences of L = n_meta + n_tokens rows of the residual stream:
+ * x, y [batch, L, d_model] dtype (distinct buffers); other arguments as for
+ * hymba_layer_prefill.  A stack of blocks chains y into the next block's x. */
+HYMBA_API hymba_status hymba_block_prefill(hymba_layer *layer, const hymba_block_weights *bw, int batch,
+                                           int n_tokens, const void *x, void *y, hymba_kv_seq *kv,
+                                           hymba_kv_cache *kv_cache, hymba_ssm_cache *ssm_cache,
+                                           void *workspace, size_t workspace_bytes, hymba_stream_t stream);
+HYMBA_API hymba_status hymba_block_decode_workspace(const hymba_layer *layer, int mlp_hidden, int batch,
+                                                    int64_t max_pos, size_t *bytes);
+/* The block for one new row per sequence: x_t, y_t [batch, d_model] dtype (distinct);
+ * other arguments as for hymba_layer_decode_step. */
+HYMBA_API hymba_status hymba_block_decode_step(hymba_layer *layer, const hymba_block_weights *bw, int batch,
+                                               int64_t pos, const void *x_t, void *y_t,
+                                               hymba_kv_cache *kv_cache, hymba_ssm_cache *ssm_cache,
+                                               void *workspace, size_t workspace_bytes, hymba_stream_t stream);
+
 /* ---- status and diagnostics -------------------------------------------- */
 
 /* Synchronises `stream`, then reports a pending CUDA error or a device-side

@@ -375,3 +375,55 @@ def layer_decode(x_t, pos: int, w: dict, s: Spec, cache: dict, kv_cache: dict | 
     f = fuse(o, y_ssm, _f64(w["beta_attn"]), _f64(w["beta_ssm"]), s.eps)
     Y = f @ _f64(w["w_out"]).T
     return Y[0], new
+
+
+# ---------------------------------------------------------------------------
+# The Hymba block and a stack of blocks (Hymba Fig. 4 (b) and Appendix E Table 11:
+# the hybrid-head module and an MLP, each behind a norm and inside a residual)
+# ---------------------------------------------------------------------------
+# Readings (the pages give Fig. 4's caption and the MLP width only): pre-norm, an RMS norm
+# with a learnable weight before the mixer and before the MLP; a residual around each; the
+# MLP gated by SiLU, down(SiLU(x W_gate^T) * (x W_up^T)), the form whose parameter count,
+# with the module of this layer and a tied embedding of a 32K vocabulary, gives the
+# printed 1.52B of Table 11 (an ungated MLP gives 1.2B).
+
+def rms_norm(x: np.ndarray, weight: np.ndarray, eps: float) -> np.ndarray:
+    """x / sqrt(mean(x^2) + eps) * weight over the last axis."""
+    return rms_normalise(x, eps) * weight
+
+
+def mlp(x: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
+    return (silu(x @ w_gate.T) * (x @ w_up.T)) @ w_down.T
+
+
+def block_prefill(xt, w: dict, s: Spec, kv_from: dict | None = None, capacity: int | None = None):
+    """One block over one sequence X~ [L, d] (the residual stream): h = x + M(norm1(x)),
+    out = h + MLP(norm2(h)).  w: the layer's weights plus norm1, norm2 [d], w_gate, w_up
+    [F, d], w_down [d, F].  Returns (out, the mixer's result dict)."""
+    xt = _f64(xt)
+    mix = layer_prefill(rms_norm(xt, _f64(w["norm1"]), s.eps), w, s, kv_from=kv_from, capacity=capacity)
+    h = xt + mix["Y"]
+    out = h + mlp(rms_norm(h, _f64(w["norm2"]), s.eps), _f64(w["w_gate"]), _f64(w["w_up"]), _f64(w["w_down"]))
+    return out, mix
+
+
+def block_decode(x_t, pos: int, w: dict, s: Spec, cache: dict, kv_cache: dict | None = None):
+    """The block for one new row: (out [d], the mixer's new cache)."""
+    x_t = _f64(x_t)
+    y, new = layer_decode(rms_norm(x_t, _f64(w["norm1"]), s.eps), pos, w, s, cache, kv_cache=kv_cache)
+    h = x_t + y
+    out = h + mlp(rms_norm(h[None, :], _f64(w["norm2"]), s.eps), _f64(w["w_gate"]), _f64(w["w_up"]),
+                  _f64(w["w_down"]))[0]
+    return out, new
+
+
+def stack_prefill(xt, weights: list, specs: list, producers: list):
+    """A stack of blocks over one sequence X~ [L, d]: block l reads block l-1's output;
+    producers[l] is None for a block that owns its K/V, else the index of the block whose
+    K/V it shares.  Returns the last output and every block's mixer result."""
+    x = _f64(xt)
+    mixes = []
+    for w, s, p in zip(weights, specs, producers):
+        x, mix = block_prefill(x, w, s, kv_from=None if p is None else mixes[p])
+        mixes.append(mix)
+    return x, mixes

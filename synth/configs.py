@@ -175,6 +175,25 @@ def layer_weights(w: Workload, layer: int, consumer: bool = False, device="cpu",
     return out
 
 
+def block_weights(w: Workload, layer: int, mlp_hidden: int, device="cpu", std: float = 0.02) -> dict:
+    """Seeded weights of a block's norms and MLP (the mixer's come from layer_weights):
+    norm1, norm2 [d] fp32 ~ U(0.5, 1.5); w_gate, w_up [F, d] and w_down [d, F] N(0, std) in
+    the storage dtype; and w_gate_up [2F, d], the gate and up rows interleaved (row 2i =
+    w_gate row i, row 2i+1 = w_up row i), the layout the library takes."""
+    d = w.dims.d_model
+    dt = torch_dtype(w.dtype)
+    pre = f"{w.name}/L{layer}/block/"
+    s = w.seed
+    wg = gen.normal_tensor((mlp_hidden, d), s, pre + "w_gate", std, device=device).to(dt)
+    wu = gen.normal_tensor((mlp_hidden, d), s, pre + "w_up", std, device=device).to(dt)
+    return dict(
+        norm1=gen.uniform_tensor((d,), s, pre + "norm1", 0.5, 1.5, device=device),
+        norm2=gen.uniform_tensor((d,), s, pre + "norm2", 0.5, 1.5, device=device),
+        w_gate=wg, w_up=wu,
+        w_gate_up=torch.stack([wg, wu], dim=1).reshape(2 * mlp_hidden, d).contiguous(),
+        w_down=gen.normal_tensor((d, mlp_hidden), s, pre + "w_down", std, device=device).to(dt))
+
+
 def meta_tokens(w: Workload, device="cpu", std: float = DEFAULT_STD.meta) -> torch.Tensor:
     """The m learnable meta rows R (seeded), [m, d_model], storage dtype."""
     return gen.normal_tensor((w.n_meta, w.dims.d_model), w.seed, f"{w.name}/meta", std,

@@ -57,3 +57,26 @@ def layer_prefill(xt, w: dict, s: O.Spec, kv_from: dict | None = None) -> dict:
     f = bf16(O.fuse(o, y_ssm, w["beta_attn"], w["beta_ssm"], s.eps))
     Y = bf16(f @ np.asarray(w["w_out"], np.float64).T)
     return dict(q=q, k=k, v=v, x_ssm=xs, gate=gate, o=o, u=u, delta=delta, y_ssm=y_ssm, f=f, Y=Y, h=h)
+
+
+def block_prefill(xt, w: dict, s: O.Spec, kv_from: dict | None = None):
+    """The block (norm1, mixer, residual, norm2, gated MLP, residual) with the bf16 roundings
+    of the CUDA path: the normed rows, the residual stream after each half and the MLP's
+    hidden rows are stored in bf16.  Returns (out, the mixer's result dict)."""
+    xt = np.asarray(xt, dtype=np.float64)
+    xn = bf16(O.rms_norm(xt, np.asarray(w["norm1"], np.float64), s.eps))
+    mix = layer_prefill(xn, w, s, kv_from=kv_from)
+    h = bf16(xt + mix["f"] @ np.asarray(w["w_out"], np.float64).T)
+    hn = bf16(O.rms_norm(h, np.asarray(w["norm2"], np.float64), s.eps))
+    hid = bf16(O.silu(hn @ np.asarray(w["w_gate"], np.float64).T) * (hn @ np.asarray(w["w_up"], np.float64).T))
+    out = bf16(h + hid @ np.asarray(w["w_down"], np.float64).T)
+    return out, mix
+
+
+def stack_prefill(xt, weights: list, specs: list, producers: list):
+    x = np.asarray(xt, dtype=np.float64)
+    mixes = []
+    for w, s, p in zip(weights, specs, producers):
+        x, mix = block_prefill(x, w, s, kv_from=None if p is None else mixes[p])
+        mixes.append(mix)
+    return x, mixes

@@ -332,3 +332,27 @@ def test_rope_configuration_is_validated():
     finally:
         hy.hymba_layer_destroy(h)
         hy.hymba_layer_destroy(plain)
+
+
+def test_block_calls_validate_before_launch():
+    p = hy.hymba_layer_create(_cfg(), _fake_weights())
+    A = 1 << 44
+    try:
+        bw = hy.hymba_block_weights(A, A, A, A, 5504)
+        ws = hy.hymba_block_prefill_workspace(p, 5504, 2, 100)
+        assert ws > hy.hymba_layer_prefill_workspace(p, 2, 100)
+        kv = hy.hymba_kv_seq(A, A, 0, 0, 0)
+        for bad in (hy.hymba_block_weights(A, A, A, A, 5500),      # not a multiple of 8
+                    hy.hymba_block_weights(A, None, A, A, 5504),   # missing norm
+                    hy.hymba_block_weights(A, A, A + 4, A, 5504)):  # misaligned
+            with pytest.raises(hy.HymbaError):
+                hy.hymba_block_prefill(p, bad, 2, 100, A, A + (1 << 32), kv, None, None, A, ws)
+        with pytest.raises(hy.HymbaError) as e:   # the output may not alias the input
+            hy.hymba_block_prefill(p, bw, 2, 100, A, A, kv, None, None, A, ws)
+        assert e.value.status == hy.HYMBA_ERR_INVALID_ARG
+        with pytest.raises(hy.HymbaError) as e:
+            hy.hymba_block_prefill(p, bw, 2, 100, A, A + (1 << 32), kv, None, None, A, ws - 256)
+        assert e.value.status == hy.HYMBA_ERR_WORKSPACE
+        assert hy.hymba_block_decode_workspace(p, 5504, 128, 8320) > hy.hymba_layer_decode_workspace(p, 128, 8320)
+    finally:
+        hy.hymba_layer_destroy(p)

@@ -479,3 +479,99 @@ def test_p12_rms_normalise():
     n = O.rms_normalise(x, 0.0)
     np.testing.assert_allclose(np.sqrt((n ** 2).mean(1)), 1.0, rtol=1e-14)
     np.testing.assert_allclose(n * np.sqrt((x ** 2).mean(1, keepdims=True)), x, rtol=1e-14)
+
+
+# --- the block and the stack (Fig. 4 (b); Table 11) ----------------------------------------------
+
+def _block_weights(s, seed, consumer=False, F=12):
+    r = np.random.default_rng(seed)
+    w = _small.weights(s, seed=seed, consumer=consumer)
+    d = s.d_model
+    w.update(norm1=r.uniform(0.5, 1.5, d), norm2=r.uniform(0.5, 1.5, d), w_gate=r.normal(0, 0.3, (F, d)),
+             w_up=r.normal(0, 0.3, (F, d)), w_down=r.normal(0, 0.3, (d, F)))
+    return w
+
+
+def test_block_with_zero_branches_is_the_identity():
+    s = _small.spec()
+    w = _block_weights(s, 41)
+    w["w_out"] = np.zeros_like(w["w_out"])
+    w["w_down"] = np.zeros_like(w["w_down"])
+    x = _small.x_tilde(s, 12)
+    out, _ = O.block_prefill(x, w, s)
+    np.testing.assert_array_equal(out, x)
+
+
+def test_mlp_and_norm_against_scalar_loops():
+    import math
+    rng = np.random.default_rng(42)
+    d, F = 5, 3
+    x = rng.normal(size=(2, d))
+    wg, wu, wd = rng.normal(size=(F, d)), rng.normal(size=(F, d)), rng.normal(size=(d, F))
+    nw = rng.uniform(0.5, 1.5, d)
+    got = O.mlp(x, wg, wu, wd)
+    gn = O.rms_norm(x, nw, 1e-6)
+    for r in range(2):
+        ms = sum(v * v for v in x[r]) / d
+        for c in range(d):
+            assert abs(gn[r, c] - x[r, c] / math.sqrt(ms + 1e-6) * nw[c]) < 1e-12
+        hid = []
+        for f in range(F):
+            g = sum(x[r, k] * wg[f, k] for k in range(d))
+            u = sum(x[r, k] * wu[f, k] for k in range(d))
+            hid.append(g / (1.0 + math.exp(-g)) * u)
+        for c in range(d):
+            assert abs(got[r, c] - sum(hid[f] * wd[c, f] for f in range(F))) < 1e-10
+
+
+@pytest.mark.parametrize("glob", [False, True])
+def test_block_decode_after_prefill(glob):
+    s = _small.spec(m=3, W=4, is_global=glob)
+    wp, wc = _block_weights(s, 43), _block_weights(s, 44, consumer=True)
+    L = 14
+    x = _small.x_tilde(s, L + 1)
+    cap = L + 1 if glob else None
+    full_p, mix_fp = O.block_prefill(x, wp, s, capacity=cap)
+    full_c, _ = O.block_prefill(full_p, wc, s, kv_from=mix_fp)
+    pre_p, mix_p = O.block_prefill(x[:L], wp, s, capacity=cap)
+    pre_c, mix_c = O.block_prefill(pre_p, wc, s, kv_from=mix_p)
+    yp, newp = O.block_decode(x[L], L, wp, s, dict(k=mix_p["k_cache"], v=mix_p["v_cache"], ssm=mix_p["h"],
+                                                   conv=mix_p["conv"]))
+    np.testing.assert_allclose(yp, full_p[L], rtol=1e-11, atol=1e-12)
+    yc, _ = O.block_decode(yp, L, wc, s, dict(ssm=mix_c["h"], conv=mix_c["conv"]), kv_cache=newp)
+    np.testing.assert_allclose(yc, full_c[L], rtol=1e-11, atol=1e-12)
+
+
+def test_stack_chains_blocks_and_shares_kv():
+    s = _small.spec(m=2, W=3)
+    ws = [_block_weights(s, 50), _block_weights(s, 51, consumer=True), _block_weights(s, 52)]
+    x = _small.x_tilde(s, 9)
+    out, mixes = O.stack_prefill(x, ws, [s, s, s], [None, 0, None])
+    a, m0 = O.block_prefill(x, ws[0], s)
+    b, _ = O.block_prefill(a, ws[1], s, kv_from=m0)
+    c, _ = O.block_prefill(b, ws[2], s)
+    np.testing.assert_array_equal(out, c)
+    assert mixes[1]["k"] is mixes[0]["k"]  # the consumer attends over its producer's K/V
+
+
+def test_parameter_count_reading_of_the_mlp():
+    """Table 11 prints 1.52B parameters for the 1.5B model.  With this layer's module
+    (K/V projections only in the 18 layers that own K/V), a tied embedding of a 32K
+    vocabulary and a gated MLP (gate, up, down) the count is 1.52B; an ungated MLP
+    (up, down) would give 1.24B."""
+    g = json.load(open(os.path.join(GOLDEN, "parameter_count.json")))
+    t = g["table11_1p5b"]
+    d, H, G, N, F = t["d_model"], t["n_heads"], t["n_kv_heads"], t["d_state"], t["mlp_hidden"]
+    E, dq, R, K = 3200, 64, 100, 4
+    dv = E // H
+    owners = t["global_layers"] + 15
+    consumers = t["blocks"] - owners
+    def mixer(own):
+        P = H * dq + (G * (dq + dv) if own else 0) + 2 * E
+        return P * d + E * K + E + (R + 2 * N) * E + E * R + E + E * N + E + 2 * E + d * E + 2 * d
+    mixers = owners * mixer(True) + consumers * mixer(False)
+    emb = g["assumed_vocab"] * d + 128 * d   # tied embedding + meta tokens
+    gated = mixers + t["blocks"] * 3 * d * F + emb
+    ungated = mixers + t["blocks"] * 2 * d * F + emb
+    assert abs(gated - g["printed"]["parameters_1p5b"]) < 0.01e9, gated
+    assert abs(ungated - g["printed"]["parameters_1p5b"]) > 0.25e9, ungated

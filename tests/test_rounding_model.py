@@ -139,3 +139,25 @@ def test_planted_scan_mistakes_fail_the_bounds():
     y, _ = O.selective_scan(ref2["u"], ref2["delta"], -np.exp(wt2["a_log"]), ref2["B"], ref2["C"],
                             0 * wt2["d_skip"])
     assert _fails(y * O.silu(ref2["z"]), ref2["y_ssm"], mag2["y_ssm"])
+
+
+def test_block_stack_rounding_within_the_chained_bound():
+    """Four blocks (global, sliding-window producer, consumer, global) with the bf16
+    roundings of the CUDA path: the stack's output error stays within 0.6 of the
+    two-chained-layer bound that the GPU test applies to it."""
+    D = LayerDims(d_model=256, n_heads=4, n_kv_heads=2, head_dim_qk=64, d_inner=512)
+    w = Workload("block_stack", D, "bf16", 2, 16, 200, 64)
+    layout = [(True, None), (False, None), (False, 1), (True, None)]
+    ws, specs, prods = [], [], []
+    for l, (g, p) in enumerate(layout):
+        lw = {k: H.to64(v) for k, v in synth.configs.layer_weights(w, l, consumer=p is not None).items()}
+        lw.update({k: H.to64(v) for k, v in synth.configs.block_weights(w, l, 512).items()})
+        ws.append(lw)
+        specs.append(H.spec_of(w, g))
+        prods.append(p)
+    for b in range(2):
+        x = H.to64(synth.configs.x_tilde(w)[b])
+        r, _ = O.stack_prefill(x, ws, specs, prods)
+        e, _ = E.stack_prefill(x, ws, specs, prods)
+        ratio = float((np.abs(e - r) / (H.CHAIN2_ATOL + H.CHAIN2_RTOL * np.abs(r))).max())
+        assert ratio <= 0.6, ratio
