@@ -128,10 +128,15 @@ class ClockSampler:
 # ---------------------------------------------------------------------------------------------
 # our path
 # ---------------------------------------------------------------------------------------------
+BRANCH_CHUNKS = 4  # batch chunks of the concurrent prefill (the two branches side by side)
+
+
 class Prefill:
     """The two KV-sharing prefill layers of the headline workload.  A step computes the
     two layers' meta-token caches (batch 1: the m meta rows are the same in every sequence,
-    Hymba §2.3) and then prefills the B x n real rows of both layers from them."""
+    Hymba §2.3) and then prefills the B x n real rows of both layers from them.  The
+    layers exist twice over the same weights: with the concurrent schedule (the timed step)
+    and with the serial one (the per-kernel figures, each kernel alone on the GPU)."""
 
     def __init__(self, w, dev):
         import hybrid_attention_ssm_head_b200 as hy
@@ -141,15 +146,18 @@ class Prefill:
         d = w.dims
         B, L, n = w.batch, w.seq_rows, w.n_tokens
         self.B, self.L, self.n = B, L, n
-        self.wts, self.handles = [], []
+        self.wts, self.handles, self.handles_serial = [], [], []
         for layer, consumer in ((0, False), (1, True)):
             wt = {k: v.contiguous() for k, v in
                   synth.configs.layer_weights(w, layer, consumer=consumer, device=dev).items()}
-            cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner, d.d_state,
-                                 d.d_conv, d.rank, w.n_meta, w.window, False, "bf16")
             self.wts.append(wt)
-            self.handles.append(hy.hymba_layer_create(cfg, hy.make_weights(wt)))
+            for hs, chunks in ((self.handles, BRANCH_CHUNKS), (self.handles_serial, 0)):
+                cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner, d.d_state,
+                                     d.d_conv, d.rank, w.n_meta, w.window, False, "bf16",
+                                     branch_chunks=chunks)
+                hs.append(hy.hymba_layer_create(cfg, hy.make_weights(wt)))
         hy.hymba_kv_share_bind(self.handles[1], self.handles[0])
+        hy.hymba_kv_share_bind(self.handles_serial[1], self.handles_serial[0])
         m = w.n_meta
         self.m = m
         self.meta_x = synth.configs.meta_tokens(w, device=dev)          # R [m, d]
@@ -173,22 +181,23 @@ class Prefill:
                 bufs["k"].data_ptr() if layer == 0 else None, bufs["v"].data_ptr() if layer == 0 else None,
                 bufs["h"].data_ptr(), bufs["conv"].data_ptr(), bufs["y"].data_ptr(), 0))
         nb = max(max(hy.hymba_layer_prefill_cached_workspace(h, B, n), hy.hymba_layer_meta_workspace(h))
-                 for h in self.handles)
+                 for h in self.handles + self.handles_serial)
         self.ws = torch.empty(nb, dtype=torch.uint8, device=dev)
         self._full = None
 
-    def run(self, stream, x=None, y=None):
+    def run(self, stream, x=None, y=None, serial=False):
         """One step: both layers' meta caches, then both layers over the real rows."""
         hy = self.hy
         x = self.x if x is None else x
         y = self.y2 if y is None else y
-        hy.hymba_layer_meta_precompute(self.handles[0], self.meta_x, self.metas[0], None, self.ws,
+        hs = self.handles_serial if serial else self.handles
+        hy.hymba_layer_meta_precompute(hs[0], self.meta_x, self.metas[0], None, self.ws,
                                        self.ws.numel(), stream)
-        hy.hymba_layer_meta_precompute(self.handles[1], self.meta_bufs[0]["y"], self.metas[1], self.metas[0],
+        hy.hymba_layer_meta_precompute(hs[1], self.meta_bufs[0]["y"], self.metas[1], self.metas[0],
                                        self.ws, self.ws.numel(), stream)
-        hy.hymba_layer_prefill_cached(self.handles[0], self.B, self.n, x, self.y1, self.metas[0], self.kv, None,
+        hy.hymba_layer_prefill_cached(hs[0], self.B, self.n, x, self.y1, self.metas[0], self.kv, None,
                                       None, self.ws, self.ws.numel(), stream)
-        hy.hymba_layer_prefill_cached(self.handles[1], self.B, self.n, self.y1, y, self.metas[1], self.kv, None,
+        hy.hymba_layer_prefill_cached(hs[1], self.B, self.n, self.y1, y, self.metas[1], self.kv, None,
                                       None, self.ws, self.ws.numel(), stream)
 
     def run_full(self, stream):
@@ -326,18 +335,19 @@ MUFU_OPS_PER_CLK_SM = 16  # MUFU (ex2/rcp/lg2) results per clock per SM on sm_10
 SCAN_MUFU_PER_CHANNEL_STEP = 16  # the 16 decays exp2(delta A) (the gate SiLU(z) comes precomputed)
 
 
-def kernel_fractions(pre, dec, prof, dprof, peaks, sm_mhz, sms):
+def kernel_fractions(pre, dec, prof, dprof, peaks, sm_mhz, sms, layer_calls):
     """Each hot kernel's achieved rate against its bound: algorithmic FLOPs (tensor-bound
-    kernels) or bytes (memory-bound kernels) over the CUDA-event time the library's
-    profiler measured for it inside the timed region.  The scan is also reported against
-    its MUFU floor (its 16 MUFU operations per channel-step at the sampled SM clock)."""
+    kernels) or bytes (memory-bound kernels) of one layer over the CUDA-event time the
+    library's profiler measured for it (summed over a layer's batch chunks; `layer_calls`
+    layer prefills were profiled).  The scan is also reported against its MUFU floor (its
+    16 MUFU operations per channel-step at the sampled SM clock)."""
     d, w = pre.w.dims, pre.w
     B, L = pre.B, pre.L
     M = B * pre.n  # the prefill's main launches run over the real rows (the meta rows are cached)
     E, H, R, N = d.d_inner, d.n_heads, d.rank, d.d_state
     hbm = peaks.get("hbm_gbs", 6650.0)
     tens = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops", 1400.0))
-    pm = {n: ms / c for n, c, _, ms in prof if c}
+    pm = {n: ms / layer_calls for n, c, _, ms in prof if c}
     out = {}
 
     def tensor(name, flops):
@@ -429,6 +439,21 @@ def run_ours(args, rank, world, dev):
     prof = hy.hymba_profile_collect()
     hy.hymba_profile_enable(False)
     clocks = sampler.stop() if rank == 0 else None
+    # the serial schedule (every kernel alone on the GPU): per-kernel figures and step time
+    steps_serial = max(1, min(args.steps, 3))
+    pre.run(stream, serial=True)
+    torch.cuda.synchronize()
+    hy.hymba_profile_enable(True)
+    hy.hymba_profile_collect()
+    es0, es1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    es0.record(stream)
+    for _ in range(steps_serial):
+        pre.run(stream, serial=True)
+    es1.record(stream)
+    torch.cuda.synchronize()
+    sprof = hy.hymba_profile_collect()
+    hy.hymba_profile_enable(False)
+    serial_ms = max_over_ranks([es0.elapsed_time(es1) / steps_serial], dev, world)[0]
     # for comparison: the same two layers without the meta cache (every sequence's m + n rows)
     steps_full = max(1, min(args.steps, 3))
     pre.run_full(stream)
@@ -467,9 +492,10 @@ def run_ours(args, rank, world, dev):
     # roofline of the dominant kernel: the input projection GEMM (tensor-bound)
     pmap = {n: (c, ms) for n, c, _, ms in prof}
     c_in, ms_in = pmap.get("in_proj", (0, 0.0))
+    # (the concurrent schedule launches it once per batch chunk: the FLOPs of all its launches
+    # in the timed region over the sum of their CUDA-event durations)
     fl = pre.in_proj_flops()
-    flops_per_launch = sum(fl) / 2.0
-    achieved = (flops_per_launch * c_in) / (ms_in / 1e3) / 1e12 if ms_in > 0 else None
+    achieved = (sum(fl) * args.steps) / (ms_in / 1e3) / 1e12 if ms_in > 0 else None
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     roof = {"kernel": "in_proj (gemm_tc_kernel<256,bf16>)", "bound": "tensor",
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -547,7 +573,8 @@ def run_ours(args, rank, world, dev):
 
     sm_mhz = clocks.get("sm_mhz") if clocks else None
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    kernels = kernel_fractions(pre, dec, prof, dprof, peaks, sm_mhz, sms)
+    kernels = kernel_fractions(pre, dec, prof, dprof, peaks, sm_mhz, sms, 2 * args.steps)
+    kernels_serial = kernel_fractions(pre, dec, sprof, dprof, peaks, sm_mhz, sms, 2 * steps_serial)
 
     if rank != 0:
         return None
@@ -563,6 +590,8 @@ def run_ours(args, rank, world, dev):
                    "l2": "inputs larger than L2 (no flush)"},
         "prefill_ms_per_step": pre_ms / args.steps,
         "prefill_without_meta_cache_ms_per_step": full_ms,
+        "prefill_serial_ms_per_step": serial_ms,
+        "branch_chunks": BRANCH_CHUNKS,
         "decode_ms_per_step": dec_ms / args.steps,
         "decode_tok_s": dec_tok_s,
         "prefill_tflops": step_flops * args.steps / (pre_ms / 1e3) / 1e12,
@@ -576,6 +605,9 @@ def run_ours(args, rank, world, dev):
         "decode_steps_profile": {n: {"calls": c, "kernels": k, "ms_per_call": ms / c if c else None}
                                  for n, c, k, ms in dprof},
         "kernels": kernels,
+        "kernels_serial": kernels_serial,
+        "steps_profile_serial": {n: {"calls": c, "kernels": k, "ms_per_call": ms / c if c else None}
+                                 for n, c, k, ms in sprof},
         "gpu_launches": pre_launches + dec_kernels_per_step * args.steps,
         "clocks": clocks,
         "e2e": e2e,
@@ -689,8 +721,23 @@ def run_case(args, dev):
     prof = hy.hymba_profile_collect()
     hy.hymba_profile_enable(False)
     hy.hymba_stream_status(stream)
-    print(json.dumps({"case": args.case, "steps": args.steps, "profile": {
-        n: {"calls": c, "kernels": kk, "ms_per_call": ms / c} for n, c, kk, ms in prof}}), flush=True)
+    out = {"case": args.case, "steps": args.steps, "profile": {
+        n: {"calls": c, "kernels": kk, "ms_per_call": ms / c} for n, c, kk, ms in prof}}
+    if args.case in ("decode", "decode-b32"):
+        # the step as the headline times it: one CUDA graph replay per step
+        dec.capture()
+        for _ in range(3):
+            dec.graph.replay()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        t0.record()
+        for _ in range(args.steps):
+            dec.graph.replay()
+        t1.record()
+        torch.cuda.synchronize()
+        hy.hymba_stream_status(stream)
+        out["graph_ms_per_step"] = t0.elapsed_time(t1) / args.steps
+    print(json.dumps(out), flush=True)
 
 
 def main():

@@ -29,7 +29,7 @@ class hymba_layer_config(C.Structure):
                 ("d_state", C.c_int), ("d_conv", C.c_int), ("dt_rank", C.c_int),
                 ("n_meta", C.c_int), ("window", C.c_int), ("is_global", C.c_int),
                 ("dtype", C.c_int), ("rms_eps", C.c_float), ("softmax_scale", C.c_float),
-                ("rope_base", C.c_float)]
+                ("rope_base", C.c_float), ("branch_chunks", C.c_int)]
 
 
 class hymba_layer_weights(C.Structure):
@@ -375,11 +375,13 @@ def hymba_profile_collect(max_entries: int = 64) -> list[tuple[str, int, int, fl
 # ---- marshalling helpers ---------------------------------------------------------------
 
 def make_config(d_model, n_heads, n_kv_heads, head_dim_qk, d_inner, d_state, d_conv, dt_rank,
-                n_meta, window, is_global, dtype: str, rms_eps=1e-6, softmax_scale=0.0, rope_base=0.0):
+                n_meta, window, is_global, dtype: str, rms_eps=1e-6, softmax_scale=0.0, rope_base=0.0,
+                branch_chunks=4):
+    """branch_chunks: batch chunks of the concurrent prefill (0 or 1: serial order)."""
     return hymba_layer_config(d_model, n_heads, n_kv_heads, head_dim_qk, d_inner // n_heads, d_inner,
                               d_state, d_conv, dt_rank, n_meta, window if not is_global else 0,
                               int(bool(is_global)), HYMBA_BF16 if dtype == "bf16" else HYMBA_F32,
-                              rms_eps, softmax_scale, rope_base)
+                              rms_eps, softmax_scale, rope_base, branch_chunks)
 
 
 def make_weights(w: dict) -> hymba_layer_weights:

@@ -39,6 +39,26 @@ long long wait_limit_cycles() {
   if (v <= 0) v = kDefaultWaitLimit;
   return std::max(v, kMinWaitLimit);
 }
+static thread_local bool t_pdl = false;
+bool pdl_enabled() { return t_pdl; }
+PdlScope::PdlScope() : prev(t_pdl) { t_pdl = true; }
+PdlScope::~PdlScope() { t_pdl = prev; }
+
+static thread_local bool t_prio_set = false;
+static thread_local int t_prio = 0;
+bool launch_priority(int *prio) {
+  if (t_prio_set) *prio = t_prio;
+  return t_prio_set;
+}
+PrioScope::PrioScope(int prio) : prev_set(t_prio_set), prev(t_prio) {
+  t_prio_set = true;
+  t_prio = prio;
+}
+PrioScope::~PrioScope() {
+  t_prio_set = prev_set;
+  t_prio = prev;
+}
+
 static std::atomic<int> g_stall{0};
 int take_debug_stall() {
   int v = g_stall.load();
@@ -113,13 +133,58 @@ class ProfScope {
 };
 }  // namespace
 
+// Side stream of the concurrent prefill (branch_chunks >= 2) and its events: one fork
+// event, then per chunk one after its dt_proj and one after its scan.
+constexpr int kMaxBranchChunks = 8;
+constexpr int kBranchEvents = 1 + 2 * kMaxBranchChunks;
+struct BranchStreams {
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev[kBranchEvents] = {};
+  int prio_hi = 0;  // the greatest scheduling priority of the device (main chain)
+  bool ready = false;
+};
+
 struct hymba_layer {
   hymba_layer_config cfg;
   hymba_layer_weights w;
   uint64_t id;
   const hymba_layer *producer;  // non-null for a K/V-sharing consumer
   uint64_t producer_id;
+  BranchStreams br;
 };
+
+static void branch_release(BranchStreams &b) {
+  for (cudaEvent_t &e : b.ev)
+    if (e) {
+      cudaEventDestroy(e);
+      e = nullptr;
+    }
+  if (b.side) cudaStreamDestroy(b.side);
+  b.side = nullptr;
+  b.ready = false;
+}
+// Creates the side stream (lowest priority, non-blocking) and the events on the current
+// device.  False (and nothing kept) when that fails, e.g. without a device.
+static bool branch_create(BranchStreams &b) {
+  if (b.ready) return true;
+  int least = 0, greatest = 0;
+  if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+      cudaStreamCreateWithPriority(&b.side, cudaStreamNonBlocking, least) != cudaSuccess) {
+    cudaGetLastError();
+    b.side = nullptr;
+    return false;
+  }
+  for (cudaEvent_t &e : b.ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      cudaGetLastError();
+      e = nullptr;
+      branch_release(b);
+      return false;
+    }
+  b.prio_hi = greatest;
+  b.ready = true;
+  return true;
+}
 
 static std::atomic<uint64_t> g_next_id{1};
 
@@ -180,6 +245,8 @@ hymba_status hymba_layer_create(const hymba_layer_config *cfg, const hymba_layer
   if (!(c.rope_base >= 0.f) || !std::isfinite(c.rope_base)) FAIL(HYMBA_ERR_INVALID_ARG, "rope_base < 0");
   if (c.rope_base > 0.f && (c.rope_base <= 1.f || (c.head_dim_qk & (c.head_dim_qk - 1)) || c.head_dim_qk < 2))
     FAIL(HYMBA_ERR_UNSUPPORTED, "rotary embedding needs a base > 1 and a power-of-two head_dim_qk");
+  if (c.branch_chunks < 0 || c.branch_chunks > kMaxBranchChunks)
+    FAIL(HYMBA_ERR_INVALID_ARG, "branch_chunks %d outside 0..%d", c.branch_chunks, kMaxBranchChunks);
   if (c.d_state != 16) FAIL(HYMBA_ERR_UNSUPPORTED, "d_state must be 16");
   if (c.d_conv > 4) FAIL(HYMBA_ERR_UNSUPPORTED, "d_conv must be <= 4");
   if (c.dt_rank % 4) FAIL(HYMBA_ERR_UNSUPPORTED, "dt_rank must be a multiple of 4 (16-byte rows of W_dt)");
@@ -208,11 +275,18 @@ hymba_status hymba_layer_create(const hymba_layer_config *cfg, const hymba_layer
   L->id = g_next_id.fetch_add(1);
   L->producer = nullptr;
   L->producer_id = 0;
+  // the concurrent prefill's side stream, on the current device (retried at the first
+  // prefill where no device was usable here)
+  if (c.branch_chunks >= 2) branch_create(L->br);
   *out = L;
   return HYMBA_OK;
 }
 
-void hymba_layer_destroy(hymba_layer *layer) { delete layer; }
+void hymba_layer_destroy(hymba_layer *layer) {
+  if (!layer) return;
+  branch_release(layer->br);
+  delete layer;
+}
 
 int hymba_layer_is_consumer(const hymba_layer *layer) { return layer && layer->producer ? 1 : 0; }
 
@@ -236,6 +310,14 @@ hymba_status hymba_kv_share_bind(hymba_layer *consumer, const hymba_layer *produ
 // ---------------------------------------------------------------------------
 // prefill
 // ---------------------------------------------------------------------------
+// Batch chunks of the concurrent prefill: *n chunks of *bc sequences (the last one may be
+// shorter); n = 1 runs the serial order.
+static void branch_split(const hymba_layer_config &c, int batch, int *n, int *bc) {
+  const int want = c.branch_chunks >= 2 ? std::min(c.branch_chunks, batch) : 1;
+  *bc = (batch + want - 1) / want;
+  *n = (batch + *bc - 1) / *bc;
+}
+
 // Workspace of a prefill whose intermediates have `rows` rows per sequence: all L = m + n
 // rows, or the n real rows when the meta rows come from a precomputed meta cache.
 static hymba_status prefill_layout_rows(const hymba_layer *layer, int batch, long long rows,
@@ -261,6 +343,8 @@ static hymba_status prefill_layout_rows(const hymba_layer *layer, int batch, lon
   o->y_ssm = take(M * E * es);
   o->o_attn = take(M * E * es);
   o->fused = take(M * E * es);
+  // the scan's chunk states for the whole batch (a concurrent prefill's batch chunks scan
+  // with the whole batch's time chunks, one after another, in the same region)
   size_t sf = scan_workspace_floats(batch, (int)rows, c.d_inner, c.d_state, nullptr);
   if (scan_floats) *scan_floats = sf;
   take(sf * 4);  // scan chunk states, after `fused`
@@ -371,6 +455,14 @@ static const char *step_name(const PrefillRun &r, int step) {
   return names[r.meta ? 1 : 0][step];
 }
 
+// Byte pointer to element `elems` of a buffer of `es`-byte elements.
+static void *elem_at(void *base, long long elems, size_t es) {
+  return base ? reinterpret_cast<char *>(base) + elems * (long long)es : nullptr;
+}
+static const void *celem_at(const void *base, long long elems, size_t es) {
+  return base ? reinterpret_cast<const char *>(base) + elems * (long long)es : nullptr;
+}
+
 static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun &r, hymba_kv_seq *kv,
                                 hymba_kv_cache *kv_cache, hymba_ssm_cache *ssm_cache, void *workspace,
                                 const hymba_prefill_layout &lay, cudaStream_t stream) {
@@ -380,6 +472,7 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
   const long long M = (long long)batch * r.rows;
   const size_t es = esize(c.dtype);
   const int E = c.d_inner;
+  const int XW = xdbl_width(c);
   hymba_status st;
   if (M > 0x7fffffffLL) FAIL(HYMBA_ERR_UNSUPPORTED, "too many rows");
 
@@ -389,125 +482,139 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
   void *delta = ws + lay.delta, *yssm = ws + lay.y_ssm, *o = ws + lay.o_attn, *f = ws + lay.fused;
   float *scan_ws = reinterpret_cast<float *>(ws + lay.fused + up256((size_t)M * E * es));
 
+  // rotary table of positions 0..L-1 (§2.5 RoPE), shared by every sequence
+  float2 *rope_tab = nullptr;
+  if (c.rope_base > 0.f) {
+    rope_tab = reinterpret_cast<float2 *>(ws + lay.rope);
+    if ((st = rope_table(rope_tab, L, 0, c.head_dim_qk, c.rope_base, stream)) != HYMBA_OK) return st;
+  }
+
+  // The steps over the sequences b0 .. b0+nb-1 (rows m0 = b0 * rows .. of the intermediates).
   // 1. input projection (§2.1 W_in_proj) -> Q, K, V, x_ssm, SiLU(z); K and V go to their
   //    rows q_off.. of each sequence of the full-length K/V
-  {
-    ProfScope prof_scope(stream, step_name(r, 0));
+  auto in_proj = [&](int b0, int nb, cudaStream_t s) -> hymba_status {
+    ProfScope prof_scope(s, step_name(r, 0));
+    const long long m0 = (long long)b0 * r.rows;
     GemmArgs g{};
-    g.A = r.x;
+    g.A = celem_at(r.x, m0 * c.d_model, es);
     g.lda = c.d_model;
     g.B = layer->w.w_in;
     g.ldb = c.d_model;
-    g.M = (int)M;
+    g.M = (int)((long long)nb * r.rows);
     g.N = qk_width(c) + (consumer ? 0 : k_width(c) + v_width(c)) + 2 * E;
     g.K = c.d_model;
     g.elem = (int)es;
-    g.epi = in_proj_epilogue(c, consumer, q, qk_width(c), kv->k, kv->v, k_width(c), v_width(c), 0, 0,
-                             xs, z, E);
+    g.epi = in_proj_epilogue(c, consumer, elem_at(q, m0 * qk_width(c), es), qk_width(c),
+                             consumer ? nullptr : elem_at(kv->k, (long long)b0 * L * k_width(c), es),
+                             consumer ? nullptr : elem_at(kv->v, (long long)b0 * L * v_width(c), es),
+                             k_width(c), v_width(c), 0, 0, elem_at(xs, m0 * E, es), elem_at(z, m0 * E, es), E);
     if (!consumer && r.q_off > 0) {
       g.epi.seg[1].rmap = g.epi.seg[2].rmap = 1;
       g.epi.rmap_rows = r.rows;
       g.epi.rmap_stride = L;
       g.epi.rmap_off = r.q_off;
     }
-    if (c.rope_base > 0.f) {
-      // Q and K rotated in the epilogue (§2.5 RoPE), positions q_off.. of each sequence
-      float2 *tab = reinterpret_cast<float2 *>(ws + lay.rope);
-      if ((st = rope_table(tab, L, 0, c.head_dim_qk, c.rope_base, stream)) != HYMBA_OK) return st;
-      g.epi.rope_tab = tab;
+    if (rope_tab) {
+      // Q and K rotated in the epilogue, positions q_off.. of each sequence
+      g.epi.rope_tab = rope_tab;
       g.epi.rope_rows = r.rows;
       g.epi.rope_off = r.q_off;
       g.epi.rope_hd = c.head_dim_qk;
       g.epi.seg[0].rope = 1;
       if (!consumer) g.epi.seg[1].rope = 1;
     }
-    if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
-  }
+    return gemm(g, c.dtype, s);
+  };
   // 2. causal conv + SiLU -> u (and the conv state)
-  {
-    ProfScope prof_scope(stream, step_name(r, 1));
+  auto conv = [&](int b0, int nb, cudaStream_t s) -> hymba_status {
+    ProfScope prof_scope(s, step_name(r, 1));
+    const long long m0 = (long long)b0 * r.rows;
     ConvArgs a{};
-    a.x = xs;
+    a.x = elem_at(xs, m0 * E, es);
     a.ld_x = E;
-    a.u = u;
+    a.u = elem_at(u, m0 * E, es);
     a.w = layer->w.conv_w;
     a.bias = layer->w.conv_b;
-    a.conv_state = ssm_cache ? ssm_cache->conv : nullptr;
+    a.conv_state = ssm_cache ? elem_at(ssm_cache->conv, (long long)b0 * (c.d_conv - 1) * E, es) : nullptr;
     a.hist = r.conv0;
-    a.B = batch;
+    a.B = nb;
     a.L = r.rows;
     a.E = E;
     a.K = c.d_conv;
-    if ((st = conv_silu(a, c.dtype, stream)) != HYMBA_OK) return st;
-  }
+    return conv_silu(a, c.dtype, s);
+  };
   // 3. x_proj -> [delta_r, B, C] (fp32)
-  {
-    ProfScope prof_scope(stream, step_name(r, 2));
+  auto x_proj = [&](int b0, int nb, cudaStream_t s) -> hymba_status {
+    ProfScope prof_scope(s, step_name(r, 2));
+    const long long m0 = (long long)b0 * r.rows;
     GemmArgs g{};
-    g.A = u;
+    g.A = elem_at(u, m0 * E, es);
     g.lda = E;
     g.B = layer->w.w_x;
     g.ldb = E;
-    g.M = (int)M;
-    g.N = xdbl_width(c);
+    g.M = (int)((long long)nb * r.rows);
+    g.N = XW;
     g.K = E;
     g.elem = (int)es;
-    g.epi.seg[0] = seg(xdbl, xdbl_width(c), 0, xdbl_width(c), 1, es);
+    g.epi.seg[0] = seg(xdbl + m0 * XW, XW, 0, XW, 1, es);
     g.epi.nseg = 1;
-    if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
-  }
+    return gemm(g, c.dtype, s);
+  };
   // 4. dt_proj + bias + softplus -> delta (tf32 on the tensor cores for the bf16 path)
-  {
-    ProfScope prof_scope(stream, step_name(r, 3));
+  auto dt_proj = [&](int b0, int nb, cudaStream_t s) -> hymba_status {
+    ProfScope prof_scope(s, step_name(r, 3));
+    const long long m0 = (long long)b0 * r.rows;
     GemmArgs g{};
-    g.A = xdbl;
-    g.lda = xdbl_width(c);
+    g.A = xdbl + m0 * XW;
+    g.lda = XW;
     g.B = layer->w.w_dt;
     g.ldb = c.dt_rank;
-    g.M = (int)M;
+    g.M = (int)((long long)nb * r.rows);
     g.N = E;
     g.K = c.dt_rank;
     g.elem = 4;
-    g.epi.seg[0] = seg(delta, E, 0, E, c.dtype == HYMBA_F32, es);
+    g.epi.seg[0] = seg(elem_at(delta, m0 * E, es), E, 0, E, c.dtype == HYMBA_F32, es);
     g.epi.nseg = 1;
     g.epi.bias = layer->w.b_dt;
     g.epi.act = 1;
-    st = c.dtype == HYMBA_BF16 ? gemm_tc(g, stream) : gemm_simt_f32(g, stream);
-    if (st != HYMBA_OK) return st;
-  }
+    return c.dtype == HYMBA_BF16 ? gemm_tc(g, s) : gemm_simt_f32(g, s);
+  };
   // 5. selective scan + D skip, times the gate SiLU(z) -> y_ssm (and the final state)
-  {
-    ProfScope prof_scope(stream, step_name(r, 4));
+  auto scan = [&](int b0, int nb, cudaStream_t s) -> hymba_status {
+    ProfScope prof_scope(s, step_name(r, 4));
+    const long long m0 = (long long)b0 * r.rows;
     ScanArgs a{};
-    a.u = u;
-    a.delta = delta;
-    a.z = z;
+    a.u = elem_at(u, m0 * E, es);
+    a.delta = elem_at(delta, m0 * E, es);
+    a.z = elem_at(z, m0 * E, es);
     a.ld_z = E;
-    a.bc = xdbl;
-    a.ld_bc = xdbl_width(c);
+    a.bc = xdbl + m0 * XW;
+    a.ld_bc = XW;
     a.bc_col = c.dt_rank;
     a.a_log = layer->w.a_log;
     a.d_skip = layer->w.d_skip;
-    a.y = yssm;
-    a.h_out = ssm_cache ? ssm_cache->h : nullptr;
+    a.y = elem_at(yssm, m0 * E, es);
+    a.h_out = ssm_cache ? ssm_cache->h + (long long)b0 * E * c.d_state : nullptr;
     a.h_in = r.h0;
     a.h_in_bstride = 0;
-    a.B = batch;
+    a.B = nb;
     a.L = r.rows;
     a.E = E;
     a.N = c.d_state;
     a.chunk_ws = scan_ws;
-    if ((st = selective_scan(a, c.dtype, stream)) != HYMBA_OK) return st;
-  }
+    a.time_chunks = scan_time_chunks(batch, r.rows, E);
+    return selective_scan(a, c.dtype, s);
+  };
   // 6. attention heads over the own or the producer's K/V
-  {
-    ProfScope prof_scope(stream, step_name(r, 5));
+  auto attention = [&](int b0, int nb, cudaStream_t s) -> hymba_status {
+    ProfScope prof_scope(s, step_name(r, 5));
+    const long long m0 = (long long)b0 * r.rows;
     AttnArgs a{};
-    a.q = q;
-    a.k = kv->k;
-    a.v = kv->v;
-    a.o = o;
-    a.B = batch;
+    a.q = elem_at(q, m0 * qk_width(c), es);
+    a.k = elem_at(kv->k, (long long)b0 * L * k_width(c), es);
+    a.v = elem_at(kv->v, (long long)b0 * L * v_width(c), es);
+    a.o = elem_at(o, m0 * E, es);
+    a.B = nb;
     a.L = L;
     a.q_off = r.q_off;
     a.Lq = r.rows;
@@ -519,40 +626,99 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
     a.window = c.window;
     a.is_global = c.is_global;
     a.scale = score_scale(c);
-    if ((st = attention_prefill(a, c.dtype, stream)) != HYMBA_OK) return st;
-  }
+    return attention_prefill(a, c.dtype, s);
+  };
   // 7. norm, beta, mean (Eq. 3)
-  {
-    ProfScope prof_scope(stream, step_name(r, 6));
+  auto fuse = [&](int b0, int nb, cudaStream_t s) -> hymba_status {
+    ProfScope prof_scope(s, step_name(r, 6));
+    const long long m0 = (long long)b0 * r.rows;
     FuseArgs a{};
-    a.o = o;
-    a.y = yssm;
+    a.o = elem_at(o, m0 * E, es);
+    a.y = elem_at(yssm, m0 * E, es);
     a.beta_attn = layer->w.beta_attn;
     a.beta_ssm = layer->w.beta_ssm;
-    a.f = f;
-    a.M = (int)M;
+    a.f = elem_at(f, m0 * E, es);
+    a.M = (int)((long long)nb * r.rows);
     a.E = E;
     a.eps = c.rms_eps;
-    if ((st = fuse_branches(a, c.dtype, stream)) != HYMBA_OK) return st;
-  }
-  // 8. output projection
-  {
-    ProfScope prof_scope(stream, step_name(r, 7));
+    return fuse_branches(a, c.dtype, s);
+  };
+  // 8. output projection (plus the residual in a block)
+  auto out_proj = [&](int b0, int nb, cudaStream_t s) -> hymba_status {
+    ProfScope prof_scope(s, step_name(r, 7));
+    const long long m0 = (long long)b0 * r.rows;
     GemmArgs g{};
-    g.A = f;
+    g.A = elem_at(f, m0 * E, es);
     g.lda = E;
     g.B = layer->w.w_out;
     g.ldb = E;
-    g.M = (int)M;
+    g.M = (int)((long long)nb * r.rows);
     g.N = c.d_model;
     g.K = E;
     g.elem = (int)es;
-    g.epi.seg[0] = seg(r.y, c.d_model, 0, c.d_model, c.dtype == HYMBA_F32, es);
-    g.epi.seg[0].resid = r.resid;
+    g.epi.seg[0] = seg(elem_at(r.y, m0 * c.d_model, es), c.d_model, 0, c.d_model, c.dtype == HYMBA_F32, es);
+    g.epi.seg[0].resid = celem_at(r.resid, m0 * c.d_model, es);
     g.epi.seg[0].ld_resid = c.d_model;
     g.epi.nseg = 1;
     g.stall = take_debug_stall();
-    if ((st = gemm(g, c.dtype, stream)) != HYMBA_OK) return st;
+    return gemm(g, c.dtype, s);
+  };
+
+  int nch = 1, bc = batch;
+  branch_split(c, batch, &nch, &bc);
+  if (nch > 1 && !branch_create(layer->br)) {
+    set_error("could not create the concurrent prefill's side stream: %s", cudaGetErrorString(cudaGetLastError()));
+    return HYMBA_ERR_CUDA;
+  }
+  if (nch == 1) {
+    // serial order on the caller's stream
+    if ((st = in_proj(0, batch, stream)) != HYMBA_OK) return st;
+    if ((st = conv(0, batch, stream)) != HYMBA_OK) return st;
+    if ((st = x_proj(0, batch, stream)) != HYMBA_OK) return st;
+    if ((st = dt_proj(0, batch, stream)) != HYMBA_OK) return st;
+    if ((st = scan(0, batch, stream)) != HYMBA_OK) return st;
+    if ((st = attention(0, batch, stream)) != HYMBA_OK) return st;
+    if ((st = fuse(0, batch, stream)) != HYMBA_OK) return st;
+    if ((st = out_proj(0, batch, stream)) != HYMBA_OK) return st;
+  } else {
+    // The two branches side by side: chunk k's scan (MUFU-bound, one small CTA per SM beside
+    // a GEMM CTA) runs on the low-priority side stream while the caller's stream, at the
+    // device's highest priority, runs chunk k's attention and chunk k+1's projections; the
+    // last chunk's scan runs beside the first chunks' output projections.
+    BranchStreams &br = layer->br;
+    auto check = [](cudaError_t e, const char *what) -> hymba_status {
+      if (e == cudaSuccess) return HYMBA_OK;
+      set_error("%s failed: %s", what, cudaGetErrorString(e));
+      return HYMBA_ERR_CUDA;
+    };
+    cudaEvent_t ev_fork = br.ev[0];
+    if ((st = check(cudaEventRecord(ev_fork, stream), "cudaEventRecord")) != HYMBA_OK) return st;
+    if ((st = check(cudaStreamWaitEvent(br.side, ev_fork, 0), "cudaStreamWaitEvent")) != HYMBA_OK) return st;
+    for (int k = 0; k < nch; ++k) {
+      const int b0 = k * bc, nb = std::min(bc, batch - b0);
+      cudaEvent_t ev_dt = br.ev[1 + 2 * k], ev_scan = br.ev[2 + 2 * k];
+      {
+        PrioScope hi(br.prio_hi);
+        if ((st = in_proj(b0, nb, stream)) != HYMBA_OK) return st;
+        if ((st = conv(b0, nb, stream)) != HYMBA_OK) return st;
+        if ((st = x_proj(b0, nb, stream)) != HYMBA_OK) return st;
+        if ((st = dt_proj(b0, nb, stream)) != HYMBA_OK) return st;
+      }
+      if ((st = check(cudaEventRecord(ev_dt, stream), "cudaEventRecord")) != HYMBA_OK) return st;
+      if ((st = check(cudaStreamWaitEvent(br.side, ev_dt, 0), "cudaStreamWaitEvent")) != HYMBA_OK) return st;
+      if ((st = scan(b0, nb, br.side)) != HYMBA_OK) return st;
+      if ((st = check(cudaEventRecord(ev_scan, br.side), "cudaEventRecord")) != HYMBA_OK) return st;
+      PrioScope hi(br.prio_hi);
+      if ((st = attention(b0, nb, stream)) != HYMBA_OK) return st;
+    }
+    for (int k = 0; k < nch; ++k) {
+      const int b0 = k * bc, nb = std::min(bc, batch - b0);
+      if ((st = check(cudaStreamWaitEvent(stream, br.ev[2 + 2 * k], 0), "cudaStreamWaitEvent")) != HYMBA_OK)
+        return st;
+      PrioScope hi(br.prio_hi);
+      if ((st = fuse(b0, nb, stream)) != HYMBA_OK) return st;
+      if ((st = out_proj(b0, nb, stream)) != HYMBA_OK) return st;
+    }
   }
   // 9. decode K/V store
   if (kv_cache) {
@@ -842,6 +1008,8 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
   hymba_status st;
   const long long slot = (c.is_global || pos < c.n_meta) ? pos : c.n_meta + (pos - c.n_meta) % c.window;
   const long long cap = kv_cache->capacity;
+  // the step's kernels are launched programmatically: each starts while its predecessor ends
+  PdlScope pdl;
 
   // 1. input projection; a K/V owner writes this token's K/V straight into its slot
   {

@@ -166,17 +166,19 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s0)[32], const uint
 }
 // P for 32 keys of a row: exp2(s * scale - m) packed to bf16 pairs; returns the fp32
 // sum as a pair of partial sums.  Scale and shift run as packed fp32x2 FMAs; one key
-// pair in four takes its exponentials from the degree-3 polynomial on the FMA pipe
+// pair in eight takes its exponentials from the degree-3 polynomial on the FMA pipe
 // (relative error 7.5e-5, well inside the bf16 rounding of P) and the others from
-// the MUFU, so that the two pipes share the exponentials.
-template <int POLY8>
+// the MUFU.  The kernel is bound by issue more than by the MUFU: on a batch-32 layer
+// 0, 1, 2, 3 pairs of eight ran within 2 % of each other (1 fastest) and 4, 5, 6 pairs
+// were 6-17 % slower.
+constexpr int kPolyPairsOf8 = 1;  // key pairs of every eight on the polynomial
 __device__ __forceinline__ float2 p_pack(const uint32_t (&v)[32], uint32_t (&pk)[16], float2 scale2,
                                          float2 nm2) {
   float2 ls[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
   for (int e = 0; e < 32; e += 2) {
     const float2 x = ffma2(make_float2(__uint_as_float(v[e]), __uint_as_float(v[e + 1])), scale2, nm2);
-    const float2 p = ((e >> 1) & 7) < POLY8 ? exp2_poly2<3>(x) : make_float2(ex2(x.x), ex2(x.y));
+    const float2 p = ((e >> 1) & 7) < kPolyPairsOf8 ? exp2_poly2<3>(x) : make_float2(ex2(x.x), ex2(x.y));
     ls[(e >> 1) & 1] = fadd2(ls[(e >> 1) & 1], p);
     pk[e >> 1] = pack_bf16x2(p.x, p.y);
   }
@@ -199,12 +201,13 @@ __device__ __forceinline__ void p_store(const uint32_t (&pk)[16], int c, int r, 
 // item's Q and first K/V tiles stream in, and its first S = Q K^T is issued, while the
 // current item's last tile is still in the softmax; the softmax warpgroups write the
 // finished item's O between its last tile and the next item's first.
-template <int POLY8>
 __global__ void __launch_bounds__(fa::THREADS, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                        int L, int q_off, int B, int H, int Hkv, int n_meta, int window, int is_global,
                        float scale_log2, int npairs, long long wlim) {
+  pdl_wait();
+  pdl_trigger();
   using namespace fa;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -458,8 +461,8 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
         const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
         const float2 nm2 = make_float2(nm, nm), scale2 = make_float2(scale_log2, scale_log2);
         uint32_t pk0[16], pk1[16], pk2[16], pk3[16];
-        const float2 ps = fadd2(fadd2(p_pack<POLY8>(s0, pk0, scale2, nm2), p_pack<POLY8>(s1, pk1, scale2, nm2)),
-                                fadd2(p_pack<POLY8>(s2, pk2, scale2, nm2), p_pack<POLY8>(s3, pk3, scale2, nm2)));
+        const float2 ps = fadd2(fadd2(p_pack(s0, pk0, scale2, nm2), p_pack(s1, pk1, scale2, nm2)),
+                                fadd2(p_pack(s2, pk2, scale2, nm2), p_pack(s3, pk3, scale2, nm2)));
         l_run += ps.x + ps.y;
         if (__any_sync(0xffffffffu, resc)) {
           // O grows by the new max: rescale it once the previous tile's P V has retired
@@ -535,14 +538,13 @@ __global__ void __launch_bounds__(fa::THREADS, 1)
   }
 }
 
-template <int POLY8>
 static hymba_status attention_prefill_tc(const AttnArgs &a, cudaStream_t s) {
   using namespace fa;
   static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
   if (!attr_set.done(dev)) {
-    if (cudaFuncSetAttribute(attn_fwd_tc_kernel<POLY8>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
+    if (cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) !=
         cudaSuccess) {
       set_error("cudaFuncSetAttribute(attention smem) failed");
       return HYMBA_ERR_CUDA;
@@ -571,9 +573,9 @@ static hymba_status attention_prefill_tc(const AttnArgs &a, cudaStream_t s) {
   const long long items = (long long)npairs * a.H * a.B;
   if (items == 0) return HYMBA_OK;
   const unsigned grid = (unsigned)std::min<long long>(items, sms);
-  attn_fwd_tc_kernel<POLY8><<<grid, THREADS, SMEM, s>>>(
-      tq, tk, tv, to, a.L, a.q_off, a.B, a.H, a.Hkv, a.n_meta, a.window,
-      a.is_global, a.scale * 1.4426950408889634f, npairs, wait_limit_cycles());
+  launch_kernel(attn_fwd_tc_kernel, dim3(grid), dim3(THREADS), (size_t)SMEM, s, tq, tk, tv, to, a.L, a.q_off, a.B,
+                a.H, a.Hkv, a.n_meta, a.window, a.is_global, a.scale * 1.4426950408889634f, npairs,
+                wait_limit_cycles());
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -591,6 +593,8 @@ __global__ void attn_fwd_simt_kernel(const T *__restrict__ q, const T *__restric
                                      const T *__restrict__ v, T *__restrict__ o, int B, int L, int q_off,
                                      int Lq, int H, int Hkv, int dqk, int dv, int n_meta, int window,
                                      int is_global, float scale) {
+  pdl_wait();
+  pdl_trigger();
   const long long wid = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= (long long)B * Lq * H) return;
@@ -637,14 +641,7 @@ hymba_status attention_prefill(const AttnArgs &a, hymba_dtype dt, cudaStream_t s
       set_error("bf16 attention kernel supports head_dim_qk 64 and head_dim_v 128 only");
       return HYMBA_ERR_UNSUPPORTED;
     }
-    static const int poly8 = [] { const char *e = getenv("HYMBA_EXP_POLY8"); return e ? atoi(e) : 2; }();
-    switch (poly8) {
-      case 3: return attention_prefill_tc<3>(a, s);
-      case 4: return attention_prefill_tc<4>(a, s);
-      case 5: return attention_prefill_tc<5>(a, s);
-      case 6: return attention_prefill_tc<6>(a, s);
-      default: return attention_prefill_tc<2>(a, s);
-    }
+    return attention_prefill_tc(a, s);
   }
   if (a.dv > 256) {
     set_error("fp32 attention supports head_dim_v <= 256");
@@ -653,9 +650,9 @@ hymba_status attention_prefill(const AttnArgs &a, hymba_dtype dt, cudaStream_t s
   const long long warps = (long long)a.B * a.Lq * a.H;
   const int tpb = 256;
   const long long blocks = (warps * 32 + tpb - 1) / tpb;
-  attn_fwd_simt_kernel<float><<<(unsigned)blocks, tpb, 0, s>>>(
-      (const float *)a.q, (const float *)a.k, (const float *)a.v, (float *)a.o, a.B, a.L, a.q_off, a.Lq,
-      a.H, a.Hkv, a.dqk, a.dv, a.n_meta, a.window, a.is_global, a.scale);
+  launch_kernel(attn_fwd_simt_kernel<float>, dim3((unsigned)blocks), dim3(tpb), 0, s, (const float *)a.q,
+                (const float *)a.k, (const float *)a.v, (float *)a.o, a.B, a.L, a.q_off, a.Lq, a.H, a.Hkv,
+                a.dqk, a.dv, a.n_meta, a.window, a.is_global, a.scale);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -910,20 +907,24 @@ __global__ void __launch_bounds__(128)
 }
 
 // ---- bf16 decode attention on the tensor cores (mma.sync m16n8k16) ---------------
-// Persistent: the work is the list of 64-slot chunks of every (sequence, kv head),
+// Persistent: the work is the list of SLOTS-slot chunks of every (sequence, kv head),
 // item i = (b * Hkv + g) * nchunks + chunk, cut into equal contiguous ranges, one per
-// CTA (two CTAs per SM).  A CTA streams its chunks through four shared-memory stages by
+// CTA (two CTAs per SM).  A CTA streams its chunks through STAGES shared-memory stages by
 // 3-D TMA (128-byte swizzle, rows past the store's capacity read as zero), the copies of
-// the next three chunks in flight while the current one is computed, across (sequence, kv
-// head) boundaries too.  Warp w takes keys 16w..16w+15 of every chunk: S = Q K^T with
+// the next chunks in flight while the current one is computed, across (sequence, kv
+// head) boundaries too.  Warp w takes keys KW*w..KW*w+KW-1 of every chunk (KW = SLOTS/4):
+// S = Q K^T with
 // the query heads of the group in rows 0..rep-1 of a 16-row tile, an online softmax in
 // registers, O += P V with V fragments from ldmatrix.trans.  Where a run of chunks of
 // one (sequence, kv head) ends inside the CTA's range, the four warps' states are
 // merged in shared memory into one partial (max, sum, O) per query head, stored at the
 // slot of the run's first chunk; the combine kernel reads the run-start slots.
 namespace dtc {
-constexpr int SLOTS = 64;                   // slots per chunk: 16 per warp
-constexpr int STAGES = 4;                   // chunks in flight per CTA: three ahead of the one computed
+constexpr int SLOTS = 128;                  // slots per chunk
+constexpr int STAGES = 2;                   // chunks in flight per CTA: one ahead of the one computed
+constexpr int KW = SLOTS / 4;               // keys per warp
+constexpr int NT = KW / 8;                  // 8-key n-tiles of S per warp
+constexpr int KS = KW / 16;                 // 16-key k-steps of P V per warp
 constexpr int K_BYTES = SLOTS * 128;        // 64 bf16 per slot
 constexpr int V_BYTES = SLOTS * 256;        // two 64-column boxes
 constexpr int STAGE = K_BYTES + V_BYTES;
@@ -932,7 +933,7 @@ constexpr int MAXREP = 8;
 __host__ __device__ constexpr int merge_bytes(int rep) { return 4 * rep * 130 * 4; }
 __host__ __device__ constexpr int smem_bytes(int rep) { return STAGES * STAGE + merge_bytes(rep) + 8 * STAGES + 1024; }
 constexpr int CTAS_PER_SM = 2;
-static_assert(SLOTS == 64, "the warps' key mapping takes 16 slots each");
+static_assert(SLOTS % 64 == 0 && SLOTS <= 256, "whole 16-key steps per warp; TMA box rows <= 256");
 }  // namespace dtc
 
 // First chunk of every run: a run starts at chunk 0 of a (sequence, kv head) or at the
@@ -972,6 +973,8 @@ __global__ void __launch_bounds__(128)
                           int Hkv, long long pos, int n_meta, int window, int is_global,
                           float scale_log2, long long n_items, long long per, long long wlim) {
   using namespace dtc;
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t dsm_raw[];
   uint8_t *sm = dsm_raw + ((1024 - (smem_u32(dsm_raw) & 1023)) & 1023);
   const int rep = H / Hkv;
@@ -1035,15 +1038,15 @@ __global__ void __launch_bounds__(128)
     if (__syncthreads_or(!ok)) { ok = false; break; }
     const uint32_t kb = smem_u32(sm + st * STAGE), vb = kb + K_BYTES;
     const long long s0 = (long long)chunk * SLOTS;
-    // ---- S = Q K^T for this warp's 16 keys (2 n-tiles of 8 keys) ----
-    float sacc[2][4];
+    // ---- S = Q K^T for this warp's KW keys (NT n-tiles of 8 keys) ----
+    float sacc[NT][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const int key = warp * 16 + nt * 8 + (lane & 7);
+    for (int nt = 0; nt < NT; ++nt) {
+      const int key = warp * KW + nt * 8 + (lane & 7);
 #pragma unroll
       for (int kp = 0; kp < 2; ++kp) {  // two k-steps per ldmatrix.x4
         const int ch = kp * 4 + (lane >> 3);  // 16-byte chunk of the key row (8 dims)
@@ -1056,10 +1059,10 @@ __global__ void __launch_bounds__(128)
     // ---- online softmax, row gr (values sacc[nt][0..1], keys 8nt + 2gc + {0,1}) ----
     float mx = -INFINITY;
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int key = warp * 16 + nt * 8 + 2 * gc + e;
+        const int key = warp * KW + nt * 8 + 2 * gc + e;
         const bool valid = dec_key_valid(s0 + key, nslots, pos, n_meta, window, is_global);
         const float x = valid ? sacc[nt][e] * scale_log2 : -INFINITY;
         sacc[nt][e] = x;
@@ -1072,9 +1075,9 @@ __global__ void __launch_bounds__(128)
     const float alpha = m_run == -INFINITY ? 0.f : ex2(m_run - mref);
     m_run = m_new;
     float lsum = 0.f;
-    uint32_t pa[2];  // P as the A fragment of one 16-key step: a0a1 (n-tile 0) / a4a5 (n-tile 1)
+    uint32_t pa[NT];  // P as A fragments: [k-step kk][a0a1 (n-tile 2kk) / a4a5 (n-tile 2kk+1)]
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int nt = 0; nt < NT; ++nt) {
       const float p0 = ex2(sacc[nt][0] - mref), p1 = ex2(sacc[nt][1] - mref);
       lsum += p0 + p1;
       pa[nt] = pack_bf16x2(p0, p1);
@@ -1087,10 +1090,10 @@ __global__ void __launch_bounds__(128)
       oacc[nt][0] *= alpha;
       oacc[nt][1] *= alpha;
     }
-    // ---- O += P V (16 n-tiles of 8 value columns, one k-step of 16 keys) ----
-    {
-      const int kk = 0;
-      const int key = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    // ---- O += P V (16 n-tiles of 8 value columns, KS k-steps of 16 keys) ----
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+      const int key = warp * KW + kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int np = 0; np < 8; ++np) {  // pairs of n-tiles per ldmatrix.x4.trans
         const int chg = np * 2 + (lane >> 4);  // 16-byte chunk of value columns (0..15)
@@ -1099,7 +1102,6 @@ __global__ void __launch_bounds__(128)
         ldsm_x4_t(addr, b0, b1, b2, b3);
         mma16816(oacc[2 * np], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b0, b1);
         mma16816(oacc[2 * np + 1], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b2, b3);
-        (void)kk;
       }
     }
     __syncthreads();  // every warp is done with stage st
@@ -1260,9 +1262,9 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
     const long long n_items = (long long)a.B * a.Hkv * nchunks;
     const long long grid_tc = std::min<long long>(n_items, (long long)dtc::CTAS_PER_SM * sms);
     const long long per = (n_items + grid_tc - 1) / grid_tc;
-    attn_decode_tc_kernel<<<(unsigned)((n_items + per - 1) / per), 128, dtc::smem_bytes(rep), s>>>(
-        tk, tv, (const __nv_bfloat16 *)a.q, a.partial, a.H, a.Hkv, a.pos, a.n_meta, a.window,
-        a.is_global, sl2, n_items, per, wait_limit_cycles());
+    launch_kernel(attn_decode_tc_kernel, dim3((unsigned)((n_items + per - 1) / per)), dim3(128),
+                  (size_t)dtc::smem_bytes(rep), s, tk, tv, (const __nv_bfloat16 *)a.q, a.partial, a.H, a.Hkv,
+                  (long long)a.pos, a.n_meta, a.window, a.is_global, sl2, n_items, per, wait_limit_cycles());
     if (a.fuse_later) {
       a.nchunks_out = nchunks;
       a.per_out = per;
@@ -1343,6 +1345,8 @@ __global__ void kv_emit_kernel(const T *__restrict__ kseq, const T *__restrict__
                                T *__restrict__ kc, T *__restrict__ vc, int B, int L, int Hkv,
                                int dqk, int dv, int cap, int n_meta, int window, int is_global,
                                long long n_keep, int meta_keep, long long start) {
+  pdl_wait();
+  pdl_trigger();
   const long long total = (long long)B * Hkv * n_keep;
   const long long idx = (long long)blockIdx.x * blockDim.y + threadIdx.y;
   if (idx >= total) return;
@@ -1376,14 +1380,14 @@ hymba_status kv_cache_emit(const KvEmitArgs &a, hymba_dtype dt, cudaStream_t s) 
   dim3 block(32, 8);
   const long long blocks = (total + 7) / 8;
   if (dt == HYMBA_BF16)
-    kv_emit_kernel<__nv_bfloat16><<<(unsigned)blocks, block, 0, s>>>(
-        (const __nv_bfloat16 *)a.k_seq, (const __nv_bfloat16 *)a.v_seq, (__nv_bfloat16 *)a.k_cache,
-        (__nv_bfloat16 *)a.v_cache, a.B, a.L, a.Hkv, a.dqk, a.dv, a.cap, a.n_meta, a.window,
-        a.is_global, n_keep, meta_keep, start);
+    launch_kernel(kv_emit_kernel<__nv_bfloat16>, dim3((unsigned)blocks), block, 0, s,
+                  (const __nv_bfloat16 *)a.k_seq, (const __nv_bfloat16 *)a.v_seq, (__nv_bfloat16 *)a.k_cache,
+                  (__nv_bfloat16 *)a.v_cache, a.B, a.L, a.Hkv, a.dqk, a.dv, a.cap, a.n_meta, a.window,
+                  a.is_global, n_keep, meta_keep, start);
   else
-    kv_emit_kernel<float><<<(unsigned)blocks, block, 0, s>>>(
-        (const float *)a.k_seq, (const float *)a.v_seq, (float *)a.k_cache, (float *)a.v_cache, a.B,
-        a.L, a.Hkv, a.dqk, a.dv, a.cap, a.n_meta, a.window, a.is_global, n_keep, meta_keep, start);
+    launch_kernel(kv_emit_kernel<float>, dim3((unsigned)blocks), block, 0, s, (const float *)a.k_seq,
+                  (const float *)a.v_seq, (float *)a.k_cache, (float *)a.v_cache, a.B, a.L, a.Hkv, a.dqk,
+                  a.dv, a.cap, a.n_meta, a.window, a.is_global, n_keep, meta_keep, start);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -305,6 +305,31 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
 }
+// Hint: bring one tile of a 2-D tensor map into L2 (no shared memory, no completion).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+// Hint: bring `bytes` (a multiple of 16, 16-byte aligned address) into L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with the programmatic-serialisation
+// attribute may begin while the kernel before it in the stream is still running.  Before
+// pdl_wait() it touches only what no kernel of the library writes (weights, its own
+// shared memory and barriers, L2 prefetch hints); pdl_wait() returns once the preceding
+// grid has completed and its writes are visible (at once for a normal launch).  Every
+// CTA of such a kernel calls pdl_wait() before it reads or writes any other global
+// memory, so completion stays transitive along the stream.  pdl_trigger() lets the next
+// kernel in the stream start its own prologue.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation MMA (cta_group::1)

@@ -37,6 +37,8 @@ hymba_status exp2_poly_eval(int degree, const float *x, float *y, long long n, c
 
 // Rotary table in double precision (the angle of a late position is large), stored fp32.
 __global__ void rope_table_kernel(float2 *tab, int npos, long long pos0, int hd, double log2_base) {
+  pdl_wait();
+  pdl_trigger();
   const int hp = hd >> 1;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (long long)npos * hp) return;
@@ -51,7 +53,8 @@ __global__ void rope_table_kernel(float2 *tab, int npos, long long pos0, int hd,
 hymba_status rope_table(float2 *tab, int npos, long long pos0, int hd, float base, cudaStream_t s) {
   const long long n = (long long)npos * (hd / 2);
   if (n <= 0) return HYMBA_OK;
-  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(tab, npos, pos0, hd, log2((double)base));
+  launch_kernel(rope_table_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, tab, npos, pos0, hd,
+                log2((double)base));
   note_launch(1);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -47,6 +47,8 @@ __device__ __forceinline__ void unpack16(const uint4 &raw, float (&v)[16 / sizeo
 // more rows fit on an SM; they are unpacked again for the output pass.
 template <typename T, int NV>
 __global__ void __launch_bounds__(128) fuse_kernel(FuseArgs a) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int V = 16 / sizeof(T);
   __shared__ float red[2][4];
   const long long row = blockIdx.x;
@@ -122,6 +124,8 @@ __global__ void __launch_bounds__(128) fuse_kernel(FuseArgs a) {
 // Rows wider than the register path: two passes, the second from L1/L2.
 template <typename T>
 __global__ void __launch_bounds__(256) fuse_wide_kernel(FuseArgs a) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int V = 16 / sizeof(T);
   __shared__ float red[2][8];
   const long long row = blockIdx.x;
@@ -181,14 +185,14 @@ hymba_status fuse_branches(const FuseArgs &a, hymba_dtype dt, cudaStream_t s) {
   const bool regs = a.E <= 128 * V * 4;
   if (dt == HYMBA_BF16) {
     if (regs)
-      fuse_kernel<__nv_bfloat16, 4><<<a.M, 128, 0, s>>>(a);
+      launch_kernel(fuse_kernel<__nv_bfloat16, 4>, dim3(a.M), dim3(128), 0, s, a);
     else
-      fuse_wide_kernel<__nv_bfloat16><<<a.M, 256, 0, s>>>(a);
+      launch_kernel(fuse_wide_kernel<__nv_bfloat16>, dim3(a.M), dim3(256), 0, s, a);
   } else {
     if (regs)
-      fuse_kernel<float, 4><<<a.M, 128, 0, s>>>(a);
+      launch_kernel(fuse_kernel<float, 4>, dim3(a.M), dim3(128), 0, s, a);
     else
-      fuse_wide_kernel<float><<<a.M, 256, 0, s>>>(a);
+      launch_kernel(fuse_wide_kernel<float>, dim3(a.M), dim3(256), 0, s, a);
   }
   note_launch(1);
   cudaError_t e = cudaGetLastError();
@@ -204,6 +208,8 @@ hymba_status fuse_branches(const FuseArgs &a, hymba_dtype dt, cudaStream_t s) {
 // weights 2^(m_r - M) / L; the merged O (fp32, four values per lane) stays in registers
 // for the two RMS norms.
 __global__ void __launch_bounds__(1024) fuse_decode_kernel(FuseDecodeArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float red[2][32];
   const int b = blockIdx.x, h = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rep = a.H / a.Hkv, E = a.H * a.dv;
@@ -295,7 +301,7 @@ hymba_status fuse_decode(const FuseDecodeArgs &a, cudaStream_t s) {
     set_error("fuse_decode needs d_v 128 and at most 32 heads");
     return HYMBA_ERR_UNSUPPORTED;
   }
-  fuse_decode_kernel<<<a.B, 32 * a.H, 0, s>>>(a);
+  launch_kernel(fuse_decode_kernel, dim3(a.B), dim3(32 * a.H), 0, s, a);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

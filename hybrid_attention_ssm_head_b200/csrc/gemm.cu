@@ -338,6 +338,8 @@ template <int BN, int ELEM, int EPI>
 __global__ void __launch_bounds__(576, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    int M, int N, int K, Epilogue epi, long long wlim, int stall) {
+  pdl_wait();
+  pdl_trigger();
   using C = TcCfg<BN, ELEM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -596,6 +598,20 @@ __global__ void __launch_bounds__(128, 1)
     tma_prefetch_desc(&tmW);
     tma_prefetch_desc(&tmX);
   }
+  __syncthreads();
+  // The weights are no kernel's output: the first stages' weight tiles are requested, and
+  // the rest of this CTA's weight slice is hinted into L2, before the wait for the
+  // preceding kernel (whose tail they overlap under a programmatic launch).
+  const int npre = min(STAGES, kb1 - kb0);
+  if (warp == 0 && lane == 0) {
+    for (int i = 0; i < npre; ++i) {
+      mbar_arrive_expect_tx(&full[i], C::STAGE);
+      tma_load_2d(smem + i * C::STAGE, &tmW, &full[i], (kb0 + i) * BK, mt * BM);
+    }
+    for (int kb = kb0 + npre; kb < kb1; ++kb) tma_prefetch_l2_2d(&tmW, kb * BK, mt * BM);
+  }
+  pdl_wait();
+  pdl_trigger();
   if (warp == 1) {
     tmem_alloc(tmem_slot, BN);
     tmem_relinquish();
@@ -611,13 +627,17 @@ __global__ void __launch_bounds__(128, 1)
     uint32_t ph = 0, issued[STAGES] = {0, 0, 0, 0};
     bool ok = true;
     for (int kb = kb0; kb < kb1; ++kb) {
-      if (!mbar_wait(&empty[st], ph ^ 1u, &g_err_gemm, wlim)) {
-        ok = false;
-        break;
+      if (kb - kb0 < npre) {  // the weight tile of this (fresh) stage is already on its way
+        tma_load_2d(smem + st * C::STAGE + W_BYTES, &tmX, &full[st], kb * BK, 0);
+      } else {
+        if (!mbar_wait(&empty[st], ph ^ 1u, &g_err_gemm, wlim)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[st], C::STAGE);
+        tma_load_2d(smem + st * C::STAGE, &tmW, &full[st], kb * BK, mt * BM);
+        tma_load_2d(smem + st * C::STAGE + W_BYTES, &tmX, &full[st], kb * BK, 0);
       }
-      mbar_arrive_expect_tx(&full[st], C::STAGE);
-      tma_load_2d(smem + st * C::STAGE, &tmW, &full[st], kb * BK, mt * BM);
-      tma_load_2d(smem + st * C::STAGE + W_BYTES, &tmX, &full[st], kb * BK, 0);
       ++issued[st];
       if (++st == STAGES) {
         st = 0;
@@ -735,13 +755,13 @@ static hymba_status launch_ws(const GemmArgs &g, cudaStream_t s) {
   cfg.blockDim = dim3(128, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[3];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = launch_attrs(attr, 1);
   cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_ws_kernel<BN, CL>, tw, tx, g.N, g.M, g.K, g.epi,
                                      wait_limit_cycles());
   note_launch(1);
@@ -816,8 +836,8 @@ static hymba_status launch_tc(const GemmArgs &g, cudaStream_t s) {
   if (!make_tmap(&tb, g.B, dt, 2, db, sb, bb)) return HYMBA_ERR_CUDA;
   const long long tiles = (long long)((g.M + 127) / 128) * ((g.N + BN - 1) / BN);
   const int grid = (int)std::min<long long>(tiles, num_sms());
-  gemm_tc_kernel<BN, ELEM, EPI><<<grid, 576, C::SMEM, s>>>(ta, tb, g.M, g.N, g.K, g.epi,
-                                                     wait_limit_cycles(), g.stall);
+  launch_kernel(gemm_tc_kernel<BN, ELEM, EPI>, dim3(grid), dim3(576), (size_t)C::SMEM, s, ta, tb, g.M, g.N, g.K,
+                g.epi, wait_limit_cycles(), g.stall);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -870,6 +890,8 @@ hymba_status gemm_tc(const GemmArgs &g, cudaStream_t s) {
 __global__ void __launch_bounds__(256)
     gemm_simt_f32_kernel(const float *__restrict__ A, long long lda, const float *__restrict__ B,
                          long long ldb, int M, int N, int K, Epilogue epi) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
   const int tid = threadIdx.x;
@@ -946,9 +968,8 @@ __global__ void __launch_bounds__(256)
 
 hymba_status gemm_simt_f32(const GemmArgs &g, cudaStream_t s) {
   dim3 grid((g.N + 63) / 64, (g.M + 63) / 64);
-  gemm_simt_f32_kernel<<<grid, 256, 0, s>>>(reinterpret_cast<const float *>(g.A), g.lda,
-                                            reinterpret_cast<const float *>(g.B), g.ldb, g.M, g.N,
-                                            g.K, g.epi);
+  launch_kernel(gemm_simt_f32_kernel, grid, dim3(256), 0, s, reinterpret_cast<const float *>(g.A), g.lda,
+                reinterpret_cast<const float *>(g.B), g.ldb, g.M, g.N, g.K, g.epi);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -27,6 +27,61 @@ struct DeviceOnce {
 };
 
 
+// Programmatic dependent launch.  While a PdlScope is alive on the calling thread, the
+// kernels launched through launch_kernel (and the weight-streaming GEMM) carry the
+// programmatic-serialisation attribute, so that each may start its prologue while the
+// kernel before it in the stream finishes; every such kernel calls pdl_wait() (see
+// common.cuh) in every CTA before it touches memory that another kernel writes.
+bool pdl_enabled();
+struct PdlScope {
+  bool prev;
+  PdlScope();
+  ~PdlScope();
+  PdlScope(const PdlScope &) = delete;
+  PdlScope &operator=(const PdlScope &) = delete;
+};
+// Launch priority.  While a PrioScope is alive on the calling thread, the kernels launched
+// through launch_kernel (and the tensor-core GEMMs) carry that scheduling priority (lower
+// numbers first), so that their pending CTAs take freed SM space before those of a
+// lower-priority kernel running beside them.
+bool launch_priority(int *prio);
+struct PrioScope {
+  bool prev_set;
+  int prev;
+  explicit PrioScope(int prio);
+  ~PrioScope();
+  PrioScope(const PrioScope &) = delete;
+  PrioScope &operator=(const PrioScope &) = delete;
+};
+// The launch attributes of the calling thread's scopes, appended to attr[n..]; returns n.
+inline unsigned launch_attrs(cudaLaunchAttribute *attr, unsigned n) {
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  int prio = 0;
+  if (launch_priority(&prio)) {
+    attr[n].id = cudaLaunchAttributePriority;
+    attr[n].val.priority = prio;
+    ++n;
+  }
+  return n;
+}
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  cfg.attrs = attr;
+  cfg.numAttrs = launch_attrs(attr, 0);
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Args &&>(args)...);
+}
+
 // Where a GEMM output column goes.  Column c in [col0, col1) of the product is
 // written to  ptr + row*ld_row + ((c-col0)/inner)*ld_group + (c-col0)%inner
 // (element offsets), as fp32 (f32 = 1) or bf16 (f32 = 0).
@@ -120,8 +175,12 @@ struct ScanArgs {
   long long h_in_bstride;  // apart (0: one state for every sequence); zero when null
   int B, L, E, N;
   float *chunk_ws;     // workspace for the chunked scan (see scan_workspace_floats)
+  int time_chunks;     // time chunks of the scan (0: chosen from B, L, E); a batch split into
+                       // parts passes the whole batch's count, so every part rounds alike
 };
 size_t scan_workspace_floats(int B, int L, int E, int N, int *chunks_out);
+// The scan's time chunks for B sequences of L steps and E channels.
+int scan_time_chunks(int B, int L, int E);
 hymba_status selective_scan(const ScanArgs &a, hymba_dtype dt, cudaStream_t s);
 
 // ---- fused norm / beta / mean -------------------------------------------

@@ -104,6 +104,8 @@ __device__ __forceinline__ void unpack16(const uint4 &raw, float (&v)[16 / sizeo
 // vector per channel) and the bias are fetched once for all kConvTB rows.
 template <typename T>
 __global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int V = Vec16<T>::N;
   constexpr int NR = kConvTB + 3;
   const int nvec = a.E / V;
@@ -213,9 +215,9 @@ hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s) {
   if (n == 0) return HYMBA_OK;
   const unsigned blocks = (unsigned)((n + 127) / 128);
   if (dt == HYMBA_BF16)
-    conv_silu_kernel<__nv_bfloat16><<<blocks, 128, 0, s>>>(a);
+    launch_kernel(conv_silu_kernel<__nv_bfloat16>, dim3(blocks), dim3(128), 0, s, a);
   else
-    conv_silu_kernel<float><<<blocks, 128, 0, s>>>(a);
+    launch_kernel(conv_silu_kernel<float>, dim3(blocks), dim3(128), 0, s, a);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
@@ -236,6 +238,8 @@ __global__ void __launch_bounds__(256) dec_conv_kernel(DecodeSsmArgs a) {
   constexpr int V = 16 / sizeof(T);
   const int nv = a.E / V;
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (idx >= (long long)a.B * nv) return;
   const int b = (int)(idx / nv), c0 = (int)(idx % nv) * V;
   const int K = a.K;
@@ -323,15 +327,8 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
   const int nrows = min(kScanRows, a.B - b0);
   const int ch = tid % kScanCh, rg = tid / kScanCh;  // channel, group of four rows
   const int c = cbase + ch;
-  // the states of this thread's four rows: issued first, consumed last
-  float4 hv[4][kStates / 4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int b = min(b0 + rg * 4 + k, a.B - 1);  // rows past the batch re-read the last row
-    const float4 *hp = reinterpret_cast<const float4 *>(a.h + ((long long)b * a.E + c) * kStates);
-#pragma unroll
-    for (int q = 0; q < kStates / 4; ++q) hv[k][q] = hp[q];
-  }
+  // Before the wait for the preceding kernel: the weights (W_dt slice, A, biases) and an
+  // L2 hint for this CTA's state rows (2 KB per sequence).
   {
     const float *src = a.w_dt + (long long)cbase * R;
     const int per_row = R / 4;
@@ -341,14 +338,7 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
     }
     for (int idx = tid; idx < kScanCh * (lay.RP - R); idx += 128)
       wdt[(idx / (lay.RP - R)) * lay.WS + R + idx % (lay.RP - R)] = 0.f;
-    const float *xsrc = a.xdbl + (long long)b0 * NJ;
-    for (int idx = tid; idx < nrows * (NJ / 4); idx += 128) {
-      const int r = idx / (NJ / 4), pc = idx % (NJ / 4);
-      cp_async16(xs + r * lay.XS + pc * 4, xsrc + (long long)r * NJ + pc * 4);
-    }
-    for (int idx = tid; idx < (kScanRows - nrows) * lay.RP; idx += 128)
-      xs[(nrows + idx / lay.RP) * lay.XS + idx % lay.RP] = 0.f;
-    cp_async_commit();
+    if (tid < nrows) prefetch_l2_bulk(a.h + ((long long)(b0 + tid) * a.E + cbase) * kStates, kScanCh * kStates * 4);
   }
   float A2[kStates];
   {
@@ -363,6 +353,27 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
     }
   }
   const float bdt = __ldg(a.b_dt + c), Dc = __ldg(a.d_skip + c);
+  pdl_wait();
+  pdl_trigger();
+  // the states of this thread's four rows
+  float4 hv[4][kStates / 4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int b = min(b0 + rg * 4 + k, a.B - 1);  // rows past the batch re-read the last row
+    const float4 *hp = reinterpret_cast<const float4 *>(a.h + ((long long)b * a.E + c) * kStates);
+#pragma unroll
+    for (int q = 0; q < kStates / 4; ++q) hv[k][q] = hp[q];
+  }
+  {
+    const float *xsrc = a.xdbl + (long long)b0 * NJ;
+    for (int idx = tid; idx < nrows * (NJ / 4); idx += 128) {
+      const int r = idx / (NJ / 4), pc = idx % (NJ / 4);
+      cp_async16(xs + r * lay.XS + pc * 4, xsrc + (long long)r * NJ + pc * 4);
+    }
+    for (int idx = tid; idx < (kScanRows - nrows) * lay.RP; idx += 128)
+      xs[(nrows + idx / lay.RP) * lay.XS + idx % lay.RP] = 0.f;
+    cp_async_commit();
+  }
   const T *u = reinterpret_cast<const T *>(a.u);
   const T *z = reinterpret_cast<const T *>(a.z);
   T ur[4], zr[4];
@@ -419,7 +430,7 @@ template <typename T>
 static hymba_status decode_conv_t(const DecodeSsmArgs &a, cudaStream_t s) {
   constexpr int V = 16 / sizeof(T);
   const long long n = (long long)a.B * (a.E / V);
-  dec_conv_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(a);
+  launch_kernel(dec_conv_kernel<T>, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, a);
   return HYMBA_OK;
 }
 
@@ -442,7 +453,7 @@ static hymba_status decode_scan_t(const DecodeSsmArgs &a, cudaStream_t s) {
     attr_set.mark(dev);
   }
   dim3 grid(a.E / kScanCh, (a.B + kScanRows - 1) / kScanRows);
-  dec_scan_kernel<T><<<grid, 128, smem, s>>>(a);
+  launch_kernel(dec_scan_kernel<T>, grid, dim3(128), (size_t)smem, s, a);
   return HYMBA_OK;
 }
 
@@ -707,6 +718,8 @@ static int scan_chunks(int B, int L, int E) {
   return (int)std::max(1LL, std::min(c, maxc));
 }
 
+int scan_time_chunks(int B, int L, int E) { return scan_chunks(B, L, E); }
+
 size_t scan_workspace_floats(int B, int L, int E, int N, int *chunks_out) {
   const int ch = scan_chunks(B, L, E);
   if (chunks_out) *chunks_out = ch;
@@ -747,6 +760,7 @@ hymba_status selective_scan(const ScanArgs &a, hymba_dtype dt, cudaStream_t s) {
   }
   int chunks = 1;
   scan_workspace_floats(a.B, a.L, a.E, a.N, &chunks);
+  if (a.time_chunks > 0) chunks = std::min(a.time_chunks, std::max(1, a.L));
   const int Tc = (a.L + chunks - 1) / chunks;
   float *hend = nullptr, *hstart = nullptr, *dsum = nullptr;
   if (chunks > 1) {

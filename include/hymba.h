@@ -86,6 +86,18 @@ typedef struct {
                         turned by p * rope_base^(-2i/head_dim_qk) at X~ position p, applied
                         by the input projection (head_dim_qk a power of two).  Layers that
                         share K/V must use the same base. */
+  int branch_chunks; /* the two branches side by side (Fig. 1 and §2.1: the attention and
+                        SSM heads read the same input in parallel; the OpenReview reply on
+                        speed proposes two CUDA streams).  0 or 1: every step of a prefill
+                        runs in order on the caller's stream.  n in 2..8: the prefill splits
+                        the batch into min(n, batch) chunks; each chunk's selective scan runs
+                        on the handle's own low-priority side stream, beside the next chunk's
+                        projections and attention (raised priority), and the caller's stream
+                        waits for it before that chunk's fusion.  The results are the same
+                        bits as the serial order.  The side stream and its events belong to
+                        the handle (created with it, on the device current at creation), so
+                        a handle with n >= 2 takes its prefill calls from one host thread at
+                        a time.  Decode steps are unaffected. */
 } hymba_layer_config;
 
 /* Weights of one layer (device pointers, kept by the handle, never copied).

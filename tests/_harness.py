@@ -40,7 +40,7 @@ class GpuLayer:
     """One layer: seeded weights on the device and its C-ABI handle."""
 
     def __init__(self, w: Workload, layer: int, consumer: bool = False, is_global: bool | None = None,
-                 std=DEFAULT_STD, tag: str = "", device="cuda"):
+                 std=DEFAULT_STD, tag: str = "", device="cuda", branch_chunks: int = 4):
         self.workload = w
         self.is_global = (w.window <= 0) if is_global is None else is_global
         self.consumer = consumer
@@ -50,7 +50,8 @@ class GpuLayer:
         d = w.dims
         self.cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner,
                                   d.d_state, d.d_conv, d.rank, w.n_meta, w.window,
-                                  self.is_global, w.dtype, rope_base=w.rope_base)
+                                  self.is_global, w.dtype, rope_base=w.rope_base,
+                                  branch_chunks=branch_chunks)
         self.handle = hy.hymba_layer_create(self.cfg, hy.make_weights(self.dev))
         self.spec = spec_of(w, self.is_global)
 

@@ -51,6 +51,8 @@ def test_create_validates_configuration():
         (dict(window=0), hy.HYMBA_ERR_INVALID_ARG),
         (dict(head_dim_qk=32), hy.HYMBA_ERR_UNSUPPORTED),     # bf16 attention kernel shape
         (dict(d_conv=5), hy.HYMBA_ERR_UNSUPPORTED),
+        (dict(branch_chunks=-1), hy.HYMBA_ERR_INVALID_ARG),
+        (dict(branch_chunks=9), hy.HYMBA_ERR_INVALID_ARG),
     ]
     for kw, want in bad:
         with pytest.raises(hy.HymbaError) as e:
@@ -356,3 +358,22 @@ def test_block_calls_validate_before_launch():
         assert hy.hymba_block_decode_workspace(p, 5504, 128, 8320) > hy.hymba_layer_decode_workspace(p, 128, 8320)
     finally:
         hy.hymba_layer_destroy(p)
+
+
+def test_branch_chunks_workspace():
+    """The concurrent prefill's chunks share one scan chunk-state region sized for the
+    largest chunk; every chunking of a batch gets a workspace (no device needed)."""
+    sizes = {}
+    for chunks in (0, 1, 2, 3, 8):
+        h = hy.hymba_layer_create(_cfg(branch_chunks=chunks), _fake_weights())
+        try:
+            for batch in (1, 2, 5, 128):
+                sizes[(chunks, batch)] = hy.hymba_layer_prefill_workspace(h, batch, 1000)
+        finally:
+            hy.hymba_layer_destroy(h)
+    for batch in (1, 2, 5, 128):
+        assert sizes[(0, batch)] == sizes[(1, batch)]
+        for chunks in (2, 3, 8):
+            assert sizes[(chunks, batch)] > 0
+    # batch 1 never splits
+    assert len({sizes[(c, 1)] for c in (0, 1, 2, 3, 8)}) == 1
