@@ -138,11 +138,12 @@ class Prefill:
     layers exist twice over the same weights: with the concurrent schedule (the timed step)
     and with the serial one (the per-kernel figures, each kernel alone on the GPU)."""
 
-    def __init__(self, w, dev):
+    def __init__(self, w, dev, branch_chunks=BRANCH_CHUNKS):
         import hybrid_attention_ssm_head_b200 as hy
         import synth
         self.hy = hy
         self.w = w
+        self.branch_chunks = branch_chunks
         d = w.dims
         B, L, n = w.batch, w.seq_rows, w.n_tokens
         self.B, self.L, self.n = B, L, n
@@ -151,7 +152,7 @@ class Prefill:
             wt = {k: v.contiguous() for k, v in
                   synth.configs.layer_weights(w, layer, consumer=consumer, device=dev).items()}
             self.wts.append(wt)
-            for hs, chunks in ((self.handles, BRANCH_CHUNKS), (self.handles_serial, 0)):
+            for hs, chunks in ((self.handles, branch_chunks), (self.handles_serial, 0)):
                 cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner, d.d_state,
                                      d.d_conv, d.rank, w.n_meta, w.window, False, "bf16",
                                      branch_chunks=chunks)
@@ -400,7 +401,7 @@ def run_ours(args, rank, world, dev):
     torch.cuda.set_device(dev)
     w3, w4 = synth.configs.CFG3, synth.configs.CFG4
     t_setup = time.time()
-    pre = Prefill(w3, dev)
+    pre = Prefill(w3, dev, branch_chunks=args.branch_chunks)
     dec = Decode(w4, dev)
     torch.cuda.synchronize()
     setup_s = time.time() - t_setup
@@ -591,7 +592,7 @@ def run_ours(args, rank, world, dev):
         "prefill_ms_per_step": pre_ms / args.steps,
         "prefill_without_meta_cache_ms_per_step": full_ms,
         "prefill_serial_ms_per_step": serial_ms,
-        "branch_chunks": BRANCH_CHUNKS,
+        "branch_chunks": pre.branch_chunks,
         "decode_ms_per_step": dec_ms / args.steps,
         "decode_tok_s": dec_tok_s,
         "prefill_tflops": step_flops * args.steps / (pre_ms / 1e3) / 1e12,
@@ -748,6 +749,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--branch-chunks", type=int, default=BRANCH_CHUNKS,
+                    help="batch chunks of the concurrent prefill (0: serial schedule)")
     ap.add_argument("--case", choices=["headline", "cfg1", "cfg2", "b32", "decode", "decode-b32"], default="headline",
                     help="headline: the benchmark; others: a smaller run for profiling")
     args = ap.parse_args()

@@ -63,7 +63,7 @@ class hymba_block_weights(C.Structure):
 
 class hymba_prefill_layout(C.Structure):
     _fields_ = [(n, C.c_size_t) for n in ("q", "x_ssm", "gate", "u", "xdbl", "delta", "y_ssm",
-                                          "o_attn", "fused", "rope", "total")]
+                                          "o_attn", "fused", "rope", "sched", "total")]
 
 
 class hymba_profile_entry(C.Structure):

@@ -310,6 +310,9 @@ hymba_status hymba_kv_share_bind(hymba_layer *consumer, const hymba_layer *produ
 // ---------------------------------------------------------------------------
 // prefill
 // ---------------------------------------------------------------------------
+// Work counters of the persistent kernels in a prefill's workspace (one per launch).
+constexpr int kSchedCounters = 64;
+
 // Batch chunks of the concurrent prefill: *n chunks of *bc sequences (the last one may be
 // shorter); n = 1 runs the serial order.
 static void branch_split(const hymba_layer_config &c, int batch, int *n, int *bc) {
@@ -350,6 +353,7 @@ static hymba_status prefill_layout_rows(const hymba_layer *layer, int batch, lon
   take(sf * 4);  // scan chunk states, after `fused`
   // rotary table of the positions 0..L-1 (none without a rotary embedding)
   o->rope = take(c.rope_base > 0.f ? (size_t)(rows + c.n_meta) * (c.head_dim_qk / 2) * 8 : 0);
+  o->sched = take(kSchedCounters * sizeof(unsigned));
   o->total = off;
   return HYMBA_OK;
 }
@@ -481,6 +485,12 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
   float *xdbl = reinterpret_cast<float *>(ws + lay.xdbl);
   void *delta = ws + lay.delta, *yssm = ws + lay.y_ssm, *o = ws + lay.o_attn, *f = ws + lay.fused;
   float *scan_ws = reinterpret_cast<float *>(ws + lay.fused + up256((size_t)M * E * es));
+  // work counters of this call's persistent GEMMs, one per launch
+  unsigned *sched = reinterpret_cast<unsigned *>(ws + lay.sched);
+  int next_ctr = 0;
+  auto take_ctr = [&]() -> unsigned * { return next_ctr < kSchedCounters ? sched + next_ctr++ : nullptr; };
+  if (cudaMemsetAsync(sched, 0, kSchedCounters * sizeof(unsigned), stream) != cudaSuccess)
+    FAIL(HYMBA_ERR_CUDA, "cudaMemsetAsync(work counters): %s", cudaGetErrorString(cudaGetLastError()));
 
   // rotary table of positions 0..L-1 (§2.5 RoPE), shared by every sequence
   float2 *rope_tab = nullptr;
@@ -523,6 +533,7 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
       g.epi.seg[0].rope = 1;
       if (!consumer) g.epi.seg[1].rope = 1;
     }
+    g.tile_ctr = take_ctr();
     return gemm(g, c.dtype, s);
   };
   // 2. causal conv + SiLU -> u (and the conv state)
@@ -558,6 +569,7 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
     g.elem = (int)es;
     g.epi.seg[0] = seg(xdbl + m0 * XW, XW, 0, XW, 1, es);
     g.epi.nseg = 1;
+    g.tile_ctr = take_ctr();
     return gemm(g, c.dtype, s);
   };
   // 4. dt_proj + bias + softplus -> delta (tf32 on the tensor cores for the bf16 path)
@@ -577,6 +589,7 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
     g.epi.nseg = 1;
     g.epi.bias = layer->w.b_dt;
     g.epi.act = 1;
+    g.tile_ctr = take_ctr();
     return c.dtype == HYMBA_BF16 ? gemm_tc(g, s) : gemm_simt_f32(g, s);
   };
   // 5. selective scan + D skip, times the gate SiLU(z) -> y_ssm (and the final state)
@@ -661,6 +674,7 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
     g.epi.seg[0].ld_resid = c.d_model;
     g.epi.nseg = 1;
     g.stall = take_debug_stall();
+    g.tile_ctr = take_ctr();
     return gemm(g, c.dtype, s);
   };
 

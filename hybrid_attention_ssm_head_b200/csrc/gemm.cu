@@ -329,15 +329,20 @@ struct TcCfg {
   static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
                                    : (2 * BN <= 256) ? 256 : 512;
   static constexpr uint32_t IDESC = make_idesc(BN, ELEM == 2 ? 1 : 2, 0, 0);
-  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8 + 16;  // + static smem: Epilogue
+  static constexpr int SCHED = 8;  // tile ids in flight from the producer to the MMA and epilogue warps
+  static constexpr int BAR_BYTES = (2 * STAGES + 5 + 2 * SCHED) * 8 + SCHED * 4 + 16;  // + static smem: Epilogue
   static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0, N <= 256");
 };
 
+// Tile order: with a work counter (tile_ctr), the producer takes the next tile with an
+// atomic add and hands its id to the MMA warp and the epilogue warps through a ring of
+// SCHED slots in shared memory (so a CTA that starts late, e.g. behind other kernels'
+// CTAs on its SM, takes fewer tiles); without one, CTA b takes tiles b, b + grid, ...
 template <int BN, int ELEM, int EPI>
 __global__ void __launch_bounds__(576, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   int M, int N, int K, Epilogue epi, long long wlim, int stall) {
+                   int M, int N, int K, Epilogue epi, long long wlim, int stall, unsigned *tile_ctr) {
   pdl_wait();
   pdl_trigger();
   using C = TcCfg<BN, ELEM>;
@@ -350,7 +355,11 @@ __global__ void __launch_bounds__(576, 1)
   uint64_t *tfull = empty + C::STAGES;
   uint64_t *tempty = tfull + 2;
   uint64_t *never = tempty + 2;  // nothing arrives on it: the wait of a stalled MMA warp
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(never + 1);
+  uint64_t *sfull = never + 1;       // [SCHED] a tile id is in the slot
+  uint64_t *sempty = sfull + C::SCHED;  // [SCHED] the MMA warp and the 16 epilogue warps have read it
+  int *stile = reinterpret_cast<int *>(sempty + C::SCHED);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(stile + C::SCHED);
+  const bool dyn = tile_ctr != nullptr;
   // Segment table in shared memory: per-column routing then indexes smem, not
   // kernel parameters.
   __shared__ Epilogue s_epi;
@@ -373,6 +382,10 @@ __global__ void __launch_bounds__(576, 1)
       mbar_init(&tempty[a], 512);
     }
     mbar_init(never, 1);
+    for (int i = 0; i < C::SCHED; ++i) {
+      mbar_init(&sfull[i], 1);
+      mbar_init(&sempty[i], 17);
+    }
     fence_barrier_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
@@ -393,7 +406,23 @@ __global__ void __launch_bounds__(576, 1)
       uint32_t phase = 0;
       uint32_t issued[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       bool ok = true;
-      for (long long u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      int si = 0;
+      uint32_t sph = 0;
+      for (long long u = dyn ? (long long)atomicAdd(tile_ctr, 1u) : blockIdx.x; ok;
+           u = dyn ? (long long)atomicAdd(tile_ctr, 1u) : u + gridDim.x) {
+        if (dyn) {  // publish the tile id (or the end) to the MMA and epilogue warps
+          if (!mbar_wait(&sempty[si], sph ^ 1u, &g_err_gemm, wlim)) {
+            ok = false;
+            break;
+          }
+          stile[si] = u < units ? (int)u : -1;
+          mbar_arrive(&sfull[si]);
+          if (++si == C::SCHED) {
+            si = 0;
+            sph ^= 1u;
+          }
+        }
+        if (u >= units) break;
         const int mt = int(u / n_tiles), nt = int(u % n_tiles);
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, &g_err_gemm, wlim)) {
@@ -426,7 +455,23 @@ __global__ void __launch_bounds__(576, 1)
       // A stalled launch (the bounded-wait test) waits for an arrival that never comes
       // instead of issuing its first MMA; it then takes the abort path below.
       bool ok = !stall || mbar_wait(never, 0, &g_err_gemm, wlim);
-      for (long long u = blockIdx.x; u < units && ok; u += gridDim.x) {
+      int si = 0;
+      uint32_t sph = 0;
+      for (long long u = blockIdx.x; ok; u += gridDim.x) {
+        if (dyn) {
+          if (!mbar_wait(&sfull[si], sph, &g_err_gemm, wlim)) {
+            ok = false;
+            break;
+          }
+          u = stile[si];
+          mbar_arrive(&sempty[si]);
+          if (++si == C::SCHED) {
+            si = 0;
+            sph ^= 1u;
+          }
+          if (u < 0) break;
+        }
+        if (u >= units) break;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, &g_err_gemm, wlim)) {
           ok = false;
           break;
@@ -478,7 +523,21 @@ __global__ void __launch_bounds__(576, 1)
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (long long u = blockIdx.x; u < units; u += gridDim.x) {
+    int si = 0;
+    uint32_t sph = 0;
+    for (long long u = blockIdx.x;; u += gridDim.x) {
+      if (dyn) {
+        if (!mbar_wait(&sfull[si], sph, &g_err_gemm, wlim)) break;
+        u = stile[si];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sempty[si]);
+        if (++si == C::SCHED) {
+          si = 0;
+          sph ^= 1u;
+        }
+        if (u < 0) break;
+      }
+      if (u >= units) break;
       const int mt = int(u / n_tiles), nt = int(u % n_tiles);
       constexpr int NCH = (BN + 63) / 64;
       if (!mbar_wait(&tfull[acc], acc_phase, &g_err_gemm, wlim)) break;
@@ -837,7 +896,7 @@ static hymba_status launch_tc(const GemmArgs &g, cudaStream_t s) {
   const long long tiles = (long long)((g.M + 127) / 128) * ((g.N + BN - 1) / BN);
   const int grid = (int)std::min<long long>(tiles, num_sms());
   launch_kernel(gemm_tc_kernel<BN, ELEM, EPI>, dim3(grid), dim3(576), (size_t)C::SMEM, s, ta, tb, g.M, g.N, g.K,
-                g.epi, wait_limit_cycles(), g.stall);
+                g.epi, wait_limit_cycles(), g.stall, g.tile_ctr);
   note_launch(1);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {

@@ -135,6 +135,9 @@ struct GemmArgs {
   int elem;    // 2: bf16 operands; 4: fp32 operands
   Epilogue epi;
   int stall;   // tensor-core path: the MMA warp waits for an arrival that never comes
+  unsigned *tile_ctr;  // tensor-core path: a zeroed counter -> tiles handed out in the order
+                       // CTAs ask for them (CTAs that start late take fewer); null -> each
+                       // CTA takes every gridDim-th tile
 };
 
 // Tensor-core path (tcgen05 + TMA).  elem 2 -> kind::f16 (bf16), 4 -> kind::tf32.

@@ -190,6 +190,8 @@ typedef struct {
   size_t o_attn;  /* [M, E] attention     dtype */
   size_t fused;   /* [M, E] Eq. 3 inside W_out(.)  dtype */
   size_t rope;    /* [L, d_qk/2] (cos, sin) fp32 pairs of the rotary embedding (if any) */
+  size_t sched;   /* [64] uint32 work counters of the persistent kernels (zeroed by each
+                     prefill; each launch of the call takes one) */
   size_t total;
 } hymba_prefill_layout;
 HYMBA_API hymba_status hymba_layer_prefill_layout(const hymba_layer *layer, int batch, int n_tokens,
