@@ -41,10 +41,12 @@ UNIT = "tok/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one in_proj launch from an ncu capture of the current kernel
 # (dram__bytes_{read,write}.sum of the in_proj launch of `bench.py --case b32`), scaled by
-# rows to one producer launch of the headline prefill (B x n = 1,048,576 real rows); None
-# while the kernel has changed since the last capture.
-IN_PROJ_TRAFFIC = None
-IN_PROJ_TRAFFIC_BASIS = "no capture of the current kernel yet"
+# rows to one producer launch of the headline's concurrent prefill (a batch chunk, 32 x 8192
+# = 262,144 real rows); None while the kernel has changed since the last capture.
+IN_PROJ_TRAFFIC = 5.53e9
+IN_PROJ_TRAFFIC_BASIS = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the in_proj launch of "
+                         "`bench.py --case b32 --branch-chunks 0` (778 MB, 36,864 rows), scaled by rows to one "
+                         "launch of the concurrent prefill (a chunk of 32 sequences x 8192 rows)")
 
 
 def max_over_ranks(vals, device, world: int):
@@ -498,11 +500,19 @@ def run_ours(args, rank, world, dev):
     fl = pre.in_proj_flops()
     achieved = (sum(fl) * args.steps) / (ms_in / 1e3) / 1e12 if ms_in > 0 else None
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    # the same kernel in the serial pass (alone on the GPU, no scan beside it)
+    smap = {n: (c, ms) for n, c, _, ms in sprof}
+    _, ms_alone = smap.get("in_proj", (0, 0.0))
+    alone = (sum(fl) * steps_serial) / (ms_alone / 1e3) / 1e12 if ms_alone > 0 else None
     roof = {"kernel": "in_proj (gemm_tc_kernel<256,bf16>)", "bound": "tensor",
             "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": (achieved / peak) if achieved else None, "traffic": IN_PROJ_TRAFFIC,
             "traffic_basis": IN_PROJ_TRAFFIC_BASIS,
-            "peak_source": f"{peak_src} bf16_tflops_sustained"}
+            "peak_source": f"{peak_src} bf16_tflops_sustained",
+            "timing": "timed region: the concurrent step, the scan of the previous batch chunk "
+                      "running beside this kernel",
+            "alone": {"achieved": alone, "frac": (alone / peak) if alone else None,
+                      "timing": "the serial pass after the timed region"}}
     step_flops = pre.flops()
     dec_bytes = dec.hbm_bytes()
 
@@ -690,6 +700,10 @@ def run_case(args, dev):
             _replace(synth.configs.CFG4, name="decode_b32", batch=32)
         dec = Decode(w4, dev)
         run = lambda: dec.run(stream)  # noqa: E731
+    elif args.case == "prefill":
+        # the headline prefill step alone (both layers, meta caches + real rows)
+        pre = Prefill(synth.configs.CFG3, dev, branch_chunks=args.branch_chunks)
+        run = lambda: pre.run(stream, serial=args.branch_chunks < 2)  # noqa: E731
     else:
         from dataclasses import replace as _replace
         w = {"cfg1": synth.configs.CFG1, "cfg2": synth.configs.CFG2,
@@ -700,7 +714,8 @@ def run_case(args, dev):
         d = w.dims
         wt = {k: v.contiguous() for k, v in synth.configs.layer_weights(w, 0, device=dev).items()}
         cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner, d.d_state,
-                             d.d_conv, d.rank, w.n_meta, w.window, w.window <= 0, "bf16")
+                             d.d_conv, d.rank, w.n_meta, w.window, w.window <= 0, "bf16",
+                             branch_chunks=args.branch_chunks)
         h = hy.hymba_layer_create(cfg, hy.make_weights(wt))
         B, L = w.batch, w.seq_rows
         x = synth.configs.x_tilde(w, device=dev)
@@ -751,7 +766,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--branch-chunks", type=int, default=BRANCH_CHUNKS,
                     help="batch chunks of the concurrent prefill (0: serial schedule)")
-    ap.add_argument("--case", choices=["headline", "cfg1", "cfg2", "b32", "decode", "decode-b32"], default="headline",
+    ap.add_argument("--case", choices=["headline", "prefill", "cfg1", "cfg2", "b32", "decode", "decode-b32"],
+                    default="headline",
                     help="headline: the benchmark; others: a smaller run for profiling")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))

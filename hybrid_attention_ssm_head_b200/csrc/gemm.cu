@@ -208,6 +208,27 @@ __device__ __forceinline__ void epi_bias16(const Epilogue &e, int n0, int N, flo
 template <int EPI>
 __device__ __forceinline__ void epi_store16(const Epilogue &e, long long m, long long mk, int rp, int n0,
                                             int N, const uint32_t (&r)[16], const float (&bias)[16]) {
+  if constexpr ((EPI & kEpiSoftplus) != 0) {
+    // dt_proj: one plain segment, bias and softplus of every column (checked on the host)
+    const EpiSeg &g = e.seg[0];
+    if (n0 + 16 <= N && g.vec_ok && !g.f32) {
+      float o[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) o[i] = softplus_f(__uint_as_float(r[i]) + bias[i]);
+      __nv_bfloat16 *p = reinterpret_cast<__nv_bfloat16 *>(g.ptr) + m * g.ld_row + (n0 - g.col0);
+      if (g.vec32) {
+        st_global_v8(p, pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                     pack_bf16x2(o[6], o[7]), pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]),
+                     pack_bf16x2(o[12], o[13]), pack_bf16x2(o[14], o[15]));
+      } else {
+        st_global_v4(p, pack_bf16x2(o[0], o[1]), pack_bf16x2(o[2], o[3]), pack_bf16x2(o[4], o[5]),
+                     pack_bf16x2(o[6], o[7]));
+        st_global_v4(p + 8, pack_bf16x2(o[8], o[9]), pack_bf16x2(o[10], o[11]), pack_bf16x2(o[12], o[13]),
+                     pack_bf16x2(o[14], o[15]));
+      }
+      return;
+    }
+  }
   float v[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
@@ -557,6 +578,15 @@ __global__ void __launch_bounds__(576, 1)
           const int c = sub * 16 + 64 * (k0 + k);
           if (k0 + k < NCH && c < BN) tmem_ld16(t_row + c, r[k]);  // uniform per warp
         }
+        // the softplus epilogue's bias: its loads overlap the tensor-memory loads
+        float pbias[(EPI & kEpiSoftplus) ? BATCH : 1][16];
+        if constexpr ((EPI & kEpiSoftplus) != 0) {
+#pragma unroll
+          for (int k = 0; k < BATCH; ++k) {
+            const int n0 = nt * BN + sub * 16 + 64 * (k0 + k);
+            if (k0 + k < NCH && n0 < N) epi_bias16(s_epi, n0, N, pbias[k]);
+          }
+        }
         tmem_wait_ld();
         if (k0 + BATCH >= NCH) {
           tc_fence_before();
@@ -567,9 +597,13 @@ __global__ void __launch_bounds__(576, 1)
           const int c = sub * 16 + 64 * (k0 + k);
           const int n0 = nt * BN + c;
           if (k0 + k < NCH && c < BN && n0 < N && m < M) {
-            float bias[16];
-            if (s_epi.bias) epi_bias16(s_epi, n0, N, bias);
-            epi_store16<EPI>(s_epi, m, mk, rp, n0, N, r[k], bias);
+            if constexpr ((EPI & kEpiSoftplus) != 0) {
+              epi_store16<EPI>(s_epi, m, mk, rp, n0, N, r[k], pbias[k]);
+            } else {
+              float bias[16];
+              if (s_epi.bias) epi_bias16(s_epi, n0, N, bias);
+              epi_store16<EPI>(s_epi, m, mk, rp, n0, N, r[k], bias);
+            }
           }
         }
       }
@@ -862,6 +896,9 @@ hymba_status gemm_ws(const GemmArgs &g, cudaStream_t s) {
 // The epilogue features a product needs (kEpi* flags).
 static int epi_flags(const Epilogue &e) {
   int f = 0;
+  if (e.act == 1 && e.bias && e.nseg == 1 && !e.seg[0].f32 && !e.seg[0].act && !e.seg[0].resid &&
+      !e.seg[0].rmap && !e.seg[0].rope && e.seg[0].inner >= e.seg[0].col1 - e.seg[0].col0)
+    f |= kEpiSoftplus;
   if (e.nseg > 1 || e.rmap_rows > 0 || e.rope_tab) f |= kEpiRoute;
   for (int i = 0; i < e.nseg; ++i) {
     if (e.seg[i].rmap || e.seg[i].rope) f |= kEpiRoute;
@@ -911,7 +948,7 @@ hymba_status gemm_tc(const GemmArgs &g, cudaStream_t s) {
   // (decode) so that more CTAs stream the weights.
   const bool small_m = g.M <= 128;
   if (g.elem == 2) {
-    const int f = epi_flags(g.epi);
+    const int f = epi_flags(g.epi) & ~kEpiSoftplus;  // a bf16 softplus takes the generic epilogue
     if (f == kEpiRoute) {  // the input projection
       if (small_m) return launch_tc<64, 2, kEpiRoute>(g, s);
       return launch_tc<256, 2, kEpiRoute>(g, s);
@@ -936,6 +973,9 @@ hymba_status gemm_tc(const GemmArgs &g, cudaStream_t s) {
   }
   if (g.elem == 4) {
     if (small_m) return launch_tc<64, 4, 0>(g, s);
+    // dt_proj (bias + softplus, one plain bf16 segment): 128-wide tiles, two 16-column chunks
+    // per epilogue warp, the bias loaded while the accumulator is read
+    if (epi_flags(g.epi) == kEpiSoftplus && g.N % 128 == 0) return launch_tc<128, 4, kEpiSoftplus>(g, s);
     if (g.N % 160 == 0) return launch_tc<160, 4, 0>(g, s);
     return launch_tc<128, 4, 0>(g, s);
   }

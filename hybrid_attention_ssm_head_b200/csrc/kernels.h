@@ -106,6 +106,7 @@ struct EpiSeg {
 constexpr int kEpiRoute = 1;  // several segments, row remap, rotary embedding
 constexpr int kEpiResid = 2;  // residual add
 constexpr int kEpiGlu = 4;    // gated SiLU of column pairs
+constexpr int kEpiSoftplus = 8;  // bias + softplus into one plain segment (dt_proj)
 
 struct Epilogue {
   EpiSeg seg[5];
