@@ -646,7 +646,7 @@ static int num_sms() {
 //   all four warps   : tensor memory -> shared partial tile; the cluster reduction
 // ---------------------------------------------------------------------------
 namespace wsg {
-constexpr int BM = 128, BK = 64, STAGES = 4;
+constexpr int BM = 128, BK = 64, STAGES = 3;  // 3 stages: 5.43 ms per decode step, 4: 5.49, 2: 5.52
 constexpr int W_BYTES = BM * 128;
 template <int BN>
 struct Cfg {
@@ -717,7 +717,7 @@ __global__ void __launch_bounds__(128, 1)
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer ----------------
     int st = 0;
-    uint32_t ph = 0, issued[STAGES] = {0, 0, 0, 0};
+    uint32_t ph = 0, issued[STAGES] = {};
     bool ok = true;
     for (int kb = kb0; kb < kb1; ++kb) {
       if (kb - kb0 < npre) {  // the weight tile of this (fresh) stage is already on its way
