@@ -312,6 +312,8 @@ hymba_status hymba_kv_share_bind(hymba_layer *consumer, const hymba_layer *produ
 // ---------------------------------------------------------------------------
 // Work counters of the persistent kernels in a prefill's workspace (one per launch).
 constexpr int kSchedCounters = 64;
+// Launch order of the concurrent prefill's main chain (see prefill_run).
+constexpr int kBranchOrder = 0;
 
 // Batch chunks of the concurrent prefill: *n chunks of *bc sequences (the last one may be
 // shorter); n = 1 runs the serial order.
@@ -406,8 +408,9 @@ static hymba_status gemm(const GemmArgs &g, hymba_dtype dt, cudaStream_t s) {
   return gemm_simt_f32(g, s);
 }
 // The decode step's projections: a few activation rows against a whole weight matrix.
+static bool gemm_decode_streams(const GemmArgs &g, hymba_dtype dt) { return dt == HYMBA_BF16 && g.M <= 256; }
 static hymba_status gemm_decode(const GemmArgs &g, hymba_dtype dt, cudaStream_t s) {
-  if (dt == HYMBA_BF16 && g.M <= 256) return gemm_ws(g, s);
+  if (gemm_decode_streams(g, dt)) return gemm_ws(g, s);
   return gemm(g, dt, s);
 }
 
@@ -708,12 +711,19 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
     cudaEvent_t ev_fork = br.ev[0];
     if ((st = check(cudaEventRecord(ev_fork, stream), "cudaEventRecord")) != HYMBA_OK) return st;
     if ((st = check(cudaStreamWaitEvent(br.side, ev_fork, 0), "cudaStreamWaitEvent")) != HYMBA_OK) return st;
+    // kBranchOrder 0: per chunk in_proj .. dt_proj, fork its scan, then its attention;
+    // 1: every chunk's in_proj first; 2: every chunk's attention after all projections
+    if (kBranchOrder == 1) {
+      PrioScope hi(br.prio_hi);
+      for (int k = 0; k < nch; ++k)
+        if ((st = in_proj(k * bc, std::min(bc, batch - k * bc), stream)) != HYMBA_OK) return st;
+    }
     for (int k = 0; k < nch; ++k) {
       const int b0 = k * bc, nb = std::min(bc, batch - b0);
       cudaEvent_t ev_dt = br.ev[1 + 2 * k], ev_scan = br.ev[2 + 2 * k];
       {
         PrioScope hi(br.prio_hi);
-        if ((st = in_proj(b0, nb, stream)) != HYMBA_OK) return st;
+        if (kBranchOrder != 1 && (st = in_proj(b0, nb, stream)) != HYMBA_OK) return st;
         if ((st = conv(b0, nb, stream)) != HYMBA_OK) return st;
         if ((st = x_proj(b0, nb, stream)) != HYMBA_OK) return st;
         if ((st = dt_proj(b0, nb, stream)) != HYMBA_OK) return st;
@@ -722,8 +732,15 @@ static hymba_status prefill_run(hymba_layer *layer, int batch, const PrefillRun 
       if ((st = check(cudaStreamWaitEvent(br.side, ev_dt, 0), "cudaStreamWaitEvent")) != HYMBA_OK) return st;
       if ((st = scan(b0, nb, br.side)) != HYMBA_OK) return st;
       if ((st = check(cudaEventRecord(ev_scan, br.side), "cudaEventRecord")) != HYMBA_OK) return st;
+      if (kBranchOrder != 2) {
+        PrioScope hi(br.prio_hi);
+        if ((st = attention(b0, nb, stream)) != HYMBA_OK) return st;
+      }
+    }
+    if (kBranchOrder == 2) {
       PrioScope hi(br.prio_hi);
-      if ((st = attention(b0, nb, stream)) != HYMBA_OK) return st;
+      for (int k = 0; k < nch; ++k)
+        if ((st = attention(k * bc, std::min(bc, batch - k * bc), stream)) != HYMBA_OK) return st;
     }
     for (int k = 0; k < nch; ++k) {
       const int b0 = k * bc, nb = std::min(bc, batch - b0);
@@ -1025,6 +1042,7 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
   // the step's kernels are launched programmatically: each starts while its predecessor ends
   PdlScope pdl;
 
+  bool xdbl_zeroed = false;
   // 1. input projection; a K/V owner writes this token's K/V straight into its slot
   {
     ProfScope prof_scope(stream, "dec_in_proj");
@@ -1054,9 +1072,15 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
       g.epi.seg[0].rope = 1;
       if (!consumer) g.epi.seg[1].rope = 1;
     }
+    if (gemm_decode_streams(g, c.dtype)) {  // its launch also zeroes the x_proj accumulator
+      g.epi.zero = xdbl;
+      g.epi.zero_n = (long long)batch * xdbl_width(c);
+      xdbl_zeroed = true;
+    }
     if ((st = gemm_decode(g, c.dtype, stream)) != HYMBA_OK) return st;
   }
-  // 2-5. SSM branch: conv + SiLU, x_proj, then dt_proj + softplus + one scan step + gate
+  // 2-5. SSM branch: conv + SiLU and x_proj (partial sums added into xdbl, zeroed by the
+  //      input projection's launch or a memset), then dt_proj + softplus + one scan step + gate
   {
     ProfScope prof_scope(stream, "dec_ssm");
     DecodeSsmArgs a{};
@@ -1068,6 +1092,8 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
     a.conv_w = layer->w.conv_w;
     a.conv_b = layer->w.conv_b;
     a.xdbl = xdbl;
+    a.xdbl_acc = xdbl;
+    a.w_x = layer->w.w_x;
     a.u = u;
     a.w_dt = layer->w.w_dt;
     a.b_dt = layer->w.b_dt;
@@ -1080,19 +1106,10 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
     a.K = c.d_conv;
     a.R = c.dt_rank;
     a.N = c.d_state;
-    if ((st = decode_conv(a, c.dtype, stream)) != HYMBA_OK) return st;
-    GemmArgs g{};
-    g.A = u;
-    g.lda = E;
-    g.B = layer->w.w_x;
-    g.ldb = E;
-    g.M = batch;
-    g.N = xdbl_width(c);
-    g.K = E;
-    g.elem = (int)es;
-    g.epi.seg[0] = seg(xdbl, xdbl_width(c), 0, xdbl_width(c), 1, es);
-    g.epi.nseg = 1;
-    if ((st = gemm_decode(g, c.dtype, stream)) != HYMBA_OK) return st;
+    if (!xdbl_zeroed &&
+        cudaMemsetAsync(xdbl, 0, (size_t)batch * xdbl_width(c) * sizeof(float), stream) != cudaSuccess)
+      FAIL(HYMBA_ERR_CUDA, "cudaMemsetAsync(xdbl): %s", cudaGetErrorString(cudaGetLastError()));
+    if ((st = decode_conv_xproj(a, c.dtype, stream)) != HYMBA_OK) return st;
     if ((st = decode_scan(a, c.dtype, stream)) != HYMBA_OK) return st;
   }
   // 6. single-query attention over the store

@@ -705,6 +705,11 @@ __global__ void __launch_bounds__(128, 1)
   }
   pdl_wait();
   pdl_trigger();
+  if (epi.zero) {  // an accumulator the next kernel adds into
+    const long long nth = (long long)gridDim.x * gridDim.y * blockDim.x;
+    for (long long i = ((long long)blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + tid; i < epi.zero_n; i += nth)
+      epi.zero[i] = 0.f;
+  }
   if (warp == 1) {
     tmem_alloc(tmem_slot, BN);
     tmem_relinquish();

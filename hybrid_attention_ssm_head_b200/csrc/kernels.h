@@ -124,6 +124,8 @@ struct Epilogue {
   int rope_rows, rope_off, rope_hd;
   const float *bias;  // per product column (nullable)
   int act;            // 0 = identity, 1 = softplus
+  float *zero;        // weight-streaming GEMM: zero_n floats set to 0 by the launch (after it
+  long long zero_n;   // has waited for the preceding kernel); for the next kernel's accumulator
 };
 
 // out[m, n] = epi( sum_k A[m, k] * B[n, k] )  (A: [M, K], B: [N, K], row-major)
@@ -277,6 +279,8 @@ struct DecodeSsmArgs {
   void *conv_state;    // [B, K-1, E] in/out
   const float *conv_w, *conv_b;  // [E, K], [E]
   const float *xdbl;   // [B, R + 2N] fp32: delta_r, B, C of the new token
+  float *xdbl_acc;     // the same buffer, zeroed beforehand, accumulated by the conv kernel
+  const void *w_x;     // [R + 2N, E] x_proj weights (dtype)
   void *u;             // [B, E] conv + SiLU output
   const float *w_dt, *b_dt;      // [E, R], [E]
   const float *a_log, *d_skip;   // [E, N], [E]
@@ -284,8 +288,9 @@ struct DecodeSsmArgs {
   void *y;             // [B, E] gated output
   int B, E, K, R, N;
 };
-// u = SiLU(conv(window, x) + b); the conv window advanced in place.
-hymba_status decode_conv(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s);
+// u = SiLU(conv(window, x) + b), the conv window advanced in place, and x_proj:
+// xdbl_acc += u W_x^T (xdbl_acc zeroed beforehand; fp32 atomic adds of per-CTA partials).
+hymba_status decode_conv_xproj(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s);
 // delta = softplus(delta_r W_dt^T + b_dt), one recurrence step, y = (C.h + D u) * gate.
 hymba_status decode_scan(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s);
 

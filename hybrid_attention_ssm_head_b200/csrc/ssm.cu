@@ -228,46 +228,124 @@ hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
-// decode SSM branch: conv + SiLU, then (after the x_proj GEMM) dt_proj + softplus +
-// one recurrence step + gate
+// decode SSM branch: conv + SiLU and x_proj, then dt_proj + softplus + one recurrence
+// step + gate
 // ---------------------------------------------------------------------------
-// (1) One thread per (sequence, 8 channels): u = SiLU(conv(window, x) + b), the window
-//     advanced by one row in conv_state.  16-byte loads and stores.
-template <typename T>
-__global__ void __launch_bounds__(256) dec_conv_kernel(DecodeSsmArgs a) {
-  constexpr int V = 16 / sizeof(T);
-  const int nv = a.E / V;
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+// (1) CTA = 16 sequences x CH channels, 256 threads: u = SiLU(conv(window, x) + b) for its
+//     channels (window advanced in conv_state, u stored), then its share of x_proj,
+//     xdbl[b, j] += sum over its channels of u[b, c] W_x[j, c], added atomically (E / CH
+//     partial sums per output; the buffer is zeroed by the launch before).  The W_x slice
+//     arrives by cp.async while the convolution runs (it is requested before the wait for
+//     the preceding kernel); every global load of the convolution is issued before the
+//     first store.
+constexpr int kDecRows = 16;
+template <typename T, int CH>
+__global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
+  constexpr int ROWB = CH * (int)sizeof(T) + 16;  // padded row of the W_x slice (conflict-free 16-byte reads)
+  constexpr int PIECES = CH * (int)sizeof(T) / 16;
+  constexpr int RPT = kDecRows * CH / 256;         // conv rows per thread
+  extern __shared__ __align__(16) uint8_t dsm_x[];
+  float *us = reinterpret_cast<float *>(dsm_x);    // [CH][kDecRows] u, channel-major (broadcast reads)
+  uint8_t *wxs = dsm_x + CH * kDecRows * 4;        // [NJ][ROWB] W_x slice
+  const int NJ = a.R + 2 * a.N;
+  const int cbase = blockIdx.x * CH;
+  const int b0 = blockIdx.y * kDecRows;
+  const int tid = threadIdx.x;
+  const T *wx = reinterpret_cast<const T *>(a.w_x);
+  for (int idx = tid; idx < NJ * PIECES; idx += 256) {
+    const int j = idx / PIECES, pc = idx % PIECES;
+    cp_async16(wxs + j * ROWB + pc * 16, wx + (long long)j * a.E + cbase + pc * (16 / (int)sizeof(T)));
+  }
+  cp_async_commit();
+  const int K = a.K;
+  const int ch = tid % CH, c = cbase + ch;
+  float w[3];  // taps of the window rows (oldest first); wlast multiplies the new row
+#pragma unroll
+  for (int k = 0; k < 3; ++k) w[k] = k < K - 1 ? __ldg(a.conv_w + c * K + k) : 0.f;
+  const float wlast = __ldg(a.conv_w + c * K + K - 1);
+  const float bias = __ldg(a.conv_b + c);
   pdl_wait();
   pdl_trigger();
-  if (idx >= (long long)a.B * nv) return;
-  const int b = (int)(idx / nv), c0 = (int)(idx % nv) * V;
-  const int K = a.K;
-  T *cs = reinterpret_cast<T *>(a.conv_state) + (long long)b * (K - 1) * a.E + c0;
-  uint4 raw[4];  // window rows (oldest first), then the new row x
+  // conv + SiLU: thread -> channel tid % CH, rows tid / CH + k * (256 / CH).  Every load
+  // is issued unconditionally (rows past the batch read a valid row and are discarded)
+  // and kept raw until all of them are in flight, so their latencies overlap.
+  {
+    T *cs = reinterpret_cast<T *>(a.conv_state);
+    const T *x = reinterpret_cast<const T *>(a.x);
+    T *u = reinterpret_cast<T *>(a.u);
+    T raw[RPT][4];  // window rows oldest first; the new row x last
 #pragma unroll
-  for (int t = 0; t < 3; ++t)
-    raw[t] = t < K - 1 ? *reinterpret_cast<const uint4 *>(cs + (long long)t * a.E) : make_uint4(0, 0, 0, 0);
-  raw[3] = __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const T *>(a.x) + (long long)b * a.ld_x + c0));
-  float xv[4][V];
+    for (int k = 0; k < RPT; ++k) {
+      const int bb = min(b0 + tid / CH + k * (256 / CH), a.B - 1);
+      if (K > 1) {  // uniform: no window rows at all for a one-tap convolution
 #pragma unroll
-  for (int t = 0; t < 4; ++t) unpack16<T>(raw[t], xv[t]);
-  float o[V];
+        for (int t = 0; t < 3; ++t) raw[k][t] = cs[((long long)bb * (K - 1) + min(t, K - 2)) * a.E + c];
+      }
+      raw[k][3] = x[(long long)bb * a.ld_x + c];
+    }
 #pragma unroll
-  for (int i = 0; i < V; ++i) {
-    const float *w = a.conv_w + (long long)(c0 + i) * K;
-    float acc = __ldg(a.conv_b + c0 + i);
+    for (int k = 0; k < RPT; ++k) {
+      const int r = tid / CH + k * (256 / CH), b = b0 + r;
+      float acc = bias;
 #pragma unroll
-    for (int t = 0; t < 3; ++t)
-      if (t < K - 1) acc = fmaf(__ldg(w + t), xv[t][i], acc);
-    acc = fmaf(__ldg(w + K - 1), xv[3][i], acc);
-    o[i] = silu_f(acc);
+      for (int t = 0; t < 3; ++t)
+        if (t < K - 1) acc = fmaf(w[t], Store<T>::to_f(raw[k][t]), acc);
+      acc = fmaf(wlast, Store<T>::to_f(raw[k][3]), acc);
+      float uv = 0.f;
+      if (b < a.B) {
+        uv = silu_f(acc);
+        u[(long long)b * a.E + c] = Store<T>::from_f(uv);
+        // the window advances by one row: rows 1..K-2 move down, x becomes the newest
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+          if (t < K - 1)
+            cs[((long long)b * (K - 1) + t) * a.E + c] = t + 1 < K - 1 ? raw[k][t + 1] : raw[k][3];
+      }
+      us[ch * kDecRows + r] = uv;
+    }
   }
-  store_vec<T>(reinterpret_cast<T *>(a.u) + (long long)b * a.E + c0, o);
-  // the window advances by one row: rows 1..K-2 move down, x becomes the newest
+  cp_async_wait<0>();
+  __syncthreads();
+  // x_proj share: thread -> output column j, all 16 rows, 16-byte reads of the W_x row
+  for (int j = tid; j < NJ; j += 256) {
+    float acc[kDecRows];
 #pragma unroll
-  for (int t = 0; t < 3; ++t)
-    if (t < K - 1) *reinterpret_cast<uint4 *>(cs + (long long)t * a.E) = t + 1 < K - 1 ? raw[t + 1] : raw[3];
+    for (int r = 0; r < kDecRows; ++r) acc[r] = 0.f;
+    const uint8_t *wrow = wxs + j * ROWB;
+#pragma unroll 2
+    for (int pc = 0; pc < PIECES; ++pc) {
+      const uint4 raw = *reinterpret_cast<const uint4 *>(wrow + pc * 16);
+      float wv[16 / sizeof(T)];
+      if constexpr (sizeof(T) == 2) {
+        const uint32_t q[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          wv[2 * i] = bf16_lo(q[i]);
+          wv[2 * i + 1] = bf16_hi(q[i]);
+        }
+      } else {
+        wv[0] = __uint_as_float(raw.x);
+        wv[1] = __uint_as_float(raw.y);
+        wv[2] = __uint_as_float(raw.z);
+        wv[3] = __uint_as_float(raw.w);
+      }
+#pragma unroll
+      for (int i = 0; i < (int)(16 / sizeof(T)); ++i) {
+        const float4 *u4 = reinterpret_cast<const float4 *>(us + (pc * (16 / (int)sizeof(T)) + i) * kDecRows);
+#pragma unroll
+        for (int q = 0; q < kDecRows / 4; ++q) {
+          const float4 v = u4[q];
+          acc[4 * q] = fmaf(v.x, wv[i], acc[4 * q]);
+          acc[4 * q + 1] = fmaf(v.y, wv[i], acc[4 * q + 1]);
+          acc[4 * q + 2] = fmaf(v.z, wv[i], acc[4 * q + 2]);
+          acc[4 * q + 3] = fmaf(v.w, wv[i], acc[4 * q + 3]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kDecRows; ++r)
+      if (b0 + r < a.B) atomicAdd(&a.xdbl_acc[(long long)(b0 + r) * NJ + j], acc[r]);
+  }
 }
 
 // (2) CTA = 16 sequences x 32 channels, 128 threads; thread (channel c, rows 4g..4g+3).
@@ -426,11 +504,27 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
   }
 }
 
-template <typename T>
-static hymba_status decode_conv_t(const DecodeSsmArgs &a, cudaStream_t s) {
-  constexpr int V = 16 / sizeof(T);
-  const long long n = (long long)a.B * (a.E / V);
-  launch_kernel(dec_conv_kernel<T>, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, a);
+template <typename T, int CH>
+static hymba_status decode_conv_xproj_t(const DecodeSsmArgs &a, cudaStream_t s) {
+  const int NJ = a.R + 2 * a.N;
+  const int smem = CH * kDecRows * 4 + NJ * (CH * (int)sizeof(T) + 16);
+  if (smem > 200 * 1024) {
+    set_error("decode SSM: dt_rank %d too large for the conv + x_proj kernel", a.R);
+    return HYMBA_ERR_UNSUPPORTED;
+  }
+  static DeviceOnce attr_set;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_set.done(dev)) {
+    if (cudaFuncSetAttribute(dec_conv_xproj_kernel<T, CH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             200 * 1024) != cudaSuccess) {
+      set_error("cudaFuncSetAttribute(decode conv smem) failed");
+      return HYMBA_ERR_CUDA;
+    }
+    attr_set.mark(dev);
+  }
+  dim3 grid(a.E / CH, (a.B + kDecRows - 1) / kDecRows);
+  launch_kernel(dec_conv_xproj_kernel<T, CH>, grid, dim3(256), (size_t)smem, s, a);
   return HYMBA_OK;
 }
 
@@ -476,12 +570,15 @@ static hymba_status launched(const char *what) {
   return HYMBA_OK;
 }
 
-hymba_status decode_conv(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s) {
+hymba_status decode_conv_xproj(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s) {
   hymba_status st = decode_check(a, dt);
   if (st != HYMBA_OK) return st;
-  st = dt == HYMBA_BF16 ? decode_conv_t<__nv_bfloat16>(a, s) : decode_conv_t<float>(a, s);
+  if (dt == HYMBA_BF16)
+    st = a.E % 128 == 0 ? decode_conv_xproj_t<__nv_bfloat16, 128>(a, s) : decode_conv_xproj_t<__nv_bfloat16, 32>(a, s);
+  else
+    st = a.E % 128 == 0 ? decode_conv_xproj_t<float, 128>(a, s) : decode_conv_xproj_t<float, 32>(a, s);
   if (st != HYMBA_OK) return st;
-  return launched("conv");
+  return launched("conv + x_proj");
 }
 
 hymba_status decode_scan(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s) {

@@ -128,7 +128,7 @@ def test_decode_global_more_runs_than_a_warp():
     lay.close()
 
 
-@pytest.mark.parametrize("batch", [129, 200])
+@pytest.mark.parametrize("batch", [129, 200, 300])
 def test_decode_batch_over_128_rows(batch):
     """More than 128 sequences: the decode projections take 256-row activation tiles."""
     w = synth.configs.Workload(f"edge_dec_b{batch}", DIMS_BF16_SMALL, "bf16", batch, 16, 40, 32)
