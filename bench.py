@@ -259,7 +259,7 @@ def visible_pairs(L, m, W, is_global):
 class Decode:
     """One decode step of the 32-layer stack (one new token per sequence)."""
 
-    def __init__(self, w, dev):
+    def __init__(self, w, dev, branch_chunks=BRANCH_CHUNKS):
         import hybrid_attention_ssm_head_b200 as hy
         import synth
         self.hy = hy
@@ -275,7 +275,8 @@ class Decode:
             wt = {k: v.contiguous() for k, v in
                   synth.configs.layer_weights(w, l, consumer=consumer, device=dev).items()}
             cfg = hy.make_config(d.d_model, d.n_heads, d.n_kv_heads, d.head_dim_qk, d.d_inner, d.d_state,
-                                 d.d_conv, d.rank, w.n_meta, w.window, is_global, "bf16")
+                                 d.d_conv, d.rank, w.n_meta, w.window, is_global, "bf16",
+                                 branch_chunks=branch_chunks)
             h = hy.hymba_layer_create(cfg, hy.make_weights(wt))
             cap = self.pos + 1 if is_global else w.n_meta + w.window
             caches = synth.configs.decode_caches(w, l, cap, consumer, device=dev)
@@ -404,7 +405,10 @@ def run_ours(args, rank, world, dev):
     w3, w4 = synth.configs.CFG3, synth.configs.CFG4
     t_setup = time.time()
     pre = Prefill(w3, dev, branch_chunks=args.branch_chunks)
-    dec = Decode(w4, dev)
+    # the decode stack in the serial order: the side-by-side decode measured the same step
+    # time (5.057 against 5.059 ms), and the serial one gives per-kernel events that are not
+    # stretched by the other branch's kernels running beside them
+    dec = Decode(w4, dev, branch_chunks=0)
     torch.cuda.synchronize()
     setup_s = time.time() - t_setup
     stream = torch.cuda.current_stream()
@@ -698,7 +702,7 @@ def run_case(args, dev):
         from dataclasses import replace as _replace
         w4 = synth.configs.CFG4 if args.case == "decode" else \
             _replace(synth.configs.CFG4, name="decode_b32", batch=32)
-        dec = Decode(w4, dev)
+        dec = Decode(w4, dev, branch_chunks=args.branch_chunks)
         run = lambda: dec.run(stream)  # noqa: E731
     elif args.case == "prefill":
         # the headline prefill step alone (both layers, meta caches + real rows)

@@ -946,7 +946,7 @@ hymba_status hymba_layer_prefill_cached(hymba_layer *layer, int batch, int n_tok
 // decode
 // ---------------------------------------------------------------------------
 struct DecodeLayout {
-  size_t q, x_ssm, z, u, xdbl, y_ssm, o, f, part, rope, total;
+  size_t q, x_ssm, z, u, xacc, y_ssm, o, f, part, rope, total;
 };
 
 static DecodeLayout decode_layout(const hymba_layer_config &c, int batch, long long pos) {
@@ -962,7 +962,7 @@ static DecodeLayout decode_layout(const hymba_layer_config &c, int batch, long l
   d.x_ssm = take(B * E * es);
   d.z = take(B * E * es);
   d.u = take(B * E * es);
-  d.xdbl = take(B * xdbl_width(c) * 4);
+  d.xacc = take(B * xdbl_width(c) * 8 + B * 4);  // x_proj result as 64-bit fixed point, then [B] flags
   d.y_ssm = take(B * E * es);
   d.o = take(B * E * es);
   d.f = take(B * E * es);
@@ -1020,7 +1020,7 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
   const int E = c.d_inner;
   char *ws = reinterpret_cast<char *>(workspace);
   void *q = ws + d.q, *xs = ws + d.x_ssm, *z = ws + d.z, *u = ws + d.u;
-  float *xdbl = reinterpret_cast<float *>(ws + d.xdbl);
+  long long *xacc = reinterpret_cast<long long *>(ws + d.xacc);
   void *yssm = ws + d.y_ssm, *o = ws + d.o, *f = ws + d.f;
   float *part = reinterpret_cast<float *>(ws + d.part);
   hymba_status st;
@@ -1029,7 +1029,9 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
   // the step's kernels are launched programmatically: each starts while its predecessor ends
   PdlScope pdl;
 
-  bool xdbl_zeroed = false;
+  const long long xacc_n = (long long)batch * xdbl_width(c);
+  unsigned *xbad = reinterpret_cast<unsigned *>(xacc + xacc_n);
+  bool xacc_zeroed = false;
   // 1. input projection; a K/V owner writes this token's K/V straight into its slot
   {
     ProfScope prof_scope(stream, "dec_in_proj");
@@ -1060,16 +1062,27 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
       if (!consumer) g.epi.seg[1].rope = 1;
     }
     if (gemm_decode_streams(g, c.dtype)) {  // its launch also zeroes the x_proj accumulator
-      g.epi.zero = xdbl;
-      g.epi.zero_n = (long long)batch * xdbl_width(c);
-      xdbl_zeroed = true;
+      g.epi.zero = reinterpret_cast<float *>(xacc);
+      g.epi.zero_n = 2 * xacc_n + batch;  // the 64-bit sums (pairs of zero words), then the flags
+      xacc_zeroed = true;
     }
     if ((st = gemm_decode(g, c.dtype, stream)) != HYMBA_OK) return st;
   }
-  // 2-5. SSM branch: conv + SiLU and x_proj (partial sums added into xdbl, zeroed by the
-  //      input projection's launch or a memset), then dt_proj + softplus + one scan step + gate
+  // The two branches side by side when the handle has a side stream (branch_chunks >= 2):
+  // the SSM branch there, at the highest priority (short launches), beside the attention.
+  BranchStreams &br = layer->br;
+  const bool side_by_side = c.branch_chunks >= 2 && br.ready;
+  cudaStream_t ssm_stream = side_by_side ? br.side : stream;
+  if (side_by_side) {
+    if (cudaEventRecord(br.ev[0], stream) != cudaSuccess || cudaStreamWaitEvent(br.side, br.ev[0], 0) != cudaSuccess)
+      FAIL(HYMBA_ERR_CUDA, "decode fork: %s", cudaGetErrorString(cudaGetLastError()));
+  }
+  // 2-5. SSM branch: conv + SiLU and x_proj (per-CTA shares added as fixed-point integers
+  //      into an accumulator zeroed by the input projection's launch or a memset), then
+  //      dt_proj + softplus + one scan step + gate
   {
-    ProfScope prof_scope(stream, "dec_ssm");
+    ProfScope prof_scope(ssm_stream, "dec_ssm");
+    PrioScope prio(side_by_side ? br.prio_hi : 0);
     DecodeSsmArgs a{};
     a.x = xs;
     a.ld_x = E;
@@ -1078,8 +1091,8 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
     a.conv_state = ssm_cache->conv;
     a.conv_w = layer->w.conv_w;
     a.conv_b = layer->w.conv_b;
-    a.xdbl = xdbl;
-    a.xdbl_acc = xdbl;
+    a.xacc = xacc;
+    a.xbad = xbad;
     a.w_x = layer->w.w_x;
     a.u = u;
     a.w_dt = layer->w.w_dt;
@@ -1093,12 +1106,14 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
     a.K = c.d_conv;
     a.R = c.dt_rank;
     a.N = c.d_state;
-    if (!xdbl_zeroed &&
-        cudaMemsetAsync(xdbl, 0, (size_t)batch * xdbl_width(c) * sizeof(float), stream) != cudaSuccess)
-      FAIL(HYMBA_ERR_CUDA, "cudaMemsetAsync(xdbl): %s", cudaGetErrorString(cudaGetLastError()));
-    if ((st = decode_conv_xproj(a, c.dtype, stream)) != HYMBA_OK) return st;
-    if ((st = decode_scan(a, c.dtype, stream)) != HYMBA_OK) return st;
+    if (!xacc_zeroed &&
+        cudaMemsetAsync(xacc, 0, (size_t)xacc_n * sizeof(long long) + (size_t)batch * 4, ssm_stream) != cudaSuccess)
+      FAIL(HYMBA_ERR_CUDA, "cudaMemsetAsync(x_proj accumulator): %s", cudaGetErrorString(cudaGetLastError()));
+    if ((st = decode_conv_xproj(a, c.dtype, ssm_stream)) != HYMBA_OK) return st;
+    if ((st = decode_scan(a, c.dtype, ssm_stream)) != HYMBA_OK) return st;
   }
+  if (side_by_side && cudaEventRecord(br.ev[1], br.side) != cudaSuccess)
+    FAIL(HYMBA_ERR_CUDA, "decode join: %s", cudaGetErrorString(cudaGetLastError()));
   // 6. single-query attention over the store
   int fuse_nchunks = 0;
   long long fuse_per = 1;
@@ -1128,6 +1143,8 @@ static hymba_status decode_run(hymba_layer *layer, int batch, int64_t pos, const
     fuse_nchunks = a.nchunks_out;
     fuse_per = a.per_out;
   }
+  if (side_by_side && cudaStreamWaitEvent(stream, br.ev[1], 0) != cudaSuccess)
+    FAIL(HYMBA_ERR_CUDA, "decode join: %s", cudaGetErrorString(cudaGetLastError()));
   // 7. norm, beta, mean
   if (fuse_nchunks > 0) {
     ProfScope prof_scope(stream, "dec_fuse");

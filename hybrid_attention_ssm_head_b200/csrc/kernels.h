@@ -278,8 +278,11 @@ struct DecodeSsmArgs {
   long long ld_z;
   void *conv_state;    // [B, K-1, E] in/out
   const float *conv_w, *conv_b;  // [E, K], [E]
-  const float *xdbl;   // [B, R + 2N] fp32: delta_r, B, C of the new token
-  float *xdbl_acc;     // the same buffer, zeroed beforehand, accumulated by the conv kernel
+  long long *xacc;     // [B, R + 2N] delta_r, B, C of the new token as fixed-point integers
+                       // (value * 2^32), zeroed beforehand, summed by the conv kernel's
+                       // integer atomic adds (the same bits whatever the order)
+  unsigned *xbad;      // [B] zeroed beforehand: set where a share was not finite or
+                       // |share| >= 2^31 (that row's delta_r, B, C are then NaN)
   const void *w_x;     // [R + 2N, E] x_proj weights (dtype)
   void *u;             // [B, E] conv + SiLU output
   const float *w_dt, *b_dt;      // [E, R], [E]
@@ -289,7 +292,7 @@ struct DecodeSsmArgs {
   int B, E, K, R, N;
 };
 // u = SiLU(conv(window, x) + b), the conv window advanced in place, and x_proj:
-// xdbl_acc += u W_x^T (xdbl_acc zeroed beforehand; fp32 atomic adds of per-CTA partials).
+// xacc += u W_x^T per channel block, in fixed point (xacc zeroed beforehand).
 hymba_status decode_conv_xproj(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s);
 // delta = softplus(delta_r W_dt^T + b_dt), one recurrence step, y = (C.h + D u) * gate.
 hymba_status decode_scan(const DecodeSsmArgs &a, hymba_dtype dt, cudaStream_t s);

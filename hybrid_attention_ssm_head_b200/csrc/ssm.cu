@@ -232,13 +232,17 @@ hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s) {
 // step + gate
 // ---------------------------------------------------------------------------
 // (1) CTA = 16 sequences x CH channels, 256 threads: u = SiLU(conv(window, x) + b) for its
-//     channels (window advanced in conv_state, u stored), then its share of x_proj,
-//     xdbl[b, j] += sum over its channels of u[b, c] W_x[j, c], added atomically (E / CH
-//     partial sums per output; the buffer is zeroed by the launch before).  The W_x slice
-//     arrives by cp.async while the convolution runs (it is requested before the wait for
-//     the preceding kernel); every global load of the convolution is issued before the
-//     first store.
+//     channels (window advanced in conv_state, u stored), then its share of x_proj, the
+//     sums over its channels of u[b, c] W_x[j, c], added into xacc as 64-bit fixed-point
+//     integers (value * 2^32, rounded): integer addition is associative, so the sum of the
+//     E / CH shares has the same bits whichever CTA adds first (|value| < 2^31; the
+//     rounding, 2^-33 per share, is far below the fp32 rounding of the share itself for
+//     any value above 2^-9).  The W_x slice arrives by cp.async while the convolution runs
+//     (it is requested before the wait for the preceding kernel); every global load of the
+//     convolution is issued before the first store.
 constexpr int kDecRows = 16;
+constexpr float kXprojFix = 4294967296.0f;       // 2^32
+constexpr float kXprojUnfix = 2.3283064365386963e-10f;  // 2^-32
 template <typename T, int CH>
 __global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
   constexpr int ROWB = CH * (int)sizeof(T) + 16;  // padded row of the W_x slice (conflict-free 16-byte reads)
@@ -344,7 +348,13 @@ __global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
     }
 #pragma unroll
     for (int r = 0; r < kDecRows; ++r)
-      if (b0 + r < a.B) atomicAdd(&a.xdbl_acc[(long long)(b0 + r) * NJ + j], acc[r]);
+      if (b0 + r < a.B) {
+        if (fabsf(acc[r]) < 2147483648.0f)  // false for NaN too
+          atomicAdd(reinterpret_cast<unsigned long long *>(a.xacc + (long long)(b0 + r) * NJ + j),
+                    (unsigned long long)__float2ll_rn(acc[r] * kXprojFix));
+        else
+          atomicOr(a.xbad + b0 + r, 1u);
+      }
   }
 }
 
@@ -443,10 +453,14 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
     for (int q = 0; q < kStates / 4; ++q) hv[k][q] = hp[q];
   }
   {
-    const float *xsrc = a.xdbl + (long long)b0 * NJ;
-    for (int idx = tid; idx < nrows * (NJ / 4); idx += 128) {
-      const int r = idx / (NJ / 4), pc = idx % (NJ / 4);
-      cp_async16(xs + r * lay.XS + pc * 4, xsrc + (long long)r * NJ + pc * 4);
+    // delta_r, B, C of the rows: fixed-point sums of the conv kernel's x_proj shares
+    const longlong2 *xsrc = reinterpret_cast<const longlong2 *>(a.xacc + (long long)b0 * NJ);
+    for (int idx = tid; idx < nrows * (NJ / 2); idx += 128) {
+      const int r = idx / (NJ / 2), pc = idx % (NJ / 2);
+      const longlong2 v = xsrc[(long long)r * (NJ / 2) + pc];
+      float2 f = make_float2(__ll2float_rn(v.x) * kXprojUnfix, __ll2float_rn(v.y) * kXprojUnfix);
+      if (a.xbad[b0 + r]) f = make_float2(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+      *reinterpret_cast<float2 *>(xs + r * lay.XS + 2 * pc) = f;
     }
     for (int idx = tid; idx < (kScanRows - nrows) * lay.RP; idx += 128)
       xs[(nrows + idx / lay.RP) * lay.XS + idx % lay.RP] = 0.f;

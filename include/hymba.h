@@ -96,8 +96,9 @@ typedef struct {
                         waits for it before that chunk's fusion.  The results are the same
                         bits as the serial order.  The side stream and its events belong to
                         the handle (created with it, on the device current at creation), so
-                        a handle with n >= 2 takes its prefill calls from one host thread at
-                        a time.  Decode steps are unaffected. */
+                        a handle with n >= 2 takes its prefill and decode calls from one host
+                        thread at a time.  A decode step of such a handle runs its SSM branch
+                        on the side stream beside the attention (same bits as in order). */
 } hymba_layer_config;
 
 /* Weights of one layer (device pointers, kept by the handle, never copied).

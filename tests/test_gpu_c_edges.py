@@ -105,6 +105,33 @@ def test_nan_inputs_propagate_without_fault():
     lay.close()
 
 
+def test_decode_nan_row_stays_in_its_row():
+    """A NaN in one sequence's new row reaches that sequence's decode output and SSM state
+    (the x_proj shares are summed as fixed-point integers, which hold no NaN: the row is
+    flagged and its delta_r, B, C become NaN), and the other sequences match the oracle."""
+    w = synth.configs.Workload("edge_dec_nan", DIMS_BF16_SMALL, "bf16", 3, 16, 60, 32)
+    lay = H.GpuLayer(w, 0)
+    pos = w.n_meta + w.n_tokens
+    cap = w.n_meta + w.window
+    c = {k: t.contiguous() for k, t in synth.configs.decode_caches(w, 0, cap, False, device="cuda").items()}
+    kvc = hy.hymba_kv_cache(c["k"].data_ptr(), c["v"].data_ptr(), w.batch, cap, 0)
+    ssm = hy.hymba_ssm_cache(c["ssm"].data_ptr(), c["conv"].data_ptr())
+    dws = H.workspace(hy.hymba_layer_decode_workspace(lay.handle, w.batch, pos))
+    xt = synth.gen.normal_tensor((w.batch, w.dims.d_model), 0, "edge_dec_nan/x", device="cuda").to(torch.bfloat16)
+    xt[1, 7] = float("nan")
+    yt = torch.empty_like(xt)
+    hy.hymba_layer_decode_step(lay.handle, w.batch, pos, xt, yt, kvc, ssm, dws, dws.numel(),
+                               torch.cuda.current_stream())
+    hy.hymba_stream_status(torch.cuda.current_stream())
+    assert torch.isnan(yt[1]).all()
+    assert torch.isnan(c["ssm"][1]).any()
+    for b in (0, 2):
+        cache = {k: H.to64(t) for k, t in synth.configs.decode_caches(w, 0, cap, False, batch_index=b).items()}
+        yo, _ = O.layer_decode(H.to64(xt[b]), pos, H.oracle_weights(lay.cpu), lay.spec, cache)
+        H.close_bf16(H.to64(yt[b]), yo, f"decode y, clean sequence {b}")
+    lay.close()
+
+
 def test_decode_global_more_runs_than_a_warp():
     """Batch 1 on a long global layer: few (sequence, kv head, chunk) items, so every chunk
     of the store becomes its own run of the persistent decode attention (35 runs per head),

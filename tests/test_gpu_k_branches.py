@@ -135,3 +135,31 @@ def test_concurrent_prefill_captured_in_a_graph():
     assert torch.equal(h, eager["h"]) and torch.equal(conv, eager["conv"])
     del g
     lay.close()
+
+
+@pytest.mark.parametrize("glob", [False, True])
+def test_decode_side_by_side_equals_serial_bitwise(glob):
+    """With a side stream the decode step runs its SSM branch there, beside the attention:
+    the same kernels on the same inputs, so the same bits as the serial order."""
+    w = Workload(f"branch_dec_{glob}", DIMS_SMALL_BF16, "bf16", 6, 128, 200, 0 if glob else 64)
+    d = w.dims
+    pos = w.seq_rows
+    cap = pos + 4 if glob else w.n_meta + w.window
+    x_new = synth.gen.normal_tensor((w.batch, d.d_model), 0, f"{w.name}/xnew", device="cuda").to(torch.bfloat16)
+    outs = []
+    for chunks in (0, 4):
+        lay = H.GpuLayer(w, 0, is_global=glob, branch_chunks=chunks)
+        c = {k: v.cuda().contiguous() for k, v in synth.configs.decode_caches(w, 0, cap, False).items()}
+        kvc = hy.hymba_kv_cache(c["k"].data_ptr(), c["v"].data_ptr(), w.batch, cap, 0)
+        ssm = hy.hymba_ssm_cache(c["ssm"].data_ptr(), c["conv"].data_ptr())
+        ws = H.workspace(hy.hymba_layer_decode_workspace(lay.handle, w.batch, pos))
+        ys = []
+        for step in range(3):  # three tokens: the caches carry each step into the next
+            y = torch.empty_like(x_new)
+            hy.hymba_layer_decode_step(lay.handle, w.batch, pos + step, x_new, y, kvc, ssm, ws, ws.numel(),
+                                       torch.cuda.current_stream())
+            ys.append(y)
+        hy.hymba_stream_status(torch.cuda.current_stream())
+        outs.append(dict(y=torch.stack(ys), k=c["k"], v=c["v"], h=c["ssm"], conv=c["conv"]))
+        lay.close()
+    _equal(outs[0], outs[1], "decode")
