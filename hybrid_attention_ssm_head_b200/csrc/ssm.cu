@@ -45,68 +45,49 @@ __device__ __forceinline__ float2 decay2(float2 x) {
 // ---------------------------------------------------------------------------
 // causal conv + SiLU (prefill)
 // ---------------------------------------------------------------------------
-template <typename T>
-struct Vec16 {
-  static constexpr int N = 16 / sizeof(T);
-};
-
-template <typename T>
-__device__ __forceinline__ void load_vec(const T *p, float (&v)[Vec16<T>::N]) {
-  uint4 raw = *reinterpret_cast<const uint4 *>(p);
-  if constexpr (sizeof(T) == 2) {
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = __low2float(h[i]);
-      v[2 * i + 1] = __high2float(h[i]);
-    }
-  } else {
-    const float *f = reinterpret_cast<const float *>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = f[i];
-  }
-}
-template <typename T>
-__device__ __forceinline__ void store_vec(T *p, const float (&v)[Vec16<T>::N]) {
-  uint4 raw;
-  if constexpr (sizeof(T) == 2) {
-    uint32_t *w = reinterpret_cast<uint32_t *>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-  } else {
-    float *f = reinterpret_cast<float *>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) f[i] = v[i];
-  }
-  *reinterpret_cast<uint4 *>(p) = raw;
-}
-
 constexpr int kConvTB = 16;
 
+// Four channels of one row as one vector load/store: 8 bytes of bf16, 16 of fp32.
 template <typename T>
-__device__ __forceinline__ void unpack16(const uint4 &raw, float (&v)[16 / sizeof(T)]) {
-  if constexpr (sizeof(T) == 2) {
-    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[2 * i] = bf16_lo(w[i]);
-      v[2 * i + 1] = bf16_hi(w[i]);
-    }
-  } else {
-    const float *f = reinterpret_cast<const float *>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) v[i] = f[i];
+struct ConvVec;
+template <>
+struct ConvVec<__nv_bfloat16> {
+  using R = uint2;
+  static __device__ __forceinline__ void unpack(const R &r, float (&v)[4]) {
+    v[0] = bf16_lo(r.x);
+    v[1] = bf16_hi(r.x);
+    v[2] = bf16_lo(r.y);
+    v[3] = bf16_hi(r.y);
   }
-}
+  static __device__ __forceinline__ R pack(const float (&v)[4]) {
+    return make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+  }
+};
+template <>
+struct ConvVec<float> {
+  using R = uint4;
+  static __device__ __forceinline__ void unpack(const R &r, float (&v)[4]) {
+    v[0] = __uint_as_float(r.x);
+    v[1] = __uint_as_float(r.y);
+    v[2] = __uint_as_float(r.z);
+    v[3] = __uint_as_float(r.w);
+  }
+  static __device__ __forceinline__ R pack(const float (&v)[4]) {
+    return make_uint4(__float_as_uint(v[0]), __float_as_uint(v[1]), __float_as_uint(v[2]), __float_as_uint(v[3]));
+  }
+};
 
-// One thread: VEC channels x kConvTB rows.  Its kConvTB + 3 input rows are loaded
-// up front as 16-byte vectors (coalesced across the warp); the taps (one 16-byte
-// vector per channel) and the bias are fetched once for all kConvTB rows.
+// One thread: 4 channels x kConvTB rows.  Its kConvTB + 3 input rows are loaded up front
+// as vectors (coalesced across the warp); the taps (one float4 per channel) and the bias
+// are fetched once for all kConvTB rows.  Four channels per thread (not eight) keep the
+// thread near 80 registers, so that enough warps are resident to cover the loads.
 template <typename T>
 __global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
   pdl_wait();
   pdl_trigger();
-  constexpr int V = Vec16<T>::N;
+  using CV = ConvVec<T>;
+  using R = typename CV::R;
+  constexpr int V = 4;
   constexpr int NR = kConvTB + 3;
   const int nvec = a.E / V;
   const int tblocks = (a.L + kConvTB - 1) / kConvTB;
@@ -122,11 +103,11 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
   T *u = reinterpret_cast<T *>(a.u);
   const int t0 = tb * kConvTB;
   static_assert(kConvTB >= 3, "the history rows must fall in the first block");
-  uint4 raw[NR];  // raw[r] = x[t0 - 3 + r]: the history rows before row 0, zero past the end
+  R raw[NR];  // raw[r] = x[t0 - 3 + r]: the history rows before row 0, zero past the end
 #pragma unroll
   for (int r = 0; r < NR; ++r) {  // unconditional loads (clamped row), replaced afterwards
     const int t = min(max(t0 - 3 + r, 0), a.L - 1);
-    raw[r] = __ldg(reinterpret_cast<const uint4 *>(x + ((long long)b * a.L + t) * a.ld_x + c0));
+    raw[r] = __ldg(reinterpret_cast<const R *>(x + ((long long)b * a.L + t) * a.ld_x + c0));
   }
 #pragma unroll
   for (int r = 0; r < 3; ++r) {  // rows before 0 exist only in the first block
@@ -134,16 +115,15 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
     if (t < 0) {
       const int hr = K - 1 + t;  // history row (oldest first); taps past K are zero
       raw[r] = (a.hist && hr >= 0)
-                   ? __ldg(reinterpret_cast<const uint4 *>(reinterpret_cast<const T *>(a.hist) +
-                                                           (long long)hr * a.E + c0))
-                   : make_uint4(0, 0, 0, 0);
+                   ? __ldg(reinterpret_cast<const R *>(reinterpret_cast<const T *>(a.hist) + (long long)hr * a.E + c0))
+                   : R{};
     }
   }
 #pragma unroll
   for (int r = 3; r < NR; ++r)
-    if (t0 - 3 + r >= a.L) raw[r] = make_uint4(0, 0, 0, 0);
+    if (t0 - 3 + r >= a.L) raw[r] = R{};
   // wj[j][i] multiplies x[t - 3 + j] for channel c0 + i (taps right-aligned)
-  float wj[4][V], bias[V];
+  float wj[4][V];
   if (K == 4) {
 #pragma unroll
     for (int i = 0; i < V; ++i) {
@@ -162,24 +142,18 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
         wj[j][i] = k >= 0 ? __ldg(a.w + (c0 + i) * K + k) : 0.f;
       }
   }
-#pragma unroll
-  for (int i = 0; i < V; i += 4) {
-    const float4 b4 = __ldg(reinterpret_cast<const float4 *>(a.bias + c0 + i));
-    bias[i] = b4.x;
-    bias[i + 1] = b4.y;
-    bias[i + 2] = b4.z;
-    bias[i + 3] = b4.w;
-  }
+  const float4 b4 = __ldg(reinterpret_cast<const float4 *>(a.bias + c0));
+  const float bias[V] = {b4.x, b4.y, b4.z, b4.w};
   float xv[4][V];  // rolling window of converted rows t-3 .. t
 #pragma unroll
-  for (int j = 0; j < 3; ++j) unpack16<T>(raw[j], xv[j + 1]);
+  for (int j = 0; j < 3; ++j) CV::unpack(raw[j], xv[j + 1]);
 #pragma unroll
   for (int tt = 0; tt < kConvTB; ++tt) {
 #pragma unroll
     for (int j = 0; j < 3; ++j)
 #pragma unroll
       for (int i = 0; i < V; ++i) xv[j][i] = xv[j + 1][i];
-    unpack16<T>(raw[tt + 3], xv[3]);
+    CV::unpack(raw[tt + 3], xv[3]);
     const int t = t0 + tt;
     if (t < a.L) {
       float o[V];
@@ -190,28 +164,24 @@ __global__ void __launch_bounds__(128) conv_silu_kernel(ConvArgs a) {
         for (int j = 0; j < 4; ++j) acc = fmaf(wj[j][i], xv[j][i], acc);
         o[i] = silu_f(acc);
       }
-      store_vec<T>(u + ((long long)b * a.L + t) * a.E + c0, o);
+      *reinterpret_cast<R *>(u + ((long long)b * a.L + t) * a.E + c0) = CV::pack(o);
     }
   }
   if (a.conv_state && t0 + kConvTB >= a.L) {
-    // the last K-1 rows of x, oldest first: x[L-K+1+r] = raw[L-K+4+r-t0]
+    // the last K-1 rows of x, oldest first: x[L-K+1+r] = raw[L-K+4+r-t0] (copied as they are)
     T *cs = reinterpret_cast<T *>(a.conv_state);
     const int base = a.L - K + 4 - t0;
 #pragma unroll
     for (int rr = 0; rr < NR; ++rr) {
       const int r = rr - base;
-      if (r >= 0 && r < K - 1) {
-        float v[V];
-        unpack16<T>(raw[rr], v);
-        store_vec<T>(cs + ((long long)b * (K - 1) + r) * a.E + c0, v);
-      }
+      if (r >= 0 && r < K - 1) *reinterpret_cast<R *>(cs + ((long long)b * (K - 1) + r) * a.E + c0) = raw[rr];
     }
   }
 }
 
 hymba_status conv_silu(const ConvArgs &a, hymba_dtype dt, cudaStream_t s) {
-  const int V = dt == HYMBA_BF16 ? 8 : 4;
-  const long long n = (long long)a.B * ((a.L + kConvTB - 1) / kConvTB) * (a.E / V);
+  (void)dt;
+  const long long n = (long long)a.B * ((a.L + kConvTB - 1) / kConvTB) * (a.E / 4);
   if (n == 0) return HYMBA_OK;
   const unsigned blocks = (unsigned)((n + 127) / 128);
   if (dt == HYMBA_BF16)
