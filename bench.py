@@ -107,7 +107,7 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.thread.join(timeout=2)
-        sm, mx, reasons = [], [], set()
+        sm, mx, pw, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             parts = [p.strip() for p in ln.split(",")]
@@ -118,13 +118,17 @@ class ClockSampler:
                 mx.append(float(parts[2]))
             except ValueError:
                 continue
+            try:
+                pw.append(float(parts[3]))
+            except ValueError:
+                pass
             for nm, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
                     reasons.add(nm)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "power_w": statistics.median(pw) if pw else None}
 
 
 # ---------------------------------------------------------------------------------------------
@@ -450,6 +454,10 @@ def run_ours(args, rank, world, dev):
     steps_serial = max(1, min(args.steps, 3))
     pre.run(stream, serial=True)
     torch.cuda.synchronize()
+    sampler_s = ClockSampler(torch.cuda.current_device())
+    if rank == 0:
+        sampler_s.start()
+        time.sleep(0.3)
     hy.hymba_profile_enable(True)
     hy.hymba_profile_collect()
     es0, es1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -460,6 +468,7 @@ def run_ours(args, rank, world, dev):
     torch.cuda.synchronize()
     sprof = hy.hymba_profile_collect()
     hy.hymba_profile_enable(False)
+    clocks_serial = sampler_s.stop() if rank == 0 else None
     serial_ms = max_over_ranks([es0.elapsed_time(es1) / steps_serial], dev, world)[0]
     # for comparison: the same two layers without the meta cache (every sequence's m + n rows)
     steps_full = max(1, min(args.steps, 3))
@@ -606,6 +615,7 @@ def run_ours(args, rank, world, dev):
         "prefill_ms_per_step": pre_ms / args.steps,
         "prefill_without_meta_cache_ms_per_step": full_ms,
         "prefill_serial_ms_per_step": serial_ms,
+        "clocks_serial": clocks_serial,
         "branch_chunks": pre.branch_chunks,
         "decode_ms_per_step": dec_ms / args.steps,
         "decode_tok_s": dec_tok_s,
