@@ -906,36 +906,6 @@ __global__ void __launch_bounds__(128)
   }
 }
 
-// ---- bf16 decode attention on the tensor cores (mma.sync m16n8k16) ---------------
-// Persistent: the work is the list of SLOTS-slot chunks of every (sequence, kv head),
-// item i = (b * Hkv + g) * nchunks + chunk, cut into equal contiguous ranges, one per
-// CTA (two CTAs per SM).  A CTA streams its chunks through STAGES shared-memory stages by
-// 3-D TMA (128-byte swizzle, rows past the store's capacity read as zero), the copies of
-// the next chunks in flight while the current one is computed, across (sequence, kv
-// head) boundaries too.  Warp w takes keys KW*w..KW*w+KW-1 of every chunk (KW = SLOTS/4):
-// S = Q K^T with
-// the query heads of the group in rows 0..rep-1 of a 16-row tile, an online softmax in
-// registers, O += P V with V fragments from ldmatrix.trans.  Where a run of chunks of
-// one (sequence, kv head) ends inside the CTA's range, the four warps' states are
-// merged in shared memory into one partial (max, sum, O) per query head, stored at the
-// slot of the run's first chunk; the combine kernel reads the run-start slots.
-namespace dtc {
-constexpr int SLOTS = 128;                  // slots per chunk
-constexpr int STAGES = 2;                   // chunks in flight per CTA: one ahead of the one computed
-constexpr int KW = SLOTS / 4;               // keys per warp
-constexpr int NT = KW / 8;                  // 8-key n-tiles of S per warp
-constexpr int KS = KW / 16;                 // 16-key k-steps of P V per warp
-constexpr int K_BYTES = SLOTS * 128;        // 64 bf16 per slot
-constexpr int V_BYTES = SLOTS * 256;        // two 64-column boxes
-constexpr int STAGE = K_BYTES + V_BYTES;
-constexpr int MAXREP = 8;
-// merge buffer [4 warps][rep][130] floats after the stages: two CTAs per SM for rep <= 5
-__host__ __device__ constexpr int merge_bytes(int rep) { return 4 * rep * 130 * 4; }
-__host__ __device__ constexpr int smem_bytes(int rep) { return STAGES * STAGE + merge_bytes(rep) + 8 * STAGES + 1024; }
-constexpr int CTAS_PER_SM = 2;
-static_assert(SLOTS % 64 == 0 && SLOTS <= 256, "whole 16-key steps per warp; TMA box rows <= 256");
-}  // namespace dtc
-
 // First chunk of every run: a run starts at chunk 0 of a (sequence, kv head) or at the
 // first item of a CTA's range.
 __host__ __device__ __forceinline__ bool dec_run_start(long long item, int chunk, long long per) {
@@ -967,21 +937,53 @@ __device__ __forceinline__ uint32_t sw128(int row, int ch) {
   return uint32_t(row * 128 + ((ch ^ (row & 7)) << 4));
 }
 
-__global__ void __launch_bounds__(128)
+// ---- bf16 decode attention on the tensor cores (mma.sync m16n8k16) ---------------
+// Persistent: the work is the list of 128-slot chunks of every (sequence, kv head), item
+// i = (b * Hkv + g) * nchunks + chunk, cut into equal contiguous ranges, one per CTA (two
+// CTAs per SM).  A CTA streams its chunks through two shared-memory stages by 3-D TMA
+// (128-byte swizzle, rows past the store's capacity read as zero), the next chunk's copy
+// in flight while the current one is computed, across (sequence, kv head) boundaries too.
+// Eight warps; warp w takes keys 16w..16w+15 of every chunk:
+//   S = Q K^T with the query heads of the group in rows 0..rep-1 of a 16-row tile (two
+//   8-key n-tiles), an online softmax in registers, then O^T += V^T P^T, in which the
+//   value columns fill the 16 MMA rows (eight 16-column m-tiles) and the query heads the
+//   8 columns, so no MMA row of the P V product is idle and O takes 32 registers.  The S
+//   fragment of a head row (keys 2gc, 2gc+1 of an n-tile) is already the B fragment of
+//   P^T, and V^T comes from ldmatrix.trans of the natural [slot][column] tile.
+// Where a run of chunks of one (sequence, kv head) ends inside the CTA's range, the eight
+// warps' states are merged in shared memory (warps 4..7 into 0..3, then the four) into one
+// partial (max, sum, O) per query head, stored at the slot of the run's first chunk; the
+// branch fuse kernel merges the run-start slots.
+namespace dtc {
+constexpr int SLOTS = 128;
+constexpr int STAGES = 2;
+constexpr int WARPS = 8;
+constexpr int THREADS = WARPS * 32;
+constexpr int KW = SLOTS / WARPS;  // 16 keys per warp: one k-step of P V
+constexpr int K_BYTES = SLOTS * 128;
+constexpr int V_BYTES = SLOTS * 256;
+constexpr int STAGE = K_BYTES + V_BYTES;
+// merge buffer [4][rep][130] floats: warps 4..7 merge into warps 0..3 first
+__host__ __device__ constexpr int merge_bytes(int rep) { return 4 * rep * 130 * 4; }
+__host__ __device__ constexpr int smem_bytes(int rep) { return STAGES * STAGE + merge_bytes(rep) + 8 * STAGES + 1024; }
+constexpr int CTAS_PER_SM = 2;
+static_assert(KW == 16, "one 16-key k-step per warp");
+}  // namespace dtc
+
+__global__ void __launch_bounds__(dtc::THREADS, 2)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                          const __nv_bfloat16 *__restrict__ q, float *__restrict__ part, int H,
-                          int Hkv, long long pos, int n_meta, int window, int is_global,
-                          float scale_log2, long long n_items, long long per, long long wlim) {
+                           const __nv_bfloat16 *__restrict__ q, float *__restrict__ part, int H,
+                           int Hkv, long long pos, int n_meta, int window, int is_global,
+                           float scale_log2, long long n_items, long long per, long long wlim) {
   using namespace dtc;
-  pdl_wait();
-  pdl_trigger();
   extern __shared__ uint8_t dsm_raw[];
   uint8_t *sm = dsm_raw + ((1024 - (smem_u32(dsm_raw) & 1023)) & 1023);
   const int rep = H / Hkv;
-  float *mw = reinterpret_cast<float *>(sm + STAGES * STAGE);                         // [4 warps][rep][130]
+  float *mw = reinterpret_cast<float *>(sm + STAGES * STAGE);                             // [4][rep][130]
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + STAGES * STAGE + merge_bytes(rep));  // [STAGES]
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int gr = lane >> 2, gc = lane & 3;  // mma group row / column pair
+  const int h0 = 2 * gc, h1 = 2 * gc + 1;   // the query heads of this lane's O^T columns
   const long long nslots = dec_slots(pos, n_meta, window, is_global);
   const int nchunks = (int)((nslots + SLOTS - 1) / SLOTS);
   const long long i0 = (long long)blockIdx.x * per;
@@ -998,19 +1000,46 @@ __global__ void __launch_bounds__(128)
     tma_load_3d(dst + K_BYTES, &tmV, &full[st], 0, s0, bg);
     tma_load_3d(dst + K_BYTES + V_BYTES / 2, &tmV, &full[st], 64, s0, bg);
   };
+  // The first chunks are requested before the wait for the preceding kernel, up to the
+  // chunk that holds this step's slot (written by the step's input projection, which may
+  // be the preceding kernel).  Every other slot was written by an earlier step, and when a
+  // kernel starts, the kernel two launches before it in the stream has completed.
+  const int new_chunk = (int)(kv_slot_of(pos, n_meta, window, is_global) / SLOTS);
+  int issued = 0;
   if (tid == 0) {
     for (int st = 0; st < STAGES; ++st) mbar_init(&full[st], 1);
     fence_barrier_init();
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    for (; issued < min(STAGES, nloc) && (int)((i0 + issued) % nchunks) != new_chunk; ++issued) issue(issued);
   }
+  pdl_wait();
+  pdl_trigger();
   __syncthreads();
-  int issued = 0;
   if (tid == 0)
     for (; issued < min(STAGES, nloc); ++issued) issue(issued);
-  float m_run = -INFINITY, l_run = 0.f;  // row gr of this warp
-  float oacc[16][4];
+  float m_run = -INFINITY, l_run = 0.f;  // head gr, over this warp's keys of the run
+  float oacc[8][4];  // m-tile mt: [0], [1] = (column 16mt+gr; heads h0, h1), [2], [3] = column +8
   uint32_t qa[4][2];  // Q fragments [k-step][a0a1 / a4a5]; rows 8..15 are zero
+  // this warp's (max, sum, O) for the heads below rep into merge slot `slot`
+  auto put = [&](int slot) {
+    float *base = mw + slot * rep * 130;
+    if (gr < rep && gc == 0) {
+      base[gr * 130] = m_run;
+      base[gr * 130 + 1] = l_run;
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      if (h0 < rep) {
+        base[h0 * 130 + 2 + 16 * mt + gr] = oacc[mt][0];
+        base[h0 * 130 + 2 + 16 * mt + gr + 8] = oacc[mt][2];
+      }
+      if (h1 < rep) {
+        base[h1 * 130 + 2 + 16 * mt + gr] = oacc[mt][1];
+        base[h1 * 130 + 2 + 16 * mt + gr + 8] = oacc[mt][3];
+      }
+    }
+  };
   bool ok = true;
   int k = 0;
   for (; k < nloc; ++k) {
@@ -1021,9 +1050,9 @@ __global__ void __launch_bounds__(128)
       m_run = -INFINITY;
       l_run = 0.f;
 #pragma unroll
-      for (int nt = 0; nt < 16; ++nt)
+      for (int mt = 0; mt < 8; ++mt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) oacc[nt][e] = 0.f;
+        for (int e = 0; e < 4; ++e) oacc[mt][e] = 0.f;
       const bool live = gr < rep;
       const uint32_t *qr =
           reinterpret_cast<const uint32_t *>(q + ((long long)b * H + g * rep + (live ? gr : 0)) * 64);
@@ -1038,28 +1067,28 @@ __global__ void __launch_bounds__(128)
     if (__syncthreads_or(!ok)) { ok = false; break; }
     const uint32_t kb = smem_u32(sm + st * STAGE), vb = kb + K_BYTES;
     const long long s0 = (long long)chunk * SLOTS;
-    // ---- S = Q K^T for this warp's KW keys (NT n-tiles of 8 keys) ----
-    float sacc[NT][4];
+    // ---- S = Q K^T for this warp's 16 keys (two n-tiles of 8) ----
+    float sacc[2][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[nt][e] = 0.f;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
+    for (int nt = 0; nt < 2; ++nt) {
       const int key = warp * KW + nt * 8 + (lane & 7);
 #pragma unroll
       for (int kp = 0; kp < 2; ++kp) {  // two k-steps per ldmatrix.x4
-        const int ch = kp * 4 + (lane >> 3);  // 16-byte chunk of the key row (8 dims)
+        const int ch = kp * 4 + (lane >> 3);
         uint32_t b0, b1, b2, b3;
         ldsm_x4(kb + sw128(key, ch), b0, b1, b2, b3);
         mma16816(sacc[nt], qa[2 * kp][0], 0u, qa[2 * kp][1], 0u, b0, b1);
         mma16816(sacc[nt], qa[2 * kp + 1][0], 0u, qa[2 * kp + 1][1], 0u, b2, b3);
       }
     }
-    // ---- online softmax, row gr (values sacc[nt][0..1], keys 8nt + 2gc + {0,1}) ----
+    // ---- online softmax, head gr (values sacc[nt][0..1], keys 8nt + 2gc + {0,1}) ----
     float mx = -INFINITY;
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int key = warp * KW + nt * 8 + 2 * gc + e;
@@ -1074,55 +1103,67 @@ __global__ void __launch_bounds__(128)
     const float mref = m_new == -INFINITY ? 0.f : m_new;
     const float alpha = m_run == -INFINITY ? 0.f : ex2(m_run - mref);
     m_run = m_new;
-    float lsum = 0.f;
-    uint32_t pa[NT];  // P as A fragments: [k-step kk][a0a1 (n-tile 2kk) / a4a5 (n-tile 2kk+1)]
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const float p0 = ex2(sacc[nt][0] - mref), p1 = ex2(sacc[nt][1] - mref);
-      lsum += p0 + p1;
-      pa[nt] = pack_bf16x2(p0, p1);
-    }
+    const float p00 = ex2(sacc[0][0] - mref), p01 = ex2(sacc[0][1] - mref);
+    const float p10 = ex2(sacc[1][0] - mref), p11 = ex2(sacc[1][1] - mref);
+    // P^T as the B fragment: b0b1 = keys 2gc, 2gc+1 of head gr, b2b3 = keys 8 + 2gc, 9 + 2gc
+    const uint32_t pb0 = pack_bf16x2(p00, p01), pb1 = pack_bf16x2(p10, p11);
+    float lsum = (p00 + p01) + (p10 + p11);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
     lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
     l_run = fmaf(l_run, alpha, lsum);
+    // rescale by the alphas of heads h0, h1 (held by the lanes of rows h0, h1)
+    const float al0 = __shfl_sync(0xffffffffu, alpha, h0 * 4), al1 = __shfl_sync(0xffffffffu, alpha, h1 * 4);
+    // ---- O^T += V^T P^T: eight m-tiles of 16 value columns, one 16-key k-step ----
+    {
+      const int j = lane >> 3;  // ldmatrix matrix: keys (j >> 1) * 8.., columns 8 (j & 1)..
+      const int key = warp * KW + (j >> 1) * 8 + (lane & 7);
 #pragma unroll
-    for (int nt = 0; nt < 16; ++nt) {
-      oacc[nt][0] *= alpha;
-      oacc[nt][1] *= alpha;
-    }
-    // ---- O += P V (16 n-tiles of 8 value columns, KS k-steps of 16 keys) ----
-#pragma unroll
-    for (int kk = 0; kk < KS; ++kk) {
-      const int key = warp * KW + kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-      for (int np = 0; np < 8; ++np) {  // pairs of n-tiles per ldmatrix.x4.trans
-        const int chg = np * 2 + (lane >> 4);  // 16-byte chunk of value columns (0..15)
+      for (int mt = 0; mt < 8; ++mt) {
+        const int chg = 2 * mt + (j & 1);  // 16-byte chunk of value columns (0..15)
         const uint32_t addr = vb + (chg >> 3) * (V_BYTES / 2) + sw128(key, chg & 7);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(addr, b0, b1, b2, b3);
-        mma16816(oacc[2 * np], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b0, b1);
-        mma16816(oacc[2 * np + 1], pa[2 * kk], 0u, pa[2 * kk + 1], 0u, b2, b3);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(addr, a0, a1, a2, a3);
+        oacc[mt][0] *= al0;
+        oacc[mt][1] *= al1;
+        oacc[mt][2] *= al0;
+        oacc[mt][3] *= al1;
+        mma16816(oacc[mt], a0, a1, a2, a3, pb0, pb1);
       }
     }
     __syncthreads();  // every warp is done with stage st
     if (tid == 0 && issued < nloc) issue(issued++);
     if (chunk == nchunks - 1 || k == nloc - 1) {
-      // the run ends: merge the four warps, rows 0..rep-1, into the run-start slot
-      if (gr < rep) {
-        float *row = mw + (warp * rep + gr) * 130;
-        if (gc == 0) {
-          row[0] = m_run;
-          row[1] = l_run;
-        }
+      // the run ends: warps 4..7 merge into warps 0..3, then the four into the run-start slot
+      if (warp >= 4) put(warp - 4);
+      __syncthreads();
+      if (warp < 4) {
+        const float *base = mw + warp * rep * 130;
+        const float m2 = gr < rep ? base[gr * 130] : -INFINITY;
+        const float l2 = gr < rep ? base[gr * 130 + 1] : 0.f;
+        const float M = fmaxf(m_run, m2);
+        const float s1 = m_run == -INFINITY ? 0.f : ex2(m_run - M);
+        const float s2 = m2 == -INFINITY ? 0.f : ex2(m2 - M);
+        l_run = l_run * s1 + l2 * s2;
+        m_run = M;
+        const float a10 = __shfl_sync(0xffffffffu, s1, h0 * 4), a11 = __shfl_sync(0xffffffffu, s1, h1 * 4);
+        const float a20 = __shfl_sync(0xffffffffu, s2, h0 * 4), a21 = __shfl_sync(0xffffffffu, s2, h1 * 4);
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          row[2 + nt * 8 + 2 * gc] = oacc[nt][0];
-          row[2 + nt * 8 + 2 * gc + 1] = oacc[nt][1];
+        for (int mt = 0; mt < 8; ++mt) {
+          const float o00 = h0 < rep ? base[h0 * 130 + 2 + 16 * mt + gr] : 0.f;
+          const float o02 = h0 < rep ? base[h0 * 130 + 2 + 16 * mt + gr + 8] : 0.f;
+          const float o11 = h1 < rep ? base[h1 * 130 + 2 + 16 * mt + gr] : 0.f;
+          const float o13 = h1 < rep ? base[h1 * 130 + 2 + 16 * mt + gr + 8] : 0.f;
+          oacc[mt][0] = oacc[mt][0] * a10 + o00 * a20;
+          oacc[mt][2] = oacc[mt][2] * a10 + o02 * a20;
+          oacc[mt][1] = oacc[mt][1] * a11 + o11 * a21;
+          oacc[mt][3] = oacc[mt][3] * a11 + o13 * a21;
         }
       }
+      __syncthreads();  // warps 0..3 have read the slots they now overwrite
+      if (warp < 4) put(warp);
       __syncthreads();
       const int run_chunk = (int)(max(i0, it - chunk) - (it - chunk));  // the run began at item max(i0, it - chunk)
-      for (int idx = tid; idx < rep * 130; idx += 128) {
+      for (int idx = tid; idx < rep * 130; idx += THREADS) {
         const int r = idx / 130, col = idx % 130;
         float M = -INFINITY;
 #pragma unroll
@@ -1240,7 +1281,7 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
     cudaGetDevice(&dev);
     if (!attr_tc.done(dev)) {
       if (cudaFuncSetAttribute(attn_decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               dtc::smem_bytes(dtc::MAXREP)) != cudaSuccess) {
+                               dtc::smem_bytes(DEC_MAXREP)) != cudaSuccess) {
         set_error("cudaFuncSetAttribute(decode attention smem) failed");
         return HYMBA_ERR_CUDA;
       }
@@ -1262,7 +1303,7 @@ hymba_status attention_decode(DecodeAttnArgs &a, hymba_dtype dt, cudaStream_t s)
     const long long n_items = (long long)a.B * a.Hkv * nchunks;
     const long long grid_tc = std::min<long long>(n_items, (long long)dtc::CTAS_PER_SM * sms);
     const long long per = (n_items + grid_tc - 1) / grid_tc;
-    launch_kernel(attn_decode_tc_kernel, dim3((unsigned)((n_items + per - 1) / per)), dim3(128),
+    launch_kernel(attn_decode_tc_kernel, dim3((unsigned)((n_items + per - 1) / per)), dim3(dtc::THREADS),
                   (size_t)dtc::smem_bytes(rep), s, tk, tv, (const __nv_bfloat16 *)a.q, a.partial, a.H, a.Hkv,
                   (long long)a.pos, a.n_meta, a.window, a.is_global, sl2, n_items, per, wait_limit_cycles());
     if (a.fuse_later) {

@@ -238,11 +238,13 @@ __global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
   for (int k = 0; k < 3; ++k) w[k] = k < K - 1 ? __ldg(a.conv_w + c * K + k) : 0.f;
   const float wlast = __ldg(a.conv_w + c * K + K - 1);
   const float bias = __ldg(a.conv_b + c);
-  pdl_wait();
-  pdl_trigger();
   // conv + SiLU: thread -> channel tid % CH, rows tid / CH + k * (256 / CH).  Every load
   // is issued unconditionally (rows past the batch read a valid row and are discarded)
-  // and kept raw until all of them are in flight, so their latencies overlap.
+  // and kept raw until all of them are in flight, so their latencies overlap.  The window
+  // rows are requested before the wait for the preceding kernel: this layer's conv state
+  // was last written by this kernel in the previous step, and when a kernel starts, the
+  // kernel two launches before it in the stream has completed (each kernel lets its
+  // dependents start only after its own wait), so no write to it can be in flight.
   {
     T *cs = reinterpret_cast<T *>(a.conv_state);
     const T *x = reinterpret_cast<const T *>(a.x);
@@ -255,6 +257,12 @@ __global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
 #pragma unroll
         for (int t = 0; t < 3; ++t) raw[k][t] = cs[((long long)bb * (K - 1) + min(t, K - 2)) * a.E + c];
       }
+    }
+    pdl_wait();
+    pdl_trigger();
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int bb = min(b0 + tid / CH + k * (256 / CH), a.B - 1);
       raw[k][3] = x[(long long)bb * a.ld_x + c];
     }
 #pragma unroll
@@ -385,8 +393,8 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
   const int nrows = min(kScanRows, a.B - b0);
   const int ch = tid % kScanCh, rg = tid / kScanCh;  // channel, group of four rows
   const int c = cbase + ch;
-  // Before the wait for the preceding kernel: the weights (W_dt slice, A, biases) and an
-  // L2 hint for this CTA's state rows (2 KB per sequence).
+  // Before the wait for the preceding kernel: the weights (W_dt slice, A, biases) and the
+  // state rows (below).
   {
     const float *src = a.w_dt + (long long)cbase * R;
     const int per_row = R / 4;
@@ -396,7 +404,6 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
     }
     for (int idx = tid; idx < kScanCh * (lay.RP - R); idx += 128)
       wdt[(idx / (lay.RP - R)) * lay.WS + R + idx % (lay.RP - R)] = 0.f;
-    if (tid < nrows) prefetch_l2_bulk(a.h + ((long long)(b0 + tid) * a.E + cbase) * kStates, kScanCh * kStates * 4);
   }
   float A2[kStates];
   {
@@ -411,9 +418,10 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
     }
   }
   const float bdt = __ldg(a.b_dt + c), Dc = __ldg(a.d_skip + c);
-  pdl_wait();
-  pdl_trigger();
-  // the states of this thread's four rows
+  // The states of this thread's four rows, requested before the wait for the preceding
+  // kernel: the state was last written by this kernel in the previous step, and when a
+  // kernel starts, the kernel two launches before it in the stream has completed (each
+  // kernel lets its dependents start only after its own wait).
   float4 hv[4][kStates / 4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -422,6 +430,8 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
 #pragma unroll
     for (int q = 0; q < kStates / 4; ++q) hv[k][q] = hp[q];
   }
+  pdl_wait();
+  pdl_trigger();
   {
     // delta_r, B, C of the rows: fixed-point sums of the conv kernel's x_proj shares
     const longlong2 *xsrc = reinterpret_cast<const longlong2 *>(a.xacc + (long long)b0 * NJ);
@@ -452,6 +462,7 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
     const int g = lane >> 2, t = lane & 3;
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     const float *wr = wdt + (warp * 8 + g) * lay.WS;
+#pragma unroll 4
     for (int k0 = 0; k0 < lay.RP; k0 += 8) {
       const uint32_t a0 = to_tf32(xs[g * lay.XS + k0 + t]), a1 = to_tf32(xs[(g + 8) * lay.XS + k0 + t]);
       const uint32_t a2 = to_tf32(xs[g * lay.XS + k0 + t + 4]), a3 = to_tf32(xs[(g + 8) * lay.XS + k0 + t + 4]);
