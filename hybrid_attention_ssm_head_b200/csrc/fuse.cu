@@ -208,15 +208,27 @@ hymba_status fuse_branches(const FuseArgs &a, hymba_dtype dt, cudaStream_t s) {
 // weights 2^(m_r - M) / L; the merged O (fp32, four values per lane) stays in registers
 // for the two RMS norms.
 __global__ void __launch_bounds__(1024) fuse_decode_kernel(FuseDecodeArgs a) {
-  pdl_wait();
-  pdl_trigger();
   __shared__ float red[2][32];
   const int b = blockIdx.x, h = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rep = a.H / a.Hkv, E = a.H * a.dv;
   const bool live = h < a.H;
-  float4 ov = make_float4(0.f, 0.f, 0.f, 0.f), yv = ov;
+  const int c = h * a.dv + 4 * lane;
+  // beta before the wait for the preceding kernels; the SSM branch's output row after it
+  // (the scan step that writes it is a direct predecessor when it ran on a side stream
+  // joined into this one, and may then still be running when this kernel starts)
+  float4 ba = make_float4(0.f, 0.f, 0.f, 0.f), bs = ba, yv = ba;
+  if (live) {
+    ba = *reinterpret_cast<const float4 *>(a.beta_attn + c);
+    bs = *reinterpret_cast<const float4 *>(a.beta_ssm + c);
+  }
+  pdl_wait();
+  pdl_trigger();
+  float4 ov = make_float4(0.f, 0.f, 0.f, 0.f);
   float so = 0.f, sy = 0.f;
   if (live) {
+    const uint2 raw = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(a.y) +
+                                                       (long long)b * E + c);
+    yv = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
     const int g = h / rep;
     const long long item0 = ((long long)b * a.Hkv + g) * a.nchunks;
     const long long r0 = item0 % a.per;
@@ -225,39 +237,71 @@ __global__ void __launch_bounds__(1024) fuse_decode_kernel(FuseDecodeArgs a) {
     if (cfirst < a.nchunks) nruns += 1 + (int)((a.nchunks - 1 - cfirst) / a.per);
     const float *base = a.part + ((long long)b * a.H + h) * a.nchunks * (a.dv + 2);
     auto run = [&](long long k) { return base + (k == 0 ? 0 : cfirst + (k - 1) * a.per) * (a.dv + 2); };
-    // the runs' (max, sum) pairs, 32 runs per round across the lanes
-    float M = -INFINITY;
-    for (int k0 = 0; k0 < nruns; k0 += 32)
-      if (k0 + lane < nruns) M = fmaxf(M, run(k0 + lane)[0]);
+    constexpr int KR = 4;  // up to KR runs: every (max, sum) and O requested at once
+    if (nruns <= KR) {
+      float2 ml[KR];
+      float4 o[KR];
 #pragma unroll
-    for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float L = 0.f;
-    for (int k0 = 0; k0 < nruns; k0 += 32) {
-      if (k0 + lane < nruns) {
-        const float *r = run(k0 + lane);
-        if (r[0] != -INFINITY) L = fmaf(r[1], ex2_ftz(r[0] - M), L);
+      for (int k = 0; k < KR; ++k) {
+        ml[k] = make_float2(-INFINITY, 0.f);
+        o[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k < nruns) {
+          const float *r = run(k);
+          ml[k] = *reinterpret_cast<const float2 *>(r);
+          // O starts at offset 2 (8-byte aligned): two float2 loads per lane
+          const float2 p0 = *reinterpret_cast<const float2 *>(r + 2 + 4 * lane);
+          const float2 p1 = *reinterpret_cast<const float2 *>(r + 2 + 4 * lane + 2);
+          o[k] = make_float4(p0.x, p0.y, p1.x, p1.y);
+        }
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < KR; ++k) M = fmaxf(M, ml[k].x);
+      float L = 0.f;
+#pragma unroll
+      for (int k = 0; k < KR; ++k)
+        if (ml[k].x != -INFINITY) L = fmaf(ml[k].y, ex2_ftz(ml[k].x - M), L);
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+      for (int k = 0; k < KR; ++k) {
+        if (ml[k].x == -INFINITY) continue;
+        const float w = ex2_ftz(ml[k].x - M) * inv;
+        ov.x = fmaf(o[k].x, w, ov.x);
+        ov.y = fmaf(o[k].y, w, ov.y);
+        ov.z = fmaf(o[k].z, w, ov.z);
+        ov.w = fmaf(o[k].w, w, ov.w);
+      }
+    } else {
+      // the runs' (max, sum) pairs, 32 runs per round across the lanes
+      float M = -INFINITY;
+      for (int k0 = 0; k0 < nruns; k0 += 32)
+        if (k0 + lane < nruns) M = fmaxf(M, run(k0 + lane)[0]);
+#pragma unroll
+      for (int off = 16; off; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+      float L = 0.f;
+      for (int k0 = 0; k0 < nruns; k0 += 32) {
+        if (k0 + lane < nruns) {
+          const float *r = run(k0 + lane);
+          if (r[0] != -INFINITY) L = fmaf(r[1], ex2_ftz(r[0] - M), L);
+        }
+      }
+#pragma unroll
+      for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      for (int k = 0; k < nruns; ++k) {
+        const float *r = run(k);
+        const float mk = r[0];
+        if (mk == -INFINITY) continue;
+        const float w = ex2_ftz(mk - M) * inv;
+        const float2 p0 = *reinterpret_cast<const float2 *>(r + 2 + 4 * lane);
+        const float2 p1 = *reinterpret_cast<const float2 *>(r + 2 + 4 * lane + 2);
+        ov.x = fmaf(p0.x, w, ov.x);
+        ov.y = fmaf(p0.y, w, ov.y);
+        ov.z = fmaf(p1.x, w, ov.z);
+        ov.w = fmaf(p1.y, w, ov.w);
       }
     }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    for (int k = 0; k < nruns; ++k) {
-      const float *r = run(k);
-      const float mk = r[0];
-      if (mk == -INFINITY) continue;
-      const float w = ex2_ftz(mk - M) * inv;
-      // O starts at offset 2 (8-byte aligned): two float2 loads per lane
-      const float2 p0 = *reinterpret_cast<const float2 *>(r + 2 + 4 * lane);
-      const float2 p1 = *reinterpret_cast<const float2 *>(r + 2 + 4 * lane + 2);
-      ov.x = fmaf(p0.x, w, ov.x);
-      ov.y = fmaf(p0.y, w, ov.y);
-      ov.z = fmaf(p1.x, w, ov.z);
-      ov.w = fmaf(p1.y, w, ov.w);
-    }
     so = ov.x * ov.x + ov.y * ov.y + ov.z * ov.z + ov.w * ov.w;
-    const uint2 raw = *reinterpret_cast<const uint2 *>(reinterpret_cast<const __nv_bfloat16 *>(a.y) +
-                                                       (long long)b * E + h * a.dv + 4 * lane);
-    yv = make_float4(bf16_lo(raw.x), bf16_hi(raw.x), bf16_lo(raw.y), bf16_hi(raw.y));
     sy = yv.x * yv.x + yv.y * yv.y + yv.z * yv.z + yv.w * yv.w;
   }
 #pragma unroll
@@ -287,9 +331,6 @@ __global__ void __launch_bounds__(1024) fuse_decode_kernel(FuseDecodeArgs a) {
   if (!live) return;
   const float ro = 0.5f * rsqrtf(red[0][0] / E + a.eps);
   const float ry = 0.5f * rsqrtf(red[1][0] / E + a.eps);
-  const int c = h * a.dv + 4 * lane;
-  const float4 ba = *reinterpret_cast<const float4 *>(a.beta_attn + c);
-  const float4 bs = *reinterpret_cast<const float4 *>(a.beta_ssm + c);
   uint2 outw;
   outw.x = pack_bf16x2(fmaf(ba.x * ro, ov.x, bs.x * ry * yv.x), fmaf(ba.y * ro, ov.y, bs.y * ry * yv.y));
   outw.y = pack_bf16x2(fmaf(ba.z * ro, ov.z, bs.z * ry * yv.z), fmaf(ba.w * ro, ov.w, bs.w * ry * yv.w));

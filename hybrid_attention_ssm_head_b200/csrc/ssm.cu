@@ -241,10 +241,11 @@ __global__ void __launch_bounds__(256) dec_conv_xproj_kernel(DecodeSsmArgs a) {
   // conv + SiLU: thread -> channel tid % CH, rows tid / CH + k * (256 / CH).  Every load
   // is issued unconditionally (rows past the batch read a valid row and are discarded)
   // and kept raw until all of them are in flight, so their latencies overlap.  The window
-  // rows are requested before the wait for the preceding kernel: this layer's conv state
-  // was last written by this kernel in the previous step, and when a kernel starts, the
-  // kernel two launches before it in the stream has completed (each kernel lets its
-  // dependents start only after its own wait), so no write to it can be in flight.
+  // rows are requested before the wait for the preceding kernels: this layer's conv state
+  // was last written by this kernel in the previous step, which is not a direct
+  // predecessor; since every kernel of the step waits in every CTA before it lets its
+  // dependents start, every kernel but the direct predecessors has completed when this one
+  // starts, so no write to the window can be in flight.
   {
     T *cs = reinterpret_cast<T *>(a.conv_state);
     const T *x = reinterpret_cast<const T *>(a.x);
@@ -419,9 +420,9 @@ __global__ void __launch_bounds__(128, 4) dec_scan_kernel(DecodeSsmArgs a) {
   }
   const float bdt = __ldg(a.b_dt + c), Dc = __ldg(a.d_skip + c);
   // The states of this thread's four rows, requested before the wait for the preceding
-  // kernel: the state was last written by this kernel in the previous step, and when a
-  // kernel starts, the kernel two launches before it in the stream has completed (each
-  // kernel lets its dependents start only after its own wait).
+  // kernels: the state was last written by this kernel in the previous step, which is not
+  // a direct predecessor, and every kernel but the direct predecessors has completed when
+  // this one starts (each kernel lets its dependents start only after its own wait).
   float4 hv[4][kStates / 4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
