@@ -643,18 +643,24 @@ static int num_sms() {
 // row, 16 output columns per store).  No atomics, no second pass.
 //   warp 0, one lane : TMA producer (weight tile and activation rows, 4-stage ring)
 //   warp 1, one lane : tcgen05.mma (M = 128, N = BN) into tensor memory
-//   all four warps   : tensor memory -> shared partial tile; the cluster reduction
+//   all four warps   : tensor memory -> shared partial tile; the cluster reduction with
+//                      16-byte distributed-shared-memory loads into a local tile of the
+//                      CTA's rows, then the epilogue from there
 // ---------------------------------------------------------------------------
 namespace wsg {
 constexpr int BM = 128, BK = 64, STAGES = 3;  // 3 stages: 5.43 ms per decode step, 4: 5.49, 2: 5.52
 constexpr int W_BYTES = BM * 128;
-template <int BN>
+template <int BN, int CL>
 struct Cfg {
   static constexpr int X_BYTES = BN * 128;
   static constexpr int STAGE = W_BYTES + X_BYTES;
-  static constexpr int PSTRIDE = BN + 1;  // floats per partial row: conflict-free both ways
+  // floats per partial row: a multiple of 4 (16-byte rows pieces) that is 16 bytes past a
+  // multiple of 128 bytes, so eight rows' 16-byte stores fall in eight different bank groups
+  static constexpr int PSTRIDE = BN + 4;
   static constexpr int P_BYTES = BM * PSTRIDE * 4;
-  static constexpr int BODY = STAGE * STAGES > P_BYTES ? STAGE * STAGES : P_BYTES;
+  // clusters of 4 or more: the CTA's BM / CL reduced rows after the partial tile
+  static constexpr int R_BYTES = CL >= 4 ? (BM / CL) * PSTRIDE * 4 : 0;
+  static constexpr int BODY = STAGE * STAGES > P_BYTES + R_BYTES ? STAGE * STAGES : P_BYTES + R_BYTES;
   static constexpr int SMEM = BODY + (2 * STAGES + 1) * 8 + 16 + 1024;
   static constexpr uint32_t IDESC = make_idesc(BN, 1, 0, 0);
 };
@@ -664,7 +670,7 @@ template <int BN, int CL>
 __global__ void __launch_bounds__(128, 1)
     gemm_ws_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, int Nout,
                    int B, int K, Epilogue epi, long long wlim) {
-  using C = wsg::Cfg<BN>;
+  using C = wsg::Cfg<BN, CL>;
   using namespace wsg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
@@ -770,7 +776,8 @@ __global__ void __launch_bounds__(128, 1)
   __syncthreads();  // the producer has drained: the stages are free for the partial tile
   tc_fence_after();
   {
-    // tensor memory -> this CTA's partial tile, part[row of W][activation row]
+    // tensor memory -> this CTA's partial tile, part[row of W][activation row], 16 bytes
+    // per store
     const int f = warp * 32 + lane;
     const uint32_t t_row = tmem + (uint32_t(warp * 32) << 16);
 #pragma unroll 1
@@ -779,14 +786,43 @@ __global__ void __launch_bounds__(128, 1)
       tmem_ld32(t_row + c, r);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) part[f * C::PSTRIDE + c + j] = acc_ok ? __uint_as_float(r[j]) : 0.f;
+      for (int j = 0; j < 32; j += 4)
+        *reinterpret_cast<float4 *>(part + f * C::PSTRIDE + c + j) =
+            acc_ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                 __uint_as_float(r[j + 3]))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
   tc_fence_before();
   cluster_sync();  // every partial tile of the cluster is written
-  {
-    constexpr int F = BM / CL;  // weight rows this CTA reduces and stores
+  constexpr int F = BM / CL;  // weight rows this CTA reduces and stores
+  // Clusters of 4 or more: the sums of this CTA's rows first go to a local tile [F][PSTRIDE]
+  // (each of the CL-fold 16-byte loads feeds four sums); smaller clusters sum the few remote
+  // values inside the store loop, whose loads then overlap the stores.
+  float *red = part + BM * C::PSTRIDE;
+  if constexpr (CL >= 4) {
+    // the CL partials of rows rank*F .. rank*F + F - 1: 16-byte loads, consecutive threads
+    // on consecutive pieces of a row (activation rows past the batch are not summed)
     const uint32_t pbase = smem_u32(part);
+    const int quads = (min(B, BN) + 3) / 4;
+#pragma unroll 4  // several rows' loads in flight at once
+    for (int it = tid; it < F * quads; it += 128) {
+      const int fl = it / quads, q = it - fl * quads;
+      const uint32_t off = (uint32_t)((((int)rank * F + fl) * C::PSTRIDE + 4 * q) * 4);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < CL; ++c) {
+        const float4 v = ld_shared_cluster_v4(map_shared_rank(pbase, (uint32_t)c) + off);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      *reinterpret_cast<float4 *>(red + fl * C::PSTRIDE + 4 * q) = acc;
+    }
+  }
+  __syncthreads();
+  {
 #pragma unroll 1
     for (int b = tid; b < B && b < BN; b += 128) {
       const long long m = b;
@@ -797,19 +833,24 @@ __global__ void __launch_bounds__(128, 1)
         const int f0 = (int)rank * F + j;
         const int n0 = mt * BM + f0;
         if (n0 >= Nout) break;
-        float acc[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] = 0.f;
-#pragma unroll
-        for (int c = 0; c < CL; ++c) {
-          const uint32_t remote = map_shared_rank(pbase, (uint32_t)c);
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            acc[i] += ld_shared_cluster_f32(remote + (uint32_t)(((f0 + i) * C::PSTRIDE + b) * 4));
-        }
         uint32_t bits[16];
+        if constexpr (CL >= 4) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) bits[i] = __float_as_uint(acc[i]);
+          for (int i = 0; i < 16; ++i) bits[i] = __float_as_uint(red[(j + i) * C::PSTRIDE + b]);
+        } else {
+          float acc[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] = 0.f;
+#pragma unroll
+          for (int c = 0; c < CL; ++c) {
+            const uint32_t remote = map_shared_rank(smem_u32(part), (uint32_t)c);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              acc[i] += ld_shared_cluster_f32(remote + (uint32_t)(((f0 + i) * C::PSTRIDE + b) * 4));
+          }
+#pragma unroll
+          for (int i = 0; i < 16; ++i) bits[i] = __float_as_uint(acc[i]);
+        }
         float bias[16];
         if (s_epi.bias) epi_bias16(s_epi, n0, Nout, bias);
         epi_store16<kEpiRoute | kEpiResid | kEpiGlu>(s_epi, m, mk, rp, n0, Nout, bits, bias);
@@ -827,7 +868,7 @@ __global__ void __launch_bounds__(128, 1)
 
 template <int BN, int CL>
 static hymba_status launch_ws(const GemmArgs &g, cudaStream_t s) {
-  using C = wsg::Cfg<BN>;
+  using C = wsg::Cfg<BN, CL>;
   static DeviceOnce attr_set;
   int dev = 0;
   cudaGetDevice(&dev);
