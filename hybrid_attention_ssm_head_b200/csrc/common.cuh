@@ -312,21 +312,16 @@ __device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x
                "r"(x), "r"(y)
                : "memory");
 }
-// Hint: bring `bytes` (a multiple of 16, 16-byte aligned address) into L2.
-__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
-               : "memory");
-}
-
 // ---------------------------------------------------------------------------
 // Programmatic dependent launch.  A kernel launched with the programmatic-serialisation
-// attribute may begin while the kernel before it in the stream is still running.  Before
-// pdl_wait() it touches only what no kernel of the library writes (weights, its own
-// shared memory and barriers, L2 prefetch hints); pdl_wait() returns once the preceding
-// grid has completed and its writes are visible (at once for a normal launch).  Every
-// CTA of such a kernel calls pdl_wait() before it reads or writes any other global
-// memory, so completion stays transitive along the stream.  pdl_trigger() lets the next
-// kernel in the stream start its own prologue.
+// attribute may begin while the kernel before it in the stream is still running.
+// pdl_wait() returns once the preceding grids have completed and their writes are visible
+// (at once for a normal launch).  Every CTA of such a kernel calls pdl_wait() before
+// pdl_trigger(), which lets the next kernel start its own prologue, so when a kernel starts,
+// every kernel but its direct predecessors has completed.  Before pdl_wait() a kernel
+// therefore reads only weights, its own shared memory and barriers, and data that no
+// direct predecessor writes (a decode kernel's own state from the previous step); it
+// writes global memory only after pdl_wait().
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
